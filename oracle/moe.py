@@ -1,0 +1,153 @@
+"""Mixture-of-Experts expert layer: router top-k, token permutation, the
+NVFP4 grouped expert GEMM with residual compensation, SwiGLU, combine.
+
+Oracle module (test infrastructure only, see ``oracle/__init__``).
+
+Method statements followed:
+* [QUADS-fr §1] / [QUADS-es §1]: the rollout runs MoE layers with native
+  NVFP4 W4A4 GEMMs (4-bit weights, 4-bit activations).
+* [QUADS-fr §2.2.B] / [QUADS-es §2.2.B]: on the high-residual channels a
+  correction term is computed and added to the quantized output, keeping the
+  W4A4 GEMM for the bulk of the work.  Here: Y = g_a g_w (deq_unit(A) .
+  deq_unit(W)^T) + R . Wc^T with R the BF16 residual on the channel set C
+  and Wc the weight columns of C (an operand: by default the dequantized
+  weights, so that selecting every channel gives exactly X . deq(W)^T).
+* [TRACE] "Fonctionnement, côté ingénierie": the router's choice of experts
+  is discrete, so small numeric differences can change which experts run.
+
+Readings where the pages are silent (each also listed in the design doc):
+* Router: experts ordered by (logit descending, index ascending), first k
+  taken; weights are the softmax over the k selected logits (renorm=True) or
+  the full softmax restricted to them (renorm=False).
+* Permutation: stable counting sort of the (token, slot) pairs by expert in
+  increasing token*k + slot order; each expert's segment is padded to a
+  multiple of 128 rows (the tensor-core tile height); pad rows are zero.
+* SwiGLU: the gate/up GEMM output row is [gate (F) | up (F)];
+  h = silu(gate) * up, silu(v) = v / (1 + exp(-v)).
+* Combine: y_t = sum over slots s = 0..k-1 of w[t, s] * Y[row_of[t, s]].
+"""
+import numpy as np
+
+from .formats import bf16_rne, f32
+from .nvfp4 import dequant_unit
+
+PAD = 128
+
+
+def router_topk(logits, k, renorm=True):
+    """Returns (idx [T, k] int32, w [T, k] float64)."""
+    l = np.asarray(logits, dtype=np.float64)
+    T, E = l.shape
+    order = np.argsort(-l, axis=1, kind="stable")      # stable: lower index first on ties
+    idx = order[:, :k].astype(np.int32)
+    sel = np.take_along_axis(l, idx, axis=1)
+    if renorm:
+        z = np.exp(sel - sel.max(axis=1, keepdims=True))
+        w = z / z.sum(axis=1, keepdims=True)
+    else:
+        zall = np.exp(l - l.max(axis=1, keepdims=True))
+        w = np.take_along_axis(zall, idx, axis=1) / zall.sum(axis=1, keepdims=True)
+    return idx, w
+
+
+def permute(idx, E):
+    """Stable counting sort of the flattened (token, slot) pairs by expert.
+
+    Returns (expert_off [E+1] int32, 128-padded; row_of [T*k] int32, the
+    expert-ordered row of pair i = t*k + s; src_of [expert_off[E]] int32,
+    the token of each expert-ordered row or -1 for a pad row)."""
+    flat = np.asarray(idx, dtype=np.int64).reshape(-1)
+    k = np.asarray(idx).shape[1]
+    counts = np.bincount(flat, minlength=E)
+    padded = -(-counts // PAD) * PAD
+    off = np.concatenate([[0], np.cumsum(padded)]).astype(np.int32)
+    order = np.argsort(flat, kind="stable")            # pairs grouped by expert, in pair order
+    first_of = np.concatenate([[0], np.cumsum(counts)])[:-1]
+    rank = np.arange(len(flat)) - first_of[flat[order]]
+    row_of = np.empty(len(flat), dtype=np.int32)
+    row_of[order] = off[flat[order]] + rank
+    src_of = np.full(int(off[-1]), -1, dtype=np.int32)
+    src_of[row_of] = (np.arange(len(flat)) // k).astype(np.int32)
+    return off, row_of, src_of
+
+
+def gather_rows(a, src_of):
+    """Rows of a in expert order; pad rows (src -1) are zero."""
+    a = np.asarray(a)
+    out = np.zeros((len(src_of),) + a.shape[1:], dtype=a.dtype)
+    ok = np.asarray(src_of) >= 0
+    out[ok] = a[np.asarray(src_of)[ok]]
+    return out
+
+
+def expert_of_rows(expert_off):
+    """Expert index of every row [0, expert_off[-1])."""
+    off = np.asarray(expert_off, dtype=np.int64)
+    return np.repeat(np.arange(len(off) - 1), np.diff(off))
+
+
+def grouped_gemm(a_codes, a_scales, g_a, w_codes, w_scales, g_w, expert_off,
+                 resid=None, wc=None):
+    """For every expert e and its rows [off[e], off[e+1]):
+        Y = g_a[e] * g_w[e] * deq_unit(A) . deq_unit(W_e)^T + R . Wc_e^T
+    in float64.  a_* are [R, K] codes / [R, K/16] scales (unpacked),
+    w_* are [E, N, K] / [E, N, K/16]; g_a is a scalar or [E]; resid is
+    [R, nc] (BF16-exact values) and wc [E, N, nc].
+
+    Returns (Y [R, N], absdot [R, N]) where absdot is sum |a*b| over every
+    product term, compensation included (the tolerance's scale)."""
+    off = np.asarray(expert_off, dtype=np.int64)
+    E = len(off) - 1
+    g_a = np.broadcast_to(np.asarray(g_a, dtype=np.float64), (E,))
+    R = int(off[-1])
+    N = np.asarray(w_codes).shape[1]
+    Y = np.zeros((R, N))
+    absdot = np.zeros((R, N))
+    for e in range(E):
+        lo, hi = int(off[e]), int(off[e + 1])
+        if hi == lo:
+            continue
+        A = dequant_unit(a_codes[lo:hi], a_scales[lo:hi])
+        W = dequant_unit(w_codes[e], w_scales[e])
+        G = g_a[e] * float(g_w[e])
+        Y[lo:hi] = G * (A @ W.T)
+        absdot[lo:hi] = abs(G) * (np.abs(A) @ np.abs(W).T)
+        if resid is not None and wc is not None and np.asarray(resid).shape[1] > 0:
+            Rr = np.asarray(resid, dtype=np.float64)[lo:hi]
+            Wc = np.asarray(wc, dtype=np.float64)[e]
+            Y[lo:hi] += Rr @ Wc.T
+            absdot[lo:hi] += np.abs(Rr) @ np.abs(Wc).T
+    return Y, absdot
+
+
+def swiglu(y):
+    """h = silu(gate) * up with y = [gate | up] along the last axis, float64."""
+    y = np.asarray(y, dtype=np.float64)
+    F = y.shape[1] // 2
+    gate, up = y[:, :F], y[:, F:]
+    return gate / (1.0 + np.exp(-gate)) * up
+
+
+def combine(y, row_of, w, k):
+    """y_t = sum_s w[t, s] * Y[row_of[t*k + s]], slots in order, float64."""
+    y = np.asarray(y, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    T = w.shape[0]
+    rows = np.asarray(row_of).reshape(T, k)
+    out = np.zeros((T, y.shape[1]))
+    for s in range(k):
+        out += w[:, s:s + 1] * y[rows[:, s]]
+    return out
+
+
+def per_token_gap(y_rollout, y_trainer):
+    """Per-token L2 distance between two layer outputs, relative to the
+    trainer output's norm (a reported diagnostic; parity unpinned)."""
+    a = np.asarray(y_rollout, dtype=np.float64)
+    b = np.asarray(y_trainer, dtype=np.float64)
+    return np.linalg.norm(a - b, axis=1) / np.maximum(np.linalg.norm(b, axis=1), 1e-30)
+
+
+def bf16_out(v):
+    """Round float64 results to BF16 via float32 (as a BF16 store does)."""
+    return bf16_rne(f32(v))

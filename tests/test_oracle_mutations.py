@@ -1,0 +1,145 @@
+"""Plant plausible mistakes in the CPU oracle (monkeypatched, CPU only) and
+check that at least one pin catches each of them."""
+import numpy as np
+import pytest
+
+from oracle import formats as F
+from oracle import moe as M
+from oracle import nvfp4 as Q
+from tests import oracle_pins as P
+
+
+def _e2m1_ties_up(v):
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    lv = F.E2M1_LEVELS
+    lo = np.clip(np.searchsorted(lv, a, side="right") - 1, 0, 7)
+    hi = np.minimum(lo + 1, 7)
+    up = (lv[hi] - a) <= (a - lv[lo])
+    idx = np.where(a >= 6, 7, lo + up)
+    return ((np.signbit(v).astype(np.int64) << 3) | idx).astype(np.uint8)
+
+
+def _e2m1_no_sign(v):
+    return F.e2m1_rne_code(np.abs(np.asarray(v, dtype=np.float64)))
+
+
+def _e4m3_truncate(t):
+    t = np.minimum(np.asarray(t, dtype=np.float64), 448.0)
+    with np.errstate(divide="ignore"):
+        e = np.maximum(np.floor(np.log2(np.where(t > 0, t, 1.0))), -6.0)
+    q = np.exp2(e - 3.0)
+    return F.e4m3_rn_satfinite_code(np.floor(t / q) * q)
+
+
+def _tensor_scale_wrong(amax):
+    return F.f32(np.float64(amax) / (6.0 * 256.0))
+
+
+_orig_gemm = M.grouped_gemm
+
+
+def _gemm_no_comp(a_codes, a_scales, g_a, w_codes, w_scales, g_w, off, resid=None, wc=None):
+    return _orig_gemm(a_codes, a_scales, g_a, w_codes, w_scales, g_w, off)
+
+
+def _gemm_no_gw(a_codes, a_scales, g_a, w_codes, w_scales, g_w, off, resid=None, wc=None):
+    return _orig_gemm(a_codes, a_scales, g_a, w_codes, w_scales, np.ones_like(np.asarray(g_w)),
+                      off, resid, wc)
+
+
+def _router_ties_high(logits, k, renorm=True):
+    l = np.asarray(logits, dtype=np.float64)
+    E = l.shape[1]
+    idx, w = M.__dict__["_orig_router"](l[:, ::-1], k, renorm)
+    return (E - 1 - idx).astype(np.int32), w
+
+
+_orig_permute = M.permute
+
+
+def _permute_reversed(idx, E):
+    off, row_of, src_of = _orig_permute(idx, E)
+    flat = np.asarray(idx).reshape(-1)
+    row2 = row_of.copy()
+    for e in range(E):
+        sel = np.flatnonzero(flat == e)
+        row2[sel] = row_of[sel][::-1]
+    src2 = np.full_like(src_of, -1)
+    k = np.asarray(idx).shape[1]
+    src2[row2] = np.arange(len(flat)) // k
+    return off, row2, src2
+
+
+def _combine_transposed(y, row_of, w, k):
+    T = np.asarray(w).shape[0]
+    r = np.asarray(row_of).reshape(T, k).T.reshape(-1)[:T * k]
+    return M.__dict__["_orig_combine"](y, r.reshape(-1), w, k)
+
+
+def _resid_sign(x, codes, scales, g):
+    return F.f32(Q.dequant_f32(codes, scales, g) - np.asarray(x, dtype=np.float64))
+
+
+def _bf16_truncate(v):
+    u = np.asarray(v, dtype=np.float32).view(np.uint32)
+    return ((u >> np.uint32(16)) << np.uint32(16)).view(np.float32).astype(np.float64)
+
+
+def _swiglu_wrong(y):
+    y = np.asarray(y, dtype=np.float64)
+    Fh = y.shape[1] // 2
+    g, u = y[:, :Fh], y[:, Fh:]
+    return u / (1.0 + np.exp(-u)) * g
+
+
+def _pack_swapped(codes):
+    c = np.asarray(codes, dtype=np.uint8)
+    return (c[..., 1::2] | (c[..., 0::2] << 4)).astype(np.uint8)
+
+
+def _select_ties_high(scores, n):
+    s = np.asarray(scores, dtype=np.float64)
+    order = np.lexsort((-np.arange(len(s)), -s))
+    return np.sort(order[:n]).astype(np.int32)
+
+
+def _div_instead_of_recip(x, g):
+    # divides by 2*S: a wrong element scale (dropped factor)
+    x = np.asarray(x, dtype=np.float64)
+    codes, s = Q.__dict__["_orig_qws"](x * 0.5, g)
+    return codes, s
+
+
+MUTATIONS = {
+    "e2m1_ties_away": [(F, "e2m1_rne_code", _e2m1_ties_up), (Q, "e2m1_rne_code", _e2m1_ties_up)],
+    "e2m1_drops_sign": [(F, "e2m1_rne_code", _e2m1_no_sign), (Q, "e2m1_rne_code", _e2m1_no_sign)],
+    "e4m3_truncates": [(F, "e4m3_rn_satfinite_code", _e4m3_truncate),
+                       (Q, "e4m3_rn_satfinite_code", _e4m3_truncate)],
+    "tensor_scale_constant": [(Q, "tensor_scale", _tensor_scale_wrong)],
+    "gemm_drops_compensation": [(M, "grouped_gemm", _gemm_no_comp)],
+    "gemm_drops_weight_scale": [(M, "grouped_gemm", _gemm_no_gw)],
+    "router_ties_to_high_index": [(M, "_orig_router", M.router_topk), (M, "router_topk", _router_ties_high)],
+    "permute_unstable": [(M, "permute", _permute_reversed)],
+    "combine_slot_index": [(M, "_orig_combine", M.combine), (M, "combine", _combine_transposed)],
+    "residual_sign": [(Q, "residual_f32", _resid_sign)],
+    "bf16_truncates": [(F, "bf16_rne", _bf16_truncate), (Q, "bf16_rne", _bf16_truncate)],
+    "swiglu_gate_up_swapped": [(M, "swiglu", _swiglu_wrong)],
+    "nibble_order": [(F, "pack_nibbles", _pack_swapped)],
+    "channel_ties_to_high_index": [(Q, "select_channels", _select_ties_high)],
+    "element_scale_dropped_factor": [(Q, "_orig_qws", Q.quantize_with_scale),
+                                     (Q, "quantize_with_scale", _div_instead_of_recip)],
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_mutation_is_caught(name, monkeypatch):
+    for mod, attr, fn in MUTATIONS[name]:
+        monkeypatch.setattr(mod, attr, fn, raising=False)
+    failures = []
+    for pin in P.ALL_PINS:
+        try:
+            pin()
+        except Exception as exc:        # noqa: BLE001 -- any failure counts as caught
+            failures.append((pin.__name__, type(exc).__name__))
+    assert failures, f"mutation {name} passed every pin"
