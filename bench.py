@@ -1,0 +1,428 @@
+"""Benchmark of the NVFP4 MoE train/rollout alignment path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+One step = one pass of the whole path over one batch of the 2048-token,
+8-expert MoE layer (hidden 1024, top-2, SwiGLU ffn 2048, 32 + 32 compensation
+channels): weight sync (amax + fake-quant of both expert weight tensors,
+which also writes the rollout's NVFP4 weights and compensation columns),
+the rollout forward (amax + quantize x with residual channels, router top-k,
+permutation, gather, grouped NVFP4 gate/up GEMM with compensation, SwiGLU
+with per-expert amax, per-expert quantize of h with residual channels,
+grouped down GEMM with compensation, combine), the TRACE record export, the
+trainer replay of both recorded tensors against the trainer's activation,
+and the straight-through backward accumulated into both master gradients.
+
+value = FLOPs of the two grouped GEMMs (FP4 products + BF16 compensation,
+algorithmic: routed rows only) per step, summed over ranks, / max-over-ranks
+step time.  Multi-GPU runs are data-parallel replicas (each rank its own
+batch, no collective on the path): weak scaling.
+
+--impl reference times the CPU oracle (float64 numpy) on a bounded sample of
+the same workload (one eighth of the tokens and of the experts' weight
+syncs per step) on the host cores; under torchrun only rank 0 runs it.
+"""
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 MoE grouped-GEMM TFLOPS (% FP4 peak); quantize/replay GB/s (% HBM)"
+UNIT = "TFLOP/s"
+DEFAULT_WORKLOAD = "moe_t2048_h1024_e8k2_f2048"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP4_OVER_BF16 = 4.0          # nominal dense ratio (9 / 2.25 PFLOP/s)
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------- accounting
+
+
+def gemm_flops(cfg, counts=None):
+    """Algorithmic FLOPs of both grouped GEMMs for T*k routed rows."""
+    R = cfg.T * cfg.k
+    fp4 = 2 * R * (2 * cfg.F) * cfg.H + 2 * R * cfg.H * cfg.F
+    comp = 2 * R * (2 * cfg.F) * cfg.n_chan + 2 * R * cfg.H * cfg.n_chan_f
+    return fp4, comp
+
+
+def kernel_work(cfg, rpad):
+    """Algorithmic bytes (HBM) or FLOPs per launch of every kernel in a step,
+    and which roofline bounds it."""
+    T, H, E, k, F = cfg.T, cfg.H, cfg.E, cfg.k, cfg.F
+    nc, ncf = cfg.n_chan, cfg.n_chan_f
+    R = T * k
+    wgu = E * 2 * F * H
+    wd = E * H * F
+    q = 0.5 + 1.0 / 16                      # codes + scales per element
+    w = {
+        "amax_w_gate_up": ("hbm", 2.0 * wgu),
+        "fakequant_w_gate_up": ("hbm", wgu * (2 + 2 + q) + E * 2 * F * nc * 2),
+        "amax_w_down": ("hbm", 2.0 * wd),
+        "fakequant_w_down": ("hbm", wd * (2 + 2 + q) + E * H * ncf * 2),
+        "amax_x": ("hbm", 2.0 * T * H),
+        "quantize_x": ("hbm", T * H * (2 + q) + T * nc * 2),
+        "router_topk": ("hbm", T * E * 4 + R * 8),
+        "permute": ("hbm", R * 4 * 3),
+        "gather": ("hbm", (R + T) * (H * q + nc * 2)),
+        "gemm_gate_up": ("tensor", 2.0 * R * 2 * F * H + 2.0 * R * 2 * F * nc),
+        "swiglu": ("hbm", rpad * (2 * F * 2 + F * 2)),
+        "quantize_h": ("hbm", rpad * F * (2 + q) + rpad * ncf * 2),
+        "gemm_down": ("tensor", 2.0 * R * H * F + 2.0 * R * H * ncf),
+        "combine": ("hbm", R * H * 2 + T * H * 2),
+        "replay_x": ("hbm", T * H * (q + 2 + 2)),
+        "replay_h": ("hbm", rpad * F * (q + 2)),
+        "ste_backward_gate_up": ("hbm", wgu * 6.0),
+        "ste_backward_down": ("hbm", wd * 6.0),
+    }
+    return w
+
+
+# ------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """nvidia-smi samples of this GPU's SM clock and throttle reasons."""
+
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            if self.uuid and self.uuid not in parts[0]:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# -------------------------------------------------------------------- oracle
+
+
+class OracleSample:
+    """Bounded CPU sample of the workload for the oracle: per run, the
+    weight sync and straight-through backward of E/frac_experts experts and
+    the rollout forward + record replay of T/frac_tokens tokens.  Inputs and
+    every expert's NVFP4 weights (which the forward needs) are prepared once,
+    outside the timing."""
+
+    def __init__(self, cfg, frac_tokens=8, frac_experts=8, seed=0):
+        import numpy as np
+        from oracle import layer as OL
+        from oracle import nvfp4 as Q
+        from train_alignment_b200 import workloads as W
+        self.OL, self.Q, self.cfg = OL, Q, cfg
+        inp = W.moe_layer_inputs(cfg, seed=seed, device="cpu")
+        self.T_s = max(cfg.T // frac_tokens, 1)
+        self.E_s = max(cfg.E // frac_experts, 1)
+        self.x = inp["x"][:self.T_s].float().numpy().astype(np.float64)
+        self.logits = inp["logits"][:self.T_s].numpy().astype(np.float64)
+        self.w_gu = inp["w_gu"].float().numpy().astype(np.float64)
+        self.w_d = inp["w_d"].float().numpy().astype(np.float64)
+        r = np.random.default_rng(seed)
+        self.chan_x = Q.pad_channels(np.sort(r.choice(cfg.H, cfg.n_chan, replace=False)))
+        self.chan_h = Q.pad_channels(np.sort(r.choice(cfg.F, cfg.n_chan_f, replace=False)))
+        self.wgu_all = OL.weight_sync(self.w_gu, self.chan_x)
+        self.wd_all = OL.weight_sync(self.w_d, self.chan_h)
+        R = self.T_s * cfg.k
+        self.flops = 2 * R * 2 * cfg.F * cfg.H + 2 * R * cfg.H * cfg.F + 2 * R * 2 * cfg.F * cfg.n_chan + \
+            2 * R * cfg.H * cfg.n_chan_f
+        self.desc = (f"oracle (float64 numpy) on {self.T_s} of {cfg.T} tokens and the weight sync + STE "
+                     f"backward of {self.E_s} of {cfg.E} experts per step")
+
+    def run(self):
+        OL, Q, E_s = self.OL, self.Q, self.E_s
+        t0 = time.perf_counter()
+        OL.weight_sync(self.w_gu[:E_s], self.chan_x)
+        OL.weight_sync(self.w_d[:E_s], self.chan_h)
+        fwd = OL.rollout_forward(self.x, self.logits, self.wgu_all, self.wd_all, self.chan_x, self.chan_h,
+                                 self.cfg.k)
+        OL.trainer_replay(fwd, self.x, self.chan_x, self.chan_h)
+        Q.ste_backward(self.w_gu[:E_s], self.w_gu[:E_s])
+        Q.ste_backward(self.w_d[:E_s], self.w_d[:E_s])
+        return time.perf_counter() - t0
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:  # noqa: BLE001
+        return 1
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    from train_alignment_b200 import workloads as W
+    cfg = W.CONFIGS[args.workload]
+    sample = OracleSample(cfg, 8, 8, seed=0)
+    for _ in range(args.warmup):
+        sample.run()
+    times = [sample.run() for _ in range(args.steps)]
+    flops, desc = sample.flops, sample.desc
+    ms = 1e3 * sum(times) / len(times)
+    value = flops / (ms * 1e-3) / 1e12
+    cores = blas_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "k": cfg.k, "F": cfg.F,
+                       "n_chan": cfg.n_chan, "n_chan_f": cfg.n_chan_f, "sample": desc},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# -------------------------------------------------------------------- ours
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from train_alignment_b200 import binding as B
+    from train_alignment_b200 import layer as L
+    from train_alignment_b200 import workloads as W
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    B.load()
+    cfg = W.CONFIGS[args.workload]
+    inp = W.moe_layer_inputs(cfg, seed=rank, device=dev)
+    layer = L.build_layer(cfg, inp, dev)
+    x, logits = inp["x"], inp["logits"]
+    x_train = W.engine_drift(x, 1e-2, seed=rank, device=dev)
+    g_gu = W.random_bf16(layer.w_gu.shape, 100 + rank, 1e-3, dev)
+    g_d = W.random_bf16(layer.w_d.shape, 200 + rank, 1e-3, dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        layer.step(x, logits, x_train, g_gu, g_d)
+    torch.cuda.synchronize()
+    assert B.device_status() == B.OK, B.last_error()
+    rpad = int(layer.expert_off[-1].item())
+
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:  # noqa: BLE001
+        pass
+    clocks = ClockSampler(uuid)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    launches0 = B.launch_count()
+    timers = []
+    for _ in range(args.steps):
+        flush.zero_()                                   # L2 flush, outside the events
+        t = L.StageTimer(True)
+        layer.step(x, logits, x_train, g_gu, g_d, timer=t)
+        timers.append(t)
+    torch.cuda.synchronize()
+    barrier()
+    launches = B.launch_count() - launches0
+    clk = clocks.stop()
+    assert B.device_status() == B.OK, B.last_error()
+    step_ms = [t.marks[0][1].elapsed_time(t.marks[-1][1]) for t in timers]
+    ms = sum(step_ms) / len(step_ms)
+    per_kernel = {}
+    for t in timers:
+        for name, v in t.durations_ms().items():
+            per_kernel[name] = per_kernel.get(name, 0.0) + v / len(timers)
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    fp4, comp = gemm_flops(cfg)
+    value = world * (fp4 + comp) / (ms * 1e-3) / 1e12
+
+    # roofline of the dominant kernel
+    peaks, peak_src = load_peaks()
+    work = kernel_work(cfg, rpad)
+    dom = max(per_kernel, key=per_kernel.get)
+    bound, amount = work[dom]
+    dur = per_kernel[dom] * 1e-3
+    if bound == "hbm":
+        achieved, peak, unit = amount / dur / 1e9, peaks["hbm_gbs"], "GB/s"
+    else:
+        achieved, peak, unit = amount / dur / 1e12, peaks["bf16_tflops_sustained"] * FP4_OVER_BF16, "TFLOP/s"
+    kernels = {}
+    for name, dms in per_kernel.items():
+        b, a = work.get(name, ("hbm", 0.0))
+        if b == "hbm":
+            kernels[name] = {"ms": dms, "GB/s": a / (dms * 1e-3) / 1e9, "frac_hbm": a / (dms * 1e-3) / 1e9 /
+                             peaks["hbm_gbs"]}
+        else:
+            tf = a / (dms * 1e-3) / 1e12
+            kernels[name] = {"ms": dms, "TFLOP/s": tf, "frac_fp4": tf / (peaks["bf16_tflops_sustained"] *
+                                                                          FP4_OVER_BF16)}
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as f:
+            traffic = json.load(f).get(f"{cfg.name}:{dom}")
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        x_h = x.cpu().pin_memory()
+        l_h = logits.cpu().pin_memory()
+        xt_h = x_train.cpu().pin_memory()
+        out_h = torch.empty(tuple(layer.out.shape), dtype=torch.bfloat16).pin_memory()
+        cnt_h = torch.empty(2, dtype=torch.int64).pin_memory()
+        x_d, l_d, xt_d = torch.empty_like(x), torch.empty_like(logits), torch.empty_like(x_train)
+        e_times = []
+        for i in range(args.warmup + args.steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            x_d.copy_(x_h, non_blocking=True)
+            l_d.copy_(l_h, non_blocking=True)
+            xt_d.copy_(xt_h, non_blocking=True)
+            out = layer.step(x_d, l_d, xt_d, g_gu, g_d)
+            out_h.copy_(out, non_blocking=True)
+            cnt_h.copy_(layer.counts, non_blocking=True)
+            e1.record()
+            e1.synchronize()
+            if i >= args.warmup:
+                e_times.append(e0.elapsed_time(e1))
+        e_ms = sum(e_times) / len(e_times)
+        if world > 1:
+            tt = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e_ms = float(tt.item())
+        h2d = x.numel() * 2 + logits.numel() * 4 + x_train.numel() * 2
+        d2h = layer.out.numel() * 2 + 16
+        e2e = {"value": world * (fp4 + comp) / (e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e_ms,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        sample = OracleSample(cfg, 1, 1, seed=0)
+        dt, flops, desc = sample.run(), sample.flops, sample.desc
+        cpu = {"value": flops / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": desc + f"; {dt:.1f} s", "seconds": dt}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "nvfp4(e2m1+e4m3)/bf16", "data": "synthetic",
+        "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "k": cfg.k, "F": cfg.F,
+                   "n_chan": cfg.n_chan, "n_chan_f": cfg.n_chan_f, "rows_padded": rpad,
+                   "parallelism": f"dp{world} (replicas, no collective)",
+                   "l2": "flushed between steps (256 MiB memset outside the timed events)",
+                   "gemm_flops_per_step": fp4 + comp},
+        "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"{peak_src}" + (" (bf16 sustained x 4)" if bound == "tensor" else "")},
+        "kernels": kernels,
+        "clocks": clk,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,338 @@
+/*
+ * quads.h -- C ABI of libquads.so: the NVFP4 Mixture-of-Experts expert layer
+ * of RL rollout/trainer alignment, as hand-written CUDA for sm_100a (B200).
+ *
+ * Sources cited below by short tag:
+ *   [QUADS-fr] "QUADS: Stabilizing NVFP4 Reinforcement Learning for MoE via
+ *              QUantization-error Alignment across Dual Sides", gist.science
+ *              French summary, "Résumé Technique" sections 1-5.
+ *   [QUADS-es] the same paper, gist.science Spanish summary, sections 1-5.
+ *   [TRACE]    "TRACE : un entraînement conscient de la quantification guidé
+ *              par le rollout pour le RL en FP4 des modèles MoE", sns.style.
+ *   [format]   the public NVFP4 format: E2M1 elements, one E4M3 scale per 16
+ *              consecutive elements along K, one FP32 per-tensor scale.
+ *
+ * Conventions (all entry points):
+ *   - Pointers named in comments as "device" point to GPU memory owned by the
+ *     caller; the library keeps no reference after the call is enqueued.
+ *     The library allocates no memory: calls that need scratch take a
+ *     caller-provided workspace whose size a *_workspace_bytes() query gives.
+ *   - Every call is asynchronous on the given stream (NULL = legacy default
+ *     stream) and does not synchronize, except quads_device_status().
+ *   - BF16 tensors are passed as uint16_t bit patterns; E2M1 codes are packed
+ *     two per byte (element 2j in the low nibble of byte j); E4M3 block scales
+ *     are one byte each.
+ *   - Scale layouts: QUADS_SCALES_LINEAR = [rows][K/16] row-major;
+ *     QUADS_SCALES_TILED = the tensor-core layout: tiles of 128 rows x 4
+ *     scales (512 bytes) in row-major tile order, rows padded to a multiple
+ *     of 128 and K/16 to a multiple of 4 with zero scales; inside a tile row r
+ *     and scale column c sit at byte (r % 32) * 16 + (r / 32) * 4 + c.
+ *     quads_scales_bytes() gives the size of either layout.
+ *   - Arguments are validated on the host before anything is launched. A
+ *     negative return value is an error; quads_last_error() (thread-local)
+ *     describes the last one.  Launch failures return QUADS_ERR_CUDA.
+ *   - The per-tensor scale g is a decode scale: value = e2m1 * e4m3 * g, with
+ *     g = fp32(amax / 2688) (2688 = 6 * 448).  Element codes are
+ *     E2M1_RNE(fp32(x * fp32(1 / fp32(e4m3 * g)))) and the block scale is
+ *     E4M3_RN_satfinite(fp32(amax_block / fp32(6 * g))).  A block whose scale
+ *     is 0 gets signed-zero codes.  Inputs must be finite; a tensor amax must
+ *     be 0 or at least 2^-100.
+ */
+#ifndef QUADS_H
+#define QUADS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* quads_stream_t;   /* a cudaStream_t */
+
+enum {
+  QUADS_OK = 0,
+  QUADS_ERR_INVALID_ARG = -1,       /* null pointer, negative or inconsistent size, misalignment */
+  QUADS_ERR_UNSUPPORTED_SHAPE = -2, /* a size outside what the kernels support */
+  QUADS_ERR_CUDA = -3,              /* a CUDA runtime/launch error */
+  QUADS_ERR_TIMEOUT = -4,           /* a bounded device-side wait gave up */
+  QUADS_ERR_BAD_RECORD = -5         /* a TRACE record failed validation */
+};
+
+enum { QUADS_SCALES_LINEAR = 0, QUADS_SCALES_TILED = 1 };
+enum { QUADS_OUT_BF16 = 0, QUADS_OUT_F32 = 1 };
+
+/* Message of the last error on this thread ("" if none). */
+const char* quads_last_error(void);
+/* ABI version of this header (1). */
+int quads_abi_version(void);
+/* Number of kernels this library has launched in this process. */
+uint64_t quads_launch_count(void);
+/* Synchronizes the stream, then returns QUADS_ERR_TIMEOUT if a kernel of this
+ * library recorded a timed-out wait on the current device since the last call
+ * (and clears the record), QUADS_OK otherwise. */
+int quads_device_status(quads_stream_t stream);
+/* Self-test of the bounded waits: launches one block that waits on a barrier
+ * nothing will complete, with the given limit in nanoseconds (<= 10 s); the
+ * wait gives up, records a timeout and the kernel returns.  A following
+ * quads_device_status() returns QUADS_ERR_TIMEOUT. */
+int quads_selftest_bounded_wait(uint64_t timeout_ns, quads_stream_t stream);
+
+/* Bytes of a scale array of `rows` x K/16 scales in the given layout. */
+size_t quads_scales_bytes(int64_t rows, int64_t K, int scale_layout);
+
+/* ---------------------------------------------------------------- a1: amax
+ * Per-group max |x| of a BF16 matrix (the tensor statistic behind the FP32
+ * per-tensor scale, [format]).  Rows are split into groups either by
+ * group_off (device int32 [n_groups + 1], ascending, group_off[0] = 0) or,
+ * when group_off is NULL, into n_groups groups of rows / n_groups rows each.
+ * amax_out: device float[n_groups], overwritten.  K % 16 == 0, ld_x >= K,
+ * ld_x % 8 == 0, x 16-byte aligned. */
+int quads_amax_bf16(const uint16_t* x, int64_t rows, int64_t K, int64_t ld_x,
+                    const int32_t* group_off, int n_groups, float* amax_out,
+                    quads_stream_t stream);
+
+/* ------------------------------------------------- a2 + a3: NVFP4 quantize
+ * NVFP4-quantizes a BF16 matrix x [rows][K] (row stride ld_x elements) with
+ * one per-tensor scale per row group (see quads_amax_bf16 for groups).
+ * [TRACE] "Fonctionnement": block scaling, one 4-bit value per element, the
+ * rounding direction a discrete choice; [format] block = 16 elements along
+ * K, E4M3 scale, FP32 tensor scale; [QUADS-fr §2.2.B] the residual of the
+ * high-residual channels feeds the rollout's compensation.
+ *   amax_in   device float[n_groups] calibrated amax, or NULL: the amax is
+ *             computed from x first (needs the workspace).
+ *   codes     device uint8 [rows][K/2], packed E2M1.
+ *   scales    device uint8, quads_scales_bytes(rows, K, scale_layout) bytes.
+ *   g_out     device float[n_groups]: the per-tensor decode scales.
+ *   chan      device int32[n_chan] or NULL: the compensation channels, valid
+ *             entries (0 <= c < K) strictly ascending and first, then -1
+ *             padding.  n_chan <= 256.
+ *   resid_out device uint16 (BF16) [rows][n_chan] or NULL:
+ *             r = bf16(fp32(x - fp32(deq(q(x))))) on each channel, 0 on padding.
+ *   ws        device workspace of quads_quantize_workspace_bytes(n_groups)
+ *             bytes (may be NULL when amax_in is given).
+ * Constraints: K % 16 == 0, K <= 65536, n_groups >= 1 (<= 1024 with
+ * group_off), rows >= 0. */
+size_t quads_quantize_workspace_bytes(int n_groups);
+int quads_quantize_nvfp4(const uint16_t* x, int64_t rows, int64_t K, int64_t ld_x,
+                         const int32_t* group_off, int n_groups, const float* amax_in,
+                         uint8_t* codes, uint8_t* scales, int scale_layout, float* g_out,
+                         const int32_t* chan, int n_chan, uint16_t* resid_out,
+                         void* ws, size_t ws_bytes, quads_stream_t stream);
+
+/* --------------------------------------------------------------- dequant
+ * deq = e2m1 * e4m3 * g of a quantized matrix (the rollout's weight or
+ * activation as the trainer sees it, [QUADS-fr §2.1]).  g: device
+ * float[n_groups] (groups as in quads_amax_bf16).  out: device BF16 or FP32
+ * [rows][K] per out_dtype (QUADS_OUT_BF16 rounds the FP32 value to BF16). */
+int quads_dequant(const uint8_t* codes, const uint8_t* scales, int scale_layout,
+                  const float* g, const int32_t* group_off, int n_groups,
+                  int64_t rows, int64_t K, void* out, int out_dtype,
+                  quads_stream_t stream);
+
+/* ---------------------------------------------- calibration of the channels
+ * [QUADS-fr §2.2.B]: a binary mask picks the channels with the largest
+ * residual magnitude.  scores: device float[K], score_c = sum over rows of
+ * |fp32(x - fp32(deq(q(x))))| for the tensor's own quantization (amax_in as
+ * in quads_quantize_nvfp4), summed in a fixed order.  Needs
+ * quads_channel_scores_workspace_bytes(rows, K) bytes of workspace. */
+size_t quads_channel_scores_workspace_bytes(int64_t rows, int64_t K);
+int quads_channel_scores(const uint16_t* x, int64_t rows, int64_t K, const float* amax_in,
+                         float* scores, void* ws, size_t ws_bytes, quads_stream_t stream);
+/* The n_sel channels with the largest score (ties: lower index), written to
+ * chan_out (device int32[n_sel]) in ascending channel order.  K <= 16384. */
+int quads_select_channels(const float* scores, int64_t K, int n_sel, int32_t* chan_out,
+                          quads_stream_t stream);
+
+/* ------------------------------------------------------------ a4: router
+ * Top-k experts per token from FP32 logits [T][E] (E <= 256, k <= 8,
+ * k <= E): experts ordered by (logit desc, index asc).  topk_w = softmax
+ * over the k selected logits (renorm = 1) or the full softmax at the
+ * selected experts (renorm = 0).  The router's choice is discrete
+ * ([TRACE] "Fonctionnement").  topk_idx: device int32 [T][k]; topk_w:
+ * device float [T][k]. */
+int quads_moe_router_topk(const float* logits, int64_t T, int E, int k, int renorm,
+                          int32_t* topk_idx, float* topk_w, quads_stream_t stream);
+
+/* ------------------------------------------------------- a5: permutation
+ * Stable counting sort of the (token, slot) pairs by expert, in increasing
+ * token * k + slot order, each expert's segment padded to a multiple of 128
+ * rows.  Outputs (device): expert_off int32[E + 1]; row_of int32[T * k] (the
+ * expert-ordered row of each pair); src_of int32[rows_cap] (the token of each
+ * expert-ordered row, -1 on pad rows; rows >= expert_off[E] are untouched).
+ * rows_cap = quads_moe_rows_capacity(T, k, E) bounds expert_off[E].
+ * Workspace: quads_moe_permute_workspace_bytes(T, k, E). */
+int64_t quads_moe_rows_capacity(int64_t T, int k, int E);
+size_t quads_moe_permute_workspace_bytes(int64_t T, int k, int E);
+int quads_moe_permute(const int32_t* topk_idx, int64_t T, int k, int E,
+                      int32_t* expert_off, int32_t* row_of, int32_t* src_of,
+                      void* ws, size_t ws_bytes, quads_stream_t stream);
+/* Gathers the quantized activation rows into expert order: pa_codes
+ * [rows_cap][K/2], pa_scales (tiled layout over rows_cap rows) and pa_resid
+ * [rows_cap][n_chan] from a_codes [T][K/2], a_scales (linear layout) and
+ * a_resid [T][n_chan] (both resid pointers NULL when n_chan == 0).  Pad rows
+ * get zero codes, scales and residuals.  K % 64 == 0. */
+int quads_moe_gather(const int32_t* src_of, const int32_t* expert_off, int E, int64_t rows_cap,
+                     const uint8_t* a_codes, const uint8_t* a_scales, int64_t K,
+                     const uint16_t* a_resid, int n_chan,
+                     uint8_t* pa_codes, uint8_t* pa_scales, uint16_t* pa_resid,
+                     quads_stream_t stream);
+/* Router + permutation + gather in one call (same arguments as above). */
+int quads_moe_route_permute(const float* logits, int64_t T, int E, int k, int renorm,
+                            int32_t* topk_idx, float* topk_w, int32_t* expert_off,
+                            int32_t* row_of, int32_t* src_of, int64_t rows_cap,
+                            const uint8_t* a_codes, const uint8_t* a_scales, int64_t K,
+                            const uint16_t* a_resid, int n_chan,
+                            uint8_t* pa_codes, uint8_t* pa_scales, uint16_t* pa_resid,
+                            void* ws, size_t ws_bytes, quads_stream_t stream);
+
+/* -------------------------------- a6: NVFP4 grouped GEMM + compensation
+ * For every expert e and its rows [off[e], off[e+1]) of the expert-ordered
+ * activations ([QUADS-fr §1] native W4A4 GEMM; [QUADS-fr §2.2.B] the
+ * residual correction added to the quantized output):
+ *   Y[r][n] = g_a(e) * g_w[e] * sum_k e2m1(A)e4m3(A) * e2m1(W_e)e4m3(W_e)
+ *           + sum_j a_resid[r][j] * w_resid[e][n][j]
+ * accumulated in FP32 on the tensor cores (tcgen05 block-scaled FP4 MMA for
+ * the first term, BF16 MMA for the second), stored as BF16.
+ *   a_codes  [rows_cap][K/2], a_scales tiled over rows_cap rows;
+ *   g_a      device float[E] if g_a_per_expert else float[1];
+ *   w_codes  [E][N][K/2] (row n = output feature n), w_scales tiled over
+ *            E*N rows; g_w device float[E];
+ *   expert_off device int32[E + 1], 128-row aligned, expert_off[E] <= rows_cap;
+ *   a_resid  [rows_cap][n_chan] BF16, w_resid [E][N][n_chan] BF16 (both NULL
+ *            when n_chan == 0);
+ *   y        [rows_cap][N] BF16; rows >= expert_off[E] are untouched.
+ * Constraints: 1 <= E <= 256, N % 128 == 0, K % 64 == 0, rows_cap % 128 == 0,
+ * n_chan % 16 == 0, n_chan <= 128; all matrix pointers 16-byte aligned.
+ * A device wait that exceeds ~4 s records a timeout (quads_device_status). */
+int quads_moe_grouped_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales,
+                                 const float* g_a, int g_a_per_expert,
+                                 const uint8_t* w_codes, const uint8_t* w_scales, const float* g_w,
+                                 const int32_t* expert_off, int E, int64_t rows_cap,
+                                 int64_t N, int64_t K,
+                                 const uint16_t* a_resid, const uint16_t* w_resid, int n_chan,
+                                 uint16_t* y, quads_stream_t stream);
+
+/* --------------------------------------------------------- a7: SwiGLU
+ * h[r][j] = bf16(silu(Y[r][j]) * Y[r][F + j]) for rows r < expert_off[E],
+ * silu(v) = v / (1 + exp(-v)), computed in FP32 from the BF16 gate/up GEMM
+ * output y [rows_cap][2F].  amax_out (device float[E], nullable, overwritten)
+ * receives the per-expert max |h| for the re-quantization of h.  F % 8 == 0. */
+int quads_swiglu(const uint16_t* y, int64_t rows_cap, int64_t F,
+                 const int32_t* expert_off, int E, uint16_t* h, float* amax_out,
+                 quads_stream_t stream);
+
+/* --------------------------------------------------------- a8: combine
+ * out[t] = bf16(sum over s = 0..k-1 of topk_w[t][s] * Y[row_of[t*k + s]]),
+ * FP32 accumulation in slot order.  y [rows_cap][H], out [T][H], H % 8 == 0. */
+int quads_moe_unpermute_combine(const uint16_t* y, const int32_t* row_of, const float* topk_w,
+                                int64_t T, int k, int64_t H, uint16_t* out,
+                                quads_stream_t stream);
+
+/* ------------------------------------------ a9: weight fake-quant + STE
+ * [QUADS-fr §2.2.A] asymmetric W4A16 QAT: the trainer's forward sees its
+ * BF16 master weights fake-quantized onto the rollout's NVFP4 grid
+ * ([QUADS-fr §2.1]: the same quantize-dequantize path as the rollout).  One
+ * pass over n_mat matrices [rows][K] (one per-tensor scale each) writes:
+ *   w_fq     BF16 [n_mat][rows][K]: bf16(e2m1 * e4m3 * g) if fold_global,
+ *            else the exact e2m1 * e4m3 (g then applies to the matmul output);
+ *   codes    (nullable) packed E2M1 [n_mat][rows][K/2] -- the rollout's
+ *            weights, identical to quads_quantize_nvfp4 of the same matrix;
+ *   scales   (nullable) tiled layout over n_mat * rows rows (rows % 128 == 0)
+ *            or linear when rows % 128 != 0;
+ *   g_out    device float[n_mat];
+ *   w_chan   (nullable) BF16 [n_mat][rows][n_chan]: the compensation weight
+ *            operand, column chan[j] of bf16(deq(W)) (chan_raw = 0) or of the
+ *            input W itself (chan_raw = 1); 0 on padding channels.
+ *   amax_in  device float[n_mat] per-matrix amax (e.g. from quads_amax_bf16),
+ *            or NULL: computed first, which needs the workspace of
+ *            quads_quantize_workspace_bytes(n_mat) bytes. */
+int quads_fakequant_weight_ste(const uint16_t* w, int64_t n_mat, int64_t rows, int64_t K,
+                               const float* amax_in, int fold_global, uint16_t* w_fq,
+                               uint8_t* codes, uint8_t* scales, float* g_out,
+                               const int32_t* chan, int n_chan, int chan_raw, uint16_t* w_chan,
+                               void* ws, size_t ws_bytes, quads_stream_t stream);
+/* Straight-through backward: grad_w = grad_wfq (accumulate = 0) or
+ * grad_w = bf16(fp32(grad_w + grad_wfq)) (accumulate = 1); n BF16 elements. */
+int quads_fakequant_weight_ste_backward(const uint16_t* grad_wfq, uint16_t* grad_w, int64_t n,
+                                        int accumulate, quads_stream_t stream);
+
+/* ------------------------------------------- a10 + a11: TRACE record
+ * [TRACE] "L'idée centrale": the rollout records its quantization results of
+ * the deep layers (mantissa and scale factors) and the trainer reproduces
+ * that rounding; "Impact": the engine exports, the trainer consumes.
+ *
+ * One record per layer: a header followed by 256-byte aligned sections.  A
+ * record holds up to two quantized tensors (slot 0: the gate/up GEMM input
+ * X in token order; slot 1: the down GEMM input h in expert order) and the
+ * router's top-k indices.  All offsets are bytes from the record start. */
+#define TRACE_QRECORD_MAGIC 0x31434552u   /* "REC1" little-endian */
+#define TRACE_QRECORD_VERSION 1u
+#define TRACE_MAX_TENSORS 2
+
+typedef struct trace_qtensor_desc {
+  int64_t rows, K;
+  int32_t n_groups;        /* per-tensor scales (1, or one per expert) */
+  int32_t n_chan;          /* compensation channels (0: none) */
+  int32_t scale_layout;    /* QUADS_SCALES_LINEAR / QUADS_SCALES_TILED */
+  int32_t present;         /* 1 if this slot holds a tensor */
+  uint64_t codes_off, scales_off, g_off, group_off_off, chan_off, resid_off;
+  uint64_t codes_bytes, scales_bytes;
+} trace_qtensor_desc;
+
+typedef struct trace_qrecord_header {
+  uint32_t magic, version;
+  int32_t layer_id;
+  int32_t k;               /* experts per token (0: no routing section) */
+  int64_t T;               /* tokens */
+  uint64_t total_bytes;
+  uint64_t topk_idx_off;   /* int32 [T][k] */
+  trace_qtensor_desc t[TRACE_MAX_TENSORS];
+} trace_qrecord_header;
+
+/* What one slot of a record holds, as device pointers (all owned by the
+ * caller): codes, scales, g[n_groups], group_off[n_groups + 1] (NULL when
+ * n_groups == 1), chan[n_chan] and resid[rows][n_chan] (NULL when
+ * n_chan == 0). */
+typedef struct trace_qtensor_src {
+  int64_t rows, K;
+  int32_t n_groups, n_chan, scale_layout, present;
+  const uint8_t* codes;
+  const uint8_t* scales;
+  const float* g;
+  const int32_t* group_off;
+  const int32_t* chan;
+  const uint16_t* resid;
+} trace_qtensor_src;
+
+/* Fills *hdr (host memory) with the layout of a record for these tensors and
+ * returns its total size in bytes (0 on invalid arguments). */
+size_t trace_qrecord_layout(int layer_id, int64_t T, int k,
+                            const trace_qtensor_src* tensors, int n_tensors,
+                            trace_qrecord_header* hdr);
+/* Writes the record (header + copies of every section) into `record`
+ * (device, record_bytes >= trace_qrecord_layout(...), 256-byte aligned).
+ * topk_idx: device int32 [T][k] or NULL when k == 0. */
+int trace_export_qrecord(int layer_id, int64_t T, int k, const int32_t* topk_idx,
+                         const trace_qtensor_src* tensors, int n_tensors,
+                         void* record, size_t record_bytes, quads_stream_t stream);
+/* Trainer replay of slot `which` of a record (device memory):
+ *   x_hat [rows][K] BF16 = bf16(fp32(deq) + r) on the compensation channels,
+ *         bf16(deq) elsewhere -- the operand the rollout's compensated GEMM
+ *         effectively used;
+ *   x_train (nullable) BF16 [rows][K]: the trainer's own activation; its
+ *         quantization with the recorded per-tensor scale is compared with
+ *         the record, and the numbers of differing element codes and block
+ *         scales are added to counts[0] and counts[1] (device uint64[2]).
+ * The record is validated on the device (magic, version, layer id, slot,
+ * shape, bounds within record_bytes); a bad record writes nothing and sets
+ * *status (device int32) to QUADS_ERR_BAD_RECORD, else *status = 0. */
+int trace_replay_qrecord(const void* record, size_t record_bytes, int layer_id, int which,
+                         int64_t rows, int64_t K, const uint16_t* x_train,
+                         uint16_t* x_hat, unsigned long long* counts, int32_t* status,
+                         quads_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QUADS_H */

@@ -1,0 +1,53 @@
+"""Test-side conversions between torch tensors and the oracle's numpy arrays,
+and the float tolerance.  Shared by the GPU parity tests; holds none of the
+method's arithmetic."""
+import numpy as np
+import torch
+
+from oracle import formats as F
+
+
+def bf16_np(t):
+    """BF16 torch tensor (any device) -> float64 numpy array of its values."""
+    return t.detach().to("cpu").to(torch.float32).numpy().astype(np.float64)
+
+
+def bf16_torch(a, device="cuda"):
+    """float64 numpy array of BF16-exact values -> BF16 torch tensor."""
+    return torch.from_numpy(np.asarray(a, dtype=np.float32)).to(torch.bfloat16).to(device)
+
+
+def u8_np(t):
+    return t.detach().to("cpu").numpy().astype(np.uint8)
+
+
+def unpack_codes(packed_t):
+    return F.unpack_nibbles(u8_np(packed_t))
+
+
+def assert_close_tol(got, ref, absdot, rel=1e-2, dot=1e-3, what=""):
+    """Per-element |got - ref| <= rel*|ref| + dot*sum|a*b| (the float parity bar)."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    bound = rel * np.abs(ref) + dot * np.asarray(absdot, dtype=np.float64)
+    err = np.abs(got - ref)
+    bad = err > bound
+    if bad.any():
+        i = np.flatnonzero(bad.ravel())[:5]
+        raise AssertionError(f"{what}: {bad.sum()} of {bad.size} elements out of tolerance; "
+                             f"first: got {got.ravel()[i]}, ref {ref.ravel()[i]}, bound {bound.ravel()[i]}")
+
+
+def assert_bits_equal(got, ref, what=""):
+    got = np.asarray(got)
+    ref = np.asarray(ref)
+    assert got.shape == ref.shape, (what, got.shape, ref.shape)
+    bad = got != ref
+    if bad.any():
+        i = np.flatnonzero(bad.ravel())[:8]
+        raise AssertionError(f"{what}: {bad.sum()} of {bad.size} differ; first at {i}: got {got.ravel()[i]}, "
+                             f"ref {ref.ravel()[i]}")
+
+
+def f32_of(t):
+    return t.detach().to("cpu").numpy().astype(np.float64)

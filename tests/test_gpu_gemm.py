@@ -1,0 +1,130 @@
+"""The tcgen05 NVFP4 grouped GEMM with residual compensation against the CPU
+oracle: per element |err| <= 1e-2 |ref| + 1e-3 sum|a b| (compensation terms
+included).  Inputs (codes, scales, residuals, weights) come from the oracle's
+quantizer on seeded BF16 data."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import formats as F
+from oracle import moe as M
+from oracle import nvfp4 as Q
+from tests.helpers import assert_close_tol, bf16_np, bf16_torch
+from train_alignment_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+def _problem(counts, N, K, nc, seed, x_scale=1.0):
+    """Expert-ordered activations with the given per-expert row counts,
+    quantized by the oracle; weights per expert quantized by the oracle."""
+    r = np.random.default_rng(seed)
+    E = len(counts)
+    padded = [-(-c // 128) * 128 for c in counts]
+    off = np.concatenate([[0], np.cumsum(padded)]).astype(np.int32)
+    R = int(off[-1])
+    cap = R + 128                                    # spare rows past the last expert
+    x = np.zeros((cap, K))
+    for e in range(E):
+        x[off[e]:off[e] + counts[e]] = r.standard_normal((counts[e], K)) * x_scale
+    ch_out = r.choice(K, 3, replace=False)
+    x[:, ch_out] *= 16
+    x = F.bf16_rne(x.astype(np.float32))
+    a_c, a_s, g_a = Q.quantize(x[:R])
+    chan = Q.pad_channels(Q.select_channels(Q.channel_scores(x[:R]), nc - 5) if nc else np.zeros(0, int), 16) \
+        if nc else None
+    w = F.bf16_rne((r.standard_normal((E, N, K)) * 0.02).astype(np.float32))
+    wq = [Q.quantize(w[e]) for e in range(E)]
+    w_c = np.stack([q[0] for q in wq])
+    w_s = np.stack([q[1] for q in wq])
+    g_w = np.array([q[2] for q in wq])
+    resid = wc = None
+    if nc:
+        resid = Q.residual_channels(x[:R], a_c, a_s, g_a, chan)
+        wc = np.zeros((E, N, nc))
+        for e in range(E):
+            deq = F.bf16_rne(F.f32(Q.dequant(w_c[e], w_s[e], g_w[e])))
+            for j, c in enumerate(chan):
+                if c >= 0:
+                    wc[e, :, j] = deq[:, c]
+    return dict(E=E, N=N, K=K, nc=nc, off=off, cap=cap, R=R, a_c=a_c, a_s=a_s, g_a=g_a, w_c=w_c, w_s=w_s,
+                g_w=g_w, resid=resid, wc=wc)
+
+
+def _run_gpu(lib, p):
+    E, N, K, cap, R = p["E"], p["N"], p["K"], p["cap"], p["R"]
+    a_codes = np.zeros((cap, K // 2), np.uint8)
+    a_codes[:R] = F.pack_nibbles(p["a_c"])
+    a_scales = np.zeros((cap, K // 16), np.uint8)
+    a_scales[:R] = p["a_s"]
+    w_codes = F.pack_nibbles(p["w_c"])
+    w_scales = F.scales_to_tiled(p["w_s"].reshape(E * N, K // 16))
+    dev = "cuda"
+    args = dict(
+        a_codes=torch.from_numpy(a_codes).to(dev), a_scales=torch.from_numpy(F.scales_to_tiled(a_scales)).to(dev),
+        g_a=torch.tensor([p["g_a"]], dtype=torch.float32, device=dev),
+        w_codes=torch.from_numpy(np.ascontiguousarray(w_codes)).to(dev), w_scales=torch.from_numpy(w_scales).to(dev),
+        g_w=torch.tensor(p["g_w"], dtype=torch.float32, device=dev),
+        expert_off=torch.from_numpy(p["off"]).to(dev), E=E, rows_cap=cap, N=N, K=K)
+    if p["nc"]:
+        resid = np.zeros((cap, p["nc"]))
+        resid[:R] = p["resid"]
+        args["a_resid"] = bf16_torch(resid)
+        args["w_resid"] = bf16_torch(p["wc"])
+    y = torch.full((cap, N), float("nan"), dtype=torch.bfloat16, device=dev)
+    lib.moe_grouped_gemm_nvfp4(y=y, **args)
+    assert lib.device_status() == lib.OK
+    torch.cuda.synchronize()
+    return bf16_np(y)
+
+
+def _oracle(p):
+    return M.grouped_gemm(p["a_c"], p["a_s"], p["g_a"], p["w_c"], p["w_s"], p["g_w"], p["off"], p["resid"], p["wc"])
+
+
+@pytest.mark.parametrize("counts,N,K,nc", [
+    ([64], 128, 64, 0),                 # one tile, one MMA along K
+    ([100], 128, 256, 0),               # one stage
+    ([64], 512, 256, 16),               # the single-linear shape with compensation
+    ([130, 0, 257], 256, 512, 32),      # empty expert, ragged experts, two stages
+    ([128, 300], 128, 320, 16),         # partial last stage (K % 256 = 64)
+    ([500, 20, 1000, 3], 384, 1024, 64),
+    ([256], 128, 4096, 128),            # long K, widest compensation
+])
+def test_grouped_gemm_parity(cuda_lib, counts, N, K, nc):
+    p = _problem(counts, N, K, nc, seed=sum(counts) + N + K + nc)
+    got = _run_gpu(cuda_lib, p)
+    ref, absdot = _oracle(p)
+    R = p["R"]
+    assert_close_tol(got[:R], ref, absdot, what="grouped gemm")
+    assert np.all(np.isnan(got[R:])), "rows past expert_off[E] must be untouched"
+
+
+def test_compensation_changes_output(cuda_lib):
+    """The compensation term is really added: without it the result differs
+    from the compensated one by R . Wc."""
+    p = _problem([200, 90], 128, 256, 32, seed=99)
+    y1 = _run_gpu(cuda_lib, p)
+    p0 = dict(p, nc=0, resid=None, wc=None)
+    y0 = _run_gpu(cuda_lib, p0)
+    R = p["R"]
+    corr = np.zeros((R, 128))
+    for e in range(2):
+        lo, hi = p["off"][e], p["off"][e + 1]
+        corr[lo:hi] = p["resid"][lo:hi] @ p["wc"][e].T
+    assert_close_tol(y1[:R] - y0[:R], corr, np.abs(y1[:R]) + np.abs(y0[:R]) + 1e-3, rel=1e-2, dot=1e-2,
+                     what="compensation delta")
+
+
+def test_grouped_gemm_bench_layer_shape(cuda_lib):
+    """The gate/up GEMM of the 2048-token, 8-expert layer (N = 4096, K = 1024,
+    32 compensation channels) in full, with the layer's routing."""
+    cfg = W.MOE_T2048
+    r = np.random.default_rng(7)
+    l = W.router_logits(cfg.T, cfg.E, "normal", torch.Generator().manual_seed(1), "cpu").numpy()
+    idx, _ = M.router_topk(l.astype(np.float64), cfg.k)
+    counts = np.bincount(idx.ravel(), minlength=cfg.E).tolist()
+    p = _problem(counts, 2 * cfg.F, cfg.H, cfg.n_chan, seed=5)
+    got = _run_gpu(cuda_lib, p)
+    ref, absdot = _oracle(p)
+    assert_close_tol(got[:p["R"]], ref, absdot, what="gate/up gemm")

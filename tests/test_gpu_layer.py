@@ -1,0 +1,109 @@
+"""One full step of the 2048-token, 8-expert layer (hidden 1024, ffn 2048,
+32 + 32 compensation channels) on the GPU against the oracle's composition of
+the same steps on the same seeded inputs.
+
+Bit-exact: input quantization, residuals, routing, permutation, weight
+fake-quant / rollout weights / compensation columns, replayed operand and
+mismatch counts.  Float: the gate/up GEMM within the tolerance.  Past the
+first BF16 GEMM output the two paths can round an intermediate differently
+(FP32 vs FP64 accumulation order before the BF16 store), which can flip an
+NVFP4 code of h; those flips are counted and bounded, and the layer output is
+checked per element with the tolerance on all but a bounded fraction."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import formats as F
+from oracle import layer as OL
+from oracle import nvfp4 as Q
+from tests.helpers import (assert_bits_equal, assert_close_tol, bf16_np, f32_of, u8_np, unpack_codes)
+from train_alignment_b200 import layer as L
+from train_alignment_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def run(cuda_lib):
+    cfg = W.MOE_T2048
+    inp = W.moe_layer_inputs(cfg, seed=0, device="cpu")
+    r = np.random.default_rng(0)
+    chan_x = Q.pad_channels(np.sort(r.choice(cfg.H, cfg.n_chan - 3, replace=False)))
+    chan_h = Q.pad_channels(np.sort(r.choice(cfg.F, cfg.n_chan_f - 7, replace=False)))
+    x_train = W.engine_drift(inp["x"], 1e-2, seed=0)
+    dev = "cuda"
+    layer = L.MoELayer(cfg, inp["w_gu"].to(dev), inp["w_d"].to(dev), torch.from_numpy(chan_x),
+                       torch.from_numpy(chan_h), dev)
+    g_gu = W.random_bf16(layer.w_gu.shape, 1, 1e-3, dev)
+    g_d = W.random_bf16(layer.w_d.shape, 2, 1e-3, dev)
+    layer.reset_counts()
+    layer.step(inp["x"].to(dev), inp["logits"].to(dev), x_train.to(dev), g_gu, g_d)
+    assert cuda_lib.device_status() == cuda_lib.OK
+    torch.cuda.synchronize()
+    ref = OL.step(bf16_np(inp["x"]), inp["logits"].numpy().astype(np.float64), bf16_np(x_train),
+                  bf16_np(inp["w_gu"]), bf16_np(inp["w_d"]), chan_x, chan_h, cfg.k,
+                  grad_gu_fq=bf16_np(g_gu), grad_gu=np.zeros(tuple(layer.w_gu.shape)))
+    return cfg, layer, ref
+
+
+def test_weights(run):
+    cfg, layer, ref = run
+    E, F2, H = cfg.E, 2 * cfg.F, cfg.H
+    assert_bits_equal(unpack_codes(layer.w_gu_codes), ref["wgu"]["codes"], "w_gu codes")
+    s = F.scales_from_tiled(u8_np(layer.w_gu_scales), E * F2, H // 16).reshape(E, F2, H // 16)
+    assert_bits_equal(s, ref["wgu"]["scales"], "w_gu scales")
+    assert_bits_equal(f32_of(layer.g_w_gu).astype(np.float32), ref["wgu"]["g"].astype(np.float32), "g_w")
+    assert_bits_equal(F.bf16_bits(bf16_np(layer.w_gu_fq)), F.bf16_bits(ref["wgu"]["w_fq"]), "w_gu_fq")
+    assert_bits_equal(F.bf16_bits(bf16_np(layer.wc_gu)), F.bf16_bits(ref["wgu"]["wc"]), "wc_gu")
+    assert_bits_equal(unpack_codes(layer.w_d_codes), ref["wd"]["codes"], "w_d codes")
+    assert_bits_equal(F.bf16_bits(bf16_np(layer.wc_d)), F.bf16_bits(ref["wd"]["wc"]), "wc_d")
+
+
+def test_rollout_input_and_routing(run):
+    cfg, layer, ref = run
+    f = ref["fwd"]
+    assert_bits_equal(unpack_codes(layer.x_codes), f["cx"], "x codes")
+    assert_bits_equal(u8_np(layer.x_scales).reshape(cfg.T, cfg.H // 16), f["sx"], "x scales")
+    assert np.float32(f32_of(layer.g_x)[0]) == np.float32(f["gx"])
+    assert_bits_equal(F.bf16_bits(bf16_np(layer.x_resid)), F.bf16_bits(f["rx"]), "x resid")
+    assert_bits_equal(f32_of(layer.topk_idx).astype(np.int64), f["idx"].astype(np.int64), "topk idx")
+    assert np.allclose(f32_of(layer.topk_w), f["w"], rtol=2e-6)
+    assert_bits_equal(f32_of(layer.expert_off).astype(np.int64), f["off"].astype(np.int64), "expert_off")
+    assert_bits_equal(f32_of(layer.row_of).astype(np.int64), f["row_of"].astype(np.int64), "row_of")
+
+
+def test_gate_up_gemm(run):
+    cfg, layer, ref = run
+    f = ref["fwd"]
+    n = int(f["off"][-1])
+    assert_close_tol(bf16_np(layer.y_gu)[:n], f["y1"], f["absdot1"], what="gate/up GEMM")
+
+
+def test_h_and_output(run):
+    cfg, layer, ref = run
+    f = ref["fwd"]
+    n = int(f["off"][-1])
+    h = bf16_np(layer.h)[:n]
+    frac_h = np.mean(h != f["h"])
+    assert frac_h < 5e-3, f"h differs in {frac_h:.2e} of elements"
+    code_flip = np.mean(unpack_codes(layer.h_codes)[:n] != f["ch"])
+    assert code_flip < 5e-3, f"h codes differ in {code_flip:.2e} of elements"
+    out = bf16_np(layer.out)
+    err = np.abs(out - f["out"])
+    scale = np.abs(f["out"]) * 1e-2 + 1e-3 * np.sqrt(np.mean(f["out"] ** 2))
+    frac_bad = np.mean(err > scale)
+    assert frac_bad < 1e-2, f"{frac_bad:.2e} of outputs outside the tolerance"
+    rel = np.linalg.norm(out - f["out"]) / np.linalg.norm(f["out"])
+    assert rel < 1e-2, rel
+
+
+def test_replay(run):
+    cfg, layer, ref = run
+    assert int(layer.status.item()) == 0 and int(layer.status_h.item()) == 0
+    assert_bits_equal(F.bf16_bits(bf16_np(layer.x_hat)), F.bf16_bits(ref["x_hat"]), "x_hat")
+    assert f32_of(layer.counts).astype(np.int64).tolist() == [ref["code_mismatches"], ref["scale_mismatches"]]
+
+
+def test_ste(run):
+    cfg, layer, ref = run
+    assert_bits_equal(F.bf16_bits(bf16_np(layer.grad_gu)), F.bf16_bits(ref["grad"]), "grad_gu")

@@ -1,0 +1,401 @@
+"""Thin ctypes binding of libquads.so (the C ABI in include/quads.h).
+
+Argument marshalling only: every function passes torch tensors' device
+pointers, sizes and the current CUDA stream to the library and raises
+QuadsError on a non-zero status.  Output tensors are allocated with torch
+when the caller does not pass them.  There is no fallback: if the library is
+missing, load() raises.
+"""
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libquads.so")
+_lib = None
+
+OK = 0
+ERR_INVALID_ARG = -1
+ERR_UNSUPPORTED_SHAPE = -2
+ERR_CUDA = -3
+ERR_TIMEOUT = -4
+ERR_BAD_RECORD = -5
+SCALES_LINEAR = 0
+SCALES_TILED = 1
+OUT_BF16 = 0
+OUT_F32 = 1
+TRACE_MAX_TENSORS = 2
+
+c_i64, c_i32, c_sz, c_vp, c_u64 = ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_uint64
+
+
+class QuadsError(RuntimeError):
+    def __init__(self, code, where, msg):
+        super().__init__(f"{where} failed with status {code}: {msg}")
+        self.code = code
+
+
+class TraceQTensorDesc(ctypes.Structure):
+    _fields_ = [("rows", c_i64), ("K", c_i64), ("n_groups", ctypes.c_int32), ("n_chan", ctypes.c_int32),
+                ("scale_layout", ctypes.c_int32), ("present", ctypes.c_int32),
+                ("codes_off", c_u64), ("scales_off", c_u64), ("g_off", c_u64), ("group_off_off", c_u64),
+                ("chan_off", c_u64), ("resid_off", c_u64), ("codes_bytes", c_u64), ("scales_bytes", c_u64)]
+
+
+class TraceQRecordHeader(ctypes.Structure):
+    _fields_ = [("magic", ctypes.c_uint32), ("version", ctypes.c_uint32), ("layer_id", ctypes.c_int32),
+                ("k", ctypes.c_int32), ("T", c_i64), ("total_bytes", c_u64), ("topk_idx_off", c_u64),
+                ("t", TraceQTensorDesc * TRACE_MAX_TENSORS)]
+
+
+class TraceQTensorSrc(ctypes.Structure):
+    _fields_ = [("rows", c_i64), ("K", c_i64), ("n_groups", ctypes.c_int32), ("n_chan", ctypes.c_int32),
+                ("scale_layout", ctypes.c_int32), ("present", ctypes.c_int32),
+                ("codes", c_vp), ("scales", c_vp), ("g", c_vp), ("group_off", c_vp), ("chan", c_vp),
+                ("resid", c_vp)]
+
+
+_SIGS = {
+    "quads_last_error": (ctypes.c_char_p, []),
+    "quads_abi_version": (c_i32, []),
+    "quads_launch_count": (c_u64, []),
+    "quads_device_status": (c_i32, [c_vp]),
+    "quads_selftest_bounded_wait": (c_i32, [c_u64, c_vp]),
+    "quads_scales_bytes": (c_sz, [c_i64, c_i64, c_i32]),
+    "quads_amax_bf16": (c_i32, [c_vp, c_i64, c_i64, c_i64, c_vp, c_i32, c_vp, c_vp]),
+    "quads_quantize_workspace_bytes": (c_sz, [c_i32]),
+    "quads_quantize_nvfp4": (c_i32, [c_vp, c_i64, c_i64, c_i64, c_vp, c_i32, c_vp, c_vp, c_vp, c_i32, c_vp,
+                                     c_vp, c_i32, c_vp, c_vp, c_sz, c_vp]),
+    "quads_dequant": (c_i32, [c_vp, c_vp, c_i32, c_vp, c_vp, c_i32, c_i64, c_i64, c_vp, c_i32, c_vp]),
+    "quads_channel_scores_workspace_bytes": (c_sz, [c_i64, c_i64]),
+    "quads_channel_scores": (c_i32, [c_vp, c_i64, c_i64, c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "quads_select_channels": (c_i32, [c_vp, c_i64, c_i32, c_vp, c_vp]),
+    "quads_moe_router_topk": (c_i32, [c_vp, c_i64, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp]),
+    "quads_moe_rows_capacity": (c_i64, [c_i64, c_i32, c_i32]),
+    "quads_moe_permute_workspace_bytes": (c_sz, [c_i64, c_i32, c_i32]),
+    "quads_moe_permute": (c_i32, [c_vp, c_i64, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "quads_moe_gather": (c_i32, [c_vp, c_vp, c_i32, c_i64, c_vp, c_vp, c_i64, c_vp, c_i32, c_vp, c_vp, c_vp,
+                                 c_vp]),
+    "quads_moe_route_permute": (c_i32, [c_vp, c_i64, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_i64,
+                                        c_vp, c_vp, c_i64, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "quads_moe_grouped_gemm_nvfp4": (c_i32, [c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_i32, c_i64, c_i64,
+                                             c_i64, c_vp, c_vp, c_i32, c_vp, c_vp]),
+    "quads_swiglu": (c_i32, [c_vp, c_i64, c_i64, c_vp, c_i32, c_vp, c_vp, c_vp]),
+    "quads_moe_unpermute_combine": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i32, c_i64, c_vp, c_vp]),
+    "quads_fakequant_weight_ste": (c_i32, [c_vp, c_i64, c_i64, c_i64, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_i32,
+                                           c_i32, c_vp, c_vp, c_sz, c_vp]),
+    "quads_fakequant_weight_ste_backward": (c_i32, [c_vp, c_vp, c_i64, c_i32, c_vp]),
+    "trace_qrecord_layout": (c_sz, [c_i32, c_i64, c_i32, c_vp, c_i32, c_vp]),
+    "trace_export_qrecord": (c_i32, [c_i32, c_i64, c_i32, c_vp, c_vp, c_i32, c_vp, c_sz, c_vp]),
+    "trace_replay_qrecord": (c_i32, [c_vp, c_sz, c_i32, c_i32, c_i64, c_i64, c_vp, c_vp, c_vp, c_vp, c_vp]),
+}
+
+
+def load(path=None):
+    """Load libquads.so (raises if it is missing; there is no fallback)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    p = path or _LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(f"{p} is missing: build it with `python -m train_alignment_b200.build`")
+    lib = ctypes.CDLL(p)
+    for name, (res, args) in _SIGS.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = lib
+    return lib
+
+
+def exported_symbols():
+    return list(_SIGS)
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _s():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _check(rc, where):
+    if rc != OK:
+        raise QuadsError(rc, where, load().quads_last_error().decode())
+
+
+def _dev(t, dtype, name):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _bits(t):
+    """BF16 tensors travel as their uint16 bit patterns."""
+    return t
+
+
+def _empty(shape, dtype, device):
+    return torch.empty(shape, dtype=dtype, device=device)
+
+
+# ------------------------------------------------------------------ status
+
+
+def last_error():
+    return load().quads_last_error().decode()
+
+
+def launch_count():
+    return int(load().quads_launch_count())
+
+
+def device_status():
+    return int(load().quads_device_status(_s()))
+
+
+def selftest_bounded_wait(timeout_ns):
+    _check(load().quads_selftest_bounded_wait(int(timeout_ns), _s()), "quads_selftest_bounded_wait")
+
+
+def scales_bytes(rows, K, layout):
+    return int(load().quads_scales_bytes(rows, K, layout))
+
+
+# ---------------------------------------------------------------- quantize
+
+
+def quantize_workspace_bytes(n_groups):
+    return int(load().quads_quantize_workspace_bytes(n_groups))
+
+
+def amax_bf16(x, group_off=None, n_groups=1, out=None):
+    _dev(x, torch.bfloat16, "x")
+    rows, K = x.shape
+    out = out if out is not None else _empty((n_groups,), torch.float32, x.device)
+    _check(load().quads_amax_bf16(_p(x), rows, K, K, _p(group_off), n_groups, _p(out), _s()), "quads_amax_bf16")
+    return out
+
+
+def quantize_nvfp4(x, *, group_off=None, n_groups=1, amax_in=None, scale_layout=SCALES_LINEAR, chan=None,
+                   codes=None, scales=None, g_out=None, resid_out=None, ws=None):
+    """Returns (codes [rows, K/2] u8, scales u8, g [n_groups] f32, resid [rows, n_chan] bf16 or None)."""
+    _dev(x, torch.bfloat16, "x")
+    rows, K = x.shape
+    dev = x.device
+    n_chan = 0 if chan is None else int(chan.numel())
+    codes = codes if codes is not None else _empty((rows, K // 2), torch.uint8, dev)
+    scales = scales if scales is not None else _empty((scales_bytes(rows, K, scale_layout),), torch.uint8, dev)
+    g_out = g_out if g_out is not None else _empty((n_groups,), torch.float32, dev)
+    if n_chan and resid_out is None:
+        resid_out = _empty((rows, n_chan), torch.bfloat16, dev)
+    if amax_in is None and ws is None:
+        ws = _empty((quantize_workspace_bytes(n_groups),), torch.uint8, dev)
+    _check(load().quads_quantize_nvfp4(
+        _p(x), rows, K, K, _p(group_off), n_groups, _p(amax_in), _p(codes), _p(scales), scale_layout, _p(g_out),
+        _p(chan), n_chan, _p(resid_out) if n_chan else None, _p(ws), 0 if ws is None else ws.numel(), _s()),
+        "quads_quantize_nvfp4")
+    return codes, scales, g_out, (resid_out if n_chan else None)
+
+
+def dequant(codes, scales, scale_layout, g, rows, K, group_off=None, n_groups=1, out_dtype=OUT_BF16, out=None):
+    dt = torch.bfloat16 if out_dtype == OUT_BF16 else torch.float32
+    out = out if out is not None else _empty((rows, K), dt, codes.device)
+    _check(load().quads_dequant(_p(codes), _p(scales), scale_layout, _p(g), _p(group_off), n_groups, rows, K,
+                                _p(out), out_dtype, _s()), "quads_dequant")
+    return out
+
+
+def channel_scores(x, amax_in=None):
+    _dev(x, torch.bfloat16, "x")
+    rows, K = x.shape
+    ws = _empty((int(load().quads_channel_scores_workspace_bytes(rows, K)),), torch.uint8, x.device)
+    out = _empty((K,), torch.float32, x.device)
+    _check(load().quads_channel_scores(_p(x), rows, K, _p(amax_in), _p(out), _p(ws), ws.numel(), _s()),
+           "quads_channel_scores")
+    return out
+
+
+def select_channels(scores, n_sel):
+    out = _empty((n_sel,), torch.int32, scores.device)
+    _check(load().quads_select_channels(_p(scores), scores.numel(), n_sel, _p(out), _s()), "quads_select_channels")
+    return out
+
+
+# --------------------------------------------------------------------- MoE
+
+
+def moe_rows_capacity(T, k, E):
+    return int(load().quads_moe_rows_capacity(T, k, E))
+
+
+def moe_permute_workspace_bytes(T, k, E):
+    return int(load().quads_moe_permute_workspace_bytes(T, k, E))
+
+
+def moe_router_topk(logits, k, renorm=True, idx=None, w=None):
+    _dev(logits, torch.float32, "logits")
+    T, E = logits.shape
+    idx = idx if idx is not None else _empty((T, k), torch.int32, logits.device)
+    w = w if w is not None else _empty((T, k), torch.float32, logits.device)
+    _check(load().quads_moe_router_topk(_p(logits), T, E, k, 1 if renorm else 0, _p(idx), _p(w), _s()),
+           "quads_moe_router_topk")
+    return idx, w
+
+
+def moe_permute(topk_idx, E, expert_off=None, row_of=None, src_of=None, ws=None):
+    _dev(topk_idx, torch.int32, "topk_idx")
+    T, k = topk_idx.shape
+    dev = topk_idx.device
+    cap = moe_rows_capacity(T, k, E)
+    expert_off = expert_off if expert_off is not None else _empty((E + 1,), torch.int32, dev)
+    row_of = row_of if row_of is not None else _empty((T * k,), torch.int32, dev)
+    src_of = src_of if src_of is not None else _empty((cap,), torch.int32, dev)
+    ws = ws if ws is not None else _empty((moe_permute_workspace_bytes(T, k, E),), torch.uint8, dev)
+    _check(load().quads_moe_permute(_p(topk_idx), T, k, E, _p(expert_off), _p(row_of), _p(src_of), _p(ws),
+                                    ws.numel(), _s()), "quads_moe_permute")
+    return expert_off, row_of, src_of
+
+
+def moe_gather(src_of, expert_off, E, rows_cap, a_codes, a_scales, K, a_resid=None, pa_codes=None,
+               pa_scales=None, pa_resid=None):
+    dev = a_codes.device
+    n_chan = 0 if a_resid is None else a_resid.shape[1]
+    pa_codes = pa_codes if pa_codes is not None else _empty((rows_cap, K // 2), torch.uint8, dev)
+    pa_scales = pa_scales if pa_scales is not None else _empty((scales_bytes(rows_cap, K, SCALES_TILED),),
+                                                               torch.uint8, dev)
+    if n_chan and pa_resid is None:
+        pa_resid = _empty((rows_cap, n_chan), torch.bfloat16, dev)
+    _check(load().quads_moe_gather(_p(src_of), _p(expert_off), E, rows_cap, _p(a_codes), _p(a_scales), K,
+                                   _p(a_resid), n_chan, _p(pa_codes), _p(pa_scales),
+                                   _p(pa_resid) if n_chan else None, _s()), "quads_moe_gather")
+    return pa_codes, pa_scales, (pa_resid if n_chan else None)
+
+
+def moe_grouped_gemm_nvfp4(a_codes, a_scales, g_a, w_codes, w_scales, g_w, expert_off, E, rows_cap, N, K,
+                           a_resid=None, w_resid=None, y=None):
+    n_chan = 0 if a_resid is None else a_resid.shape[1]
+    y = y if y is not None else _empty((rows_cap, N), torch.bfloat16, a_codes.device)
+    per_expert = 1 if g_a.numel() == E and E > 1 else 0
+    _check(load().quads_moe_grouped_gemm_nvfp4(
+        _p(a_codes), _p(a_scales), _p(g_a), per_expert, _p(w_codes), _p(w_scales), _p(g_w), _p(expert_off), E,
+        rows_cap, N, K, _p(a_resid), _p(w_resid), n_chan, _p(y), _s()), "quads_moe_grouped_gemm_nvfp4")
+    return y
+
+
+def swiglu(y, F, expert_off, E, h=None, amax=None, want_amax=True):
+    rows_cap = y.shape[0]
+    h = h if h is not None else _empty((rows_cap, F), torch.bfloat16, y.device)
+    if want_amax and amax is None:
+        amax = _empty((E,), torch.float32, y.device)
+    _check(load().quads_swiglu(_p(y), rows_cap, F, _p(expert_off), E, _p(h), _p(amax) if want_amax else None,
+                               _s()), "quads_swiglu")
+    return h, (amax if want_amax else None)
+
+
+def moe_unpermute_combine(y, row_of, topk_w, T, k, H, out=None):
+    out = out if out is not None else _empty((T, H), torch.bfloat16, y.device)
+    _check(load().quads_moe_unpermute_combine(_p(y), _p(row_of), _p(topk_w), T, k, H, _p(out), _s()),
+           "quads_moe_unpermute_combine")
+    return out
+
+
+# ------------------------------------------------------------ fake-quant
+
+
+def fakequant_weight_ste(w, fold_global=True, chan=None, chan_raw=False, want_codes=True, w_fq=None, codes=None,
+                         scales=None, g_out=None, w_chan=None, ws=None, amax_in=None):
+    """w: [n_mat, rows, K] bf16.  Returns (w_fq, codes, scales, g, w_chan)."""
+    _dev(w, torch.bfloat16, "w")
+    n_mat, rows, K = w.shape
+    dev = w.device
+    n_chan = 0 if chan is None else int(chan.numel())
+    layout = SCALES_TILED if rows % 128 == 0 else SCALES_LINEAR
+    w_fq = w_fq if w_fq is not None else _empty((n_mat, rows, K), torch.bfloat16, dev)
+    if want_codes:
+        codes = codes if codes is not None else _empty((n_mat, rows, K // 2), torch.uint8, dev)
+        scales = scales if scales is not None else _empty((scales_bytes(n_mat * rows, K, layout),), torch.uint8,
+                                                          dev)
+    g_out = g_out if g_out is not None else _empty((n_mat,), torch.float32, dev)
+    if n_chan and w_chan is None:
+        w_chan = _empty((n_mat, rows, n_chan), torch.bfloat16, dev)
+    if amax_in is None and ws is None:
+        ws = _empty((quantize_workspace_bytes(n_mat),), torch.uint8, dev)
+    _check(load().quads_fakequant_weight_ste(
+        _p(w), n_mat, rows, K, _p(amax_in), 1 if fold_global else 0, _p(w_fq), _p(codes) if want_codes else None,
+        _p(scales) if want_codes else None, _p(g_out), _p(chan), n_chan, 1 if chan_raw else 0,
+        _p(w_chan) if n_chan else None, _p(ws), 0 if ws is None else ws.numel(), _s()),
+        "quads_fakequant_weight_ste")
+    return w_fq, (codes if want_codes else None), (scales if want_codes else None), g_out, \
+        (w_chan if n_chan else None)
+
+
+def fakequant_weight_ste_backward(grad_wfq, grad_w=None, accumulate=False):
+    grad_w = grad_w if grad_w is not None else torch.empty_like(grad_wfq)
+    _check(load().quads_fakequant_weight_ste_backward(_p(grad_wfq), _p(grad_w), grad_wfq.numel(),
+                                                      1 if accumulate else 0, _s()),
+           "quads_fakequant_weight_ste_backward")
+    return grad_w
+
+
+# ---------------------------------------------------------------- TRACE
+
+
+def qtensor_src(codes, scales, g, rows, K, scale_layout, group_off=None, chan=None, resid=None):
+    """Description of one recorded tensor (keeps the tensors alive via ._keep)."""
+    s = TraceQTensorSrc()
+    s.rows, s.K = rows, K
+    s.n_groups = int(g.numel())
+    s.n_chan = 0 if chan is None else int(chan.numel())
+    s.scale_layout = scale_layout
+    s.present = 1
+    s.codes, s.scales, s.g = codes.data_ptr(), scales.data_ptr(), g.data_ptr()
+    s.group_off = group_off.data_ptr() if (group_off is not None and s.n_groups > 1) else None
+    s.chan = chan.data_ptr() if s.n_chan else None
+    s.resid = resid.data_ptr() if s.n_chan else None
+    s._keep = (codes, scales, g, group_off, chan, resid)
+    return s
+
+
+def _src_array(tensors):
+    arr = (TraceQTensorSrc * TRACE_MAX_TENSORS)()
+    for i, t in enumerate(tensors):
+        if t is not None:
+            arr[i] = t
+    return arr
+
+
+def trace_qrecord_layout(layer_id, T, k, tensors):
+    hdr = TraceQRecordHeader()
+    arr = _src_array(tensors)
+    n = int(load().trace_qrecord_layout(layer_id, T, k, ctypes.cast(arr, c_vp), len(tensors), ctypes.byref(hdr)))
+    if n == 0:
+        raise QuadsError(ERR_INVALID_ARG, "trace_qrecord_layout", "invalid record description")
+    return n, hdr
+
+
+def trace_export_qrecord(layer_id, T, k, topk_idx, tensors, record=None):
+    n, _ = trace_qrecord_layout(layer_id, T, k, tensors)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    record = record if record is not None else _empty((n,), torch.uint8, dev)
+    arr = _src_array(tensors)
+    _check(load().trace_export_qrecord(layer_id, T, k, _p(topk_idx), ctypes.cast(arr, c_vp), len(tensors),
+                                       _p(record), record.numel(), _s()), "trace_export_qrecord")
+    return record
+
+
+def trace_replay_qrecord(record, layer_id, which, rows, K, x_train=None, x_hat=None, counts=None, status=None):
+    dev = record.device
+    x_hat = x_hat if x_hat is not None else _empty((rows, K), torch.bfloat16, dev)
+    if x_train is not None and counts is None:
+        counts = torch.zeros(2, dtype=torch.int64, device=dev)
+    status = status if status is not None else _empty((1,), torch.int32, dev)
+    _check(load().trace_replay_qrecord(_p(record), record.numel(), layer_id, which, rows, K, _p(x_train),
+                                       _p(x_hat), _p(counts), _p(status), _s()), "trace_replay_qrecord")
+    return x_hat, counts, status

@@ -1,0 +1,578 @@
+// NVFP4 grouped expert GEMM with QUADS residual compensation, for sm_100a.
+//
+// Method: the rollout runs its MoE expert GEMMs as native NVFP4 W4A4
+// ([QUADS-fr §1]); on the high-residual input channels a correction term is
+// computed and added to the quantized output, so that the W4A4 GEMM still
+// does the bulk of the work ([QUADS-fr §2.2.B], [QUADS-es §2.2.B]):
+//   Y = g_a g_w (A_fp4 (x) W_fp4) + R_C . Wc
+//
+// Design (one persistent CTA per SM, 192 threads, warp-specialized):
+//   warp 0 lane 0  TMA producer: 128x256 FP4 tiles of A and W (128-byte
+//                  swizzle) and their 512-byte block-scale tiles (bulk copy)
+//                  into a multi-stage shared-memory ring; per output tile the
+//                  BF16 compensation operands R [128 x |C|] and Wc [128 x |C|]
+//                  (32-byte swizzle, 16 channels per box).
+//   warp 1         allocates 512 TMEM columns; lane 0 issues tcgen05.cp of the
+//                  scales into TMEM and tcgen05.mma kind::mxf4nvf4 (block16
+//                  E4M3 scales, K = 64 per instruction) into a double-buffered
+//                  FP32 accumulator, then tcgen05.mma kind::f16 (BF16) for
+//                  R_C . Wc into a second accumulator.
+//   warps 2..5     epilogue: tcgen05.ld both accumulators, y = G * acc + comp,
+//                  BF16 stores.
+// TMEM columns: [0,128) and [128,256) main accumulators, [256,384) the
+// compensation accumulator, [384,448) two buffers of scale factors.
+// Tiles are (expert, 128-row block, 128-column block); experts' row segments
+// are 128-aligned by the permutation, so no tile straddles two experts.
+// No TMA multicast is used anywhere.
+//
+// Every wait on an mbarrier is bounded (a global-timer limit); on expiry the
+// kernel records a timeout in a device status word, lets in-flight copies and
+// MMAs finish (bounded again), frees its TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+
+namespace quads {
+
+__device__ unsigned int g_wait_status = 0u;
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 128;
+constexpr int kStageRowBytes = 128;                 // 256 FP4 elements per row per stage
+constexpr int kMmaKBytes = 32;                      // 64 FP4 elements per MMA
+constexpr int kABytes = BM * kStageRowBytes;        // 16384
+constexpr int kBBytes = BN * kStageRowBytes;        // 16384
+constexpr int kSfBytes = 4 * 512;                   // scales of 4 MMAs for 128 rows
+constexpr int kStageBytes = kABytes + kBBytes + 2 * kSfBytes;   // 36864
+constexpr int kCompChunkBytes = 128 * 32;           // 128 rows x 16 BF16
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kCompCol = 256;
+constexpr uint32_t kSfCol = 384;
+constexpr int kMaxStages = 8;
+constexpr int kMaxChan = 128;
+constexpr uint64_t kGemmTimeoutNs = 4000000000ull;
+constexpr uint64_t kDrainTimeoutNs = 500000000ull;
+
+// Instruction descriptors (tcgen05 "instruction descriptor" format):
+// kind::mxf4nvf4: A/B format E2M1 (1) at bits 7-9 / 10-12, K-major, N>>3 at
+// bit 17, scale format UE4M3 (0) at bit 23, M>>4 at bit 24, dense K = 64.
+constexpr uint32_t kIdescFp4 = (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+// kind::f16: D format F32 (1) at bits 4-5, A/B BF16 (1), K-major, N>>3, M>>4.
+constexpr uint32_t kIdescBf16 =
+    (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+
+struct GemmParams {
+  const uint8_t* a_scales;
+  const uint8_t* w_scales;
+  const float* g_a;
+  const float* g_w;
+  const int32_t* expert_off;
+  uint16_t* y;
+  int g_a_per_expert;
+  int E;
+  int N;
+  int K;
+  int n_chan;
+  int stages;
+  uint64_t timeout_ns;
+};
+
+// ------------------------------------------------------------ PTX wrappers
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t global_timer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase with the given parity.  Returns false if the
+// limit expired (recording a timeout and raising the CTA's abort flag) or if
+// another role already aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          uint64_t limit_ns) {
+  if (mbar_test(bar, parity)) return true;
+  const uint64_t t0 = global_timer();
+  while (true) {
+    if (mbar_test(bar, parity)) return true;
+    if (abort_flag != nullptr && *abort_flag) return false;
+    if (global_timer() - t0 > limit_ns) {
+      if (abort_flag != nullptr) *abort_flag = 1;
+      atomicOr(&g_wait_status, 1u);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+          "r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+// 32 rows x 16 bytes of scales from shared memory into TMEM, replicated to the
+// four 32-lane quarters.
+__device__ __forceinline__ void tc_copy_scales(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+__device__ __forceinline__ void mma_fp4(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+__device__ __forceinline__ void mma_bf16(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_load32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptors (tcgen05 format: start >> 4 at bit 0,
+// leading-byte offset >> 4 at bit 16, stride-byte offset >> 4 at bit 32,
+// version 1 at bit 46, swizzle mode at bit 61).
+__device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t addr) {
+  return uint64_t((addr >> 4) & 0x3FFFu) | (uint64_t(1) << 16) | (uint64_t(1024 >> 4) << 32) | (uint64_t(1) << 46) |
+         (uint64_t(2) << 61);
+}
+__device__ __forceinline__ uint64_t desc_kmajor_sw32(uint32_t addr) {
+  return uint64_t((addr >> 4) & 0x3FFFu) | (uint64_t(1) << 16) | (uint64_t(256 >> 4) << 32) | (uint64_t(1) << 46) |
+         (uint64_t(6) << 61);
+}
+// 32 rows of 16 bytes, contiguous: 8-row core matrices 128 bytes apart.
+__device__ __forceinline__ uint64_t desc_scales(uint32_t addr) {
+  return uint64_t((addr >> 4) & 0x3FFFu) | (uint64_t(128 >> 4) << 16) | (uint64_t(128 >> 4) << 32) |
+         (uint64_t(1) << 46);
+}
+
+__device__ __forceinline__ int expert_of_row(const int32_t* off_s, int E, int row) {
+  int lo = 0, hi = E - 1;                 // last expert whose segment starts at or before row
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (off_s[mid] <= row) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// ------------------------------------------------------------------ kernel
+
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                        const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_wc,
+                        GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* const base_ptr = smem_raw + (base - raw);
+  const int S = p.stages;
+  const int nch = p.n_chan / 16;
+  const uint32_t comp_r = base + S * kStageBytes;
+  const uint32_t comp_wc = comp_r + nch * kCompChunkBytes;
+  const uint32_t bar0 = comp_wc + nch * kCompChunkBytes;           // 8-byte aligned
+  // barrier addresses
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
+  const uint32_t comp_full = bar0 + 8u * (2 * S);
+  const uint32_t comp_empty = comp_full + 8;
+  const uint32_t acc_full0 = comp_full + 16;       // two barriers
+  const uint32_t acc_empty0 = comp_full + 32;      // two barriers
+  const uint32_t compacc_empty = comp_full + 48;
+  const uint32_t drain_bar = comp_full + 56;
+  uint8_t* const misc = base_ptr + (comp_full + 64 - base);
+  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(misc);
+  volatile int* const abort_flag = reinterpret_cast<volatile int*>(misc + 4);
+  int32_t* const off_s = reinterpret_cast<int32_t*>(misc + 16);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    mbar_init(comp_full, 1);
+    mbar_init(comp_empty, 1);
+    mbar_init(acc_full0, 1);
+    mbar_init(acc_full0 + 8, 1);
+    mbar_init(acc_empty0, 4);
+    mbar_init(acc_empty0 + 8, 4);
+    mbar_init(compacc_empty, 4);
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  for (int i = threadIdx.x; i <= p.E; i += blockDim.x) off_s[i] = p.expert_off[i];
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int n_ntiles = p.N / BN;
+  const int total = (off_s[p.E] / BM) * n_ntiles;
+  const int nkb_total = p.K / 64;                 // MMAs along K
+  const int nks = (nkb_total + 3) / 4;            // pipeline stages along K
+  const int n_col_tiles = nkb_total;              // 512-byte scale tiles per 128-row band
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ producer
+    int it = 0;
+    uint32_t cph = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      const int mt = t / n_ntiles, nt = t - mt * n_ntiles;
+      const int m0 = mt * BM;
+      const int e = expert_of_row(off_s, p.E, m0);
+      const int brow = e * p.N + nt * BN;
+      for (int ks = 0; ks < nks; ++ks, ++it) {
+        const int s = it % S;
+        const uint32_t ph = (it / S) & 1;
+        if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+        const int nkb = min(4, nkb_total - ks * 4);
+        const uint32_t st = base + s * kStageBytes;
+        mbar_expect_tx(full_bar(s), kABytes + kBBytes + 2 * nkb * 512);
+        tma_load_2d(st, &tm_a, ks * kStageRowBytes, m0, full_bar(s));
+        tma_load_2d(st + kABytes, &tm_b, ks * kStageRowBytes, brow, full_bar(s));
+        bulk_load(st + kABytes + kBBytes, p.a_scales + (static_cast<int64_t>(mt) * n_col_tiles + ks * 4) * 512,
+                  nkb * 512, full_bar(s));
+        bulk_load(st + kABytes + kBBytes + kSfBytes,
+                  p.w_scales + (static_cast<int64_t>(brow / BM) * n_col_tiles + ks * 4) * 512, nkb * 512,
+                  full_bar(s));
+      }
+      if (ok && nch) {
+        if (!mbar_wait(comp_empty, cph ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+        mbar_expect_tx(comp_full, 2 * nch * kCompChunkBytes);
+        for (int j = 0; j < nch; ++j) {
+          tma_load_2d(comp_r + j * kCompChunkBytes, &tm_r, j * 16, m0, comp_full);
+          tma_load_2d(comp_wc + j * kCompChunkBytes, &tm_wc, j * 16, brow, comp_full);
+        }
+        cph ^= 1u;
+      }
+    }
+    if (!ok) {
+      // let every copy this thread issued land before the CTA can exit
+      for (int i = (it > S ? it - S : 0); i < it; ++i)
+        mbar_wait(full_bar(i % S), (i / S) & 1, nullptr, kDrainTimeoutNs);
+      if (nch) mbar_wait(comp_full, cph ^ 1u, nullptr, kDrainTimeoutNs);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------------------------------------------------------- MMA
+    int it = 0, tc = 0;
+    uint32_t cph = 0, caph = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++tc) {
+      const int buf = tc & 1;
+      const uint32_t aph = (tc >> 1) & 1;
+      if (!mbar_wait(acc_empty0 + 8 * buf, aph ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t dacc = tmem + buf * BN;
+      for (int ks = 0; ks < nks; ++ks, ++it) {
+        const int s = it % S;
+        const uint32_t ph = (it / S) & 1;
+        if (!mbar_wait(full_bar(s), ph, abort_flag, p.timeout_ns)) { ok = false; break; }
+        tc_fence_after();
+        const int nkb = min(4, nkb_total - ks * 4);
+        const uint32_t st = base + s * kStageBytes;
+        const uint32_t tsfa = tmem + kSfCol + (it & 1) * 32;
+        const uint32_t tsfb = tsfa + 16;
+        for (int kb = 0; kb < nkb; ++kb) {
+          tc_copy_scales(tsfa + kb * 4, desc_scales(st + kABytes + kBBytes + kb * 512));
+          tc_copy_scales(tsfb + kb * 4, desc_scales(st + kABytes + kBBytes + kSfBytes + kb * 512));
+        }
+        for (int kb = 0; kb < nkb; ++kb) {
+          mma_fp4(dacc, desc_kmajor_sw128(st + kb * kMmaKBytes), desc_kmajor_sw128(st + kABytes + kb * kMmaKBytes),
+                  kIdescFp4, tsfa + kb * 4, tsfb + kb * 4, (ks | kb) != 0 ? 1u : 0u);
+        }
+        tc_commit(empty_bar(s));
+      }
+      if (!ok) break;
+      if (nch) {
+        if (!mbar_wait(comp_full, cph, abort_flag, p.timeout_ns)) { ok = false; break; }
+        tc_fence_after();
+        cph ^= 1u;
+        if (!mbar_wait(compacc_empty, caph ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+        tc_fence_after();
+        caph ^= 1u;
+        for (int j = 0; j < nch; ++j)
+          mma_bf16(tmem + kCompCol, desc_kmajor_sw32(comp_r + j * kCompChunkBytes),
+                   desc_kmajor_sw32(comp_wc + j * kCompChunkBytes), kIdescBf16, j != 0 ? 1u : 0u);
+        tc_commit(comp_empty);
+      }
+      tc_commit(acc_full0 + 8 * buf);
+    }
+    if (!ok) {
+      // wait for every MMA and scale copy already issued before TMEM is freed
+      tc_commit(drain_bar);
+      mbar_wait(drain_bar, 0, nullptr, kDrainTimeoutNs);
+    }
+  } else if (warp >= 2) {
+    // ----------------------------------------------------------- epilogue
+    const int q = warp & 3;                       // TMEM lane quarter of this warp
+    int tc = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++tc) {
+      const int mt = t / n_ntiles, nt = t - mt * n_ntiles;
+      const int m0 = mt * BM;
+      const int e = expert_of_row(off_s, p.E, m0);
+      const int buf = tc & 1;
+      const uint32_t ph = (tc >> 1) & 1;
+      if (!mbar_wait(acc_full0 + 8 * buf, ph, abort_flag, p.timeout_ns)) break;
+      tc_fence_after();
+      const float G = __fmul_rn(p.g_a[p.g_a_per_expert ? e : 0], p.g_w[e]);
+      const int64_t row = m0 + q * 32 + lane;
+      uint16_t* const yrow = p.y + row * p.N + nt * BN;
+      const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32], w[32];
+        tmem_load32(lane_base + buf * BN + c * 32, v);
+        if (nch) tmem_load32(lane_base + kCompCol + c * 32, w);
+        tmem_wait_ld();
+        uint32_t o[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          float a0 = __uint_as_float(v[2 * j]) * G, a1 = __uint_as_float(v[2 * j + 1]) * G;
+          if (nch) {
+            a0 += __uint_as_float(w[2 * j]);
+            a1 += __uint_as_float(w[2 * j + 1]);
+          }
+          o[j] = pack_bf16x2(a0, a1);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(yrow + c * 32);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) dst[j] = make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(acc_empty0 + 8 * buf);
+        if (nch) mbar_arrive(compacc_empty);
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+// One thread waits on a barrier that nothing completes; the bounded wait
+// gives up after limit_ns and records the timeout.
+__global__ void bounded_wait_selftest_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_addr(&bar), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    mbar_wait(smem_addr(&bar), 0, reinterpret_cast<volatile int*>(&abort_flag), limit_ns);
+  }
+}
+
+// ------------------------------------------------------------------- host
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+int make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t elem_bytes, uint64_t inner,
+                uint64_t outer, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return set_error(QUADS_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * elem_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return set_error(QUADS_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return QUADS_OK;
+}
+
+size_t gemm_smem_bytes(int stages, int n_chan, int E) {
+  return 1024 + static_cast<size_t>(stages) * kStageBytes + static_cast<size_t>(n_chan / 16) * 2 * kCompChunkBytes +
+         static_cast<size_t>(2 * stages + 8) * 8 + 16 + static_cast<size_t>(E + 1) * 4;
+}
+
+}  // namespace
+}  // namespace quads
+
+using namespace quads;
+
+extern "C" {
+
+int quads_moe_grouped_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_a,
+                                 int g_a_per_expert, const uint8_t* w_codes, const uint8_t* w_scales, const float* g_w,
+                                 const int32_t* expert_off, int E, int64_t rows_cap, int64_t N, int64_t K,
+                                 const uint16_t* a_resid, const uint16_t* w_resid, int n_chan, uint16_t* y,
+                                 quads_stream_t stream) {
+  clear_error();
+  QUADS_REQUIRE(E >= 1 && E <= 256, QUADS_ERR_UNSUPPORTED_SHAPE, "E must be in [1, 256]");
+  QUADS_REQUIRE(N > 0 && N % BN == 0 && N <= (int64_t(1) << 20), QUADS_ERR_UNSUPPORTED_SHAPE,
+                "N (%lld) must be a positive multiple of 128", (long long)N);
+  QUADS_REQUIRE(K > 0 && K % 64 == 0 && K <= (int64_t(1) << 20), QUADS_ERR_UNSUPPORTED_SHAPE,
+                "K (%lld) must be a positive multiple of 64", (long long)K);
+  QUADS_REQUIRE(rows_cap >= 0 && rows_cap % BM == 0 && rows_cap < (int64_t(1) << 31), QUADS_ERR_INVALID_ARG,
+                "rows_cap must be a multiple of 128");
+  QUADS_REQUIRE(E * N < (int64_t(1) << 31), QUADS_ERR_UNSUPPORTED_SHAPE, "E * N too large");
+  QUADS_REQUIRE(n_chan >= 0 && n_chan % 16 == 0 && n_chan <= kMaxChan, QUADS_ERR_UNSUPPORTED_SHAPE,
+                "n_chan must be a multiple of 16 in [0, %d]", kMaxChan);
+  QUADS_REQUIRE(a_codes && a_scales && g_a && w_codes && w_scales && g_w && expert_off && y, QUADS_ERR_INVALID_ARG,
+                "null pointer");
+  QUADS_REQUIRE(n_chan == 0 || (a_resid && w_resid), QUADS_ERR_INVALID_ARG, "a_resid and w_resid required");
+  QUADS_REQUIRE(aligned(a_codes, 16) && aligned(w_codes, 16) && aligned(a_scales, 16) && aligned(w_scales, 16) &&
+                    aligned(y, 16) && (n_chan == 0 || (aligned(a_resid, 16) && aligned(w_resid, 16))),
+                QUADS_ERR_INVALID_ARG, "matrix pointers must be 16-byte aligned");
+  if (rows_cap == 0) return QUADS_OK;
+
+  CUtensorMap tm_a, tm_b, tm_r, tm_wc;
+  QUADS_TRY(make_map_2d(&tm_a, a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, rows_cap, kStageRowBytes, BM,
+                        CU_TENSOR_MAP_SWIZZLE_128B));
+  QUADS_TRY(make_map_2d(&tm_b, w_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, E * N, kStageRowBytes, BN,
+                        CU_TENSOR_MAP_SWIZZLE_128B));
+  if (n_chan) {
+    QUADS_TRY(make_map_2d(&tm_r, a_resid, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, n_chan, rows_cap, 16, BM,
+                          CU_TENSOR_MAP_SWIZZLE_32B));
+    QUADS_TRY(make_map_2d(&tm_wc, w_resid, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, n_chan, E * N, 16, BN,
+                          CU_TENSOR_MAP_SWIZZLE_32B));
+  } else {
+    tm_r = tm_a;
+    tm_wc = tm_a;
+  }
+  const size_t smem_cap = 232448;   // 227 KB per block on sm_100
+  int stages = kMaxStages;
+  while (stages >= 2 && gemm_smem_bytes(stages, n_chan, E) > smem_cap) --stages;
+  QUADS_REQUIRE(stages >= 2, QUADS_ERR_UNSUPPORTED_SHAPE, "not enough shared memory for two stages");
+  const size_t smem = gemm_smem_bytes(stages, n_chan, E);
+  if (cudaFuncSetAttribute(grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return set_error(QUADS_ERR_CUDA, "cannot set %zu bytes of shared memory", smem);
+  GemmParams p;
+  p.a_scales = a_scales;
+  p.w_scales = w_scales;
+  p.g_a = g_a;
+  p.g_w = g_w;
+  p.expert_off = expert_off;
+  p.y = y;
+  p.g_a_per_expert = g_a_per_expert ? 1 : 0;
+  p.E = E;
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.n_chan = n_chan;
+  p.stages = stages;
+  p.timeout_ns = kGemmTimeoutNs;
+  const int64_t max_tiles = (rows_cap / BM) * (N / BN);
+  int grid = num_sms();
+  if (grid > max_tiles) grid = static_cast<int>(max_tiles);
+  grouped_gemm_kernel<<<grid, kThreads, smem, stream>>>(tm_a, tm_b, tm_r, tm_wc, p);
+  count_launches(1);
+  return check_launch("grouped_gemm_kernel");
+}
+
+int quads_device_status(quads_stream_t stream) {
+  clear_error();
+  if (cudaStreamSynchronize(stream) != cudaSuccess)
+    return set_error(QUADS_ERR_CUDA, "stream synchronize failed: %s", cudaGetErrorString(cudaGetLastError()));
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_wait_status, sizeof(v)) != cudaSuccess)
+    return set_error(QUADS_ERR_CUDA, "cannot read the device status word");
+  if (v) {
+    unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_wait_status, &zero, sizeof(zero)) != cudaSuccess)
+      return set_error(QUADS_ERR_CUDA, "cannot clear the device status word");
+    return set_error(QUADS_ERR_TIMEOUT, "a device-side wait timed out");
+  }
+  return QUADS_OK;
+}
+
+int quads_selftest_bounded_wait(uint64_t timeout_ns, quads_stream_t stream) {
+  clear_error();
+  QUADS_REQUIRE(timeout_ns > 0 && timeout_ns <= 10000000000ull, QUADS_ERR_INVALID_ARG,
+                "timeout must be in (0, 10 s]");
+  bounded_wait_selftest_kernel<<<1, 32, 0, stream>>>(timeout_ns);
+  count_launches(1);
+  return check_launch("bounded_wait_selftest_kernel");
+}
+
+}  // extern "C"

@@ -1,0 +1,607 @@
+// NVFP4 quantization kernels: per-group amax, quantize (+ residual channels,
+// + weight fake-quant outputs), dequantize, channel calibration, STE backward.
+//
+// Method: [TRACE] "Fonctionnement, côté ingénierie" (block scaling, one 4-bit
+// value per element, rounding direction as a discrete choice); [format]
+// (16-element blocks along K, E4M3 block scale, FP32 per-tensor scale);
+// [QUADS-fr §2.2.B] (residual on the high-residual channels);
+// [QUADS-fr §2.2.A] (trainer weights fake-quantized onto the rollout's grid,
+// straight-through backward).
+//
+// Every kernel is HBM-bound: one thread owns one 16-element block (32 bytes of
+// BF16 in, 8 bytes of codes and 1 scale byte out), a warp covers 32
+// consecutive blocks of a row (1 KB contiguous), grids are grid-stride loops
+// sized to a multiple of the SM count.
+#include <cstdio>
+
+#include "common.cuh"
+
+namespace quads {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kMaxGroupsSmem = 1024;
+constexpr int kMaxChan = 256;
+
+int grid_for(int64_t work, int per_block = kThreads) {
+  int64_t g = ceil_div(work, per_block);
+  int64_t cap = static_cast<int64_t>(num_sms()) * 8;
+  if (g > cap) g = cap;
+  if (g < 1) g = 1;
+  return static_cast<int>(g);
+}
+
+// --------------------------------------------------------------------- amax
+
+__global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t* __restrict__ x, int64_t rows,
+                                                        int64_t K, int64_t ld, const int32_t* group_off,
+                                                        int n_groups, int64_t uniform_rows,
+                                                        unsigned int* __restrict__ out_bits) {
+  extern __shared__ int32_t smem[];
+  int32_t* off_s = smem;                                   // n_groups + 1 (explicit groups)
+  unsigned int* amax_s = reinterpret_cast<unsigned int*>(smem + n_groups + 1);
+  for (int i = threadIdx.x; i <= n_groups; i += blockDim.x) {
+    if (group_off != nullptr) off_s[i] = group_off[i];
+    if (i < n_groups) amax_s[i] = 0u;
+  }
+  __syncthreads();
+  RowGroups grp{group_off ? off_s : nullptr, n_groups, uniform_rows};
+  const int64_t nkb = K / 16;
+  const int64_t total = rows * nkb;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t wstride = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t base = warp0 * 32; base < total; base += wstride * 32) {
+    int64_t b = base + lane;
+    unsigned int m = 0u;
+    int gid = 0;
+    if (b < total) {
+      int64_t row = b / nkb, kb = b - row * nkb;
+      uint32_t w[8];
+      load_bf16x16(x + row * ld + kb * 16, w);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        m = max(m, w[i] & 0x7FFFu);
+        m = max(m, (w[i] >> 16) & 0x7FFFu);
+      }
+      gid = grp.of(row);
+    }
+    int gid0 = __shfl_sync(0xffffffffu, gid, 0);
+    bool same = __all_sync(0xffffffffu, (b >= total) || gid == gid0);
+    if (same) {
+      unsigned int wm = __reduce_max_sync(0xffffffffu, m);
+      if (lane == 0 && wm) atomicMax(&amax_s[gid0], wm);
+    } else if (b < total && m) {
+      atomicMax(&amax_s[gid], m);
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < n_groups; i += blockDim.x)
+    if (amax_s[i]) atomicMax(&out_bits[i], amax_s[i] << 16);
+}
+
+// ----------------------------------------------------------------- quantize
+
+struct QuantArgs {
+  const uint16_t* x;
+  int64_t rows, K, ld;
+  const int32_t* group_off;
+  int n_groups;
+  int64_t uniform_rows;
+  const float* amax;       // [n_groups]
+  uint8_t* codes;          // [rows][K/2] or null
+  uint8_t* scales;         // or null
+  int scale_layout;
+  float* g_out;            // [n_groups] or null
+  const int32_t* chan;     // [n_chan]
+  int n_chan;
+  uint16_t* resid;         // [rows][n_chan] or null
+  int resid_mode;          // 0: residual, 1: bf16(deq), 2: the input itself
+  uint16_t* w_fq;          // [rows][K] or null
+  int fold;                // w_fq = bf16(deq) (1) or e2m1 * e4m3 (0)
+};
+
+__global__ void __launch_bounds__(kThreads) quantize_kernel(QuantArgs a) {
+  extern __shared__ int32_t smem[];
+  const int64_t nkb = a.K / 16;
+  const int n = a.n_groups;
+  int32_t* off_s = smem;                                   // n + 1
+  float* g_s = reinterpret_cast<float*>(smem + n + 1);     // n
+  int32_t* mask_s = smem + 2 * n + 1;                      // nkb (only with channels)
+  int32_t* first_s = mask_s + (a.n_chan ? nkb : 0);        // nkb
+  int32_t* pad_s = first_s + (a.n_chan ? nkb : 0);         // n_chan + 1 (count first)
+  for (int i = threadIdx.x; i <= n; i += blockDim.x) {
+    if (a.group_off != nullptr) off_s[i] = a.group_off[i];
+    if (i < n) {
+      float g = __fdiv_rn(a.amax[i], kNvfp4Range);
+      g_s[i] = g;
+      if (blockIdx.x == 0 && a.g_out != nullptr) a.g_out[i] = g;
+    }
+  }
+  if (a.n_chan) {
+    for (int64_t i = threadIdx.x; i < nkb; i += blockDim.x) { mask_s[i] = 0; first_s[i] = 0x7FFFFFFF; }
+    if (threadIdx.x == 0) pad_s[0] = 0;
+  }
+  __syncthreads();
+  if (a.n_chan) {
+    for (int j = threadIdx.x; j < a.n_chan; j += blockDim.x) {
+      int c = a.chan[j];
+      if (c >= 0 && c < a.K) {
+        atomicOr(&mask_s[c >> 4], 1 << (c & 15));
+        atomicMin(&first_s[c >> 4], j);
+      } else {
+        int p = atomicAdd(&pad_s[0], 1);
+        pad_s[1 + p] = j;
+      }
+    }
+    __syncthreads();
+  }
+  RowGroups grp{a.group_off ? off_s : nullptr, n, a.uniform_rows};
+  const bool tiled = a.scale_layout == QUADS_SCALES_TILED;
+  const int64_t nkb_e = tiled ? ceil_div(nkb, 4) * 4 : nkb;
+  const int64_t rows_e = tiled ? ceil_div(a.rows, 128) * 128 : a.rows;
+  const int64_t ncol_tiles = nkb_e / 4;
+  const int64_t total = rows_e * nkb_e;
+  const int npad = a.n_chan ? pad_s[0] : 0;
+  for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < total;
+       b += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = b / nkb_e, kb = b - row * nkb_e;
+    const bool real = row < a.rows && kb < nkb;
+    uint32_t scale = 0;
+    if (real) {
+      QBlock q;
+      uint32_t w[8];
+      load_bf16x16(a.x + row * a.ld + kb * 16, w);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        q.x[2 * i] = bf16_bits_to_float(w[i] & 0xFFFFu);
+        q.x[2 * i + 1] = bf16_bits_to_float(w[i] >> 16);
+      }
+      const float g = g_s[grp.of(row)];
+      quantize_block(q, g);
+      scale = q.scale;
+      if (a.codes) {
+        uint2 c;
+        // byte j holds elements 2j (low nibble) and 2j+1: nibble order == element order
+        c.x = q.codes_lo;
+        c.y = q.codes_hi;
+        *reinterpret_cast<uint2*>(a.codes + row * (a.K / 2) + kb * 8) = c;
+      }
+      if (a.w_fq) {
+        uint32_t o[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float v0 = __fmul_rn(e2m1_value(qblock_code(q, 2 * i)), q.sv);
+          float v1 = __fmul_rn(e2m1_value(qblock_code(q, 2 * i + 1)), q.sv);
+          if (a.fold) { v0 = __fmul_rn(v0, g); v1 = __fmul_rn(v1, g); }
+          o[i] = pack_bf16x2(v0, v1);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(a.w_fq + row * a.K + kb * 16);
+        dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+        dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+      }
+      if (a.resid) {
+        uint32_t m = static_cast<uint32_t>(mask_s[kb]);
+        if (m) {
+          int j = first_s[kb];
+          while (m) {
+            int bit = __ffs(m) - 1;
+            m &= m - 1;
+            float v;
+            if (a.resid_mode == 2) {
+              v = q.x[bit];
+            } else {
+              float dq = deq_f32(qblock_code(q, bit), q.sv, g);
+              v = (a.resid_mode == 1) ? dq : __fsub_rn(q.x[bit], dq);
+            }
+            a.resid[row * a.n_chan + j] = static_cast<uint16_t>(float_to_bf16_bits(v));
+            ++j;
+          }
+        }
+        if (kb == 0)
+          for (int p = 0; p < npad; ++p) a.resid[row * a.n_chan + pad_s[1 + p]] = 0;
+      }
+    }
+    if (a.scales && (real || tiled)) {
+      int64_t off = tiled ? tiled_scale_offset(row, kb, ncol_tiles) : row * nkb + kb;
+      a.scales[off] = static_cast<uint8_t>(scale);
+    }
+  }
+}
+
+size_t quantize_smem(int n_groups, int64_t K, int n_chan) {
+  size_t s = (2 * static_cast<size_t>(n_groups) + 1) * 4;
+  if (n_chan) s += (2 * static_cast<size_t>(K / 16) + n_chan + 1) * 4;
+  return s;
+}
+
+// --------------------------------------------------------------- dequantize
+
+__global__ void __launch_bounds__(kThreads) dequant_kernel(const uint8_t* __restrict__ codes,
+                                                           const uint8_t* __restrict__ scales, int layout,
+                                                           const float* __restrict__ g, const int32_t* group_off,
+                                                           int n_groups, int64_t uniform_rows, int64_t rows,
+                                                           int64_t K, void* out, int out_dtype) {
+  extern __shared__ int32_t smem[];
+  for (int i = threadIdx.x; i <= n_groups; i += blockDim.x)
+    if (group_off) smem[i] = group_off[i];
+  __syncthreads();
+  RowGroups grp{group_off ? smem : nullptr, n_groups, uniform_rows};
+  const int64_t nkb = K / 16, ncol_tiles = ceil_div(nkb, 4);
+  const int64_t total = rows * nkb;
+  for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < total;
+       b += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = b / nkb, kb = b - row * nkb;
+    const uint2 c = __ldg(reinterpret_cast<const uint2*>(codes + row * (K / 2) + kb * 8));
+    const uint32_t s = scales[layout == QUADS_SCALES_TILED ? tiled_scale_offset(row, kb, ncol_tiles)
+                                                           : row * nkb + kb];
+    const float sv = e4m3_value(s);
+    const float gg = g[grp.of(row)];
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v[i] = deq_f32((c.x >> (4 * i)) & 15u, sv, gg);
+      v[8 + i] = deq_f32((c.y >> (4 * i)) & 15u, sv, gg);
+    }
+    if (out_dtype == QUADS_OUT_F32) {
+      float4* d = reinterpret_cast<float4*>(static_cast<float*>(out) + row * K + kb * 16);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    } else {
+      uint4* d = reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + row * K + kb * 16);
+      d[0] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                        pack_bf16x2(v[6], v[7]));
+      d[1] = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
+                        pack_bf16x2(v[14], v[15]));
+    }
+  }
+}
+
+// ------------------------------------------------------ channel calibration
+
+constexpr int kScoreRows = 256;   // rows per partial sum
+
+// partial[chunk][K]: sum over the chunk's rows (in row order) of |fp32 residual|.
+__global__ void __launch_bounds__(kThreads) channel_partial_kernel(const uint16_t* __restrict__ x,
+                                                                   int64_t rows, int64_t K,
+                                                                   const float* __restrict__ amax,
+                                                                   float* __restrict__ partial) {
+  const int64_t nkb = K / 16;
+  const int64_t kb = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t chunk = blockIdx.y;
+  if (kb >= nkb) return;
+  const float g = __fdiv_rn(amax[0], kNvfp4Range);
+  float acc[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) acc[i] = 0.0f;
+  const int64_t r0 = chunk * kScoreRows, r1 = min(rows, r0 + kScoreRows);
+  for (int64_t row = r0; row < r1; ++row) {
+    QBlock q;
+    uint32_t w[8];
+    load_bf16x16(x + row * K + kb * 16, w);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      q.x[2 * i] = bf16_bits_to_float(w[i] & 0xFFFFu);
+      q.x[2 * i + 1] = bf16_bits_to_float(w[i] >> 16);
+    }
+    quantize_block(q, g);
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      acc[i] = __fadd_rn(acc[i], fabsf(__fsub_rn(q.x[i], deq_f32(qblock_code(q, i), q.sv, g))));
+  }
+  float* dst = partial + chunk * K + kb * 16;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) dst[i] = acc[i];
+}
+
+__global__ void channel_reduce_kernel(const float* __restrict__ partial, int64_t n_chunks, int64_t K,
+                                      float* __restrict__ scores) {
+  int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (c >= K) return;
+  float s = 0.0f;
+  for (int64_t i = 0; i < n_chunks; ++i) s = __fadd_rn(s, partial[i * K + c]);
+  scores[c] = s;
+}
+
+// One block: rank every channel by (score desc, index asc), keep rank < n_sel,
+// write the kept channels in ascending order.
+__global__ void __launch_bounds__(1024) select_kernel(const float* __restrict__ scores, int K, int n_sel,
+                                                      int32_t* __restrict__ chan_out) {
+  extern __shared__ float s_scores[];
+  __shared__ int warp_tot[32];
+  __shared__ int carry;
+  for (int i = threadIdx.x; i < K; i += blockDim.x) s_scores[i] = scores[i];
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  for (int base = 0; base < K; base += blockDim.x) {
+    int c = base + threadIdx.x;
+    int keep = 0;
+    if (c < K) {
+      float v = s_scores[c];
+      int rank = 0;
+      for (int j = 0; j < K; ++j) {
+        float u = s_scores[j];
+        rank += (u > v) || (u == v && j < c);
+      }
+      keep = rank < n_sel;
+    }
+    unsigned int bal = __ballot_sync(0xffffffffu, keep);
+    int before = __popc(bal & ((1u << lane) - 1u));
+    if (lane == 0) warp_tot[wid] = __popc(bal);
+    __syncthreads();
+    int wbase = 0;
+    for (int w = 0; w < wid; ++w) wbase += warp_tot[w];
+    if (keep) chan_out[carry + wbase + before] = c;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int t = 0;
+      for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += warp_tot[w];
+      carry += t;
+    }
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------ STE backward
+
+__global__ void ste_backward_kernel(const uint16_t* __restrict__ gfq, uint16_t* __restrict__ gw, int64_t n,
+                                    int accumulate) {
+  const int64_t nv = n / 8;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nv;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    uint4 a = __ldg(reinterpret_cast<const uint4*>(gfq) + i);
+    if (accumulate) {
+      uint4 b = reinterpret_cast<const uint4*>(gw)[i];
+      uint32_t* pa = reinterpret_cast<uint32_t*>(&a);
+      const uint32_t* pb = reinterpret_cast<const uint32_t*>(&b);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float lo = __fadd_rn(bf16_bits_to_float(pa[j] & 0xFFFFu), bf16_bits_to_float(pb[j] & 0xFFFFu));
+        float hi = __fadd_rn(bf16_bits_to_float(pa[j] >> 16), bf16_bits_to_float(pb[j] >> 16));
+        pa[j] = pack_bf16x2(lo, hi);
+      }
+    }
+    reinterpret_cast<uint4*>(gw)[i] = a;
+  }
+  // tail (n % 8 elements) handled by the first thread
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    for (int64_t i = nv * 8; i < n; ++i) {
+      if (accumulate)
+        gw[i] = static_cast<uint16_t>(
+            float_to_bf16_bits(__fadd_rn(bf16_bits_to_float(gfq[i]), bf16_bits_to_float(gw[i]))));
+      else
+        gw[i] = gfq[i];
+    }
+  }
+}
+
+// ------------------------------------------------------------- host helpers
+
+int validate_matrix(const void* x, int64_t rows, int64_t K, int64_t ld) {
+  QUADS_REQUIRE(rows >= 0 && K > 0, QUADS_ERR_INVALID_ARG, "rows must be >= 0 and K > 0");
+  QUADS_REQUIRE(K % 16 == 0, QUADS_ERR_UNSUPPORTED_SHAPE, "K (%lld) must be a multiple of 16", (long long)K);
+  QUADS_REQUIRE(K <= 65536, QUADS_ERR_UNSUPPORTED_SHAPE, "K (%lld) above 65536", (long long)K);
+  QUADS_REQUIRE(ld >= K && ld % 8 == 0, QUADS_ERR_INVALID_ARG, "ld (%lld) must be >= K and a multiple of 8",
+                (long long)ld);
+  QUADS_REQUIRE(rows == 0 || (x != nullptr && aligned(x, 16)), QUADS_ERR_INVALID_ARG,
+                "input must be non-null and 16-byte aligned");
+  return QUADS_OK;
+}
+
+int validate_groups(const int32_t* group_off, int n_groups, int64_t rows) {
+  QUADS_REQUIRE(n_groups >= 1, QUADS_ERR_INVALID_ARG, "n_groups must be >= 1");
+  if (group_off) {
+    QUADS_REQUIRE(n_groups <= kMaxGroupsSmem, QUADS_ERR_UNSUPPORTED_SHAPE, "n_groups above %d", kMaxGroupsSmem);
+  } else {
+    QUADS_REQUIRE(rows % n_groups == 0, QUADS_ERR_INVALID_ARG,
+                  "without group offsets, rows (%lld) must be a multiple of n_groups (%d)", (long long)rows,
+                  n_groups);
+    QUADS_REQUIRE(n_groups <= kMaxGroupsSmem, QUADS_ERR_UNSUPPORTED_SHAPE, "n_groups above %d", kMaxGroupsSmem);
+  }
+  return QUADS_OK;
+}
+
+int launch_amax(const uint16_t* x, int64_t rows, int64_t K, int64_t ld, const int32_t* group_off, int n_groups,
+                float* amax_out, cudaStream_t s) {
+  if (cudaMemsetAsync(amax_out, 0, sizeof(float) * n_groups, s) != cudaSuccess)
+    return set_error(QUADS_ERR_CUDA, "memset of the amax output failed");
+  if (rows == 0) return QUADS_OK;
+  int64_t uniform = group_off ? 0 : rows / n_groups;
+  size_t smem = (2 * static_cast<size_t>(n_groups) + 1) * 4;
+  amax_kernel<<<grid_for(rows * (K / 16)), kThreads, smem, s>>>(x, rows, K, ld, group_off, n_groups,
+                                                                uniform ? uniform : 1,
+                                                                reinterpret_cast<unsigned int*>(amax_out));
+  count_launches(1);
+  return check_launch("amax_kernel");
+}
+
+int launch_quantize(QuantArgs a, cudaStream_t s) {
+  int64_t nkb = a.K / 16;
+  bool tiled = a.scale_layout == QUADS_SCALES_TILED;
+  int64_t total = (tiled ? ceil_div(a.rows, 128) * 128 : a.rows) * (tiled ? ceil_div(nkb, 4) * 4 : nkb);
+  if (total == 0) return QUADS_OK;
+  size_t smem = quantize_smem(a.n_groups, a.K, a.n_chan);
+  if (smem > 48 * 1024) {
+    if (cudaFuncSetAttribute(quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return set_error(QUADS_ERR_CUDA, "cannot raise shared memory of quantize_kernel");
+  }
+  quantize_kernel<<<grid_for(total), kThreads, smem, s>>>(a);
+  count_launches(1);
+  return check_launch("quantize_kernel");
+}
+
+}  // namespace
+}  // namespace quads
+
+using namespace quads;
+
+extern "C" {
+
+size_t quads_quantize_workspace_bytes(int n_groups) {
+  if (n_groups < 1) return 0;
+  return static_cast<size_t>(ceil_div(static_cast<int64_t>(n_groups) * 4, 256) * 256);
+}
+
+int quads_amax_bf16(const uint16_t* x, int64_t rows, int64_t K, int64_t ld_x, const int32_t* group_off,
+                    int n_groups, float* amax_out, quads_stream_t stream) {
+  clear_error();
+  QUADS_TRY(validate_matrix(x, rows, K, ld_x));
+  QUADS_TRY(validate_groups(group_off, n_groups, rows));
+  QUADS_REQUIRE(amax_out != nullptr, QUADS_ERR_INVALID_ARG, "amax_out is null");
+  return launch_amax(x, rows, K, ld_x, group_off, n_groups, amax_out, stream);
+}
+
+int quads_quantize_nvfp4(const uint16_t* x, int64_t rows, int64_t K, int64_t ld_x, const int32_t* group_off,
+                         int n_groups, const float* amax_in, uint8_t* codes, uint8_t* scales, int scale_layout,
+                         float* g_out, const int32_t* chan, int n_chan, uint16_t* resid_out, void* ws,
+                         size_t ws_bytes, quads_stream_t stream) {
+  clear_error();
+  QUADS_TRY(validate_matrix(x, rows, K, ld_x));
+  QUADS_TRY(validate_groups(group_off, n_groups, rows));
+  QUADS_REQUIRE(scale_layout == QUADS_SCALES_LINEAR || scale_layout == QUADS_SCALES_TILED,
+                QUADS_ERR_INVALID_ARG, "unknown scale layout %d", scale_layout);
+  QUADS_REQUIRE(codes && scales && g_out, QUADS_ERR_INVALID_ARG, "codes, scales and g_out must be non-null");
+  QUADS_REQUIRE(aligned(codes, 8), QUADS_ERR_INVALID_ARG, "codes must be 8-byte aligned");
+  QUADS_REQUIRE(n_chan >= 0 && n_chan <= kMaxChan, QUADS_ERR_UNSUPPORTED_SHAPE, "n_chan must be in [0, %d]",
+                kMaxChan);
+  QUADS_REQUIRE(n_chan == 0 || (chan && resid_out), QUADS_ERR_INVALID_ARG,
+                "chan and resid_out are required when n_chan > 0");
+  const float* amax = amax_in;
+  if (amax == nullptr) {
+    QUADS_REQUIRE(ws != nullptr && ws_bytes >= quads_quantize_workspace_bytes(n_groups), QUADS_ERR_INVALID_ARG,
+                  "workspace of %zu bytes required when amax_in is NULL", quads_quantize_workspace_bytes(n_groups));
+    QUADS_TRY(launch_amax(x, rows, K, ld_x, group_off, n_groups, static_cast<float*>(ws), stream));
+    amax = static_cast<const float*>(ws);
+  }
+  QuantArgs a{};
+  a.x = x; a.rows = rows; a.K = K; a.ld = ld_x;
+  a.group_off = group_off; a.n_groups = n_groups; a.uniform_rows = group_off ? 1 : (rows ? rows / n_groups : 1);
+  a.amax = amax; a.codes = codes; a.scales = scales; a.scale_layout = scale_layout; a.g_out = g_out;
+  a.chan = chan; a.n_chan = n_chan; a.resid = n_chan ? resid_out : nullptr; a.resid_mode = 0;
+  a.w_fq = nullptr; a.fold = 1;
+  if (rows == 0) {
+    // still publish g (computed from the given or zero amax) and the padded scale tiles
+    if (cudaMemsetAsync(g_out, 0, sizeof(float) * n_groups, stream) != cudaSuccess)
+      return set_error(QUADS_ERR_CUDA, "memset failed");
+    return QUADS_OK;
+  }
+  return launch_quantize(a, stream);
+}
+
+int quads_dequant(const uint8_t* codes, const uint8_t* scales, int scale_layout, const float* g,
+                  const int32_t* group_off, int n_groups, int64_t rows, int64_t K, void* out, int out_dtype,
+                  quads_stream_t stream) {
+  clear_error();
+  QUADS_REQUIRE(rows >= 0 && K > 0 && K % 16 == 0, QUADS_ERR_UNSUPPORTED_SHAPE, "K must be a positive multiple of 16");
+  QUADS_TRY(validate_groups(group_off, n_groups, rows));
+  QUADS_REQUIRE(scale_layout == QUADS_SCALES_LINEAR || scale_layout == QUADS_SCALES_TILED,
+                QUADS_ERR_INVALID_ARG, "unknown scale layout %d", scale_layout);
+  QUADS_REQUIRE(out_dtype == QUADS_OUT_BF16 || out_dtype == QUADS_OUT_F32, QUADS_ERR_INVALID_ARG,
+                "unknown output dtype %d", out_dtype);
+  if (rows == 0) return QUADS_OK;
+  QUADS_REQUIRE(codes && scales && g && out, QUADS_ERR_INVALID_ARG, "null pointer");
+  QUADS_REQUIRE(aligned(codes, 8) && aligned(out, 16), QUADS_ERR_INVALID_ARG,
+                "codes must be 8-byte and out 16-byte aligned");
+  size_t smem = group_off ? (static_cast<size_t>(n_groups) + 1) * 4 : 0;
+  dequant_kernel<<<grid_for(rows * (K / 16)), kThreads, smem, stream>>>(
+      codes, scales, scale_layout, g, group_off, n_groups, group_off ? 1 : rows / n_groups, rows, K, out, out_dtype);
+  count_launches(1);
+  return check_launch("dequant_kernel");
+}
+
+size_t quads_channel_scores_workspace_bytes(int64_t rows, int64_t K) {
+  if (rows <= 0 || K <= 0) return 256;
+  return 256 + static_cast<size_t>(ceil_div(rows, kScoreRows)) * static_cast<size_t>(K) * 4;
+}
+
+int quads_channel_scores(const uint16_t* x, int64_t rows, int64_t K, const float* amax_in, float* scores, void* ws,
+                         size_t ws_bytes, quads_stream_t stream) {
+  clear_error();
+  QUADS_TRY(validate_matrix(x, rows, K, K));
+  QUADS_REQUIRE(rows > 0, QUADS_ERR_INVALID_ARG, "rows must be > 0");
+  QUADS_REQUIRE(scores != nullptr, QUADS_ERR_INVALID_ARG, "scores is null");
+  QUADS_REQUIRE(ws && ws_bytes >= quads_channel_scores_workspace_bytes(rows, K), QUADS_ERR_INVALID_ARG,
+                "workspace of %zu bytes required", quads_channel_scores_workspace_bytes(rows, K));
+  float* amax = static_cast<float*>(ws);
+  if (amax_in) {
+    if (cudaMemcpyAsync(amax, amax_in, 4, cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
+      return set_error(QUADS_ERR_CUDA, "copy of amax failed");
+  } else {
+    QUADS_TRY(launch_amax(x, rows, K, K, nullptr, 1, amax, stream));
+  }
+  float* partial = reinterpret_cast<float*>(static_cast<char*>(ws) + 256);
+  int64_t n_chunks = ceil_div(rows, kScoreRows);
+  int64_t nkb = K / 16;
+  dim3 grid(static_cast<unsigned>(ceil_div(nkb, 128)), static_cast<unsigned>(n_chunks));
+  channel_partial_kernel<<<grid, 128, 0, stream>>>(x, rows, K, amax, partial);
+  count_launches(1);
+  QUADS_TRY(check_launch("channel_partial_kernel"));
+  channel_reduce_kernel<<<static_cast<unsigned>(ceil_div(K, 256)), 256, 0, stream>>>(partial, n_chunks, K, scores);
+  count_launches(1);
+  return check_launch("channel_reduce_kernel");
+}
+
+int quads_select_channels(const float* scores, int64_t K, int n_sel, int32_t* chan_out, quads_stream_t stream) {
+  clear_error();
+  QUADS_REQUIRE(scores && chan_out, QUADS_ERR_INVALID_ARG, "null pointer");
+  QUADS_REQUIRE(K > 0 && K <= 16384, QUADS_ERR_UNSUPPORTED_SHAPE, "K must be in [1, 16384]");
+  QUADS_REQUIRE(n_sel >= 0 && n_sel <= K, QUADS_ERR_INVALID_ARG, "n_sel must be in [0, K]");
+  if (n_sel == 0) return QUADS_OK;
+  size_t smem = static_cast<size_t>(K) * 4;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+          cudaSuccess)
+    return set_error(QUADS_ERR_CUDA, "cannot raise shared memory of select_kernel");
+  select_kernel<<<1, 1024, smem, stream>>>(scores, static_cast<int>(K), n_sel, chan_out);
+  count_launches(1);
+  return check_launch("select_kernel");
+}
+
+int quads_fakequant_weight_ste(const uint16_t* w, int64_t n_mat, int64_t rows, int64_t K, const float* amax_in,
+                               int fold_global,
+                               uint16_t* w_fq, uint8_t* codes, uint8_t* scales, float* g_out, const int32_t* chan,
+                               int n_chan, int chan_raw, uint16_t* w_chan, void* ws, size_t ws_bytes,
+                               quads_stream_t stream) {
+  clear_error();
+  QUADS_REQUIRE(n_mat >= 1 && n_mat <= kMaxGroupsSmem, QUADS_ERR_UNSUPPORTED_SHAPE, "n_mat must be in [1, %d]",
+                kMaxGroupsSmem);
+  QUADS_TRY(validate_matrix(w, n_mat * rows, K, K));
+  QUADS_REQUIRE(rows > 0, QUADS_ERR_INVALID_ARG, "rows must be > 0");
+  QUADS_REQUIRE(g_out != nullptr, QUADS_ERR_INVALID_ARG, "g_out is null");
+  QUADS_REQUIRE(w_fq == nullptr || aligned(w_fq, 16), QUADS_ERR_INVALID_ARG, "w_fq must be 16-byte aligned");
+  QUADS_REQUIRE(codes == nullptr || aligned(codes, 8), QUADS_ERR_INVALID_ARG, "codes must be 8-byte aligned");
+  QUADS_REQUIRE(n_chan >= 0 && n_chan <= kMaxChan, QUADS_ERR_UNSUPPORTED_SHAPE, "n_chan must be in [0, %d]",
+                kMaxChan);
+  QUADS_REQUIRE(n_chan == 0 || (chan && w_chan), QUADS_ERR_INVALID_ARG, "chan and w_chan required with n_chan > 0");
+  const float* amax = amax_in;
+  if (amax == nullptr) {
+    QUADS_REQUIRE(ws && ws_bytes >= quads_quantize_workspace_bytes(static_cast<int>(n_mat)), QUADS_ERR_INVALID_ARG,
+                  "workspace of %zu bytes required", quads_quantize_workspace_bytes(static_cast<int>(n_mat)));
+    QUADS_TRY(launch_amax(w, n_mat * rows, K, K, nullptr, static_cast<int>(n_mat), static_cast<float*>(ws), stream));
+    amax = static_cast<const float*>(ws);
+  }
+  QuantArgs a{};
+  a.x = w; a.rows = n_mat * rows; a.K = K; a.ld = K;
+  a.group_off = nullptr; a.n_groups = static_cast<int>(n_mat); a.uniform_rows = rows;
+  a.amax = amax; a.codes = codes; a.scales = scales;
+  a.scale_layout = (rows % 128 == 0) ? QUADS_SCALES_TILED : QUADS_SCALES_LINEAR;
+  a.g_out = g_out; a.chan = chan; a.n_chan = n_chan; a.resid = n_chan ? w_chan : nullptr;
+  a.resid_mode = chan_raw ? 2 : 1; a.w_fq = w_fq; a.fold = fold_global ? 1 : 0;
+  return launch_quantize(a, stream);
+}
+
+int quads_fakequant_weight_ste_backward(const uint16_t* grad_wfq, uint16_t* grad_w, int64_t n, int accumulate,
+                                        quads_stream_t stream) {
+  clear_error();
+  QUADS_REQUIRE(n >= 0, QUADS_ERR_INVALID_ARG, "n must be >= 0");
+  if (n == 0) return QUADS_OK;
+  QUADS_REQUIRE(grad_wfq && grad_w && aligned(grad_wfq, 16) && aligned(grad_w, 16), QUADS_ERR_INVALID_ARG,
+                "gradients must be non-null and 16-byte aligned");
+  ste_backward_kernel<<<grid_for(ceil_div(n, 8)), kThreads, 0, stream>>>(grad_wfq, grad_w, n, accumulate);
+  count_launches(1);
+  return check_launch("ste_backward_kernel");
+}
+
+}  // extern "C"

@@ -1,0 +1,217 @@
+"""One NVFP4 MoE expert layer on both sides of RL alignment, driven through
+the C ABI (every step runs in libquads kernels; torch only allocates).
+
+Rollout side ([QUADS-fr §1], [QUADS-fr §2.2.B]): NVFP4 quantization of the
+layer input with the residual of the calibrated high-residual channels,
+top-k routing and expert permutation, the NVFP4 grouped gate/up GEMM with
+compensation, SwiGLU, per-expert NVFP4 re-quantization of h with its own
+compensation channels, the grouped down GEMM with compensation, and the
+weighted combine.
+
+Trainer side ([QUADS-fr §2.2.A], [TRACE]): weight fake-quant onto the
+rollout's grid (one pass also produces the rollout's NVFP4 weights and the
+compensation weight columns), the straight-through backward accumulated
+into the master gradient, the export of the rollout's quantization record
+and its replay against the trainer's activation.
+"""
+from dataclasses import dataclass
+
+import torch
+
+from . import binding as B
+from .workloads import MoEConfig
+
+
+@dataclass
+class StageTimer:
+    """Optional CUDA-event marks between stages (on the current stream)."""
+    enabled: bool = False
+
+    def __post_init__(self):
+        self.marks = []
+
+    def mark(self, name):
+        if self.enabled:
+            ev = torch.cuda.Event(enable_timing=True)
+            ev.record()
+            self.marks.append((name, ev))
+
+    def durations_ms(self):
+        out = {}
+        for (_, e0), (name, e1) in zip(self.marks, self.marks[1:]):
+            out[name] = out.get(name, 0.0) + e0.elapsed_time(e1)
+        return out
+
+
+class MoELayer:
+    """Weights, calibrated channel sets and every buffer of one layer at a
+    fixed token count; step() runs the whole path without allocating."""
+
+    def __init__(self, cfg: MoEConfig, w_gu, w_d, chan_x, chan_h, device="cuda"):
+        self.cfg = cfg
+        T, H, E, k, F = cfg.T, cfg.H, cfg.E, cfg.k, cfg.F
+        dev = torch.device(device)
+        self.dev = dev
+        self.w_gu = w_gu.contiguous()                   # [E, 2F, H] trainer master weights
+        self.w_d = w_d.contiguous()                     # [E, H, F]
+        self.chan_x = chan_x.to(dev, torch.int32).contiguous()
+        self.chan_h = chan_h.to(dev, torch.int32).contiguous()
+        self.nc_x = int(self.chan_x.numel())
+        self.nc_h = int(self.chan_h.numel())
+        cap = B.moe_rows_capacity(T, k, E)
+        self.cap = cap
+        e = lambda shape, dt: torch.empty(shape, dtype=dt, device=dev)
+        bf, u8, f32, i32 = torch.bfloat16, torch.uint8, torch.float32, torch.int32
+        # weight sync outputs
+        self.w_gu_fq, self.w_d_fq = e((E, 2 * F, H), bf), e((E, H, F), bf)
+        self.w_gu_codes, self.w_d_codes = e((E, 2 * F, H // 2), u8), e((E, H, F // 2), u8)
+        self.w_gu_scales = e((B.scales_bytes(E * 2 * F, H, B.SCALES_TILED),), u8)
+        self.w_d_scales = e((B.scales_bytes(E * H, F, B.SCALES_TILED),), u8)
+        self.g_w_gu, self.g_w_d = e((E,), f32), e((E,), f32)
+        self.amax_w_gu, self.amax_w_d, self.amax_x = e((E,), f32), e((E,), f32), e((1,), f32)
+        self.wc_gu, self.wc_d = e((E, 2 * F, self.nc_x), bf), e((E, H, self.nc_h), bf)
+        self.ws_w = e((B.quantize_workspace_bytes(E),), u8)
+        # STE gradients (master gradient accumulated in place)
+        self.grad_gu, self.grad_d = torch.zeros_like(self.w_gu), torch.zeros_like(self.w_d)
+        # rollout activations
+        self.x_codes, self.x_scales = e((T, H // 2), u8), e((B.scales_bytes(T, H, B.SCALES_LINEAR),), u8)
+        self.g_x, self.x_resid, self.ws_x = e((1,), f32), e((T, self.nc_x), bf), e((B.quantize_workspace_bytes(1),), u8)
+        self.topk_idx, self.topk_w = e((T, k), i32), e((T, k), f32)
+        self.expert_off, self.row_of, self.src_of = e((E + 1,), i32), e((T * k,), i32), e((cap,), i32)
+        self.ws_perm = e((B.moe_permute_workspace_bytes(T, k, E),), u8)
+        self.pa_codes, self.pa_scales = e((cap, H // 2), u8), e((B.scales_bytes(cap, H, B.SCALES_TILED),), u8)
+        self.pa_resid = e((cap, self.nc_x), bf)
+        self.y_gu = e((cap, 2 * F), bf)
+        self.h, self.amax_h = e((cap, F), bf), e((E,), f32)
+        self.h_codes, self.h_scales = e((cap, F // 2), u8), e((B.scales_bytes(cap, F, B.SCALES_TILED),), u8)
+        self.g_h, self.h_resid = e((E,), f32), e((cap, self.nc_h), bf)
+        self.y_d = e((cap, H), bf)
+        self.out = e((T, H), bf)
+        # TRACE record and replay outputs
+        self._tsrc = [
+            B.qtensor_src(self.x_codes, self.x_scales, self.g_x, T, H, B.SCALES_LINEAR, chan=self.chan_x,
+                          resid=self.x_resid),
+            B.qtensor_src(self.h_codes, self.h_scales, self.g_h, cap, F, B.SCALES_TILED, group_off=self.expert_off,
+                          chan=self.chan_h, resid=self.h_resid),
+        ]
+        self.record_bytes, _ = B.trace_qrecord_layout(0, T, k, self._tsrc)
+        self.record = e((self.record_bytes,), u8)
+        self.x_hat, self.h_hat = e((T, H), bf), e((cap, F), bf)
+        self.counts, self.status = torch.zeros(2, dtype=torch.int64, device=dev), e((1,), i32)
+        self.status_h = e((1,), i32)
+
+    # ---------------------------------------------------------------- stages
+
+    def weight_sync(self, timer=None):
+        """Trainer fake-quant + the rollout's NVFP4 weights: one amax pass and
+        one quantize pass per weight tensor."""
+        cfg = self.cfg
+        t = timer or StageTimer(False)
+        E, F, H = cfg.E, cfg.F, cfg.H
+        B.amax_bf16(self.w_gu.view(E * 2 * F, H), n_groups=E, out=self.amax_w_gu)
+        t.mark("amax_w_gate_up")
+        B.fakequant_weight_ste(self.w_gu, True, self.chan_x, False, True, self.w_gu_fq, self.w_gu_codes,
+                               self.w_gu_scales, self.g_w_gu, self.wc_gu, None, self.amax_w_gu)
+        t.mark("fakequant_w_gate_up")
+        B.amax_bf16(self.w_d.view(E * H, F), n_groups=E, out=self.amax_w_d)
+        t.mark("amax_w_down")
+        B.fakequant_weight_ste(self.w_d, True, self.chan_h, False, True, self.w_d_fq, self.w_d_codes,
+                               self.w_d_scales, self.g_w_d, self.wc_d, None, self.amax_w_d)
+        t.mark("fakequant_w_down")
+
+    def ste_backward(self, grad_gu_fq, grad_d_fq, timer=None):
+        t = timer or StageTimer(False)
+        B.fakequant_weight_ste_backward(grad_gu_fq, self.grad_gu, accumulate=True)
+        t.mark("ste_backward_gate_up")
+        B.fakequant_weight_ste_backward(grad_d_fq, self.grad_d, accumulate=True)
+        t.mark("ste_backward_down")
+
+    def rollout_forward(self, x, logits, timer=None):
+        cfg = self.cfg
+        T, H, E, k, F = cfg.T, cfg.H, cfg.E, cfg.k, cfg.F
+        t = timer or StageTimer(False)
+        B.amax_bf16(x, out=self.amax_x)
+        t.mark("amax_x")
+        B.quantize_nvfp4(x, amax_in=self.amax_x, scale_layout=B.SCALES_LINEAR, chan=self.chan_x,
+                         codes=self.x_codes, scales=self.x_scales, g_out=self.g_x, resid_out=self.x_resid)
+        t.mark("quantize_x")
+        B.moe_router_topk(logits, k, True, idx=self.topk_idx, w=self.topk_w)
+        t.mark("router_topk")
+        B.moe_permute(self.topk_idx, E, self.expert_off, self.row_of, self.src_of, self.ws_perm)
+        t.mark("permute")
+        B.moe_gather(self.src_of, self.expert_off, E, self.cap, self.x_codes, self.x_scales, H, self.x_resid,
+                     self.pa_codes, self.pa_scales, self.pa_resid)
+        t.mark("gather")
+        B.moe_grouped_gemm_nvfp4(self.pa_codes, self.pa_scales, self.g_x, self.w_gu_codes, self.w_gu_scales,
+                                 self.g_w_gu, self.expert_off, E, self.cap, 2 * F, H, self.pa_resid, self.wc_gu,
+                                 y=self.y_gu)
+        t.mark("gemm_gate_up")
+        B.swiglu(self.y_gu, F, self.expert_off, E, h=self.h, amax=self.amax_h)
+        t.mark("swiglu")
+        B.quantize_nvfp4(self.h, group_off=self.expert_off, n_groups=E, amax_in=self.amax_h,
+                         scale_layout=B.SCALES_TILED, chan=self.chan_h, codes=self.h_codes, scales=self.h_scales,
+                         g_out=self.g_h, resid_out=self.h_resid)
+        t.mark("quantize_h")
+        B.moe_grouped_gemm_nvfp4(self.h_codes, self.h_scales, self.g_h, self.w_d_codes, self.w_d_scales,
+                                 self.g_w_d, self.expert_off, E, self.cap, H, F, self.h_resid, self.wc_d,
+                                 y=self.y_d)
+        t.mark("gemm_down")
+        B.moe_unpermute_combine(self.y_d, self.row_of, self.topk_w, T, k, H, out=self.out)
+        t.mark("combine")
+        return self.out
+
+    def export(self, layer_id=0):
+        B.trace_export_qrecord(layer_id, self.cfg.T, self.cfg.k, self.topk_idx, self._tsrc, record=self.record)
+
+    def trainer_replay(self, x_train, layer_id=0, timer=None):
+        cfg = self.cfg
+        t = timer or StageTimer(False)
+        B.trace_replay_qrecord(self.record, layer_id, 0, cfg.T, cfg.H, x_train=x_train, x_hat=self.x_hat,
+                               counts=self.counts, status=self.status)
+        t.mark("replay_x")
+        B.trace_replay_qrecord(self.record, layer_id, 1, self.cap, cfg.F, x_hat=self.h_hat, status=self.status_h)
+        t.mark("replay_h")
+
+    def step(self, x, logits, x_train, grad_gu_fq, grad_d_fq, timer=None, layer_id=0):
+        """One pass of the whole path over one batch.  The replay's mismatch
+        counters accumulate across steps (zero them with reset_counts())."""
+        t = timer or StageTimer(False)
+        t.mark("start")
+        self.weight_sync(t)
+        out = self.rollout_forward(x, logits, t)
+        self.export(layer_id)
+        t.mark("export")
+        self.trainer_replay(x_train, layer_id, t)
+        self.ste_backward(grad_gu_fq, grad_d_fq, t)
+        return out
+
+    def reset_counts(self):
+        self.counts.zero_()
+
+
+def calibrate_channels(x, n_sel):
+    """Calibrated high-residual channel set (device kernels), padded with -1
+    to a multiple of 16."""
+    K = x.shape[1]
+    scores = B.channel_scores(x)
+    sel = B.select_channels(scores, n_sel)
+    n_pad = -(-n_sel // 16) * 16
+    out = torch.full((n_pad,), -1, dtype=torch.int32, device=x.device)
+    out[:n_sel] = sel
+    return out
+
+
+def build_layer(cfg: MoEConfig, inputs, device="cuda"):
+    """Layer from generated inputs: channel sets calibrated on the layer's own
+    batch (X for the gate/up input, the uncompensated h for the down input)."""
+    x, logits = inputs["x"], inputs["logits"]
+    chan_x = calibrate_channels(x, cfg.n_chan)
+    empty = torch.full((16,), -1, dtype=torch.int32, device=device)
+    probe = MoELayer(cfg, inputs["w_gu"], inputs["w_d"], chan_x, empty, device)
+    probe.weight_sync()
+    probe.rollout_forward(x, logits)
+    torch.cuda.synchronize()
+    n_rows = int(probe.expert_off[-1].item())
+    chan_h = calibrate_channels(probe.h[:n_rows].contiguous(), cfg.n_chan_f)
+    del probe
+    return MoELayer(cfg, inputs["w_gu"], inputs["w_d"], chan_x, chan_h, device)
