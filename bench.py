@@ -71,6 +71,22 @@ def load_peaks():
 # --------------------------------------------------------------- accounting
 
 
+def max_over_ranks(v, world, device=None):
+    """The slowest rank's value (every rank takes part; NCCL or gloo)."""
+    if world == 1:
+        return float(v)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank, world, ms):
+    """Aggregate throughput: every rank's work over the slowest rank's time."""
+    return world * flops_per_rank / (ms * 1e-3) / 1e12
+
+
 def gemm_flops(cfg, counts=None):
     """Algorithmic FLOPs of both grouped GEMMs for T*k routed rows."""
     R = cfg.T * cfg.k
@@ -316,12 +332,9 @@ def run_ours(args):
     for t in timers:
         for name, v in t.durations_ms().items():
             per_kernel[name] = per_kernel.get(name, 0.0) + v / len(timers)
-    if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(ms, world, dev)
     fp4, comp = gemm_flops(cfg)
-    value = world * (fp4 + comp) / (ms * 1e-3) / 1e12
+    value = whole_job_tflops(fp4 + comp, world, ms)
 
     # roofline of the dominant kernel
     peaks, peak_src = load_peaks()
@@ -373,14 +386,10 @@ def run_ours(args):
             e1.synchronize()
             if i >= args.warmup:
                 e_times.append(e0.elapsed_time(e1))
-        e_ms = sum(e_times) / len(e_times)
-        if world > 1:
-            tt = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e_ms = float(tt.item())
+        e_ms = max_over_ranks(sum(e_times) / len(e_times), world, dev)
         h2d = x.numel() * 2 + logits.numel() * 4 + x_train.numel() * 2
         d2h = layer.out.numel() * 2 + 16
-        e2e = {"value": world * (fp4 + comp) / (e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e_ms,
+        e2e = {"value": whole_job_tflops(fp4 + comp, world, e_ms), "unit": UNIT, "ms_per_step": e_ms,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     cpu = None
