@@ -120,6 +120,32 @@ int quads_quantize_nvfp4(const uint16_t* x, int64_t rows, int64_t K, int64_t ld_
                          const int32_t* chan, int n_chan, uint16_t* resid_out,
                          void* ws, size_t ws_bytes, quads_stream_t stream);
 
+/* The same quantization as quads_quantize_nvfp4, for callers that cannot
+ * give this library any device memory beyond their inputs and outputs: code
+ * whose GPU memory is all owned by another allocator (a framework's pool, an
+ * arena sized once at start-up), plugin interfaces with no way to pass a
+ * workspace, latency-critical loops that cannot afford an allocation.  The
+ * pages have no counterpart: this is a deployment convenience, not a step of
+ * the method.
+ *   - It allocates nothing and takes no workspace.  The one scratch it needs
+ *     (one FP32 amax per row group, used when amax_in is NULL) lives in a
+ *     4 KiB file-scope device array that every GPU which loads the library
+ *     holds until the process exits.
+ *   - n_groups <= 1024; larger requests return QUADS_ERR_UNSUPPORTED_SHAPE
+ *     before anything is launched.  All other arguments and limits are those
+ *     of quads_quantize_nvfp4.
+ *   - The first call with a given device current looks up the array's device
+ *     address on that device (cudaGetSymbolAddress); make that first call
+ *     before any stream capture.
+ *   - Every call reuses the same array and clears it before use.  Calls that
+ *     can run at the same time on one GPU (other streams, other host threads)
+ *     race on it: serialize them. */
+int quads_quantize_nvfp4_noalloc(const uint16_t* x, int64_t rows, int64_t K, int64_t ld_x,
+                                 const int32_t* group_off, int n_groups, const float* amax_in,
+                                 uint8_t* codes, uint8_t* scales, int scale_layout, float* g_out,
+                                 const int32_t* chan, int n_chan, uint16_t* resid_out,
+                                 quads_stream_t stream);
+
 /* --------------------------------------------------------------- dequant
  * deq = e2m1 * e4m3 * g of a quantized matrix (the rollout's weight or
  * activation as the trainer sees it, [QUADS-fr §2.1]).  g: device

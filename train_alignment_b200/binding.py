@@ -66,6 +66,8 @@ _SIGS = {
     "quads_quantize_workspace_bytes": (c_sz, [c_i32]),
     "quads_quantize_nvfp4": (c_i32, [c_vp, c_i64, c_i64, c_i64, c_vp, c_i32, c_vp, c_vp, c_vp, c_i32, c_vp,
                                      c_vp, c_i32, c_vp, c_vp, c_sz, c_vp]),
+    "quads_quantize_nvfp4_noalloc": (c_i32, [c_vp, c_i64, c_i64, c_i64, c_vp, c_i32, c_vp, c_vp, c_vp, c_i32,
+                                             c_vp, c_vp, c_i32, c_vp, c_vp]),
     "quads_dequant": (c_i32, [c_vp, c_vp, c_i32, c_vp, c_vp, c_i32, c_i64, c_i64, c_vp, c_i32, c_vp]),
     "quads_channel_scores_workspace_bytes": (c_sz, [c_i64, c_i64]),
     "quads_channel_scores": (c_i32, [c_vp, c_i64, c_i64, c_vp, c_vp, c_vp, c_sz, c_vp]),

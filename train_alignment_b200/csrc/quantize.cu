@@ -13,6 +13,7 @@
 // consecutive blocks of a row (1 KB contiguous), grids are grid-stride loops
 // sized to a multiple of the SM count.
 #include <cstdio>
+#include <mutex>
 
 #include "common.cuh"
 
@@ -605,3 +606,93 @@ int quads_fakequant_weight_ste_backward(const uint16_t* grad_wfq, uint16_t* grad
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Quantize without any device allocation.
+//
+// Some callers cannot hand this library a workspace or let it obtain one:
+// code whose device memory is entirely owned by another allocator (a
+// framework's caching pool, a fixed arena sized once at start-up), plugin
+// interfaces that have no way to pass a scratch buffer through, and
+// latency-critical loops where an allocation's implicit synchronization is
+// not acceptable.  For them, this entry point keeps the only scratch the
+// quantizer needs -- one FP32 amax per row group -- in a file-scope device
+// array that the module loader places in every GPU's memory when the library
+// is loaded and that stays there until the process exits.
+//
+// The array's name is only a host-side stand-in for the device variable, so
+// host code never passes it to a kernel: the device address is obtained once
+// per device with cudaGetSymbolAddress (on the first call made with that
+// device current) and cached.  All calls share the array and it keeps the
+// last call's contents, so each call clears the part it uses before the amax
+// pass; calls that can overlap on the GPU (different streams, or different
+// host threads on one device) race on it and must be serialized by the caller.
+namespace quads {
+namespace {
+
+constexpr int kNoAllocMaxGroups = 1024;                     // 4 KiB of scratch per GPU
+static __device__ __align__(256) float g_noalloc_amax[kNoAllocMaxGroups];
+
+std::mutex g_noalloc_mutex;
+float* g_noalloc_scratch[64] = {nullptr};
+
+int noalloc_scratch(float** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+    return set_error(QUADS_ERR_CUDA, "no usable current CUDA device");
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_scratch[dev] == nullptr) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_amax);
+    if (e != cudaSuccess || p == nullptr)
+      return set_error(QUADS_ERR_CUDA, "cudaGetSymbolAddress of the quantizer scratch failed: %s",
+                       cudaGetErrorString(e));
+    g_noalloc_scratch[dev] = static_cast<float*>(p);
+  }
+  *out = g_noalloc_scratch[dev];
+  return QUADS_OK;
+}
+
+}  // namespace
+}  // namespace quads
+
+extern "C" int quads_quantize_nvfp4_noalloc(const uint16_t* x, int64_t rows, int64_t K, int64_t ld_x,
+                                            const int32_t* group_off, int n_groups, const float* amax_in,
+                                            uint8_t* codes, uint8_t* scales, int scale_layout, float* g_out,
+                                            const int32_t* chan, int n_chan, uint16_t* resid_out,
+                                            quads_stream_t stream) {
+  clear_error();
+  QUADS_TRY(validate_matrix(x, rows, K, ld_x));
+  QUADS_TRY(validate_groups(group_off, n_groups, rows));
+  QUADS_REQUIRE(n_groups <= kNoAllocMaxGroups, QUADS_ERR_UNSUPPORTED_SHAPE,
+                "the allocation-free quantizer supports at most %d row groups (got %d)", kNoAllocMaxGroups,
+                n_groups);
+  QUADS_REQUIRE(scale_layout == QUADS_SCALES_LINEAR || scale_layout == QUADS_SCALES_TILED,
+                QUADS_ERR_INVALID_ARG, "unknown scale layout %d", scale_layout);
+  QUADS_REQUIRE(codes && scales && g_out, QUADS_ERR_INVALID_ARG, "codes, scales and g_out must be non-null");
+  QUADS_REQUIRE(aligned(codes, 8), QUADS_ERR_INVALID_ARG, "codes must be 8-byte aligned");
+  QUADS_REQUIRE(n_chan >= 0 && n_chan <= kMaxChan, QUADS_ERR_UNSUPPORTED_SHAPE, "n_chan must be in [0, %d]",
+                kMaxChan);
+  QUADS_REQUIRE(n_chan == 0 || (chan && resid_out), QUADS_ERR_INVALID_ARG,
+                "chan and resid_out are required when n_chan > 0");
+  if (rows == 0) {
+    if (cudaMemsetAsync(g_out, 0, sizeof(float) * n_groups, stream) != cudaSuccess)
+      return set_error(QUADS_ERR_CUDA, "memset failed");
+    return QUADS_OK;
+  }
+  const float* amax = amax_in;
+  if (amax == nullptr) {
+    float* scratch = nullptr;
+    QUADS_TRY(noalloc_scratch(&scratch));
+    // launch_amax clears scratch[0, n_groups) before accumulating into it
+    QUADS_TRY(launch_amax(x, rows, K, ld_x, group_off, n_groups, scratch, stream));
+    amax = scratch;
+  }
+  QuantArgs a{};
+  a.x = x; a.rows = rows; a.K = K; a.ld = ld_x;
+  a.group_off = group_off; a.n_groups = n_groups; a.uniform_rows = group_off ? 1 : rows / n_groups;
+  a.amax = amax; a.codes = codes; a.scales = scales; a.scale_layout = scale_layout; a.g_out = g_out;
+  a.chan = chan; a.n_chan = n_chan; a.resid = n_chan ? resid_out : nullptr; a.resid_mode = 0;
+  a.w_fq = nullptr; a.fold = 1;
+  return launch_quantize(a, stream);
+}
