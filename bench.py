@@ -19,8 +19,9 @@ step time.  Multi-GPU runs are data-parallel replicas (each rank its own
 batch, no collective on the path): weak scaling.
 
 --impl reference times the CPU oracle (float64 numpy) on a bounded sample of
-the same workload (one eighth of the tokens and of the experts' weight
-syncs per step) on the host cores; under torchrun only rank 0 runs it.
+the same workload (the same fraction of the tokens and of the weight rows
+per step, sized so that the whole run takes about two minutes) on the host
+cores; under torchrun only rank 0 runs it.
 """
 import argparse
 import datetime
@@ -46,8 +47,8 @@ L2_FLUSH_BYTES = 256 << 20
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -189,23 +190,21 @@ class ClockSampler:
 
 
 class OracleSample:
-    """Bounded CPU sample of the workload for the oracle: per run, the
-    weight sync and straight-through backward of E/frac_experts experts and
-    the rollout forward + record replay of T/frac_tokens tokens.  Inputs and
-    every expert's NVFP4 weights (which the forward needs) are prepared once,
-    outside the timing."""
+    """Bounded CPU sample of the workload for the oracle: a fraction `frac` of
+    every part of one step -- the weight sync and straight-through backward of
+    that fraction of the weight rows, the rollout forward and record replay of
+    that fraction of the tokens.  Inputs and every expert's NVFP4 weights
+    (which the forward needs) are prepared once, outside the timing."""
 
-    def __init__(self, cfg, frac_tokens=8, frac_experts=8, seed=0):
+    def __init__(self, cfg, seed=0):
         import numpy as np
         from oracle import layer as OL
         from oracle import nvfp4 as Q
         from train_alignment_b200 import workloads as W
-        self.OL, self.Q, self.cfg = OL, Q, cfg
+        self.OL, self.Q, self.cfg, self.np = OL, Q, cfg, np
         inp = W.moe_layer_inputs(cfg, seed=seed, device="cpu")
-        self.T_s = max(cfg.T // frac_tokens, 1)
-        self.E_s = max(cfg.E // frac_experts, 1)
-        self.x = inp["x"][:self.T_s].float().numpy().astype(np.float64)
-        self.logits = inp["logits"][:self.T_s].numpy().astype(np.float64)
+        self.x = inp["x"].float().numpy().astype(np.float64)
+        self.logits = inp["logits"].numpy().astype(np.float64)
         self.w_gu = inp["w_gu"].float().numpy().astype(np.float64)
         self.w_d = inp["w_d"].float().numpy().astype(np.float64)
         r = np.random.default_rng(seed)
@@ -213,22 +212,33 @@ class OracleSample:
         self.chan_h = Q.pad_channels(np.sort(r.choice(cfg.F, cfg.n_chan_f, replace=False)))
         self.wgu_all = OL.weight_sync(self.w_gu, self.chan_x)
         self.wd_all = OL.weight_sync(self.w_d, self.chan_h)
+        self.set_fraction(1.0)
+
+    def set_fraction(self, frac):
+        cfg = self.cfg
+        self.frac = frac
+        self.T_s = max(1, int(round(cfg.T * frac)))
+        self.rows_gu = max(16, int(round(cfg.E * 2 * cfg.F * frac)))
+        self.rows_d = max(16, int(round(cfg.E * cfg.H * frac)))
         R = self.T_s * cfg.k
         self.flops = 2 * R * 2 * cfg.F * cfg.H + 2 * R * cfg.H * cfg.F + 2 * R * 2 * cfg.F * cfg.n_chan + \
             2 * R * cfg.H * cfg.n_chan_f
         self.desc = (f"oracle (float64 numpy) on {self.T_s} of {cfg.T} tokens and the weight sync + STE "
-                     f"backward of {self.E_s} of {cfg.E} experts per step")
+                     f"backward of {self.rows_gu} of {cfg.E * 2 * cfg.F} gate/up and {self.rows_d} of "
+                     f"{cfg.E * cfg.H} down weight rows per step")
 
     def run(self):
-        OL, Q, E_s = self.OL, self.Q, self.E_s
+        OL, Q, np = self.OL, self.Q, self.np
+        wgu = self.w_gu.reshape(-1, self.cfg.H)[:self.rows_gu][None]
+        wd = self.w_d.reshape(-1, self.cfg.F)[:self.rows_d][None]
         t0 = time.perf_counter()
-        OL.weight_sync(self.w_gu[:E_s], self.chan_x)
-        OL.weight_sync(self.w_d[:E_s], self.chan_h)
-        fwd = OL.rollout_forward(self.x, self.logits, self.wgu_all, self.wd_all, self.chan_x, self.chan_h,
-                                 self.cfg.k)
-        OL.trainer_replay(fwd, self.x, self.chan_x, self.chan_h)
-        Q.ste_backward(self.w_gu[:E_s], self.w_gu[:E_s])
-        Q.ste_backward(self.w_d[:E_s], self.w_d[:E_s])
+        OL.weight_sync(wgu, self.chan_x)
+        OL.weight_sync(wd, self.chan_h)
+        fwd = OL.rollout_forward(self.x[:self.T_s], self.logits[:self.T_s], self.wgu_all, self.wd_all,
+                                 self.chan_x, self.chan_h, self.cfg.k)
+        OL.trainer_replay(fwd, self.x[:self.T_s], self.chan_x, self.chan_h)
+        Q.ste_backward(wgu, wgu)
+        Q.ste_backward(wd, wd)
         return time.perf_counter() - t0
 
 
@@ -247,7 +257,12 @@ def run_reference(args):
         return 0
     from train_alignment_b200 import workloads as W
     cfg = W.CONFIGS[args.workload]
-    sample = OracleSample(cfg, 8, 8, seed=0)
+    sample = OracleSample(cfg, seed=0)
+    # size each step so that warm-up + timed steps take about two minutes
+    sample.set_fraction(1.0 / 64)
+    probe = sample.run()
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    sample.set_fraction(min(1.0, max(1.0 / 4096, budget / max(probe * 64, 1e-6))))
     for _ in range(args.warmup):
         sample.run()
     times = [sample.run() for _ in range(args.steps)]
@@ -299,10 +314,39 @@ def run_ours(args):
 
     for _ in range(max(args.warmup, 3)):
         flush.zero_()
+        n0 = B.launch_count()
         layer.step(x, logits, x_train, g_gu, g_d)
+        launches_per_step = B.launch_count() - n0
     torch.cuda.synchronize()
     assert B.device_status() == B.OK, B.last_error()
     rpad = int(layer.expert_off[-1].item())
+
+    # one step captured as a CUDA graph (stage events inside the graph)
+    timing_mode = "cuda-graph"
+    graph, gtimer = None, L.StageTimer(True, external=True)
+    try:
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            layer.step(x, logits, x_train, g_gu, g_d)
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()                  # with an event between every two kernels
+        with torch.cuda.graph(graph):
+            layer.step(x, logits, x_train, g_gu, g_d, timer=gtimer)
+        graph_plain = torch.cuda.CUDAGraph()            # the step alone
+        with torch.cuda.graph(graph_plain):
+            layer.step(x, logits, x_train, g_gu, g_d)
+        for _ in range(3):
+            flush.zero_()
+            graph.replay()
+            graph_plain.replay()
+        torch.cuda.synchronize()
+        gtimer.durations_ms()
+    except Exception as exc:  # noqa: BLE001 -- fall back to stream launches
+        graph = None
+        timing_mode = f"stream launches ({type(exc).__name__} in graph capture: {str(exc)[:120]})"
+        torch.cuda.synchronize()
 
     uuid = None
     try:
@@ -315,23 +359,42 @@ def run_ours(args):
     barrier()
     torch.cuda.synchronize()
     launches0 = B.launch_count()
-    timers = []
-    for _ in range(args.steps):
+    # timed region: exactly K steps, each the whole path, events around each step
+    step_ms = []
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
         flush.zero_()                                   # L2 flush, outside the events
-        t = L.StageTimer(True)
-        layer.step(x, logits, x_train, g_gu, g_d, timer=t)
-        timers.append(t)
+        ev[i][0].record()
+        if graph is not None:
+            graph_plain.replay()
+        else:
+            layer.step(x, logits, x_train, g_gu, g_d)
+        ev[i][1].record()
     torch.cuda.synchronize()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
     barrier()
     launches = B.launch_count() - launches0
+    if graph is not None:                               # graph replays bypass the host-side counter
+        launches = args.steps * launches_per_step
     clk = clocks.stop()
     assert B.device_status() == B.OK, B.last_error()
-    step_ms = [t.marks[0][1].elapsed_time(t.marks[-1][1]) for t in timers]
     ms = sum(step_ms) / len(step_ms)
-    per_kernel = {}
-    for t in timers:
+    # per-kernel breakdown: the same K steps again with an event between every two kernels
+    per_kernel, inst_ms = {}, []
+    for _ in range(args.steps):
+        flush.zero_()
+        if graph is not None:
+            graph.replay()
+            torch.cuda.synchronize()
+            t = gtimer
+        else:
+            t = L.StageTimer(True)
+            layer.step(x, logits, x_train, g_gu, g_d, timer=t)
+            t.marks[-1][1].synchronize()
+        inst_ms.append(t.marks[0][1].elapsed_time(t.marks[-1][1]))
         for name, v in t.durations_ms().items():
-            per_kernel[name] = per_kernel.get(name, 0.0) + v / len(timers)
+            per_kernel[name] = per_kernel.get(name, 0.0) + v / args.steps
+    assert B.device_status() == B.OK, B.last_error()
     ms = max_over_ranks(ms, world, dev)
     fp4, comp = gemm_flops(cfg)
     value = whole_job_tflops(fp4 + comp, world, ms)
@@ -394,7 +457,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        sample = OracleSample(cfg, 1, 1, seed=0)
+        sample = OracleSample(cfg, seed=0)
         dt, flops, desc = sample.run(), sample.flops, sample.desc
         cpu = {"value": flops / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                "sample": desc + f"; {dt:.1f} s", "seconds": dt}
@@ -420,6 +483,8 @@ def run_ours(args):
         "clocks": clk,
         "e2e": e2e,
         "gpu_launches": launches,
+        "timing": timing_mode,
+        "instrumented_ms_per_step": sum(inst_ms) / len(inst_ms),
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)

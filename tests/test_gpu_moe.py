@@ -33,7 +33,8 @@ def test_router_parity(cuda_lib, T, E, k, renorm):
     assert np.allclose(f32_of(w), w_ref, rtol=2e-6, atol=1e-7)
 
 
-@pytest.mark.parametrize("T,E,k", [(1, 4, 1), (300, 8, 2), (2048, 8, 2), (4096, 128, 8), (5000, 64, 4)])
+@pytest.mark.parametrize("T,E,k", [(1, 4, 1), (300, 8, 2), (2048, 8, 2), (4096, 128, 8), (5000, 64, 4),
+                                   (5000, 64, 8), (16384, 128, 8)])
 def test_permute_parity(cuda_lib, T, E, k):
     l = _logits(T, E, 7 * T + E, "zipf")
     idx_ref, _ = M.router_topk(l.numpy().astype(np.float64), k)

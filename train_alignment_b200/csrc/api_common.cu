@@ -45,6 +45,15 @@ int num_sms() {
   return g_sm_count[dev];
 }
 
+int persistent_grid(const void* kernel, int threads, size_t smem, int64_t work_blocks) {
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) != cudaSuccess || per_sm < 1)
+    per_sm = 1;
+  int64_t cap = static_cast<int64_t>(per_sm) * num_sms();
+  int64_t g = work_blocks < cap ? work_blocks : cap;
+  return static_cast<int>(g < 1 ? 1 : g);
+}
+
 }  // namespace quads
 
 extern "C" {

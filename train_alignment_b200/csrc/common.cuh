@@ -12,6 +12,9 @@ namespace quads {
 // ------------------------------------------------------------------ host side
 
 int set_error(int code, const char* fmt, ...);
+// Grid for a persistent grid-stride kernel: min(work items / per_block,
+// resident blocks per SM x SMs).
+int persistent_grid(const void* kernel, int threads, size_t smem, int64_t work_blocks);
 void clear_error();
 void count_launches(uint64_t n);
 int num_sms();
@@ -40,6 +43,20 @@ __host__ __device__ inline int64_t scale_bytes(int64_t rows, int64_t K, int layo
   return ceil_div(rows, 128) * 128 * ceil_div(nkb, 4) * 4;
 }
 
+// Division of n < 2^31 by a fixed d >= 1 with a multiply-high and a shift
+// (the round-up multiplier: s = ceil(log2 d), m = floor(2^32 (2^s - d) / d) + 1,
+// n / d = (umulhi(n, m) + n) >> s).
+struct FastDiv {
+  uint32_t d, m, s;
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+  uint32_t s = 0;
+  while ((uint64_t(1) << s) < d) ++s;
+  uint64_t m = ((uint64_t(1) << 32) * ((uint64_t(1) << s) - d)) / d + 1;
+  return FastDiv{d, static_cast<uint32_t>(m), s};
+}
+__device__ __forceinline__ uint32_t fast_div(uint32_t n, const FastDiv& f) { return (__umulhi(n, f.m) + n) >> f.s; }
+
 // ---------------------------------------------------------------- device side
 
 constexpr float kNvfp4Range = 2688.0f;   // 6 * 448
@@ -50,9 +67,11 @@ __device__ __forceinline__ uint32_t float_to_bf16_bits(float f) {
   return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f)));
 }
 
-// Two floats -> packed BF16 pair (lo in the low half).
+// Two floats -> packed BF16 pair (lo in the low half), round to nearest even.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  return float_to_bf16_bits(lo) | (float_to_bf16_bits(hi) << 16);
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 // Value of an E4M3 (fn) scale code with the sign bit clear: 4 exponent bits
@@ -87,6 +106,74 @@ __device__ __forceinline__ uint32_t e2m1x8_from_float(const float* v) {
   return out;
 }
 
+// ---- packed helpers (two fp32 in a 64-bit register: element 0 in the low half)
+
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+  return (static_cast<uint64_t>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
+}
+__device__ __forceinline__ float lo_f32(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float hi_f32(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
+// Two IEEE round-to-nearest fp32 products in one instruction.
+__device__ __forceinline__ uint64_t fmul2_rn(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// A word of two BF16 values -> the two values as fp32 (exact).
+__device__ __forceinline__ uint64_t bf16x2_to_f32x2(uint32_t w) {
+  return (static_cast<uint64_t>(w & 0xFFFF0000u) << 32) | (w << 16);
+}
+// Two floats -> BF16 pair, lo in the low half (round to nearest even), one instruction.
+__device__ __forceinline__ uint32_t f32x2_to_bf16x2(uint64_t v) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi_f32(v)), "f"(lo_f32(v)));
+  return r;
+}
+
+// Eight packed fp32 pairs (elements 2i, 2i+1 in y[i]) -> eight E2M1 codes,
+// element i in nibble i (nearest-even, saturating, sign kept).
+__device__ __forceinline__ uint32_t e2m1x8_from_pairs(const uint64_t* y) {
+  float v[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = lo_f32(y[i]);
+    v[2 * i + 1] = hi_f32(y[i]);
+  }
+  return e2m1x8_from_float(v);
+}
+
+// Eight E2M1 codes (nibble i = element i) -> four f16x2 values (exact).
+__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t codes, uint32_t (&h)[4]) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+      : "r"(codes));
+}
+// f16x2 product (exact here: both factors carry few significant bits).
+__device__ __forceinline__ uint32_t hmul2_rn(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+// f16x2 -> two fp32 (exact).
+__device__ __forceinline__ uint64_t f16x2_to_f32x2(uint32_t h) {
+  float lo, hi;
+  asm("{\n\t.reg .f16 l, u;\n\tmov.b32 {l, u}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, u;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(h));
+  return pack_f32x2(lo, hi);
+}
+// An E4M3 scale value (exactly representable in f16) as an f16x2 pair.
+__device__ __forceinline__ uint32_t f16x2_splat(float v) {
+  uint32_t r;
+  asm("{\n\t.reg .f16 t;\n\tcvt.rn.f16.f32 t, %1;\n\tmov.b32 %0, {t, t};\n\t}" : "=r"(r) : "f"(v));
+  return r;
+}
+
 // Value of a 4-bit E2M1 code: magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6}.
 __device__ __forceinline__ float e2m1_value(uint32_t c) {
   uint32_t m = c & 7u;
@@ -104,11 +191,11 @@ __device__ __forceinline__ int64_t tiled_scale_offset(int64_t row, int64_t kb, i
 struct RowGroups {
   const int32_t* off_smem;   // n + 1 entries, or nullptr
   int n;
-  int64_t uniform_rows;
+  FastDiv uniform;           // rows per group when off_smem is null
   __device__ __forceinline__ int of(int64_t row) const {
     if (off_smem == nullptr) {
       if (n == 1) return 0;
-      return static_cast<int>(row / uniform_rows);
+      return static_cast<int>(fast_div(static_cast<uint32_t>(row), uniform));
     }
     int lo = 0, hi = n - 1;             // last i with off[i] <= row
     while (lo < hi) {
@@ -180,6 +267,65 @@ __device__ __forceinline__ uint32_t qblock_code(const QBlock& b, int i) {
 // fp32(val(q) * val(s) * g) -- exact product of the first two, one rounding.
 __device__ __forceinline__ float deq_f32(uint32_t code, float sv, float g) {
   return __fmul_rn(__fmul_rn(e2m1_value(code), sv), g);
+}
+
+// One quantized block: codes (nibble i = element i), E4M3 scale and its value.
+struct QCore {
+  uint32_t lo, hi, scale;
+  float sv;
+};
+
+// The quantizer on 16 BF16 values given as 8 packed words (element 2i in the
+// low half of w[i]); same operations and rounding as quantize_block.
+__device__ __forceinline__ QCore quant_core(const uint32_t (&w)[8], float g) {
+  uint32_t m = 0u;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m = __vmaxu2(m, w[i] & 0x7FFF7FFFu);
+  const float amax = bf16_bits_to_float(max(m & 0xFFFFu, m >> 16));
+  uint32_t s = 0;
+  if (g != 0.0f) s = e4m3_from_float(__fdiv_rn(amax, __fmul_rn(6.0f, g)));
+  QCore r;
+  r.scale = s;
+  r.sv = e4m3_value(s);
+  const float S = __fmul_rn(r.sv, g);
+  if (S == 0.0f) {
+    uint32_t lo = 0, hi = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      lo |= ((w[i] >> 15) & 1u) << (8 * i + 3) | ((w[i] >> 31) & 1u) << (8 * i + 7);
+      hi |= ((w[4 + i] >> 15) & 1u) << (8 * i + 3) | ((w[4 + i] >> 31) & 1u) << (8 * i + 7);
+    }
+    r.lo = lo;
+    r.hi = hi;
+    return r;
+  }
+  const float inv = __frcp_rn(S);
+  const uint64_t inv2 = pack_f32x2(inv, inv);
+  uint64_t y[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) y[i] = fmul2_rn(bf16x2_to_f32x2(w[i]), inv2);
+  r.lo = e2m1x8_from_pairs(y);
+  r.hi = e2m1x8_from_pairs(y + 4);
+  return r;
+}
+
+// BF16 of the dequantized block: fp32(e2m1 * e4m3 * g) (fold) or the exact
+// e2m1 * e4m3; the products e2m1 * e4m3 are exact in f16.
+__device__ __forceinline__ void deq_block_bf16(const QCore& q, float g, int fold, uint32_t (&out)[8]) {
+  uint32_t h[8];
+  uint32_t h0[4], h1[4];
+  e2m1x8_to_f16x2(q.lo, h0);
+  e2m1x8_to_f16x2(q.hi, h1);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) { h[i] = h0[i]; h[4 + i] = h1[i]; }
+  const uint32_t sv2 = f16x2_splat(q.sv);
+  const uint64_t g2 = pack_f32x2(g, g);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    uint64_t f = f16x2_to_f32x2(hmul2_rn(h[i], sv2));
+    if (fold) f = fmul2_rn(f, g2);
+    out[i] = f32x2_to_bf16x2(f);
+  }
 }
 
 }  // namespace quads

@@ -6,21 +6,24 @@
 // does the bulk of the work ([QUADS-fr §2.2.B], [QUADS-es §2.2.B]):
 //   Y = g_a g_w (A_fp4 (x) W_fp4) + R_C . Wc
 //
-// Design (one persistent CTA per SM, 192 threads, warp-specialized):
+// Design (one persistent CTA per SM, 224 threads, warp-specialized):
 //   warp 0 lane 0  TMA producer: 128x256 FP4 tiles of A and W (128-byte
 //                  swizzle) and their 512-byte block-scale tiles (bulk copy)
 //                  into a multi-stage shared-memory ring; per output tile the
 //                  BF16 compensation operands R [128 x |C|] and Wc [128 x |C|]
 //                  (32-byte swizzle, 16 channels per box).
-//   warp 1         allocates 512 TMEM columns; lane 0 issues tcgen05.cp of the
-//                  scales into TMEM and tcgen05.mma kind::mxf4nvf4 (block16
+//   warp 6 lane 0  copies each stage's block scales into a TMEM slot
+//                  (tcgen05.cp), signalling the MMA thread per slot;
+//   warp 1         allocates 512 TMEM columns; lane 0 issues
+//                  tcgen05.mma kind::mxf4nvf4 (block16
 //                  E4M3 scales, K = 64 per instruction) into a double-buffered
 //                  FP32 accumulator, then tcgen05.mma kind::f16 (BF16) for
 //                  R_C . Wc into a second accumulator.
 //   warps 2..5     epilogue: tcgen05.ld both accumulators, y = G * acc + comp,
-//                  BF16 stores.
+//                  BF16 rows staged in shared memory, TMA tensor stores of
+//                  32 x 32 boxes.
 // TMEM columns: [0,128) and [128,256) main accumulators, [256,384) the
-// compensation accumulator, [384,448) two buffers of scale factors.
+// compensation accumulator, [384,512) four slots of scale factors.
 // Tiles are (expert, 128-row block, 128-column block); experts' row segments
 // are 128-aligned by the permutation, so no tile straddles two experts.
 // No TMA multicast is used anywhere.
@@ -50,7 +53,10 @@ constexpr int kBBytes = BN * kStageRowBytes;        // 16384
 constexpr int kSfBytes = 4 * 512;                   // scales of 4 MMAs for 128 rows
 constexpr int kStageBytes = kABytes + kBBytes + 2 * kSfBytes;   // 36864
 constexpr int kCompChunkBytes = 128 * 32;           // 128 rows x 16 BF16
-constexpr int kThreads = 192;
+constexpr int kOutChunkBytes = 32 * 64;             // 32 rows x 32 BF16 output columns
+constexpr int kOutStageBytes = 4 * 2 * kOutChunkBytes;   // 4 epilogue warps, 2 buffers each
+constexpr int kThreads = 224;                    // 7 warps
+constexpr int kSfSlots = 4;                      // scale-factor buffers in TMEM
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kCompCol = 256;
 constexpr uint32_t kSfCol = 384;
@@ -145,6 +151,24 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
                : "memory");
 }
 
+// Store a box of the output from shared memory through TMA (bulk-group
+// completion tracked by the issuing thread).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(src)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
 __device__ __forceinline__ void tmem_alloc(uint32_t slot, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot), "r"(ncols) : "memory");
 }
@@ -225,7 +249,7 @@ __device__ __forceinline__ int expert_of_row(const int32_t* off_s, int E, int ro
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                         const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_wc,
-                        GemmParams p) {
+                        const __grid_constant__ CUtensorMap tm_y, GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -234,7 +258,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nch = p.n_chan / 16;
   const uint32_t comp_r = base + S * kStageBytes;
   const uint32_t comp_wc = comp_r + nch * kCompChunkBytes;
-  const uint32_t bar0 = comp_wc + nch * kCompChunkBytes;           // 8-byte aligned
+  const uint32_t out_stage = comp_wc + nch * kCompChunkBytes;     // 1024-byte aligned
+  const uint32_t bar0 = out_stage + kOutStageBytes;                 // 8-byte aligned
   // barrier addresses
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
@@ -244,10 +269,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t acc_empty0 = comp_full + 32;      // two barriers
   const uint32_t compacc_empty = comp_full + 48;
   const uint32_t drain_bar = comp_full + 56;
-  uint8_t* const misc = base_ptr + (comp_full + 64 - base);
+  auto sf_full = [&](int i) { return comp_full + 64 + 8u * i; };            // kSfSlots barriers
+  auto sf_empty = [&](int i) { return comp_full + 64 + 8u * (kSfSlots + i); };
+  const uint32_t sf_drain = comp_full + 64 + 8u * (2 * kSfSlots);
+  uint8_t* const misc = base_ptr + (sf_drain + 8 - base);
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(misc);
   volatile int* const abort_flag = reinterpret_cast<volatile int*>(misc + 4);
   int32_t* const off_s = reinterpret_cast<int32_t*>(misc + 16);
+  float* const gscale_s = reinterpret_cast<float*>(off_s + p.E + 1);   // g_a(e) * g_w[e]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -263,6 +292,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(acc_empty0 + 8, 4);
     mbar_init(compacc_empty, 4);
     mbar_init(drain_bar, 1);
+    for (int i = 0; i < kSfSlots; ++i) {
+      mbar_init(sf_full(i), 1);
+      mbar_init(sf_empty(i), 1);
+    }
+    mbar_init(sf_drain, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -270,7 +304,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(smem_addr(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
-  for (int i = threadIdx.x; i <= p.E; i += blockDim.x) off_s[i] = p.expert_off[i];
+  for (int i = threadIdx.x; i <= p.E; i += blockDim.x) {
+    off_s[i] = p.expert_off[i];
+    if (i < p.E) gscale_s[i] = __fmul_rn(p.g_a[p.g_a_per_expert ? i : 0], p.g_w[i]);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -337,21 +374,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int ks = 0; ks < nks; ++ks, ++it) {
         const int s = it % S;
         const uint32_t ph = (it / S) & 1;
+        const int slot = it % kSfSlots;
         if (!mbar_wait(full_bar(s), ph, abort_flag, p.timeout_ns)) { ok = false; break; }
+        if (!mbar_wait(sf_full(slot), (it / kSfSlots) & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
         tc_fence_after();
         const int nkb = min(4, nkb_total - ks * 4);
         const uint32_t st = base + s * kStageBytes;
-        const uint32_t tsfa = tmem + kSfCol + (it & 1) * 32;
+        const uint32_t tsfa = tmem + kSfCol + slot * 32;
         const uint32_t tsfb = tsfa + 16;
-        for (int kb = 0; kb < nkb; ++kb) {
-          tc_copy_scales(tsfa + kb * 4, desc_scales(st + kABytes + kBBytes + kb * 512));
-          tc_copy_scales(tsfb + kb * 4, desc_scales(st + kABytes + kBBytes + kSfBytes + kb * 512));
-        }
         for (int kb = 0; kb < nkb; ++kb) {
           mma_fp4(dacc, desc_kmajor_sw128(st + kb * kMmaKBytes), desc_kmajor_sw128(st + kABytes + kb * kMmaKBytes),
                   kIdescFp4, tsfa + kb * 4, tsfb + kb * 4, (ks | kb) != 0 ? 1u : 0u);
         }
         tc_commit(empty_bar(s));
+        tc_commit(sf_empty(slot));
       }
       if (!ok) break;
       if (nch) {
@@ -373,10 +409,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit(drain_bar);
       mbar_wait(drain_bar, 0, nullptr, kDrainTimeoutNs);
     }
-  } else if (warp >= 2) {
+  } else if (warp == 6 && lane == 0) {
+    // ------------------------------------------------------- scale copies
+    // Copies each stage's block scales from shared memory into a TMEM slot
+    // (one tcgen05.cp per 128 rows x 4 scales) so that the MMA thread only
+    // issues MMAs; copies and MMAs then overlap.
+    int it = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      for (int ks = 0; ks < nks; ++ks, ++it) {
+        const int s = it % S, slot = it % kSfSlots;
+        if (!mbar_wait(full_bar(s), (it / S) & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+        if (!mbar_wait(sf_empty(slot), ((it / kSfSlots) & 1) ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+        tc_fence_after();
+        const int nkb = min(4, nkb_total - ks * 4);
+        const uint32_t st = base + s * kStageBytes;
+        const uint32_t tsfa = tmem + kSfCol + slot * 32;
+        for (int kb = 0; kb < nkb; ++kb) {
+          tc_copy_scales(tsfa + kb * 4, desc_scales(st + kABytes + kBBytes + kb * 512));
+          tc_copy_scales(tsfa + 16 + kb * 4, desc_scales(st + kABytes + kBBytes + kSfBytes + kb * 512));
+        }
+        tc_commit(sf_full(slot));
+      }
+    }
+    if (!ok) {
+      tc_commit(sf_drain);
+      mbar_wait(sf_drain, 0, nullptr, kDrainTimeoutNs);
+    }
+  } else if (warp >= 2 && warp <= 5) {
     // ----------------------------------------------------------- epilogue
-    const int q = warp & 3;                       // TMEM lane quarter of this warp
-    int tc = 0;
+    // Each warp owns 32 accumulator rows (its TMEM lane quarter).  Per
+    // 32-column chunk: TMEM -> registers -> y = G * acc + comp -> BF16 row in
+    // a 2 KB shared buffer -> one TMA store of the 32 x 32 box.  Two buffers
+    // per warp; a buffer is rewritten only after its previous store has read it.
+    const int q = warp & 3;
+    const uint32_t stg = out_stage + (warp - 2) * 2 * kOutChunkBytes;
+    int tc = 0, nstore = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++tc) {
       const int mt = t / n_ntiles, nt = t - mt * n_ntiles;
       const int m0 = mt * BM;
@@ -385,16 +453,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t ph = (tc >> 1) & 1;
       if (!mbar_wait(acc_full0 + 8 * buf, ph, abort_flag, p.timeout_ns)) break;
       tc_fence_after();
-      const float G = __fmul_rn(p.g_a[p.g_a_per_expert ? e : 0], p.g_w[e]);
-      const int64_t row = m0 + q * 32 + lane;
-      uint16_t* const yrow = p.y + row * p.N + nt * BN;
+      const float G = gscale_s[e];
       const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = 0; c < BN / 32; ++c, ++nstore) {
         uint32_t v[32], w[32];
         tmem_load32(lane_base + buf * BN + c * 32, v);
         if (nch) tmem_load32(lane_base + kCompCol + c * 32, w);
         tmem_wait_ld();
+        if (c == BN / 32 - 1) {
+          // every TMEM read of this tile is done: hand the accumulators back
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(acc_empty0 + 8 * buf);
+            if (nch) mbar_arrive(compacc_empty);
+          }
+        }
         uint32_t o[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
@@ -405,17 +480,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           o[j] = pack_bf16x2(a0, a1);
         }
-        uint4* dst = reinterpret_cast<uint4*>(yrow + c * 32);
+        const uint32_t sb = stg + (nstore & 1) * kOutChunkBytes;
+        if (lane == 0) bulk_wait_read_1();
+        __syncwarp();
+        const uint32_t row_addr = sb + lane * 64;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) dst[j] = make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(acc_empty0 + 8 * buf);
-        if (nch) mbar_arrive(compacc_empty);
+        for (int j = 0; j < 4; ++j) st_shared_v4(row_addr + j * 16, o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tm_y, sb, nt * BN + c * 32, m0 + q * 32);
+          bulk_commit();
+        }
       }
     }
+    if (lane == 0) bulk_wait_all();
   }
   __syncwarp();
   tc_fence_before();
@@ -472,7 +551,8 @@ int make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64
 
 size_t gemm_smem_bytes(int stages, int n_chan, int E) {
   return 1024 + static_cast<size_t>(stages) * kStageBytes + static_cast<size_t>(n_chan / 16) * 2 * kCompChunkBytes +
-         static_cast<size_t>(2 * stages + 8) * 8 + 16 + static_cast<size_t>(E + 1) * 4;
+         kOutStageBytes + static_cast<size_t>(2 * stages + 9 + 2 * kSfSlots) * 8 + 16 +
+         static_cast<size_t>(2 * E + 1) * 4;
 }
 
 }  // namespace
@@ -506,7 +586,7 @@ int quads_moe_grouped_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales
                 QUADS_ERR_INVALID_ARG, "matrix pointers must be 16-byte aligned");
   if (rows_cap == 0) return QUADS_OK;
 
-  CUtensorMap tm_a, tm_b, tm_r, tm_wc;
+  CUtensorMap tm_a, tm_b, tm_r, tm_wc, tm_y;
   QUADS_TRY(make_map_2d(&tm_a, a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, rows_cap, kStageRowBytes, BM,
                         CU_TENSOR_MAP_SWIZZLE_128B));
   QUADS_TRY(make_map_2d(&tm_b, w_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, E * N, kStageRowBytes, BN,
@@ -520,6 +600,8 @@ int quads_moe_grouped_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales
     tm_r = tm_a;
     tm_wc = tm_a;
   }
+  QUADS_TRY(make_map_2d(&tm_y, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, rows_cap, 32, 32,
+                        CU_TENSOR_MAP_SWIZZLE_NONE));
   const size_t smem_cap = 232448;   // 227 KB per block on sm_100
   int stages = kMaxStages;
   while (stages >= 2 && gemm_smem_bytes(stages, n_chan, E) > smem_cap) --stages;
@@ -545,7 +627,7 @@ int quads_moe_grouped_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales
   const int64_t max_tiles = (rows_cap / BM) * (N / BN);
   int grid = num_sms();
   if (grid > max_tiles) grid = static_cast<int>(max_tiles);
-  grouped_gemm_kernel<<<grid, kThreads, smem, stream>>>(tm_a, tm_b, tm_r, tm_wc, p);
+  grouped_gemm_kernel<<<grid, kThreads, smem, stream>>>(tm_a, tm_b, tm_r, tm_wc, tm_y, p);
   count_launches(1);
   return check_launch("grouped_gemm_kernel");
 }

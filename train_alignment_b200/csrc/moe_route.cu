@@ -163,6 +163,66 @@ __global__ void __launch_bounds__(kRankThreads) rank_kernel(const int32_t* __res
   }
 }
 
+// Whole permutation in one block for small batches (<= kSmallPairs pairs):
+// histogram, padded offsets, pad rows and the in-order ranking.
+constexpr int kSmallThreads = 1024;
+constexpr int kSmallPairs = 32768;
+
+__global__ void __launch_bounds__(kSmallThreads) permute_small_kernel(const int32_t* __restrict__ idx,
+                                                                      int n_pairs, int k, int E,
+                                                                      int32_t* __restrict__ expert_off,
+                                                                      int32_t* __restrict__ row_of,
+                                                                      int32_t* __restrict__ src_of) {
+  constexpr int kWarps = kSmallThreads / 32;
+  __shared__ int32_t cnt[kMaxE];
+  __shared__ int32_t running[kMaxE];
+  __shared__ int32_t padded[kMaxE];
+  __shared__ int32_t wcnt[kWarps][kMaxE];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < E; i += blockDim.x) cnt[i] = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i < n_pairs; i += blockDim.x) {
+    const int e = idx[i];
+    if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
+  }
+  __syncthreads();
+  if (threadIdx.x < E) padded[threadIdx.x] = (cnt[threadIdx.x] + 127) / 128 * 128;
+  __syncthreads();
+  if (threadIdx.x < E) {
+    const int e = threadIdx.x;
+    int off = 0;
+    for (int j = 0; j < e; ++j) off += padded[j];
+    expert_off[e] = off;
+    running[e] = off;
+    for (int r = off + cnt[e]; r < off + padded[e]; ++r) src_of[r] = -1;
+    if (e == E - 1) expert_off[E] = off + padded[e];
+  }
+  for (int r0 = 0; r0 < n_pairs; r0 += kSmallThreads) {
+    for (int i = threadIdx.x; i < kWarps * kMaxE; i += blockDim.x) (&wcnt[0][0])[i] = 0;
+    __syncthreads();
+    const int i = r0 + threadIdx.x;
+    const bool valid = i < n_pairs;
+    const int e = valid ? idx[i] : -1;
+    const unsigned int peers = __match_any_sync(0xffffffffu, e);
+    const int rank_w = __popc(peers & ((1u << lane) - 1u));
+    if (valid && lane == __ffs(peers) - 1 && e >= 0 && e < E) wcnt[wid][e] = __popc(peers);
+    __syncthreads();
+    if (valid && e >= 0 && e < E) {
+      int pos = running[e] + rank_w;
+      for (int w = 0; w < wid; ++w) pos += wcnt[w][e];
+      row_of[i] = pos;
+      src_of[pos] = i / k;
+    }
+    __syncthreads();
+    for (int x = threadIdx.x; x < E; x += blockDim.x) {
+      int add = 0;
+      for (int w = 0; w < kWarps; ++w) add += wcnt[w][x];
+      running[x] += add;
+    }
+    __syncthreads();
+  }
+}
+
 // ------------------------------------------------------------------- gather
 
 // One warp per expert-ordered row p < expert_off[E].
@@ -209,7 +269,7 @@ __global__ void __launch_bounds__(256) swiglu_kernel(const uint16_t* __restrict_
     if (i < E) am_s[i] = 0u;
   }
   __syncthreads();
-  RowGroups grp{off_s, E, 1};
+  RowGroups grp{off_s, E, FastDiv{1u, 1u, 0u}};
   const int64_t rows = off_s[E];
   const int64_t per_row = F / 8;
   const int64_t total = rows * per_row;
@@ -229,7 +289,7 @@ __global__ void __launch_bounds__(256) swiglu_kernel(const uint16_t* __restrict_
       for (int hl = 0; hl < 2; ++hl) {
         float gt = bf16_bits_to_float(hl ? (gp[j] >> 16) : (gp[j] & 0xFFFFu));
         float ut = bf16_bits_to_float(hl ? (up[j] >> 16) : (up[j] & 0xFFFFu));
-        float sg = __fdiv_rn(gt, __fadd_rn(1.0f, expf(-gt)));
+        float sg = __fdividef(gt, 1.0f + __expf(-gt));   // relative error ~1e-6, far below BF16 rounding
         r[hl] = __fmul_rn(sg, ut);
       }
       o[j] = pack_bf16x2(r[0], r[1]);
@@ -330,6 +390,12 @@ int quads_moe_permute(const int32_t* topk_idx, int64_t T, int k, int E, int32_t*
   QUADS_REQUIRE(ws && ws_bytes >= quads_moe_permute_workspace_bytes(T, k, E), QUADS_ERR_INVALID_ARG,
                 "workspace of %zu bytes required", quads_moe_permute_workspace_bytes(T, k, E));
   const int64_t n_pairs = T * k;
+  if (n_pairs <= kSmallPairs) {
+    permute_small_kernel<<<1, kSmallThreads, 0, stream>>>(topk_idx, static_cast<int>(n_pairs), k, E, expert_off,
+                                                          row_of, src_of);
+    count_launches(1);
+    return check_launch("permute_small_kernel");
+  }
   int n_chunks = static_cast<int>(ceil_div(n_pairs, kChunk));
   if (n_chunks < 1) n_chunks = 1;
   int32_t* cnt = static_cast<int32_t*>(ws);

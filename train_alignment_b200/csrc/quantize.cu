@@ -23,10 +23,11 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kMaxGroupsSmem = 1024;
 constexpr int kMaxChan = 256;
+constexpr int64_t kMaxBlocks = int64_t(1) << 31;
 
 int grid_for(int64_t work, int per_block = kThreads) {
   int64_t g = ceil_div(work, per_block);
-  int64_t cap = static_cast<int64_t>(num_sms()) * 8;
+  int64_t cap = static_cast<int64_t>(num_sms()) * 16;
   if (g > cap) g = cap;
   if (g < 1) g = 1;
   return static_cast<int>(g);
@@ -34,10 +35,11 @@ int grid_for(int64_t work, int per_block = kThreads) {
 
 // --------------------------------------------------------------------- amax
 
-__global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t* __restrict__ x, int64_t rows,
-                                                        int64_t K, int64_t ld, const int32_t* group_off,
-                                                        int n_groups, int64_t uniform_rows,
-                                                        unsigned int* __restrict__ out_bits) {
+// One warp per row; each lane reads 32 bytes (16 elements) per pass, four
+// passes in flight; |x| maxima on the BF16 bit patterns, two per word.
+__global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t K,
+                                                        int64_t ld, const int32_t* group_off, int n_groups,
+                                                        FastDiv uniform, unsigned int* __restrict__ out_bits) {
   extern __shared__ int32_t smem[];
   int32_t* off_s = smem;                                   // n_groups + 1 (explicit groups)
   unsigned int* amax_s = reinterpret_cast<unsigned int*>(smem + n_groups + 1);
@@ -46,34 +48,39 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t* __restri
     if (i < n_groups) amax_s[i] = 0u;
   }
   __syncthreads();
-  RowGroups grp{group_off ? off_s : nullptr, n_groups, uniform_rows};
-  const int64_t nkb = K / 16;
-  const int64_t total = rows * nkb;
+  RowGroups grp{group_off ? off_s : nullptr, n_groups, uniform};
   const int lane = threadIdx.x & 31;
-  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t wstride = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  for (int64_t base = warp0 * 32; base < total; base += wstride * 32) {
-    int64_t b = base + lane;
-    unsigned int m = 0u;
-    int gid = 0;
-    if (b < total) {
-      int64_t row = b / nkb, kb = b - row * nkb;
-      uint32_t w[8];
-      load_bf16x16(x + row * ld + kb * 16, w);
+  const int nkb = static_cast<int>(K / 16);
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  // each warp takes rows r and r + warps together: 4 loads of 32 bytes per lane in flight
+  for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
+       row += 2 * warps) {
+    const int64_t row2 = row + warps;
+    const bool two = row2 < rows;
+    uint32_t m = 0u, m2 = 0u;
+    for (int kb0 = 0; kb0 < nkb; kb0 += 2 * 32) {
+      uint32_t w[4][8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        m = max(m, w[i] & 0x7FFFu);
-        m = max(m, (w[i] >> 16) & 0x7FFFu);
+      for (int u = 0; u < 4; ++u) {
+        const int kb = kb0 + (u & 1) * 32 + lane;
+        const int64_t r = (u < 2) ? row : row2;
+        if (kb < nkb && (u < 2 || two)) load_bf16x16(x + r * ld + kb * 16, w[u]);
       }
-      gid = grp.of(row);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int kb = kb0 + (u & 1) * 32 + lane;
+        if (kb < nkb && (u < 2 || two)) {
+          uint32_t& acc = (u < 2) ? m : m2;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc = __vmaxu2(acc, w[u][i] & 0x7FFF7FFFu);
+        }
+      }
     }
-    int gid0 = __shfl_sync(0xffffffffu, gid, 0);
-    bool same = __all_sync(0xffffffffu, (b >= total) || gid == gid0);
-    if (same) {
-      unsigned int wm = __reduce_max_sync(0xffffffffu, m);
-      if (lane == 0 && wm) atomicMax(&amax_s[gid0], wm);
-    } else if (b < total && m) {
-      atomicMax(&amax_s[gid], m);
+    const unsigned int wm = __reduce_max_sync(0xffffffffu, max(m & 0xFFFFu, m >> 16));
+    const unsigned int wm2 = __reduce_max_sync(0xffffffffu, max(m2 & 0xFFFFu, m2 >> 16));
+    if (lane == 0) {
+      if (wm) atomicMax(&amax_s[grp.of(row)], wm);
+      if (two && wm2) atomicMax(&amax_s[grp.of(row2)], wm2);
     }
   }
   __syncthreads();
@@ -100,119 +107,136 @@ struct QuantArgs {
   int resid_mode;          // 0: residual, 1: bf16(deq), 2: the input itself
   uint16_t* w_fq;          // [rows][K] or null
   int fold;                // w_fq = bf16(deq) (1) or e2m1 * e4m3 (0)
+  FastDiv uniform_div;     // filled by launch_quantize: rows per group (uniform groups)
 };
 
-__global__ void __launch_bounds__(kThreads) quantize_kernel(QuantArgs a) {
+// One warp per row, lanes along K (32 blocks of 16 elements per pass, two
+// passes in flight).  The residual channels of a pass are extracted
+// cooperatively: lane j takes channel slot j and fetches its element, code and
+// scale from the lane that owns the block by warp shuffles, then the warp
+// writes the row's residual slots as one contiguous store.
+__global__ void __launch_bounds__(kThreads, 3) quantize_kernel(QuantArgs a) {
   extern __shared__ int32_t smem[];
-  const int64_t nkb = a.K / 16;
   const int n = a.n_groups;
+  const int nkb = static_cast<int>(a.K / 16);
+  const int npass = (nkb + 31) / 32;
   int32_t* off_s = smem;                                   // n + 1
   float* g_s = reinterpret_cast<float*>(smem + n + 1);     // n
-  int32_t* mask_s = smem + 2 * n + 1;                      // nkb (only with channels)
-  int32_t* first_s = mask_s + (a.n_chan ? nkb : 0);        // nkb
-  int32_t* pad_s = first_s + (a.n_chan ? nkb : 0);         // n_chan + 1 (count first)
+  int32_t* pass_slot = smem + 2 * n + 1;                   // npass + 1 (with channels)
+  int32_t* chan_s = pass_slot + npass + 1;                 // n_chan
+  __shared__ int n_valid_s;
   for (int i = threadIdx.x; i <= n; i += blockDim.x) {
     if (a.group_off != nullptr) off_s[i] = a.group_off[i];
     if (i < n) {
-      float g = __fdiv_rn(a.amax[i], kNvfp4Range);
+      const float g = __fdiv_rn(a.amax[i], kNvfp4Range);
       g_s[i] = g;
       if (blockIdx.x == 0 && a.g_out != nullptr) a.g_out[i] = g;
     }
   }
   if (a.n_chan) {
-    for (int64_t i = threadIdx.x; i < nkb; i += blockDim.x) { mask_s[i] = 0; first_s[i] = 0x7FFFFFFF; }
-    if (threadIdx.x == 0) pad_s[0] = 0;
+    for (int j = threadIdx.x; j < a.n_chan; j += blockDim.x) chan_s[j] = a.chan[j];
+    __syncthreads();
+    // valid channels are ascending and first: slots of pass p are
+    // [#valid < 512 p, #valid < 512 (p + 1))
+    for (int p = threadIdx.x; p <= npass; p += blockDim.x) {
+      int cnt = 0;
+      for (int j = 0; j < a.n_chan; ++j) {
+        const int c = chan_s[j];
+        cnt += (c >= 0 && c < a.K && c < 512 * p) ? 1 : 0;
+      }
+      pass_slot[p] = cnt;
+    }
+    if (threadIdx.x == 0) {
+      int cnt = 0;
+      for (int j = 0; j < a.n_chan; ++j) cnt += (chan_s[j] >= 0 && chan_s[j] < a.K) ? 1 : 0;
+      n_valid_s = cnt;
+    }
   }
   __syncthreads();
-  if (a.n_chan) {
-    for (int j = threadIdx.x; j < a.n_chan; j += blockDim.x) {
-      int c = a.chan[j];
-      if (c >= 0 && c < a.K) {
-        atomicOr(&mask_s[c >> 4], 1 << (c & 15));
-        atomicMin(&first_s[c >> 4], j);
-      } else {
-        int p = atomicAdd(&pad_s[0], 1);
-        pad_s[1 + p] = j;
-      }
-    }
-    __syncthreads();
-  }
-  RowGroups grp{a.group_off ? off_s : nullptr, n, a.uniform_rows};
+  RowGroups grp{a.group_off ? off_s : nullptr, n, a.uniform_div};
   const bool tiled = a.scale_layout == QUADS_SCALES_TILED;
-  const int64_t nkb_e = tiled ? ceil_div(nkb, 4) * 4 : nkb;
-  const int64_t rows_e = tiled ? ceil_div(a.rows, 128) * 128 : a.rows;
+  const int64_t rows_valid = a.group_off ? min(a.rows, static_cast<int64_t>(off_s[n])) : a.rows;
+  const int64_t rows_e = tiled ? ceil_div(rows_valid, 128) * 128 : rows_valid;
+  const int nkb_e = tiled ? (nkb + 3) / 4 * 4 : nkb;
   const int64_t ncol_tiles = nkb_e / 4;
-  const int64_t total = rows_e * nkb_e;
-  const int npad = a.n_chan ? pad_s[0] : 0;
-  for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < total;
-       b += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t row = b / nkb_e, kb = b - row * nkb_e;
-    const bool real = row < a.rows && kb < nkb;
-    uint32_t scale = 0;
-    if (real) {
-      QBlock q;
-      uint32_t w[8];
-      load_bf16x16(a.x + row * a.ld + kb * 16, w);
+  const int n_valid = a.n_chan ? n_valid_s : 0;
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows_e;
+       row += warps) {
+    if (row >= rows_valid) {                           // padding rows of the last tiled band
+      if (a.scales)
+        for (int kb = lane; kb < nkb_e; kb += 32) a.scales[tiled_scale_offset(row, kb, ncol_tiles)] = 0;
+      continue;
+    }
+    const float g = g_s[grp.of(row)];
+    const uint16_t* xr = a.x + row * a.ld;
+    for (int p0 = 0; p0 < npass; p0 += 2) {
+      uint32_t w[2][8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        q.x[2 * i] = bf16_bits_to_float(w[i] & 0xFFFFu);
-        q.x[2 * i + 1] = bf16_bits_to_float(w[i] >> 16);
+      for (int u = 0; u < 2; ++u) {
+        const int kb = (p0 + u) * 32 + lane;
+        if (kb < nkb) load_bf16x16(xr + kb * 16, w[u]);
       }
-      const float g = g_s[grp.of(row)];
-      quantize_block(q, g);
-      scale = q.scale;
-      if (a.codes) {
-        uint2 c;
-        // byte j holds elements 2j (low nibble) and 2j+1: nibble order == element order
-        c.x = q.codes_lo;
-        c.y = q.codes_hi;
-        *reinterpret_cast<uint2*>(a.codes + row * (a.K / 2) + kb * 8) = c;
-      }
-      if (a.w_fq) {
-        uint32_t o[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          float v0 = __fmul_rn(e2m1_value(qblock_code(q, 2 * i)), q.sv);
-          float v1 = __fmul_rn(e2m1_value(qblock_code(q, 2 * i + 1)), q.sv);
-          if (a.fold) { v0 = __fmul_rn(v0, g); v1 = __fmul_rn(v1, g); }
-          o[i] = pack_bf16x2(v0, v1);
-        }
-        uint4* dst = reinterpret_cast<uint4*>(a.w_fq + row * a.K + kb * 16);
-        dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-        dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
-      }
-      if (a.resid) {
-        uint32_t m = static_cast<uint32_t>(mask_s[kb]);
-        if (m) {
-          int j = first_s[kb];
-          while (m) {
-            int bit = __ffs(m) - 1;
-            m &= m - 1;
-            float v;
-            if (a.resid_mode == 2) {
-              v = q.x[bit];
-            } else {
-              float dq = deq_f32(qblock_code(q, bit), q.sv, g);
-              v = (a.resid_mode == 1) ? dq : __fsub_rn(q.x[bit], dq);
-            }
-            a.resid[row * a.n_chan + j] = static_cast<uint16_t>(float_to_bf16_bits(v));
-            ++j;
+      for (int u = 0; u < 2; ++u) {
+        const int p = p0 + u;
+        if (p >= npass) break;                         // warp-uniform
+        const int kb = p * 32 + lane;
+        QCore q{0u, 0u, 0u, 0.0f};
+        if (kb < nkb) {
+          q = quant_core(w[u], g);
+          if (a.codes)
+            *reinterpret_cast<uint2*>(a.codes + row * (a.K / 2) + kb * 8) = make_uint2(q.lo, q.hi);
+          if (a.w_fq) {
+            uint32_t o[8];
+            deq_block_bf16(q, g, a.fold, o);
+            uint4* dst = reinterpret_cast<uint4*>(a.w_fq + row * a.K + kb * 16);
+            dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+            dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
           }
         }
-        if (kb == 0)
-          for (int p = 0; p < npad; ++p) a.resid[row * a.n_chan + pad_s[1 + p]] = 0;
+        if (a.scales && kb < nkb_e)
+          a.scales[tiled ? tiled_scale_offset(row, kb, ncol_tiles) : row * nkb + kb] =
+              static_cast<uint8_t>(q.scale);
+        if (a.resid) {
+          const int slo = pass_slot[p], shi = pass_slot[p + 1];
+          for (int j0 = slo; j0 < shi; j0 += 32) {       // warp-uniform
+            const int j = j0 + lane;
+            const bool act = j < shi;
+            const int c = act ? chan_s[j] : 512 * p;
+            const int src = (c - 512 * p) >> 4, bit = c & 15;
+            uint32_t word = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const uint32_t v = __shfl_sync(0xffffffffu, w[u][i], src);
+              word = ((bit >> 1) == i) ? v : word;
+            }
+            const uint32_t cl = __shfl_sync(0xffffffffu, q.lo, src);
+            const uint32_t ch = __shfl_sync(0xffffffffu, q.hi, src);
+            const float sv = __shfl_sync(0xffffffffu, q.sv, src);
+            const float xv = bf16_bits_to_float((bit & 1) ? (word >> 16) : (word & 0xFFFFu));
+            const uint32_t code = (((bit < 8) ? cl : ch) >> (4 * (bit & 7))) & 15u;
+            float v;
+            if (a.resid_mode == 2) {
+              v = xv;
+            } else {
+              const float dq = deq_f32(code, sv, g);
+              v = (a.resid_mode == 1) ? dq : __fsub_rn(xv, dq);
+            }
+            if (act) a.resid[row * a.n_chan + j] = static_cast<uint16_t>(float_to_bf16_bits(v));
+          }
+        }
       }
     }
-    if (a.scales && (real || tiled)) {
-      int64_t off = tiled ? tiled_scale_offset(row, kb, ncol_tiles) : row * nkb + kb;
-      a.scales[off] = static_cast<uint8_t>(scale);
-    }
+    if (a.resid)
+      for (int j = n_valid + lane; j < a.n_chan; j += 32) a.resid[row * a.n_chan + j] = 0;
   }
 }
 
 size_t quantize_smem(int n_groups, int64_t K, int n_chan) {
   size_t s = (2 * static_cast<size_t>(n_groups) + 1) * 4;
-  if (n_chan) s += (2 * static_cast<size_t>(K / 16) + n_chan + 1) * 4;
+  if (n_chan) s += (static_cast<size_t>((K / 16 + 31) / 32) + 1 + n_chan) * 4;
   return s;
 }
 
@@ -221,21 +245,21 @@ size_t quantize_smem(int n_groups, int64_t K, int n_chan) {
 __global__ void __launch_bounds__(kThreads) dequant_kernel(const uint8_t* __restrict__ codes,
                                                            const uint8_t* __restrict__ scales, int layout,
                                                            const float* __restrict__ g, const int32_t* group_off,
-                                                           int n_groups, int64_t uniform_rows, int64_t rows,
-                                                           int64_t K, void* out, int out_dtype) {
+                                                           int n_groups, FastDiv uniform, uint32_t total,
+                                                           uint32_t nkb, FastDiv nkb_div, int64_t K, void* out,
+                                                           int out_dtype) {
   extern __shared__ int32_t smem[];
   for (int i = threadIdx.x; i <= n_groups; i += blockDim.x)
     if (group_off) smem[i] = group_off[i];
   __syncthreads();
-  RowGroups grp{group_off ? smem : nullptr, n_groups, uniform_rows};
-  const int64_t nkb = K / 16, ncol_tiles = ceil_div(nkb, 4);
-  const int64_t total = rows * nkb;
-  for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < total;
-       b += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t row = b / nkb, kb = b - row * nkb;
-    const uint2 c = __ldg(reinterpret_cast<const uint2*>(codes + row * (K / 2) + kb * 8));
+  RowGroups grp{group_off ? smem : nullptr, n_groups, uniform};
+  const uint32_t ncol_tiles = (nkb + 3) / 4;
+  const uint32_t stride = gridDim.x * blockDim.x;
+  for (uint32_t b = blockIdx.x * blockDim.x + threadIdx.x; b < total; b += stride) {
+    const uint32_t row = fast_div(b, nkb_div), kb = b - row * nkb;
+    const uint2 c = __ldg(reinterpret_cast<const uint2*>(codes + static_cast<int64_t>(row) * (K / 2) + kb * 8));
     const uint32_t s = scales[layout == QUADS_SCALES_TILED ? tiled_scale_offset(row, kb, ncol_tiles)
-                                                           : row * nkb + kb];
+                                                           : static_cast<int64_t>(b)];
     const float sv = e4m3_value(s);
     const float gg = g[grp.of(row)];
     float v[16];
@@ -245,11 +269,11 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const uint8_t* __rest
       v[8 + i] = deq_f32((c.y >> (4 * i)) & 15u, sv, gg);
     }
     if (out_dtype == QUADS_OUT_F32) {
-      float4* d = reinterpret_cast<float4*>(static_cast<float*>(out) + row * K + kb * 16);
+      float4* d = reinterpret_cast<float4*>(static_cast<float*>(out) + static_cast<int64_t>(row) * K + kb * 16);
 #pragma unroll
       for (int i = 0; i < 4; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
     } else {
-      uint4* d = reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + row * K + kb * 16);
+      uint4* d = reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + static_cast<int64_t>(row) * K + kb * 16);
       d[0] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
                         pack_bf16x2(v[6], v[7]));
       d[1] = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
@@ -408,27 +432,30 @@ int launch_amax(const uint16_t* x, int64_t rows, int64_t K, int64_t ld, const in
   if (cudaMemsetAsync(amax_out, 0, sizeof(float) * n_groups, s) != cudaSuccess)
     return set_error(QUADS_ERR_CUDA, "memset of the amax output failed");
   if (rows == 0) return QUADS_OK;
-  int64_t uniform = group_off ? 0 : rows / n_groups;
+  QUADS_REQUIRE(rows < kMaxBlocks, QUADS_ERR_UNSUPPORTED_SHAPE, "too many rows");
+  const uint32_t uniform = group_off ? 1u : static_cast<uint32_t>(rows / n_groups);
   size_t smem = (2 * static_cast<size_t>(n_groups) + 1) * 4;
-  amax_kernel<<<grid_for(rows * (K / 16)), kThreads, smem, s>>>(x, rows, K, ld, group_off, n_groups,
-                                                                uniform ? uniform : 1,
-                                                                reinterpret_cast<unsigned int*>(amax_out));
+  const int grid = persistent_grid(reinterpret_cast<const void*>(amax_kernel), kThreads, smem, ceil_div(rows, 16));
+  amax_kernel<<<grid, kThreads, smem, s>>>(x, rows, K, ld, group_off, n_groups,
+                                                          make_fastdiv(uniform ? uniform : 1u),
+                                                          reinterpret_cast<unsigned int*>(amax_out));
   count_launches(1);
   return check_launch("amax_kernel");
 }
 
 int launch_quantize(QuantArgs a, cudaStream_t s) {
-  int64_t nkb = a.K / 16;
-  bool tiled = a.scale_layout == QUADS_SCALES_TILED;
-  int64_t total = (tiled ? ceil_div(a.rows, 128) * 128 : a.rows) * (tiled ? ceil_div(nkb, 4) * 4 : nkb);
-  if (total == 0) return QUADS_OK;
-  size_t smem = quantize_smem(a.n_groups, a.K, a.n_chan);
+  if (a.rows == 0) return QUADS_OK;
+  QUADS_REQUIRE(a.rows < kMaxBlocks, QUADS_ERR_UNSUPPORTED_SHAPE, "too many rows");
+  a.uniform_div = make_fastdiv(a.group_off ? 1u : static_cast<uint32_t>(a.uniform_rows > 0 ? a.uniform_rows : 1));
+  const size_t smem = quantize_smem(a.n_groups, a.K, a.n_chan);
   if (smem > 48 * 1024) {
     if (cudaFuncSetAttribute(quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return set_error(QUADS_ERR_CUDA, "cannot raise shared memory of quantize_kernel");
   }
-  quantize_kernel<<<grid_for(total), kThreads, smem, s>>>(a);
+  const int64_t rows_e = a.scale_layout == QUADS_SCALES_TILED ? ceil_div(a.rows, 128) * 128 : a.rows;
+  const int grid = persistent_grid(reinterpret_cast<const void*>(quantize_kernel), kThreads, smem, ceil_div(rows_e, 8));
+  quantize_kernel<<<grid, kThreads, smem, s>>>(a);
   count_launches(1);
   return check_launch("quantize_kernel");
 }
@@ -505,9 +532,14 @@ int quads_dequant(const uint8_t* codes, const uint8_t* scales, int scale_layout,
   QUADS_REQUIRE(codes && scales && g && out, QUADS_ERR_INVALID_ARG, "null pointer");
   QUADS_REQUIRE(aligned(codes, 8) && aligned(out, 16), QUADS_ERR_INVALID_ARG,
                 "codes must be 8-byte and out 16-byte aligned");
+  const int64_t total = rows * (K / 16);
+  QUADS_REQUIRE(total < kMaxBlocks, QUADS_ERR_UNSUPPORTED_SHAPE, "tensor above 2^31 blocks of 16");
   size_t smem = group_off ? (static_cast<size_t>(n_groups) + 1) * 4 : 0;
-  dequant_kernel<<<grid_for(rows * (K / 16)), kThreads, smem, stream>>>(
-      codes, scales, scale_layout, g, group_off, n_groups, group_off ? 1 : rows / n_groups, rows, K, out, out_dtype);
+  const uint32_t uniform = group_off ? 1u : static_cast<uint32_t>(rows / n_groups);
+  dequant_kernel<<<grid_for(total), kThreads, smem, stream>>>(
+      codes, scales, scale_layout, g, group_off, n_groups, make_fastdiv(uniform ? uniform : 1u),
+      static_cast<uint32_t>(total), static_cast<uint32_t>(K / 16), make_fastdiv(static_cast<uint32_t>(K / 16)), K,
+      out, out_dtype);
   count_launches(1);
   return check_launch("dequant_kernel");
 }

@@ -68,6 +68,7 @@ struct ReplayArgs {
   uint16_t* x_hat;
   unsigned long long* counts;
   int32_t* status;
+  FastDiv nkb_div;         // K / 16 (checked against the record on the device)
 };
 
 __device__ bool record_ok(const ReplayArgs& a, const trace_qrecord_header& h) {
@@ -77,6 +78,7 @@ __device__ bool record_ok(const ReplayArgs& a, const trace_qrecord_header& h) {
   const trace_qtensor_desc& d = h.t[a.which];
   if (!d.present || d.rows != a.rows || d.K != a.K) return false;
   if (d.K <= 0 || d.K % 16 != 0 || d.K > 65536 || d.rows < 0) return false;
+  if (d.rows * (d.K / 16) >= (int64_t(1) << 31)) return false;
   if (d.n_groups < 1 || d.n_groups > 1024 || d.n_chan < 0 || d.n_chan > 256) return false;
   if (d.scale_layout != QUADS_SCALES_LINEAR && d.scale_layout != QUADS_SCALES_TILED) return false;
   const uint64_t cb = static_cast<uint64_t>(d.rows) * (d.K / 2);
@@ -91,7 +93,7 @@ __device__ bool record_ok(const ReplayArgs& a, const trace_qrecord_header& h) {
   return true;
 }
 
-__global__ void __launch_bounds__(kThreads) replay_kernel(ReplayArgs a) {
+__global__ void __launch_bounds__(kThreads, 3) replay_kernel(ReplayArgs a) {
   extern __shared__ int32_t smem[];
   __shared__ trace_qrecord_header h;
   __shared__ int ok;
@@ -104,11 +106,13 @@ __global__ void __launch_bounds__(kThreads) replay_kernel(ReplayArgs a) {
   if (!ok) return;
   const trace_qtensor_desc d = h.t[a.which];
   const int n = d.n_groups;
-  const int64_t K = d.K, nkb = K / 16;
+  const int64_t K = d.K;
+  const int nkb = static_cast<int>(K / 16);
+  const int npass = (nkb + 31) / 32;
   int32_t* off_s = smem;                                   // n + 1
   float* g_s = reinterpret_cast<float*>(smem + n + 1);     // n
-  int32_t* mask_s = smem + 2 * n + 1;                      // nkb
-  int32_t* first_s = mask_s + nkb;                         // nkb
+  int32_t* pass_slot = smem + 2 * n + 1;                   // npass + 1
+  int32_t* chan_s = pass_slot + npass + 1;                 // n_chan
   const float* g_rec = reinterpret_cast<const float*>(a.record + d.g_off);
   const int32_t* goff_rec = reinterpret_cast<const int32_t*>(a.record + d.group_off_off);
   const int32_t* chan_rec = reinterpret_cast<const int32_t*>(a.record + d.chan_off);
@@ -118,68 +122,91 @@ __global__ void __launch_bounds__(kThreads) replay_kernel(ReplayArgs a) {
     if (i < n) g_s[i] = g_rec[i];
   }
   if (d.n_chan) {
-    for (int64_t i = threadIdx.x; i < nkb; i += blockDim.x) { mask_s[i] = 0; first_s[i] = 0x7FFFFFFF; }
+    for (int j = threadIdx.x; j < d.n_chan; j += blockDim.x) chan_s[j] = chan_rec[j];
     __syncthreads();
-    for (int j = threadIdx.x; j < d.n_chan; j += blockDim.x) {
-      int c = chan_rec[j];
-      if (c >= 0 && c < K) {
-        atomicOr(&mask_s[c >> 4], 1 << (c & 15));
-        atomicMin(&first_s[c >> 4], j);
+    for (int p = threadIdx.x; p <= npass; p += blockDim.x) {
+      int cnt = 0;
+      for (int j = 0; j < d.n_chan; ++j) {
+        const int c = chan_s[j];
+        cnt += (c >= 0 && c < K && c < 512 * p) ? 1 : 0;
       }
+      pass_slot[p] = cnt;
     }
   }
   __syncthreads();
-  RowGroups grp{n > 1 ? off_s : nullptr, n, 1};
+  RowGroups grp{n > 1 ? off_s : nullptr, n, FastDiv{1u, 1u, 0u}};
   const uint8_t* codes = a.record + d.codes_off;
   const uint8_t* scales = a.record + d.scales_off;
   const bool tiled = d.scale_layout == QUADS_SCALES_TILED;
   const int64_t ncol_tiles = ceil_div(nkb, 4);
-  const int64_t total = d.rows * nkb;
+  // rows past the last group's end hold no data (expert-ordered padding capacity)
+  const int64_t rows = (n > 1) ? min(d.rows, static_cast<int64_t>(off_s[n])) : d.rows;
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   unsigned long long code_mis = 0, scale_mis = 0;
-  for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < total;
-       b += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t row = b / nkb, kb = b - row * nkb;
-    const uint2 c = *reinterpret_cast<const uint2*>(codes + row * (K / 2) + kb * 8);
-    const uint32_t s = scales[tiled ? tiled_scale_offset(row, kb, ncol_tiles) : row * nkb + kb];
-    const float sv = e4m3_value(s);
+  for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
+       row += warps) {
     const float g = g_s[grp.of(row)];
-    float v[16];
+    for (int p0 = 0; p0 < npass; p0 += 2) {
+      uint2 cw[2];
+      uint32_t sc[2], xw[2][8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      v[i] = deq_f32((c.x >> (4 * i)) & 15u, sv, g);
-      v[8 + i] = deq_f32((c.y >> (4 * i)) & 15u, sv, g);
-    }
-    if (d.n_chan) {
-      uint32_t m = static_cast<uint32_t>(mask_s[kb]);
-      int j = m ? first_s[kb] : 0;
-      while (m) {
-        int bit = __ffs(m) - 1;
-        m &= m - 1;
-        v[bit] = __fadd_rn(v[bit], bf16_bits_to_float(resid_rec[row * d.n_chan + j]));
-        ++j;
+      for (int u = 0; u < 2; ++u) {
+        const int kb = (p0 + u) * 32 + lane;
+        if (kb < nkb) {
+          cw[u] = *reinterpret_cast<const uint2*>(codes + row * (K / 2) + kb * 8);
+          sc[u] = scales[tiled ? tiled_scale_offset(row, kb, ncol_tiles) : row * nkb + kb];
+          if (a.x_train) load_bf16x16(a.x_train + row * K + kb * 16, xw[u]);
+        }
       }
-    }
-    uint4* dst = reinterpret_cast<uint4*>(a.x_hat + row * K + kb * 16);
-    dst[0] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                        pack_bf16x2(v[6], v[7]));
-    dst[1] = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
-                        pack_bf16x2(v[14], v[15]));
-    if (a.x_train) {
-      QBlock q;
-      uint32_t w[8];
-      load_bf16x16(a.x_train + row * K + kb * 16, w);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        q.x[2 * i] = bf16_bits_to_float(w[i] & 0xFFFFu);
-        q.x[2 * i + 1] = bf16_bits_to_float(w[i] >> 16);
+      for (int u = 0; u < 2; ++u) {
+        const int p = p0 + u;
+        if (p >= npass) break;                         // warp-uniform
+        const int kb = p * 32 + lane;
+        QCore q{0u, 0u, 0u, 0.0f};
+        if (kb < nkb) {
+          q.lo = cw[u].x;
+          q.hi = cw[u].y;
+          q.scale = sc[u];
+          q.sv = e4m3_value(sc[u]);
+          uint32_t o[8];
+          deq_block_bf16(q, g, 1, o);
+          uint4* dst = reinterpret_cast<uint4*>(a.x_hat + row * K + kb * 16);
+          dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+          dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+          if (a.x_train) {
+            const QCore t = quant_core(xw[u], g);
+            // nibbles that differ: OR-fold each nibble onto its low bit, count
+            uint32_t d0 = t.lo ^ q.lo, d1 = t.hi ^ q.hi;
+            d0 = (d0 | (d0 >> 1) | (d0 >> 2) | (d0 >> 3)) & 0x11111111u;
+            d1 = (d1 | (d1 >> 1) | (d1 >> 2) | (d1 >> 3)) & 0x11111111u;
+            code_mis += __popc(d0) + __popc(d1);
+            scale_mis += (t.scale != q.scale) ? 1u : 0u;
+          }
+        }
+        if (d.n_chan) {
+          // compensation channels of this pass: x_hat = bf16(fp32(deq) + r),
+          // rewritten after the block stores above
+          __syncwarp();
+          const int slo = pass_slot[p], shi = pass_slot[p + 1];
+          for (int j0 = slo; j0 < shi; j0 += 32) {       // warp-uniform
+            const int j = j0 + lane;
+            const bool act = j < shi;
+            const int c = act ? chan_s[j] : 512 * p;
+            const int src = (c - 512 * p) >> 4, bit = c & 15;
+            const uint32_t cl = __shfl_sync(0xffffffffu, q.lo, src);
+            const uint32_t ch = __shfl_sync(0xffffffffu, q.hi, src);
+            const float sv = __shfl_sync(0xffffffffu, q.sv, src);
+            if (act) {
+              const uint32_t code = (((bit < 8) ? cl : ch) >> (4 * (bit & 7))) & 15u;
+              const float v = __fadd_rn(deq_f32(code, sv, g), bf16_bits_to_float(resid_rec[row * d.n_chan + j]));
+              a.x_hat[row * K + c] = static_cast<uint16_t>(float_to_bf16_bits(v));
+            }
+          }
+          __syncwarp();
+        }
       }
-      quantize_block(q, g);
-      // nibbles that differ: OR-fold each nibble onto its low bit, count
-      uint32_t d0 = q.codes_lo ^ c.x, d1 = q.codes_hi ^ c.y;
-      d0 = (d0 | (d0 >> 1) | (d0 >> 2) | (d0 >> 3)) & 0x11111111u;
-      d1 = (d1 | (d1 >> 1) | (d1 >> 2) | (d1 >> 3)) & 0x11111111u;
-      code_mis += __popc(d0) + __popc(d1);
-      scale_mis += (q.scale != s) ? 1u : 0u;
     }
   }
   if (a.x_train) {
@@ -297,17 +324,17 @@ int trace_replay_qrecord(const void* record, size_t record_bytes, int layer_id, 
   QUADS_REQUIRE(aligned(x_hat, 16) && (!x_train || aligned(x_train, 16)), QUADS_ERR_INVALID_ARG,
                 "x_hat and x_train must be 16-byte aligned");
   QUADS_REQUIRE(!x_train || counts, QUADS_ERR_INVALID_ARG, "counts required with x_train");
+  QUADS_REQUIRE(rows * (K / 16) < (int64_t(1) << 31), QUADS_ERR_UNSUPPORTED_SHAPE, "tensor above 2^31 blocks");
   ReplayArgs a{static_cast<const uint8_t*>(record), record_bytes, layer_id, which, rows, K, x_train, x_hat, counts,
-               status};
-  // worst-case shared memory: group offsets and scales for 1024 groups, channel tables for K/16 blocks
-  size_t smem = (2 * 1024 + 1) * 4 + 2 * static_cast<size_t>(K / 16) * 4;
+               status, make_fastdiv(static_cast<uint32_t>(K / 16))};
+  // worst case: group offsets and scales of 1024 groups, the pass table and 256 channels
+  size_t smem = (2 * 1024 + 1) * 4 + (static_cast<size_t>((K / 16 + 31) / 32) + 1 + 256) * 4;
   if (smem > 48 * 1024 &&
       cudaFuncSetAttribute(replay_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
           cudaSuccess)
     return set_error(QUADS_ERR_CUDA, "cannot raise shared memory of replay_kernel");
-  int64_t work = rows * (K / 16);
-  int64_t g = ceil_div(work, kThreads), cap = static_cast<int64_t>(num_sms()) * 8;
-  replay_kernel<<<static_cast<unsigned>(g < 1 ? 1 : (g > cap ? cap : g)), kThreads, smem, stream>>>(a);
+  const int grid = persistent_grid(reinterpret_cast<const void*>(replay_kernel), kThreads, smem, ceil_div(rows, 8));
+  replay_kernel<<<grid, kThreads, smem, stream>>>(a);
   count_launches(1);
   return check_launch("replay_kernel");
 }

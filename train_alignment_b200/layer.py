@@ -24,15 +24,18 @@ from .workloads import MoEConfig
 
 @dataclass
 class StageTimer:
-    """Optional CUDA-event marks between stages (on the current stream)."""
+    """Optional CUDA-event marks between stages (on the current stream).
+    external=True records them as external event nodes, which is how timing
+    events are captured into a CUDA graph and re-recorded at every replay."""
     enabled: bool = False
+    external: bool = False
 
     def __post_init__(self):
         self.marks = []
 
     def mark(self, name):
         if self.enabled:
-            ev = torch.cuda.Event(enable_timing=True)
+            ev = torch.cuda.Event(enable_timing=True, external=self.external)
             ev.record()
             self.marks.append((name, ev))
 
