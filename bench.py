@@ -69,6 +69,52 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+# Which source files build each kernel of the step; a DRAM-traffic figure
+# recorded from an ncu capture is reported only while the hash of these
+# files still equals the one recorded with it.
+KERNEL_SOURCES = {
+    "quantize.cu": ("amax_w", "fakequant_w_gate_up", "fakequant_w_down", "amax_x", "quantize_x", "quantize_h",
+                    "ste_backward"),
+    "grouped_gemm.cu": ("gemm_gate_up", "gemm_gate_up_swiglu", "gemm_down"),
+    "moe_route.cu": ("router_topk", "permute", "gather", "swiglu", "combine"),
+    "trace_record.cu": ("export", "replay_x", "replay_h"),
+}
+
+
+def source_hash(kernel):
+    import hashlib
+    csrc = os.path.join(ROOT, "train_alignment_b200", "csrc")
+    for src, names in KERNEL_SOURCES.items():
+        if kernel in names:
+            h = hashlib.sha256()
+            for f in (src, "common.cuh"):
+                with open(os.path.join(csrc, f), "rb") as fh:
+                    h.update(fh.read())
+            return h.hexdigest()[:12]
+    return None
+
+
+def recorded_traffic(workload, kernel):
+    """DRAM bytes (read + write) per launch of `kernel` from the table in
+    profiles/traffic.md, or None when there is no row or the kernel's sources
+    changed since the capture."""
+    path = os.path.join(ROOT, "profiles", "traffic.md")
+    if not os.path.exists(path):
+        return None
+    want = source_hash(kernel)
+    with open(path) as f:
+        for line in f:
+            cells = [c.strip().strip("`") for c in line.strip().strip("|").split("|")]
+            if len(cells) < 6 or cells[0] != workload or cells[1] != kernel:
+                continue
+            try:
+                rd, wr = float(cells[2]), float(cells[3])
+            except ValueError:
+                continue
+            return rd + wr if cells[5] == want else None
+    return None
+
+
 # --------------------------------------------------------------- accounting
 
 
@@ -106,9 +152,8 @@ def kernel_work(cfg, rpad):
     wd = E * H * F
     q = 0.5 + 1.0 / 16                      # codes + scales per element
     w = {
-        "amax_w_gate_up": ("hbm", 2.0 * wgu),
+        "amax_w": ("hbm", 2.0 * (wgu + wd)),
         "fakequant_w_gate_up": ("hbm", wgu * (2 + 2 + q) + E * 2 * F * nc * 2),
-        "amax_w_down": ("hbm", 2.0 * wd),
         "fakequant_w_down": ("hbm", wd * (2 + 2 + q) + E * H * ncf * 2),
         "amax_x": ("hbm", 2.0 * T * H),
         "quantize_x": ("hbm", T * H * (2 + q) + T * nc * 2),
@@ -116,14 +161,15 @@ def kernel_work(cfg, rpad):
         "permute": ("hbm", R * 4 * 3),
         "gather": ("hbm", (R + T) * (H * q + nc * 2)),
         "gemm_gate_up": ("tensor", 2.0 * R * 2 * F * H + 2.0 * R * 2 * F * nc),
+        "gemm_gate_up_swiglu": ("tensor", 2.0 * R * 2 * F * H + 2.0 * R * 2 * F * nc),
         "swiglu": ("hbm", rpad * (2 * F * 2 + F * 2)),
         "quantize_h": ("hbm", rpad * F * (2 + q) + rpad * ncf * 2),
         "gemm_down": ("tensor", 2.0 * R * H * F + 2.0 * R * H * ncf),
         "combine": ("hbm", R * H * 2 + T * H * 2),
+        "export": ("hbm", 2.0 * (T * H * q + T * nc * 2 + rpad * F * q + rpad * ncf * 2)),
         "replay_x": ("hbm", T * H * (q + 2 + 2)),
         "replay_h": ("hbm", rpad * F * (q + 2)),
-        "ste_backward_gate_up": ("hbm", wgu * 6.0),
-        "ste_backward_down": ("hbm", wd * 6.0),
+        "ste_backward": ("hbm", (wgu + wd) * 6.0),
     }
     return w
 
@@ -304,8 +350,9 @@ def run_ours(args):
     layer = L.build_layer(cfg, inp, dev)
     x, logits = inp["x"], inp["logits"]
     x_train = W.engine_drift(x, 1e-2, seed=rank, device=dev)
-    g_gu = W.random_bf16(layer.w_gu.shape, 100 + rank, 1e-3, dev)
-    g_d = W.random_bf16(layer.w_d.shape, 200 + rank, 1e-3, dev)
+    g_all, g_gu, g_d = layer.grad_fq_buffers()          # both weight gradients in one allocation
+    g_gu.copy_(W.random_bf16(layer.w_gu.shape, 100 + rank, 1e-3, dev))
+    g_d.copy_(W.random_bf16(layer.w_d.shape, 200 + rank, 1e-3, dev))
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     def barrier():
@@ -419,11 +466,7 @@ def run_ours(args):
             tf = a / (dms * 1e-3) / 1e12
             kernels[name] = {"ms": dms, "TFLOP/s": tf, "frac_fp4": tf / (peaks["bf16_tflops_sustained"] *
                                                                           FP4_OVER_BF16)}
-    traffic = None
-    tpath = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tpath):
-        with open(tpath) as f:
-            traffic = json.load(f).get(f"{cfg.name}:{dom}")
+    traffic = recorded_traffic(cfg.name, dom)
 
     # end to end through the public API with host buffers
     e2e = None

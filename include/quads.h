@@ -239,6 +239,26 @@ int quads_moe_grouped_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales
                                  const uint16_t* a_resid, const uint16_t* w_resid, int n_chan,
                                  uint16_t* y, quads_stream_t stream);
 
+/* a6 + a7 in one pass: the gate/up grouped GEMM with the SwiGLU applied in
+ * the epilogue.  The operands are those of quads_moe_grouped_gemm_nvfp4 with
+ * N = 2F, except that the W rows (w_codes, w_scales, w_resid) are in the
+ * 64-row interleaved gate/up order that quads_fakequant_weight_ste_gate_up
+ * writes.  Each 128-row tile then holds gate rows 64b..64b+63 followed by the
+ * matching up rows.  Writes
+ *   h[r][f] = bf16(silu(y_gate[r][f]) * y_up[r][f]),
+ * where y_gate and y_up are the BF16 GEMM outputs exactly as
+ * quads_moe_grouped_gemm_nvfp4 would store them.  SwiGLU is computed in FP32
+ * as in quads_swiglu.  h is [rows_cap][F] BF16.  amax_out (device float[E],
+ * nullable, overwritten) receives the per-expert max |h|.  F % 64 == 0. */
+int quads_moe_grouped_gemm_nvfp4_swiglu(const uint8_t* a_codes, const uint8_t* a_scales,
+                                        const float* g_a, int g_a_per_expert,
+                                        const uint8_t* w_codes, const uint8_t* w_scales,
+                                        const float* g_w, const int32_t* expert_off, int E,
+                                        int64_t rows_cap, int64_t F, int64_t K,
+                                        const uint16_t* a_resid, const uint16_t* w_resid,
+                                        int n_chan, uint16_t* h, float* amax_out,
+                                        quads_stream_t stream);
+
 /* --------------------------------------------------------- a7: SwiGLU
  * h[r][j] = bf16(silu(Y[r][j]) * Y[r][F + j]) for rows r < expert_off[E],
  * silu(v) = v / (1 + exp(-v)), computed in FP32 from the BF16 gate/up GEMM
@@ -278,6 +298,19 @@ int quads_fakequant_weight_ste(const uint16_t* w, int64_t n_mat, int64_t rows, i
                                uint8_t* codes, uint8_t* scales, float* g_out,
                                const int32_t* chan, int n_chan, int chan_raw, uint16_t* w_chan,
                                void* ws, size_t ws_bytes, quads_stream_t stream);
+/* The same pass for gate/up weight matrices [n_mat][rows][K] whose first
+ * rows / 2 rows are the gate projection and the rest the up projection
+ * (rows % 128 == 0).  w_fq keeps the input row order.  codes, scales
+ * (tiled) and w_chan are written with each matrix's rows interleaved in blocks
+ * of 64: gate rows 64b..64b+63 go to rows 128b..128b+63, and up rows
+ * 64b..64b+63 go to rows 128b+64..128b+127.  That way every 128-row tile of
+ * the rollout's weights holds matching gate and up rows.  This is the operand
+ * layout of quads_moe_grouped_gemm_nvfp4_swiglu. */
+int quads_fakequant_weight_ste_gate_up(const uint16_t* w, int64_t n_mat, int64_t rows, int64_t K,
+                                       const float* amax_in, int fold_global, uint16_t* w_fq,
+                                       uint8_t* codes, uint8_t* scales, float* g_out,
+                                       const int32_t* chan, int n_chan, int chan_raw, uint16_t* w_chan,
+                                       void* ws, size_t ws_bytes, quads_stream_t stream);
 /* Straight-through backward: grad_w = grad_wfq (accumulate = 0) or
  * grad_w = bf16(fp32(grad_w + grad_wfq)) (accumulate = 1); n BF16 elements. */
 int quads_fakequant_weight_ste_backward(const uint16_t* grad_wfq, uint16_t* grad_w, int64_t n,
@@ -332,13 +365,17 @@ typedef struct trace_qtensor_src {
 } trace_qtensor_src;
 
 /* Fills *hdr (host memory) with the layout of a record for these tensors and
- * returns its total size in bytes (0 on invalid arguments). */
+ * returns its total size in bytes (0 on invalid arguments).  Only the sizes
+ * in `tensors` are read (the pointers may be NULL), so a producer can place
+ * its outputs at the returned offsets of the record before exporting. */
 size_t trace_qrecord_layout(int layer_id, int64_t T, int k,
                             const trace_qtensor_src* tensors, int n_tensors,
                             trace_qrecord_header* hdr);
 /* Writes the record (header + copies of every section) into `record`
  * (device, record_bytes >= trace_qrecord_layout(...), 256-byte aligned).
- * topk_idx: device int32 [T][k] or NULL when k == 0. */
+ * topk_idx: device int32 [T][k] or NULL when k == 0.  A section whose source
+ * pointer already equals its place in the record (a producer that wrote its
+ * output into the record) is not copied. */
 int trace_export_qrecord(int layer_id, int64_t T, int k, const int32_t* topk_idx,
                          const trace_qtensor_src* tensors, int n_tensors,
                          void* record, size_t record_bytes, quads_stream_t stream);

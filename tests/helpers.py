@@ -51,3 +51,11 @@ def assert_bits_equal(got, ref, what=""):
 
 def f32_of(t):
     return t.detach().to("cpu").numpy().astype(np.float64)
+
+
+def gate_up_interleave_index(F):
+    """Row order of gate/up weights interleaved in blocks of 64: destination
+    row 128 b + j holds gate row 64 b + j (j < 64) or up row F + 64 b + j - 64."""
+    dst = np.arange(2 * F)
+    b, j = dst // 128, dst % 128
+    return np.where(j < 64, 64 * b + j, F + 64 * b + (j - 64))

@@ -9,7 +9,7 @@ import torch
 from oracle import formats as F
 from oracle import moe as M
 from oracle import nvfp4 as Q
-from tests.helpers import assert_close_tol, bf16_np, bf16_torch
+from tests.helpers import assert_bits_equal, assert_close_tol, bf16_np, bf16_torch, f32_of, gate_up_interleave_index
 from train_alignment_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
@@ -128,3 +128,73 @@ def test_grouped_gemm_bench_layer_shape(cuda_lib):
     got = _run_gpu(cuda_lib, p)
     ref, absdot = _oracle(p)
     assert_close_tol(got[:p["R"]], ref, absdot, what="gate/up gemm")
+
+
+def _gpu_args(p, w_c, w_s, wc):
+    E, N, K, cap, R = p["E"], p["N"], p["K"], p["cap"], p["R"]
+    a_codes = np.zeros((cap, K // 2), np.uint8)
+    a_codes[:R] = F.pack_nibbles(p["a_c"])
+    a_scales = np.zeros((cap, K // 16), np.uint8)
+    a_scales[:R] = p["a_s"]
+    dev = "cuda"
+    args = dict(
+        a_codes=torch.from_numpy(a_codes).to(dev), a_scales=torch.from_numpy(F.scales_to_tiled(a_scales)).to(dev),
+        g_a=torch.tensor([p["g_a"]], dtype=torch.float32, device=dev),
+        w_codes=torch.from_numpy(np.ascontiguousarray(F.pack_nibbles(w_c))).to(dev),
+        w_scales=torch.from_numpy(F.scales_to_tiled(w_s.reshape(E * N, K // 16))).to(dev),
+        g_w=torch.tensor(p["g_w"], dtype=torch.float32, device=dev),
+        expert_off=torch.from_numpy(p["off"]).to(dev), E=E, rows_cap=cap, K=K)
+    if p["nc"]:
+        resid = np.zeros((cap, p["nc"]))
+        resid[:R] = p["resid"]
+        args["a_resid"] = bf16_torch(resid)
+        args["w_resid"] = bf16_torch(np.ascontiguousarray(wc))
+    return args
+
+
+@pytest.mark.parametrize("counts,F_,K,nc", [
+    ([64], 64, 64, 0),                  # one tile: 64 gate + 64 up columns
+    ([130, 0, 257], 128, 512, 32),      # empty expert, ragged experts
+    ([500, 20, 1000, 3], 192, 1024, 64),
+])
+def test_grouped_gemm_swiglu_parity(cuda_lib, counts, F_, K, nc):
+    """Gate/up GEMM with the SwiGLU in its epilogue, on weights in the 64-row
+    interleaved gate/up order: h against the oracle's SwiGLU of the oracle's
+    GEMM (tolerance propagated through SwiGLU), bit for bit against the plain
+    GEMM followed by the SwiGLU kernel, and the per-expert amax exact."""
+    p = _problem(counts, 2 * F_, K, nc, seed=3 * sum(counts) + F_ + K + nc)
+    perm = gate_up_interleave_index(F_)
+    wc_il = p["wc"][:, perm] if nc else None
+    args = _gpu_args(p, p["w_c"][:, perm], p["w_s"][:, perm], wc_il)
+    E, cap, R = p["E"], p["cap"], p["R"]
+    h = torch.full((cap, F_), float("nan"), dtype=torch.bfloat16, device="cuda")
+    h, amax = cuda_lib.moe_grouped_gemm_nvfp4_swiglu(F=F_, h=h, **args)
+    torch.cuda.synchronize()
+    assert cuda_lib.device_status() == cuda_lib.OK
+    got = bf16_np(h)
+    assert np.all(np.isnan(got[R:])), "rows past expert_off[E] must be untouched"
+    # against the oracle: y within the GEMM tolerance, carried through SwiGLU
+    y_ref, absdot = _oracle(p)
+    tol_y = 1e-2 * np.abs(y_ref) + 1e-3 * absdot
+    g, u = y_ref[:, :F_], y_ref[:, F_:]
+    sig = 1.0 / (1.0 + np.exp(-g))
+    h_ref = M.swiglu(F.bf16_rne(y_ref.astype(np.float32)))
+    dsilu = np.abs(sig * (1.0 + g * (1.0 - sig)))
+    tol_h = dsilu * (np.abs(u) + tol_y[:, F_:]) * tol_y[:, :F_] + np.abs(g * sig) * tol_y[:, F_:] + \
+        2.0 ** -7 * np.abs(h_ref) + 1e-30
+    err = np.abs(got[:R] - h_ref)
+    assert np.all(err <= tol_h), f"{np.sum(err > tol_h)} of {err.size} h values outside the tolerance"
+    # against the plain GEMM (same operands) + the SwiGLU kernel: identical bits
+    y_il = torch.full((cap, 2 * F_), float("nan"), dtype=torch.bfloat16, device="cuda")
+    cuda_lib.moe_grouped_gemm_nvfp4(N=2 * F_, y=y_il, **args)
+    inv = np.argsort(perm)
+    y_nat = y_il[:, torch.from_numpy(inv).cuda()].contiguous()
+    h2, amax2 = cuda_lib.swiglu(y_nat, F_, args["expert_off"], E)
+    torch.cuda.synchronize()
+    assert_bits_equal(F.bf16_bits(got[:R]), F.bf16_bits(bf16_np(h2)[:R]), "fused vs separate SwiGLU")
+    a = f32_of(amax)
+    for e in range(E):
+        lo, hi = p["off"][e], p["off"][e + 1]
+        want = np.max(np.abs(got[lo:hi])) if hi > lo else 0.0
+        assert a[e] == want, (e, a[e], want)
+    assert_bits_equal(a.astype(np.float32), f32_of(amax2).astype(np.float32), "amax vs SwiGLU kernel")

@@ -16,15 +16,16 @@ import torch
 from oracle import formats as F
 from oracle import layer as OL
 from oracle import nvfp4 as Q
-from tests.helpers import (assert_bits_equal, assert_close_tol, bf16_np, f32_of, u8_np, unpack_codes)
+from tests.helpers import (assert_bits_equal, assert_close_tol, bf16_np, f32_of, gate_up_interleave_index, u8_np,
+                           unpack_codes)
 from train_alignment_b200 import layer as L
 from train_alignment_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(scope="module")
-def run(cuda_lib):
+@pytest.fixture(scope="module", params=[True, False], ids=["fused_swiglu", "separate_swiglu"])
+def run(cuda_lib, request):
     cfg = W.MOE_T2048
     inp = W.moe_layer_inputs(cfg, seed=0, device="cpu")
     r = np.random.default_rng(0)
@@ -33,9 +34,10 @@ def run(cuda_lib):
     x_train = W.engine_drift(inp["x"], 1e-2, seed=0)
     dev = "cuda"
     layer = L.MoELayer(cfg, inp["w_gu"].to(dev), inp["w_d"].to(dev), torch.from_numpy(chan_x),
-                       torch.from_numpy(chan_h), dev)
-    g_gu = W.random_bf16(layer.w_gu.shape, 1, 1e-3, dev)
-    g_d = W.random_bf16(layer.w_d.shape, 2, 1e-3, dev)
+                       torch.from_numpy(chan_h), dev, fuse_swiglu=request.param)
+    _, g_gu, g_d = layer.grad_fq_buffers()
+    g_gu.copy_(W.random_bf16(layer.w_gu.shape, 1, 1e-3, dev))
+    g_d.copy_(W.random_bf16(layer.w_d.shape, 2, 1e-3, dev))
     layer.reset_counts()
     layer.step(inp["x"].to(dev), inp["logits"].to(dev), x_train.to(dev), g_gu, g_d)
     assert cuda_lib.device_status() == cuda_lib.OK
@@ -43,18 +45,21 @@ def run(cuda_lib):
     ref = OL.step(bf16_np(inp["x"]), inp["logits"].numpy().astype(np.float64), bf16_np(x_train),
                   bf16_np(inp["w_gu"]), bf16_np(inp["w_d"]), chan_x, chan_h, cfg.k,
                   grad_gu_fq=bf16_np(g_gu), grad_gu=np.zeros(tuple(layer.w_gu.shape)))
+    ref["grad_d"] = bf16_np(g_d)          # accumulated onto a zero master gradient: itself
     return cfg, layer, ref
 
 
 def test_weights(run):
     cfg, layer, ref = run
     E, F2, H = cfg.E, 2 * cfg.F, cfg.H
-    assert_bits_equal(unpack_codes(layer.w_gu_codes), ref["wgu"]["codes"], "w_gu codes")
+    # the rollout's gate/up weights are in the interleaved order when SwiGLU is fused
+    perm = gate_up_interleave_index(cfg.F) if layer.fuse_swiglu else np.arange(F2)
+    assert_bits_equal(unpack_codes(layer.w_gu_codes), ref["wgu"]["codes"][:, perm], "w_gu codes")
     s = F.scales_from_tiled(u8_np(layer.w_gu_scales), E * F2, H // 16).reshape(E, F2, H // 16)
-    assert_bits_equal(s, ref["wgu"]["scales"], "w_gu scales")
+    assert_bits_equal(s, ref["wgu"]["scales"][:, perm], "w_gu scales")
     assert_bits_equal(f32_of(layer.g_w_gu).astype(np.float32), ref["wgu"]["g"].astype(np.float32), "g_w")
     assert_bits_equal(F.bf16_bits(bf16_np(layer.w_gu_fq)), F.bf16_bits(ref["wgu"]["w_fq"]), "w_gu_fq")
-    assert_bits_equal(F.bf16_bits(bf16_np(layer.wc_gu)), F.bf16_bits(ref["wgu"]["wc"]), "wc_gu")
+    assert_bits_equal(F.bf16_bits(bf16_np(layer.wc_gu)), F.bf16_bits(ref["wgu"]["wc"][:, perm]), "wc_gu")
     assert_bits_equal(unpack_codes(layer.w_d_codes), ref["wd"]["codes"], "w_d codes")
     assert_bits_equal(F.bf16_bits(bf16_np(layer.wc_d)), F.bf16_bits(ref["wd"]["wc"]), "wc_d")
 
@@ -74,6 +79,8 @@ def test_rollout_input_and_routing(run):
 
 def test_gate_up_gemm(run):
     cfg, layer, ref = run
+    if layer.fuse_swiglu:
+        pytest.skip("y is not stored when SwiGLU runs in the GEMM epilogue (h is checked instead)")
     f = ref["fwd"]
     n = int(f["off"][-1])
     assert_close_tol(bf16_np(layer.y_gu)[:n], f["y1"], f["absdot1"], what="gate/up GEMM")
@@ -107,3 +114,4 @@ def test_replay(run):
 def test_ste(run):
     cfg, layer, ref = run
     assert_bits_equal(F.bf16_bits(bf16_np(layer.grad_gu)), F.bf16_bits(ref["grad"]), "grad_gu")
+    assert_bits_equal(F.bf16_bits(bf16_np(layer.grad_d)), F.bf16_bits(ref["grad_d"]), "grad_d")

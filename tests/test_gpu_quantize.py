@@ -8,7 +8,8 @@ import torch
 
 from oracle import formats as F
 from oracle import nvfp4 as Q
-from tests.helpers import (assert_bits_equal, bf16_np, bf16_torch, f32_of, u8_np, unpack_codes)
+from tests.helpers import (assert_bits_equal, bf16_np, bf16_torch, f32_of, gate_up_interleave_index, u8_np,
+                           unpack_codes)
 from train_alignment_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
@@ -102,6 +103,40 @@ def test_quantize_grouped(cuda_lib):
     _check_quant(cuda_lib, x, 1, group_off=off)
 
 
+def _every_block_max(tensor_amax, seed, binades=13):
+    """Rows of 16-element blocks per group: one block for every BF16 value v in
+    [A 2^-binades, A] as the block maximum (the other 15 elements below it,
+    random signs), so that every block-scale ratio amax_b / fp32(6 g) that can
+    round to a non-zero E4M3 code occurs."""
+    r = np.random.default_rng(seed)
+    blocks, off = [], [0]
+    for A in tensor_amax:
+        a_bits = int(F.bf16_bits(np.array([A], dtype=np.float32))[0])
+        lo_bits = int(F.bf16_bits(np.array([A * 2.0 ** -binades], dtype=np.float32))[0])
+        vals = F.bf16_from_bits(np.arange(lo_bits, a_bits + 1, dtype=np.uint16)).astype(np.float64)
+        n = (len(vals) + 31) // 32 * 32                 # whole rows of 32 blocks
+        vals = np.concatenate([vals, np.full(n - len(vals), A)])
+        b = vals[:, None] * r.uniform(0, 1, (n, 16))
+        b[np.arange(n), r.integers(0, 16, n)] = vals
+        b *= r.choice([-1.0, 1.0], (n, 16))
+        blocks.append(F.bf16_rne(b.astype(np.float32)).reshape(n // 32, 512))
+        off.append(off[-1] + n // 32)
+    return np.concatenate(blocks), off
+
+
+@pytest.mark.parametrize("n_groups", [8, 40])
+def test_quantize_every_block_scale(cuda_lib, n_groups):
+    """Every BF16 block maximum over 13 binades below the tensor maximum, for
+    tensor maxima from 2^-80 to 2^80 (the smallest ones below the range where
+    the quantizer's quotient shortcut applies): codes and scales bit-exact
+    against the oracle.  8 groups use the per-group scale table, 40 do not."""
+    r = np.random.default_rng(100 + n_groups)
+    A = F.bf16_rne((2.0 ** r.uniform(-80, 80, n_groups) * r.uniform(1, 2, n_groups)).astype(np.float32))
+    A[:3] = F.bf16_rne(np.array([2.0 ** -70, 448.0, 1.0], dtype=np.float32))
+    x, off = _every_block_max(A.astype(np.float64), n_groups)
+    _check_quant(cuda_lib, x, 1, group_off=off)
+
+
 def test_amax_groups(cuda_lib):
     x = _x(500, 128, 10)
     off = [0, 100, 100, 500]
@@ -154,6 +189,34 @@ def test_fakequant_parity(cuda_lib, fold):
     c1, s1, g1, _ = cuda_lib.quantize_nvfp4(wt[1].contiguous(), scale_layout=cuda_lib.SCALES_TILED)
     torch.cuda.synchronize()
     assert_bits_equal(unpack_codes(c1), c_all[1], "rollout vs trainer codes")
+
+
+@pytest.mark.parametrize("fold", [True, False])
+def test_fakequant_gate_up_interleaved(cuda_lib, fold):
+    """The gate/up variant: W_fq in the input order, the rollout's codes,
+    scales and compensation columns in the 64-row interleaved gate/up order."""
+    r = np.random.default_rng(13)
+    n_mat, F_, K = 2, 192, 128
+    rows = 2 * F_
+    w = F.bf16_rne((r.standard_normal((n_mat, rows, K)) * 0.02).astype(np.float32))
+    chan = [3, 64, 100, -1]
+    wt = bf16_torch(w)
+    ch = torch.tensor(chan, dtype=torch.int32, device="cuda")
+    w_fq, codes, scales, g, w_chan = cuda_lib.fakequant_weight_ste(wt, fold_global=fold, chan=ch, gate_up=True)
+    torch.cuda.synchronize()
+    perm = gate_up_interleave_index(F_)
+    s_all = F.scales_from_tiled(u8_np(scales), n_mat * rows, K // 16).reshape(n_mat, rows, K // 16)
+    c_all = unpack_codes(codes)
+    for m in range(n_mat):
+        wf_ref, c_ref, s_ref, g_ref = Q.fakequant_weight(w[m], fold_global=fold)
+        assert_bits_equal(F.bf16_bits(bf16_np(w_fq[m])), F.bf16_bits(wf_ref), f"w_fq[{m}]")
+        assert_bits_equal(c_all[m], c_ref[perm], f"codes[{m}]")
+        assert_bits_equal(s_all[m], s_ref[perm], f"scales[{m}]")
+        assert np.float32(f32_of(g)[m]) == np.float32(g_ref)
+        deq = F.bf16_rne(F.f32(Q.dequant(c_ref, s_ref, g_ref)))
+        for j, c in enumerate(chan):
+            want = deq[perm, c] if c >= 0 else np.zeros(rows)
+            assert_bits_equal(F.bf16_bits(bf16_np(w_chan[m][:, j])), F.bf16_bits(want), "w_chan")
 
 
 @pytest.mark.parametrize("accumulate", [False, True])

@@ -82,10 +82,14 @@ _SIGS = {
                                         c_vp, c_vp, c_i64, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
     "quads_moe_grouped_gemm_nvfp4": (c_i32, [c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_i32, c_i64, c_i64,
                                              c_i64, c_vp, c_vp, c_i32, c_vp, c_vp]),
+    "quads_moe_grouped_gemm_nvfp4_swiglu": (c_i32, [c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_i32, c_i64,
+                                                    c_i64, c_i64, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp]),
     "quads_swiglu": (c_i32, [c_vp, c_i64, c_i64, c_vp, c_i32, c_vp, c_vp, c_vp]),
     "quads_moe_unpermute_combine": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i32, c_i64, c_vp, c_vp]),
     "quads_fakequant_weight_ste": (c_i32, [c_vp, c_i64, c_i64, c_i64, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_i32,
                                            c_i32, c_vp, c_vp, c_sz, c_vp]),
+    "quads_fakequant_weight_ste_gate_up": (c_i32, [c_vp, c_i64, c_i64, c_i64, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp,
+                                                   c_vp, c_i32, c_i32, c_vp, c_vp, c_sz, c_vp]),
     "quads_fakequant_weight_ste_backward": (c_i32, [c_vp, c_vp, c_i64, c_i32, c_vp]),
     "trace_qrecord_layout": (c_sz, [c_i32, c_i64, c_i32, c_vp, c_i32, c_vp]),
     "trace_export_qrecord": (c_i32, [c_i32, c_i64, c_i32, c_vp, c_vp, c_i32, c_vp, c_sz, c_vp]),
@@ -291,6 +295,22 @@ def moe_grouped_gemm_nvfp4(a_codes, a_scales, g_a, w_codes, w_scales, g_w, exper
     return y
 
 
+def moe_grouped_gemm_nvfp4_swiglu(a_codes, a_scales, g_a, w_codes, w_scales, g_w, expert_off, E, rows_cap, F, K,
+                                  a_resid=None, w_resid=None, h=None, amax=None, want_amax=True):
+    """Gate/up GEMM with SwiGLU fused; W rows in the 64-row interleaved
+    gate/up order.  Returns (h [rows_cap, F], per-expert amax or None)."""
+    n_chan = 0 if a_resid is None else a_resid.shape[1]
+    h = h if h is not None else _empty((rows_cap, F), torch.bfloat16, a_codes.device)
+    if want_amax and amax is None:
+        amax = _empty((E,), torch.float32, a_codes.device)
+    per_expert = 1 if g_a.numel() == E and E > 1 else 0
+    _check(load().quads_moe_grouped_gemm_nvfp4_swiglu(
+        _p(a_codes), _p(a_scales), _p(g_a), per_expert, _p(w_codes), _p(w_scales), _p(g_w), _p(expert_off), E,
+        rows_cap, F, K, _p(a_resid), _p(w_resid), n_chan, _p(h), _p(amax) if want_amax else None, _s()),
+        "quads_moe_grouped_gemm_nvfp4_swiglu")
+    return h, (amax if want_amax else None)
+
+
 def swiglu(y, F, expert_off, E, h=None, amax=None, want_amax=True):
     rows_cap = y.shape[0]
     h = h if h is not None else _empty((rows_cap, F), torch.bfloat16, y.device)
@@ -312,8 +332,10 @@ def moe_unpermute_combine(y, row_of, topk_w, T, k, H, out=None):
 
 
 def fakequant_weight_ste(w, fold_global=True, chan=None, chan_raw=False, want_codes=True, w_fq=None, codes=None,
-                         scales=None, g_out=None, w_chan=None, ws=None, amax_in=None):
-    """w: [n_mat, rows, K] bf16.  Returns (w_fq, codes, scales, g, w_chan)."""
+                         scales=None, g_out=None, w_chan=None, ws=None, amax_in=None, gate_up=False):
+    """w: [n_mat, rows, K] bf16.  Returns (w_fq, codes, scales, g, w_chan).
+    gate_up=True: codes, scales and w_chan in the 64-row gate/up interleaved
+    order of quads_fakequant_weight_ste_gate_up."""
     _dev(w, torch.bfloat16, "w")
     n_mat, rows, K = w.shape
     dev = w.device
@@ -329,11 +351,11 @@ def fakequant_weight_ste(w, fold_global=True, chan=None, chan_raw=False, want_co
         w_chan = _empty((n_mat, rows, n_chan), torch.bfloat16, dev)
     if amax_in is None and ws is None:
         ws = _empty((quantize_workspace_bytes(n_mat),), torch.uint8, dev)
-    _check(load().quads_fakequant_weight_ste(
+    name = "quads_fakequant_weight_ste_gate_up" if gate_up else "quads_fakequant_weight_ste"
+    _check(getattr(load(), name)(
         _p(w), n_mat, rows, K, _p(amax_in), 1 if fold_global else 0, _p(w_fq), _p(codes) if want_codes else None,
         _p(scales) if want_codes else None, _p(g_out), _p(chan), n_chan, 1 if chan_raw else 0,
-        _p(w_chan) if n_chan else None, _p(ws), 0 if ws is None else ws.numel(), _s()),
-        "quads_fakequant_weight_ste")
+        _p(w_chan) if n_chan else None, _p(ws), 0 if ws is None else ws.numel(), _s()), name)
     return w_fq, (codes if want_codes else None), (scales if want_codes else None), g_out, \
         (w_chan if n_chan else None)
 
@@ -363,6 +385,33 @@ def qtensor_src(codes, scales, g, rows, K, scale_layout, group_off=None, chan=No
     s.resid = resid.data_ptr() if s.n_chan else None
     s._keep = (codes, scales, g, group_off, chan, resid)
     return s
+
+
+def qtensor_shape(rows, K, scale_layout, n_groups=1, n_chan=0):
+    """A record slot described by its sizes only (for trace_qrecord_layout)."""
+    s = TraceQTensorSrc()
+    s.rows, s.K, s.n_groups, s.n_chan, s.scale_layout, s.present = rows, K, n_groups, n_chan, scale_layout, 1
+    return s
+
+
+def record_views(record, hdr, which):
+    """Views of slot `which` of a record laid out by trace_qrecord_layout:
+    codes, scales (u8), g (f32), group_off and chan (i32), resid (bf16), each
+    None when the slot has no such section."""
+    d = hdr.t[which]
+
+    def sec(off, nbytes, dtype):
+        return record[off:off + nbytes].view(dtype)
+
+    ng, nc, rows = int(d.n_groups), int(d.n_chan), int(d.rows)
+    return {
+        "codes": sec(d.codes_off, d.codes_bytes, torch.uint8),
+        "scales": sec(d.scales_off, d.scales_bytes, torch.uint8),
+        "g": sec(d.g_off, 4 * ng, torch.float32),
+        "group_off": sec(d.group_off_off, 4 * (ng + 1), torch.int32) if ng > 1 else None,
+        "chan": sec(d.chan_off, 4 * nc, torch.int32) if nc else None,
+        "resid": sec(d.resid_off, 2 * nc * rows, torch.bfloat16) if nc else None,
+    }
 
 
 def _src_array(tensors):

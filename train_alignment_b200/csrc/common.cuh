@@ -275,19 +275,72 @@ struct QCore {
   float sv;
 };
 
+// Per-group constants of the block-scale computation: the per-tensor scale g,
+// d = fp32(6 g), rd = fp32(1 / d) when the division below may use it (0
+// otherwise), and optionally a table tab[s] = {S, fp32(1 / S)} with
+// S = fp32(val(s) g) for every E4M3 code s in [0, 128).
+struct QConsts {
+  float g, d, rd;
+  const float2* tab;
+};
+
+__device__ __forceinline__ QConsts make_qconsts(float g, const float2* tab = nullptr) {
+  QConsts c;
+  c.g = g;
+  c.d = __fmul_rn(6.0f, g);
+  c.rd = (c.d >= 0x1p-60f) ? __frcp_rn(c.d) : 0.0f;
+  c.tab = tab;
+  return c;
+}
+
+// Entry s of the {S, 1/S} table of a group.
+__device__ __forceinline__ float2 scale_table_entry(uint32_t s, float g) {
+  const float S = __fmul_rn(e4m3_value(s), g);
+  return make_float2(S, S != 0.0f ? __frcp_rn(S) : 0.0f);
+}
+
+// fp32(amax / d), correctly rounded.  With rd = fp32(1/d), q = fp32(amax rd)
+// is within one ulp of the quotient, the remainder amax - d q is exact in one
+// FMA, and fp32(q + rem rd) is the correctly rounded quotient (Markstein's
+// theorem; P. Markstein, IBM J. Res. Develop. 34(1), 1990).  rd is set only
+// for d >= 2^-60, where every remainder that can change an E4M3 scale stays a
+// normal number; smaller d takes the full division.
+__device__ __forceinline__ float block_ratio(float amax, const QConsts& c) {
+  if (c.rd == 0.0f) return __fdiv_rn(amax, c.d);
+  const float q = __fmul_rn(amax, c.rd);
+  const float rem = __fmaf_rn(-c.d, q, amax);
+  return __fmaf_rn(rem, c.rd, q);
+}
+
+// {val(s), val(s)} as an f16x2 pair (exact: E4M3 values are f16 values).
+__device__ __forceinline__ uint32_t e4m3_splat_f16x2(uint32_t s) {
+  uint32_t r;
+  const uint16_t in = static_cast<uint16_t>(s | (s << 8));
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(in));
+  return r;
+}
+
 // The quantizer on 16 BF16 values given as 8 packed words (element 2i in the
 // low half of w[i]); same operations and rounding as quantize_block.
-__device__ __forceinline__ QCore quant_core(const uint32_t (&w)[8], float g) {
+__device__ __forceinline__ QCore quant_core(const uint32_t (&w)[8], const QConsts& c) {
   uint32_t m = 0u;
 #pragma unroll
   for (int i = 0; i < 8; ++i) m = __vmaxu2(m, w[i] & 0x7FFF7FFFu);
   const float amax = bf16_bits_to_float(max(m & 0xFFFFu, m >> 16));
   uint32_t s = 0;
-  if (g != 0.0f) s = e4m3_from_float(__fdiv_rn(amax, __fmul_rn(6.0f, g)));
+  if (c.g != 0.0f) s = e4m3_from_float(block_ratio(amax, c));
   QCore r;
   r.scale = s;
   r.sv = e4m3_value(s);
-  const float S = __fmul_rn(r.sv, g);
+  float S, inv;
+  if (c.tab != nullptr) {
+    const float2 e = c.tab[s];
+    S = e.x;
+    inv = e.y;
+  } else {
+    S = __fmul_rn(r.sv, c.g);
+    inv = (S != 0.0f) ? __frcp_rn(S) : 0.0f;
+  }
   if (S == 0.0f) {
     uint32_t lo = 0, hi = 0;
 #pragma unroll
@@ -299,7 +352,6 @@ __device__ __forceinline__ QCore quant_core(const uint32_t (&w)[8], float g) {
     r.hi = hi;
     return r;
   }
-  const float inv = __frcp_rn(S);
   const uint64_t inv2 = pack_f32x2(inv, inv);
   uint64_t y[8];
 #pragma unroll
@@ -308,6 +360,8 @@ __device__ __forceinline__ QCore quant_core(const uint32_t (&w)[8], float g) {
   r.hi = e2m1x8_from_pairs(y + 4);
   return r;
 }
+
+__device__ __forceinline__ QCore quant_core(const uint32_t (&w)[8], float g) { return quant_core(w, make_qconsts(g)); }
 
 // BF16 of the dequantized block: fp32(e2m1 * e4m3 * g) (fold) or the exact
 // e2m1 * e4m3; the products e2m1 * e4m3 are exact in f16.
@@ -318,7 +372,7 @@ __device__ __forceinline__ void deq_block_bf16(const QCore& q, float g, int fold
   e2m1x8_to_f16x2(q.hi, h1);
 #pragma unroll
   for (int i = 0; i < 4; ++i) { h[i] = h0[i]; h[4 + i] = h1[i]; }
-  const uint32_t sv2 = f16x2_splat(q.sv);
+  const uint32_t sv2 = e4m3_splat_f16x2(q.scale);
   const uint64_t g2 = pack_f32x2(g, g);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {

@@ -20,8 +20,8 @@
 //                  FP32 accumulator, then tcgen05.mma kind::f16 (BF16) for
 //                  R_C . Wc into a second accumulator.
 //   warps 2..5     epilogue: tcgen05.ld both accumulators, y = G * acc + comp,
-//                  BF16 rows staged in shared memory, TMA tensor stores of
-//                  32 x 32 boxes.
+//                  BF16 rows staged in shared memory (64-byte swizzle),
+//                  TMA tensor stores of 32 x 32 boxes.
 // TMEM columns: [0,128) and [128,256) main accumulators, [256,384) the
 // compensation accumulator, [384,512) four slots of scale factors.
 // Tiles are (expert, 128-row block, 128-column block); experts' row segments
@@ -80,6 +80,7 @@ struct GemmParams {
   const float* g_w;
   const int32_t* expert_off;
   uint16_t* y;
+  unsigned int* amax_bits;   // SwiGLU epilogue: per-expert max |h| (float bits), or null
   int g_a_per_expert;
   int E;
   int N;
@@ -246,6 +247,16 @@ __device__ __forceinline__ int expert_of_row(const int32_t* off_s, int E, int ro
 
 // ------------------------------------------------------------------ kernel
 
+// One output before rounding: fp32(G * acc + comp) in one FMA, or
+// fp32(G * acc) without compensation.
+__device__ __forceinline__ float epi_value(uint32_t acc, float G, bool has_comp, uint32_t comp) {
+  return has_comp ? __fmaf_rn(__uint_as_float(acc), G, __uint_as_float(comp)) : __fmul_rn(__uint_as_float(acc), G);
+}
+
+// kSwiglu: the W rows of every 128-row tile are 64 gate rows then the 64
+// matching up rows; the epilogue writes h = silu(y_gate) * y_up (64 columns
+// per tile) instead of y, and the per-expert max |h|.
+template <bool kSwiglu>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                         const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_wc,
@@ -455,42 +466,85 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const float G = gscale_s[e];
       const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      constexpr int kChunks = kSwiglu ? BN / 64 : BN / 32;   // 32 output columns each
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c, ++nstore) {
-        uint32_t v[32], w[32];
-        tmem_load32(lane_base + buf * BN + c * 32, v);
-        if (nch) tmem_load32(lane_base + kCompCol + c * 32, w);
-        tmem_wait_ld();
-        if (c == BN / 32 - 1) {
-          // every TMEM read of this tile is done: hand the accumulators back
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(acc_empty0 + 8 * buf);
-            if (nch) mbar_arrive(compacc_empty);
-          }
-        }
+      for (int c = 0; c < kChunks; ++c, ++nstore) {
         uint32_t o[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          float a0 = __uint_as_float(v[2 * j]) * G, a1 = __uint_as_float(v[2 * j + 1]) * G;
-          if (nch) {
-            a0 += __uint_as_float(w[2 * j]);
-            a1 += __uint_as_float(w[2 * j + 1]);
+        unsigned int hmax = 0u;
+        if constexpr (!kSwiglu) {
+          uint32_t v[32], w[32];
+          tmem_load32(lane_base + buf * BN + c * 32, v);
+          if (nch) tmem_load32(lane_base + kCompCol + c * 32, w);
+          tmem_wait_ld();
+          if (c == kChunks - 1) {
+            // every TMEM read of this tile is done: hand the accumulators back
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+              mbar_arrive(acc_empty0 + 8 * buf);
+              if (nch) mbar_arrive(compacc_empty);
+            }
           }
-          o[j] = pack_bf16x2(a0, a1);
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            o[j] = pack_bf16x2(epi_value(v[2 * j], G, nch, w[2 * j]),
+                               epi_value(v[2 * j + 1], G, nch, w[2 * j + 1]));
+        } else {
+          // gate columns [32c, 32c + 32) and the matching up columns 64 further
+          uint32_t vg[32], vu[32], wg[32], wu[32];
+          tmem_load32(lane_base + buf * BN + c * 32, vg);
+          tmem_load32(lane_base + buf * BN + 64 + c * 32, vu);
+          if (nch) {
+            tmem_load32(lane_base + kCompCol + c * 32, wg);
+            tmem_load32(lane_base + kCompCol + 64 + c * 32, wu);
+          }
+          tmem_wait_ld();
+          if (c == kChunks - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+              mbar_arrive(acc_empty0 + 8 * buf);
+              if (nch) mbar_arrive(compacc_empty);
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            // y rounded to BF16 exactly as the plain epilogue stores it, then
+            // SwiGLU in FP32 as quads_swiglu computes it from that y
+            const uint32_t yg = pack_bf16x2(epi_value(vg[2 * j], G, nch, wg[2 * j]),
+                                            epi_value(vg[2 * j + 1], G, nch, wg[2 * j + 1]));
+            const uint32_t yu = pack_bf16x2(epi_value(vu[2 * j], G, nch, wu[2 * j]),
+                                            epi_value(vu[2 * j + 1], G, nch, wu[2 * j + 1]));
+            float r[2];
+#pragma unroll
+            for (int hl = 0; hl < 2; ++hl) {
+              const float gt = bf16_bits_to_float(hl ? (yg >> 16) : (yg & 0xFFFFu));
+              const float ut = bf16_bits_to_float(hl ? (yu >> 16) : (yu & 0xFFFFu));
+              r[hl] = __fmul_rn(__fdividef(gt, 1.0f + __expf(-gt)), ut);
+            }
+            o[j] = pack_bf16x2(r[0], r[1]);
+            hmax = max(hmax, max(o[j] & 0x7FFFu, (o[j] >> 16) & 0x7FFFu));
+          }
         }
         const uint32_t sb = stg + (nstore & 1) * kOutChunkBytes;
         if (lane == 0) bulk_wait_read_1();
         __syncwarp();
+        // 64-byte swizzle (the store's tensor map): 16-byte chunk j of row r sits
+        // at chunk j ^ ((r >> 1) & 3), so the 32 lanes' row stores hit all banks
         const uint32_t row_addr = sb + lane * 64;
+        const uint32_t sw = (lane >> 1) & 3u;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) st_shared_v4(row_addr + j * 16, o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+        for (int j = 0; j < 4; ++j)
+          st_shared_v4(row_addr + ((j ^ sw) << 4), o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(&tm_y, sb, nt * BN + c * 32, m0 + q * 32);
+          tma_store_2d(&tm_y, sb, (kSwiglu ? nt * (BN / 2) : nt * BN) + c * 32, m0 + q * 32);
           bulk_commit();
+        }
+        if constexpr (kSwiglu) {
+          hmax = __reduce_max_sync(0xffffffffu, hmax);
+          if (lane == 0 && hmax != 0u && p.amax_bits != nullptr) atomicMax(&p.amax_bits[e], hmax << 16);
         }
       }
     }
@@ -562,12 +616,16 @@ using namespace quads;
 
 extern "C" {
 
-int quads_moe_grouped_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_a,
-                                 int g_a_per_expert, const uint8_t* w_codes, const uint8_t* w_scales, const float* g_w,
-                                 const int32_t* expert_off, int E, int64_t rows_cap, int64_t N, int64_t K,
-                                 const uint16_t* a_resid, const uint16_t* w_resid, int n_chan, uint16_t* y,
-                                 quads_stream_t stream) {
-  clear_error();
+}  // extern "C"
+
+namespace quads {
+namespace {
+
+template <bool kSwiglu>
+int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_a, int g_a_per_expert,
+                const uint8_t* w_codes, const uint8_t* w_scales, const float* g_w, const int32_t* expert_off, int E,
+                int64_t rows_cap, int64_t N, int64_t K, const uint16_t* a_resid, const uint16_t* w_resid, int n_chan,
+                uint16_t* y, float* amax_out, cudaStream_t stream) {
   QUADS_REQUIRE(E >= 1 && E <= 256, QUADS_ERR_UNSUPPORTED_SHAPE, "E must be in [1, 256]");
   QUADS_REQUIRE(N > 0 && N % BN == 0 && N <= (int64_t(1) << 20), QUADS_ERR_UNSUPPORTED_SHAPE,
                 "N (%lld) must be a positive multiple of 128", (long long)N);
@@ -584,6 +642,8 @@ int quads_moe_grouped_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales
   QUADS_REQUIRE(aligned(a_codes, 16) && aligned(w_codes, 16) && aligned(a_scales, 16) && aligned(w_scales, 16) &&
                     aligned(y, 16) && (n_chan == 0 || (aligned(a_resid, 16) && aligned(w_resid, 16))),
                 QUADS_ERR_INVALID_ARG, "matrix pointers must be 16-byte aligned");
+  if (kSwiglu && amax_out && cudaMemsetAsync(amax_out, 0, sizeof(float) * E, stream) != cudaSuccess)
+    return set_error(QUADS_ERR_CUDA, "memset of amax_out failed");
   if (rows_cap == 0) return QUADS_OK;
 
   CUtensorMap tm_a, tm_b, tm_r, tm_wc, tm_y;
@@ -600,14 +660,14 @@ int quads_moe_grouped_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales
     tm_r = tm_a;
     tm_wc = tm_a;
   }
-  QUADS_TRY(make_map_2d(&tm_y, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, rows_cap, 32, 32,
-                        CU_TENSOR_MAP_SWIZZLE_NONE));
+  QUADS_TRY(make_map_2d(&tm_y, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kSwiglu ? N / 2 : N, rows_cap, 32, 32,
+                        CU_TENSOR_MAP_SWIZZLE_64B));
   const size_t smem_cap = 232448;   // 227 KB per block on sm_100
   int stages = kMaxStages;
   while (stages >= 2 && gemm_smem_bytes(stages, n_chan, E) > smem_cap) --stages;
   QUADS_REQUIRE(stages >= 2, QUADS_ERR_UNSUPPORTED_SHAPE, "not enough shared memory for two stages");
   const size_t smem = gemm_smem_bytes(stages, n_chan, E);
-  if (cudaFuncSetAttribute(grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(grouped_gemm_kernel<kSwiglu>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return set_error(QUADS_ERR_CUDA, "cannot set %zu bytes of shared memory", smem);
   GemmParams p;
@@ -617,6 +677,7 @@ int quads_moe_grouped_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales
   p.g_w = g_w;
   p.expert_off = expert_off;
   p.y = y;
+  p.amax_bits = reinterpret_cast<unsigned int*>(amax_out);
   p.g_a_per_expert = g_a_per_expert ? 1 : 0;
   p.E = E;
   p.N = static_cast<int>(N);
@@ -627,9 +688,36 @@ int quads_moe_grouped_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales
   const int64_t max_tiles = (rows_cap / BM) * (N / BN);
   int grid = num_sms();
   if (grid > max_tiles) grid = static_cast<int>(max_tiles);
-  grouped_gemm_kernel<<<grid, kThreads, smem, stream>>>(tm_a, tm_b, tm_r, tm_wc, tm_y, p);
+  grouped_gemm_kernel<kSwiglu><<<grid, kThreads, smem, stream>>>(tm_a, tm_b, tm_r, tm_wc, tm_y, p);
   count_launches(1);
   return check_launch("grouped_gemm_kernel");
+}
+
+}  // namespace
+}  // namespace quads
+
+extern "C" {
+
+int quads_moe_grouped_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_a,
+                                 int g_a_per_expert, const uint8_t* w_codes, const uint8_t* w_scales, const float* g_w,
+                                 const int32_t* expert_off, int E, int64_t rows_cap, int64_t N, int64_t K,
+                                 const uint16_t* a_resid, const uint16_t* w_resid, int n_chan, uint16_t* y,
+                                 quads_stream_t stream) {
+  clear_error();
+  return launch_gemm<false>(a_codes, a_scales, g_a, g_a_per_expert, w_codes, w_scales, g_w, expert_off, E, rows_cap,
+                            N, K, a_resid, w_resid, n_chan, y, nullptr, stream);
+}
+
+int quads_moe_grouped_gemm_nvfp4_swiglu(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_a,
+                                        int g_a_per_expert, const uint8_t* w_codes, const uint8_t* w_scales,
+                                        const float* g_w, const int32_t* expert_off, int E, int64_t rows_cap,
+                                        int64_t F, int64_t K, const uint16_t* a_resid, const uint16_t* w_resid,
+                                        int n_chan, uint16_t* h, float* amax_out, quads_stream_t stream) {
+  clear_error();
+  QUADS_REQUIRE(F > 0 && F % 64 == 0, QUADS_ERR_UNSUPPORTED_SHAPE, "F (%lld) must be a positive multiple of 64",
+                (long long)F);
+  return launch_gemm<true>(a_codes, a_scales, g_a, g_a_per_expert, w_codes, w_scales, g_w, expert_off, E, rows_cap,
+                           2 * F, K, a_resid, w_resid, n_chan, h, amax_out, stream);
 }
 
 int quads_device_status(quads_stream_t stream) {

@@ -177,13 +177,16 @@ __global__ void __launch_bounds__(kSmallThreads) permute_small_kernel(const int3
   __shared__ int32_t cnt[kMaxE];
   __shared__ int32_t running[kMaxE];
   __shared__ int32_t padded[kMaxE];
-  __shared__ int32_t wcnt[kWarps][kMaxE];
+  __shared__ int32_t wcnt[kWarps * kMaxE];             // [warp][expert], stride E
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < E; i += blockDim.x) cnt[i] = 0;
   __syncthreads();
-  for (int i = threadIdx.x; i < n_pairs; i += blockDim.x) {
-    const int e = idx[i];
-    if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
+  // warp-aggregated histogram: one shared atomic per distinct expert in a warp
+  for (int i0 = 0; i0 < n_pairs; i0 += blockDim.x) {
+    const int i = i0 + threadIdx.x;
+    const int e = (i < n_pairs) ? idx[i] : -1;
+    const unsigned int peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && e < E && lane == __ffs(peers) - 1) atomicAdd(&cnt[e], __popc(peers));
   }
   __syncthreads();
   if (threadIdx.x < E) padded[threadIdx.x] = (cnt[threadIdx.x] + 127) / 128 * 128;
@@ -198,25 +201,25 @@ __global__ void __launch_bounds__(kSmallThreads) permute_small_kernel(const int3
     if (e == E - 1) expert_off[E] = off + padded[e];
   }
   for (int r0 = 0; r0 < n_pairs; r0 += kSmallThreads) {
-    for (int i = threadIdx.x; i < kWarps * kMaxE; i += blockDim.x) (&wcnt[0][0])[i] = 0;
+    for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) wcnt[i] = 0;
     __syncthreads();
     const int i = r0 + threadIdx.x;
     const bool valid = i < n_pairs;
     const int e = valid ? idx[i] : -1;
     const unsigned int peers = __match_any_sync(0xffffffffu, e);
     const int rank_w = __popc(peers & ((1u << lane) - 1u));
-    if (valid && lane == __ffs(peers) - 1 && e >= 0 && e < E) wcnt[wid][e] = __popc(peers);
+    if (valid && lane == __ffs(peers) - 1 && e >= 0 && e < E) wcnt[wid * E + e] = __popc(peers);
     __syncthreads();
     if (valid && e >= 0 && e < E) {
       int pos = running[e] + rank_w;
-      for (int w = 0; w < wid; ++w) pos += wcnt[w][e];
+      for (int w = 0; w < wid; ++w) pos += wcnt[w * E + e];
       row_of[i] = pos;
       src_of[pos] = i / k;
     }
     __syncthreads();
     for (int x = threadIdx.x; x < E; x += blockDim.x) {
       int add = 0;
-      for (int w = 0; w < kWarps; ++w) add += wcnt[w][x];
+      for (int w = 0; w < kWarps; ++w) add += wcnt[w * E + x];
       running[x] += add;
     }
     __syncthreads();
@@ -320,22 +323,40 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
     rows[s] = row_of[t * k + s];
     ws[s] = w[t * k + s];
   }
-  for (int64_t c = lane * 8; c < H; c += 32 * 8) {
-    float acc[8];
+  // four 8-column chunks per lane per iteration: the k x 4 loads of a slot are
+  // independent, so they are in flight together
+  for (int64_t c0 = lane * 8; c0 < H; c0 += 4 * 32 * 8) {
+    float acc[4][8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[u][j] = 0.0f;
     for (int s = 0; s < k; ++s) {
-      uint4 v = __ldg(reinterpret_cast<const uint4*>(y + static_cast<int64_t>(rows[s]) * H + c));
-      const uint32_t* p = reinterpret_cast<const uint32_t*>(&v);
+      uint4 v[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        acc[2 * j] = __fmaf_rn(ws[s], bf16_bits_to_float(p[j] & 0xFFFFu), acc[2 * j]);
-        acc[2 * j + 1] = __fmaf_rn(ws[s], bf16_bits_to_float(p[j] >> 16), acc[2 * j + 1]);
+      for (int u = 0; u < 4; ++u) {
+        const int64_t c = c0 + u * 256;
+        v[u] = c < H ? __ldg(reinterpret_cast<const uint4*>(y + static_cast<int64_t>(rows[s]) * H + c))
+                     : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t* p = reinterpret_cast<const uint32_t*>(&v[u]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          acc[u][2 * j] = __fmaf_rn(ws[s], bf16_bits_to_float(p[j] & 0xFFFFu), acc[u][2 * j]);
+          acc[u][2 * j + 1] = __fmaf_rn(ws[s], bf16_bits_to_float(p[j] >> 16), acc[u][2 * j + 1]);
+        }
       }
     }
-    *reinterpret_cast<uint4*>(out + t * H + c) =
-        make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
-                   pack_bf16x2(acc[6], acc[7]));
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t c = c0 + u * 256;
+      if (c < H)
+        *reinterpret_cast<uint4*>(out + t * H + c) =
+            make_uint4(pack_bf16x2(acc[u][0], acc[u][1]), pack_bf16x2(acc[u][2], acc[u][3]),
+                       pack_bf16x2(acc[u][4], acc[u][5]), pack_bf16x2(acc[u][6], acc[u][7]));
+    }
   }
 }
 

@@ -8,10 +8,12 @@
 // [QUADS-fr §2.2.A] (trainer weights fake-quantized onto the rollout's grid,
 // straight-through backward).
 //
-// Every kernel is HBM-bound: one thread owns one 16-element block (32 bytes of
-// BF16 in, 8 bytes of codes and 1 scale byte out), a warp covers 32
-// consecutive blocks of a row (1 KB contiguous), grids are grid-stride loops
-// sized to a multiple of the SM count.
+// Every kernel is HBM-bound.  amax and quantize take one warp per row: a lane
+// owns one 16-element block per pass (32 bytes of BF16 in; 8 bytes of codes
+// and one scale byte out), a pass covers 32 consecutive blocks (1 KB), and a
+// warp keeps two passes of loads in flight.  Grids are persistent: as many
+// CTAs as fit on the SMs at once.  The elementwise kernels (dequantize, STE
+// backward) are grid-stride loops.
 #include <cstdio>
 #include <mutex>
 
@@ -23,6 +25,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kMaxGroupsSmem = 1024;
 constexpr int kMaxChan = 256;
+constexpr int kTabGroups = 16;     // up to this many groups get a {S, 1/S} table in shared memory
 constexpr int64_t kMaxBlocks = int64_t(1) << 31;
 
 int grid_for(int64_t work, int per_block = kThreads) {
@@ -107,6 +110,9 @@ struct QuantArgs {
   int resid_mode;          // 0: residual, 1: bf16(deq), 2: the input itself
   uint16_t* w_fq;          // [rows][K] or null
   int fold;                // w_fq = bf16(deq) (1) or e2m1 * e4m3 (0)
+  int64_t ilv_half;        // > 0: codes, scales and resid rows of each group of
+                           // 2 * ilv_half rows interleaved in blocks of 64 (first
+                           // half 64 rows, second half 64 rows, ...); 0: input order
   FastDiv uniform_div;     // filled by launch_quantize: rows per group (uniform groups)
 };
 
@@ -115,11 +121,14 @@ struct QuantArgs {
 // cooperatively: lane j takes channel slot j and fetches its element, code and
 // scale from the lane that owns the block by warp shuffles, then the warp
 // writes the row's residual slots as one contiguous store.
-__global__ void __launch_bounds__(kThreads, 3) quantize_kernel(QuantArgs a) {
-  extern __shared__ int32_t smem[];
+__global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a) {
+  extern __shared__ int32_t smem_q[];
   const int n = a.n_groups;
   const int nkb = static_cast<int>(a.K / 16);
   const int npass = (nkb + 31) / 32;
+  const bool use_tab = n <= kTabGroups;
+  float2* tab = reinterpret_cast<float2*>(smem_q);         // n x 128 {S, 1/S} (few groups)
+  int32_t* smem = smem_q + (use_tab ? n * 128 * 2 : 0);
   int32_t* off_s = smem;                                   // n + 1
   float* g_s = reinterpret_cast<float*>(smem + n + 1);     // n
   int32_t* pass_slot = smem + 2 * n + 1;                   // npass + 1 (with channels)
@@ -133,6 +142,9 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_kernel(QuantArgs a) {
       if (blockIdx.x == 0 && a.g_out != nullptr) a.g_out[i] = g;
     }
   }
+  if (use_tab)
+    for (int i = threadIdx.x; i < n * 128; i += blockDim.x)
+      tab[i] = scale_table_entry(i & 127, __fdiv_rn(a.amax[i >> 7], kNvfp4Range));
   if (a.n_chan) {
     for (int j = threadIdx.x; j < a.n_chan; j += blockDim.x) chan_s[j] = a.chan[j];
     __syncthreads();
@@ -169,8 +181,17 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_kernel(QuantArgs a) {
         for (int kb = lane; kb < nkb_e; kb += 32) a.scales[tiled_scale_offset(row, kb, ncol_tiles)] = 0;
       continue;
     }
-    const float g = g_s[grp.of(row)];
+    const int gi = grp.of(row);
+    const float g = g_s[gi];
+    const QConsts qc = make_qconsts(g, use_tab ? tab + gi * 128 : nullptr);
     const uint16_t* xr = a.x + row * a.ld;
+    int64_t drow = row;                                // row of the codes, scales and resid outputs
+    if (a.ilv_half) {
+      const int64_t base = static_cast<int64_t>(gi) * 2 * a.ilv_half, loc = row - base;
+      const bool second = loc >= a.ilv_half;
+      const int64_t f = second ? loc - a.ilv_half : loc;
+      drow = base + (f >> 6) * 128 + (second ? 64 : 0) + (f & 63);
+    }
     for (int p0 = 0; p0 < npass; p0 += 2) {
       uint32_t w[2][8];
 #pragma unroll
@@ -185,9 +206,9 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_kernel(QuantArgs a) {
         const int kb = p * 32 + lane;
         QCore q{0u, 0u, 0u, 0.0f};
         if (kb < nkb) {
-          q = quant_core(w[u], g);
+          q = quant_core(w[u], qc);
           if (a.codes)
-            *reinterpret_cast<uint2*>(a.codes + row * (a.K / 2) + kb * 8) = make_uint2(q.lo, q.hi);
+            *reinterpret_cast<uint2*>(a.codes + drow * (a.K / 2) + kb * 8) = make_uint2(q.lo, q.hi);
           if (a.w_fq) {
             uint32_t o[8];
             deq_block_bf16(q, g, a.fold, o);
@@ -197,45 +218,52 @@ __global__ void __launch_bounds__(kThreads, 3) quantize_kernel(QuantArgs a) {
           }
         }
         if (a.scales && kb < nkb_e)
-          a.scales[tiled ? tiled_scale_offset(row, kb, ncol_tiles) : row * nkb + kb] =
+          a.scales[tiled ? tiled_scale_offset(drow, kb, ncol_tiles) : drow * nkb + kb] =
               static_cast<uint8_t>(q.scale);
         if (a.resid) {
+          // Channel slot j of this pass is taken by lane j % 32.  The element
+          // itself is read back through L2 (the input row, or, for bf16(deq)
+          // with the scale folded, the W_fq row this warp has just written);
+          // its code and block scale come from the owning lane by shuffles.
           const int slo = pass_slot[p], shi = pass_slot[p + 1];
+          const bool from_fq = a.resid_mode == 1 && a.fold && a.w_fq != nullptr;
+          if (from_fq) __syncwarp();                     // this warp's W_fq stores are visible to it
           for (int j0 = slo; j0 < shi; j0 += 32) {       // warp-uniform
             const int j = j0 + lane;
             const bool act = j < shi;
             const int c = act ? chan_s[j] : 512 * p;
             const int src = (c - 512 * p) >> 4, bit = c & 15;
-            uint32_t word = 0;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const uint32_t v = __shfl_sync(0xffffffffu, w[u][i], src);
-              word = ((bit >> 1) == i) ? v : word;
-            }
-            const uint32_t cl = __shfl_sync(0xffffffffu, q.lo, src);
-            const uint32_t ch = __shfl_sync(0xffffffffu, q.hi, src);
-            const float sv = __shfl_sync(0xffffffffu, q.sv, src);
-            const float xv = bf16_bits_to_float((bit & 1) ? (word >> 16) : (word & 0xFFFFu));
-            const uint32_t code = (((bit < 8) ? cl : ch) >> (4 * (bit & 7))) & 15u;
-            float v;
-            if (a.resid_mode == 2) {
-              v = xv;
+            uint32_t vb;
+            if (from_fq) {
+              vb = act ? a.w_fq[row * a.K + c] : 0u;
             } else {
-              const float dq = deq_f32(code, sv, g);
-              v = (a.resid_mode == 1) ? dq : __fsub_rn(xv, dq);
+              const uint32_t cl = __shfl_sync(0xffffffffu, q.lo, src);
+              const uint32_t ch = __shfl_sync(0xffffffffu, q.hi, src);
+              const float sv = __shfl_sync(0xffffffffu, q.sv, src);
+              const float xv = act ? bf16_bits_to_float(__ldg(xr + c)) : 0.0f;
+              const uint32_t code = (((bit < 8) ? cl : ch) >> (4 * (bit & 7))) & 15u;
+              float v;
+              if (a.resid_mode == 2) {
+                v = xv;
+              } else {
+                const float dq = deq_f32(code, sv, g);
+                v = (a.resid_mode == 1) ? dq : __fsub_rn(xv, dq);
+              }
+              vb = float_to_bf16_bits(v);
             }
-            if (act) a.resid[row * a.n_chan + j] = static_cast<uint16_t>(float_to_bf16_bits(v));
+            if (act) a.resid[drow * a.n_chan + j] = static_cast<uint16_t>(vb);
           }
         }
       }
     }
     if (a.resid)
-      for (int j = n_valid + lane; j < a.n_chan; j += 32) a.resid[row * a.n_chan + j] = 0;
+      for (int j = n_valid + lane; j < a.n_chan; j += 32) a.resid[drow * a.n_chan + j] = 0;
   }
 }
 
 size_t quantize_smem(int n_groups, int64_t K, int n_chan) {
   size_t s = (2 * static_cast<size_t>(n_groups) + 1) * 4;
+  if (n_groups <= kTabGroups) s += static_cast<size_t>(n_groups) * 128 * sizeof(float2);
   if (n_chan) s += (static_cast<size_t>((K / 16 + 31) / 32) + 1 + n_chan) * 4;
   return s;
 }
@@ -592,12 +620,15 @@ int quads_select_channels(const float* scores, int64_t K, int n_sel, int32_t* ch
   return check_launch("select_kernel");
 }
 
-int quads_fakequant_weight_ste(const uint16_t* w, int64_t n_mat, int64_t rows, int64_t K, const float* amax_in,
-                               int fold_global,
-                               uint16_t* w_fq, uint8_t* codes, uint8_t* scales, float* g_out, const int32_t* chan,
-                               int n_chan, int chan_raw, uint16_t* w_chan, void* ws, size_t ws_bytes,
-                               quads_stream_t stream) {
-  clear_error();
+}  // extern "C"
+
+namespace quads {
+namespace {
+
+int fakequant_impl(const uint16_t* w, int64_t n_mat, int64_t rows, int64_t K, const float* amax_in, int fold_global,
+                   uint16_t* w_fq, uint8_t* codes, uint8_t* scales, float* g_out, const int32_t* chan, int n_chan,
+                   int chan_raw, uint16_t* w_chan, void* ws, size_t ws_bytes, int64_t ilv_half,
+                   quads_stream_t stream) {
   QUADS_REQUIRE(n_mat >= 1 && n_mat <= kMaxGroupsSmem, QUADS_ERR_UNSUPPORTED_SHAPE, "n_mat must be in [1, %d]",
                 kMaxGroupsSmem);
   QUADS_TRY(validate_matrix(w, n_mat * rows, K, K));
@@ -622,7 +653,34 @@ int quads_fakequant_weight_ste(const uint16_t* w, int64_t n_mat, int64_t rows, i
   a.scale_layout = (rows % 128 == 0) ? QUADS_SCALES_TILED : QUADS_SCALES_LINEAR;
   a.g_out = g_out; a.chan = chan; a.n_chan = n_chan; a.resid = n_chan ? w_chan : nullptr;
   a.resid_mode = chan_raw ? 2 : 1; a.w_fq = w_fq; a.fold = fold_global ? 1 : 0;
+  a.ilv_half = ilv_half;
   return launch_quantize(a, stream);
+}
+
+}  // namespace
+}  // namespace quads
+
+extern "C" {
+
+int quads_fakequant_weight_ste(const uint16_t* w, int64_t n_mat, int64_t rows, int64_t K, const float* amax_in,
+                               int fold_global,
+                               uint16_t* w_fq, uint8_t* codes, uint8_t* scales, float* g_out, const int32_t* chan,
+                               int n_chan, int chan_raw, uint16_t* w_chan, void* ws, size_t ws_bytes,
+                               quads_stream_t stream) {
+  clear_error();
+  return fakequant_impl(w, n_mat, rows, K, amax_in, fold_global, w_fq, codes, scales, g_out, chan, n_chan, chan_raw,
+                        w_chan, ws, ws_bytes, 0, stream);
+}
+
+int quads_fakequant_weight_ste_gate_up(const uint16_t* w, int64_t n_mat, int64_t rows, int64_t K,
+                                       const float* amax_in, int fold_global, uint16_t* w_fq, uint8_t* codes,
+                                       uint8_t* scales, float* g_out, const int32_t* chan, int n_chan, int chan_raw,
+                                       uint16_t* w_chan, void* ws, size_t ws_bytes, quads_stream_t stream) {
+  clear_error();
+  QUADS_REQUIRE(rows > 0 && rows % 128 == 0, QUADS_ERR_UNSUPPORTED_SHAPE,
+                "rows (gate and up) must be a positive multiple of 128");
+  return fakequant_impl(w, n_mat, rows, K, amax_in, fold_global, w_fq, codes, scales, g_out, chan, n_chan, chan_raw,
+                        w_chan, ws, ws_bytes, rows / 2, stream);
 }
 
 int quads_fakequant_weight_ste_backward(const uint16_t* grad_wfq, uint16_t* grad_w, int64_t n, int accumulate,

@@ -97,8 +97,11 @@ __global__ void __launch_bounds__(kThreads, 3) replay_kernel(ReplayArgs a) {
   extern __shared__ int32_t smem[];
   __shared__ trace_qrecord_header h;
   __shared__ int ok;
+  static_assert(sizeof(trace_qrecord_header) % 4 == 0, "header is copied as 32-bit words");
+  for (int i = threadIdx.x; i < static_cast<int>(sizeof(h) / 4); i += blockDim.x)
+    reinterpret_cast<uint32_t*>(&h)[i] = reinterpret_cast<const uint32_t*>(a.record)[i];
+  __syncthreads();
   if (threadIdx.x == 0) {
-    memcpy(&h, a.record, sizeof(h));
     ok = record_ok(a, h) ? 1 : 0;
     if (blockIdx.x == 0) *a.status = ok ? QUADS_OK : QUADS_ERR_BAD_RECORD;
   }
@@ -147,6 +150,7 @@ __global__ void __launch_bounds__(kThreads, 3) replay_kernel(ReplayArgs a) {
   for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
        row += warps) {
     const float g = g_s[grp.of(row)];
+    const QConsts qc = make_qconsts(g);
     for (int p0 = 0; p0 < npass; p0 += 2) {
       uint2 cw[2];
       uint32_t sc[2], xw[2][8];
@@ -176,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 3) replay_kernel(ReplayArgs a) {
           dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
           dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
           if (a.x_train) {
-            const QCore t = quant_core(xw[u], g);
+            const QCore t = quant_core(xw[u], qc);
             // nibbles that differ: OR-fold each nibble onto its low bit, count
             uint32_t d0 = t.lo ^ q.lo, d1 = t.hi ^ q.hi;
             d0 = (d0 | (d0 >> 1) | (d0 >> 2) | (d0 >> 3)) & 0x11111111u;
@@ -280,6 +284,7 @@ int trace_export_qrecord(int layer_id, int64_t T, int k, const int32_t* topk_idx
   auto add = [&](const void* src, uint64_t off, uint64_t bytes) -> int {
     if (bytes == 0) return QUADS_OK;
     if (!src) return set_error(QUADS_ERR_INVALID_ARG, "null section pointer");
+    if (src == static_cast<const uint8_t*>(record) + off) return QUADS_OK;   // produced in place
     a.seg[n].src = static_cast<const uint8_t*>(src);
     a.seg[n].dst_off = off;
     a.seg[n].bytes = bytes;

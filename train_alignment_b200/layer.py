@@ -14,6 +14,7 @@ compensation weight columns), the straight-through backward accumulated
 into the master gradient, the export of the rollout's quantization record
 and its replay against the trainer's activation.
 """
+import math
 from dataclasses import dataclass
 
 import torch
@@ -50,44 +51,77 @@ class MoELayer:
     """Weights, calibrated channel sets and every buffer of one layer at a
     fixed token count; step() runs the whole path without allocating."""
 
-    def __init__(self, cfg: MoEConfig, w_gu, w_d, chan_x, chan_h, device="cuda"):
+    def __init__(self, cfg: MoEConfig, w_gu, w_d, chan_x, chan_h, device="cuda", fuse_swiglu=None):
         self.cfg = cfg
         T, H, E, k, F = cfg.T, cfg.H, cfg.E, cfg.k, cfg.F
         dev = torch.device(device)
         self.dev = dev
-        self.w_gu = w_gu.contiguous()                   # [E, 2F, H] trainer master weights
-        self.w_d = w_d.contiguous()                     # [E, H, F]
-        self.chan_x = chan_x.to(dev, torch.int32).contiguous()
-        self.chan_h = chan_h.to(dev, torch.int32).contiguous()
-        self.nc_x = int(self.chan_x.numel())
-        self.nc_h = int(self.chan_h.numel())
+        # trainer master weights, both matrices in one allocation (gate/up
+        # [E, 2F, H] then down [E, H, F]) so that one amax pass covers both
+        n_gu, n_d = E * 2 * F * H, E * H * F
+        self.n_gu, self.n_d = n_gu, n_d
+        self.w_all = torch.empty(n_gu + n_d, dtype=torch.bfloat16, device=dev)
+        self.w_all[:n_gu].copy_(w_gu.reshape(-1))
+        self.w_all[n_gu:].copy_(w_d.reshape(-1))
+        self.w_gu = self.w_all[:n_gu].view(E, 2 * F, H)
+        self.w_d = self.w_all[n_gu:].view(E, H, F)
+        # rows of a common width for the joint amax: each expert matrix is a group
+        kw = math.gcd(H, F)
+        self.amax_k = kw if kw % 16 == 0 else 0
+        if self.amax_k:
+            offs = [e * 2 * F * H // kw for e in range(E)] + [(n_gu + e * H * F) // kw for e in range(E + 1)]
+            self.w_groups = torch.tensor(offs, dtype=torch.int32, device=dev)
+        # SwiGLU in the gate/up GEMM's epilogue (rollout gate/up weights kept
+        # in the 64-row interleaved gate/up order), else a separate pass
+        self.fuse_swiglu = (F % 64 == 0) if fuse_swiglu is None else bool(fuse_swiglu)
+        self.nc_x = int(chan_x.numel())
+        self.nc_h = int(chan_h.numel())
         cap = B.moe_rows_capacity(T, k, E)
         self.cap = cap
         e = lambda shape, dt: torch.empty(shape, dtype=dt, device=dev)
         bf, u8, f32, i32 = torch.bfloat16, torch.uint8, torch.float32, torch.int32
+        # TRACE record: the rollout's kernels write the recorded tensors (codes,
+        # scales, per-tensor scales, residuals, expert offsets, top-k indices)
+        # straight into their sections, so the export writes only the header
+        slot_x = B.qtensor_shape(T, H, B.SCALES_LINEAR, 1, self.nc_x)
+        slot_h = B.qtensor_shape(cap, F, B.SCALES_TILED, E, self.nc_h)
+        self.record_bytes, hdr = B.trace_qrecord_layout(0, T, k, [slot_x, slot_h])
+        self.record = torch.zeros(self.record_bytes, dtype=u8, device=dev)
+        vx, vh = B.record_views(self.record, hdr, 0), B.record_views(self.record, hdr, 1)
+        none_i32 = torch.empty(0, dtype=i32, device=dev)
+        self.chan_x = vx["chan"] if self.nc_x else none_i32
+        self.chan_h = vh["chan"] if self.nc_h else none_i32
+        self.chan_x.copy_(chan_x.to(dev, torch.int32))
+        self.chan_h.copy_(chan_h.to(dev, torch.int32))
         # weight sync outputs
         self.w_gu_fq, self.w_d_fq = e((E, 2 * F, H), bf), e((E, H, F), bf)
         self.w_gu_codes, self.w_d_codes = e((E, 2 * F, H // 2), u8), e((E, H, F // 2), u8)
         self.w_gu_scales = e((B.scales_bytes(E * 2 * F, H, B.SCALES_TILED),), u8)
         self.w_d_scales = e((B.scales_bytes(E * H, F, B.SCALES_TILED),), u8)
         self.g_w_gu, self.g_w_d = e((E,), f32), e((E,), f32)
-        self.amax_w_gu, self.amax_w_d, self.amax_x = e((E,), f32), e((E,), f32), e((1,), f32)
+        self.amax_w_all, self.amax_x = e((2 * E,), f32), e((1,), f32)
+        self.amax_w_gu, self.amax_w_d = self.amax_w_all[:E], self.amax_w_all[E:]
         self.wc_gu, self.wc_d = e((E, 2 * F, self.nc_x), bf), e((E, H, self.nc_h), bf)
         self.ws_w = e((B.quantize_workspace_bytes(E),), u8)
         # STE gradients (master gradient accumulated in place)
-        self.grad_gu, self.grad_d = torch.zeros_like(self.w_gu), torch.zeros_like(self.w_d)
+        self.grad_all = torch.zeros_like(self.w_all)
+        self.grad_gu, self.grad_d = self.grad_all[:n_gu].view(E, 2 * F, H), self.grad_all[n_gu:].view(E, H, F)
         # rollout activations
-        self.x_codes, self.x_scales = e((T, H // 2), u8), e((B.scales_bytes(T, H, B.SCALES_LINEAR),), u8)
-        self.g_x, self.x_resid, self.ws_x = e((1,), f32), e((T, self.nc_x), bf), e((B.quantize_workspace_bytes(1),), u8)
-        self.topk_idx, self.topk_w = e((T, k), i32), e((T, k), f32)
-        self.expert_off, self.row_of, self.src_of = e((E + 1,), i32), e((T * k,), i32), e((cap,), i32)
+        self.x_codes, self.x_scales = vx["codes"].view(T, H // 2), vx["scales"]
+        self.g_x = vx["g"]
+        self.x_resid = vx["resid"].view(T, self.nc_x) if self.nc_x else None
+        self.ws_x = e((B.quantize_workspace_bytes(1),), u8)
+        self.topk_idx = self.record[hdr.topk_idx_off:hdr.topk_idx_off + 4 * T * k].view(i32).view(T, k)
+        self.topk_w = e((T, k), f32)
+        self.expert_off, self.row_of, self.src_of = vh["group_off"], e((T * k,), i32), e((cap,), i32)
         self.ws_perm = e((B.moe_permute_workspace_bytes(T, k, E),), u8)
         self.pa_codes, self.pa_scales = e((cap, H // 2), u8), e((B.scales_bytes(cap, H, B.SCALES_TILED),), u8)
         self.pa_resid = e((cap, self.nc_x), bf)
-        self.y_gu = e((cap, 2 * F), bf)
+        self.y_gu = None if self.fuse_swiglu else e((cap, 2 * F), bf)
         self.h, self.amax_h = e((cap, F), bf), e((E,), f32)
-        self.h_codes, self.h_scales = e((cap, F // 2), u8), e((B.scales_bytes(cap, F, B.SCALES_TILED),), u8)
-        self.g_h, self.h_resid = e((E,), f32), e((cap, self.nc_h), bf)
+        self.h_codes, self.h_scales = vh["codes"].view(cap, F // 2), vh["scales"]
+        self.g_h = vh["g"]
+        self.h_resid = vh["resid"].view(cap, self.nc_h) if self.nc_h else None
         self.y_d = e((cap, H), bf)
         self.out = e((T, H), bf)
         # TRACE record and replay outputs
@@ -97,8 +131,6 @@ class MoELayer:
             B.qtensor_src(self.h_codes, self.h_scales, self.g_h, cap, F, B.SCALES_TILED, group_off=self.expert_off,
                           chan=self.chan_h, resid=self.h_resid),
         ]
-        self.record_bytes, _ = B.trace_qrecord_layout(0, T, k, self._tsrc)
-        self.record = e((self.record_bytes,), u8)
         self.x_hat, self.h_hat = e((T, H), bf), e((cap, F), bf)
         self.counts, self.status = torch.zeros(2, dtype=torch.int64, device=dev), e((1,), i32)
         self.status_h = e((1,), i32)
@@ -106,28 +138,45 @@ class MoELayer:
     # ---------------------------------------------------------------- stages
 
     def weight_sync(self, timer=None):
-        """Trainer fake-quant + the rollout's NVFP4 weights: one amax pass and
-        one quantize pass per weight tensor."""
+        """Trainer fake-quant + the rollout's NVFP4 weights: one amax pass over
+        both weight tensors, then one quantize pass per weight tensor."""
         cfg = self.cfg
         t = timer or StageTimer(False)
         E, F, H = cfg.E, cfg.F, cfg.H
-        B.amax_bf16(self.w_gu.view(E * 2 * F, H), n_groups=E, out=self.amax_w_gu)
-        t.mark("amax_w_gate_up")
+        if self.amax_k:
+            B.amax_bf16(self.w_all.view(-1, self.amax_k), self.w_groups, 2 * E, out=self.amax_w_all)
+            t.mark("amax_w")
+        else:
+            B.amax_bf16(self.w_gu.view(E * 2 * F, H), n_groups=E, out=self.amax_w_gu)
+            B.amax_bf16(self.w_d.view(E * H, F), n_groups=E, out=self.amax_w_d)
+            t.mark("amax_w")
         B.fakequant_weight_ste(self.w_gu, True, self.chan_x, False, True, self.w_gu_fq, self.w_gu_codes,
-                               self.w_gu_scales, self.g_w_gu, self.wc_gu, None, self.amax_w_gu)
+                               self.w_gu_scales, self.g_w_gu, self.wc_gu, None, self.amax_w_gu,
+                               gate_up=self.fuse_swiglu)
         t.mark("fakequant_w_gate_up")
-        B.amax_bf16(self.w_d.view(E * H, F), n_groups=E, out=self.amax_w_d)
-        t.mark("amax_w_down")
         B.fakequant_weight_ste(self.w_d, True, self.chan_h, False, True, self.w_d_fq, self.w_d_codes,
                                self.w_d_scales, self.g_w_d, self.wc_d, None, self.amax_w_d)
         t.mark("fakequant_w_down")
 
     def ste_backward(self, grad_gu_fq, grad_d_fq, timer=None):
+        """Straight-through backward of both weight tensors, accumulated into
+        the master gradient; one pass when the two incoming gradients are
+        adjacent in one allocation (as grad_fq_buffers() makes them)."""
         t = timer or StageTimer(False)
-        B.fakequant_weight_ste_backward(grad_gu_fq, self.grad_gu, accumulate=True)
-        t.mark("ste_backward_gate_up")
-        B.fakequant_weight_ste_backward(grad_d_fq, self.grad_d, accumulate=True)
-        t.mark("ste_backward_down")
+        flat = _adjacent(grad_gu_fq, grad_d_fq)
+        if flat is not None:
+            B.fakequant_weight_ste_backward(flat, self.grad_all, accumulate=True)
+        else:
+            B.fakequant_weight_ste_backward(grad_gu_fq, self.grad_gu, accumulate=True)
+            B.fakequant_weight_ste_backward(grad_d_fq, self.grad_d, accumulate=True)
+        t.mark("ste_backward")
+
+    def grad_fq_buffers(self):
+        """(flat, gate/up view, down view): one allocation for the gradients
+        with respect to both fake-quantized weights."""
+        flat = torch.empty_like(self.w_all)
+        E, F, H = self.cfg.E, self.cfg.F, self.cfg.H
+        return flat, flat[:self.n_gu].view(E, 2 * F, H), flat[self.n_gu:].view(E, H, F)
 
     def rollout_forward(self, x, logits, timer=None):
         cfg = self.cfg
@@ -145,12 +194,18 @@ class MoELayer:
         B.moe_gather(self.src_of, self.expert_off, E, self.cap, self.x_codes, self.x_scales, H, self.x_resid,
                      self.pa_codes, self.pa_scales, self.pa_resid)
         t.mark("gather")
-        B.moe_grouped_gemm_nvfp4(self.pa_codes, self.pa_scales, self.g_x, self.w_gu_codes, self.w_gu_scales,
-                                 self.g_w_gu, self.expert_off, E, self.cap, 2 * F, H, self.pa_resid, self.wc_gu,
-                                 y=self.y_gu)
-        t.mark("gemm_gate_up")
-        B.swiglu(self.y_gu, F, self.expert_off, E, h=self.h, amax=self.amax_h)
-        t.mark("swiglu")
+        if self.fuse_swiglu:
+            B.moe_grouped_gemm_nvfp4_swiglu(self.pa_codes, self.pa_scales, self.g_x, self.w_gu_codes,
+                                            self.w_gu_scales, self.g_w_gu, self.expert_off, E, self.cap, F, H,
+                                            self.pa_resid, self.wc_gu, h=self.h, amax=self.amax_h)
+            t.mark("gemm_gate_up_swiglu")
+        else:
+            B.moe_grouped_gemm_nvfp4(self.pa_codes, self.pa_scales, self.g_x, self.w_gu_codes, self.w_gu_scales,
+                                     self.g_w_gu, self.expert_off, E, self.cap, 2 * F, H, self.pa_resid, self.wc_gu,
+                                     y=self.y_gu)
+            t.mark("gemm_gate_up")
+            B.swiglu(self.y_gu, F, self.expert_off, E, h=self.h, amax=self.amax_h)
+            t.mark("swiglu")
         B.quantize_nvfp4(self.h, group_off=self.expert_off, n_groups=E, amax_in=self.amax_h,
                          scale_layout=B.SCALES_TILED, chan=self.chan_h, codes=self.h_codes, scales=self.h_scales,
                          g_out=self.g_h, resid_out=self.h_resid)
@@ -190,6 +245,17 @@ class MoELayer:
 
     def reset_counts(self):
         self.counts.zero_()
+
+
+def _adjacent(a, b):
+    """A flat view over a then b when b directly follows a in one storage."""
+    if a.dtype != b.dtype or a.device != b.device or not (a.is_contiguous() and b.is_contiguous()):
+        return None
+    if a.untyped_storage().data_ptr() != b.untyped_storage().data_ptr():
+        return None
+    if b.storage_offset() != a.storage_offset() + a.numel():
+        return None
+    return torch.as_strided(a, (a.numel() + b.numel(),), (1,), a.storage_offset())
 
 
 def calibrate_channels(x, n_sel):
