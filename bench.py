@@ -53,6 +53,7 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the standalone quantize/replay size sweep")
     return ap.parse_args()
 
 
@@ -172,6 +173,66 @@ def kernel_work(cfg, rpad):
         "ste_backward": ("hbm", (wgu + wd) * 6.0),
     }
     return w
+
+
+# ------------------------------------------------------ quantize / replay sweep
+
+SWEEP_LOG2 = (20, 22, 24, 26, 28, 30)       # BF16 elements, rows of 4096
+
+
+def quantize_replay_sweep(dev, hbm_gbs, reps=10):
+    """Standalone NVFP4 quantize (amax given: 2 B in, 0.5625 B out per element)
+    and TRACE replay with the mismatch count (0.5625 B record + 2 B x_train in,
+    2 B x_hat out) on [n / 4096, 4096] BF16 activations with Student-t (nu = 3)
+    channel scales.  L2 is flushed before every timed launch; sizes up to 2^24
+    elements fit in L2 nonetheless."""
+    import torch
+    from train_alignment_b200 import binding as B
+    from train_alignment_b200 import workloads as W
+    out = []
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for lg in SWEEP_LOG2:
+        n = 1 << lg
+        rows, K = n // 4096, 4096
+        gen = torch.Generator(device=dev).manual_seed(lg)
+        x = W.activations(rows, K, "student_t", 0, 1.0, gen, dev)
+        amax = B.amax_bf16(x)
+        codes = torch.empty(rows, K // 2, dtype=torch.uint8, device=dev)
+        scales = torch.empty(B.scales_bytes(rows, K, B.SCALES_LINEAR), dtype=torch.uint8, device=dev)
+        g = torch.empty(1, dtype=torch.float32, device=dev)
+        q = lambda: B.quantize_nvfp4(x, amax_in=amax, codes=codes, scales=scales, g_out=g)
+
+        def timed(fn):
+            fn()
+            ts = []
+            for _ in range(reps):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                fn()
+                e1.record()
+                e1.synchronize()
+                ts.append(e0.elapsed_time(e1))
+            return sum(ts) / len(ts)
+
+        tq = timed(q)
+        src = [B.qtensor_src(codes, scales, g, rows, K, B.SCALES_LINEAR)]
+        record = B.trace_export_qrecord(0, rows, 0, None, src)
+        x_hat = torch.empty_like(x)
+        counts = torch.zeros(2, dtype=torch.int64, device=dev)
+        status = torch.empty(1, dtype=torch.int32, device=dev)
+        r = lambda: B.trace_replay_qrecord(record, 0, 0, rows, K, x_train=x, x_hat=x_hat, counts=counts,
+                                           status=status)
+        tr = timed(r)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0 and int(counts[0].item()) == 0, "replay of the rollout's own input"
+        gq = n * (2 + 0.5625) / (tq * 1e-3) / 1e9
+        gr = n * (0.5625 + 2 + 2) / (tr * 1e-3) / 1e9
+        out.append({"elements": n, "quantize_us": tq * 1e3, "quantize_gbs": gq, "quantize_frac": gq / hbm_gbs,
+                    "replay_us": tr * 1e3, "replay_gbs": gr, "replay_frac": gr / hbm_gbs})
+        del x, codes, scales, record, x_hat
+        torch.cuda.empty_cache()
+    return out
 
 
 # ------------------------------------------------------------------- clocks
@@ -498,6 +559,10 @@ def run_ours(args):
         e2e = {"value": whole_job_tflops(fp4 + comp, world, e_ms), "unit": UNIT, "ms_per_step": e_ms,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
+    sweep = None
+    if not args.no_sweep:
+        sweep = quantize_replay_sweep(dev, peaks["hbm_gbs"])
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         sample = OracleSample(cfg, seed=0)
@@ -528,6 +593,7 @@ def run_ours(args):
         "gpu_launches": launches,
         "timing": timing_mode,
         "instrumented_ms_per_step": sum(inst_ms) / len(inst_ms),
+        "quantize_replay_sweep": sweep,
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)

@@ -6,14 +6,17 @@
 // does the bulk of the work ([QUADS-fr §2.2.B], [QUADS-es §2.2.B]):
 //   Y = g_a g_w (A_fp4 (x) W_fp4) + R_C . Wc
 //
-// Design (one persistent CTA per SM, 224 threads, warp-specialized):
+// Design (one persistent CTA per SM, 320 threads, warp-specialized):
 //   warp 0 lane 0  TMA producer: 128x256 FP4 tiles of A and W (128-byte
 //                  swizzle) and their 512-byte block-scale tiles (bulk copy)
 //                  into a multi-stage shared-memory ring; per output tile the
 //                  BF16 compensation operands R [128 x |C|] and Wc [128 x |C|]
 //                  (32-byte swizzle, 16 channels per box).
-//   warp 6 lane 0  copies each stage's block scales into a TMEM slot
-//                  (tcgen05.cp), signalling the MMA thread per slot;
+//   warps 6..9     one per TMEM lane quarter: load each stage's block scales
+//                  from shared memory and write them into a TMEM slot with
+//                  tcgen05.st (two per warp and stage), then signal the MMA
+//                  thread.  A tcgen05.cp per 512-byte tile would cost the
+//                  issuing thread more than the MMAs that read the scales.
 //   warp 1         allocates 512 TMEM columns; lane 0 issues
 //                  tcgen05.mma kind::mxf4nvf4 (block16
 //                  E4M3 scales, K = 64 per instruction) into a double-buffered
@@ -55,7 +58,7 @@ constexpr int kStageBytes = kABytes + kBBytes + 2 * kSfBytes;   // 36864
 constexpr int kCompChunkBytes = 128 * 32;           // 128 rows x 16 BF16
 constexpr int kOutChunkBytes = 32 * 64;             // 32 rows x 32 BF16 output columns
 constexpr int kOutStageBytes = 4 * 2 * kOutChunkBytes;   // 4 epilogue warps, 2 buffers each
-constexpr int kThreads = 224;                    // 7 warps
+constexpr int kThreads = 320;                    // 10 warps
 constexpr int kSfSlots = 4;                      // scale-factor buffers in TMEM
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kCompCol = 256;
@@ -184,11 +187,21 @@ __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
-// 32 rows x 16 bytes of scales from shared memory into TMEM, replicated to the
-// four 32-lane quarters.
-__device__ __forceinline__ void tc_copy_scales(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
 }
+// 16 consecutive TMEM columns of this warp's 32 lanes from registers.
+__device__ __forceinline__ void tmem_store16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void mma_fp4(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa, uint32_t sfb,
                                         uint32_t accumulate) {
   asm volatile(
@@ -229,11 +242,6 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t addr) {
 __device__ __forceinline__ uint64_t desc_kmajor_sw32(uint32_t addr) {
   return uint64_t((addr >> 4) & 0x3FFFu) | (uint64_t(1) << 16) | (uint64_t(256 >> 4) << 32) | (uint64_t(1) << 46) |
          (uint64_t(6) << 61);
-}
-// 32 rows of 16 bytes, contiguous: 8-row core matrices 128 bytes apart.
-__device__ __forceinline__ uint64_t desc_scales(uint32_t addr) {
-  return uint64_t((addr >> 4) & 0x3FFFu) | (uint64_t(128 >> 4) << 16) | (uint64_t(128 >> 4) << 32) |
-         (uint64_t(1) << 46);
 }
 
 __device__ __forceinline__ int expert_of_row(const int32_t* off_s, int E, int row) {
@@ -282,8 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t drain_bar = comp_full + 56;
   auto sf_full = [&](int i) { return comp_full + 64 + 8u * i; };            // kSfSlots barriers
   auto sf_empty = [&](int i) { return comp_full + 64 + 8u * (kSfSlots + i); };
-  const uint32_t sf_drain = comp_full + 64 + 8u * (2 * kSfSlots);
-  uint8_t* const misc = base_ptr + (sf_drain + 8 - base);
+  uint8_t* const misc = base_ptr + (comp_full + 64 + 8u * (2 * kSfSlots) + 8 - base);
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(misc);
   volatile int* const abort_flag = reinterpret_cast<volatile int*>(misc + 4);
   int32_t* const off_s = reinterpret_cast<int32_t*>(misc + 16);
@@ -304,10 +311,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(compacc_empty, 4);
     mbar_init(drain_bar, 1);
     for (int i = 0; i < kSfSlots; ++i) {
-      mbar_init(sf_full(i), 1);
+      mbar_init(sf_full(i), 4);                 // one arrival per scale warp
       mbar_init(sf_empty(i), 1);
     }
-    mbar_init(sf_drain, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -420,32 +426,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit(drain_bar);
       mbar_wait(drain_bar, 0, nullptr, kDrainTimeoutNs);
     }
-  } else if (warp == 6 && lane == 0) {
-    // ------------------------------------------------------- scale copies
-    // Copies each stage's block scales from shared memory into a TMEM slot
-    // (one tcgen05.cp per 128 rows x 4 scales) so that the MMA thread only
-    // issues MMAs; copies and MMAs then overlap.
+  } else if (warp >= 6) {
+    // ------------------------------------------------------- block scales
+    // Warps 6..9, one per TMEM lane quarter q: lane i of the quarter reads
+    // row i (16 bytes: rows i, i + 32, i + 64, i + 96 x 4 scales) of each of
+    // the stage's 512-byte scale tiles and writes them to the slot's columns
+    // (4 per 64-wide K block), the layout the block-scaled MMA reads for all
+    // 128 rows.  Two tcgen05.st per warp and stage.
     int it = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
       for (int ks = 0; ks < nks; ++ks, ++it) {
         const int s = it % S, slot = it % kSfSlots;
-        if (!mbar_wait(full_bar(s), (it / S) & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
-        if (!mbar_wait(sf_empty(slot), ((it / kSfSlots) & 1) ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+        bool w_ok = mbar_wait(full_bar(s), (it / S) & 1, abort_flag, p.timeout_ns);
+        if (w_ok) w_ok = mbar_wait(sf_empty(slot), ((it / kSfSlots) & 1) ^ 1u, abort_flag, p.timeout_ns);
+        if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
         tc_fence_after();
-        const int nkb = min(4, nkb_total - ks * 4);
-        const uint32_t st = base + s * kStageBytes;
-        const uint32_t tsfa = tmem + kSfCol + slot * 32;
-        for (int kb = 0; kb < nkb; ++kb) {
-          tc_copy_scales(tsfa + kb * 4, desc_scales(st + kABytes + kBBytes + kb * 512));
-          tc_copy_scales(tsfa + 16 + kb * 4, desc_scales(st + kABytes + kBBytes + kSfBytes + kb * 512));
+        const uint32_t sf = base + s * kStageBytes + kABytes + kBBytes + lane * 16;
+        const uint32_t tsf = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + kSfCol + slot * 32;
+        uint32_t ra[16], rb[16];
+#pragma unroll
+        for (int kb = 0; kb < 4; ++kb) {        // tiles past the stage's last K block are never read
+          const uint4 a = ld_shared_v4(sf + kb * 512);
+          const uint4 b = ld_shared_v4(sf + kSfBytes + kb * 512);
+          ra[4 * kb] = a.x; ra[4 * kb + 1] = a.y; ra[4 * kb + 2] = a.z; ra[4 * kb + 3] = a.w;
+          rb[4 * kb] = b.x; rb[4 * kb + 1] = b.y; rb[4 * kb + 2] = b.z; rb[4 * kb + 3] = b.w;
         }
-        tc_commit(sf_full(slot));
+        tmem_store16(tsf, ra);
+        tmem_store16(tsf + 16, rb);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sf_full(slot));
       }
-    }
-    if (!ok) {
-      tc_commit(sf_drain);
-      mbar_wait(sf_drain, 0, nullptr, kDrainTimeoutNs);
     }
   } else if (warp >= 2 && warp <= 5) {
     // ----------------------------------------------------------- epilogue

@@ -166,63 +166,115 @@ __global__ void __launch_bounds__(kRankThreads) rank_kernel(const int32_t* __res
 // Whole permutation in one block for small batches (<= kSmallPairs pairs):
 // histogram, padded offsets, pad rows and the in-order ranking.
 constexpr int kSmallThreads = 1024;
-constexpr int kSmallPairs = 32768;
+constexpr int kSmallWarps = kSmallThreads / 32;
+constexpr int kSmallPerLane = 32;
+constexpr int kSmallPairs = kSmallThreads * kSmallPerLane;   // 32768
 
+// The whole permutation in one CTA for up to 32768 routed pairs.  Warp w owns
+// the contiguous pairs [w P, (w + 1) P) (P a multiple of 32), held in
+// registers (the expert of pair w P + 32 j + lane as 16 bits), read from
+// global memory once:
+//   1. per-warp expert histogram: one shared-memory add per distinct expert
+//      among the 32 lanes (__match_any_sync), warp-synchronous;
+//   2. per expert, the exclusive prefix over warps (one thread per expert),
+//      and the 128-padded expert offsets (a warp-shuffle scan);
+//   3. stable ranks: pair i of expert e goes to offset(e) + #(earlier pairs
+//      of e in earlier warps) + #(earlier pairs of e in this warp).
+// Padding rows of every expert segment get src_of = -1.
 __global__ void __launch_bounds__(kSmallThreads) permute_small_kernel(const int32_t* __restrict__ idx,
                                                                       int n_pairs, int k, int E,
                                                                       int32_t* __restrict__ expert_off,
                                                                       int32_t* __restrict__ row_of,
                                                                       int32_t* __restrict__ src_of) {
-  constexpr int kWarps = kSmallThreads / 32;
-  __shared__ int32_t cnt[kMaxE];
-  __shared__ int32_t running[kMaxE];
-  __shared__ int32_t padded[kMaxE];
-  __shared__ int32_t wcnt[kWarps * kMaxE];             // [warp][expert], stride E
+  __shared__ int32_t wbase[kSmallWarps * kMaxE];        // [warp][expert]: count, then first row
+  __shared__ int32_t cnt_s[kMaxE];
+  __shared__ int32_t off_s[kMaxE + 1];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  for (int i = threadIdx.x; i < E; i += blockDim.x) cnt[i] = 0;
+  const int per_warp = ((n_pairs + kSmallWarps - 1) / kSmallWarps + 31) & ~31;
+  const int J = per_warp / 32;                          // <= kSmallPerLane
+  const int w0 = wid * per_warp;
+  // expert of pair j of this lane as 16 bits (-1: no pair / out of range), two per register
+  uint32_t vp[kSmallPerLane / 2];
+#pragma unroll
+  for (int j = 0; j < kSmallPerLane; j += 2) {
+    int e2[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int i = w0 + (j + u) * 32 + lane;
+      const int e = (j + u < J && i < n_pairs) ? __ldg(idx + i) : -1;
+      e2[u] = (e >= 0 && e < E) ? e : -1;
+    }
+    vp[j / 2] = (static_cast<uint32_t>(e2[0]) & 0xFFFFu) | (static_cast<uint32_t>(e2[1]) << 16);
+  }
+  auto v_of = [&](int j) { return static_cast<int>(static_cast<int16_t>(vp[j >> 1] >> (16 * (j & 1)))); };
+  for (int i = threadIdx.x; i < kSmallWarps * E; i += blockDim.x) wbase[i] = 0;
   __syncthreads();
-  // warp-aggregated histogram: one shared atomic per distinct expert in a warp
-  for (int i0 = 0; i0 < n_pairs; i0 += blockDim.x) {
-    const int i = i0 + threadIdx.x;
-    const int e = (i < n_pairs) ? idx[i] : -1;
-    const unsigned int peers = __match_any_sync(0xffffffffu, e);
-    if (e >= 0 && e < E && lane == __ffs(peers) - 1) atomicAdd(&cnt[e], __popc(peers));
+  // 1. per-warp histogram
+#pragma unroll
+  for (int j = 0; j < kSmallPerLane; ++j) {
+    if (j < J) {                                        // warp-uniform
+      const int e = v_of(j);
+      const unsigned int peers = __match_any_sync(0xffffffffu, e);
+      if (e >= 0 && lane == __ffs(peers) - 1) wbase[wid * E + e] += __popc(peers);
+      __syncwarp();
+    }
   }
   __syncthreads();
-  if (threadIdx.x < E) padded[threadIdx.x] = (cnt[threadIdx.x] + 127) / 128 * 128;
-  __syncthreads();
+  // 2a. per expert: exclusive prefix over warps, total count
   if (threadIdx.x < E) {
     const int e = threadIdx.x;
-    int off = 0;
-    for (int j = 0; j < e; ++j) off += padded[j];
-    expert_off[e] = off;
-    running[e] = off;
-    for (int r = off + cnt[e]; r < off + padded[e]; ++r) src_of[r] = -1;
-    if (e == E - 1) expert_off[E] = off + padded[e];
+    int run = 0;
+    for (int w = 0; w < kSmallWarps; ++w) {
+      const int c = wbase[w * E + e];
+      wbase[w * E + e] = run;
+      run += c;
+    }
+    cnt_s[e] = run;
   }
-  for (int r0 = 0; r0 < n_pairs; r0 += kSmallThreads) {
-    for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) wcnt[i] = 0;
-    __syncthreads();
-    const int i = r0 + threadIdx.x;
-    const bool valid = i < n_pairs;
-    const int e = valid ? idx[i] : -1;
-    const unsigned int peers = __match_any_sync(0xffffffffu, e);
-    const int rank_w = __popc(peers & ((1u << lane) - 1u));
-    if (valid && lane == __ffs(peers) - 1 && e >= 0 && e < E) wcnt[wid * E + e] = __popc(peers);
-    __syncthreads();
-    if (valid && e >= 0 && e < E) {
-      int pos = running[e] + rank_w;
-      for (int w = 0; w < wid; ++w) pos += wcnt[w * E + e];
-      row_of[i] = pos;
-      src_of[pos] = i / k;
+  __syncthreads();
+  // 2b. expert offsets: exclusive scan of the 128-padded counts (8 experts per lane)
+  if (wid == 0) {
+    int loc[8], sum = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int e = lane * 8 + q;
+      loc[q] = sum;
+      sum += (e < E) ? (cnt_s[e] + 127) / 128 * 128 : 0;
     }
-    __syncthreads();
-    for (int x = threadIdx.x; x < E; x += blockDim.x) {
-      int add = 0;
-      for (int w = 0; w < kWarps; ++w) add += wcnt[w * E + x];
-      running[x] += add;
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
     }
-    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      if (lane * 8 + q < E) off_s[lane * 8 + q] = incl - sum + loc[q];
+    if (lane == 31) off_s[E] = incl;
+  }
+  __syncthreads();
+  const int total_rows = off_s[E];
+  for (int i = threadIdx.x; i <= E; i += blockDim.x) expert_off[i] = off_s[i];
+  for (int r = threadIdx.x; r < total_rows; r += blockDim.x) src_of[r] = -1;   // overwritten below for real rows
+  for (int i = threadIdx.x; i < kSmallWarps * E; i += blockDim.x) wbase[i] += off_s[i % E];
+  __syncthreads();                                      // also orders the -1 fill before the row writes
+  // 3. stable ranks
+  const unsigned int lt = (1u << lane) - 1u;
+#pragma unroll
+  for (int j = 0; j < kSmallPerLane; ++j) {
+    if (j < J) {                                        // warp-uniform
+      const int e = v_of(j);
+      const unsigned int peers = __match_any_sync(0xffffffffu, e);
+      if (e >= 0) {
+        const int i = w0 + j * 32 + lane;
+        const int pos = wbase[wid * E + e] + __popc(peers & lt);
+        row_of[i] = pos;
+        src_of[pos] = i / k;
+      }
+      __syncwarp();
+      if (e >= 0 && lane == __ffs(peers) - 1) wbase[wid * E + e] += __popc(peers);
+      __syncwarp();
+    }
   }
 }
 

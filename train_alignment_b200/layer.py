@@ -15,7 +15,6 @@ into the master gradient, the export of the rollout's quantization record
 and its replay against the trainer's activation.
 """
 import math
-from dataclasses import dataclass
 
 import torch
 
@@ -23,28 +22,43 @@ from . import binding as B
 from .workloads import MoEConfig
 
 
-@dataclass
 class StageTimer:
-    """Optional CUDA-event marks between stages (on the current stream).
-    external=True records them as external event nodes, which is how timing
-    events are captured into a CUDA graph and re-recorded at every replay."""
-    enabled: bool = False
-    external: bool = False
+    """Optional CUDA-event marks between stages, one chain per stream: mark()
+    records on the current stream, and a stage's duration is the time between
+    its mark and the previous mark of the same stream.  external=True records
+    them as external event nodes, which is how timing events are captured into
+    a CUDA graph and re-recorded at every replay.  Marks named "start", or
+    starting with "wait" or "join", end no kernel stage."""
 
-    def __post_init__(self):
-        self.marks = []
+    def __init__(self, enabled=False, external=False):
+        self.enabled = enabled
+        self.external = external
+        self.chains = {}
 
     def mark(self, name):
         if self.enabled:
+            s = torch.cuda.current_stream()
             ev = torch.cuda.Event(enable_timing=True, external=self.external)
-            ev.record()
-            self.marks.append((name, ev))
+            ev.record(s)
+            self.chains.setdefault(s.cuda_stream, []).append((name, ev))
+
+    @property
+    def marks(self):
+        """The chain of the first stream marked (the step's own stream)."""
+        return next(iter(self.chains.values())) if self.chains else []
 
     def durations_ms(self):
         out = {}
-        for (_, e0), (name, e1) in zip(self.marks, self.marks[1:]):
-            out[name] = out.get(name, 0.0) + e0.elapsed_time(e1)
+        for chain in self.chains.values():
+            for (_, e0), (name, e1) in zip(chain, chain[1:]):
+                if not is_stage(name):
+                    continue
+                out[name] = out.get(name, 0.0) + e0.elapsed_time(e1)
         return out
+
+
+def is_stage(name):
+    return name != "start" and not name.startswith("wait") and not name.startswith("join")
 
 
 class MoELayer:
@@ -56,20 +70,22 @@ class MoELayer:
         T, H, E, k, F = cfg.T, cfg.H, cfg.E, cfg.k, cfg.F
         dev = torch.device(device)
         self.dev = dev
-        # trainer master weights, both matrices in one allocation (gate/up
-        # [E, 2F, H] then down [E, H, F]) so that one amax pass covers both
+        # trainer master weights, both matrices in one allocation so that one
+        # amax pass covers both: down [E, H, F] first, then gate/up [E, 2F, H].
+        # The amax pass reads gate/up last, so much of it is still in L2 when
+        # the gate/up fake-quant reads it again right after.
         n_gu, n_d = E * 2 * F * H, E * H * F
         self.n_gu, self.n_d = n_gu, n_d
-        self.w_all = torch.empty(n_gu + n_d, dtype=torch.bfloat16, device=dev)
-        self.w_all[:n_gu].copy_(w_gu.reshape(-1))
-        self.w_all[n_gu:].copy_(w_d.reshape(-1))
-        self.w_gu = self.w_all[:n_gu].view(E, 2 * F, H)
-        self.w_d = self.w_all[n_gu:].view(E, H, F)
+        self.w_all = torch.empty(n_d + n_gu, dtype=torch.bfloat16, device=dev)
+        self.w_all[:n_d].copy_(w_d.reshape(-1))
+        self.w_all[n_d:].copy_(w_gu.reshape(-1))
+        self.w_d = self.w_all[:n_d].view(E, H, F)
+        self.w_gu = self.w_all[n_d:].view(E, 2 * F, H)
         # rows of a common width for the joint amax: each expert matrix is a group
         kw = math.gcd(H, F)
         self.amax_k = kw if kw % 16 == 0 else 0
         if self.amax_k:
-            offs = [e * 2 * F * H // kw for e in range(E)] + [(n_gu + e * H * F) // kw for e in range(E + 1)]
+            offs = [e * H * F // kw for e in range(E)] + [(n_d + e * 2 * F * H) // kw for e in range(E + 1)]
             self.w_groups = torch.tensor(offs, dtype=torch.int32, device=dev)
         # SwiGLU in the gate/up GEMM's epilogue (rollout gate/up weights kept
         # in the 64-row interleaved gate/up order), else a separate pass
@@ -99,12 +115,12 @@ class MoELayer:
         self.w_gu_scales = e((B.scales_bytes(E * 2 * F, H, B.SCALES_TILED),), u8)
         self.w_d_scales = e((B.scales_bytes(E * H, F, B.SCALES_TILED),), u8)
         self.g_w_gu, self.g_w_d = e((E,), f32), e((E,), f32)
-        self.amax_w_all, self.amax_x = e((2 * E,), f32), e((1,), f32)
-        self.amax_w_gu, self.amax_w_d = self.amax_w_all[:E], self.amax_w_all[E:]
+        self.amax_w_all, self.amax_x = e((2 * E,), f32), e((1,), f32)   # down experts, then gate/up
+        self.amax_w_d, self.amax_w_gu = self.amax_w_all[:E], self.amax_w_all[E:]
         self.wc_gu, self.wc_d = e((E, 2 * F, self.nc_x), bf), e((E, H, self.nc_h), bf)
         self.ws_w = e((B.quantize_workspace_bytes(E),), u8)
         # STE gradients (master gradient accumulated in place)
-        self.grad_all = torch.zeros_like(self.w_all)
+        self.grad_all = torch.zeros(n_gu + n_d, dtype=torch.bfloat16, device=dev)   # gate/up, then down
         self.grad_gu, self.grad_d = self.grad_all[:n_gu].view(E, 2 * F, H), self.grad_all[n_gu:].view(E, H, F)
         # rollout activations
         self.x_codes, self.x_scales = vx["codes"].view(T, H // 2), vx["scales"]
@@ -134,26 +150,36 @@ class MoELayer:
         self.x_hat, self.h_hat = e((T, H), bf), e((cap, F), bf)
         self.counts, self.status = torch.zeros(2, dtype=torch.int64, device=dev), e((1,), i32)
         self.status_h = e((1,), i32)
+        # the weight side of a step runs on its own stream (see step())
+        self.side = torch.cuda.Stream(device=dev)
+        self.ev_w_gu, self.ev_w_d = torch.cuda.Event(), torch.cuda.Event()
 
     # ---------------------------------------------------------------- stages
 
     def weight_sync(self, timer=None):
         """Trainer fake-quant + the rollout's NVFP4 weights: one amax pass over
         both weight tensors, then one quantize pass per weight tensor."""
-        cfg = self.cfg
         t = timer or StageTimer(False)
-        E, F, H = cfg.E, cfg.F, cfg.H
+        self._amax_w(t)
+        self._fakequant_gate_up(t)
+        self._fakequant_down(t)
+
+    def _amax_w(self, t):
+        E, F, H = self.cfg.E, self.cfg.F, self.cfg.H
         if self.amax_k:
             B.amax_bf16(self.w_all.view(-1, self.amax_k), self.w_groups, 2 * E, out=self.amax_w_all)
-            t.mark("amax_w")
         else:
             B.amax_bf16(self.w_gu.view(E * 2 * F, H), n_groups=E, out=self.amax_w_gu)
             B.amax_bf16(self.w_d.view(E * H, F), n_groups=E, out=self.amax_w_d)
-            t.mark("amax_w")
+        t.mark("amax_w")
+
+    def _fakequant_gate_up(self, t):
         B.fakequant_weight_ste(self.w_gu, True, self.chan_x, False, True, self.w_gu_fq, self.w_gu_codes,
                                self.w_gu_scales, self.g_w_gu, self.wc_gu, None, self.amax_w_gu,
                                gate_up=self.fuse_swiglu)
         t.mark("fakequant_w_gate_up")
+
+    def _fakequant_down(self, t):
         B.fakequant_weight_ste(self.w_d, True, self.chan_h, False, True, self.w_d_fq, self.w_d_codes,
                                self.w_d_scales, self.g_w_d, self.wc_d, None, self.amax_w_d)
         t.mark("fakequant_w_down")
@@ -174,14 +200,21 @@ class MoELayer:
     def grad_fq_buffers(self):
         """(flat, gate/up view, down view): one allocation for the gradients
         with respect to both fake-quantized weights."""
-        flat = torch.empty_like(self.w_all)
+        flat = torch.empty_like(self.grad_all)
         E, F, H = self.cfg.E, self.cfg.F, self.cfg.H
         return flat, flat[:self.n_gu].view(E, 2 * F, H), flat[self.n_gu:].view(E, H, F)
 
     def rollout_forward(self, x, logits, timer=None):
-        cfg = self.cfg
-        T, H, E, k, F = cfg.T, cfg.H, cfg.E, cfg.k, cfg.F
+        """The rollout side of the layer on the current stream (the weights
+        must be synced)."""
         t = timer or StageTimer(False)
+        self._rollout_front(x, logits, t)
+        self._rollout_gate_up(t)
+        return self._rollout_down(t)
+
+    def _rollout_front(self, x, logits, t):
+        cfg = self.cfg
+        T, H, E, k = cfg.T, cfg.H, cfg.E, cfg.k
         B.amax_bf16(x, out=self.amax_x)
         t.mark("amax_x")
         B.quantize_nvfp4(x, amax_in=self.amax_x, scale_layout=B.SCALES_LINEAR, chan=self.chan_x,
@@ -194,6 +227,10 @@ class MoELayer:
         B.moe_gather(self.src_of, self.expert_off, E, self.cap, self.x_codes, self.x_scales, H, self.x_resid,
                      self.pa_codes, self.pa_scales, self.pa_resid)
         t.mark("gather")
+
+    def _rollout_gate_up(self, t):
+        cfg = self.cfg
+        H, E, F = cfg.H, cfg.E, cfg.F
         if self.fuse_swiglu:
             B.moe_grouped_gemm_nvfp4_swiglu(self.pa_codes, self.pa_scales, self.g_x, self.w_gu_codes,
                                             self.w_gu_scales, self.g_w_gu, self.expert_off, E, self.cap, F, H,
@@ -206,6 +243,10 @@ class MoELayer:
             t.mark("gemm_gate_up")
             B.swiglu(self.y_gu, F, self.expert_off, E, h=self.h, amax=self.amax_h)
             t.mark("swiglu")
+
+    def _rollout_down(self, t):
+        cfg = self.cfg
+        T, H, E, k, F = cfg.T, cfg.H, cfg.E, cfg.k, cfg.F
         B.quantize_nvfp4(self.h, group_off=self.expert_off, n_groups=E, amax_in=self.amax_h,
                          scale_layout=B.SCALES_TILED, chan=self.chan_h, codes=self.h_codes, scales=self.h_scales,
                          g_out=self.g_h, resid_out=self.h_resid)
@@ -231,16 +272,39 @@ class MoELayer:
         t.mark("replay_h")
 
     def step(self, x, logits, x_train, grad_gu_fq, grad_d_fq, timer=None, layer_id=0):
-        """One pass of the whole path over one batch.  The replay's mismatch
-        counters accumulate across steps (zero them with reset_counts())."""
+        """One pass of the whole path over one batch, on two streams: the
+        weight side (amax, fake-quant of gate/up then down, STE backward) on
+        a side stream, the rollout forward, export and replay on the calling
+        stream.  Each GEMM waits only for its own weights, and the call
+        returns with the calling stream joined to the side stream.  The
+        replay's mismatch counters accumulate across steps (zero them with
+        reset_counts())."""
+        cfg = self.cfg
+        T, H, E, k, F = cfg.T, cfg.H, cfg.E, cfg.k, cfg.F
         t = timer or StageTimer(False)
+        main = torch.cuda.current_stream()
         t.mark("start")
-        self.weight_sync(t)
-        out = self.rollout_forward(x, logits, t)
+        self.side.wait_stream(main)
+        with torch.cuda.stream(self.side):
+            t.mark("start")
+            self._amax_w(t)
+            self._fakequant_gate_up(t)
+            self.ev_w_gu.record(self.side)
+            self._fakequant_down(t)
+            self.ev_w_d.record(self.side)
+            self.ste_backward(grad_gu_fq, grad_d_fq, t)
+        self._rollout_front(x, logits, t)
+        main.wait_event(self.ev_w_gu)
+        t.mark("wait_w_gate_up")
+        self._rollout_gate_up(t)
+        main.wait_event(self.ev_w_d)
+        t.mark("wait_w_down")
+        out = self._rollout_down(t)
         self.export(layer_id)
         t.mark("export")
         self.trainer_replay(x_train, layer_id, t)
-        self.ste_backward(grad_gu_fq, grad_d_fq, t)
+        main.wait_stream(self.side)
+        t.mark("join")
         return out
 
     def reset_counts(self):
