@@ -744,8 +744,10 @@ int quads_device_status(quads_stream_t stream) {
     unsigned int zero = 0;
     if (cudaMemcpyToSymbol(g_wait_status, &zero, sizeof(zero)) != cudaSuccess)
       return set_error(QUADS_ERR_CUDA, "cannot clear the device status word");
-    return set_error(QUADS_ERR_TIMEOUT, "a device-side wait timed out");
   }
+  const int q = take_quantize_wait_status();
+  if (q < 0) return set_error(QUADS_ERR_CUDA, "cannot read the quantizer's status word");
+  if (v || q) return set_error(QUADS_ERR_TIMEOUT, "a device-side wait timed out");
   return QUADS_OK;
 }
 
