@@ -54,6 +54,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sweep", action="store_true", help="skip the standalone quantize/replay size sweep")
+    ap.add_argument("--serial", action="store_true", help="run the step on one stream (no weight-side overlap)")
     return ap.parse_args()
 
 
@@ -408,7 +409,7 @@ def run_ours(args):
     B.load()
     cfg = W.CONFIGS[args.workload]
     inp = W.moe_layer_inputs(cfg, seed=rank, device=dev)
-    layer = L.build_layer(cfg, inp, dev)
+    layer = L.build_layer(cfg, inp, dev, overlap=not args.serial)
     x, logits = inp["x"], inp["logits"]
     x_train = W.engine_drift(x, 1e-2, seed=rank, device=dev)
     g_all, g_gu, g_d = layer.grad_fq_buffers()          # both weight gradients in one allocation
@@ -582,6 +583,7 @@ def run_ours(args):
         "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "k": cfg.k, "F": cfg.F,
                    "n_chan": cfg.n_chan, "n_chan_f": cfg.n_chan_f, "rows_padded": rpad,
                    "parallelism": f"dp{world} (replicas, no collective)",
+                   "schedule": "one stream" if args.serial else "two streams (weight side overlapped)",
                    "l2": "flushed between steps (256 MiB memset outside the timed events)",
                    "gemm_flops_per_step": fp4 + comp},
         "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,

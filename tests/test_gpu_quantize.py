@@ -137,6 +137,21 @@ def test_quantize_every_block_scale(cuda_lib, n_groups):
     _check_quant(cuda_lib, x, 1, group_off=off)
 
 
+def test_amax_strided_rows(cuda_lib):
+    """Rows with a stride above K take the row kernel; contiguous rows the
+    flat one: both give the exact max |x| per group."""
+    x = _x(300, 256 + 64, 15)
+    full = bf16_torch(x)
+    view = full[:, :256]                      # row stride 320 elements
+    off = [0, 7, 7, 300]
+    t_off = torch.tensor(off, dtype=torch.int32, device="cuda")
+    got_s = f32_of(cuda_lib.amax_bf16(view, t_off, 3))
+    got_c = f32_of(cuda_lib.amax_bf16(view.contiguous(), t_off, 3))
+    want = [np.max(np.abs(x[0:7, :256])), 0.0, np.max(np.abs(x[7:300, :256]))]
+    assert_bits_equal(got_s, np.array(want), "amax strided")
+    assert_bits_equal(got_c, np.array(want), "amax contiguous")
+
+
 def test_amax_groups(cuda_lib):
     x = _x(500, 128, 10)
     off = [0, 100, 100, 500]

@@ -181,11 +181,17 @@ def quantize_workspace_bytes(n_groups):
     return int(load().quads_quantize_workspace_bytes(n_groups))
 
 
+def _rows_view(x, name):
+    """A BF16 matrix whose rows may be strided (row stride = ld elements)."""
+    if not x.is_cuda or x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError(f"{name} must be a CUDA bfloat16 matrix with unit column stride")
+    return x.shape[0], x.shape[1], x.stride(0)
+
+
 def amax_bf16(x, group_off=None, n_groups=1, out=None):
-    _dev(x, torch.bfloat16, "x")
-    rows, K = x.shape
+    rows, K, ld = _rows_view(x, "x")
     out = out if out is not None else _empty((n_groups,), torch.float32, x.device)
-    _check(load().quads_amax_bf16(_p(x), rows, K, K, _p(group_off), n_groups, _p(out), _s()), "quads_amax_bf16")
+    _check(load().quads_amax_bf16(_p(x), rows, K, ld, _p(group_off), n_groups, _p(out), _s()), "quads_amax_bf16")
     return out
 
 

@@ -21,9 +21,6 @@ int num_sms();
 
 // Returns QUADS_ERR_CUDA (with a message) if the last launch failed.
 int check_launch(const char* what);
-// Reads and clears the timeout flag of the staged quantize kernels (quantize.cu):
-// 1 if a bounded wait there gave up since the last call, 0 if not, -1 on a CUDA error.
-int take_quantize_wait_status();
 
 #define QUADS_REQUIRE(cond, code, ...)                 \
   do {                                                 \
@@ -62,49 +59,6 @@ __device__ __forceinline__ uint32_t fast_div(uint32_t n, const FastDiv& f) { ret
 
 // ---------------------------------------------------------------- device side
 
-// Asynchronous bulk copies global -> shared with mbarrier completion (used to
-// stage rows of HBM-bound kernels without holding them in registers).
-__device__ __forceinline__ uint64_t gtimer_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-__device__ __forceinline__ void mb_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mb_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ bool mb_test(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Waits for the phase with the given parity for at most limit_ns; false on expiry.
-__device__ __forceinline__ bool mb_wait_bounded(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
-  if (mb_test(bar, parity)) return true;
-  const uint64_t t0 = gtimer_ns();
-  while (!mb_test(bar, parity))
-    if (gtimer_ns() - t0 > limit_ns) return false;
-  return true;
-}
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-               "l"(src), "r"(bytes), "r"(bar)
-               : "memory");
-}
-__device__ __forceinline__ void fence_proxy_async_cta() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
 
 constexpr float kNvfp4Range = 2688.0f;   // 6 * 448
 

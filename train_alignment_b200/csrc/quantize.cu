@@ -91,6 +91,57 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t* __restri
     if (amax_s[i]) atomicMax(&out_bits[i], amax_s[i] << 16);
 }
 
+// Contiguous rows (ld == K): the groups are contiguous ranges of 16-byte
+// vectors, swept with a grid-stride loop that keeps eight 16-byte loads per
+// thread in flight; one warp reduction and one atomic per warp and group.
+constexpr int kAmaxUnroll = 8;
+
+__global__ void __launch_bounds__(kThreads) amax_flat_kernel(const uint4* __restrict__ x, int64_t rows,
+                                                             int64_t vec_per_row, const int32_t* group_off,
+                                                             int n_groups, int64_t uniform_rows,
+                                                             unsigned int* __restrict__ out_bits) {
+  extern __shared__ int32_t off_a[];                       // n_groups + 1 (explicit groups)
+  if (group_off != nullptr)
+    for (int i = threadIdx.x; i <= n_groups; i += blockDim.x) off_a[i] = group_off[i];
+  __syncthreads();
+  const int64_t nth = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (int g = 0; g < n_groups; ++g) {                     // uniform across the grid
+    // as in amax_kernel, the last group runs to the last row; offsets are
+    // clamped to [0, rows] so that no read leaves the matrix
+    const int64_t r0 = min(max(group_off ? static_cast<int64_t>(off_a[g]) : g * uniform_rows, int64_t(0)), rows);
+    const int64_t r1 = g == n_groups - 1
+                           ? rows
+                           : min(max(group_off ? static_cast<int64_t>(off_a[g + 1]) : (g + 1) * uniform_rows,
+                                     int64_t(0)),
+                                 rows);
+    const int64_t v1 = r1 * vec_per_row;
+    uint32_t m = 0u;
+    int64_t v = r0 * vec_per_row + tid;
+    for (; v + (kAmaxUnroll - 1) * nth < v1; v += kAmaxUnroll * nth) {
+      uint4 r[kAmaxUnroll];
+#pragma unroll
+      for (int u = 0; u < kAmaxUnroll; ++u) r[u] = __ldg(x + v + u * nth);
+#pragma unroll
+      for (int u = 0; u < kAmaxUnroll; ++u) {
+        m = __vmaxu2(m, r[u].x & 0x7FFF7FFFu);
+        m = __vmaxu2(m, r[u].y & 0x7FFF7FFFu);
+        m = __vmaxu2(m, r[u].z & 0x7FFF7FFFu);
+        m = __vmaxu2(m, r[u].w & 0x7FFF7FFFu);
+      }
+    }
+    for (; v < v1; v += nth) {
+      const uint4 r = __ldg(x + v);
+      m = __vmaxu2(m, r.x & 0x7FFF7FFFu);
+      m = __vmaxu2(m, r.y & 0x7FFF7FFFu);
+      m = __vmaxu2(m, r.z & 0x7FFF7FFFu);
+      m = __vmaxu2(m, r.w & 0x7FFF7FFFu);
+    }
+    const unsigned int wm = __reduce_max_sync(0xffffffffu, max(m & 0xFFFFu, m >> 16));
+    if ((threadIdx.x & 31) == 0 && wm) atomicMax(&out_bits[g], wm << 16);
+  }
+}
+
 // ----------------------------------------------------------------- quantize
 
 struct QuantArgs {
@@ -116,47 +167,24 @@ struct QuantArgs {
   FastDiv uniform_div;     // filled by launch_quantize: rows per group (uniform groups)
 };
 
-// Rows are staged through shared memory by asynchronous bulk copies: each
-// warp owns a ring of kRing pass buffers (one pass = 512 elements, 1 KB of
-// BF16 = 32 blocks of 16), refilled kRing passes ahead by lane 0, so the
-// warp's loads stay in flight while it computes and no registers hold them.
-constexpr int kRing = 4;
-constexpr int kPassElems = 512;
-constexpr int kPassBytes = kPassElems * 2;
-constexpr int kWarpsPerBlock = kThreads / 32;
-constexpr size_t kRingBytes = static_cast<size_t>(kWarpsPerBlock) * kRing * (kPassBytes + 8);
-constexpr uint64_t kStageWaitNs = 4000000000ull;     // a bulk copy that has not landed in 4 s is a fault
-constexpr uint64_t kStageDrainNs = 500000000ull;
-
-__device__ unsigned int g_q_wait_status = 0u;
-
-// One warp per row, lanes along K (lane l owns block 32 p + l of pass p).
-// The residual channels of a pass are extracted cooperatively: lane j takes
-// channel slot j, reads its element from the staged pass and fetches the
-// element's code and block scale from the lane that owns the block by warp
-// shuffles; the warp then writes the row's residual slots contiguously.
+// One warp per row, lanes along K (32 blocks of 16 elements per pass, two
+// passes in flight).  The residual channels of a pass are extracted
+// cooperatively: lane j takes channel slot j and fetches its element, code and
+// scale from the lane that owns the block by warp shuffles, then the warp
+// writes the row's residual slots as one contiguous store.
 __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a) {
-  extern __shared__ __align__(128) uint8_t smem_qr[];
+  extern __shared__ int32_t smem_q[];
   const int n = a.n_groups;
   const int nkb = static_cast<int>(a.K / 16);
   const int npass = (nkb + 31) / 32;
   const bool use_tab = n <= kTabGroups;
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  uint8_t* const ring_p = smem_qr + static_cast<size_t>(wid) * kRing * kPassBytes;
-  const uint32_t ring = smem_u32(ring_p);
-  const uint32_t bars = smem_u32(smem_qr) + kWarpsPerBlock * kRing * kPassBytes + wid * kRing * 8;
-  uint8_t* const after = smem_qr + kRingBytes;
-  float2* tab = reinterpret_cast<float2*>(after);          // n x 128 {S, 1/S} (few groups)
-  int32_t* smem = reinterpret_cast<int32_t*>(after + (use_tab ? static_cast<size_t>(n) * 128 * sizeof(float2) : 0));
+  float2* tab = reinterpret_cast<float2*>(smem_q);         // n x 128 {S, 1/S} (few groups)
+  int32_t* smem = smem_q + (use_tab ? n * 128 * 2 : 0);
   int32_t* off_s = smem;                                   // n + 1
   float* g_s = reinterpret_cast<float*>(smem + n + 1);     // n
   int32_t* pass_slot = smem + 2 * n + 1;                   // npass + 1 (with channels)
   int32_t* chan_s = pass_slot + npass + 1;                 // n_chan
   __shared__ int n_valid_s;
-  if (lane == 0) {
-    for (int i = 0; i < kRing; ++i) mb_init(bars + 8 * i, 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
   for (int i = threadIdx.x; i <= n; i += blockDim.x) {
     if (a.group_off != nullptr) off_s[i] = a.group_off[i];
     if (i < n) {
@@ -177,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a) {
       int cnt = 0;
       for (int j = 0; j < a.n_chan; ++j) {
         const int c = chan_s[j];
-        cnt += (c >= 0 && c < a.K && c < kPassElems * p) ? 1 : 0;
+        cnt += (c >= 0 && c < a.K && c < 512 * p) ? 1 : 0;
       }
       pass_slot[p] = cnt;
     }
@@ -195,117 +223,97 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a) {
   const int nkb_e = tiled ? (nkb + 3) / 4 * 4 : nkb;
   const int64_t ncol_tiles = nkb_e / 4;
   const int n_valid = a.n_chan ? n_valid_s : 0;
-  const int64_t warps = static_cast<int64_t>(gridDim.x) * kWarpsPerBlock;
-  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kWarpsPerBlock + wid;
-  // padding rows of the last tiled band hold no data: zero scales
-  for (int64_t row = rows_valid + row0; row < rows_e; row += warps)
-    if (a.scales)
-      for (int kb = lane; kb < nkb_e; kb += 32) a.scales[tiled_scale_offset(row, kb, ncol_tiles)] = 0;
-  // this warp's rows row0 + r * warps (r < nr), npass staged items each
-  const int64_t nr = row0 < rows_valid ? (rows_valid - row0 + warps - 1) / warps : 0;
-  const int n_items = static_cast<int>(nr * npass);    // < 2^31: rows < 2^31 over >= 4736 warps
-  // lane 0's issue cursor: the next staged item's row and pass
-  int64_t irow = row0;
-  int ipass = 0;
-  auto issue_next = [&](int slot) {
-    const int e0 = ipass * kPassElems;
-    const uint32_t bytes = static_cast<uint32_t>(min(kPassElems, static_cast<int>(a.K) - e0)) * 2u;
-    mb_expect_tx(bars + 8 * slot, bytes);
-    bulk_g2s(ring + slot * kPassBytes, a.x + irow * a.ld + e0, bytes, bars + 8 * slot);
-    if (++ipass == npass) {
-      ipass = 0;
-      irow += warps;
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows_e;
+       row += warps) {
+    if (row >= rows_valid) {                           // padding rows of the last tiled band
+      if (a.scales)
+        for (int kb = lane; kb < nkb_e; kb += 32) a.scales[tiled_scale_offset(row, kb, ncol_tiles)] = 0;
+      continue;
     }
-  };
-  if (lane == 0)
-    for (int it = 0; it < n_items && it < kRing; ++it) issue_next(it);
-  int gi = 0;
-  float g = 0.0f;
-  QConsts qc = make_qconsts(0.0f);
-  int64_t drow = 0;
-  int64_t row = row0;
-  int p = 0;
-  for (int it = 0; it < n_items; ++it) {
-    const int slot = it % kRing;
-    if (p == 0) {
-      gi = grp.of(row);
-      g = g_s[gi];
-      qc = make_qconsts(g, use_tab ? tab + gi * 128 : nullptr);
-      drow = row;                                      // row of the codes, scales and resid outputs
-      if (a.ilv_half) {
-        const int64_t base = static_cast<int64_t>(gi) * 2 * a.ilv_half, loc = row - base;
-        const bool second = loc >= a.ilv_half;
-        const int64_t f = second ? loc - a.ilv_half : loc;
-        drow = base + (f >> 6) * 128 + (second ? 64 : 0) + (f & 63);
+    const int gi = grp.of(row);
+    const float g = g_s[gi];
+    const QConsts qc = make_qconsts(g, use_tab ? tab + gi * 128 : nullptr);
+    const uint16_t* xr = a.x + row * a.ld;
+    int64_t drow = row;                                // row of the codes, scales and resid outputs
+    if (a.ilv_half) {
+      const int64_t base = static_cast<int64_t>(gi) * 2 * a.ilv_half, loc = row - base;
+      const bool second = loc >= a.ilv_half;
+      const int64_t f = second ? loc - a.ilv_half : loc;
+      drow = base + (f >> 6) * 128 + (second ? 64 : 0) + (f & 63);
+    }
+    for (int p0 = 0; p0 < npass; p0 += 2) {
+      uint32_t w[2][8];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int kb = (p0 + u) * 32 + lane;
+        if (kb < nkb) load_bf16x16(xr + kb * 16, w[u]);
       }
-    }
-    const bool landed = mb_wait_bounded(bars + 8 * slot, static_cast<uint32_t>((it / kRing) & 1), kStageWaitNs);
-    if (!__all_sync(0xffffffffu, landed)) {
-      // record the timeout, let the copies this warp issued land, give up
-      if (lane == 0) {
-        atomicOr(&g_q_wait_status, 1u);
-        for (int j = it; j < n_items && j < it + kRing; ++j)
-          mb_wait_bounded(bars + 8 * (j % kRing), static_cast<uint32_t>((j / kRing) & 1), kStageDrainNs);
-      }
-      return;
-    }
-    const uint8_t* const buf = ring_p + slot * kPassBytes;
-    const int kb = p * 32 + lane;
-    QCore q{0u, 0u, 0u, 0.0f};
-    if (kb < nkb) {
-      const uint4 lo4 = *reinterpret_cast<const uint4*>(buf + lane * 32);
-      const uint4 hi4 = *reinterpret_cast<const uint4*>(buf + lane * 32 + 16);
-      const uint32_t w[8] = {lo4.x, lo4.y, lo4.z, lo4.w, hi4.x, hi4.y, hi4.z, hi4.w};
-      q = quant_core(w, qc);
-      if (a.codes) *reinterpret_cast<uint2*>(a.codes + drow * (a.K / 2) + kb * 8) = make_uint2(q.lo, q.hi);
-      if (a.w_fq) {
-        uint32_t o[8];
-        deq_block_bf16(q, g, a.fold, o);
-        uint4* dst = reinterpret_cast<uint4*>(a.w_fq + row * a.K + kb * 16);
-        dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-        dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
-      }
-    }
-    if (a.scales && kb < nkb_e)
-      a.scales[tiled ? tiled_scale_offset(drow, kb, ncol_tiles) : drow * nkb + kb] = static_cast<uint8_t>(q.scale);
-    if (a.resid) {
-      const int slo = pass_slot[p], shi = pass_slot[p + 1];
-      for (int j0 = slo; j0 < shi; j0 += 32) {         // warp-uniform
-        const int j = j0 + lane;
-        const bool act = j < shi;
-        const int c = act ? chan_s[j] : kPassElems * p;
-        const int src = (c - kPassElems * p) >> 4, bit = c & 15;
-        const uint32_t cl = __shfl_sync(0xffffffffu, q.lo, src);
-        const uint32_t ch = __shfl_sync(0xffffffffu, q.hi, src);
-        const float sv = __shfl_sync(0xffffffffu, q.sv, src);
-        const float xv = bf16_bits_to_float(reinterpret_cast<const uint16_t*>(buf)[c - kPassElems * p]);
-        const uint32_t code = (((bit < 8) ? cl : ch) >> (4 * (bit & 7))) & 15u;
-        float v;
-        if (a.resid_mode == 2) {
-          v = xv;
-        } else {
-          const float dq = deq_f32(code, sv, g);
-          v = (a.resid_mode == 1) ? dq : __fsub_rn(xv, dq);
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int p = p0 + u;
+        if (p >= npass) break;                         // warp-uniform
+        const int kb = p * 32 + lane;
+        QCore q{0u, 0u, 0u, 0.0f};
+        if (kb < nkb) {
+          q = quant_core(w[u], qc);
+          if (a.codes)
+            *reinterpret_cast<uint2*>(a.codes + drow * (a.K / 2) + kb * 8) = make_uint2(q.lo, q.hi);
+          if (a.w_fq) {
+            uint32_t o[8];
+            deq_block_bf16(q, g, a.fold, o);
+            uint4* dst = reinterpret_cast<uint4*>(a.w_fq + row * a.K + kb * 16);
+            dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+            dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+          }
         }
-        if (act) a.resid[drow * a.n_chan + j] = static_cast<uint16_t>(float_to_bf16_bits(v));
+        if (a.scales && kb < nkb_e)
+          a.scales[tiled ? tiled_scale_offset(drow, kb, ncol_tiles) : drow * nkb + kb] =
+              static_cast<uint8_t>(q.scale);
+        if (a.resid) {
+          // Channel slot j of this pass is taken by lane j % 32.  The element
+          // itself is read back through L2 (the input row, or, for bf16(deq)
+          // with the scale folded, the W_fq row this warp has just written);
+          // its code and block scale come from the owning lane by shuffles.
+          const int slo = pass_slot[p], shi = pass_slot[p + 1];
+          const bool from_fq = a.resid_mode == 1 && a.fold && a.w_fq != nullptr;
+          if (from_fq) __syncwarp();                     // this warp's W_fq stores are visible to it
+          for (int j0 = slo; j0 < shi; j0 += 32) {       // warp-uniform
+            const int j = j0 + lane;
+            const bool act = j < shi;
+            const int c = act ? chan_s[j] : 512 * p;
+            const int src = (c - 512 * p) >> 4, bit = c & 15;
+            uint32_t vb;
+            if (from_fq) {
+              vb = act ? a.w_fq[row * a.K + c] : 0u;
+            } else {
+              const uint32_t cl = __shfl_sync(0xffffffffu, q.lo, src);
+              const uint32_t ch = __shfl_sync(0xffffffffu, q.hi, src);
+              const float sv = __shfl_sync(0xffffffffu, q.sv, src);
+              const float xv = act ? bf16_bits_to_float(__ldg(xr + c)) : 0.0f;
+              const uint32_t code = (((bit < 8) ? cl : ch) >> (4 * (bit & 7))) & 15u;
+              float v;
+              if (a.resid_mode == 2) {
+                v = xv;
+              } else {
+                const float dq = deq_f32(code, sv, g);
+                v = (a.resid_mode == 1) ? dq : __fsub_rn(xv, dq);
+              }
+              vb = float_to_bf16_bits(v);
+            }
+            if (act) a.resid[drow * a.n_chan + j] = static_cast<uint16_t>(vb);
+          }
+        }
       }
-      if (p == npass - 1)
-        for (int j = n_valid + lane; j < a.n_chan; j += 32) a.resid[drow * a.n_chan + j] = 0;
     }
-    __syncwarp();                                      // every lane is done with the slot
-    if (lane == 0 && it + kRing < n_items) {
-      fence_proxy_async_cta();
-      issue_next(slot);
-    }
-    if (++p == npass) {
-      p = 0;
-      row += warps;
-    }
+    if (a.resid)
+      for (int j = n_valid + lane; j < a.n_chan; j += 32) a.resid[drow * a.n_chan + j] = 0;
   }
 }
 
 size_t quantize_smem(int n_groups, int64_t K, int n_chan) {
-  size_t s = kRingBytes + (2 * static_cast<size_t>(n_groups) + 1) * 4;
+  size_t s = (2 * static_cast<size_t>(n_groups) + 1) * 4;
   if (n_groups <= kTabGroups) s += static_cast<size_t>(n_groups) * 128 * sizeof(float2);
   if (n_chan) s += (static_cast<size_t>((K / 16 + 31) / 32) + 1 + n_chan) * 4;
   return s;
@@ -441,24 +449,48 @@ __global__ void __launch_bounds__(1024) select_kernel(const float* __restrict__ 
 
 // ------------------------------------------------------------ STE backward
 
-__global__ void ste_backward_kernel(const uint16_t* __restrict__ gfq, uint16_t* __restrict__ gw, int64_t n,
-                                    int accumulate) {
-  const int64_t nv = n / 8;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nv;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    uint4 a = __ldg(reinterpret_cast<const uint4*>(gfq) + i);
-    if (accumulate) {
-      uint4 b = reinterpret_cast<const uint4*>(gw)[i];
-      uint32_t* pa = reinterpret_cast<uint32_t*>(&a);
-      const uint32_t* pb = reinterpret_cast<const uint32_t*>(&b);
+// Few CTAs (two per SM), each thread with kSteUnroll 16-byte vectors of both
+// inputs in flight per iteration: enough bytes in flight to stream at HBM
+// speed while leaving the SMs' registers and warp slots to kernels that run
+// beside it on other streams.
+constexpr int kSteUnroll = 4;
+
+__device__ __forceinline__ uint4 ste_add(uint4 a, uint4 b) {
+  uint32_t* pa = reinterpret_cast<uint32_t*>(&a);
+  const uint32_t* pb = reinterpret_cast<const uint32_t*>(&b);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        float lo = __fadd_rn(bf16_bits_to_float(pa[j] & 0xFFFFu), bf16_bits_to_float(pb[j] & 0xFFFFu));
-        float hi = __fadd_rn(bf16_bits_to_float(pa[j] >> 16), bf16_bits_to_float(pb[j] >> 16));
-        pa[j] = pack_bf16x2(lo, hi);
-      }
+  for (int j = 0; j < 4; ++j) {
+    const float lo = __fadd_rn(bf16_bits_to_float(pa[j] & 0xFFFFu), bf16_bits_to_float(pb[j] & 0xFFFFu));
+    const float hi = __fadd_rn(bf16_bits_to_float(pa[j] >> 16), bf16_bits_to_float(pb[j] >> 16));
+    pa[j] = pack_bf16x2(lo, hi);
+  }
+  return a;
+}
+
+__global__ void __launch_bounds__(kThreads) ste_backward_kernel(const uint16_t* __restrict__ gfq,
+                                                                uint16_t* __restrict__ gw, int64_t n, int accumulate) {
+  const int64_t nv = n / 8;
+  const int64_t nth = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const uint4* src = reinterpret_cast<const uint4*>(gfq);
+  uint4* dst = reinterpret_cast<uint4*>(gw);
+  int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (; i + (kSteUnroll - 1) * nth < nv; i += kSteUnroll * nth) {
+    uint4 a[kSteUnroll], b[kSteUnroll];
+#pragma unroll
+    for (int u = 0; u < kSteUnroll; ++u) a[u] = __ldg(src + i + u * nth);
+    if (accumulate) {
+#pragma unroll
+      for (int u = 0; u < kSteUnroll; ++u) b[u] = dst[i + u * nth];
+#pragma unroll
+      for (int u = 0; u < kSteUnroll; ++u) a[u] = ste_add(a[u], b[u]);
     }
-    reinterpret_cast<uint4*>(gw)[i] = a;
+#pragma unroll
+    for (int u = 0; u < kSteUnroll; ++u) dst[i + u * nth] = a[u];
+  }
+  for (; i < nv; i += nth) {
+    uint4 a = __ldg(src + i);
+    if (accumulate) a = ste_add(a, dst[i]);
+    dst[i] = a;
   }
   // tail (n % 8 elements) handled by the first thread
   if (blockIdx.x == 0 && threadIdx.x == 0) {
@@ -505,6 +537,18 @@ int launch_amax(const uint16_t* x, int64_t rows, int64_t K, int64_t ld, const in
   if (rows == 0) return QUADS_OK;
   QUADS_REQUIRE(rows < kMaxBlocks, QUADS_ERR_UNSUPPORTED_SHAPE, "too many rows");
   const uint32_t uniform = group_off ? 1u : static_cast<uint32_t>(rows / n_groups);
+  if (ld == K) {
+    const size_t smem_f = (static_cast<size_t>(n_groups) + 1) * 4;
+    const int64_t nvec = rows * (K / 8);
+    // two CTAs per SM keep 64 KB per SM in flight and leave room beside them
+    const int64_t want = ceil_div(nvec, static_cast<int64_t>(kThreads) * kAmaxUnroll);
+    const int grid_f = static_cast<int>(want < 2 * num_sms() ? (want < 1 ? 1 : want) : 2 * num_sms());
+    amax_flat_kernel<<<grid_f, kThreads, smem_f, s>>>(reinterpret_cast<const uint4*>(x), rows, K / 8, group_off,
+                                                      n_groups, rows / n_groups,
+                                                      reinterpret_cast<unsigned int*>(amax_out));
+    count_launches(1);
+    return check_launch("amax_flat_kernel");
+  }
   size_t smem = (2 * static_cast<size_t>(n_groups) + 1) * 4;
   const int grid = persistent_grid(reinterpret_cast<const void*>(amax_kernel), kThreads, smem, ceil_div(rows, 16));
   amax_kernel<<<grid, kThreads, smem, s>>>(x, rows, K, ld, group_off, n_groups,
@@ -532,16 +576,6 @@ int launch_quantize(QuantArgs a, cudaStream_t s) {
 }
 
 }  // namespace
-
-int take_quantize_wait_status() {
-  unsigned int v = 0;
-  if (cudaMemcpyFromSymbol(&v, g_q_wait_status, sizeof(v)) != cudaSuccess) return -1;
-  if (v == 0) return 0;
-  const unsigned int zero = 0;
-  if (cudaMemcpyToSymbol(g_q_wait_status, &zero, sizeof(zero)) != cudaSuccess) return -1;
-  return 1;
-}
-
 }  // namespace quads
 
 using namespace quads;
@@ -743,7 +777,9 @@ int quads_fakequant_weight_ste_backward(const uint16_t* grad_wfq, uint16_t* grad
   if (n == 0) return QUADS_OK;
   QUADS_REQUIRE(grad_wfq && grad_w && aligned(grad_wfq, 16) && aligned(grad_w, 16), QUADS_ERR_INVALID_ARG,
                 "gradients must be non-null and 16-byte aligned");
-  ste_backward_kernel<<<grid_for(ceil_div(n, 8)), kThreads, 0, stream>>>(grad_wfq, grad_w, n, accumulate);
+  const int64_t want = ceil_div(ceil_div(n, 8), static_cast<int64_t>(kThreads) * kSteUnroll);
+  const int grid = static_cast<int>(want < 2 * num_sms() ? (want < 1 ? 1 : want) : 2 * num_sms());
+  ste_backward_kernel<<<grid, kThreads, 0, stream>>>(grad_wfq, grad_w, n, accumulate);
   count_launches(1);
   return check_launch("ste_backward_kernel");
 }

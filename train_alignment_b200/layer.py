@@ -65,7 +65,7 @@ class MoELayer:
     """Weights, calibrated channel sets and every buffer of one layer at a
     fixed token count; step() runs the whole path without allocating."""
 
-    def __init__(self, cfg: MoEConfig, w_gu, w_d, chan_x, chan_h, device="cuda", fuse_swiglu=None):
+    def __init__(self, cfg: MoEConfig, w_gu, w_d, chan_x, chan_h, device="cuda", fuse_swiglu=None, overlap=True):
         self.cfg = cfg
         T, H, E, k, F = cfg.T, cfg.H, cfg.E, cfg.k, cfg.F
         dev = torch.device(device)
@@ -90,6 +90,8 @@ class MoELayer:
         # SwiGLU in the gate/up GEMM's epilogue (rollout gate/up weights kept
         # in the 64-row interleaved gate/up order), else a separate pass
         self.fuse_swiglu = (F % 64 == 0) if fuse_swiglu is None else bool(fuse_swiglu)
+        # the weight side of a step on its own stream (False: one stream)
+        self.overlap = bool(overlap)
         self.nc_x = int(chan_x.numel())
         self.nc_h = int(chan_h.numel())
         cap = B.moe_rows_capacity(T, k, E)
@@ -284,6 +286,18 @@ class MoELayer:
         t = timer or StageTimer(False)
         main = torch.cuda.current_stream()
         t.mark("start")
+        if not self.overlap:
+            self._amax_w(t)
+            self._fakequant_gate_up(t)
+            self._fakequant_down(t)
+            self._rollout_front(x, logits, t)
+            self._rollout_gate_up(t)
+            out = self._rollout_down(t)
+            self.export(layer_id)
+            t.mark("export")
+            self.trainer_replay(x_train, layer_id, t)
+            self.ste_backward(grad_gu_fq, grad_d_fq, t)
+            return out
         self.side.wait_stream(main)
         with torch.cuda.stream(self.side):
             t.mark("start")
@@ -334,7 +348,7 @@ def calibrate_channels(x, n_sel):
     return out
 
 
-def build_layer(cfg: MoEConfig, inputs, device="cuda"):
+def build_layer(cfg: MoEConfig, inputs, device="cuda", overlap=True):
     """Layer from generated inputs: channel sets calibrated on the layer's own
     batch (X for the gate/up input, the uncompensated h for the down input)."""
     x, logits = inputs["x"], inputs["logits"]
@@ -347,4 +361,4 @@ def build_layer(cfg: MoEConfig, inputs, device="cuda"):
     n_rows = int(probe.expert_off[-1].item())
     chan_h = calibrate_channels(probe.h[:n_rows].contiguous(), cfg.n_chan_f)
     del probe
-    return MoELayer(cfg, inputs["w_gu"], inputs["w_d"], chan_x, chan_h, device)
+    return MoELayer(cfg, inputs["w_gu"], inputs["w_d"], chan_x, chan_h, device, overlap=overlap)
