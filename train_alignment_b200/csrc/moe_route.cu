@@ -167,8 +167,7 @@ __global__ void __launch_bounds__(kRankThreads) rank_kernel(const int32_t* __res
 // histogram, padded offsets, pad rows and the in-order ranking.
 constexpr int kSmallThreads = 1024;
 constexpr int kSmallWarps = kSmallThreads / 32;
-constexpr int kSmallPerLane = 32;
-constexpr int kSmallPairs = kSmallThreads * kSmallPerLane;   // 32768
+constexpr int kSmallPairs = kSmallThreads * 32;   // 32768: up to 32 pairs per lane
 
 // The whole permutation in one CTA for up to 32768 routed pairs.  Warp w owns
 // the contiguous pairs [w P, (w + 1) P) (P a multiple of 32), held in
@@ -181,6 +180,9 @@ constexpr int kSmallPairs = kSmallThreads * kSmallPerLane;   // 32768
 //   3. stable ranks: pair i of expert e goes to offset(e) + #(earlier pairs
 //      of e in earlier warps) + #(earlier pairs of e in this warp).
 // Padding rows of every expert segment get src_of = -1.
+// kPerLane: pairs per lane (4 or 32; the small variant keeps the unrolled
+// loops short enough to stay in the instruction cache).
+template <int kPerLane>
 __global__ void __launch_bounds__(kSmallThreads) permute_small_kernel(const int32_t* __restrict__ idx,
                                                                       int n_pairs, int k, int E,
                                                                       int32_t* __restrict__ expert_off,
@@ -191,12 +193,12 @@ __global__ void __launch_bounds__(kSmallThreads) permute_small_kernel(const int3
   __shared__ int32_t off_s[kMaxE + 1];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int per_warp = ((n_pairs + kSmallWarps - 1) / kSmallWarps + 31) & ~31;
-  const int J = per_warp / 32;                          // <= kSmallPerLane
+  const int J = per_warp / 32;                          // <= kPerLane
   const int w0 = wid * per_warp;
   // expert of pair j of this lane as 16 bits (-1: no pair / out of range), two per register
-  uint32_t vp[kSmallPerLane / 2];
+  uint32_t vp[kPerLane / 2];
 #pragma unroll
-  for (int j = 0; j < kSmallPerLane; j += 2) {
+  for (int j = 0; j < kPerLane; j += 2) {
     int e2[2];
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
@@ -211,7 +213,7 @@ __global__ void __launch_bounds__(kSmallThreads) permute_small_kernel(const int3
   __syncthreads();
   // 1. per-warp histogram
 #pragma unroll
-  for (int j = 0; j < kSmallPerLane; ++j) {
+  for (int j = 0; j < kPerLane; ++j) {
     if (j < J) {                                        // warp-uniform
       const int e = v_of(j);
       const unsigned int peers = __match_any_sync(0xffffffffu, e);
@@ -261,7 +263,7 @@ __global__ void __launch_bounds__(kSmallThreads) permute_small_kernel(const int3
   // 3. stable ranks
   const unsigned int lt = (1u << lane) - 1u;
 #pragma unroll
-  for (int j = 0; j < kSmallPerLane; ++j) {
+  for (int j = 0; j < kPerLane; ++j) {
     if (j < J) {                                        // warp-uniform
       const int e = v_of(j);
       const unsigned int peers = __match_any_sync(0xffffffffu, e);
@@ -464,8 +466,12 @@ int quads_moe_permute(const int32_t* topk_idx, int64_t T, int k, int E, int32_t*
                 "workspace of %zu bytes required", quads_moe_permute_workspace_bytes(T, k, E));
   const int64_t n_pairs = T * k;
   if (n_pairs <= kSmallPairs) {
-    permute_small_kernel<<<1, kSmallThreads, 0, stream>>>(topk_idx, static_cast<int>(n_pairs), k, E, expert_off,
-                                                          row_of, src_of);
+    if (n_pairs <= kSmallThreads * 4)
+      permute_small_kernel<4><<<1, kSmallThreads, 0, stream>>>(topk_idx, static_cast<int>(n_pairs), k, E,
+                                                               expert_off, row_of, src_of);
+    else
+      permute_small_kernel<32><<<1, kSmallThreads, 0, stream>>>(topk_idx, static_cast<int>(n_pairs), k, E,
+                                                                expert_off, row_of, src_of);
     count_launches(1);
     return check_launch("permute_small_kernel");
   }
