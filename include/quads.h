@@ -395,6 +395,21 @@ int trace_replay_qrecord(const void* record, size_t record_bytes, int layer_id, 
                          uint16_t* x_hat, unsigned long long* counts, int32_t* status,
                          quads_stream_t stream);
 
+/* ------------------------------------------------------ layer stacking
+ * The pages describe the MoE layer, not the model around it; a stack of
+ * layers is joined here in the plainest way: x_{l+1} = x_l + MoE_l(x_l), and
+ * the router logits of layer l are x_l . W_r[l].
+ *
+ * Router logits: logits[t][e] = sum over h of x[t][h] * w_r[h][e], one FP32
+ * FMA chain per output in increasing h.  x: device BF16 [T][H]; w_r: device
+ * FP32 [H][E] (row-major); logits: device FP32 [T][E].  1 <= E <= 4096. */
+int quads_router_logits(const uint16_t* x, int64_t T, int64_t H, const float* w_r, int E,
+                        float* logits, quads_stream_t stream);
+/* Residual connection: out[i] = bf16(fp32(x[i]) + fp32(y[i])) for n BF16
+ * elements (n % 8 == 0, all three 16-byte aligned; out may alias x or y). */
+int quads_residual_add(const uint16_t* x, const uint16_t* y, int64_t n, uint16_t* out,
+                       quads_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -31,6 +31,8 @@ Modules:
   moe      -- router top-k, permutation, grouped GEMM + compensation,
               SwiGLU, combine, one MoE layer
   trace    -- rollout record export and trainer replay
+  layer    -- one MoE layer on both sides, composed from the steps above
+  stack    -- router projection and residual connection between layers
 
 Pins: every function here is checked in ``tests/test_oracle_*.py`` against
 brute force, closed forms, library routines or invariants.  Functions with

@@ -13,6 +13,7 @@ import torch
 from oracle import formats as F
 from oracle import moe as M
 from oracle import nvfp4 as Q
+from oracle import stack as ST
 from oracle import trace as TR
 
 RNG = np.random.default_rng(12345)
@@ -493,6 +494,43 @@ def pin_replay_counts_drift():
     assert cm >= 1
     c2, s2 = Q.quantize_with_scale(x2, g)
     assert cm == int(np.count_nonzero(c2 != c)) and sm == int(np.count_nonzero(s2 != s))
+
+
+# ------------------------------------------------------------------ stack
+
+
+def pin_router_logits_selects_rows():
+    """One-hot inputs select rows of W_r; a sum of one-hot rows sums them."""
+    H, E = 24, 7
+    w = RNG.standard_normal((H, E))
+    eye = np.eye(H)
+    got, absdot = ST.router_logits(eye, w)
+    assert np.array_equal(got, w) and np.array_equal(absdot, np.abs(w))
+    two = np.zeros((1, H))
+    two[0, [2, 5]] = [1.0, -2.0]
+    got, _ = ST.router_logits(two, w)
+    assert np.array_equal(got[0], w[2] - 2.0 * w[5])
+
+
+def pin_router_logits_matches_torch():
+    """Against torch's float64 matmul on random inputs."""
+    x = RNG.standard_normal((13, 40))
+    w = RNG.standard_normal((40, 9))
+    got, _ = ST.router_logits(x, w)
+    ref = (torch.from_numpy(x) @ torch.from_numpy(w)).numpy()
+    assert np.allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def pin_residual_add_against_torch_rounding():
+    """bf16(fp32(x + y)) against torch's FP32 add and BF16 cast, including
+    sums that fall on BF16 midpoints and cancellations."""
+    x = F.bf16_rne(RNG.standard_normal(4000).astype(np.float32) * 8)
+    y = F.bf16_rne(RNG.standard_normal(4000).astype(np.float32) / 64)
+    y[:100] = -x[:100]                                   # exact cancellation
+    y[100:200] = x[100:200] * 2.0 ** -8                  # midpoint-sized increments
+    got = ST.residual_add(x, y)
+    ref = (torch.from_numpy(x.astype(np.float32)) + torch.from_numpy(y.astype(np.float32))).to(torch.bfloat16)
+    assert np.array_equal(got, ref.to(torch.float64).numpy())
 
 
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -91,6 +91,8 @@ _SIGS = {
     "quads_fakequant_weight_ste_gate_up": (c_i32, [c_vp, c_i64, c_i64, c_i64, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp,
                                                    c_vp, c_i32, c_i32, c_vp, c_vp, c_sz, c_vp]),
     "quads_fakequant_weight_ste_backward": (c_i32, [c_vp, c_vp, c_i64, c_i32, c_vp]),
+    "quads_router_logits": (c_i32, [c_vp, c_i64, c_i64, c_vp, c_i32, c_vp, c_vp]),
+    "quads_residual_add": (c_i32, [c_vp, c_vp, c_i64, c_vp, c_vp]),
     "trace_qrecord_layout": (c_sz, [c_i32, c_i64, c_i32, c_vp, c_i32, c_vp]),
     "trace_export_qrecord": (c_i32, [c_i32, c_i64, c_i32, c_vp, c_vp, c_i32, c_vp, c_sz, c_vp]),
     "trace_replay_qrecord": (c_i32, [c_vp, c_sz, c_i32, c_i32, c_i64, c_i64, c_vp, c_vp, c_vp, c_vp, c_vp]),
@@ -456,3 +458,26 @@ def trace_replay_qrecord(record, layer_id, which, rows, K, x_train=None, x_hat=N
     _check(load().trace_replay_qrecord(_p(record), record.numel(), layer_id, which, rows, K, _p(x_train),
                                        _p(x_hat), _p(counts), _p(status), _s()), "trace_replay_qrecord")
     return x_hat, counts, status
+
+
+# ------------------------------------------------------------ layer stacking
+
+
+def router_logits(x, w_r, out=None):
+    """logits [T, E] f32 = x [T, H] bf16 . w_r [H, E] f32."""
+    _dev(x, torch.bfloat16, "x")
+    _dev(w_r, torch.float32, "w_r")
+    T, H = x.shape
+    E = w_r.shape[1]
+    out = out if out is not None else _empty((T, E), torch.float32, x.device)
+    _check(load().quads_router_logits(_p(x), T, H, _p(w_r), E, _p(out), _s()), "quads_router_logits")
+    return out
+
+
+def residual_add(x, y, out=None):
+    """out = bf16(x + y), elementwise (out may be x)."""
+    _dev(x, torch.bfloat16, "x")
+    _dev(y, torch.bfloat16, "y")
+    out = out if out is not None else torch.empty_like(x)
+    _check(load().quads_residual_add(_p(x), _p(y), x.numel(), _p(out), _s()), "quads_residual_add")
+    return out

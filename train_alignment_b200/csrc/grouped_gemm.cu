@@ -55,7 +55,6 @@ constexpr int kABytes = BM * kStageRowBytes;        // 16384
 constexpr int kBBytes = BN * kStageRowBytes;        // 16384
 constexpr int kSfBytes = 4 * 512;                   // scales of 4 MMAs for 128 rows
 constexpr int kStageBytes = kABytes + kBBytes + 2 * kSfBytes;   // 36864
-constexpr int kBStageBytes = kBBytes + kSfBytes;                // 18432: a stage of W only (A resident)
 constexpr int kCompChunkBytes = 128 * 32;           // 128 rows x 16 BF16
 constexpr int kOutChunkBytes = 32 * 64;             // 32 rows x 32 BF16 output columns
 constexpr int kOutStageBytes = 4 * 2 * kOutChunkBytes;   // 4 epilogue warps, 2 buffers each
@@ -273,12 +272,7 @@ __device__ __forceinline__ float epi_value(uint32_t acc, float G, bool has_comp,
 // kSwiglu: the W rows of every 128-row tile are 64 gate rows then the 64
 // matching up rows; the epilogue writes h = silu(y_gate) * y_up (64 columns
 // per tile) instead of y, and the per-expert max |h|.
-// kAStat (A-stationary): every CTA takes a contiguous run of tiles in
-// (row block, column block) order, so consecutive tiles mostly share their
-// 128-row block of A.  That block's codes, scales and compensation rows are
-// loaded once into a resident region and reused across the run; the stages
-// stream W tiles and their scales only.
-template <bool kSwiglu, bool kAStat>
+template <bool kSwiglu>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                         const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_wc,
@@ -289,13 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* const base_ptr = smem_raw + (base - raw);
   const int S = p.stages;
   const int nch = p.n_chan / 16;
-  const int nkb_total = p.K / 64;                 // MMAs along K
-  const int nks = (nkb_total + 3) / 4;            // pipeline stages along K
-  const int n_col_tiles = nkb_total;              // 512-byte scale tiles per 128-row band
-  const uint32_t stage_bytes = kAStat ? kBStageBytes : kStageBytes;
-  const uint32_t a_res = base + S * stage_bytes;                    // resident A (kAStat), 1024-byte aligned
-  const uint32_t sfa_res = a_res + (kAStat ? nks * kABytes : 0);    // its scale tiles
-  const uint32_t comp_r = sfa_res + (kAStat ? nks * 4 * 512 : 0);
+  const uint32_t comp_r = base + S * kStageBytes;
   const uint32_t comp_wc = comp_r + nch * kCompChunkBytes;
   const uint32_t out_stage = comp_wc + nch * kCompChunkBytes;     // 1024-byte aligned
   const uint32_t bar0 = out_stage + kOutStageBytes;                 // 8-byte aligned
@@ -310,9 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t drain_bar = comp_full + 56;
   auto sf_full = [&](int i) { return comp_full + 64 + 8u * i; };            // kSfSlots barriers
   auto sf_empty = [&](int i) { return comp_full + 64 + 8u * (kSfSlots + i); };
-  const uint32_t a_full = comp_full + 64 + 8u * (2 * kSfSlots) + 8;   // resident A loaded (kAStat)
-  const uint32_t a_empty = a_full + 8;                                // resident A no longer read
-  uint8_t* const misc = base_ptr + (a_empty + 8 - base);
+  uint8_t* const misc = base_ptr + (comp_full + 64 + 8u * (2 * kSfSlots) + 8 - base);
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(misc);
   volatile int* const abort_flag = reinterpret_cast<volatile int*>(misc + 4);
   int32_t* const off_s = reinterpret_cast<int32_t*>(misc + 16);
@@ -336,8 +322,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(sf_full(i), 4);                 // one arrival per scale warp
       mbar_init(sf_empty(i), 1);
     }
-    mbar_init(a_full, 1);
-    mbar_init(a_empty, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -356,65 +340,40 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int n_ntiles = p.N / BN;
   const int total = (off_s[p.E] / BM) * n_ntiles;
-  // this CTA's tiles: [t_begin, t_end) with stride t_step
-  int t_begin = blockIdx.x, t_end = total, t_step = gridDim.x;
-  if constexpr (kAStat) {
-    const int q = total / static_cast<int>(gridDim.x), r = total % static_cast<int>(gridDim.x);
-    const int b = blockIdx.x;
-    t_begin = b * q + min(b, r);
-    t_end = t_begin + q + (b < r ? 1 : 0);
-    t_step = 1;
-  }
-  // row block of the tile after t in this CTA's order (-1 past the end)
-  auto next_mt = [&](int t) { return t + t_step < t_end ? (t + t_step) / n_ntiles : -1; };
+  const int nkb_total = p.K / 64;                 // MMAs along K
+  const int nks = (nkb_total + 3) / 4;            // pipeline stages along K
+  const int n_col_tiles = nkb_total;              // 512-byte scale tiles per 128-row band
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ producer
-    int it = 0, cur_mt = -1;
-    uint32_t cph = 0, a_loads = 0;
+    int it = 0;
+    uint32_t cph = 0;
     bool ok = true;
-    for (int t = t_begin; t < t_end && ok; t += t_step) {
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
       const int mt = t / n_ntiles, nt = t - mt * n_ntiles;
       const int m0 = mt * BM;
       const int e = expert_of_row(off_s, p.E, m0);
       const int brow = e * p.N + nt * BN;
-      if constexpr (kAStat) {
-        if (mt != cur_mt) {
-          // wait until the MMAs of the previous row block are done with the region
-          if (a_loads > 0 && !mbar_wait(a_empty, (a_loads - 1) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
-          mbar_expect_tx(a_full, nks * kABytes + nkb_total * 512 + nch * kCompChunkBytes);
-          for (int ks = 0; ks < nks; ++ks) tma_load_2d(a_res + ks * kABytes, &tm_a, ks * kStageRowBytes, m0, a_full);
-          bulk_load(sfa_res, p.a_scales + static_cast<int64_t>(mt) * n_col_tiles * 512, nkb_total * 512, a_full);
-          for (int j = 0; j < nch; ++j) tma_load_2d(comp_r + j * kCompChunkBytes, &tm_r, j * 16, m0, a_full);
-          cur_mt = mt;
-          ++a_loads;
-        }
-      }
       for (int ks = 0; ks < nks; ++ks, ++it) {
         const int s = it % S;
         const uint32_t ph = (it / S) & 1;
         if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
         const int nkb = min(4, nkb_total - ks * 4);
-        const uint32_t st = base + s * stage_bytes;
-        const int64_t sfb = (static_cast<int64_t>(brow / BM) * n_col_tiles + ks * 4) * 512;
-        if constexpr (kAStat) {
-          mbar_expect_tx(full_bar(s), kBBytes + nkb * 512);
-          tma_load_2d(st, &tm_b, ks * kStageRowBytes, brow, full_bar(s));
-          bulk_load(st + kBBytes, p.w_scales + sfb, nkb * 512, full_bar(s));
-        } else {
-          mbar_expect_tx(full_bar(s), kABytes + kBBytes + 2 * nkb * 512);
-          tma_load_2d(st, &tm_a, ks * kStageRowBytes, m0, full_bar(s));
-          tma_load_2d(st + kABytes, &tm_b, ks * kStageRowBytes, brow, full_bar(s));
-          bulk_load(st + kABytes + kBBytes, p.a_scales + (static_cast<int64_t>(mt) * n_col_tiles + ks * 4) * 512,
-                    nkb * 512, full_bar(s));
-          bulk_load(st + kABytes + kBBytes + kSfBytes, p.w_scales + sfb, nkb * 512, full_bar(s));
-        }
+        const uint32_t st = base + s * kStageBytes;
+        mbar_expect_tx(full_bar(s), kABytes + kBBytes + 2 * nkb * 512);
+        tma_load_2d(st, &tm_a, ks * kStageRowBytes, m0, full_bar(s));
+        tma_load_2d(st + kABytes, &tm_b, ks * kStageRowBytes, brow, full_bar(s));
+        bulk_load(st + kABytes + kBBytes, p.a_scales + (static_cast<int64_t>(mt) * n_col_tiles + ks * 4) * 512,
+                  nkb * 512, full_bar(s));
+        bulk_load(st + kABytes + kBBytes + kSfBytes,
+                  p.w_scales + (static_cast<int64_t>(brow / BM) * n_col_tiles + ks * 4) * 512, nkb * 512,
+                  full_bar(s));
       }
       if (ok && nch) {
         if (!mbar_wait(comp_empty, cph ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
-        mbar_expect_tx(comp_full, (kAStat ? 1 : 2) * nch * kCompChunkBytes);
+        mbar_expect_tx(comp_full, 2 * nch * kCompChunkBytes);
         for (int j = 0; j < nch; ++j) {
-          if constexpr (!kAStat) tma_load_2d(comp_r + j * kCompChunkBytes, &tm_r, j * 16, m0, comp_full);
+          tma_load_2d(comp_r + j * kCompChunkBytes, &tm_r, j * 16, m0, comp_full);
           tma_load_2d(comp_wc + j * kCompChunkBytes, &tm_wc, j * 16, brow, comp_full);
         }
         cph ^= 1u;
@@ -425,25 +384,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = (it > S ? it - S : 0); i < it; ++i)
         mbar_wait(full_bar(i % S), (i / S) & 1, nullptr, kDrainTimeoutNs);
       if (nch) mbar_wait(comp_full, cph ^ 1u, nullptr, kDrainTimeoutNs);
-      if (kAStat && a_loads > 0) mbar_wait(a_full, (a_loads - 1) & 1u, nullptr, kDrainTimeoutNs);
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------------------------------------------------------- MMA
-    int it = 0, tc = 0, cur_mt = -1;
-    uint32_t cph = 0, caph = 0, a_uses = 0;
+    int it = 0, tc = 0;
+    uint32_t cph = 0, caph = 0;
     bool ok = true;
-    for (int t = t_begin; t < t_end && ok; t += t_step, ++tc) {
-      const int mt = t / n_ntiles;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++tc) {
       const int buf = tc & 1;
       const uint32_t aph = (tc >> 1) & 1;
       if (!mbar_wait(acc_empty0 + 8 * buf, aph ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
-      if constexpr (kAStat) {
-        if (mt != cur_mt) {
-          if (!mbar_wait(a_full, a_uses & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
-          ++a_uses;
-          cur_mt = mt;
-        }
-      }
       tc_fence_after();
       const uint32_t dacc = tmem + buf * BN;
       for (int ks = 0; ks < nks; ++ks, ++it) {
@@ -454,13 +404,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(sf_full(slot), (it / kSfSlots) & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
         tc_fence_after();
         const int nkb = min(4, nkb_total - ks * 4);
-        const uint32_t st = base + s * stage_bytes;
-        const uint32_t a_src = kAStat ? a_res + ks * kABytes : st;
-        const uint32_t b_src = kAStat ? st : st + kABytes;
+        const uint32_t st = base + s * kStageBytes;
         const uint32_t tsfa = tmem + kSfCol + slot * 32;
         const uint32_t tsfb = tsfa + 16;
         for (int kb = 0; kb < nkb; ++kb) {
-          mma_fp4(dacc, desc_kmajor_sw128(a_src + kb * kMmaKBytes), desc_kmajor_sw128(b_src + kb * kMmaKBytes),
+          mma_fp4(dacc, desc_kmajor_sw128(st + kb * kMmaKBytes), desc_kmajor_sw128(st + kABytes + kb * kMmaKBytes),
                   kIdescFp4, tsfa + kb * 4, tsfb + kb * 4, (ks | kb) != 0 ? 1u : 0u);
         }
         tc_commit(empty_bar(s));
@@ -480,7 +428,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_commit(comp_empty);
       }
       tc_commit(acc_full0 + 8 * buf);
-      if (kAStat && next_mt(t) != mt) tc_commit(a_empty);   // the resident block is free once these MMAs finish
     }
     if (!ok) {
       // wait for every MMA and scale copy already issued before TMEM is freed
@@ -494,34 +441,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the stage's 512-byte scale tiles and writes them to the slot's columns
     // (4 per 64-wide K block), the layout the block-scaled MMA reads for all
     // 128 rows.  Two tcgen05.st per warp and stage.
-    int it = 0, cur_mt = -1;
-    uint32_t a_uses = 0;
+    int it = 0;
     bool ok = true;
-    for (int t = t_begin; t < t_end && ok; t += t_step) {
-      const int mt = t / n_ntiles;
-      if constexpr (kAStat) {
-        if (mt != cur_mt) {
-          if (!__all_sync(0xffffffffu, mbar_wait(a_full, a_uses & 1u, abort_flag, p.timeout_ns))) { ok = false; break; }
-          ++a_uses;
-          cur_mt = mt;
-        }
-      }
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
       for (int ks = 0; ks < nks; ++ks, ++it) {
         const int s = it % S, slot = it % kSfSlots;
         bool w_ok = mbar_wait(full_bar(s), (it / S) & 1, abort_flag, p.timeout_ns);
         if (w_ok) w_ok = mbar_wait(sf_empty(slot), ((it / kSfSlots) & 1) ^ 1u, abort_flag, p.timeout_ns);
         if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
         tc_fence_after();
-        // scale tiles of A (resident or in the stage) and of W (in the stage)
-        const uint32_t sfa = kAStat ? sfa_res + ks * 4 * 512 + lane * 16
-                                    : base + s * stage_bytes + kABytes + kBBytes + lane * 16;
-        const uint32_t sfb = kAStat ? base + s * stage_bytes + kBBytes + lane * 16 : sfa + kSfBytes;
+        const uint32_t sf = base + s * kStageBytes + kABytes + kBBytes + lane * 16;
         const uint32_t tsf = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + kSfCol + slot * 32;
         uint32_t ra[16], rb[16];
 #pragma unroll
         for (int kb = 0; kb < 4; ++kb) {        // tiles past the stage's last K block are never read
-          const uint4 a = ld_shared_v4(sfa + kb * 512);
-          const uint4 b = ld_shared_v4(sfb + kb * 512);
+          const uint4 a = ld_shared_v4(sf + kb * 512);
+          const uint4 b = ld_shared_v4(sf + kSfBytes + kb * 512);
           ra[4 * kb] = a.x; ra[4 * kb + 1] = a.y; ra[4 * kb + 2] = a.z; ra[4 * kb + 3] = a.w;
           rb[4 * kb] = b.x; rb[4 * kb + 1] = b.y; rb[4 * kb + 2] = b.z; rb[4 * kb + 3] = b.w;
         }
@@ -542,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;
     const uint32_t stg = out_stage + (warp - 2) * 2 * kOutChunkBytes;
     int tc = 0, nstore = 0;
-    for (int t = t_begin; t < t_end; t += t_step, ++tc) {
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++tc) {
       const int mt = t / n_ntiles, nt = t - mt * n_ntiles;
       const int m0 = mt * BM;
       const int e = expert_of_row(off_s, p.E, m0);
@@ -694,32 +629,10 @@ int make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64
   return QUADS_OK;
 }
 
-size_t gemm_smem_bytes(int stages, int n_chan, int E, bool astat, int64_t K) {
-  const size_t nks = static_cast<size_t>((K / 64 + 3) / 4);
-  const size_t stage = astat ? kBStageBytes : kStageBytes;
-  const size_t resident = astat ? nks * kABytes + nks * 4 * 512 : 0;
-  return 1024 + static_cast<size_t>(stages) * stage + resident +
-         static_cast<size_t>(n_chan / 16) * 2 * kCompChunkBytes + kOutStageBytes +
-         static_cast<size_t>(2 * stages + 9 + 2 * kSfSlots + 2) * 8 + 16 + static_cast<size_t>(2 * E + 1) * 4;
-}
-
-// Largest stage count (<= kMaxStages) that fits, or 0.
-int gemm_stages(int n_chan, int E, bool astat, int64_t K) {
-  const size_t smem_cap = 232448;   // 227 KB per block on sm_100
-  for (int st = kMaxStages; st >= 2; --st)
-    if (gemm_smem_bytes(st, n_chan, E, astat, K) <= smem_cap) return st;
-  return 0;
-}
-
-template <bool kSwiglu, bool kAStat>
-int launch_kernel(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_r, const CUtensorMap& tm_wc,
-                  const CUtensorMap& tm_y, const GemmParams& p, int grid, size_t smem, cudaStream_t stream) {
-  if (cudaFuncSetAttribute(grouped_gemm_kernel<kSwiglu, kAStat>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
-    return set_error(QUADS_ERR_CUDA, "cannot set %zu bytes of shared memory", smem);
-  grouped_gemm_kernel<kSwiglu, kAStat><<<grid, kThreads, smem, stream>>>(tm_a, tm_b, tm_r, tm_wc, tm_y, p);
-  count_launches(1);
-  return check_launch("grouped_gemm_kernel");
+size_t gemm_smem_bytes(int stages, int n_chan, int E) {
+  return 1024 + static_cast<size_t>(stages) * kStageBytes + static_cast<size_t>(n_chan / 16) * 2 * kCompChunkBytes +
+         kOutStageBytes + static_cast<size_t>(2 * stages + 9 + 2 * kSfSlots) * 8 + 16 +
+         static_cast<size_t>(2 * E + 1) * 4;
 }
 
 }  // namespace
@@ -775,13 +688,14 @@ int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_
   }
   QUADS_TRY(make_map_2d(&tm_y, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kSwiglu ? N / 2 : N, rows_cap, 32, 32,
                         CU_TENSOR_MAP_SWIZZLE_64B));
-  // A-stationary when the resident 128-row block of A still leaves a
-  // four-stage ring of W tiles; otherwise A and W both stream
-  const int st_astat = gemm_stages(n_chan, E, true, K);
-  const bool astat = st_astat >= 4;
-  const int stages = astat ? st_astat : gemm_stages(n_chan, E, false, K);
+  const size_t smem_cap = 232448;   // 227 KB per block on sm_100
+  int stages = kMaxStages;
+  while (stages >= 2 && gemm_smem_bytes(stages, n_chan, E) > smem_cap) --stages;
   QUADS_REQUIRE(stages >= 2, QUADS_ERR_UNSUPPORTED_SHAPE, "not enough shared memory for two stages");
-  const size_t smem = gemm_smem_bytes(stages, n_chan, E, astat, K);
+  const size_t smem = gemm_smem_bytes(stages, n_chan, E);
+  if (cudaFuncSetAttribute(grouped_gemm_kernel<kSwiglu>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return set_error(QUADS_ERR_CUDA, "cannot set %zu bytes of shared memory", smem);
   GemmParams p;
   p.a_scales = a_scales;
   p.w_scales = w_scales;
@@ -800,8 +714,9 @@ int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_
   const int64_t max_tiles = (rows_cap / BM) * (N / BN);
   int grid = num_sms();
   if (grid > max_tiles) grid = static_cast<int>(max_tiles);
-  return astat ? launch_kernel<kSwiglu, true>(tm_a, tm_b, tm_r, tm_wc, tm_y, p, grid, smem, stream)
-               : launch_kernel<kSwiglu, false>(tm_a, tm_b, tm_r, tm_wc, tm_y, p, grid, smem, stream);
+  grouped_gemm_kernel<kSwiglu><<<grid, kThreads, smem, stream>>>(tm_a, tm_b, tm_r, tm_wc, tm_y, p);
+  count_launches(1);
+  return check_launch("grouped_gemm_kernel");
 }
 
 }  // namespace

@@ -91,55 +91,57 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t* __restri
     if (amax_s[i]) atomicMax(&out_bits[i], amax_s[i] << 16);
 }
 
-// Contiguous rows (ld == K): the groups are contiguous ranges of 16-byte
-// vectors, swept with a grid-stride loop that keeps eight 16-byte loads per
-// thread in flight; one warp reduction and one atomic per warp and group.
+// Contiguous rows (ld == K): one grid-stride sweep over the tensor's 16-byte
+// vectors with kAmaxUnroll predicated loads per thread in flight.  A vector's
+// group follows from its row; each thread keeps a running maximum for its
+// current group and folds it into the block's shared maxima when the group
+// changes (rare: groups are long contiguous ranges), then the block folds
+// its maxima into the output.
 constexpr int kAmaxUnroll = 8;
 
 __global__ void __launch_bounds__(kThreads) amax_flat_kernel(const uint4* __restrict__ x, int64_t rows,
-                                                             int64_t vec_per_row, const int32_t* group_off,
-                                                             int n_groups, int64_t uniform_rows,
+                                                             uint32_t vec_per_row, const int32_t* group_off,
+                                                             int n_groups, FastDiv vec_div, FastDiv uniform,
                                                              unsigned int* __restrict__ out_bits) {
-  extern __shared__ int32_t off_a[];                       // n_groups + 1 (explicit groups)
-  if (group_off != nullptr)
-    for (int i = threadIdx.x; i <= n_groups; i += blockDim.x) off_a[i] = group_off[i];
-  __syncthreads();
-  const int64_t nth = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  for (int g = 0; g < n_groups; ++g) {                     // uniform across the grid
-    // as in amax_kernel, the last group runs to the last row; offsets are
-    // clamped to [0, rows] so that no read leaves the matrix
-    const int64_t r0 = min(max(group_off ? static_cast<int64_t>(off_a[g]) : g * uniform_rows, int64_t(0)), rows);
-    const int64_t r1 = g == n_groups - 1
-                           ? rows
-                           : min(max(group_off ? static_cast<int64_t>(off_a[g + 1]) : (g + 1) * uniform_rows,
-                                     int64_t(0)),
-                                 rows);
-    const int64_t v1 = r1 * vec_per_row;
-    uint32_t m = 0u;
-    int64_t v = r0 * vec_per_row + tid;
-    for (; v + (kAmaxUnroll - 1) * nth < v1; v += kAmaxUnroll * nth) {
-      uint4 r[kAmaxUnroll];
-#pragma unroll
-      for (int u = 0; u < kAmaxUnroll; ++u) r[u] = __ldg(x + v + u * nth);
-#pragma unroll
-      for (int u = 0; u < kAmaxUnroll; ++u) {
-        m = __vmaxu2(m, r[u].x & 0x7FFF7FFFu);
-        m = __vmaxu2(m, r[u].y & 0x7FFF7FFFu);
-        m = __vmaxu2(m, r[u].z & 0x7FFF7FFFu);
-        m = __vmaxu2(m, r[u].w & 0x7FFF7FFFu);
-      }
-    }
-    for (; v < v1; v += nth) {
-      const uint4 r = __ldg(x + v);
-      m = __vmaxu2(m, r.x & 0x7FFF7FFFu);
-      m = __vmaxu2(m, r.y & 0x7FFF7FFFu);
-      m = __vmaxu2(m, r.z & 0x7FFF7FFFu);
-      m = __vmaxu2(m, r.w & 0x7FFF7FFFu);
-    }
-    const unsigned int wm = __reduce_max_sync(0xffffffffu, max(m & 0xFFFFu, m >> 16));
-    if ((threadIdx.x & 31) == 0 && wm) atomicMax(&out_bits[g], wm << 16);
+  extern __shared__ int32_t sm_a[];
+  int32_t* off_a = sm_a;                                   // n_groups + 1 (explicit groups)
+  unsigned int* am_a = reinterpret_cast<unsigned int*>(sm_a + n_groups + 1);
+  for (int i = threadIdx.x; i <= n_groups; i += blockDim.x) {
+    if (group_off != nullptr) off_a[i] = group_off[i];
+    if (i < n_groups) am_a[i] = 0u;
   }
+  __syncthreads();
+  RowGroups grp{group_off ? off_a : nullptr, n_groups, uniform};
+  const int64_t nvec = rows * vec_per_row;                // < 2^31 (checked on the host)
+  const uint32_t nth = gridDim.x * blockDim.x;
+  int cur = -1;
+  uint32_t m = 0u;
+  for (uint32_t v = blockIdx.x * blockDim.x + threadIdx.x; v < nvec; v += kAmaxUnroll * nth) {
+    uint4 r[kAmaxUnroll];
+#pragma unroll
+    for (int u = 0; u < kAmaxUnroll; ++u)
+      r[u] = (v + u * nth < nvec) ? __ldg(x + v + u * nth) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int u = 0; u < kAmaxUnroll; ++u) {
+      if (v + u * nth >= nvec) break;
+      const int g = grp.of(fast_div(v + u * nth, vec_div));
+      if (g != cur) {
+        const unsigned int mm = max(m & 0xFFFFu, m >> 16);
+        if (cur >= 0 && mm) atomicMax(&am_a[cur], mm);
+        cur = g;
+        m = 0u;
+      }
+      m = __vmaxu2(m, r[u].x & 0x7FFF7FFFu);
+      m = __vmaxu2(m, r[u].y & 0x7FFF7FFFu);
+      m = __vmaxu2(m, r[u].z & 0x7FFF7FFFu);
+      m = __vmaxu2(m, r[u].w & 0x7FFF7FFFu);
+    }
+  }
+  const unsigned int mm = max(m & 0xFFFFu, m >> 16);
+  if (cur >= 0 && mm) atomicMax(&am_a[cur], mm);
+  __syncthreads();
+  for (int i = threadIdx.x; i < n_groups; i += blockDim.x)
+    if (am_a[i]) atomicMax(&out_bits[i], am_a[i] << 16);
 }
 
 // ----------------------------------------------------------------- quantize
@@ -449,10 +451,8 @@ __global__ void __launch_bounds__(1024) select_kernel(const float* __restrict__ 
 
 // ------------------------------------------------------------ STE backward
 
-// Few CTAs (two per SM), each thread with kSteUnroll 16-byte vectors of both
-// inputs in flight per iteration: enough bytes in flight to stream at HBM
-// speed while leaving the SMs' registers and warp slots to kernels that run
-// beside it on other streams.
+// Each thread keeps kSteUnroll 16-byte vectors of both inputs in flight per
+// iteration of a grid-stride loop.
 constexpr int kSteUnroll = 4;
 
 __device__ __forceinline__ uint4 ste_add(uint4 a, uint4 b) {
@@ -537,14 +537,16 @@ int launch_amax(const uint16_t* x, int64_t rows, int64_t K, int64_t ld, const in
   if (rows == 0) return QUADS_OK;
   QUADS_REQUIRE(rows < kMaxBlocks, QUADS_ERR_UNSUPPORTED_SHAPE, "too many rows");
   const uint32_t uniform = group_off ? 1u : static_cast<uint32_t>(rows / n_groups);
-  if (ld == K) {
-    const size_t smem_f = (static_cast<size_t>(n_groups) + 1) * 4;
+  if (ld == K && rows * (K / 8) < (int64_t(1) << 31)) {
+    const size_t smem_f = (2 * static_cast<size_t>(n_groups) + 1) * 4;
     const int64_t nvec = rows * (K / 8);
-    // two CTAs per SM keep 64 KB per SM in flight and leave room beside them
+    // two CTAs per SM keep 64 KB per SM in flight
     const int64_t want = ceil_div(nvec, static_cast<int64_t>(kThreads) * kAmaxUnroll);
     const int grid_f = static_cast<int>(want < 2 * num_sms() ? (want < 1 ? 1 : want) : 2 * num_sms());
-    amax_flat_kernel<<<grid_f, kThreads, smem_f, s>>>(reinterpret_cast<const uint4*>(x), rows, K / 8, group_off,
-                                                      n_groups, rows / n_groups,
+    amax_flat_kernel<<<grid_f, kThreads, smem_f, s>>>(reinterpret_cast<const uint4*>(x), rows,
+                                                      static_cast<uint32_t>(K / 8), group_off, n_groups,
+                                                      make_fastdiv(static_cast<uint32_t>(K / 8)),
+                                                      make_fastdiv(uniform ? uniform : 1u),
                                                       reinterpret_cast<unsigned int*>(amax_out));
     count_launches(1);
     return check_launch("amax_flat_kernel");
@@ -777,9 +779,8 @@ int quads_fakequant_weight_ste_backward(const uint16_t* grad_wfq, uint16_t* grad
   if (n == 0) return QUADS_OK;
   QUADS_REQUIRE(grad_wfq && grad_w && aligned(grad_wfq, 16) && aligned(grad_w, 16), QUADS_ERR_INVALID_ARG,
                 "gradients must be non-null and 16-byte aligned");
-  const int64_t want = ceil_div(ceil_div(n, 8), static_cast<int64_t>(kThreads) * kSteUnroll);
-  const int grid = static_cast<int>(want < 2 * num_sms() ? (want < 1 ? 1 : want) : 2 * num_sms());
-  ste_backward_kernel<<<grid, kThreads, 0, stream>>>(grad_wfq, grad_w, n, accumulate);
+  ste_backward_kernel<<<grid_for(ceil_div(ceil_div(n, 8), int64_t(kSteUnroll))), kThreads, 0, stream>>>(
+      grad_wfq, grad_w, n, accumulate);
   count_launches(1);
   return check_launch("ste_backward_kernel");
 }
