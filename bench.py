@@ -75,8 +75,8 @@ def load_peaks():
 # recorded from an ncu capture is reported only while the hash of these
 # files still equals the one recorded with it.
 KERNEL_SOURCES = {
-    "quantize.cu": ("amax_w", "fakequant_w_gate_up", "fakequant_w_down", "amax_x", "quantize_x", "quantize_h",
-                    "ste_backward"),
+    "quantize.cu": ("amax_w", "fakequant_w_gate_up", "fakequant_w_down", "amax_x", "quantize_x", "quantize_h"),
+    "ste_backward.cu": ("ste_backward",),
     "grouped_gemm.cu": ("gemm_gate_up", "gemm_gate_up_swiglu", "gemm_down"),
     "moe_route.cu": ("router_topk", "permute", "gather", "swiglu", "combine"),
     "trace_record.cu": ("export", "replay_x", "replay_h"),

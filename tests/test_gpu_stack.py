@@ -5,8 +5,11 @@ import pytest
 import torch
 
 from oracle import formats as F
+from oracle import moe as M
 from oracle import stack as S
 from tests.helpers import assert_bits_equal, bf16_np, bf16_torch, f32_of
+from train_alignment_b200 import stack as ST
+from train_alignment_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
 
@@ -36,3 +39,40 @@ def test_residual_add(cuda_lib, n):
     ref = S.residual_add(x, y)
     assert_bits_equal(F.bf16_bits(bf16_np(got)), F.bf16_bits(ref), "residual add")
     assert_bits_equal(F.bf16_bits(bf16_np(xt)), F.bf16_bits(ref), "residual add in place")
+
+
+def test_stack_alignment_pass(cuda_lib):
+    """The 8-layer stack (hidden 2048, 64 experts top-4, ffn 1024, 4096 tokens;
+    the last 4 layers recorded and replayed): one alignment pass runs, layer
+    0's routing agrees with the oracle's wherever the k-th and (k+1)-th
+    logits are further apart than the logits' rounding bound, every recorded
+    layer's record replays its own rollout input with zero mismatches, and
+    the per-token gap between the two sides is reported (unpinned)."""
+    cfg = W.CONFIGS["stack8_t4096_h2048_e64k4_f1024"]
+    st = ST.LayerStack(cfg, seed=0, device="cuda")
+    gap, cm, sm = st.alignment_pass(drift=1e-3)
+    torch.cuda.synchronize()
+    assert cuda_lib.device_status() == cuda_lib.OK
+    g = gap.cpu().numpy()
+    assert np.all(np.isfinite(g)) and g.shape == (cfg.T,)
+    print(f"per-token gap: median {np.median(g):.4f}, p90 {np.percentile(g, 90):.4f}, max {g.max():.4f}; "
+          f"replayed-layer mismatches: codes {cm}, scales {sm}")
+    # layer 0 routing against the oracle's logits on the same synthetic input
+    x0 = bf16_np(st.x0)
+    lg, absdot = S.router_logits(x0, st.w_r[0].cpu().numpy().astype(np.float64))
+    idx_ref, _ = M.router_topk(lg, cfg.k)
+    bound = (cfg.H + 1) * 2.0 ** -24 * absdot
+    srt = np.sort(lg, axis=1)[:, ::-1]
+    b_at = np.take_along_axis(bound, np.argsort(-lg, axis=1), axis=1)
+    clear = (srt[:, cfg.k - 1] - srt[:, cfg.k]) > (b_at[:, cfg.k - 1] + b_at[:, cfg.k])
+    assert clear.mean() > 0.99
+    got = f32_of(st.layers[0].topk_idx).astype(np.int64)
+    assert_bits_equal(got[clear], idx_ref[clear].astype(np.int64), "layer-0 routing")
+    # each record replays its own rollout input exactly
+    for l in range(cfg.layers - st.recorded, cfg.layers):
+        layer = st.layers[l]
+        layer.reset_counts()
+        layer.trainer_replay(st.x_roll[l], layer_id=l)
+        torch.cuda.synchronize()
+        assert int(layer.status.item()) == 0
+        assert f32_of(layer.counts).astype(np.int64).tolist() == [0, 0], l

@@ -91,13 +91,15 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t* __restri
     if (amax_s[i]) atomicMax(&out_bits[i], amax_s[i] << 16);
 }
 
-// Contiguous rows (ld == K): one grid-stride sweep over the tensor's 16-byte
-// vectors with kAmaxUnroll predicated loads per thread in flight.  A vector's
-// group follows from its row; each thread keeps a running maximum for its
-// current group and folds it into the block's shared maxima when the group
-// changes (rare: groups are long contiguous ranges), then the block folds
-// its maxima into the output.
+// Contiguous rows (ld == K): one sweep over the tensor in warp chunks of
+// 256 16-byte vectors (4 KB, lane l loads vectors l, l + 32, ... of the chunk:
+// eight coalesced 512-byte loads in flight per warp), chunks grid-strided
+// over the warps.  Groups are long contiguous ranges, so a chunk almost
+// always lies in one group, found once per chunk; a thread keeps a running
+// maximum for its current group and folds it into the block's shared maxima
+// when the group changes; the block then folds those into the output.
 constexpr int kAmaxUnroll = 8;
+constexpr uint32_t kAmaxChunk = 32 * kAmaxUnroll;
 
 __global__ void __launch_bounds__(kThreads) amax_flat_kernel(const uint4* __restrict__ x, int64_t rows,
                                                              uint32_t vec_per_row, const int32_t* group_off,
@@ -112,33 +114,42 @@ __global__ void __launch_bounds__(kThreads) amax_flat_kernel(const uint4* __rest
   }
   __syncthreads();
   RowGroups grp{group_off ? off_a : nullptr, n_groups, uniform};
-  const int64_t nvec = rows * vec_per_row;                // < 2^31 (checked on the host)
-  const uint32_t nth = gridDim.x * blockDim.x;
+  const uint32_t nvec = static_cast<uint32_t>(rows * vec_per_row);   // < 2^31 (checked on the host)
+  const uint32_t lane = threadIdx.x & 31;
+  const uint32_t nwarps = gridDim.x * (blockDim.x >> 5);
+  const uint32_t nchunks = (nvec + kAmaxChunk - 1) / kAmaxChunk;
   int cur = -1;
   uint32_t m = 0u;
-  for (uint32_t v = blockIdx.x * blockDim.x + threadIdx.x; v < nvec; v += kAmaxUnroll * nth) {
+  auto fold = [&](int g) {
+    const unsigned int mm = max(m & 0xFFFFu, m >> 16);
+    if (cur >= 0 && mm) atomicMax(&am_a[cur], mm);
+    cur = g;
+    m = 0u;
+  };
+  for (uint32_t c = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); c < nchunks; c += nwarps) {
+    const uint32_t base = c * kAmaxChunk;
     uint4 r[kAmaxUnroll];
 #pragma unroll
-    for (int u = 0; u < kAmaxUnroll; ++u)
-      r[u] = (v + u * nth < nvec) ? __ldg(x + v + u * nth) : make_uint4(0u, 0u, 0u, 0u);
+    for (int u = 0; u < kAmaxUnroll; ++u) {
+      const uint32_t v = base + u * 32 + lane;
+      r[u] = v < nvec ? __ldg(x + v) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    const uint32_t last = min(base + kAmaxChunk, nvec) - 1;
+    const int g0 = grp.of(fast_div(base, vec_div));
+    const bool one_group = g0 == grp.of(fast_div(last, vec_div));
 #pragma unroll
     for (int u = 0; u < kAmaxUnroll; ++u) {
-      if (v + u * nth >= nvec) break;
-      const int g = grp.of(fast_div(v + u * nth, vec_div));
-      if (g != cur) {
-        const unsigned int mm = max(m & 0xFFFFu, m >> 16);
-        if (cur >= 0 && mm) atomicMax(&am_a[cur], mm);
-        cur = g;
-        m = 0u;
-      }
+      const uint32_t v = base + u * 32 + lane;
+      if (v >= nvec) break;
+      const int g = one_group ? g0 : grp.of(fast_div(v, vec_div));
+      if (g != cur) fold(g);
       m = __vmaxu2(m, r[u].x & 0x7FFF7FFFu);
       m = __vmaxu2(m, r[u].y & 0x7FFF7FFFu);
       m = __vmaxu2(m, r[u].z & 0x7FFF7FFFu);
       m = __vmaxu2(m, r[u].w & 0x7FFF7FFFu);
     }
   }
-  const unsigned int mm = max(m & 0xFFFFu, m >> 16);
-  if (cur >= 0 && mm) atomicMax(&am_a[cur], mm);
+  fold(-1);
   __syncthreads();
   for (int i = threadIdx.x; i < n_groups; i += blockDim.x)
     if (am_a[i]) atomicMax(&out_bits[i], am_a[i] << 16);
@@ -451,58 +462,6 @@ __global__ void __launch_bounds__(1024) select_kernel(const float* __restrict__ 
 
 // ------------------------------------------------------------ STE backward
 
-// Each thread keeps kSteUnroll 16-byte vectors of both inputs in flight per
-// iteration of a grid-stride loop.
-constexpr int kSteUnroll = 4;
-
-__device__ __forceinline__ uint4 ste_add(uint4 a, uint4 b) {
-  uint32_t* pa = reinterpret_cast<uint32_t*>(&a);
-  const uint32_t* pb = reinterpret_cast<const uint32_t*>(&b);
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const float lo = __fadd_rn(bf16_bits_to_float(pa[j] & 0xFFFFu), bf16_bits_to_float(pb[j] & 0xFFFFu));
-    const float hi = __fadd_rn(bf16_bits_to_float(pa[j] >> 16), bf16_bits_to_float(pb[j] >> 16));
-    pa[j] = pack_bf16x2(lo, hi);
-  }
-  return a;
-}
-
-__global__ void __launch_bounds__(kThreads) ste_backward_kernel(const uint16_t* __restrict__ gfq,
-                                                                uint16_t* __restrict__ gw, int64_t n, int accumulate) {
-  const int64_t nv = n / 8;
-  const int64_t nth = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  const uint4* src = reinterpret_cast<const uint4*>(gfq);
-  uint4* dst = reinterpret_cast<uint4*>(gw);
-  int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  for (; i + (kSteUnroll - 1) * nth < nv; i += kSteUnroll * nth) {
-    uint4 a[kSteUnroll], b[kSteUnroll];
-#pragma unroll
-    for (int u = 0; u < kSteUnroll; ++u) a[u] = __ldg(src + i + u * nth);
-    if (accumulate) {
-#pragma unroll
-      for (int u = 0; u < kSteUnroll; ++u) b[u] = dst[i + u * nth];
-#pragma unroll
-      for (int u = 0; u < kSteUnroll; ++u) a[u] = ste_add(a[u], b[u]);
-    }
-#pragma unroll
-    for (int u = 0; u < kSteUnroll; ++u) dst[i + u * nth] = a[u];
-  }
-  for (; i < nv; i += nth) {
-    uint4 a = __ldg(src + i);
-    if (accumulate) a = ste_add(a, dst[i]);
-    dst[i] = a;
-  }
-  // tail (n % 8 elements) handled by the first thread
-  if (blockIdx.x == 0 && threadIdx.x == 0) {
-    for (int64_t i = nv * 8; i < n; ++i) {
-      if (accumulate)
-        gw[i] = static_cast<uint16_t>(
-            float_to_bf16_bits(__fadd_rn(bf16_bits_to_float(gfq[i]), bf16_bits_to_float(gw[i]))));
-      else
-        gw[i] = gfq[i];
-    }
-  }
-}
 
 // ------------------------------------------------------------- host helpers
 
@@ -540,9 +499,9 @@ int launch_amax(const uint16_t* x, int64_t rows, int64_t K, int64_t ld, const in
   if (ld == K && rows * (K / 8) < (int64_t(1) << 31)) {
     const size_t smem_f = (2 * static_cast<size_t>(n_groups) + 1) * 4;
     const int64_t nvec = rows * (K / 8);
-    // two CTAs per SM keep 64 KB per SM in flight
+    // four CTAs of 8 warps per SM: 128 KB per SM in flight
     const int64_t want = ceil_div(nvec, static_cast<int64_t>(kThreads) * kAmaxUnroll);
-    const int grid_f = static_cast<int>(want < 2 * num_sms() ? (want < 1 ? 1 : want) : 2 * num_sms());
+    const int grid_f = static_cast<int>(want < 4 * num_sms() ? (want < 1 ? 1 : want) : 4 * num_sms());
     amax_flat_kernel<<<grid_f, kThreads, smem_f, s>>>(reinterpret_cast<const uint4*>(x), rows,
                                                       static_cast<uint32_t>(K / 8), group_off, n_groups,
                                                       make_fastdiv(static_cast<uint32_t>(K / 8)),
@@ -772,18 +731,6 @@ int quads_fakequant_weight_ste_gate_up(const uint16_t* w, int64_t n_mat, int64_t
                         w_chan, ws, ws_bytes, rows / 2, stream);
 }
 
-int quads_fakequant_weight_ste_backward(const uint16_t* grad_wfq, uint16_t* grad_w, int64_t n, int accumulate,
-                                        quads_stream_t stream) {
-  clear_error();
-  QUADS_REQUIRE(n >= 0, QUADS_ERR_INVALID_ARG, "n must be >= 0");
-  if (n == 0) return QUADS_OK;
-  QUADS_REQUIRE(grad_wfq && grad_w && aligned(grad_wfq, 16) && aligned(grad_w, 16), QUADS_ERR_INVALID_ARG,
-                "gradients must be non-null and 16-byte aligned");
-  ste_backward_kernel<<<grid_for(ceil_div(ceil_div(n, 8), int64_t(kSteUnroll))), kThreads, 0, stream>>>(
-      grad_wfq, grad_w, n, accumulate);
-  count_launches(1);
-  return check_launch("ste_backward_kernel");
-}
 
 }  // extern "C"
 
