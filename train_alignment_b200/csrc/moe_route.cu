@@ -377,39 +377,42 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
     rows[s] = row_of[t * k + s];
     ws[s] = w[t * k + s];
   }
-  // four 8-column chunks per lane per iteration: the k x 4 loads of a slot are
-  // independent, so they are in flight together
-  for (int64_t c0 = lane * 8; c0 < H; c0 += 4 * 32 * 8) {
-    float acc[4][8];
+  // two 8-column chunks per lane per iteration, the loads of all k slots for
+  // both issued before any is used (up to 16 independent 16-byte loads)
+  for (int64_t c0 = lane * 8; c0 < H; c0 += 2 * 32 * 8) {
+    uint4 v[kMaxK][2];
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
+    for (int s = 0; s < kMaxK; ++s) {
+      if (s < k) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) acc[u][j] = 0.0f;
-    for (int s = 0; s < k; ++s) {
-      uint4 v[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int64_t c = c0 + u * 256;
-        v[u] = c < H ? __ldg(reinterpret_cast<const uint4*>(y + static_cast<int64_t>(rows[s]) * H + c))
-                     : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const uint32_t* p = reinterpret_cast<const uint32_t*>(&v[u]);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          acc[u][2 * j] = __fmaf_rn(ws[s], bf16_bits_to_float(p[j] & 0xFFFFu), acc[u][2 * j]);
-          acc[u][2 * j + 1] = __fmaf_rn(ws[s], bf16_bits_to_float(p[j] >> 16), acc[u][2 * j + 1]);
+        for (int u = 0; u < 2; ++u) {
+          const int64_t c = c0 + u * 256;
+          v[s][u] = c < H ? __ldg(reinterpret_cast<const uint4*>(y + static_cast<int64_t>(rows[s]) * H + c))
+                          : make_uint4(0, 0, 0, 0);
         }
       }
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < 2; ++u) {
       const int64_t c = c0 + u * 256;
+      float acc[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
+#pragma unroll
+      for (int s = 0; s < kMaxK; ++s) {
+        if (s < k) {
+          const uint32_t* p = reinterpret_cast<const uint32_t*>(&v[s][u]);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            acc[2 * j] = __fmaf_rn(ws[s], bf16_bits_to_float(p[j] & 0xFFFFu), acc[2 * j]);
+            acc[2 * j + 1] = __fmaf_rn(ws[s], bf16_bits_to_float(p[j] >> 16), acc[2 * j + 1]);
+          }
+        }
+      }
       if (c < H)
         *reinterpret_cast<uint4*>(out + t * H + c) =
-            make_uint4(pack_bf16x2(acc[u][0], acc[u][1]), pack_bf16x2(acc[u][2], acc[u][3]),
-                       pack_bf16x2(acc[u][4], acc[u][5]), pack_bf16x2(acc[u][6], acc[u][7]));
+            make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
+                       pack_bf16x2(acc[6], acc[7]));
     }
   }
 }

@@ -185,7 +185,17 @@ struct QuantArgs {
 // cooperatively: lane j takes channel slot j and fetches its element, code and
 // scale from the lane that owns the block by warp shuffles, then the warp
 // writes the row's residual slots as one contiguous store.
+// kMode: 0 any combination of outputs (runtime checks); 1 the weight
+// fake-quant (codes, scales, W_fq with g folded, compensation columns as
+// bf16(deq)); 2 the activation quantizer (codes, scales, residual channels).
+template <int kMode>
 __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a) {
+  constexpr bool kFq = kMode == 1, kAct = kMode == 2;
+  const bool has_codes = kFq || kAct || a.codes != nullptr;
+  const bool has_scales = kFq || kAct || a.scales != nullptr;
+  const bool has_wfq = kFq || (!kAct && a.w_fq != nullptr);
+  const int fold = kFq ? 1 : a.fold;
+  const int resid_mode = kFq ? 1 : (kAct ? 0 : a.resid_mode);
   extern __shared__ int32_t smem_q[];
   const int n = a.n_groups;
   const int nkb = static_cast<int>(a.K / 16);
@@ -241,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a) {
   for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows_e;
        row += warps) {
     if (row >= rows_valid) {                           // padding rows of the last tiled band
-      if (a.scales)
+      if (has_scales)
         for (int kb = lane; kb < nkb_e; kb += 32) a.scales[tiled_scale_offset(row, kb, ncol_tiles)] = 0;
       continue;
     }
@@ -256,6 +266,9 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a) {
       const int64_t f = second ? loc - a.ilv_half : loc;
       drow = base + (f >> 6) * 128 + (second ? 64 : 0) + (f & 63);
     }
+    // the row's part of the scale offsets (tiled: band, lane and quarter of the row)
+    const int64_t sbase = tiled ? ((drow >> 7) * ncol_tiles) * 512 + (drow & 31) * 16 + ((drow >> 5) & 3) * 4
+                                : drow * nkb;
     for (int p0 = 0; p0 < npass; p0 += 2) {
       uint32_t w[2][8];
 #pragma unroll
@@ -271,26 +284,25 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a) {
         QCore q{0u, 0u, 0u, 0.0f};
         if (kb < nkb) {
           q = quant_core(w[u], qc);
-          if (a.codes)
+          if (has_codes)
             *reinterpret_cast<uint2*>(a.codes + drow * (a.K / 2) + kb * 8) = make_uint2(q.lo, q.hi);
-          if (a.w_fq) {
+          if (has_wfq) {
             uint32_t o[8];
-            deq_block_bf16(q, g, a.fold, o);
+            deq_block_bf16(q, g, fold, o);
             uint4* dst = reinterpret_cast<uint4*>(a.w_fq + row * a.K + kb * 16);
             dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
             dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
           }
         }
-        if (a.scales && kb < nkb_e)
-          a.scales[tiled ? tiled_scale_offset(drow, kb, ncol_tiles) : drow * nkb + kb] =
-              static_cast<uint8_t>(q.scale);
+        if (has_scales && kb < nkb_e)
+          a.scales[sbase + (tiled ? (kb >> 2) * 512 + (kb & 3) : kb)] = static_cast<uint8_t>(q.scale);
         if (a.resid) {
           // Channel slot j of this pass is taken by lane j % 32.  The element
           // itself is read back through L2 (the input row, or, for bf16(deq)
           // with the scale folded, the W_fq row this warp has just written);
           // its code and block scale come from the owning lane by shuffles.
           const int slo = pass_slot[p], shi = pass_slot[p + 1];
-          const bool from_fq = a.resid_mode == 1 && a.fold && a.w_fq != nullptr;
+          const bool from_fq = resid_mode == 1 && fold && has_wfq;
           if (from_fq) __syncwarp();                     // this warp's W_fq stores are visible to it
           for (int j0 = slo; j0 < shi; j0 += 32) {       // warp-uniform
             const int j = j0 + lane;
@@ -307,11 +319,11 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a) {
               const float xv = act ? bf16_bits_to_float(__ldg(xr + c)) : 0.0f;
               const uint32_t code = (((bit < 8) ? cl : ch) >> (4 * (bit & 7))) & 15u;
               float v;
-              if (a.resid_mode == 2) {
+              if (resid_mode == 2) {
                 v = xv;
               } else {
                 const float dq = deq_f32(code, sv, g);
-                v = (a.resid_mode == 1) ? dq : __fsub_rn(xv, dq);
+                v = (resid_mode == 1) ? dq : __fsub_rn(xv, dq);
               }
               vb = float_to_bf16_bits(v);
             }
@@ -519,21 +531,30 @@ int launch_amax(const uint16_t* x, int64_t rows, int64_t K, int64_t ld, const in
   return check_launch("amax_kernel");
 }
 
+template <int kMode>
+int launch_quantize_mode(const QuantArgs& a, size_t smem, int64_t rows_e, cudaStream_t s) {
+  if (smem > 48 * 1024 && cudaFuncSetAttribute(quantize_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(smem)) != cudaSuccess)
+    return set_error(QUADS_ERR_CUDA, "cannot raise shared memory of quantize_kernel");
+  const int grid = persistent_grid(reinterpret_cast<const void*>(quantize_kernel<kMode>), kThreads, smem,
+                                   ceil_div(rows_e, 8));
+  quantize_kernel<kMode><<<grid, kThreads, smem, s>>>(a);
+  count_launches(1);
+  return check_launch("quantize_kernel");
+}
+
 int launch_quantize(QuantArgs a, cudaStream_t s) {
   if (a.rows == 0) return QUADS_OK;
   QUADS_REQUIRE(a.rows < kMaxBlocks, QUADS_ERR_UNSUPPORTED_SHAPE, "too many rows");
   a.uniform_div = make_fastdiv(a.group_off ? 1u : static_cast<uint32_t>(a.uniform_rows > 0 ? a.uniform_rows : 1));
   const size_t smem = quantize_smem(a.n_groups, a.K, a.n_chan);
-  if (smem > 48 * 1024) {
-    if (cudaFuncSetAttribute(quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-      return set_error(QUADS_ERR_CUDA, "cannot raise shared memory of quantize_kernel");
-  }
   const int64_t rows_e = a.scale_layout == QUADS_SCALES_TILED ? ceil_div(a.rows, 128) * 128 : a.rows;
-  const int grid = persistent_grid(reinterpret_cast<const void*>(quantize_kernel), kThreads, smem, ceil_div(rows_e, 8));
-  quantize_kernel<<<grid, kThreads, smem, s>>>(a);
-  count_launches(1);
-  return check_launch("quantize_kernel");
+  const bool any_resid = a.resid != nullptr && a.n_chan > 0;
+  if (a.codes && a.scales && a.w_fq && a.fold && (!any_resid || a.resid_mode == 1))
+    return launch_quantize_mode<1>(a, smem, rows_e, s);
+  if (a.codes && a.scales && !a.w_fq && (!any_resid || a.resid_mode == 0))
+    return launch_quantize_mode<2>(a, smem, rows_e, s);
+  return launch_quantize_mode<0>(a, smem, rows_e, s);
 }
 
 }  // namespace

@@ -30,13 +30,14 @@ class StageTimer:
     a CUDA graph and re-recorded at every replay.  Marks named "start", or
     starting with "wait" or "join", end no kernel stage."""
 
-    def __init__(self, enabled=False, external=False):
+    def __init__(self, enabled=False, external=False, only=None):
         self.enabled = enabled
         self.external = external
+        self.only = None if only is None else set(only)       # record only these marks
         self.chains = {}
 
     def mark(self, name):
-        if self.enabled:
+        if self.enabled and (self.only is None or name in self.only):
             s = torch.cuda.current_stream()
             ev = torch.cuda.Event(enable_timing=True, external=self.external)
             ev.record(s)
