@@ -55,6 +55,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sweep", action="store_true", help="skip the standalone quantize/replay size sweep")
     ap.add_argument("--serial", action="store_true", help="run the step on one stream (no weight-side overlap)")
+    ap.add_argument("--fuse-requant", action="store_true",
+                    help="quantize h in the gate/up GEMM epilogue with the previous step's amax (delayed scaling)")
     return ap.parse_args()
 
 
@@ -77,7 +79,7 @@ def load_peaks():
 KERNEL_SOURCES = {
     "quantize.cu": ("amax_w", "fakequant_w_gate_up", "fakequant_w_down", "amax_x", "quantize_x", "quantize_h"),
     "ste_backward.cu": ("ste_backward",),
-    "grouped_gemm.cu": ("gemm_gate_up", "gemm_gate_up_swiglu", "gemm_down"),
+    "grouped_gemm.cu": ("gemm_gate_up", "gemm_gate_up_swiglu", "gemm_gate_up_swiglu_quant", "gemm_down"),
     "moe_route.cu": ("router_topk", "permute", "gather", "swiglu", "combine"),
     "trace_record.cu": ("export", "replay_x", "replay_h"),
 }
@@ -164,6 +166,7 @@ def kernel_work(cfg, rpad):
         "gather": ("hbm", (R + T) * (H * q + nc * 2)),
         "gemm_gate_up": ("tensor", 2.0 * R * 2 * F * H + 2.0 * R * 2 * F * nc),
         "gemm_gate_up_swiglu": ("tensor", 2.0 * R * 2 * F * H + 2.0 * R * 2 * F * nc),
+        "gemm_gate_up_swiglu_quant": ("tensor", 2.0 * R * 2 * F * H + 2.0 * R * 2 * F * nc),
         "swiglu": ("hbm", rpad * (2 * F * 2 + F * 2)),
         "quantize_h": ("hbm", rpad * F * (2 + q) + rpad * ncf * 2),
         "gemm_down": ("tensor", 2.0 * R * H * F + 2.0 * R * H * ncf),
@@ -409,7 +412,7 @@ def run_ours(args):
     B.load()
     cfg = W.CONFIGS[args.workload]
     inp = W.moe_layer_inputs(cfg, seed=rank, device=dev)
-    layer = L.build_layer(cfg, inp, dev, overlap=not args.serial)
+    layer = L.build_layer(cfg, inp, dev, overlap=not args.serial, fuse_requant=args.fuse_requant)
     x, logits = inp["x"], inp["logits"]
     x_train = W.engine_drift(x, 1e-2, seed=rank, device=dev)
     g_all, g_gu, g_d = layer.grad_fq_buffers()          # both weight gradients in one allocation
@@ -610,7 +613,9 @@ def run_ours(args):
         "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "k": cfg.k, "F": cfg.F,
                    "n_chan": cfg.n_chan, "n_chan_f": cfg.n_chan_f, "rows_padded": rpad,
                    "parallelism": f"dp{world} (replicas, no collective)",
-                   "schedule": "one stream" if args.serial else "two streams (weight side overlapped)",
+                   "schedule": ("one stream" if args.serial else "two streams (weight side overlapped)") +
+                               ("; h quantized in the gate/up GEMM epilogue (delayed amax)" if args.fuse_requant
+                                else ""),
                    "l2": "flushed between steps (256 MiB memset outside the timed events)",
                    "gemm_flops_per_step": fp4 + comp},
         "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,

@@ -259,6 +259,32 @@ int quads_moe_grouped_gemm_nvfp4_swiglu(const uint8_t* a_codes, const uint8_t* a
                                         int n_chan, uint16_t* h, float* amax_out,
                                         quads_stream_t stream);
 
+/* a6 + a7 + the re-quantization of h in one pass: the SwiGLU GEMM above
+ * whose epilogue also NVFP4-quantizes h for the down projection.  Each
+ * expert uses the decode scale g_e = fp32(amax_h_in[e] / 2688), computed from
+ * an amax given in advance (calibrated, or the previous step's: delayed
+ * scaling).  Written:
+ *   h_codes  [rows_cap][F/2], h_scales tiled over rows_cap x F,
+ *   h_resid  [rows_cap][n_chan_h] BF16 residuals on chan_h (ascending valid
+ *            channels first, then -1; 0 on padding slots), NULL if n_chan_h = 0,
+ *   g_h_out  device float[E] = g_e.
+ * Rows below expert_off[E] are quantized, including the zero pad rows of
+ * each expert's segment.  The values written are those quads_quantize_nvfp4
+ * writes for this h with group_off = expert_off, amax_in = amax_h_in, the
+ * tiled layout and chan_h.  amax_h_out (nullable, overwritten) receives
+ * this h's per-expert max |h| (the next step's amax_h_in), and h (nullable)
+ * receives h itself in BF16.  F % 64 == 0, n_chan_h <= 256. */
+int quads_moe_grouped_gemm_nvfp4_swiglu_quant(const uint8_t* a_codes, const uint8_t* a_scales,
+                                              const float* g_a, int g_a_per_expert,
+                                              const uint8_t* w_codes, const uint8_t* w_scales,
+                                              const float* g_w, const int32_t* expert_off, int E,
+                                              int64_t rows_cap, int64_t F, int64_t K,
+                                              const uint16_t* a_resid, const uint16_t* w_resid,
+                                              int n_chan, const float* amax_h_in,
+                                              const int32_t* chan_h, int n_chan_h, uint8_t* h_codes,
+                                              uint8_t* h_scales, uint16_t* h_resid, float* g_h_out,
+                                              float* amax_h_out, uint16_t* h, quads_stream_t stream);
+
 /* --------------------------------------------------------- a7: SwiGLU
  * h[r][j] = bf16(silu(Y[r][j]) * Y[r][F + j]) for rows r < expert_off[E],
  * silu(v) = v / (1 + exp(-v)), computed in FP32 from the BF16 gate/up GEMM

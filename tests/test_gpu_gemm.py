@@ -9,7 +9,8 @@ import torch
 from oracle import formats as F
 from oracle import moe as M
 from oracle import nvfp4 as Q
-from tests.helpers import assert_bits_equal, assert_close_tol, bf16_np, bf16_torch, f32_of, gate_up_interleave_index
+from tests.helpers import (assert_bits_equal, assert_close_tol, bf16_np, bf16_torch, f32_of, gate_up_interleave_index,
+                           u8_np)
 from train_alignment_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
@@ -152,6 +153,20 @@ def _gpu_args(p, w_c, w_s, wc):
     return args
 
 
+def _swiglu_ref(p, F_):
+    """The oracle's h = SwiGLU(bf16(y)) and a bound on |h_gpu - h|: the GEMM
+    tolerance of y carried through SwiGLU, plus one BF16 rounding of h."""
+    y_ref, absdot = _oracle(p)
+    tol_y = 1e-2 * np.abs(y_ref) + 1e-3 * absdot
+    g, u = y_ref[:, :F_], y_ref[:, F_:]
+    sig = 1.0 / (1.0 + np.exp(-g))
+    h_ref = M.swiglu(F.bf16_rne(y_ref.astype(np.float32)))
+    dsilu = np.abs(sig * (1.0 + g * (1.0 - sig)))
+    tol_h = dsilu * (np.abs(u) + tol_y[:, F_:]) * tol_y[:, :F_] + np.abs(g * sig) * tol_y[:, F_:] + \
+        2.0 ** -7 * np.abs(h_ref) + 1e-30
+    return h_ref, tol_h
+
+
 @pytest.mark.parametrize("counts,F_,K,nc", [
     ([64], 64, 64, 0),                  # one tile: 64 gate + 64 up columns
     ([130, 0, 257], 128, 512, 32),      # empty expert, ragged experts
@@ -174,14 +189,7 @@ def test_grouped_gemm_swiglu_parity(cuda_lib, counts, F_, K, nc):
     got = bf16_np(h)
     assert np.all(np.isnan(got[R:])), "rows past expert_off[E] must be untouched"
     # against the oracle: y within the GEMM tolerance, carried through SwiGLU
-    y_ref, absdot = _oracle(p)
-    tol_y = 1e-2 * np.abs(y_ref) + 1e-3 * absdot
-    g, u = y_ref[:, :F_], y_ref[:, F_:]
-    sig = 1.0 / (1.0 + np.exp(-g))
-    h_ref = M.swiglu(F.bf16_rne(y_ref.astype(np.float32)))
-    dsilu = np.abs(sig * (1.0 + g * (1.0 - sig)))
-    tol_h = dsilu * (np.abs(u) + tol_y[:, F_:]) * tol_y[:, :F_] + np.abs(g * sig) * tol_y[:, F_:] + \
-        2.0 ** -7 * np.abs(h_ref) + 1e-30
+    h_ref, tol_h = _swiglu_ref(p, F_)
     err = np.abs(got[:R] - h_ref)
     assert np.all(err <= tol_h), f"{np.sum(err > tol_h)} of {err.size} h values outside the tolerance"
     # against the plain GEMM (same operands) + the SwiGLU kernel: identical bits
@@ -198,3 +206,76 @@ def test_grouped_gemm_swiglu_parity(cuda_lib, counts, F_, K, nc):
         want = np.max(np.abs(got[lo:hi])) if hi > lo else 0.0
         assert a[e] == want, (e, a[e], want)
     assert_bits_equal(a.astype(np.float32), f32_of(amax2).astype(np.float32), "amax vs SwiGLU kernel")
+
+
+@pytest.mark.parametrize("counts,F_,K,nc,nch,amax_scale", [
+    ([64], 64, 64, 0, 0, 1.0),                 # one tile, no channels on either side
+    ([130, 0, 257], 128, 512, 32, 16, 1.0),    # empty expert, ragged experts, h channels
+    ([500, 20, 1000, 3], 192, 1024, 64, 32, 0.7),   # stale amax below the true max: saturating codes
+    ([300, 40], 256, 256, 16, 48, 1.3),        # stale amax above it; channels in several 32-column chunks
+])
+def test_grouped_gemm_swiglu_quant(cuda_lib, counts, F_, K, nc, nch, amax_scale):
+    """Gate/up GEMM with SwiGLU and the NVFP4 quantization of h in one
+    epilogue: h, its codes, tiled scales, per-expert scales and channel
+    residuals identical to the SwiGLU GEMM followed by quads_quantize_nvfp4
+    with the same per-expert amax (given in advance, as delayed scaling
+    does); the dequantized h against the oracle's quantization of the
+    oracle's h within the GEMM tolerance carried through SwiGLU plus one
+    NVFP4 step of each side."""
+    p = _problem(counts, 2 * F_, K, nc, seed=5 * sum(counts) + F_ + K + nc + nch)
+    perm = gate_up_interleave_index(F_)
+    wc_il = p["wc"][:, perm] if nc else None
+    args = _gpu_args(p, p["w_c"][:, perm], p["w_s"][:, perm], wc_il)
+    E, cap, R = p["E"], p["cap"], p["R"]
+    off = p["off"]
+    # two-pass path: SwiGLU GEMM, then the quantizer with a given amax
+    h_ref_gpu, amax_true = cuda_lib.moe_grouped_gemm_nvfp4_swiglu(F=F_, **args)
+    amax_in = (amax_true * amax_scale).contiguous()
+    r = np.random.default_rng(nch + F_)
+    chan_h = None
+    if nch:
+        chan_h = torch.from_numpy(Q.pad_channels(np.sort(r.choice(F_, nch - 3, replace=False)), 16)).cuda()
+    c2, s2, g2, r2 = cuda_lib.quantize_nvfp4(h_ref_gpu[:R], group_off=args["expert_off"], n_groups=E,
+                                             amax_in=amax_in, scale_layout=cuda_lib.SCALES_TILED, chan=chan_h)
+    # fused
+    h = torch.full((cap, F_), float("nan"), dtype=torch.bfloat16, device="cuda")
+    hc = torch.full((cap, F_ // 2), 0xAB, dtype=torch.uint8, device="cuda")
+    c1, s1, r1, g1, amax1 = cuda_lib.moe_grouped_gemm_nvfp4_swiglu_quant(F=F_, amax_h_in=amax_in, chan_h=chan_h,
+                                                                        h=h, h_codes=hc, **args)
+    torch.cuda.synchronize()
+    assert cuda_lib.device_status() == cuda_lib.OK
+    assert_bits_equal(F.bf16_bits(bf16_np(h)[:R]), F.bf16_bits(bf16_np(h_ref_gpu)[:R]), "h")
+    assert np.all(np.isnan(bf16_np(h)[R:])), "rows past expert_off[E] must be untouched"
+    assert_bits_equal(u8_np(c1)[:R], u8_np(c2), "h codes")
+    assert np.all(u8_np(c1)[R:] == 0xAB), "code rows past expert_off[E] must be untouched"
+    nsb = cuda_lib.scales_bytes(R, F_, cuda_lib.SCALES_TILED)
+    assert_bits_equal(u8_np(s1)[:nsb], u8_np(s2), "h scales")
+    assert_bits_equal(f32_of(g1).astype(np.float32), f32_of(g2).astype(np.float32), "g_h")
+    assert_bits_equal(f32_of(amax1).astype(np.float32), f32_of(amax_true).astype(np.float32), "amax_h_out")
+    if nch:
+        assert_bits_equal(F.bf16_bits(bf16_np(r1)[:R]), F.bf16_bits(bf16_np(r2)), "h residuals")
+    # against the oracle: its h, quantized by its quantizer with the same amax.
+    # |Q(a) - Q(b)| <= e(a) + e(b) + |a - b|, where one NVFP4 step moves a value
+    # of a block with max m by at most max(S, m - 6 S) for the block scale
+    # S <= m (1 + 2^-4) / 6 + g (E4M3 rounding, subnormal floor) and
+    # 6 S >= min(m (1 - 2^-4), 2688 g) - 6 g (saturation at 448 when the given amax
+    # is below the data's)
+    h_or, tol_h = _swiglu_ref(p, F_)
+    amax_or = f32_of(amax_in).astype(np.float64)
+    qc, qs, qg = Q.quantize_grouped(h_or, off, amax=amax_or)
+    deq_or = np.zeros_like(h_or)
+    for e in range(E):
+        if off[e + 1] > off[e]:
+            deq_or[off[e]:off[e + 1]] = Q.dequant(qc[off[e]:off[e + 1]], qs[off[e]:off[e + 1]], qg[e])
+    deq_gpu = f32_of(cuda_lib.dequant(c1, s1, cuda_lib.SCALES_TILED, g1, R, F_, group_off=args["expert_off"],
+                                      n_groups=E, out_dtype=cuda_lib.OUT_F32))
+    g_row = np.repeat(qg, np.diff(off))[:, None]
+    m = (np.abs(h_or) + tol_h).reshape(R, F_ // 16, 16).max(axis=2)
+    m = np.repeat(m, 16, axis=1)
+    s_hi = m * (1 + 2.0 ** -4) / 6 + g_row
+    e_step = np.maximum(s_hi, m - np.minimum(m * (1 - 2.0 ** -4), 2688.0 * g_row) + 6 * g_row)
+    tol = 2 * e_step + tol_h + 1e-30
+    err = np.abs(deq_gpu - deq_or)
+    assert np.all(err <= tol), f"{np.sum(err > tol)} of {err.size} dequantized h values outside the tolerance"
+    match = np.mean(F.unpack_nibbles(u8_np(c1)[:R]) == qc)
+    assert match > 0.9, f"only {match:.3f} of the h codes match the oracle's"

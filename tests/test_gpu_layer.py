@@ -115,3 +115,45 @@ def test_ste(run):
     cfg, layer, ref = run
     assert_bits_equal(F.bf16_bits(bf16_np(layer.grad_gu)), F.bf16_bits(ref["grad"]), "grad_gu")
     assert_bits_equal(F.bf16_bits(bf16_np(layer.grad_d)), F.bf16_bits(ref["grad_d"]), "grad_d")
+
+
+def test_fused_requant_layer_matches_two_pass(cuda_lib):
+    """The layer with h's NVFP4 quantization in the gate/up GEMM epilogue
+    (delayed scaling: the per-expert scale comes from the amax held from the
+    step before) against the two-pass layer, on the same batch twice.  With
+    the held amax equal to this batch's own, the fused layer's h codes,
+    scales, residuals, per-expert scales, TRACE record and output are the
+    two-pass layer's, bit for bit; its amax_h is this step's exact amax."""
+    cfg = W.MOE_T2048
+    inp = W.moe_layer_inputs(cfg, seed=1, device="cpu")
+    r = np.random.default_rng(1)
+    chan_x = torch.from_numpy(Q.pad_channels(np.sort(r.choice(cfg.H, cfg.n_chan - 3, replace=False))))
+    chan_h = torch.from_numpy(Q.pad_channels(np.sort(r.choice(cfg.F, cfg.n_chan_f - 7, replace=False))))
+    dev = "cuda"
+    x, logits = inp["x"].to(dev), inp["logits"].to(dev)
+    x_train = W.engine_drift(inp["x"], 1e-2, seed=1).to(dev)
+    two = L.MoELayer(cfg, inp["w_gu"].to(dev), inp["w_d"].to(dev), chan_x, chan_h, dev)
+    _, g_gu, g_d = two.grad_fq_buffers()
+    g_gu.zero_()
+    g_d.zero_()
+    two.reset_counts()
+    two.step(x, logits, x_train, g_gu, g_d)
+    torch.cuda.synchronize()
+    fused = L.MoELayer(cfg, inp["w_gu"].to(dev), inp["w_d"].to(dev), chan_x, chan_h, dev, fuse_requant=True,
+                       amax_h_init=two.amax_h.clone())
+    for step in range(2):
+        fused.reset_counts()
+        fused.step(x, logits, x_train, g_gu, g_d)
+        torch.cuda.synchronize()
+        assert cuda_lib.device_status() == cuda_lib.OK
+        R = int(two.expert_off[-1].item())
+        assert_bits_equal(u8_np(fused.h_codes)[:R], u8_np(two.h_codes)[:R], f"h codes, step {step}")
+        nsb = cuda_lib.scales_bytes(R, cfg.F, cuda_lib.SCALES_TILED)
+        assert_bits_equal(u8_np(fused.h_scales)[:nsb], u8_np(two.h_scales)[:nsb], f"h scales, step {step}")
+        assert_bits_equal(F.bf16_bits(bf16_np(fused.h_resid)[:R]), F.bf16_bits(bf16_np(two.h_resid)[:R]),
+                          f"h residuals, step {step}")
+        assert_bits_equal(f32_of(fused.g_h).astype(np.float32), f32_of(two.g_h).astype(np.float32), "g_h")
+        assert_bits_equal(f32_of(fused.amax_h).astype(np.float32), f32_of(two.amax_h).astype(np.float32), "amax_h")
+        assert_bits_equal(F.bf16_bits(bf16_np(fused.out)), F.bf16_bits(bf16_np(two.out)), f"output, step {step}")
+        assert_bits_equal(u8_np(fused.record), u8_np(two.record), f"TRACE record, step {step}")
+        assert_bits_equal(f32_of(fused.counts).astype(np.int64), f32_of(two.counts).astype(np.int64), "counts")

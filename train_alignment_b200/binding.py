@@ -84,6 +84,9 @@ _SIGS = {
                                              c_i64, c_vp, c_vp, c_i32, c_vp, c_vp]),
     "quads_moe_grouped_gemm_nvfp4_swiglu": (c_i32, [c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_i32, c_i64,
                                                     c_i64, c_i64, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp]),
+    "quads_moe_grouped_gemm_nvfp4_swiglu_quant": (c_i32, [c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_i32,
+                                                          c_i64, c_i64, c_i64, c_vp, c_vp, c_i32, c_vp, c_vp, c_i32,
+                                                          c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
     "quads_swiglu": (c_i32, [c_vp, c_i64, c_i64, c_vp, c_i32, c_vp, c_vp, c_vp]),
     "quads_moe_unpermute_combine": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i32, c_i64, c_vp, c_vp]),
     "quads_fakequant_weight_ste": (c_i32, [c_vp, c_i64, c_i64, c_i64, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_i32,
@@ -317,6 +320,30 @@ def moe_grouped_gemm_nvfp4_swiglu(a_codes, a_scales, g_a, w_codes, w_scales, g_w
         rows_cap, F, K, _p(a_resid), _p(w_resid), n_chan, _p(h), _p(amax) if want_amax else None, _s()),
         "quads_moe_grouped_gemm_nvfp4_swiglu")
     return h, (amax if want_amax else None)
+
+
+def moe_grouped_gemm_nvfp4_swiglu_quant(a_codes, a_scales, g_a, w_codes, w_scales, g_w, expert_off, E, rows_cap, F,
+                                        K, amax_h_in, chan_h=None, a_resid=None, w_resid=None, h_codes=None,
+                                        h_scales=None, h_resid=None, g_h=None, amax_h_out=None, h=None):
+    """Gate/up GEMM + SwiGLU + NVFP4 quantization of h (per-expert scale from
+    amax_h_in).  Returns (h_codes, h_scales, h_resid or None, g_h, amax_h_out)."""
+    dev = a_codes.device
+    n_chan = 0 if a_resid is None else a_resid.shape[1]
+    n_chan_h = 0 if chan_h is None else int(chan_h.numel())
+    h_codes = h_codes if h_codes is not None else _empty((rows_cap, F // 2), torch.uint8, dev)
+    h_scales = h_scales if h_scales is not None else _empty((scales_bytes(rows_cap, F, SCALES_TILED),), torch.uint8,
+                                                            dev)
+    if n_chan_h and h_resid is None:
+        h_resid = _empty((rows_cap, n_chan_h), torch.bfloat16, dev)
+    g_h = g_h if g_h is not None else _empty((E,), torch.float32, dev)
+    amax_h_out = amax_h_out if amax_h_out is not None else _empty((E,), torch.float32, dev)
+    per_expert = 1 if g_a.numel() == E and E > 1 else 0
+    _check(load().quads_moe_grouped_gemm_nvfp4_swiglu_quant(
+        _p(a_codes), _p(a_scales), _p(g_a), per_expert, _p(w_codes), _p(w_scales), _p(g_w), _p(expert_off), E,
+        rows_cap, F, K, _p(a_resid), _p(w_resid), n_chan, _p(amax_h_in), _p(chan_h), n_chan_h, _p(h_codes),
+        _p(h_scales), _p(h_resid) if n_chan_h else None, _p(g_h), _p(amax_h_out), _p(h), _s()),
+        "quads_moe_grouped_gemm_nvfp4_swiglu_quant")
+    return h_codes, h_scales, (h_resid if n_chan_h else None), g_h, amax_h_out
 
 
 def swiglu(y, F, expert_off, E, h=None, amax=None, want_amax=True):

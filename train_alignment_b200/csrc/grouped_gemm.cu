@@ -84,8 +84,17 @@ struct GemmParams {
   const int32_t* expert_off;
   uint16_t* y;
   unsigned int* amax_bits;   // SwiGLU epilogue: per-expert max |h| (float bits), or null
+  // SwiGLU epilogue with NVFP4 quantization of h (per-expert scale from amax_h_in)
+  const float* amax_h_in;    // [E]
+  const int32_t* chan_h;     // [n_chan_h]: h's compensation channels
+  uint8_t* h_codes;          // [rows_cap][F/2]
+  uint8_t* h_scales;         // tiled over rows_cap x F
+  uint16_t* h_resid;         // [rows_cap][n_chan_h]
+  float* g_h_out;            // [E]
+  int n_chan_h;
   int g_a_per_expert;
   int E;
+  int rows_cap;              // rows of a_codes, y and the h outputs
   int N;
   int K;
   int n_chan;
@@ -272,7 +281,51 @@ __device__ __forceinline__ float epi_value(uint32_t acc, float G, bool has_comp,
 // kSwiglu: the W rows of every 128-row tile are 64 gate rows then the 64
 // matching up rows; the epilogue writes h = silu(y_gate) * y_up (64 columns
 // per tile) instead of y, and the per-expert max |h|.
-template <bool kSwiglu>
+// NVFP4 quantization of one lane's 32 consecutive h values (one row, h
+// columns [col0, col0 + 32), two blocks of 16) with decode scale g: codes,
+// the two tiled scales, and the residual of every compensation channel in
+// the chunk; the lane holding a row's first chunk also zeroes its padding
+// channel slots.  Same operations as quads_quantize_nvfp4 (quant_core).
+__device__ __forceinline__ void quantize_h_chunk(const GemmParams& p, const uint32_t (&o)[16], float g,
+                                                 const int32_t* chanh_s, const int32_t* hslot_s, int row, int col0,
+                                                 bool first_chunk) {
+  const int Fh = p.N / 2;
+  const QConsts qc = make_qconsts(g);
+  uint32_t w0[8], w1[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    w0[i] = o[i];
+    w1[i] = o[8 + i];
+  }
+  const QCore q0 = quant_core(w0, qc), q1 = quant_core(w1, qc);
+  const int64_t r = row;
+  *reinterpret_cast<uint4*>(p.h_codes + r * (Fh / 2) + col0 / 2) = make_uint4(q0.lo, q0.hi, q1.lo, q1.hi);
+  // blocks col0 / 16 and the next: adjacent bytes of one tiled scale row (col0 / 16 is even)
+  const int64_t so = tiled_scale_offset(r, col0 / 16, Fh / 64);
+  *reinterpret_cast<uint16_t*>(p.h_scales + so) = static_cast<uint16_t>(q0.scale | (q1.scale << 8));
+  if (p.n_chan_h) {
+    const int slo = hslot_s[col0 / 32], shi = hslot_s[col0 / 32 + 1];
+    for (int j = slo; j < shi; ++j) {
+      const int cc = chanh_s[j] - col0, b = cc >> 4, bit = cc & 15;
+      uint32_t word = 0;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) word = (i == (cc >> 1)) ? o[i] : word;
+      const float hv = bf16_bits_to_float((cc & 1) ? (word >> 16) : (word & 0xFFFFu));
+      const uint32_t lo = b ? q1.lo : q0.lo, hi = b ? q1.hi : q0.hi;
+      const uint32_t code = (((bit < 8) ? lo : hi) >> (4 * (bit & 7))) & 15u;
+      const float dq = deq_f32(code, b ? q1.sv : q0.sv, g);
+      p.h_resid[r * p.n_chan_h + j] = static_cast<uint16_t>(float_to_bf16_bits(__fsub_rn(hv, dq)));
+    }
+    if (first_chunk)
+      for (int j = hslot_s[Fh / 32]; j < p.n_chan_h; ++j) p.h_resid[r * p.n_chan_h + j] = 0;
+  }
+}
+
+// kQuant (with kSwiglu): h is also NVFP4-quantized in the epilogue with the
+// per-expert scale g_e = fp32(amax_h_in[e] / 2688): codes, tiled scales and
+// the residual channels, exactly as quads_quantize_nvfp4 of h with that
+// amax; h itself is stored only when y is non-null.
+template <bool kSwiglu, bool kQuant>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                         const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_wc,
@@ -303,6 +356,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* const abort_flag = reinterpret_cast<volatile int*>(misc + 4);
   int32_t* const off_s = reinterpret_cast<int32_t*>(misc + 16);
   float* const gscale_s = reinterpret_cast<float*>(off_s + p.E + 1);   // g_a(e) * g_w[e]
+  // kQuant: h's per-expert scale, its channels, and per 32-column chunk of h
+  // the first channel slot at or after the chunk (valid channels ascend)
+  float* const gh_s = gscale_s + p.E;                                  // E
+  int32_t* const chanh_s = reinterpret_cast<int32_t*>(gh_s + p.E);     // n_chan_h
+  int32_t* const hslot_s = chanh_s + p.n_chan_h;                       // N / 64 + 1
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -333,13 +391,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     off_s[i] = p.expert_off[i];
     if (i < p.E) gscale_s[i] = __fmul_rn(p.g_a[p.g_a_per_expert ? i : 0], p.g_w[i]);
   }
+  if constexpr (kQuant) {
+    const int Fh = p.N / 2;
+    for (int i = threadIdx.x; i < p.E; i += blockDim.x) {
+      gh_s[i] = __fdiv_rn(p.amax_h_in[i], kNvfp4Range);
+      if (blockIdx.x == 0 && p.g_h_out != nullptr) p.g_h_out[i] = gh_s[i];
+    }
+    for (int j = threadIdx.x; j < p.n_chan_h; j += blockDim.x) chanh_s[j] = p.chan_h[j];
+    __syncthreads();
+    for (int qc = threadIdx.x; qc <= Fh / 32; qc += blockDim.x) {
+      int cnt = 0;
+      for (int j = 0; j < p.n_chan_h; ++j) cnt += (chanh_s[j] >= 0 && chanh_s[j] < Fh && chanh_s[j] < 32 * qc) ? 1 : 0;
+      hslot_s[qc] = cnt;
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
   const int n_ntiles = p.N / BN;
-  const int total = (off_s[p.E] / BM) * n_ntiles;
+  // row tiles below expert_off[E], never past the buffers' rows_cap rows
+  const int total = (min(off_s[p.E], p.rows_cap) / BM) * n_ntiles;
   const int nkb_total = p.K / 64;                 // MMAs along K
   const int nks = (nkb_total + 3) / 4;            // pipeline stages along K
   const int n_col_tiles = nkb_total;              // 512-byte scale tiles per 128-row band
@@ -552,21 +625,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        const uint32_t sb = stg + (nstore & 1) * kOutChunkBytes;
-        if (lane == 0) bulk_wait_read_1();
-        __syncwarp();
-        // 64-byte swizzle (the store's tensor map): 16-byte chunk j of row r sits
-        // at chunk j ^ ((r >> 1) & 3), so the 32 lanes' row stores hit all banks
-        const uint32_t row_addr = sb + lane * 64;
-        const uint32_t sw = (lane >> 1) & 3u;
+        if constexpr (kQuant) quantize_h_chunk(p, o, gh_s[e], chanh_s, hslot_s, m0 + q * 32 + lane,
+                                               nt * (BN / 2) + c * 32, nt == 0 && c == 0);
+        if (!kQuant || p.y != nullptr) {
+          const uint32_t sb = stg + (nstore & 1) * kOutChunkBytes;
+          if (lane == 0) bulk_wait_read_1();
+          __syncwarp();
+          // 64-byte swizzle (the store's tensor map): 16-byte chunk j of row r sits
+          // at chunk j ^ ((r >> 1) & 3), so the 32 lanes' row stores hit all banks
+          const uint32_t row_addr = sb + lane * 64;
+          const uint32_t sw = (lane >> 1) & 3u;
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          st_shared_v4(row_addr + ((j ^ sw) << 4), o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(&tm_y, sb, (kSwiglu ? nt * (BN / 2) : nt * BN) + c * 32, m0 + q * 32);
-          bulk_commit();
+          for (int j = 0; j < 4; ++j)
+            st_shared_v4(row_addr + ((j ^ sw) << 4), o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tm_y, sb, (kSwiglu ? nt * (BN / 2) : nt * BN) + c * 32, m0 + q * 32);
+            bulk_commit();
+          }
         }
         if constexpr (kSwiglu) {
           hmax = __reduce_max_sync(0xffffffffu, hmax);
@@ -629,11 +706,23 @@ int make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64
   return QUADS_OK;
 }
 
-size_t gemm_smem_bytes(int stages, int n_chan, int E) {
+// extra_words: the quantizing epilogue's tables (E + n_chan_h + N / 64 + 1)
+size_t gemm_smem_bytes(int stages, int n_chan, int E, size_t extra_words = 0) {
   return 1024 + static_cast<size_t>(stages) * kStageBytes + static_cast<size_t>(n_chan / 16) * 2 * kCompChunkBytes +
          kOutStageBytes + static_cast<size_t>(2 * stages + 9 + 2 * kSfSlots) * 8 + 16 +
-         static_cast<size_t>(2 * E + 1) * 4;
+         (static_cast<size_t>(2 * E + 1) + extra_words) * 4;
 }
+
+// The quantizing epilogue's outputs (all device memory).
+struct HQuant {
+  const float* amax_in;
+  const int32_t* chan;
+  int n_chan;
+  uint8_t* codes;
+  uint8_t* scales;
+  uint16_t* resid;
+  float* g_out;
+};
 
 }  // namespace
 }  // namespace quads
@@ -647,11 +736,11 @@ extern "C" {
 namespace quads {
 namespace {
 
-template <bool kSwiglu>
+template <bool kSwiglu, bool kQuant = false>
 int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_a, int g_a_per_expert,
                 const uint8_t* w_codes, const uint8_t* w_scales, const float* g_w, const int32_t* expert_off, int E,
                 int64_t rows_cap, int64_t N, int64_t K, const uint16_t* a_resid, const uint16_t* w_resid, int n_chan,
-                uint16_t* y, float* amax_out, cudaStream_t stream) {
+                uint16_t* y, float* amax_out, cudaStream_t stream, const HQuant* hq = nullptr) {
   QUADS_REQUIRE(E >= 1 && E <= 256, QUADS_ERR_UNSUPPORTED_SHAPE, "E must be in [1, 256]");
   QUADS_REQUIRE(N > 0 && N % BN == 0 && N <= (int64_t(1) << 20), QUADS_ERR_UNSUPPORTED_SHAPE,
                 "N (%lld) must be a positive multiple of 128", (long long)N);
@@ -662,11 +751,19 @@ int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_
   QUADS_REQUIRE(E * N < (int64_t(1) << 31), QUADS_ERR_UNSUPPORTED_SHAPE, "E * N too large");
   QUADS_REQUIRE(n_chan >= 0 && n_chan % 16 == 0 && n_chan <= kMaxChan, QUADS_ERR_UNSUPPORTED_SHAPE,
                 "n_chan must be a multiple of 16 in [0, %d]", kMaxChan);
-  QUADS_REQUIRE(a_codes && a_scales && g_a && w_codes && w_scales && g_w && expert_off && y, QUADS_ERR_INVALID_ARG,
-                "null pointer");
+  QUADS_REQUIRE(a_codes && a_scales && g_a && w_codes && w_scales && g_w && expert_off && (y || kQuant),
+                QUADS_ERR_INVALID_ARG, "null pointer");
+  if constexpr (kQuant) {
+    QUADS_REQUIRE(hq && hq->amax_in && hq->codes && hq->scales && hq->g_out, QUADS_ERR_INVALID_ARG,
+                  "amax_h_in, h_codes, h_scales and g_h_out are required");
+    QUADS_REQUIRE(hq->n_chan >= 0 && hq->n_chan <= 256, QUADS_ERR_UNSUPPORTED_SHAPE, "n_chan_h must be in [0, 256]");
+    QUADS_REQUIRE(hq->n_chan == 0 || (hq->chan && hq->resid), QUADS_ERR_INVALID_ARG, "chan_h and h_resid required");
+    QUADS_REQUIRE(aligned(hq->codes, 16) && aligned(hq->scales, 16) && (!hq->resid || aligned(hq->resid, 4)),
+                  QUADS_ERR_INVALID_ARG, "h_codes and h_scales must be 16-byte aligned");
+  }
   QUADS_REQUIRE(n_chan == 0 || (a_resid && w_resid), QUADS_ERR_INVALID_ARG, "a_resid and w_resid required");
   QUADS_REQUIRE(aligned(a_codes, 16) && aligned(w_codes, 16) && aligned(a_scales, 16) && aligned(w_scales, 16) &&
-                    aligned(y, 16) && (n_chan == 0 || (aligned(a_resid, 16) && aligned(w_resid, 16))),
+                    (!y || aligned(y, 16)) && (n_chan == 0 || (aligned(a_resid, 16) && aligned(w_resid, 16))),
                 QUADS_ERR_INVALID_ARG, "matrix pointers must be 16-byte aligned");
   if (kSwiglu && amax_out && cudaMemsetAsync(amax_out, 0, sizeof(float) * E, stream) != cudaSuccess)
     return set_error(QUADS_ERR_CUDA, "memset of amax_out failed");
@@ -686,14 +783,18 @@ int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_
     tm_r = tm_a;
     tm_wc = tm_a;
   }
-  QUADS_TRY(make_map_2d(&tm_y, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kSwiglu ? N / 2 : N, rows_cap, 32, 32,
-                        CU_TENSOR_MAP_SWIZZLE_64B));
+  if (y)
+    QUADS_TRY(make_map_2d(&tm_y, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kSwiglu ? N / 2 : N, rows_cap, 32, 32,
+                          CU_TENSOR_MAP_SWIZZLE_64B));
+  else
+    tm_y = tm_a;                                  // never used: no h store
+  const size_t extra = kQuant ? static_cast<size_t>(E + hq->n_chan + N / 64 + 1) : 0;
   const size_t smem_cap = 232448;   // 227 KB per block on sm_100
   int stages = kMaxStages;
-  while (stages >= 2 && gemm_smem_bytes(stages, n_chan, E) > smem_cap) --stages;
+  while (stages >= 2 && gemm_smem_bytes(stages, n_chan, E, extra) > smem_cap) --stages;
   QUADS_REQUIRE(stages >= 2, QUADS_ERR_UNSUPPORTED_SHAPE, "not enough shared memory for two stages");
-  const size_t smem = gemm_smem_bytes(stages, n_chan, E);
-  if (cudaFuncSetAttribute(grouped_gemm_kernel<kSwiglu>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const size_t smem = gemm_smem_bytes(stages, n_chan, E, extra);
+  if (cudaFuncSetAttribute(grouped_gemm_kernel<kSwiglu, kQuant>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return set_error(QUADS_ERR_CUDA, "cannot set %zu bytes of shared memory", smem);
   GemmParams p;
@@ -704,8 +805,16 @@ int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_
   p.expert_off = expert_off;
   p.y = y;
   p.amax_bits = reinterpret_cast<unsigned int*>(amax_out);
+  p.amax_h_in = kQuant ? hq->amax_in : nullptr;
+  p.chan_h = kQuant ? hq->chan : nullptr;
+  p.n_chan_h = kQuant ? hq->n_chan : 0;
+  p.h_codes = kQuant ? hq->codes : nullptr;
+  p.h_scales = kQuant ? hq->scales : nullptr;
+  p.h_resid = kQuant ? hq->resid : nullptr;
+  p.g_h_out = kQuant ? hq->g_out : nullptr;
   p.g_a_per_expert = g_a_per_expert ? 1 : 0;
   p.E = E;
+  p.rows_cap = static_cast<int>(rows_cap);
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
   p.n_chan = n_chan;
@@ -714,7 +823,7 @@ int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_
   const int64_t max_tiles = (rows_cap / BM) * (N / BN);
   int grid = num_sms();
   if (grid > max_tiles) grid = static_cast<int>(max_tiles);
-  grouped_gemm_kernel<kSwiglu><<<grid, kThreads, smem, stream>>>(tm_a, tm_b, tm_r, tm_wc, tm_y, p);
+  grouped_gemm_kernel<kSwiglu, kQuant><<<grid, kThreads, smem, stream>>>(tm_a, tm_b, tm_r, tm_wc, tm_y, p);
   count_launches(1);
   return check_launch("grouped_gemm_kernel");
 }
@@ -732,6 +841,22 @@ int quads_moe_grouped_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales
   clear_error();
   return launch_gemm<false>(a_codes, a_scales, g_a, g_a_per_expert, w_codes, w_scales, g_w, expert_off, E, rows_cap,
                             N, K, a_resid, w_resid, n_chan, y, nullptr, stream);
+}
+
+int quads_moe_grouped_gemm_nvfp4_swiglu_quant(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_a,
+                                              int g_a_per_expert, const uint8_t* w_codes, const uint8_t* w_scales,
+                                              const float* g_w, const int32_t* expert_off, int E, int64_t rows_cap,
+                                              int64_t F, int64_t K, const uint16_t* a_resid,
+                                              const uint16_t* w_resid, int n_chan, const float* amax_h_in,
+                                              const int32_t* chan_h, int n_chan_h, uint8_t* h_codes,
+                                              uint8_t* h_scales, uint16_t* h_resid, float* g_h_out,
+                                              float* amax_h_out, uint16_t* h, quads_stream_t stream) {
+  clear_error();
+  QUADS_REQUIRE(F > 0 && F % 64 == 0, QUADS_ERR_UNSUPPORTED_SHAPE, "F (%lld) must be a positive multiple of 64",
+                (long long)F);
+  const HQuant hq{amax_h_in, chan_h, n_chan_h, h_codes, h_scales, h_resid, g_h_out};
+  return launch_gemm<true, true>(a_codes, a_scales, g_a, g_a_per_expert, w_codes, w_scales, g_w, expert_off, E,
+                                 rows_cap, 2 * F, K, a_resid, w_resid, n_chan, h, amax_h_out, stream, &hq);
 }
 
 int quads_moe_grouped_gemm_nvfp4_swiglu(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_a,

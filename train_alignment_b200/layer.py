@@ -66,7 +66,8 @@ class MoELayer:
     """Weights, calibrated channel sets and every buffer of one layer at a
     fixed token count; step() runs the whole path without allocating."""
 
-    def __init__(self, cfg: MoEConfig, w_gu, w_d, chan_x, chan_h, device="cuda", fuse_swiglu=None, overlap=True):
+    def __init__(self, cfg: MoEConfig, w_gu, w_d, chan_x, chan_h, device="cuda", fuse_swiglu=None, overlap=True,
+                 fuse_requant=False, amax_h_init=None):
         self.cfg = cfg
         T, H, E, k, F = cfg.T, cfg.H, cfg.E, cfg.k, cfg.F
         dev = torch.device(device)
@@ -91,6 +92,13 @@ class MoELayer:
         # SwiGLU in the gate/up GEMM's epilogue (rollout gate/up weights kept
         # in the 64-row interleaved gate/up order), else a separate pass
         self.fuse_swiglu = (F % 64 == 0) if fuse_swiglu is None else bool(fuse_swiglu)
+        # NVFP4 quantization of h in the same epilogue too (delayed scaling:
+        # each expert's scale comes from the previous step's max |h|, or from
+        # amax_h_init on the first step), else a separate pass with this
+        # step's exact amax
+        self.fuse_requant = bool(fuse_requant)
+        if self.fuse_requant and not self.fuse_swiglu:
+            raise ValueError("fuse_requant needs the fused SwiGLU epilogue (F % 64 == 0)")
         # the weight side of a step on its own stream (False: one stream)
         self.overlap = bool(overlap)
         self.nc_x = int(chan_x.numel())
@@ -138,6 +146,9 @@ class MoELayer:
         self.pa_resid = e((cap, self.nc_x), bf)
         self.y_gu = None if self.fuse_swiglu else e((cap, 2 * F), bf)
         self.h, self.amax_h = e((cap, F), bf), e((E,), f32)
+        self.amax_h_prev = torch.zeros(E, dtype=f32, device=dev)
+        if amax_h_init is not None:
+            self.amax_h_prev.copy_(amax_h_init)
         self.h_codes, self.h_scales = vh["codes"].view(cap, F // 2), vh["scales"]
         self.g_h = vh["g"]
         self.h_resid = vh["resid"].view(cap, self.nc_h) if self.nc_h else None
@@ -234,7 +245,15 @@ class MoELayer:
     def _rollout_gate_up(self, t):
         cfg = self.cfg
         H, E, F = cfg.H, cfg.E, cfg.F
-        if self.fuse_swiglu:
+        if self.fuse_requant:
+            B.moe_grouped_gemm_nvfp4_swiglu_quant(
+                self.pa_codes, self.pa_scales, self.g_x, self.w_gu_codes, self.w_gu_scales, self.g_w_gu,
+                self.expert_off, E, self.cap, F, H, self.amax_h_prev, chan_h=self.chan_h if self.nc_h else None,
+                a_resid=self.pa_resid, w_resid=self.wc_gu, h_codes=self.h_codes, h_scales=self.h_scales,
+                h_resid=self.h_resid, g_h=self.g_h, amax_h_out=self.amax_h)
+            t.mark("gemm_gate_up_swiglu_quant")
+            self.amax_h_prev.copy_(self.amax_h)         # the next step's scale (a 4E-byte device copy)
+        elif self.fuse_swiglu:
             B.moe_grouped_gemm_nvfp4_swiglu(self.pa_codes, self.pa_scales, self.g_x, self.w_gu_codes,
                                             self.w_gu_scales, self.g_w_gu, self.expert_off, E, self.cap, F, H,
                                             self.pa_resid, self.wc_gu, h=self.h, amax=self.amax_h)
@@ -250,10 +269,11 @@ class MoELayer:
     def _rollout_down(self, t):
         cfg = self.cfg
         T, H, E, k, F = cfg.T, cfg.H, cfg.E, cfg.k, cfg.F
-        B.quantize_nvfp4(self.h, group_off=self.expert_off, n_groups=E, amax_in=self.amax_h,
-                         scale_layout=B.SCALES_TILED, chan=self.chan_h, codes=self.h_codes, scales=self.h_scales,
-                         g_out=self.g_h, resid_out=self.h_resid)
-        t.mark("quantize_h")
+        if not self.fuse_requant:
+            B.quantize_nvfp4(self.h, group_off=self.expert_off, n_groups=E, amax_in=self.amax_h,
+                             scale_layout=B.SCALES_TILED, chan=self.chan_h, codes=self.h_codes,
+                             scales=self.h_scales, g_out=self.g_h, resid_out=self.h_resid)
+            t.mark("quantize_h")
         B.moe_grouped_gemm_nvfp4(self.h_codes, self.h_scales, self.g_h, self.w_d_codes, self.w_d_scales,
                                  self.g_w_d, self.expert_off, E, self.cap, H, F, self.h_resid, self.wc_d,
                                  y=self.y_d)
@@ -349,9 +369,11 @@ def calibrate_channels(x, n_sel):
     return out
 
 
-def build_layer(cfg: MoEConfig, inputs, device="cuda", overlap=True):
+def build_layer(cfg: MoEConfig, inputs, device="cuda", overlap=True, fuse_requant=False):
     """Layer from generated inputs: channel sets calibrated on the layer's own
-    batch (X for the gate/up input, the uncompensated h for the down input)."""
+    batch (X for the gate/up input, the uncompensated h for the down input);
+    with fuse_requant, h's first-step per-expert amax is calibrated on the
+    same batch."""
     x, logits = inputs["x"], inputs["logits"]
     chan_x = calibrate_channels(x, cfg.n_chan)
     empty = torch.full((16,), -1, dtype=torch.int32, device=device)
@@ -361,5 +383,7 @@ def build_layer(cfg: MoEConfig, inputs, device="cuda", overlap=True):
     torch.cuda.synchronize()
     n_rows = int(probe.expert_off[-1].item())
     chan_h = calibrate_channels(probe.h[:n_rows].contiguous(), cfg.n_chan_f)
+    amax_h = probe.amax_h.clone()
     del probe
-    return MoELayer(cfg, inputs["w_gu"], inputs["w_d"], chan_x, chan_h, device, overlap=overlap)
+    return MoELayer(cfg, inputs["w_gu"], inputs["w_d"], chan_x, chan_h, device, overlap=overlap,
+                    fuse_requant=fuse_requant, amax_h_init=amax_h if fuse_requant else None)
