@@ -496,6 +496,81 @@ def pin_replay_counts_drift():
     assert cm == int(np.count_nonzero(c2 != c)) and sm == int(np.count_nonzero(s2 != s))
 
 
+def _unit_scale_block(vals):
+    """One row of 32 values (two blocks) with block scales 1 and decode scale
+    1, so the scaled value y equals x."""
+    x = np.zeros((1, 32))
+    x[0, :len(vals)] = vals
+    s1 = F.e4m3_rn_satfinite_code(np.array([[1.0, 1.0]]))
+    assert np.all(F.e4m3_value(s1) == 1.0)
+    return x, s1.astype(np.uint8), np.array([1.0])
+
+
+def pin_direction_worked_values():
+    """Rounding directions worked by hand on the E2M1 grid (0, .5, 1, 1.5, 2,
+    3, 4, 6) with S = 1: nearest level, ties to the even code, saturation at
+    6 counts as rounding down; values on the grid round down."""
+    cases = [(0.0, 0), (0.25, 0), (0.3, 1), (0.75, 1), (1.0, 0), (1.25, 0), (1.3, 1), (2.5, 0), (2.6, 1),
+             (3.5, 1), (5.0, 0), (5.5, 1), (6.0, 0), (7.0, 0), (-3.5, 1), (-0.2, 0), (-1.75, 1)]
+    x, s1, g = _unit_scale_block([v for v, _ in cases])
+    codes = F.e2m1_rne_code(x)
+    bits = TR.direction_bits(x, codes, s1, g)
+    assert bits[0, :len(cases)].tolist() == [b for _, b in cases]
+    # the trainer's guided choice, worked by hand: (y_t, recorded bit) -> level
+    guided = [(3.49, 1, 4.0, True), (3.6, 0, 3.0, True), (3.6, 1, 4.0, False), (0.1, 1, 0.5, True),
+              (6.5, 1, 6.0, False), (-2.2, 1, -3.0, True), (1.0, 1, 1.5, True)]
+    xt, _, _ = _unit_scale_block([v for v, _, _, _ in guided])
+    b = np.zeros((1, 32), dtype=np.uint8)
+    b[0, :len(guided)] = [bit for _, bit, _, _ in guided]
+    c, x_hat, corr = TR.replay_direction(b, s1, g, xt)
+    assert F.e2m1_value(c[0, :len(guided)]).tolist() == [lv for _, _, lv, _ in guided]
+    assert corr == sum(1 for _, _, _, fixed in guided if fixed)
+    assert np.array_equal(x_hat[0, :len(guided)], [lv for _, _, lv, _ in guided])
+
+
+def pin_direction_replay_reproduces_rounding():
+    """With the trainer's input equal to the rollout's, the compact record
+    replays the quantizer's codes exactly (zero corrections), including
+    signed zeros, saturated blocks and all-zero blocks, and its x_hat equals
+    the full record's replay."""
+    x = _act(48, 64, 31)
+    x[3, :16] = 0.0
+    x[4, :16] = -0.0
+    x[5, 16:32] = 1e-30
+    c, s, g = Q.quantize(x)
+    bits = TR.direction_bits(x, c, s, np.full(48, g))
+    c2, x_hat, corr = TR.replay_direction(bits, s, np.full(48, g), x)
+    assert np.array_equal(c2, c) and corr == 0
+    chan = np.array([5, 17, 40, -1])
+    resid = Q.residual_channels(x, c, s, g, chan)
+    _, xh_c, _ = TR.replay_direction(bits, s, np.full(48, g), x, chan, resid)
+    xr, _, _ = TR.replay_tensor(TR.export_tensor(c, s, g, chan=chan, resid=resid))
+    assert np.array_equal(xh_c, xr)
+
+
+def pin_direction_guided_is_a_neighbour():
+    """Brute force on a drifted input: each guided magnitude is the level at
+    or below the trainer's |y_t| or the next one up, and it equals the
+    rollout's code wherever both values lie between the same two levels."""
+    x = _act(32, 64, 32)
+    c, s, g = Q.quantize(x)
+    xt = F.bf16_rne(F.f32(x * (1 + 0.05 * RNG.standard_normal(x.shape))))
+    bits = TR.direction_bits(x, c, s, np.full(32, g))
+    c2, _, _ = TR.replay_direction(bits, s, np.full(32, g), xt)
+    S = np.repeat(F.f32(F.e4m3_value(s) * g), 16, axis=1)
+    yt = F.f32(xt * F.f32(1.0 / np.where(S > 0, S, 1.0)))
+    yr = F.f32(x * F.f32(1.0 / np.where(S > 0, S, 1.0)))
+    lv = F.E2M1_LEVELS
+    for i, j in itertools.product(range(32), range(64)):
+        if S[i, j] == 0:
+            continue
+        fl_t = max(k for k in range(8) if lv[k] <= abs(yt[i, j]))
+        fl_r = max(k for k in range(8) if lv[k] <= abs(yr[i, j]))
+        assert (c2[i, j] & 7) in (fl_t, min(fl_t + 1, 7))
+        if fl_t == fl_r and np.signbit(yt[i, j]) == np.signbit(yr[i, j]):
+            assert c2[i, j] == c[i, j], (i, j)
+
+
 # ------------------------------------------------------------------ stack
 
 

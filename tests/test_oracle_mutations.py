@@ -6,6 +6,7 @@ import pytest
 from oracle import formats as F
 from oracle import moe as M
 from oracle import nvfp4 as Q
+from oracle import trace as TR
 from tests import oracle_pins as P
 
 
@@ -111,6 +112,16 @@ def _div_instead_of_recip(x, g):
     return codes, s
 
 
+def _floor_level_left(a):
+    # an off-by-one at exact grid points: the level strictly below a
+    from oracle import formats as FF
+    return np.clip(np.searchsorted(FF.E2M1_LEVELS, a, side="left") - 1, 0, 7)
+
+
+def _guided_ignores_bit(bits, scales, g_rows, x_train, chan=None, resid=None):
+    return TR.__dict__["_orig_replay_dir"](np.zeros_like(bits), scales, g_rows, x_train, chan, resid)
+
+
 MUTATIONS = {
     "e2m1_ties_away": [(F, "e2m1_rne_code", _e2m1_ties_up), (Q, "e2m1_rne_code", _e2m1_ties_up)],
     "e2m1_drops_sign": [(F, "e2m1_rne_code", _e2m1_no_sign), (Q, "e2m1_rne_code", _e2m1_no_sign)],
@@ -127,6 +138,9 @@ MUTATIONS = {
     "swiglu_gate_up_swapped": [(M, "swiglu", _swiglu_wrong)],
     "nibble_order": [(F, "pack_nibbles", _pack_swapped)],
     "channel_ties_to_high_index": [(Q, "select_channels", _select_ties_high)],
+    "direction_floor_off_by_one": [(TR, "_floor_level_index", _floor_level_left)],
+    "direction_bit_ignored": [(TR, "_orig_replay_dir", TR.replay_direction),
+                              (TR, "replay_direction", _guided_ignores_bit)],
     "element_scale_dropped_factor": [(Q, "_orig_qws", Q.quantize_with_scale),
                                      (Q, "quantize_with_scale", _div_instead_of_recip)],
 }
