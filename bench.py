@@ -82,6 +82,7 @@ KERNEL_SOURCES = {
     "grouped_gemm.cu": ("gemm_gate_up", "gemm_gate_up_swiglu", "gemm_gate_up_swiglu_quant", "gemm_down"),
     "moe_route.cu": ("router_topk", "permute", "gather", "swiglu", "combine"),
     "trace_record.cu": ("export", "replay_x", "replay_h"),
+    "trace_direction.cu": ("direction_bits", "direction_replay"),
 }
 
 
@@ -230,11 +231,24 @@ def quantize_replay_sweep(dev, hbm_gbs, reps=10):
         tr = timed(r)
         torch.cuda.synchronize()
         assert int(status.item()) == 0 and int(counts[0].item()) == 0, "replay of the rollout's own input"
+        # compact record: direction bits from x and its codes (2 + 0.5 + 1/16 B in,
+        # 1/8 B out), guided replay (1/8 + 1/16 + 2 B in, 2 B out)
+        bits = torch.empty(rows, K // 8, dtype=torch.uint8, device=dev)
+        td = timed(lambda: B.trace_direction_bits(x, codes, scales, B.SCALES_LINEAR, g, bits=bits))
+        corr = torch.zeros(1, dtype=torch.int64, device=dev)
+        tg = timed(lambda: B.trace_replay_direction(bits, scales, B.SCALES_LINEAR, g, x, x_hat=x_hat,
+                                                    corrections=corr))
+        torch.cuda.synchronize()
+        assert int(corr.item()) == 0, "guided replay of the rollout's own input"
         gq = n * (2 + 0.5625) / (tq * 1e-3) / 1e9
         gr = n * (0.5625 + 2 + 2) / (tr * 1e-3) / 1e9
+        gd = n * (2 + 0.5625 + 0.125) / (td * 1e-3) / 1e9
+        gg = n * (0.125 + 0.0625 + 2 + 2) / (tg * 1e-3) / 1e9
         out.append({"elements": n, "quantize_us": tq * 1e3, "quantize_gbs": gq, "quantize_frac": gq / hbm_gbs,
-                    "replay_us": tr * 1e3, "replay_gbs": gr, "replay_frac": gr / hbm_gbs})
-        del x, codes, scales, record, x_hat
+                    "replay_us": tr * 1e3, "replay_gbs": gr, "replay_frac": gr / hbm_gbs,
+                    "direction_bits_us": td * 1e3, "direction_bits_frac": gd / hbm_gbs,
+                    "direction_replay_us": tg * 1e3, "direction_replay_frac": gg / hbm_gbs})
+        del x, codes, scales, record, x_hat, bits
         torch.cuda.empty_cache()
     return out
 

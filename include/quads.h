@@ -421,6 +421,46 @@ int trace_replay_qrecord(const void* record, size_t record_bytes, int layer_id, 
                          uint16_t* x_hat, unsigned long long* counts, int32_t* status,
                          quads_stream_t stream);
 
+/* ------------------------------- compact record: rounding directions
+ * [TRACE] "Fonctionnement, côté ingénierie": on a block-scaled FP4 grid each
+ * value's rounding (up to the grid point above or down to the one below) is
+ * a discrete choice, and the trainer uses the rollout's record to make the
+ * same choice; [TRACE] "L'idée centrale": the cache is kept small.
+ *
+ * One bit per element replaces the 4-bit code; the block scales and the
+ * per-tensor scale(s) are kept as they are.  With S = fp32(val(s) g) and
+ * y = fp32(x * fp32(1/S)), level(y) is the index (0..7) of the largest E2M1
+ * level (0, .5, 1, 1.5, 2, 3, 4, 6) at or below |y|.
+ *
+ * trace_direction_bits: bit = 1 where the rollout's code magnitude index is
+ * above level(y) of its own input x (it rounded up), else 0; 0 in blocks
+ * with S == 0.  x [rows][K] BF16 and codes [rows][K/2] are the rollout's
+ * quantizer input and output, scales are in scale_layout, g is device
+ * float[n_groups] over row groups (group_off as in quads_quantize_nvfp4;
+ * rows past group_off[n_groups] are skipped).  bits: device [rows][K/8],
+ * element 8j + i in bit i of byte j.
+ *
+ * trace_replay_direction: the trainer's guided rounding of x_train:
+ * code = sign(y_t) | min(level(y_t) + bit, 7) (signed zeros where S == 0),
+ * x_hat = bf16(fp32(val(code) val(s) g)), and on the compensation channels
+ * chan (ascending valid channels first, then -1) x_hat = bf16(fp32(deq) + r)
+ * with r = resid [rows][n_chan] BF16.  codes_out (nullable) receives the
+ * guided codes [rows][K/2]; *corrections (device u64, nullable, accumulated)
+ * counts the elements where the guided code differs from the trainer's own
+ * nearest-even rounding with the recorded scale.  Where x_train lies between
+ * the same two levels as the rollout's x, the guided code is the rollout's.
+ * K % 16 == 0, n_groups <= 1024, n_chan <= 256; x, x_train, x_hat 16-byte
+ * aligned, codes 8-byte, bits 2-byte. */
+int trace_direction_bits(const uint16_t* x, int64_t rows, int64_t K, const uint8_t* codes,
+                         const uint8_t* scales, int scale_layout, const float* g,
+                         const int32_t* group_off, int n_groups, uint8_t* bits,
+                         quads_stream_t stream);
+int trace_replay_direction(const uint8_t* bits, const uint8_t* scales, int scale_layout,
+                           const float* g, const int32_t* group_off, int n_groups, int64_t rows,
+                           int64_t K, const uint16_t* x_train, const int32_t* chan, int n_chan,
+                           const uint16_t* resid, uint16_t* x_hat, uint8_t* codes_out,
+                           unsigned long long* corrections, quads_stream_t stream);
+
 /* ------------------------------------------------------ layer stacking
  * The pages describe the MoE layer, not the model around it; a stack of
  * layers is joined here in the plainest way: x_{l+1} = x_l + MoE_l(x_l), and

@@ -6,6 +6,7 @@ import torch
 
 from oracle import formats as F
 from oracle import moe as M
+from oracle import nvfp4 as Q
 from oracle import stack as S
 from tests.helpers import assert_bits_equal, bf16_np, bf16_torch, f32_of
 from train_alignment_b200 import stack as ST
@@ -76,3 +77,39 @@ def test_stack_alignment_pass(cuda_lib):
         torch.cuda.synchronize()
         assert int(layer.status.item()) == 0
         assert f32_of(layer.counts).astype(np.int64).tolist() == [0, 0], l
+
+
+@pytest.mark.parametrize("rows,K", [(2048, 1024), (77, 512), (1, 64)])
+def test_activation_fakequant_matches_oracle(cuda_lib, rows, K):
+    """The symmetric W4A4 trainer's activation fake-quant (one per-tensor
+    scale, the device fake-quant kernel on a single matrix) against the
+    oracle's, bit for bit; the straight-through backward passes the gradient
+    through unchanged."""
+    r = np.random.default_rng(rows + K)
+    x = F.bf16_rne((r.standard_normal((rows, K)) * np.exp(r.standard_normal((1, K)))).astype(np.float32))
+    xt = bf16_torch(x)
+    x_fq, _, _, g, _ = cuda_lib.fakequant_weight_ste(xt.unsqueeze(0), want_codes=False)
+    gy = W.random_bf16((rows, K), 3, 1.0, "cuda")
+    gx = cuda_lib.fakequant_weight_ste_backward(gy)
+    torch.cuda.synchronize()
+    ref, _, _, g_ref = Q.fakequant_weight(x)
+    assert_bits_equal(F.bf16_bits(bf16_np(x_fq[0])), F.bf16_bits(ref), "x_fq")
+    assert np.float32(f32_of(g)[0]) == np.float32(g_ref)
+    assert_bits_equal(F.bf16_bits(bf16_np(gx)), F.bf16_bits(bf16_np(gy)), "STE backward")
+
+
+def test_stack_w4a4_trainer_gap(cuda_lib):
+    """The symmetric W4A4 QAT trainer (activations fake-quantized too, no
+    compensation, no replay) on the same 8-layer stack and rollout: the pass
+    runs and its per-token gap is reported next to the replayed trainer's
+    (a diagnostic; the pages' claim is about training, which is not run)."""
+    cfg = W.CONFIGS["stack8_t4096_h2048_e64k4_f1024"]
+    st = ST.LayerStack(cfg, seed=0, device="cuda")
+    gap_q, _, _ = st.alignment_pass(drift=1e-3)
+    gap_w4, cm, sm = st.alignment_pass(drift=1e-3, w4a4=True)
+    torch.cuda.synchronize()
+    assert cuda_lib.device_status() == cuda_lib.OK
+    gq, gw = gap_q.cpu().numpy(), gap_w4.cpu().numpy()
+    assert np.all(np.isfinite(gw)) and (cm, sm) == (0, 0)
+    print(f"per-token gap, replayed trainer: median {np.median(gq):.4f}; W4A4 QAT trainer: median "
+          f"{np.median(gw):.4f}, p90 {np.percentile(gw, 90):.4f}")

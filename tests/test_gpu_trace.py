@@ -126,3 +126,96 @@ def test_bounded_wait_times_out_and_context_survives(cuda_lib):
     codes, scales, g, _ = cuda_lib.quantize_nvfp4(x)
     torch.cuda.synchronize()
     assert float(g.item()) == np.float32(1.0 / 2688.0)
+
+
+# ------------------------------------------- compact rounding-direction record
+
+
+def _direction_case(rows, K, groups, n_chan, tiled, seed, drift=0.05):
+    """Rollout input x (outlier channels, a zero block, a negative-zero
+    block), quantized by the oracle (per group when groups is given), the
+    trainer's drifted copy, and a channel set."""
+    r = np.random.default_rng(seed)
+    x = r.standard_normal((rows, K)) * np.exp(0.5 * r.standard_normal((1, K)))
+    x[:, r.choice(K, 2, replace=False)] *= 30
+    if rows > 2:
+        x[1, :16] = 0.0
+        x[2, 16:32] = -0.0
+    x = F.bf16_rne(x.astype(np.float32))
+    if groups is None:
+        off = np.array([0, rows])
+        c, s, g = Q.quantize(x)
+        gs = np.array([g])
+    else:
+        off = np.asarray(groups)
+        c, s, gs = Q.quantize_grouped(x[:off[-1]], off)
+        c = np.concatenate([c, np.zeros((rows - off[-1], K), np.uint8)])
+        s = np.concatenate([s, np.zeros((rows - off[-1], K // 16), np.uint8)])
+    g_rows = np.zeros(rows)
+    for i in range(len(off) - 1):
+        g_rows[off[i]:off[i + 1]] = gs[i]
+    xt = F.bf16_rne(F.f32(x * (1 + drift * r.standard_normal(x.shape))))
+    chan = Q.pad_channels(np.sort(r.choice(K, n_chan - 3, replace=False))) if n_chan else None
+    resid = None
+    if n_chan:
+        resid = np.zeros((rows, len(chan)))
+        for i in range(len(off) - 1):
+            lo, hi = off[i], off[i + 1]
+            if hi > lo:
+                resid[lo:hi] = Q.residual_channels(x[lo:hi], c[lo:hi], s[lo:hi], gs[i], chan)
+    return dict(x=x, xt=xt, c=c, s=s, gs=gs, g_rows=g_rows, off=off, R=int(off[-1]), chan=chan, resid=resid,
+                tiled=tiled, grouped=groups is not None)
+
+
+def _gpu_direction(lib, d):
+    dev = "cuda"
+    rows, K = d["x"].shape
+    layout = lib.SCALES_TILED if d["tiled"] else lib.SCALES_LINEAR
+    scales = F.scales_to_tiled(d["s"]) if d["tiled"] else d["s"]
+    sc = torch.from_numpy(np.ascontiguousarray(scales)).to(dev)
+    g = torch.tensor(d["gs"], dtype=torch.float32, device=dev)
+    goff = torch.from_numpy(d["off"].astype(np.int32)).to(dev) if d["grouped"] else None
+    n = len(d["gs"])
+    bits = torch.full((rows, K // 8), 0xA5, dtype=torch.uint8, device=dev)
+    cuda_lib_bits = lib.trace_direction_bits(bf16_torch(d["x"]), torch.from_numpy(F.pack_nibbles(d["c"])).to(dev),
+                                             sc, layout, g, group_off=goff, n_groups=n, bits=bits)
+    codes = torch.full((rows, K // 2), 0xA5, dtype=torch.uint8, device=dev)
+    corr = torch.zeros(1, dtype=torch.int64, device=dev)
+    x_hat = torch.full((rows, K), float("nan"), dtype=torch.bfloat16, device=dev)
+    chan = torch.from_numpy(d["chan"]).to(dev) if d["chan"] is not None else None
+    resid = bf16_torch(d["resid"]) if d["chan"] is not None else None
+    lib.trace_replay_direction(cuda_lib_bits, sc, layout, g, bf16_torch(d["xt"]), group_off=goff, n_groups=n,
+                               chan=chan, resid=resid, x_hat=x_hat, codes_out=codes, corrections=corr)
+    torch.cuda.synchronize()
+    assert lib.device_status() == lib.OK
+    return cuda_lib_bits.cpu().numpy(), codes.cpu().numpy(), bf16_np(x_hat), int(corr.item())
+
+
+@pytest.mark.parametrize("rows,K,groups,n_chan,tiled", [
+    (64, 64, None, 0, False),                          # one pass, one group
+    (333, 1040, None, 32, False),                      # ragged rows, 65 blocks: a partial third pass
+    (768, 512, [0, 128, 128, 384, 640], 16, True),     # expert-ordered h: an empty expert, padding rows past the last
+    (2048, 1024, None, 32, False),                     # the 2048-token layer input, full size
+])
+def test_direction_record_parity(cuda_lib, rows, K, groups, n_chan, tiled):
+    """The compact record's bits bit for bit against the oracle's, and the
+    trainer's guided codes, replayed operand and correction count against
+    the oracle's replay of the same bits; rows past the last group are left
+    untouched."""
+    d = _direction_case(rows, K, groups, n_chan, tiled, seed=rows + K)
+    bits, codes, x_hat, corr = _gpu_direction(cuda_lib, d)
+    R = d["R"]
+    b_ref = TR.direction_bits(d["x"][:R], d["c"][:R], d["s"][:R], d["g_rows"][:R])
+    assert_bits_equal(bits[:R], TR.pack_bits(b_ref), "direction bits")
+    assert np.all(bits[R:] == 0xA5), "rows past the last group must be untouched"
+    c_ref, xh_ref, corr_ref = TR.replay_direction(b_ref, d["s"][:R], d["g_rows"][:R], d["xt"][:R],
+                                                  d["chan"], d["resid"][:R] if d["resid"] is not None else None)
+    assert_bits_equal(codes[:R], F.pack_nibbles(c_ref), "guided codes")
+    assert_bits_equal(F.bf16_bits(x_hat[:R]), F.bf16_bits(xh_ref), "x_hat")
+    assert corr == corr_ref
+    assert np.all(np.isnan(x_hat[R:]))
+    # the rollout's own input replays its codes exactly
+    d0 = dict(d, xt=d["x"])
+    _, codes0, _, corr0 = _gpu_direction(cuda_lib, d0)
+    assert_bits_equal(codes0[:R], F.pack_nibbles(d["c"][:R]), "self-replay codes")
+    assert corr0 == 0

@@ -99,6 +99,9 @@ _SIGS = {
     "trace_qrecord_layout": (c_sz, [c_i32, c_i64, c_i32, c_vp, c_i32, c_vp]),
     "trace_export_qrecord": (c_i32, [c_i32, c_i64, c_i32, c_vp, c_vp, c_i32, c_vp, c_sz, c_vp]),
     "trace_replay_qrecord": (c_i32, [c_vp, c_sz, c_i32, c_i32, c_i64, c_i64, c_vp, c_vp, c_vp, c_vp, c_vp]),
+    "trace_direction_bits": (c_i32, [c_vp, c_i64, c_i64, c_vp, c_vp, c_i32, c_vp, c_vp, c_i32, c_vp, c_vp]),
+    "trace_replay_direction": (c_i32, [c_vp, c_vp, c_i32, c_vp, c_vp, c_i32, c_i64, c_i64, c_vp, c_vp, c_i32, c_vp,
+                                       c_vp, c_vp, c_vp, c_vp]),
 }
 
 
@@ -488,6 +491,31 @@ def trace_replay_qrecord(record, layer_id, which, rows, K, x_train=None, x_hat=N
 
 
 # ------------------------------------------------------------ layer stacking
+
+
+def trace_direction_bits(x, codes, scales, scale_layout, g, group_off=None, n_groups=1, bits=None):
+    """One rounding-direction bit per element of the rollout's quantization
+    of x: returns bits [rows, K/8] u8."""
+    _dev(x, torch.bfloat16, "x")
+    rows, K = x.shape
+    bits = bits if bits is not None else _empty((rows, K // 8), torch.uint8, x.device)
+    _check(load().trace_direction_bits(_p(x), rows, K, _p(codes), _p(scales), scale_layout, _p(g), _p(group_off),
+                                       n_groups, _p(bits), _s()), "trace_direction_bits")
+    return bits
+
+
+def trace_replay_direction(bits, scales, scale_layout, g, x_train, group_off=None, n_groups=1, chan=None,
+                           resid=None, x_hat=None, codes_out=None, corrections=None):
+    """The trainer's rounding of x_train guided by the recorded directions.
+    Returns (x_hat, codes_out or None, corrections or None)."""
+    _dev(x_train, torch.bfloat16, "x_train")
+    rows, K = x_train.shape
+    n_chan = 0 if chan is None else int(chan.numel())
+    x_hat = x_hat if x_hat is not None else _empty((rows, K), torch.bfloat16, x_train.device)
+    _check(load().trace_replay_direction(_p(bits), _p(scales), scale_layout, _p(g), _p(group_off), n_groups, rows, K,
+                                         _p(x_train), _p(chan), n_chan, _p(resid) if n_chan else None, _p(x_hat),
+                                         _p(codes_out), _p(corrections), _s()), "trace_replay_direction")
+    return x_hat, codes_out, corrections
 
 
 def router_logits(x, w_r, out=None):

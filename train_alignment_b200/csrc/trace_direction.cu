@@ -1,0 +1,290 @@
+// Compact TRACE record: one rounding-direction bit per element in place of
+// the 4-bit code, and the trainer's rounding guided by it.
+//
+// Method: [TRACE] "Fonctionnement, côté ingénierie" -- on a block-scaled FP4
+// grid the rounding of each value is a discrete choice (up to the grid point
+// above, or down to the one below); the trainer reads the rollout's record
+// and uses it to make the same choice.  [TRACE] "L'idée centrale" -- the
+// cache keeps the mantissa and the scale factors selectively, to save memory.
+//
+// For an element with block scale S = fp32(val(s) g) and y = fp32(x fp32(1/S)):
+//   level(y) = index of the largest E2M1 level <= |y| (0 .. 7; 7 = 6.0);
+//   rollout bit = 1 if its code's magnitude index is above level(y), else 0;
+//   trainer code = sign(y_t) | min(level(y_t) + bit, 7).
+// Blocks with S == 0 record 0 and replay signed zeros (the quantizer's rule).
+// The trainer keeps the recorded block and per-tensor scales, so where both
+// values lie between the same two levels the guided code is the rollout's.
+//
+// Both kernels: one warp per row, lane = 16-element block, 32 blocks per pass;
+// HBM-bound streams (direction: 2 + 0.5 B read, 0.125 B written per element;
+// replay: 2 + 0.125 B read, 2 (+ 0.5) B written).
+#include "common.cuh"
+
+namespace quads {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kMaxGroups = 1024;
+constexpr int kMaxChan = 256;
+
+struct DirArgs {
+  const uint16_t* x;          // rollout input (bits) or trainer input (replay)
+  const uint8_t* codes;       // rollout codes (bits) or null
+  const uint8_t* scales;
+  int tiled;
+  const float* g;
+  const int32_t* group_off;
+  int n_groups;
+  FastDiv uniform;            // rows per group without group_off
+  int64_t rows, K;
+  uint8_t* bits;              // written (bits) / read (replay)
+  // replay only
+  const int32_t* chan;
+  int n_chan;
+  const uint16_t* resid;
+  uint16_t* x_hat;
+  uint8_t* codes_out;
+  unsigned long long* corrections;
+};
+
+// Index of the largest E2M1 level (0, .5, 1, 1.5, 2, 3, 4, 6) at or below a >= 0.
+__device__ __forceinline__ uint32_t floor_level(float a) {
+  return static_cast<uint32_t>(a >= 0.5f) + static_cast<uint32_t>(a >= 1.0f) + static_cast<uint32_t>(a >= 1.5f) +
+         static_cast<uint32_t>(a >= 2.0f) + static_cast<uint32_t>(a >= 3.0f) + static_cast<uint32_t>(a >= 4.0f) +
+         static_cast<uint32_t>(a >= 6.0f);
+}
+
+// Shared-memory group table; returns the number of rows that belong to a group.
+__device__ __forceinline__ int64_t load_groups(const DirArgs& a, int32_t* off_s, float* g_s) {
+  const int n = a.n_groups;
+  for (int i = threadIdx.x; i <= n; i += blockDim.x) {
+    off_s[i] = a.group_off ? a.group_off[i] : 0;
+    if (i < n) g_s[i] = a.g[i];
+  }
+  __syncthreads();
+  return a.group_off ? min(a.rows, static_cast<int64_t>(off_s[n])) : a.rows;
+}
+
+__global__ void __launch_bounds__(kThreads) direction_bits_kernel(DirArgs a) {
+  extern __shared__ int32_t smem[];
+  int32_t* off_s = smem;
+  float* g_s = reinterpret_cast<float*>(smem + a.n_groups + 1);
+  const int64_t rows = load_groups(a, off_s, g_s);
+  const RowGroups grp{a.group_off ? off_s : nullptr, a.n_groups, a.uniform};
+  const int64_t K = a.K;
+  const int nkb = static_cast<int>(K / 16);
+  const int64_t ncol_tiles = ceil_div(nkb, 4);
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
+       row += warps) {
+    const float g = g_s[grp.of(row)];
+    for (int kb = lane; kb < nkb; kb += 32) {
+      const uint32_t s = a.scales[a.tiled ? tiled_scale_offset(row, kb, ncol_tiles) : row * nkb + kb];
+      const float2 e = scale_table_entry(s, g);
+      uint32_t out = 0;
+      if (e.x != 0.0f) {
+        uint32_t w[8];
+        load_bf16x16(a.x + row * K + kb * 16, w);
+        const uint2 c = __ldg(reinterpret_cast<const uint2*>(a.codes + row * (K / 2) + kb * 8));
+        const uint64_t inv2 = pack_f32x2(e.y, e.y);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint64_t y = fmul2_rn(bf16x2_to_f32x2(w[i]), inv2);
+          const uint32_t cw = (i < 4) ? c.x : c.y;
+          const uint32_t c0 = (cw >> (8 * (i & 3))) & 7u, c1 = (cw >> (8 * (i & 3) + 4)) & 7u;
+          out |= static_cast<uint32_t>(c0 > floor_level(fabsf(lo_f32(y)))) << (2 * i);
+          out |= static_cast<uint32_t>(c1 > floor_level(fabsf(hi_f32(y)))) << (2 * i + 1);
+        }
+      }
+      *reinterpret_cast<uint16_t*>(a.bits + row * (K / 8) + kb * 2) = static_cast<uint16_t>(out);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads) replay_direction_kernel(DirArgs a) {
+  extern __shared__ int32_t smem[];
+  const int n = a.n_groups;
+  const int64_t K = a.K;
+  const int nkb = static_cast<int>(K / 16);
+  const int npass = (nkb + 31) / 32;
+  int32_t* off_s = smem;                                      // n + 1
+  float* g_s = reinterpret_cast<float*>(smem + n + 1);        // n
+  int32_t* pass_slot = smem + 2 * n + 1;                      // npass + 1
+  int32_t* chan_s = pass_slot + npass + 1;                    // n_chan
+  for (int j = threadIdx.x; j < a.n_chan; j += blockDim.x) chan_s[j] = a.chan[j];
+  __syncthreads();
+  for (int p = threadIdx.x; p <= npass && a.n_chan; p += blockDim.x) {
+    int cnt = 0;                 // valid channels (ascending, first) below column 512 p
+    for (int j = 0; j < a.n_chan; ++j) cnt += (chan_s[j] >= 0 && chan_s[j] < K && chan_s[j] < 512 * p) ? 1 : 0;
+    pass_slot[p] = cnt;
+  }
+  const int64_t rows = load_groups(a, off_s, g_s);
+  const RowGroups grp{a.group_off ? off_s : nullptr, n, a.uniform};
+  const int64_t ncol_tiles = ceil_div(nkb, 4);
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  unsigned long long fixes = 0;
+  for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
+       row += warps) {
+    const float g = g_s[grp.of(row)];
+    for (int p = 0; p < npass; ++p) {
+      const int kb = p * 32 + lane;
+      QCore q{0u, 0u, 0u, 0.0f};
+      if (kb < nkb) {
+        const uint32_t s = a.scales[a.tiled ? tiled_scale_offset(row, kb, ncol_tiles) : row * nkb + kb];
+        const float2 e = scale_table_entry(s, g);
+        const uint32_t bits = *reinterpret_cast<const uint16_t*>(a.bits + row * (K / 8) + kb * 2);
+        uint32_t w[8];
+        load_bf16x16(a.x + row * K + kb * 16, w);
+        q.scale = s;
+        q.sv = e4m3_value(s);
+        if (e.x == 0.0f) {
+          // signed zeros, as the quantizer writes for a zero block scale
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            q.lo |= ((w[i] >> 15) & 1u) << (8 * i + 3) | ((w[i] >> 31) & 1u) << (8 * i + 7);
+            q.hi |= ((w[4 + i] >> 15) & 1u) << (8 * i + 3) | ((w[4 + i] >> 31) & 1u) << (8 * i + 7);
+          }
+        } else {
+          const uint64_t inv2 = pack_f32x2(e.y, e.y);
+          uint64_t y[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) y[i] = fmul2_rn(bf16x2_to_f32x2(w[i]), inv2);
+          const uint32_t own_lo = e2m1x8_from_pairs(y), own_hi = e2m1x8_from_pairs(y + 4);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float v = (i & 1) ? hi_f32(y[i >> 1]) : lo_f32(y[i >> 1]);
+            const uint32_t lvl = min(floor_level(fabsf(v)) + ((bits >> i) & 1u), 7u);
+            const uint32_t code = lvl | ((__float_as_uint(v) >> 31) << 3);
+            const uint32_t own = (((i < 8) ? own_lo : own_hi) >> (4 * (i & 7))) & 7u;
+            fixes += (own != lvl) ? 1u : 0u;
+            if (i < 8) q.lo |= code << (4 * i); else q.hi |= code << (4 * (i - 8));
+          }
+        }
+        uint32_t o[8];
+        deq_block_bf16(q, g, 1, o);
+        uint4* dst = reinterpret_cast<uint4*>(a.x_hat + row * K + kb * 16);
+        dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+        dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+        if (a.codes_out) *reinterpret_cast<uint2*>(a.codes_out + row * (K / 2) + kb * 8) = make_uint2(q.lo, q.hi);
+      }
+      if (a.n_chan) {
+        // compensation channels of this pass: x_hat = bf16(fp32(deq) + r)
+        __syncwarp();
+        const int slo = pass_slot[p], shi = pass_slot[p + 1];
+        for (int j0 = slo; j0 < shi; j0 += 32) {              // warp-uniform
+          const int j = j0 + lane;
+          const bool act = j < shi;
+          const int c = act ? chan_s[j] : 512 * p;
+          const int src = (c - 512 * p) >> 4, bit = c & 15;
+          const uint32_t cl = __shfl_sync(0xffffffffu, q.lo, src);
+          const uint32_t ch = __shfl_sync(0xffffffffu, q.hi, src);
+          const float sv = __shfl_sync(0xffffffffu, q.sv, src);
+          if (act) {
+            const uint32_t code = (((bit < 8) ? cl : ch) >> (4 * (bit & 7))) & 15u;
+            const float v = __fadd_rn(deq_f32(code, sv, g), bf16_bits_to_float(a.resid[row * a.n_chan + j]));
+            a.x_hat[row * K + c] = static_cast<uint16_t>(float_to_bf16_bits(v));
+          }
+        }
+        __syncwarp();
+      }
+    }
+  }
+  if (a.corrections) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) fixes += __shfl_xor_sync(0xffffffffu, fixes, o);
+    if (lane == 0 && fixes) atomicAdd(a.corrections, fixes);
+  }
+}
+
+int check_common(int64_t rows, int64_t K, const uint8_t* scales, int scale_layout, const float* g,
+                 const int32_t* group_off, int n_groups) {
+  QUADS_REQUIRE(rows >= 0 && K > 0 && K % 16 == 0 && K <= 65536, QUADS_ERR_UNSUPPORTED_SHAPE,
+                "K must be a positive multiple of 16 up to 65536");
+  QUADS_REQUIRE(rows * (K / 16) < (int64_t(1) << 31), QUADS_ERR_UNSUPPORTED_SHAPE, "tensor above 2^31 blocks");
+  QUADS_REQUIRE(scale_layout == QUADS_SCALES_LINEAR || scale_layout == QUADS_SCALES_TILED, QUADS_ERR_INVALID_ARG,
+                "unknown scale layout");
+  QUADS_REQUIRE(n_groups >= 1 && n_groups <= kMaxGroups, QUADS_ERR_UNSUPPORTED_SHAPE, "n_groups must be in [1, %d]",
+                kMaxGroups);
+  QUADS_REQUIRE(group_off || rows % n_groups == 0, QUADS_ERR_INVALID_ARG,
+                "without group offsets, rows must be a multiple of n_groups");
+  QUADS_REQUIRE(rows == 0 || (scales && g), QUADS_ERR_INVALID_ARG, "scales and g must be non-null");
+  return QUADS_OK;
+}
+
+DirArgs base_args(int64_t rows, int64_t K, const uint8_t* scales, int scale_layout, const float* g,
+                  const int32_t* group_off, int n_groups) {
+  DirArgs a{};
+  a.scales = scales;
+  a.tiled = scale_layout == QUADS_SCALES_TILED;
+  a.g = g;
+  a.group_off = group_off;
+  a.n_groups = n_groups;
+  a.uniform = make_fastdiv(static_cast<uint32_t>(n_groups > 1 && !group_off ? rows / n_groups : 1));
+  a.rows = rows;
+  a.K = K;
+  return a;
+}
+
+}  // namespace
+}  // namespace quads
+
+using namespace quads;
+
+extern "C" {
+
+int trace_direction_bits(const uint16_t* x, int64_t rows, int64_t K, const uint8_t* codes, const uint8_t* scales,
+                         int scale_layout, const float* g, const int32_t* group_off, int n_groups, uint8_t* bits,
+                         quads_stream_t stream) {
+  clear_error();
+  QUADS_TRY(check_common(rows, K, scales, scale_layout, g, group_off, n_groups));
+  if (rows == 0) return QUADS_OK;
+  QUADS_REQUIRE(x && codes && bits && aligned(x, 16) && aligned(codes, 8) && aligned(bits, 2), QUADS_ERR_INVALID_ARG,
+                "x (16-byte aligned), codes (8) and bits (2) must be non-null and aligned");
+  DirArgs a = base_args(rows, K, scales, scale_layout, g, group_off, n_groups);
+  a.x = x;
+  a.codes = codes;
+  a.bits = bits;
+  const size_t smem = (2 * static_cast<size_t>(n_groups) + 1) * 4;
+  const int grid = persistent_grid(reinterpret_cast<const void*>(direction_bits_kernel), kThreads, smem,
+                                   ceil_div(rows, kThreads / 32));
+  direction_bits_kernel<<<grid, kThreads, smem, stream>>>(a);
+  count_launches(1);
+  return check_launch("direction_bits_kernel");
+}
+
+int trace_replay_direction(const uint8_t* bits, const uint8_t* scales, int scale_layout, const float* g,
+                           const int32_t* group_off, int n_groups, int64_t rows, int64_t K, const uint16_t* x_train,
+                           const int32_t* chan, int n_chan, const uint16_t* resid, uint16_t* x_hat,
+                           uint8_t* codes_out, unsigned long long* corrections, quads_stream_t stream) {
+  clear_error();
+  QUADS_TRY(check_common(rows, K, scales, scale_layout, g, group_off, n_groups));
+  QUADS_REQUIRE(n_chan >= 0 && n_chan <= kMaxChan, QUADS_ERR_UNSUPPORTED_SHAPE, "n_chan must be in [0, %d]",
+                kMaxChan);
+  QUADS_REQUIRE(n_chan == 0 || (chan && resid), QUADS_ERR_INVALID_ARG, "chan and resid required with n_chan > 0");
+  if (rows == 0) return QUADS_OK;
+  QUADS_REQUIRE(bits && x_train && x_hat && aligned(bits, 2) && aligned(x_train, 16) && aligned(x_hat, 16) &&
+                    (!codes_out || aligned(codes_out, 8)),
+                QUADS_ERR_INVALID_ARG, "bits (2), x_train and x_hat (16), codes_out (8): non-null and aligned");
+  DirArgs a = base_args(rows, K, scales, scale_layout, g, group_off, n_groups);
+  a.x = x_train;
+  a.bits = const_cast<uint8_t*>(bits);
+  a.chan = chan;
+  a.n_chan = n_chan;
+  a.resid = resid;
+  a.x_hat = x_hat;
+  a.codes_out = codes_out;
+  a.corrections = corrections;
+  const size_t smem = (2 * static_cast<size_t>(n_groups) + 1 + (K / 16 + 31) / 32 + 1 + n_chan) * 4;
+  if (smem > 48 * 1024 && cudaFuncSetAttribute(replay_direction_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(smem)) != cudaSuccess)
+    return set_error(QUADS_ERR_CUDA, "cannot raise shared memory of replay_direction_kernel");
+  const int grid = persistent_grid(reinterpret_cast<const void*>(replay_direction_kernel), kThreads, smem,
+                                   ceil_div(rows, kThreads / 32));
+  replay_direction_kernel<<<grid, kThreads, smem, stream>>>(a);
+  count_launches(1);
+  return check_launch("replay_direction_kernel");
+}
+
+}  // extern "C"

@@ -20,6 +20,14 @@ The other layers route and compute on the trainer's own activations.  The
 trainer's expert FFNs are BF16 matmuls on W_fq (a plain library GEMM; the
 pages' trainer is a BF16 framework).  The per-token gap between the two
 sides' stack outputs is reported, not pinned.
+
+The symmetric W4A4 trainer ([QUADS-fr §2.2, ablation studies; §2.1]: QAT
+that fake-quantizes both weights and activations) is the ablation the pages
+report as drifting further than the asymmetric scheme: every
+layer fake-quantizes its input x (one per-tensor scale) and each expert's h
+(one scale per expert) on the NVFP4 grid, without compensation and without
+replay; its backward through those fake-quants is the same straight-through
+identity as for the weights.
 """
 import torch
 
@@ -70,17 +78,23 @@ class LayerStack:
             B.residual_add(self.x_roll[l], out, out=self.x_roll[l + 1])
         return self.x_roll[self.cfg.layers]
 
-    def _trainer_ffn(self, layer, x, idx, w):
+    def _trainer_ffn(self, layer, x, idx, w, w4a4=False):
         """BF16 MoE FFN of one layer with the fake-quantized weights:
-        y_t = sum_s w[t,s] W_d,fq[e] (silu(W_g,fq[e] x) * W_u,fq[e] x), e = idx[t,s]."""
+        y_t = sum_s w[t,s] W_d,fq[e] (silu(W_g,fq[e] x) * W_u,fq[e] x), e = idx[t,s].
+        w4a4: x (per tensor) and each expert's h (per expert) fake-quantized
+        too, by the device fake-quant kernel."""
         cfg = self.cfg
         y = torch.zeros(cfg.T, cfg.H, dtype=torch.float32, device=self.dev)
+        if w4a4:
+            x = B.fakequant_weight_ste(x.unsqueeze(0), want_codes=False)[0][0]
         flat = idx.reshape(-1).long()
         for e in torch.unique(flat).tolist():
             pos = (flat == e).nonzero().squeeze(1)
             t = pos // cfg.k
             gu = x[t] @ layer.w_gu_fq[e].t()
             h = (torch.nn.functional.silu(gu[:, :cfg.F].float()) * gu[:, cfg.F:].float()).to(torch.bfloat16)
+            if w4a4:
+                h = B.fakequant_weight_ste(h.unsqueeze(0).contiguous(), want_codes=False)[0][0]
             yd = (h @ layer.w_d_fq[e].t()).float()
             y.index_add_(0, t, yd * w.reshape(-1)[pos, None])
         return y.to(torch.bfloat16)
@@ -97,16 +111,17 @@ class LayerStack:
                 Y[off[e]:off[e + 1]] = layer.h_hat[off[e]:off[e + 1]] @ layer.w_d_fq[e].t()
         return B.moe_unpermute_combine(Y, layer.row_of, layer.topk_w, cfg.T, cfg.k, cfg.H)
 
-    def trainer(self, x0_train):
+    def trainer(self, x0_train, w4a4=False):
         """The trainer side through every layer; layer inputs in x_train[l].
         Recorded layers replay the record; returns (stack output, code
-        mismatches, scale mismatches) over the recorded layers."""
+        mismatches, scale mismatches) over the recorded layers.  w4a4: the
+        symmetric W4A4 QAT trainer instead (no replay; mismatches 0)."""
         cfg = self.cfg
         self.x_train[0].copy_(x0_train)
         code_mis = scale_mis = 0
         for l, layer in enumerate(self.layers):
             xl = self.x_train[l]
-            if self.is_recorded(l):
+            if self.is_recorded(l) and not w4a4:
                 layer.reset_counts()
                 layer.trainer_replay(xl, layer_id=l)
                 assert int(layer.status.item()) == 0 and int(layer.status_h.item()) == 0, "bad TRACE record"
@@ -117,18 +132,18 @@ class LayerStack:
             else:
                 B.router_logits(xl, self.w_r[l], out=self.logits)
                 idx, w = B.moe_router_topk(self.logits, cfg.k, True)
-                y = self._trainer_ffn(layer, xl, idx, w)
+                y = self._trainer_ffn(layer, xl, idx, w, w4a4)
             B.residual_add(xl, y, out=self.x_train[l + 1])
         return self.x_train[cfg.layers], code_mis, scale_mis
 
-    def alignment_pass(self, drift=1e-3, seed=0):
+    def alignment_pass(self, drift=1e-3, seed=0, w4a4=False):
         """One train/rollout alignment pass: rollout, then the trainer on the
         rollout's input plus N(0, drift) engine drift.  Returns the per-token
         relative gap between the two stack outputs (a reported diagnostic)
         and the mismatch counts of the replayed layers."""
         y_r = self.rollout(self.x0)
         x0_t = W.engine_drift(self.x0, drift, seed=seed, device=self.dev)
-        y_t, cm, sm = self.trainer(x0_t)
+        y_t, cm, sm = self.trainer(x0_t, w4a4=w4a4)
         a, b = y_r.float(), y_t.float()
         gap = torch.linalg.vector_norm(a - b, dim=1) / torch.linalg.vector_norm(b, dim=1).clamp_min(1e-30)
         return gap, cm, sm
