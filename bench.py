@@ -82,7 +82,6 @@ KERNEL_SOURCES = {
     "grouped_gemm.cu": ("gemm_gate_up", "gemm_gate_up_swiglu", "gemm_gate_up_swiglu_quant", "gemm_down"),
     "moe_route.cu": ("router_topk", "permute", "gather", "swiglu", "combine"),
     "trace_record.cu": ("export", "replay_x", "replay_h"),
-    "trace_direction.cu": ("direction_bits", "direction_replay"),
 }
 
 
