@@ -151,3 +151,59 @@ def per_token_gap(y_rollout, y_trainer):
 def bf16_out(v):
     """Round float64 results to BF16 via float32 (as a BF16 store does)."""
     return bf16_rne(f32(v))
+
+
+# ------------------------------------------- literal second quantization pass
+#
+# [QUADS-fr §2.2.B] / [QUADS-es §2.2.B] describe the compensation as a second
+# quantization pass over the high-residual channels whose correction is added
+# to the quantized output.  Here the residual R and the weight columns Wc are
+# themselves NVFP4-quantized and multiplied on the FP4 path.
+#
+# Reading (listed in DESIGN.md): Wc_e is quantized per expert with its own
+# amax (decode scale g_wc[e]); R is quantized per expert segment with the
+# decode scale derived from amax_r[e] = fp32(fp32(G_e / g_wc[e]) * 2688),
+# G_e = fp32(g_a g_w[e]), so that g_r g_wc equals G_e up to one rounding and
+# the correction shares the main product's per-tensor scale.  The block
+# scales of R carry its magnitude.  The layer output is then
+#   Y = G_e (deq_unit(A) . deq_unit(W_e)^T + deq_unit(q(R)) . deq_unit(q(Wc_e))^T),
+# one FP4 product over the channel-extended reduction axis.
+
+
+def fp4_comp_amax(g_a, g_w, g_wc):
+    """amax_r[e] = fp32(fp32(fp32(g_a g_w[e]) / g_wc[e]) * 2688), 0 where
+    g_wc[e] == 0."""
+    g_w = np.asarray(g_w, dtype=np.float64)
+    g_wc = np.asarray(g_wc, dtype=np.float64)
+    G = f32(np.broadcast_to(np.asarray(g_a, dtype=np.float64), g_w.shape) * g_w)
+    ratio = np.where(g_wc > 0, f32(G / np.where(g_wc > 0, g_wc, 1.0)), 0.0)
+    return f32(ratio * 2688.0)
+
+
+def fp4_compensation_operands(resid, wc, g_a, g_w, expert_off):
+    """NVFP4 operands of the FP4 correction: q(Wc_e) per expert (own amax)
+    and q(R) per expert segment with amax_r.  resid [R, nc] and wc [E, N, nc]
+    are BF16-exact values (nc a multiple of 16).  Returns (r_codes, r_scales,
+    g_r [E], wc_codes [E, N, nc], wc_scales [E, N, nc/16], g_wc [E])."""
+    from .nvfp4 import quantize, quantize_grouped
+    wc = np.asarray(wc, dtype=np.float64)
+    E = wc.shape[0]
+    q = [quantize(wc[e]) for e in range(E)]
+    wc_codes = np.stack([t[0] for t in q])
+    wc_scales = np.stack([t[1] for t in q])
+    g_wc = np.array([t[2] for t in q])
+    amax_r = fp4_comp_amax(g_a, g_w, g_wc)
+    r_codes, r_scales, g_r = quantize_grouped(resid, expert_off, amax=amax_r)
+    return r_codes, r_scales, g_r, wc_codes, wc_scales, g_wc
+
+
+def grouped_gemm_fp4_comp(a_codes, a_scales, g_a, w_codes, w_scales, g_w, expert_off, r_codes, r_scales,
+                          wc_codes, wc_scales):
+    """Y = G_e (A . W_e^T + q(R) . q(Wc_e)^T) on the NVFP4 values: the
+    grouped GEMM over the reduction axis extended by the channel columns.
+    Returns (Y, absdot) as grouped_gemm does."""
+    a_c = np.concatenate([np.asarray(a_codes), np.asarray(r_codes)], axis=1)
+    a_s = np.concatenate([np.asarray(a_scales), np.asarray(r_scales)], axis=1)
+    w_c = np.concatenate([np.asarray(w_codes), np.asarray(wc_codes)], axis=2)
+    w_s = np.concatenate([np.asarray(w_scales), np.asarray(wc_scales)], axis=2)
+    return grouped_gemm(a_c, a_s, g_a, w_c, w_s, g_w, expert_off)

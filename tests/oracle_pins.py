@@ -571,6 +571,47 @@ def pin_direction_guided_is_a_neighbour():
             assert c2[i, j] == c[i, j], (i, j)
 
 
+def pin_fp4_compensation_close_to_bf16():
+    """The FP4 correction against the BF16 one it stands for, with every
+    channel selected and Wc = deq(W): the BF16-compensated output is exactly
+    X . deq(W)^T (a closed form), and the FP4-compensated output stays within
+    the NVFP4 errors of R and Wc: |sum r wc - sum q(r) q(wc)| <=
+    sum |r - q(r)| |wc| + |q(r)| |wc - q(wc)|, with each element error at most
+    its block's max times 1/6 (half the widest level gap over the scale) plus
+    the E4M3 rounding of the scale.  It also removes most of the plain W4A4
+    error."""
+    r = np.random.default_rng(41)
+    K, N, rows = 64, 32, 40
+    x = F.bf16_rne((r.standard_normal((rows, K)) * np.exp(r.standard_normal((1, K)))).astype(np.float32))
+    w = F.bf16_rne((r.standard_normal((1, N, K)) * 0.05).astype(np.float32))
+    a_c, a_s, g_a = Q.quantize(x)
+    w_c, w_s, g_w = Q.quantize(w[0])
+    chan = np.arange(K)
+    resid = Q.residual_channels(x, a_c, a_s, g_a, chan)
+    wdeq = F.bf16_rne(F.f32(Q.dequant(w_c, w_s, g_w)))
+    off = np.array([0, rows])
+    exact = x @ Q.dequant(w_c, w_s, g_w).T
+    y_plain, _ = M.grouped_gemm(a_c, a_s, g_a, w_c[None], w_s[None], [g_w], off)
+    rc, rs, g_r, wcc, wcs, g_wc = M.fp4_compensation_operands(resid, wdeq[None], g_a, [g_w], off)
+    assert abs(g_r[0] * g_wc[0] / (g_a * g_w) - 1) < 2.0 ** -22
+    y4, _ = M.grouped_gemm_fp4_comp(a_c, a_s, g_a, w_c[None], w_s[None], [g_w], off, rc, rs, wcc, wcs)
+    qr = Q.dequant(rc, rs, g_r[0])
+    qwc = Q.dequant(wcc[0], wcs[0], g_wc[0])
+    def elem_err(v):
+        m = np.repeat(np.abs(v).reshape(v.shape[0], -1, 16).max(axis=2), 16, axis=1)
+        return m / 6.0 * (1 + 2.0 ** -3) + 1e-300
+    bound = elem_err(resid) @ np.abs(wdeq).T + np.abs(qr) @ elem_err(wdeq).T
+    # the BF16 rounding of the stored residual is inside r itself; the G_e vs
+    # g_r g_wc rounding is a relative 2^-22 of the correction
+    assert np.all(np.abs(y4 - exact) <= bound * (1 + 2.0 ** -20) + 1e-12 * np.abs(exact).max()
+                  + np.abs(resid - F.f32(x - Q.dequant(a_c, a_s, g_a))) @ np.abs(wdeq).T)
+    assert np.mean(np.abs(y4 - exact)) < 0.5 * np.mean(np.abs(y_plain - exact))
+    # a zero residual contributes nothing
+    z = M.fp4_compensation_operands(np.zeros_like(resid), wdeq[None], g_a, [g_w], off)
+    y0, _ = M.grouped_gemm_fp4_comp(a_c, a_s, g_a, w_c[None], w_s[None], [g_w], off, z[0], z[1], z[3], z[4])
+    assert np.array_equal(y0, y_plain)
+
+
 # ------------------------------------------------------------------ stack
 
 

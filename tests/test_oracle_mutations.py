@@ -122,6 +122,11 @@ def _guided_ignores_bit(bits, scales, g_rows, x_train, chan=None, resid=None):
     return TR.__dict__["_orig_replay_dir"](np.zeros_like(bits), scales, g_rows, x_train, chan, resid)
 
 
+def _comp_amax_uses_gw(g_a, g_w, g_wc):
+    # the ratio taken against the wrong per-tensor scale
+    return M.__dict__["_orig_comp_amax"](g_a, g_w, np.asarray(g_w, dtype=np.float64) * 4.0)
+
+
 MUTATIONS = {
     "e2m1_ties_away": [(F, "e2m1_rne_code", _e2m1_ties_up), (Q, "e2m1_rne_code", _e2m1_ties_up)],
     "e2m1_drops_sign": [(F, "e2m1_rne_code", _e2m1_no_sign), (Q, "e2m1_rne_code", _e2m1_no_sign)],
@@ -138,6 +143,7 @@ MUTATIONS = {
     "swiglu_gate_up_swapped": [(M, "swiglu", _swiglu_wrong)],
     "nibble_order": [(F, "pack_nibbles", _pack_swapped)],
     "channel_ties_to_high_index": [(Q, "select_channels", _select_ties_high)],
+    "fp4_comp_wrong_scale": [(M, "_orig_comp_amax", M.fp4_comp_amax), (M, "fp4_comp_amax", _comp_amax_uses_gw)],
     "direction_floor_off_by_one": [(TR, "_floor_level_index", _floor_level_left)],
     "direction_bit_ignored": [(TR, "_orig_replay_dir", TR.replay_direction),
                               (TR, "replay_direction", _guided_ignores_bit)],
