@@ -259,6 +259,43 @@ int quads_moe_grouped_gemm_nvfp4_swiglu(const uint8_t* a_codes, const uint8_t* a
                                         int n_chan, uint16_t* h, float* amax_out,
                                         quads_stream_t stream);
 
+/* The literal second quantization pass ([QUADS-fr §2.2.B]: the correction
+ * on the high-residual channels is a second quantization pass added to the
+ * quantized output): the residual channels R and the weights' channel
+ * columns Wc are NVFP4 operands, multiplied on the FP4 tensor cores in the
+ * same accumulator as the main product:
+ *   y = bf16(G_e * (sum_k a w + sum_c q(r) q(wc)))   (NVFP4 values)
+ * r_codes [rows_cap][Kc/2] and r_scales (tiled over rows_cap x Kc) are R
+ * quantized per expert segment with amax_r from quads_moe_fp4_comp_amax;
+ * wc_codes [E*N][Kc/2] and wc_scales (tiled over E*N x Kc) are Wc quantized
+ * per expert with its own amax.  Kc % 64 == 0, Kc <= 1024 (pad channel
+ * columns with zeros); everything else as quads_moe_grouped_gemm_nvfp4 with
+ * n_chan = 0.  The SwiGLU variant is quads_moe_grouped_gemm_nvfp4_swiglu with
+ * this correction. */
+int quads_moe_grouped_gemm_nvfp4_fp4comp(const uint8_t* a_codes, const uint8_t* a_scales,
+                                         const float* g_a, int g_a_per_expert,
+                                         const uint8_t* w_codes, const uint8_t* w_scales,
+                                         const float* g_w, const int32_t* expert_off, int E,
+                                         int64_t rows_cap, int64_t N, int64_t K,
+                                         const uint8_t* r_codes, const uint8_t* r_scales,
+                                         const uint8_t* wc_codes, const uint8_t* wc_scales,
+                                         int64_t Kc, uint16_t* y, quads_stream_t stream);
+int quads_moe_grouped_gemm_nvfp4_swiglu_fp4comp(const uint8_t* a_codes, const uint8_t* a_scales,
+                                                const float* g_a, int g_a_per_expert,
+                                                const uint8_t* w_codes, const uint8_t* w_scales,
+                                                const float* g_w, const int32_t* expert_off, int E,
+                                                int64_t rows_cap, int64_t F, int64_t K,
+                                                const uint8_t* r_codes, const uint8_t* r_scales,
+                                                const uint8_t* wc_codes, const uint8_t* wc_scales,
+                                                int64_t Kc, uint16_t* h, float* amax_out,
+                                                quads_stream_t stream);
+/* Per-expert amax of the residual operand above, chosen so that its decode
+ * scale times g_wc[e] is G_e = fp32(g_a g_w[e]) up to one rounding:
+ * amax_r[e] = fp32(fp32(G_e / g_wc[e]) * 2688), 0 where g_wc[e] == 0.
+ * g_a is device float[E] when g_a_per_expert, else float[1]; all device. */
+int quads_moe_fp4_comp_amax(const float* g_a, int g_a_per_expert, const float* g_w,
+                            const float* g_wc, int E, float* amax_r, quads_stream_t stream);
+
 /* a6 + a7 + the re-quantization of h in one pass: the SwiGLU GEMM above
  * whose epilogue also NVFP4-quantizes h for the down projection.  Each
  * expert uses the decode scale g_e = fp32(amax_h_in[e] / 2688), computed from

@@ -279,3 +279,70 @@ def test_grouped_gemm_swiglu_quant(cuda_lib, counts, F_, K, nc, nch, amax_scale)
     assert np.all(err <= tol), f"{np.sum(err > tol)} of {err.size} dequantized h values outside the tolerance"
     match = np.mean(F.unpack_nibbles(u8_np(c1)[:R]) == qc)
     assert match > 0.9, f"only {match:.3f} of the h codes match the oracle's"
+
+
+@pytest.mark.parametrize("counts,N,K,nc,swiglu", [
+    ([64], 128, 64, 64, False),                 # one tile, one main and one correction K block
+    ([130, 0, 257], 256, 512, 128, False),      # empty expert, ragged experts, two correction blocks
+    ([500, 20, 1000, 3], 384, 1024, 64, True),  # SwiGLU epilogue
+    ([300, 40], 256, 320, 192, False),          # partial main stage, three correction blocks
+])
+def test_grouped_gemm_fp4_comp_parity(cuda_lib, counts, N, K, nc, swiglu):
+    """The literal second quantization pass: residual channels and weight
+    channel columns NVFP4-quantized on the device (per-expert residual scale
+    from quads_moe_fp4_comp_amax) bit for bit against the oracle's operands,
+    and the GEMM over the channel-extended reduction axis against the
+    oracle's within the GEMM tolerance."""
+    p = _problem(counts, N, K, nc, seed=7 * sum(counts) + N + K + nc)
+    E, cap, R, off = p["E"], p["cap"], p["R"], p["off"]
+    rc, rs, g_r, wcc, wcs, g_wc = M.fp4_compensation_operands(p["resid"], p["wc"], p["g_a"], p["g_w"], off)
+    perm = gate_up_interleave_index(N // 2) if swiglu else np.arange(N)
+    args = _gpu_args(p, p["w_c"][:, perm], p["w_s"][:, perm], p["wc"][:, perm])
+    dev = "cuda"
+    # device operand path
+    wc_dev = args["w_resid"].reshape(E * N, nc)
+    wcc_d, wcs_d, g_wc_d, _ = cuda_lib.quantize_nvfp4(wc_dev, n_groups=E, scale_layout=cuda_lib.SCALES_TILED)
+    amax_r = cuda_lib.moe_fp4_comp_amax(args["g_a"], args["g_w"], g_wc_d, E)
+    ra = torch.zeros((cap, nc), dtype=torch.bfloat16, device=dev)
+    ra[:R] = bf16_torch(p["resid"])
+    rc_d = torch.full((cap, nc // 2), 0, dtype=torch.uint8, device=dev)
+    rs_d = torch.zeros(cuda_lib.scales_bytes(cap, nc, cuda_lib.SCALES_TILED), dtype=torch.uint8, device=dev)
+    _, _, g_r_d, _ = cuda_lib.quantize_nvfp4(ra, group_off=args["expert_off"], n_groups=E, amax_in=amax_r,
+                                             scale_layout=cuda_lib.SCALES_TILED, codes=rc_d, scales=rs_d)
+    torch.cuda.synchronize()
+    assert_bits_equal(f32_of(g_wc_d).astype(np.float32), g_wc.astype(np.float32), "g_wc")
+    assert_bits_equal(f32_of(amax_r).astype(np.float32), M.fp4_comp_amax(p["g_a"], p["g_w"], g_wc).astype(np.float32),
+                      "amax_r")
+    assert_bits_equal(f32_of(g_r_d).astype(np.float32), g_r.astype(np.float32), "g_r")
+    assert_bits_equal(u8_np(rc_d)[:R], F.pack_nibbles(rc), "residual codes")
+    assert_bits_equal(F.scales_from_tiled(u8_np(rs_d), cap, nc // 16)[:R], rs, "residual scales")
+    assert_bits_equal(u8_np(wcc_d).reshape(E, N, nc // 2), F.pack_nibbles(wcc[:, perm]), "weight-column codes")
+    # the GEMM
+    if swiglu:
+        h, amax = cuda_lib.moe_grouped_gemm_nvfp4_fp4comp(
+            args["a_codes"], args["a_scales"], args["g_a"], args["w_codes"], args["w_scales"], args["g_w"],
+            args["expert_off"], E, cap, N, K, rc_d, rs_d, wcc_d, wcs_d, nc, swiglu=True)
+    else:
+        y = torch.full((cap, N), float("nan"), dtype=torch.bfloat16, device=dev)
+        cuda_lib.moe_grouped_gemm_nvfp4_fp4comp(
+            args["a_codes"], args["a_scales"], args["g_a"], args["w_codes"], args["w_scales"], args["g_w"],
+            args["expert_off"], E, cap, N, K, rc_d, rs_d, wcc_d, wcs_d, nc, y=y)
+    torch.cuda.synchronize()
+    assert cuda_lib.device_status() == cuda_lib.OK
+    ref, absdot = M.grouped_gemm_fp4_comp(p["a_c"], p["a_s"], p["g_a"], p["w_c"], p["w_s"], p["g_w"], off, rc, rs,
+                                          wcc, wcs)
+    if not swiglu:
+        got = bf16_np(y)
+        assert_close_tol(got[:R], ref, absdot, what="grouped gemm with FP4 correction")
+        assert np.all(np.isnan(got[R:]))
+    else:
+        F_ = N // 2
+        tol_y = 1e-2 * np.abs(ref) + 1e-3 * absdot
+        g, u = ref[:, :F_], ref[:, F_:]
+        sig = 1.0 / (1.0 + np.exp(-g))
+        h_ref = M.swiglu(F.bf16_rne(ref.astype(np.float32)))
+        dsilu = np.abs(sig * (1.0 + g * (1.0 - sig)))
+        tol_h = dsilu * (np.abs(u) + tol_y[:, F_:]) * tol_y[:, :F_] + np.abs(g * sig) * tol_y[:, F_:] + \
+            2.0 ** -7 * np.abs(h_ref) + 1e-30
+        err = np.abs(bf16_np(h)[:R] - h_ref)
+        assert np.all(err <= tol_h), f"{np.sum(err > tol_h)} of {err.size} h values outside the tolerance"

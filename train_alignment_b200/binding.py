@@ -87,6 +87,12 @@ _SIGS = {
     "quads_moe_grouped_gemm_nvfp4_swiglu_quant": (c_i32, [c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_i32,
                                                           c_i64, c_i64, c_i64, c_vp, c_vp, c_i32, c_vp, c_vp, c_i32,
                                                           c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
+    "quads_moe_grouped_gemm_nvfp4_fp4comp": (c_i32, [c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_i32, c_i64,
+                                                     c_i64, c_i64, c_vp, c_vp, c_vp, c_vp, c_i64, c_vp, c_vp]),
+    "quads_moe_grouped_gemm_nvfp4_swiglu_fp4comp": (c_i32, [c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_i32,
+                                                            c_i64, c_i64, c_i64, c_vp, c_vp, c_vp, c_vp, c_i64, c_vp,
+                                                            c_vp, c_vp]),
+    "quads_moe_fp4_comp_amax": (c_i32, [c_vp, c_i32, c_vp, c_vp, c_i32, c_vp, c_vp]),
     "quads_swiglu": (c_i32, [c_vp, c_i64, c_i64, c_vp, c_i32, c_vp, c_vp, c_vp]),
     "quads_moe_unpermute_combine": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i32, c_i64, c_vp, c_vp]),
     "quads_fakequant_weight_ste": (c_i32, [c_vp, c_i64, c_i64, c_i64, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_i32,
@@ -347,6 +353,37 @@ def moe_grouped_gemm_nvfp4_swiglu_quant(a_codes, a_scales, g_a, w_codes, w_scale
         _p(h_scales), _p(h_resid) if n_chan_h else None, _p(g_h), _p(amax_h_out), _p(h), _s()),
         "quads_moe_grouped_gemm_nvfp4_swiglu_quant")
     return h_codes, h_scales, (h_resid if n_chan_h else None), g_h, amax_h_out
+
+
+def moe_grouped_gemm_nvfp4_fp4comp(a_codes, a_scales, g_a, w_codes, w_scales, g_w, expert_off, E, rows_cap, N, K,
+                                   r_codes, r_scales, wc_codes, wc_scales, Kc, y=None, swiglu=False, amax=None):
+    """Grouped GEMM with the FP4 residual correction; swiglu=True gives
+    (h [rows_cap, N/2], amax) with N = 2F, else y [rows_cap, N]."""
+    dev = a_codes.device
+    per_expert = 1 if g_a.numel() == E and E > 1 else 0
+    if swiglu:
+        F = N // 2
+        y = y if y is not None else _empty((rows_cap, F), torch.bfloat16, dev)
+        amax = amax if amax is not None else _empty((E,), torch.float32, dev)
+        _check(load().quads_moe_grouped_gemm_nvfp4_swiglu_fp4comp(
+            _p(a_codes), _p(a_scales), _p(g_a), per_expert, _p(w_codes), _p(w_scales), _p(g_w), _p(expert_off), E,
+            rows_cap, F, K, _p(r_codes), _p(r_scales), _p(wc_codes), _p(wc_scales), Kc, _p(y), _p(amax), _s()),
+            "quads_moe_grouped_gemm_nvfp4_swiglu_fp4comp")
+        return y, amax
+    y = y if y is not None else _empty((rows_cap, N), torch.bfloat16, dev)
+    _check(load().quads_moe_grouped_gemm_nvfp4_fp4comp(
+        _p(a_codes), _p(a_scales), _p(g_a), per_expert, _p(w_codes), _p(w_scales), _p(g_w), _p(expert_off), E,
+        rows_cap, N, K, _p(r_codes), _p(r_scales), _p(wc_codes), _p(wc_scales), Kc, _p(y), _s()),
+        "quads_moe_grouped_gemm_nvfp4_fp4comp")
+    return y
+
+
+def moe_fp4_comp_amax(g_a, g_w, g_wc, E, out=None):
+    out = out if out is not None else _empty((E,), torch.float32, g_w.device)
+    per_expert = 1 if g_a.numel() == E and E > 1 else 0
+    _check(load().quads_moe_fp4_comp_amax(_p(g_a), per_expert, _p(g_w), _p(g_wc), E, _p(out), _s()),
+           "quads_moe_fp4_comp_amax")
+    return out
 
 
 def swiglu(y, F, expert_off, E, h=None, amax=None, want_amax=True):

@@ -92,6 +92,11 @@ struct GemmParams {
   uint16_t* h_resid;         // [rows_cap][n_chan_h]
   float* g_h_out;            // [E]
   int n_chan_h;
+  // FP4 compensation: NVFP4 residual / weight-column operands appended to the
+  // reduction axis (nkb_comp 64-wide K blocks; tiled scales)
+  const uint8_t* a2_scales;  // [rows_cap] x Kc
+  const uint8_t* w2_scales;  // [E * N] x Kc
+  int nkb_comp;
   int g_a_per_expert;
   int E;
   int rows_cap;              // rows of a_codes, y and the h outputs
@@ -329,7 +334,8 @@ template <bool kSwiglu, bool kQuant>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                         const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_wc,
-                        const __grid_constant__ CUtensorMap tm_y, GemmParams p) {
+                        const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_a2,
+                        const __grid_constant__ CUtensorMap tm_b2, GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -414,7 +420,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // row tiles below expert_off[E], never past the buffers' rows_cap rows
   const int total = (min(off_s[p.E], p.rows_cap) / BM) * n_ntiles;
   const int nkb_total = p.K / 64;                 // MMAs along K
-  const int nks = (nkb_total + 3) / 4;            // pipeline stages along K
+  const int nks_main = (nkb_total + 3) / 4;       // pipeline stages along K
+  const int nks = nks_main + (p.nkb_comp + 3) / 4; // then the FP4 compensation's stages
   const int n_col_tiles = nkb_total;              // 512-byte scale tiles per 128-row band
 
   if (warp == 0 && lane == 0) {
@@ -431,16 +438,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = it % S;
         const uint32_t ph = (it / S) & 1;
         if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
-        const int nkb = min(4, nkb_total - ks * 4);
         const uint32_t st = base + s * kStageBytes;
-        mbar_expect_tx(full_bar(s), kABytes + kBBytes + 2 * nkb * 512);
-        tma_load_2d(st, &tm_a, ks * kStageRowBytes, m0, full_bar(s));
-        tma_load_2d(st + kABytes, &tm_b, ks * kStageRowBytes, brow, full_bar(s));
-        bulk_load(st + kABytes + kBBytes, p.a_scales + (static_cast<int64_t>(mt) * n_col_tiles + ks * 4) * 512,
-                  nkb * 512, full_bar(s));
-        bulk_load(st + kABytes + kBBytes + kSfBytes,
-                  p.w_scales + (static_cast<int64_t>(brow / BM) * n_col_tiles + ks * 4) * 512, nkb * 512,
-                  full_bar(s));
+        if (ks < nks_main) {
+          const int nkb = min(4, nkb_total - ks * 4);
+          mbar_expect_tx(full_bar(s), kABytes + kBBytes + 2 * nkb * 512);
+          tma_load_2d(st, &tm_a, ks * kStageRowBytes, m0, full_bar(s));
+          tma_load_2d(st + kABytes, &tm_b, ks * kStageRowBytes, brow, full_bar(s));
+          bulk_load(st + kABytes + kBBytes, p.a_scales + (static_cast<int64_t>(mt) * n_col_tiles + ks * 4) * 512,
+                    nkb * 512, full_bar(s));
+          bulk_load(st + kABytes + kBBytes + kSfBytes,
+                    p.w_scales + (static_cast<int64_t>(brow / BM) * n_col_tiles + ks * 4) * 512, nkb * 512,
+                    full_bar(s));
+        } else {
+          // FP4 compensation: one 128 x 32-byte box (32-byte swizzle) per K block
+          const int j0 = (ks - nks_main) * 4;
+          const int nkb = min(4, p.nkb_comp - j0);
+          mbar_expect_tx(full_bar(s), 2 * nkb * (kCompChunkBytes + 512));
+          for (int j = 0; j < nkb; ++j) {
+            tma_load_2d(st + j * kCompChunkBytes, &tm_a2, (j0 + j) * kMmaKBytes, m0, full_bar(s));
+            tma_load_2d(st + kABytes + j * kCompChunkBytes, &tm_b2, (j0 + j) * kMmaKBytes, brow, full_bar(s));
+          }
+          bulk_load(st + kABytes + kBBytes, p.a2_scales + (static_cast<int64_t>(mt) * p.nkb_comp + j0) * 512,
+                    nkb * 512, full_bar(s));
+          bulk_load(st + kABytes + kBBytes + kSfBytes,
+                    p.w2_scales + (static_cast<int64_t>(brow / BM) * p.nkb_comp + j0) * 512, nkb * 512,
+                    full_bar(s));
+        }
       }
       if (ok && nch) {
         if (!mbar_wait(comp_empty, cph ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
@@ -476,13 +499,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(full_bar(s), ph, abort_flag, p.timeout_ns)) { ok = false; break; }
         if (!mbar_wait(sf_full(slot), (it / kSfSlots) & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
         tc_fence_after();
-        const int nkb = min(4, nkb_total - ks * 4);
         const uint32_t st = base + s * kStageBytes;
         const uint32_t tsfa = tmem + kSfCol + slot * 32;
         const uint32_t tsfb = tsfa + 16;
-        for (int kb = 0; kb < nkb; ++kb) {
-          mma_fp4(dacc, desc_kmajor_sw128(st + kb * kMmaKBytes), desc_kmajor_sw128(st + kABytes + kb * kMmaKBytes),
-                  kIdescFp4, tsfa + kb * 4, tsfb + kb * 4, (ks | kb) != 0 ? 1u : 0u);
+        if (ks < nks_main) {
+          const int nkb = min(4, nkb_total - ks * 4);
+          for (int kb = 0; kb < nkb; ++kb)
+            mma_fp4(dacc, desc_kmajor_sw128(st + kb * kMmaKBytes), desc_kmajor_sw128(st + kABytes + kb * kMmaKBytes),
+                    kIdescFp4, tsfa + kb * 4, tsfb + kb * 4, (ks | kb) != 0 ? 1u : 0u);
+        } else {
+          const int nkb = min(4, p.nkb_comp - (ks - nks_main) * 4);
+          for (int kb = 0; kb < nkb; ++kb)
+            mma_fp4(dacc, desc_kmajor_sw32(st + kb * kCompChunkBytes),
+                    desc_kmajor_sw32(st + kABytes + kb * kCompChunkBytes), kIdescFp4, tsfa + kb * 4, tsfb + kb * 4,
+                    1u);
         }
         tc_commit(empty_bar(s));
         tc_commit(sf_empty(slot));
@@ -660,6 +690,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
+// Per-expert amax for the FP4 compensation's residual:
+// amax_r[e] = fp32(fp32(G_e / g_wc[e]) * 2688), G_e = fp32(g_a g_w[e]); the
+// residual's decode scale times g_wc[e] is then G_e up to one rounding.
+__global__ void fp4_comp_amax_kernel(const float* g_a, int g_a_per_expert, const float* g_w, const float* g_wc,
+                                     int E, float* amax_r) {
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const float G = __fmul_rn(g_a[g_a_per_expert ? e : 0], g_w[e]);
+    const float wc = g_wc[e];
+    amax_r[e] = wc > 0.0f ? __fmul_rn(__fdiv_rn(G, wc), kNvfp4Range) : 0.0f;
+  }
+}
+
 // One thread waits on a barrier that nothing completes; the bounded wait
 // gives up after limit_ns and records the timeout.
 __global__ void bounded_wait_selftest_kernel(uint64_t limit_ns) {
@@ -713,6 +755,17 @@ size_t gemm_smem_bytes(int stages, int n_chan, int E, size_t extra_words = 0) {
          (static_cast<size_t>(2 * E + 1) + extra_words) * 4;
 }
 
+// FP4 compensation operands (device memory): the NVFP4 residual channels of
+// the activations [rows_cap][Kc] and the weights' channel columns [E * N][Kc],
+// codes row-major, scales tiled.
+struct Fp4Comp {
+  const uint8_t* a_codes;
+  const uint8_t* a_scales;
+  const uint8_t* w_codes;
+  const uint8_t* w_scales;
+  int64_t Kc;
+};
+
 // The quantizing epilogue's outputs (all device memory).
 struct HQuant {
   const float* amax_in;
@@ -740,7 +793,8 @@ template <bool kSwiglu, bool kQuant = false>
 int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_a, int g_a_per_expert,
                 const uint8_t* w_codes, const uint8_t* w_scales, const float* g_w, const int32_t* expert_off, int E,
                 int64_t rows_cap, int64_t N, int64_t K, const uint16_t* a_resid, const uint16_t* w_resid, int n_chan,
-                uint16_t* y, float* amax_out, cudaStream_t stream, const HQuant* hq = nullptr) {
+                uint16_t* y, float* amax_out, cudaStream_t stream, const HQuant* hq = nullptr,
+                const Fp4Comp* fc = nullptr) {
   QUADS_REQUIRE(E >= 1 && E <= 256, QUADS_ERR_UNSUPPORTED_SHAPE, "E must be in [1, 256]");
   QUADS_REQUIRE(N > 0 && N % BN == 0 && N <= (int64_t(1) << 20), QUADS_ERR_UNSUPPORTED_SHAPE,
                 "N (%lld) must be a positive multiple of 128", (long long)N);
@@ -762,6 +816,14 @@ int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_
                   QUADS_ERR_INVALID_ARG, "h_codes and h_scales must be 16-byte aligned");
   }
   QUADS_REQUIRE(n_chan == 0 || (a_resid && w_resid), QUADS_ERR_INVALID_ARG, "a_resid and w_resid required");
+  if (fc) {
+    QUADS_REQUIRE(n_chan == 0, QUADS_ERR_INVALID_ARG, "BF16 and FP4 compensation are exclusive");
+    QUADS_REQUIRE(fc->Kc > 0 && fc->Kc % 64 == 0 && fc->Kc <= 1024, QUADS_ERR_UNSUPPORTED_SHAPE,
+                  "Kc (%lld) must be a positive multiple of 64 up to 1024", (long long)fc->Kc);
+    QUADS_REQUIRE(fc->a_codes && fc->a_scales && fc->w_codes && fc->w_scales && aligned(fc->a_codes, 16) &&
+                      aligned(fc->w_codes, 16) && aligned(fc->a_scales, 16) && aligned(fc->w_scales, 16),
+                  QUADS_ERR_INVALID_ARG, "FP4 compensation operands must be non-null and 16-byte aligned");
+  }
   QUADS_REQUIRE(aligned(a_codes, 16) && aligned(w_codes, 16) && aligned(a_scales, 16) && aligned(w_scales, 16) &&
                     (!y || aligned(y, 16)) && (n_chan == 0 || (aligned(a_resid, 16) && aligned(w_resid, 16))),
                 QUADS_ERR_INVALID_ARG, "matrix pointers must be 16-byte aligned");
@@ -788,6 +850,13 @@ int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_
                           CU_TENSOR_MAP_SWIZZLE_64B));
   else
     tm_y = tm_a;                                  // never used: no h store
+  CUtensorMap tm_a2 = tm_a, tm_b2 = tm_a;
+  if (fc) {
+    QUADS_TRY(make_map_2d(&tm_a2, fc->a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, fc->Kc / 2, rows_cap, kMmaKBytes,
+                          BM, CU_TENSOR_MAP_SWIZZLE_32B));
+    QUADS_TRY(make_map_2d(&tm_b2, fc->w_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, fc->Kc / 2, E * N, kMmaKBytes, BN,
+                          CU_TENSOR_MAP_SWIZZLE_32B));
+  }
   const size_t extra = kQuant ? static_cast<size_t>(E + hq->n_chan + N / 64 + 1) : 0;
   const size_t smem_cap = 232448;   // 227 KB per block on sm_100
   int stages = kMaxStages;
@@ -812,6 +881,9 @@ int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_
   p.h_scales = kQuant ? hq->scales : nullptr;
   p.h_resid = kQuant ? hq->resid : nullptr;
   p.g_h_out = kQuant ? hq->g_out : nullptr;
+  p.a2_scales = fc ? fc->a_scales : nullptr;
+  p.w2_scales = fc ? fc->w_scales : nullptr;
+  p.nkb_comp = fc ? static_cast<int>(fc->Kc / 64) : 0;
   p.g_a_per_expert = g_a_per_expert ? 1 : 0;
   p.E = E;
   p.rows_cap = static_cast<int>(rows_cap);
@@ -823,7 +895,8 @@ int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_
   const int64_t max_tiles = (rows_cap / BM) * (N / BN);
   int grid = num_sms();
   if (grid > max_tiles) grid = static_cast<int>(max_tiles);
-  grouped_gemm_kernel<kSwiglu, kQuant><<<grid, kThreads, smem, stream>>>(tm_a, tm_b, tm_r, tm_wc, tm_y, p);
+  grouped_gemm_kernel<kSwiglu, kQuant><<<grid, kThreads, smem, stream>>>(tm_a, tm_b, tm_r, tm_wc, tm_y, tm_a2, tm_b2,
+                                                                         p);
   count_launches(1);
   return check_launch("grouped_gemm_kernel");
 }
@@ -841,6 +914,43 @@ int quads_moe_grouped_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales
   clear_error();
   return launch_gemm<false>(a_codes, a_scales, g_a, g_a_per_expert, w_codes, w_scales, g_w, expert_off, E, rows_cap,
                             N, K, a_resid, w_resid, n_chan, y, nullptr, stream);
+}
+
+int quads_moe_grouped_gemm_nvfp4_fp4comp(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_a,
+                                         int g_a_per_expert, const uint8_t* w_codes, const uint8_t* w_scales,
+                                         const float* g_w, const int32_t* expert_off, int E, int64_t rows_cap,
+                                         int64_t N, int64_t K, const uint8_t* r_codes, const uint8_t* r_scales,
+                                         const uint8_t* wc_codes, const uint8_t* wc_scales, int64_t Kc, uint16_t* y,
+                                         quads_stream_t stream) {
+  clear_error();
+  const Fp4Comp fc{r_codes, r_scales, wc_codes, wc_scales, Kc};
+  return launch_gemm<false>(a_codes, a_scales, g_a, g_a_per_expert, w_codes, w_scales, g_w, expert_off, E, rows_cap,
+                            N, K, nullptr, nullptr, 0, y, nullptr, stream, nullptr, &fc);
+}
+
+int quads_moe_grouped_gemm_nvfp4_swiglu_fp4comp(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_a,
+                                                int g_a_per_expert, const uint8_t* w_codes, const uint8_t* w_scales,
+                                                const float* g_w, const int32_t* expert_off, int E, int64_t rows_cap,
+                                                int64_t F, int64_t K, const uint8_t* r_codes,
+                                                const uint8_t* r_scales, const uint8_t* wc_codes,
+                                                const uint8_t* wc_scales, int64_t Kc, uint16_t* h, float* amax_out,
+                                                quads_stream_t stream) {
+  clear_error();
+  QUADS_REQUIRE(F > 0 && F % 64 == 0, QUADS_ERR_UNSUPPORTED_SHAPE, "F (%lld) must be a positive multiple of 64",
+                (long long)F);
+  const Fp4Comp fc{r_codes, r_scales, wc_codes, wc_scales, Kc};
+  return launch_gemm<true>(a_codes, a_scales, g_a, g_a_per_expert, w_codes, w_scales, g_w, expert_off, E, rows_cap,
+                           2 * F, K, nullptr, nullptr, 0, h, amax_out, stream, nullptr, &fc);
+}
+
+int quads_moe_fp4_comp_amax(const float* g_a, int g_a_per_expert, const float* g_w, const float* g_wc, int E,
+                            float* amax_r, quads_stream_t stream) {
+  clear_error();
+  QUADS_REQUIRE(E >= 1 && E <= 4096, QUADS_ERR_UNSUPPORTED_SHAPE, "E must be in [1, 4096]");
+  QUADS_REQUIRE(g_a && g_w && g_wc && amax_r, QUADS_ERR_INVALID_ARG, "null pointer");
+  fp4_comp_amax_kernel<<<1, 256, 0, stream>>>(g_a, g_a_per_expert, g_w, g_wc, E, amax_r);
+  count_launches(1);
+  return check_launch("fp4_comp_amax_kernel");
 }
 
 int quads_moe_grouped_gemm_nvfp4_swiglu_quant(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_a,
