@@ -157,3 +157,37 @@ def test_fused_requant_layer_matches_two_pass(cuda_lib):
         assert_bits_equal(F.bf16_bits(bf16_np(fused.out)), F.bf16_bits(bf16_np(two.out)), f"output, step {step}")
         assert_bits_equal(u8_np(fused.record), u8_np(two.record), f"TRACE record, step {step}")
         assert_bits_equal(f32_of(fused.counts).astype(np.int64), f32_of(two.counts).astype(np.int64), "counts")
+
+
+def test_fp4_compensation_layer(cuda_lib):
+    """The layer with the literal second quantization pass (residual and
+    weight channel columns NVFP4-quantized, one FP4 product) next to the
+    BF16-compensated layer and an uncompensated one, on the same batch: the
+    FP4 correction keeps the output close to the BF16-corrected one and
+    removes most of the uncompensated layer's distance to it."""
+    cfg = W.MOE_T2048
+    inp = W.moe_layer_inputs(cfg, seed=2, device="cpu")
+    dev = "cuda"
+    x, logits = inp["x"].to(dev), inp["logits"].to(dev)
+    chan_x = L.calibrate_channels(x, cfg.n_chan)
+    r = np.random.default_rng(2)
+    chan_h = torch.from_numpy(Q.pad_channels(np.sort(r.choice(cfg.F, cfg.n_chan_f - 7, replace=False)))).to(dev)
+    none = torch.full((16,), -1, dtype=torch.int32, device=dev)
+    outs = {}
+    for name, cx, ch, comp in [("bf16", chan_x, chan_h, "bf16"), ("fp4", chan_x, chan_h, "fp4"),
+                               ("none", none, none, "bf16")]:
+        layer = L.MoELayer(cfg, inp["w_gu"].to(dev), inp["w_d"].to(dev), cx, ch, dev, comp=comp)
+        layer.weight_sync()
+        outs[name] = layer.rollout_forward(x, logits).float().clone()
+        torch.cuda.synchronize()
+        assert cuda_lib.device_status() == cuda_lib.OK
+        if comp == "fp4":
+            assert layer.nc_x % 64 == 0 and layer.nc_h % 64 == 0
+        del layer
+    ref = outs["bf16"]
+    d_fp4 = torch.linalg.vector_norm(outs["fp4"] - ref, dim=1) / torch.linalg.vector_norm(ref, dim=1)
+    d_none = torch.linalg.vector_norm(outs["none"] - ref, dim=1) / torch.linalg.vector_norm(ref, dim=1)
+    print(f"distance to the BF16-compensated output: FP4 correction median {d_fp4.median():.4f}, "
+          f"none {d_none.median():.4f}")
+    assert torch.isfinite(outs["fp4"]).all()
+    assert d_fp4.median() < 0.5 * d_none.median()

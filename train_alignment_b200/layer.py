@@ -67,7 +67,7 @@ class MoELayer:
     fixed token count; step() runs the whole path without allocating."""
 
     def __init__(self, cfg: MoEConfig, w_gu, w_d, chan_x, chan_h, device="cuda", fuse_swiglu=None, overlap=True,
-                 fuse_requant=False, amax_h_init=None):
+                 fuse_requant=False, amax_h_init=None, comp="bf16"):
         self.cfg = cfg
         T, H, E, k, F = cfg.T, cfg.H, cfg.E, cfg.k, cfg.F
         dev = torch.device(device)
@@ -99,6 +99,17 @@ class MoELayer:
         self.fuse_requant = bool(fuse_requant)
         if self.fuse_requant and not self.fuse_swiglu:
             raise ValueError("fuse_requant needs the fused SwiGLU epilogue (F % 64 == 0)")
+        # the compensation on the high-residual channels: "bf16" (R . Wc in
+        # BF16 on the tensor cores) or "fp4" (the literal second quantization
+        # pass: R and Wc NVFP4-quantized, multiplied in the main FP4 product;
+        # channel lists padded with -1 to multiples of 64)
+        if comp not in ("bf16", "fp4"):
+            raise ValueError(f"unknown compensation {comp!r}")
+        self.comp = comp
+        if comp == "fp4":
+            if not self.fuse_swiglu or self.fuse_requant:
+                raise ValueError("the FP4 compensation runs with the fused SwiGLU epilogue, without fuse_requant")
+            chan_x, chan_h = _pad_chan(chan_x, 64), _pad_chan(chan_h, 64)
         # the weight side of a step on its own stream (False: one stream)
         self.overlap = bool(overlap)
         self.nc_x = int(chan_x.numel())
@@ -161,6 +172,19 @@ class MoELayer:
             B.qtensor_src(self.h_codes, self.h_scales, self.g_h, cap, F, B.SCALES_TILED, group_off=self.expert_off,
                           chan=self.chan_h, resid=self.h_resid),
         ]
+        if comp == "fp4":
+            z = lambda shape, dt: torch.zeros(shape, dtype=dt, device=dev)
+            ts = lambda rows, k: e((B.scales_bytes(rows, k, B.SCALES_TILED),), u8)
+            self.wcq_gu_codes, self.wcq_gu_scales = e((E * 2 * F, self.nc_x // 2), u8), ts(E * 2 * F, self.nc_x)
+            self.wcq_d_codes, self.wcq_d_scales = e((E * H, self.nc_h // 2), u8), ts(E * H, self.nc_h)
+            self.g_wc_gu, self.g_wc_d = e((E,), f32), e((E,), f32)
+            self.ws_wc = e((B.quantize_workspace_bytes(E),), u8)
+            self.amax_r_gu, self.amax_r_d = e((E,), f32), e((E,), f32)
+            self.rq_codes, self.rq_scales = z((cap, self.nc_x // 2), u8), z((B.scales_bytes(cap, self.nc_x,
+                                                                                          B.SCALES_TILED),), u8)
+            self.rhq_codes, self.rhq_scales = z((cap, self.nc_h // 2), u8), z((B.scales_bytes(cap, self.nc_h,
+                                                                                            B.SCALES_TILED),), u8)
+            self.g_rq, self.g_rhq = e((E,), f32), e((E,), f32)
         self.x_hat, self.h_hat = e((T, H), bf), e((cap, F), bf)
         self.counts, self.status = torch.zeros(2, dtype=torch.int64, device=dev), e((1,), i32)
         self.status_h = e((1,), i32)
@@ -192,11 +216,21 @@ class MoELayer:
                                self.w_gu_scales, self.g_w_gu, self.wc_gu, None, self.amax_w_gu,
                                gate_up=self.fuse_swiglu)
         t.mark("fakequant_w_gate_up")
+        if self.comp == "fp4":
+            E, F = self.cfg.E, self.cfg.F
+            B.quantize_nvfp4(self.wc_gu.view(E * 2 * F, self.nc_x), n_groups=E, scale_layout=B.SCALES_TILED,
+                             codes=self.wcq_gu_codes, scales=self.wcq_gu_scales, g_out=self.g_wc_gu, ws=self.ws_wc)
+            t.mark("quantize_wc_gate_up")
 
     def _fakequant_down(self, t):
         B.fakequant_weight_ste(self.w_d, True, self.chan_h, False, True, self.w_d_fq, self.w_d_codes,
                                self.w_d_scales, self.g_w_d, self.wc_d, None, self.amax_w_d)
         t.mark("fakequant_w_down")
+        if self.comp == "fp4":
+            E, H = self.cfg.E, self.cfg.H
+            B.quantize_nvfp4(self.wc_d.view(E * H, self.nc_h), n_groups=E, scale_layout=B.SCALES_TILED,
+                             codes=self.wcq_d_codes, scales=self.wcq_d_scales, g_out=self.g_wc_d, ws=self.ws_wc)
+            t.mark("quantize_wc_down")
 
     def ste_backward(self, grad_gu_fq, grad_d_fq, timer=None):
         """Straight-through backward of both weight tensors, accumulated into
@@ -245,7 +279,18 @@ class MoELayer:
     def _rollout_gate_up(self, t):
         cfg = self.cfg
         H, E, F = cfg.H, cfg.E, cfg.F
-        if self.fuse_requant:
+        if self.comp == "fp4":
+            B.moe_fp4_comp_amax(self.g_x, self.g_w_gu, self.g_wc_gu, E, out=self.amax_r_gu)
+            B.quantize_nvfp4(self.pa_resid, group_off=self.expert_off, n_groups=E, amax_in=self.amax_r_gu,
+                             scale_layout=B.SCALES_TILED, codes=self.rq_codes, scales=self.rq_scales,
+                             g_out=self.g_rq)
+            t.mark("quantize_r")
+            B.moe_grouped_gemm_nvfp4_fp4comp(self.pa_codes, self.pa_scales, self.g_x, self.w_gu_codes,
+                                             self.w_gu_scales, self.g_w_gu, self.expert_off, E, self.cap, 2 * F, H,
+                                             self.rq_codes, self.rq_scales, self.wcq_gu_codes, self.wcq_gu_scales,
+                                             self.nc_x, y=self.h, swiglu=True, amax=self.amax_h)
+            t.mark("gemm_gate_up_swiglu_fp4comp")
+        elif self.fuse_requant:
             B.moe_grouped_gemm_nvfp4_swiglu_quant(
                 self.pa_codes, self.pa_scales, self.g_x, self.w_gu_codes, self.w_gu_scales, self.g_w_gu,
                 self.expert_off, E, self.cap, F, H, self.amax_h_prev, chan_h=self.chan_h if self.nc_h else None,
@@ -274,10 +319,22 @@ class MoELayer:
                              scale_layout=B.SCALES_TILED, chan=self.chan_h, codes=self.h_codes,
                              scales=self.h_scales, g_out=self.g_h, resid_out=self.h_resid)
             t.mark("quantize_h")
-        B.moe_grouped_gemm_nvfp4(self.h_codes, self.h_scales, self.g_h, self.w_d_codes, self.w_d_scales,
-                                 self.g_w_d, self.expert_off, E, self.cap, H, F, self.h_resid, self.wc_d,
-                                 y=self.y_d)
-        t.mark("gemm_down")
+        if self.comp == "fp4":
+            B.moe_fp4_comp_amax(self.g_h, self.g_w_d, self.g_wc_d, E, out=self.amax_r_d)
+            B.quantize_nvfp4(self.h_resid, group_off=self.expert_off, n_groups=E, amax_in=self.amax_r_d,
+                             scale_layout=B.SCALES_TILED, codes=self.rhq_codes, scales=self.rhq_scales,
+                             g_out=self.g_rhq)
+            t.mark("quantize_rh")
+            B.moe_grouped_gemm_nvfp4_fp4comp(self.h_codes, self.h_scales, self.g_h, self.w_d_codes, self.w_d_scales,
+                                             self.g_w_d, self.expert_off, E, self.cap, H, F, self.rhq_codes,
+                                             self.rhq_scales, self.wcq_d_codes, self.wcq_d_scales, self.nc_h,
+                                             y=self.y_d)
+            t.mark("gemm_down_fp4comp")
+        else:
+            B.moe_grouped_gemm_nvfp4(self.h_codes, self.h_scales, self.g_h, self.w_d_codes, self.w_d_scales,
+                                     self.g_w_d, self.expert_off, E, self.cap, H, F, self.h_resid, self.wc_d,
+                                     y=self.y_d)
+            t.mark("gemm_down")
         B.moe_unpermute_combine(self.y_d, self.row_of, self.topk_w, T, k, H, out=self.out)
         t.mark("combine")
         return self.out
@@ -346,6 +403,15 @@ class MoELayer:
         self.counts.zero_()
 
 
+def _pad_chan(chan, multiple):
+    """A channel list padded with -1 entries to a multiple of `multiple`."""
+    chan = torch.as_tensor(chan).to(torch.int32)
+    n = -(-chan.numel() // multiple) * multiple
+    out = torch.full((n,), -1, dtype=torch.int32, device=chan.device)
+    out[:chan.numel()] = chan
+    return out
+
+
 def _adjacent(a, b):
     """A flat view over a then b when b directly follows a in one storage."""
     if a.dtype != b.dtype or a.device != b.device or not (a.is_contiguous() and b.is_contiguous()):
@@ -369,7 +435,7 @@ def calibrate_channels(x, n_sel):
     return out
 
 
-def build_layer(cfg: MoEConfig, inputs, device="cuda", overlap=True, fuse_requant=False):
+def build_layer(cfg: MoEConfig, inputs, device="cuda", overlap=True, fuse_requant=False, comp="bf16"):
     """Layer from generated inputs: channel sets calibrated on the layer's own
     batch (X for the gate/up input, the uncompensated h for the down input);
     with fuse_requant, h's first-step per-expert amax is calibrated on the
@@ -386,4 +452,4 @@ def build_layer(cfg: MoEConfig, inputs, device="cuda", overlap=True, fuse_requan
     amax_h = probe.amax_h.clone()
     del probe
     return MoELayer(cfg, inputs["w_gu"], inputs["w_d"], chan_x, chan_h, device, overlap=overlap,
-                    fuse_requant=fuse_requant, amax_h_init=amax_h if fuse_requant else None)
+                    fuse_requant=fuse_requant, amax_h_init=amax_h if fuse_requant else None, comp=comp)
