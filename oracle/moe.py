@@ -207,3 +207,32 @@ def grouped_gemm_fp4_comp(a_codes, a_scales, g_a, w_codes, w_scales, g_w, expert
     w_c = np.concatenate([np.asarray(w_codes), np.asarray(wc_codes)], axis=2)
     w_s = np.concatenate([np.asarray(w_scales), np.asarray(wc_scales)], axis=2)
     return grouped_gemm(a_c, a_s, g_a, w_c, w_s, g_w, expert_off)
+
+
+# ------------------------------------------------ trainer-side W4A16 GEMM
+#
+# [QUADS-fr §2.2.A]: the trainer keeps BF16 activations and multiplies them
+# by its fake-quantized weights W_fq = bf16(deq(q(W))), the rollout's grid.
+# Given the weights as their NVFP4 codes, scales and per-expert scale:
+#   Y[r] = X[r] . W_fq[e]^T for every row r of expert e's segment,
+# with W_fq = bf16(fp32(val(q) val(s) g_w[e])) (the folded fake-quant).
+
+
+def grouped_gemm_w4a16(x, w_codes, w_scales, g_w, expert_off):
+    """Returns (Y [R, N] float64, absdot [R, N]) for BF16-exact x [R, K]."""
+    from .nvfp4 import dequant
+    x = np.asarray(x, dtype=np.float64)
+    off = np.asarray(expert_off, dtype=np.int64)
+    E = len(off) - 1
+    R = int(off[-1])
+    N = np.asarray(w_codes).shape[1]
+    Y = np.zeros((R, N))
+    absdot = np.zeros((R, N))
+    for e in range(E):
+        lo, hi = int(off[e]), int(off[e + 1])
+        if hi == lo:
+            continue
+        w_fq = bf16_rne(f32(dequant(w_codes[e], w_scales[e], float(g_w[e]))))
+        Y[lo:hi] = x[lo:hi] @ w_fq.T
+        absdot[lo:hi] = np.abs(x[lo:hi]) @ np.abs(w_fq).T
+    return Y, absdot

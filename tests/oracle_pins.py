@@ -612,6 +612,25 @@ def pin_fp4_compensation_close_to_bf16():
     assert np.array_equal(y0, y_plain)
 
 
+def pin_w4a16_gemm_is_fakequant_matmul():
+    """The trainer's W4A16 GEMM on the NVFP4 weights is the BF16 matmul of x
+    with the pinned weight fake-quant, per expert (torch float64 matmul as
+    the library routine); empty experts give no rows."""
+    r = np.random.default_rng(43)
+    E, N, K = 3, 16, 64
+    w = F.bf16_rne((r.standard_normal((E, N, K)) * np.array([0.01, 1.0, 30.0])[:, None, None]).astype(np.float32))
+    q = [Q.fakequant_weight(w[e]) for e in range(E)]
+    off = np.array([0, 5, 5, 12])
+    x = F.bf16_rne(r.standard_normal((12, K)).astype(np.float32))
+    y, absdot = M.grouped_gemm_w4a16(x, np.stack([t[1] for t in q]), np.stack([t[2] for t in q]),
+                                     [t[3] for t in q], off)
+    for e in range(E):
+        lo, hi = off[e], off[e + 1]
+        ref = torch.matmul(torch.from_numpy(x[lo:hi]), torch.from_numpy(q[e][0]).T).numpy()
+        assert np.allclose(y[lo:hi], ref, rtol=0, atol=1e-12 * max(1.0, np.abs(ref).max(initial=0)))
+        assert np.all(absdot[lo:hi] >= np.abs(y[lo:hi]))
+
+
 # ------------------------------------------------------------------ stack
 
 
