@@ -262,6 +262,60 @@ def quantize_replay_sweep(dev, hbm_gbs, reps=10):
     return out
 
 
+def trainer_gemm_timing(layer, dev, peaks, reps=20):
+    """The trainer's gate/up projection on the layer's expert-ordered rows:
+    the W4A16 kernel (BF16 activations, the NVFP4 weights dequantized on
+    chip, SwiGLU epilogue) against the BF16 library matmul of the same rows
+    with the stored W_fq (one per expert) it replaces.  L2 flushed before
+    each timed launch."""
+    import torch
+    from train_alignment_b200 import binding as B
+    cfg = layer.cfg
+    E, F, H = cfg.E, cfg.F, cfg.H
+    off = layer.expert_off.tolist()
+    rpad = off[-1]
+    gen = torch.Generator(device=dev).manual_seed(7)
+    x = torch.randn(layer.cap, H, generator=gen, device=dev).to(torch.bfloat16)
+    h = torch.empty(layer.cap, F, dtype=torch.bfloat16, device=dev)
+    amax = torch.empty(E, dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def timed(fn):
+        fn()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return sum(ts) / len(ts)
+
+    t_w4 = None
+    if layer.fuse_swiglu:           # the rollout's gate/up codes are in the interleaved order SwiGLU needs
+        t_w4 = timed(lambda: B.moe_grouped_gemm_w4a16(x, layer.w_gu_codes, layer.w_gu_scales, layer.g_w_gu,
+                                                      layer.expert_off, E, layer.cap, 2 * F, H, y=h, swiglu=True,
+                                                      amax=amax))
+    y = torch.empty(layer.cap, 2 * F, dtype=torch.bfloat16, device=dev)
+
+    def lib():
+        for e in range(E):
+            if off[e + 1] > off[e]:
+                torch.matmul(x[off[e]:off[e + 1]], layer.w_gu_fq[e].t(), out=y[off[e]:off[e + 1]])
+    t_lib = timed(lib)
+    rows = cfg.T * cfg.k
+    flops = 2.0 * rows * 2 * F * H
+    out = {"shape": f"{rows} routed rows ({rpad} padded) x {2 * F} x {H}, {E} experts",
+           "library_bf16_us": t_lib * 1e3, "library_bf16_tflops": flops / (t_lib * 1e-3) / 1e12,
+           "peak_bf16_tflops": peaks["bf16_tflops"]}
+    if t_w4 is not None:
+        out.update({"w4a16_swiglu_us": t_w4 * 1e3, "w4a16_tflops": flops / (t_w4 * 1e-3) / 1e12,
+                    "w4a16_frac_bf16": flops / (t_w4 * 1e-3) / 1e12 / peaks["bf16_tflops"]})
+    return out
+
+
 # ------------------------------------------------------------------- clocks
 
 
@@ -616,6 +670,7 @@ def run_ours(args):
     sweep = None
     if not args.no_sweep:
         sweep = quantize_replay_sweep(dev, peaks["hbm_gbs"])
+    trainer = trainer_gemm_timing(layer, dev, peaks) if not args.no_sweep else None
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -654,6 +709,7 @@ def run_ours(args):
         "timing": timing_mode,
         "instrumented_ms_per_step": sum(inst_ms) / len(inst_ms),
         "quantize_replay_sweep": sweep,
+        "trainer_gemm": trainer,
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)

@@ -289,6 +289,27 @@ int quads_moe_grouped_gemm_nvfp4_swiglu_fp4comp(const uint8_t* a_codes, const ui
                                                 const uint8_t* wc_codes, const uint8_t* wc_scales,
                                                 int64_t Kc, uint16_t* h, float* amax_out,
                                                 quads_stream_t stream);
+/* Trainer-side W4A16 grouped GEMM ([QUADS-fr §2.2.A]: the trainer keeps BF16
+ * activations and multiplies them by its fake-quantized weights):
+ *   y[r][n] = bf16(sum_k x[r][k] * W_fq[e][n][k]),  FP32 accumulation,
+ *   W_fq = bf16(fp32(val(q) * val(s)) * g_w[e])  (the folded fake-quant),
+ * for every row r of expert e's segment, with the weights read as their
+ * NVFP4 codes w_codes [E*N][K/2] and tiled scales (what
+ * quads_fakequant_weight_ste writes with want_codes) and dequantized on
+ * chip, so W_fq is never stored.  x [rows_cap][K] BF16, 16-byte aligned;
+ * other arguments as quads_moe_grouped_gemm_nvfp4.  The SwiGLU variant
+ * writes h [rows_cap][F] from weights in the 64-row interleaved gate/up order
+ * (N = 2F) and the per-expert max |h| (amax_out, nullable). */
+int quads_moe_grouped_gemm_w4a16(const uint16_t* x, const uint8_t* w_codes, const uint8_t* w_scales,
+                                 const float* g_w, const int32_t* expert_off, int E,
+                                 int64_t rows_cap, int64_t N, int64_t K, uint16_t* y,
+                                 quads_stream_t stream);
+int quads_moe_grouped_gemm_w4a16_swiglu(const uint16_t* x, const uint8_t* w_codes,
+                                        const uint8_t* w_scales, const float* g_w,
+                                        const int32_t* expert_off, int E, int64_t rows_cap,
+                                        int64_t F, int64_t K, uint16_t* h, float* amax_out,
+                                        quads_stream_t stream);
+
 /* Per-expert amax of the residual operand above, chosen so that its decode
  * scale times g_wc[e] is G_e = fp32(g_a g_w[e]) up to one rounding:
  * amax_r[e] = fp32(fp32(G_e / g_wc[e]) * 2688), 0 where g_wc[e] == 0.

@@ -346,3 +346,82 @@ def test_grouped_gemm_fp4_comp_parity(cuda_lib, counts, N, K, nc, swiglu):
             2.0 ** -7 * np.abs(h_ref) + 1e-30
         err = np.abs(bf16_np(h)[:R] - h_ref)
         assert np.all(err <= tol_h), f"{np.sum(err > tol_h)} of {err.size} h values outside the tolerance"
+
+
+def _w4a16_problem(counts, N, K, seed):
+    r = np.random.default_rng(seed)
+    E = len(counts)
+    padded = [-(-c // 128) * 128 for c in counts]
+    off = np.concatenate([[0], np.cumsum(padded)]).astype(np.int32)
+    R = int(off[-1])
+    cap = R + 128
+    x = np.zeros((cap, K))
+    for e in range(E):
+        x[off[e]:off[e] + counts[e]] = r.standard_normal((counts[e], K))
+    x = F.bf16_rne(x.astype(np.float32))
+    w = F.bf16_rne((r.standard_normal((E, N, K)) * 0.02).astype(np.float32))
+    wq = [Q.quantize(w[e]) for e in range(E)]
+    return dict(E=E, N=N, K=K, off=off, R=R, cap=cap, x=x, w=w, w_c=np.stack([q[0] for q in wq]),
+                w_s=np.stack([q[1] for q in wq]), g_w=np.array([q[2] for q in wq]))
+
+
+@pytest.mark.parametrize("counts,N,K", [
+    ([64], 128, 64),                   # one tile, one stage
+    ([130, 0, 257], 256, 512),         # empty expert, ragged experts
+    ([500, 20, 1000, 3], 384, 1024),
+    ([256], 128, 4096),                # long K
+])
+def test_grouped_gemm_w4a16_parity(cuda_lib, counts, N, K):
+    """The trainer-side W4A16 GEMM (BF16 activations, NVFP4 weights
+    dequantized on chip) against the oracle within the GEMM tolerance, and
+    against a plain PyTorch FP32 matmul of x with the device fake-quant's
+    W_fq; rows past expert_off[E] untouched."""
+    p = _w4a16_problem(counts, N, K, seed=sum(counts) + N + K)
+    E, cap, R, off = p["E"], p["cap"], p["R"], p["off"]
+    dev = "cuda"
+    w_codes = torch.from_numpy(np.ascontiguousarray(F.pack_nibbles(p["w_c"]))).to(dev)
+    w_scales = torch.from_numpy(F.scales_to_tiled(p["w_s"].reshape(E * N, K // 16))).to(dev)
+    g_w = torch.tensor(p["g_w"], dtype=torch.float32, device=dev)
+    x = bf16_torch(p["x"])
+    y = torch.full((cap, N), float("nan"), dtype=torch.bfloat16, device=dev)
+    cuda_lib.moe_grouped_gemm_w4a16(x, w_codes, w_scales, g_w, torch.from_numpy(off).to(dev), E, cap, N, K, y=y)
+    torch.cuda.synchronize()
+    assert cuda_lib.device_status() == cuda_lib.OK
+    got = bf16_np(y)
+    ref, absdot = M.grouped_gemm_w4a16(p["x"][:R], p["w_c"], p["w_s"], p["g_w"], off)
+    assert_close_tol(got[:R], ref, absdot, what="W4A16 GEMM")
+    assert np.all(np.isnan(got[R:]))
+    # against PyTorch: the device fake-quant's W_fq, FP32 matmul, BF16 rounding
+    w_fq = cuda_lib.fakequant_weight_ste(bf16_torch(p["w"]), want_codes=False)[0]
+    for e in range(E):
+        lo, hi = int(off[e]), int(off[e + 1])
+        if hi == lo:
+            continue
+        yt = torch.matmul(x[lo:hi].float(), w_fq[e].float().t())
+        err = (y[lo:hi].float() - yt).abs()
+        bound = 2.0 ** -8 * yt.abs() + K * 2.0 ** -22 * torch.matmul(x[lo:hi].float().abs(), w_fq[e].float().abs().t())
+        assert bool((err <= bound).all()), f"expert {e}: {int((err > bound).sum())} outside the FP32 bound"
+
+
+@pytest.mark.parametrize("counts,F_,K", [([64], 64, 64), ([500, 20, 1000, 3], 192, 1024)])
+def test_grouped_gemm_w4a16_swiglu(cuda_lib, counts, F_, K):
+    """The W4A16 GEMM with the SwiGLU epilogue on 64-row interleaved gate/up
+    weights, bit for bit against the plain W4A16 GEMM followed by the SwiGLU
+    kernel."""
+    p = _w4a16_problem(counts, 2 * F_, K, seed=11 * sum(counts) + F_ + K)
+    E, cap, R, off, N = p["E"], p["cap"], p["R"], p["off"], 2 * F_
+    perm = gate_up_interleave_index(F_)
+    dev = "cuda"
+    w_codes = torch.from_numpy(np.ascontiguousarray(F.pack_nibbles(p["w_c"][:, perm]))).to(dev)
+    w_scales = torch.from_numpy(F.scales_to_tiled(p["w_s"][:, perm].reshape(E * N, K // 16))).to(dev)
+    g_w = torch.tensor(p["g_w"], dtype=torch.float32, device=dev)
+    x = bf16_torch(p["x"])
+    offt = torch.from_numpy(off).to(dev)
+    h, amax = cuda_lib.moe_grouped_gemm_w4a16(x, w_codes, w_scales, g_w, offt, E, cap, N, K, swiglu=True)
+    y_il = cuda_lib.moe_grouped_gemm_w4a16(x, w_codes, w_scales, g_w, offt, E, cap, N, K)
+    y_nat = y_il[:, torch.from_numpy(np.argsort(perm)).cuda()].contiguous()
+    h2, amax2 = cuda_lib.swiglu(y_nat, F_, offt, E)
+    torch.cuda.synchronize()
+    assert cuda_lib.device_status() == cuda_lib.OK
+    assert_bits_equal(F.bf16_bits(bf16_np(h)[:R]), F.bf16_bits(bf16_np(h2)[:R]), "fused vs separate SwiGLU")
+    assert_bits_equal(f32_of(amax).astype(np.float32), f32_of(amax2).astype(np.float32), "amax")

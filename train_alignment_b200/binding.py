@@ -93,6 +93,9 @@ _SIGS = {
                                                             c_i64, c_i64, c_i64, c_vp, c_vp, c_vp, c_vp, c_i64, c_vp,
                                                             c_vp, c_vp]),
     "quads_moe_fp4_comp_amax": (c_i32, [c_vp, c_i32, c_vp, c_vp, c_i32, c_vp, c_vp]),
+    "quads_moe_grouped_gemm_w4a16": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_i32, c_i64, c_i64, c_i64, c_vp, c_vp]),
+    "quads_moe_grouped_gemm_w4a16_swiglu": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_i32, c_i64, c_i64, c_i64, c_vp,
+                                                    c_vp, c_vp]),
     "quads_swiglu": (c_i32, [c_vp, c_i64, c_i64, c_vp, c_i32, c_vp, c_vp, c_vp]),
     "quads_moe_unpermute_combine": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i32, c_i64, c_vp, c_vp]),
     "quads_fakequant_weight_ste": (c_i32, [c_vp, c_i64, c_i64, c_i64, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_i32,
@@ -375,6 +378,26 @@ def moe_grouped_gemm_nvfp4_fp4comp(a_codes, a_scales, g_a, w_codes, w_scales, g_
         _p(a_codes), _p(a_scales), _p(g_a), per_expert, _p(w_codes), _p(w_scales), _p(g_w), _p(expert_off), E,
         rows_cap, N, K, _p(r_codes), _p(r_scales), _p(wc_codes), _p(wc_scales), Kc, _p(y), _s()),
         "quads_moe_grouped_gemm_nvfp4_fp4comp")
+    return y
+
+
+def moe_grouped_gemm_w4a16(x, w_codes, w_scales, g_w, expert_off, E, rows_cap, N, K, y=None, swiglu=False,
+                           amax=None):
+    """Trainer GEMM: BF16 x [rows_cap, K] times the fake-quantized weights
+    given as NVFP4 codes/scales.  swiglu=True returns (h, amax) with N = 2F."""
+    _dev(x, torch.bfloat16, "x")
+    dev = x.device
+    if swiglu:
+        F = N // 2
+        y = y if y is not None else _empty((rows_cap, F), torch.bfloat16, dev)
+        amax = amax if amax is not None else _empty((E,), torch.float32, dev)
+        _check(load().quads_moe_grouped_gemm_w4a16_swiglu(_p(x), _p(w_codes), _p(w_scales), _p(g_w), _p(expert_off),
+                                                          E, rows_cap, F, K, _p(y), _p(amax), _s()),
+               "quads_moe_grouped_gemm_w4a16_swiglu")
+        return y, amax
+    y = y if y is not None else _empty((rows_cap, N), torch.bfloat16, dev)
+    _check(load().quads_moe_grouped_gemm_w4a16(_p(x), _p(w_codes), _p(w_scales), _p(g_w), _p(expert_off), E,
+                                               rows_cap, N, K, _p(y), _s()), "quads_moe_grouped_gemm_w4a16")
     return y
 
 

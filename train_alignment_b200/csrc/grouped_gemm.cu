@@ -56,6 +56,13 @@ constexpr int kBBytes = BN * kStageRowBytes;        // 16384
 constexpr int kSfBytes = 4 * 512;                   // scales of 4 MMAs for 128 rows
 constexpr int kStageBytes = kABytes + kBBytes + 2 * kSfBytes;   // 36864
 constexpr int kCompChunkBytes = 128 * 32;           // 128 rows x 16 BF16
+// W4A16 stage (K = 64): BF16 activations, the weights dequantized to BF16 by
+// the converter warps, the weights' FP4 codes and their 512-byte scale tile
+constexpr int kW16ABytes = BM * 128;                 // 128 rows x 64 BF16
+constexpr int kW16BBytes = BN * 128;
+constexpr int kW16CodeBytes = BN * 32;               // 128 rows x 64 FP4
+constexpr int kW16StageBytes = kW16ABytes + kW16BBytes + kW16CodeBytes + 1024;   // 37888 (1024-aligned)
+__host__ __device__ constexpr int stage_bytes(bool w4a16) { return w4a16 ? kW16StageBytes : kStageBytes; }
 constexpr int kOutChunkBytes = 32 * 64;             // 32 rows x 32 BF16 output columns
 constexpr int kOutStageBytes = 4 * 2 * kOutChunkBytes;   // 4 epilogue warps, 2 buffers each
 constexpr int kThreads = 320;                    // 10 warps
@@ -330,7 +337,13 @@ __device__ __forceinline__ void quantize_h_chunk(const GemmParams& p, const uint
 // per-expert scale g_e = fp32(amax_h_in[e] / 2688): codes, tiled scales and
 // the residual channels, exactly as quads_quantize_nvfp4 of h with that
 // amax; h itself is stored only when y is non-null.
-template <bool kSwiglu, bool kQuant>
+//
+// kW4A16: the trainer-side GEMM Y = X . W_fq^T with BF16 activations X and
+// the weights given as NVFP4 codes and scales: warps 6-9 turn each stage's
+// FP4 weight tile into W_fq = bf16(fp32(val(q) val(s)) g_w[e]) in shared
+// memory (the 128-byte-swizzled K-major layout the MMA reads), and the MMA
+// is kind::f16 (BF16 x BF16, FP32 accumulate); the epilogue stores fp32 acc.
+template <bool kSwiglu, bool kQuant, bool kW4A16>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                         const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_wc,
@@ -342,7 +355,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* const base_ptr = smem_raw + (base - raw);
   const int S = p.stages;
   const int nch = p.n_chan / 16;
-  const uint32_t comp_r = base + S * kStageBytes;
+  constexpr int kSB = stage_bytes(kW4A16);
+  const uint32_t comp_r = base + S * kSB;
   const uint32_t comp_wc = comp_r + nch * kCompChunkBytes;
   const uint32_t out_stage = comp_wc + nch * kCompChunkBytes;     // 1024-byte aligned
   const uint32_t bar0 = out_stage + kOutStageBytes;                 // 8-byte aligned
@@ -357,7 +371,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t drain_bar = comp_full + 56;
   auto sf_full = [&](int i) { return comp_full + 64 + 8u * i; };            // kSfSlots barriers
   auto sf_empty = [&](int i) { return comp_full + 64 + 8u * (kSfSlots + i); };
-  uint8_t* const misc = base_ptr + (comp_full + 64 + 8u * (2 * kSfSlots) + 8 - base);
+  auto conv_bar = [&](int s) { return comp_full + 64 + 8u * (2 * kSfSlots + s); };   // W4A16: S barriers
+  uint8_t* const misc = base_ptr + (comp_full + 64 + 8u * (2 * kSfSlots + S) + 8 - base);
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(misc);
   volatile int* const abort_flag = reinterpret_cast<volatile int*>(misc + 4);
   int32_t* const off_s = reinterpret_cast<int32_t*>(misc + 16);
@@ -386,6 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(sf_full(i), 4);                 // one arrival per scale warp
       mbar_init(sf_empty(i), 1);
     }
+    for (int s = 0; s < S; ++s) mbar_init(conv_bar(s), 4);   // one arrival per converter warp
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -395,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   for (int i = threadIdx.x; i <= p.E; i += blockDim.x) {
     off_s[i] = p.expert_off[i];
-    if (i < p.E) gscale_s[i] = __fmul_rn(p.g_a[p.g_a_per_expert ? i : 0], p.g_w[i]);
+    if (i < p.E) gscale_s[i] = kW4A16 ? p.g_w[i] : __fmul_rn(p.g_a[p.g_a_per_expert ? i : 0], p.g_w[i]);
   }
   if constexpr (kQuant) {
     const int Fh = p.N / 2;
@@ -420,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // row tiles below expert_off[E], never past the buffers' rows_cap rows
   const int total = (min(off_s[p.E], p.rows_cap) / BM) * n_ntiles;
   const int nkb_total = p.K / 64;                 // MMAs along K
-  const int nks_main = (nkb_total + 3) / 4;       // pipeline stages along K
+  const int nks_main = kW4A16 ? nkb_total : (nkb_total + 3) / 4;   // pipeline stages along K
   const int nks = nks_main + (p.nkb_comp + 3) / 4; // then the FP4 compensation's stages
   const int n_col_tiles = nkb_total;              // 512-byte scale tiles per 128-row band
 
@@ -438,8 +454,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = it % S;
         const uint32_t ph = (it / S) & 1;
         if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
-        const uint32_t st = base + s * kStageBytes;
-        if (ks < nks_main) {
+        const uint32_t st = base + s * kSB;
+        if constexpr (kW4A16) {
+          // BF16 activations (64 per row), FP4 weight codes, their scale tile
+          mbar_expect_tx(full_bar(s), kW16ABytes + kW16CodeBytes + 512);
+          tma_load_2d(st, &tm_a, ks * 64, m0, full_bar(s));
+          tma_load_2d(st + kW16ABytes + kW16BBytes, &tm_b, ks * kMmaKBytes, brow, full_bar(s));
+          bulk_load(st + kW16ABytes + kW16BBytes + kW16CodeBytes,
+                    p.w_scales + (static_cast<int64_t>(brow / BM) * n_col_tiles + ks) * 512, 512, full_bar(s));
+        } else if (ks < nks_main) {
           const int nkb = min(4, nkb_total - ks * 4);
           mbar_expect_tx(full_bar(s), kABytes + kBBytes + 2 * nkb * 512);
           tma_load_2d(st, &tm_a, ks * kStageRowBytes, m0, full_bar(s));
@@ -497,9 +520,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ph = (it / S) & 1;
         const int slot = it % kSfSlots;
         if (!mbar_wait(full_bar(s), ph, abort_flag, p.timeout_ns)) { ok = false; break; }
+        if constexpr (kW4A16) {
+          if (!mbar_wait(conv_bar(s), ph, abort_flag, p.timeout_ns)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t st = base + s * kSB;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)      // four K = 16 BF16 MMAs per stage
+            mma_bf16(dacc, desc_kmajor_sw128(st + kk * 32), desc_kmajor_sw128(st + kW16ABytes + kk * 32), kIdescBf16,
+                     (ks | kk) != 0 ? 1u : 0u);
+          tc_commit(empty_bar(s));
+          continue;
+        }
         if (!mbar_wait(sf_full(slot), (it / kSfSlots) & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t st = base + s * kStageBytes;
+        const uint32_t st = base + s * kSB;
         const uint32_t tsfa = tmem + kSfCol + slot * 32;
         const uint32_t tsfb = tsfa + 16;
         if (ks < nks_main) {
@@ -537,6 +571,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit(drain_bar);
       mbar_wait(drain_bar, 0, nullptr, kDrainTimeoutNs);
     }
+  } else if (kW4A16 && warp >= 6) {
+    // ------------------------------------------- W4A16 weight converters
+    // Thread r of warps 6..9 owns weight row r of the tile: its 64 FP4 codes
+    // (32 bytes) and 4 block scales become 64 BF16 values of W_fq written as
+    // row r of the 128-byte-swizzled K-major tile (16-byte chunk j at
+    // j ^ (r % 8)), the layout a TMA load with 128-byte swizzle produces.
+    const int r = (warp - 6) * 32 + lane;
+    int it = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      const int m0 = (t / n_ntiles) * BM;
+      const float g = gscale_s[expert_of_row(off_s, p.E, m0)];
+      for (int ks = 0; ks < nks; ++ks, ++it) {
+        const int s = it % S;
+        const bool w_ok = mbar_wait(full_bar(s), (it / S) & 1, abort_flag, p.timeout_ns);
+        if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+        const uint32_t st = base + s * kSB;
+        const uint32_t cw = st + kW16ABytes + kW16BBytes + r * 32;
+        const uint4 c0 = ld_shared_v4(cw), c1 = ld_shared_v4(cw + 16);
+        const uint4 sv = ld_shared_v4(st + kW16ABytes + kW16BBytes + kW16CodeBytes + (r & 31) * 16);
+        const int qr = (r >> 5) & 3;
+        const uint32_t sc = qr == 0 ? sv.x : (qr == 1 ? sv.y : (qr == 2 ? sv.z : sv.w));
+        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        const uint32_t row = st + kW16ABytes + r * 128;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const QCore q{words[2 * b], words[2 * b + 1], (sc >> (8 * b)) & 0xFFu, 0.0f};
+          uint32_t o[8];
+          deq_block_bf16(q, g, 1, o);
+          st_shared_v4(row + (static_cast<uint32_t>((2 * b) ^ (r & 7)) << 4), o[0], o[1], o[2], o[3]);
+          st_shared_v4(row + (static_cast<uint32_t>((2 * b + 1) ^ (r & 7)) << 4), o[4], o[5], o[6], o[7]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(conv_bar(s));
+      }
+    }
   } else if (warp >= 6) {
     // ------------------------------------------------------- block scales
     // Warps 6..9, one per TMEM lane quarter q: lane i of the quarter reads
@@ -553,7 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (w_ok) w_ok = mbar_wait(sf_empty(slot), ((it / kSfSlots) & 1) ^ 1u, abort_flag, p.timeout_ns);
         if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t sf = base + s * kStageBytes + kABytes + kBBytes + lane * 16;
+        const uint32_t sf = base + s * kSB + kABytes + kBBytes + lane * 16;
         const uint32_t tsf = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + kSfCol + slot * 32;
         uint32_t ra[16], rb[16];
 #pragma unroll
@@ -588,7 +659,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t ph = (tc >> 1) & 1;
       if (!mbar_wait(acc_full0 + 8 * buf, ph, abort_flag, p.timeout_ns)) break;
       tc_fence_after();
-      const float G = gscale_s[e];
+      const float G = kW4A16 ? 1.0f : gscale_s[e];      // W4A16: g_w is inside W_fq
       const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
       constexpr int kChunks = kSwiglu ? BN / 64 : BN / 32;   // 32 output columns each
 #pragma unroll 1
@@ -749,9 +820,9 @@ int make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64
 }
 
 // extra_words: the quantizing epilogue's tables (E + n_chan_h + N / 64 + 1)
-size_t gemm_smem_bytes(int stages, int n_chan, int E, size_t extra_words = 0) {
-  return 1024 + static_cast<size_t>(stages) * kStageBytes + static_cast<size_t>(n_chan / 16) * 2 * kCompChunkBytes +
-         kOutStageBytes + static_cast<size_t>(2 * stages + 9 + 2 * kSfSlots) * 8 + 16 +
+size_t gemm_smem_bytes(int stages, int n_chan, int E, size_t extra_words = 0, int stage_b = kStageBytes) {
+  return 1024 + static_cast<size_t>(stages) * stage_b + static_cast<size_t>(n_chan / 16) * 2 * kCompChunkBytes +
+         kOutStageBytes + static_cast<size_t>(3 * stages + 9 + 2 * kSfSlots) * 8 + 16 +
          (static_cast<size_t>(2 * E + 1) + extra_words) * 4;
 }
 
@@ -789,7 +860,7 @@ extern "C" {
 namespace quads {
 namespace {
 
-template <bool kSwiglu, bool kQuant = false>
+template <bool kSwiglu, bool kQuant = false, bool kW4A16 = false>
 int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_a, int g_a_per_expert,
                 const uint8_t* w_codes, const uint8_t* w_scales, const float* g_w, const int32_t* expert_off, int E,
                 int64_t rows_cap, int64_t N, int64_t K, const uint16_t* a_resid, const uint16_t* w_resid, int n_chan,
@@ -805,7 +876,8 @@ int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_
   QUADS_REQUIRE(E * N < (int64_t(1) << 31), QUADS_ERR_UNSUPPORTED_SHAPE, "E * N too large");
   QUADS_REQUIRE(n_chan >= 0 && n_chan % 16 == 0 && n_chan <= kMaxChan, QUADS_ERR_UNSUPPORTED_SHAPE,
                 "n_chan must be a multiple of 16 in [0, %d]", kMaxChan);
-  QUADS_REQUIRE(a_codes && a_scales && g_a && w_codes && w_scales && g_w && expert_off && (y || kQuant),
+  QUADS_REQUIRE(a_codes && (kW4A16 || (a_scales && g_a)) && w_codes && w_scales && g_w && expert_off &&
+                    (y || kQuant),
                 QUADS_ERR_INVALID_ARG, "null pointer");
   if constexpr (kQuant) {
     QUADS_REQUIRE(hq && hq->amax_in && hq->codes && hq->scales && hq->g_out, QUADS_ERR_INVALID_ARG,
@@ -824,7 +896,8 @@ int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_
                       aligned(fc->w_codes, 16) && aligned(fc->a_scales, 16) && aligned(fc->w_scales, 16),
                   QUADS_ERR_INVALID_ARG, "FP4 compensation operands must be non-null and 16-byte aligned");
   }
-  QUADS_REQUIRE(aligned(a_codes, 16) && aligned(w_codes, 16) && aligned(a_scales, 16) && aligned(w_scales, 16) &&
+  QUADS_REQUIRE(aligned(a_codes, 16) && aligned(w_codes, 16) && (kW4A16 || aligned(a_scales, 16)) &&
+                    aligned(w_scales, 16) &&
                     (!y || aligned(y, 16)) && (n_chan == 0 || (aligned(a_resid, 16) && aligned(w_resid, 16))),
                 QUADS_ERR_INVALID_ARG, "matrix pointers must be 16-byte aligned");
   if (kSwiglu && amax_out && cudaMemsetAsync(amax_out, 0, sizeof(float) * E, stream) != cudaSuccess)
@@ -832,10 +905,18 @@ int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_
   if (rows_cap == 0) return QUADS_OK;
 
   CUtensorMap tm_a, tm_b, tm_r, tm_wc, tm_y;
-  QUADS_TRY(make_map_2d(&tm_a, a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, rows_cap, kStageRowBytes, BM,
-                        CU_TENSOR_MAP_SWIZZLE_128B));
-  QUADS_TRY(make_map_2d(&tm_b, w_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, E * N, kStageRowBytes, BN,
-                        CU_TENSOR_MAP_SWIZZLE_128B));
+  if (kW4A16) {
+    // a_codes holds the BF16 activations [rows_cap][K]; W codes come in 32-byte rows per K = 64
+    QUADS_TRY(make_map_2d(&tm_a, a_codes, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, rows_cap, 64, BM,
+                          CU_TENSOR_MAP_SWIZZLE_128B));
+    QUADS_TRY(make_map_2d(&tm_b, w_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, E * N, kMmaKBytes, BN,
+                          CU_TENSOR_MAP_SWIZZLE_NONE));
+  } else {
+    QUADS_TRY(make_map_2d(&tm_a, a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, rows_cap, kStageRowBytes, BM,
+                          CU_TENSOR_MAP_SWIZZLE_128B));
+    QUADS_TRY(make_map_2d(&tm_b, w_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, E * N, kStageRowBytes, BN,
+                          CU_TENSOR_MAP_SWIZZLE_128B));
+  }
   if (n_chan) {
     QUADS_TRY(make_map_2d(&tm_r, a_resid, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, n_chan, rows_cap, 16, BM,
                           CU_TENSOR_MAP_SWIZZLE_32B));
@@ -860,10 +941,11 @@ int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_
   const size_t extra = kQuant ? static_cast<size_t>(E + hq->n_chan + N / 64 + 1) : 0;
   const size_t smem_cap = 232448;   // 227 KB per block on sm_100
   int stages = kMaxStages;
-  while (stages >= 2 && gemm_smem_bytes(stages, n_chan, E, extra) > smem_cap) --stages;
+  constexpr int kSB = stage_bytes(kW4A16);
+  while (stages >= 2 && gemm_smem_bytes(stages, n_chan, E, extra, kSB) > smem_cap) --stages;
   QUADS_REQUIRE(stages >= 2, QUADS_ERR_UNSUPPORTED_SHAPE, "not enough shared memory for two stages");
-  const size_t smem = gemm_smem_bytes(stages, n_chan, E, extra);
-  if (cudaFuncSetAttribute(grouped_gemm_kernel<kSwiglu, kQuant>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const size_t smem = gemm_smem_bytes(stages, n_chan, E, extra, kSB);
+  if (cudaFuncSetAttribute(grouped_gemm_kernel<kSwiglu, kQuant, kW4A16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return set_error(QUADS_ERR_CUDA, "cannot set %zu bytes of shared memory", smem);
   GemmParams p;
@@ -895,8 +977,8 @@ int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_
   const int64_t max_tiles = (rows_cap / BM) * (N / BN);
   int grid = num_sms();
   if (grid > max_tiles) grid = static_cast<int>(max_tiles);
-  grouped_gemm_kernel<kSwiglu, kQuant><<<grid, kThreads, smem, stream>>>(tm_a, tm_b, tm_r, tm_wc, tm_y, tm_a2, tm_b2,
-                                                                         p);
+  grouped_gemm_kernel<kSwiglu, kQuant, kW4A16><<<grid, kThreads, smem, stream>>>(tm_a, tm_b, tm_r, tm_wc, tm_y,
+                                                                                 tm_a2, tm_b2, p);
   count_launches(1);
   return check_launch("grouped_gemm_kernel");
 }
@@ -941,6 +1023,25 @@ int quads_moe_grouped_gemm_nvfp4_swiglu_fp4comp(const uint8_t* a_codes, const ui
   const Fp4Comp fc{r_codes, r_scales, wc_codes, wc_scales, Kc};
   return launch_gemm<true>(a_codes, a_scales, g_a, g_a_per_expert, w_codes, w_scales, g_w, expert_off, E, rows_cap,
                            2 * F, K, nullptr, nullptr, 0, h, amax_out, stream, nullptr, &fc);
+}
+
+int quads_moe_grouped_gemm_w4a16(const uint16_t* x, const uint8_t* w_codes, const uint8_t* w_scales,
+                                 const float* g_w, const int32_t* expert_off, int E, int64_t rows_cap, int64_t N,
+                                 int64_t K, uint16_t* y, quads_stream_t stream) {
+  clear_error();
+  return launch_gemm<false, false, true>(reinterpret_cast<const uint8_t*>(x), nullptr, nullptr, 0, w_codes, w_scales,
+                                         g_w, expert_off, E, rows_cap, N, K, nullptr, nullptr, 0, y, nullptr, stream);
+}
+
+int quads_moe_grouped_gemm_w4a16_swiglu(const uint16_t* x, const uint8_t* w_codes, const uint8_t* w_scales,
+                                        const float* g_w, const int32_t* expert_off, int E, int64_t rows_cap,
+                                        int64_t F, int64_t K, uint16_t* h, float* amax_out, quads_stream_t stream) {
+  clear_error();
+  QUADS_REQUIRE(F > 0 && F % 64 == 0, QUADS_ERR_UNSUPPORTED_SHAPE, "F (%lld) must be a positive multiple of 64",
+                (long long)F);
+  return launch_gemm<true, false, true>(reinterpret_cast<const uint8_t*>(x), nullptr, nullptr, 0, w_codes, w_scales,
+                                        g_w, expert_off, E, rows_cap, 2 * F, K, nullptr, nullptr, 0, h, amax_out,
+                                        stream);
 }
 
 int quads_moe_fp4_comp_amax(const float* g_a, int g_a_per_expert, const float* g_w, const float* g_wc, int E,
