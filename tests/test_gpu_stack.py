@@ -113,3 +113,25 @@ def test_stack_w4a4_trainer_gap(cuda_lib):
     assert np.all(np.isfinite(gw)) and (cm, sm) == (0, 0)
     print(f"per-token gap, replayed trainer: median {np.median(gq):.4f}; W4A4 QAT trainer: median "
           f"{np.median(gw):.4f}, p90 {np.percentile(gw, 90):.4f}")
+
+
+def test_stack_trainer_w4a16_matches_library(cuda_lib):
+    """The stack's trainer side on the W4A16 kernels (NVFP4 weight codes
+    dequantized on chip) against the same trainer on per-expert BF16 library
+    matmuls with the stored W_fq: the two differ only in FP32 accumulation
+    order and the rounding of intermediate BF16 values, so their outputs
+    agree to a small relative distance per token."""
+    cfg = W.CONFIGS["stack8_t4096_h2048_e64k4_f1024"]
+    st = ST.LayerStack(cfg, seed=0, device="cuda")
+    st.rollout(st.x0)
+    x0_t = W.engine_drift(st.x0, 1e-3, seed=0, device="cuda")
+    y_w4, cm, sm = st.trainer(x0_t)
+    y_w4 = y_w4.float().clone()
+    st.trainer_gemm = "library"
+    y_lib, cm2, sm2 = st.trainer(x0_t)
+    torch.cuda.synchronize()
+    assert cuda_lib.device_status() == cuda_lib.OK
+    assert (cm, sm) == (cm2, sm2)
+    d = torch.linalg.vector_norm(y_w4 - y_lib.float(), dim=1) / torch.linalg.vector_norm(y_lib.float(), dim=1)
+    print(f"W4A16 vs library trainer: per-token relative distance median {d.median():.2e}, max {d.max():.2e}")
+    assert d.median() < 1e-2

@@ -17,9 +17,12 @@ weights W_fq.  In the recorded layers the trainer replays the record
   - the mismatches of its own rounding of the layer input against the
     record are counted.
 The other layers route and compute on the trainer's own activations.  The
-trainer's expert FFNs are BF16 matmuls on W_fq (a plain library GEMM; the
-pages' trainer is a BF16 framework).  The per-token gap between the two
-sides' stack outputs is reported, not pinned.
+trainer's expert FFNs are BF16 x W_fq products ([QUADS-fr §2.2.A]): by
+default the W4A16 grouped GEMM, which reads the weights as their NVFP4 codes
+and dequantizes them on chip (gate/up with the SwiGLU epilogue, then down,
+then the combine kernel); trainer_gemm="library" runs per-expert BF16 library
+matmuls on the stored W_fq instead.  The per-token gap between the two sides'
+stack outputs is reported, not pinned.
 
 The symmetric W4A4 trainer ([QUADS-fr §2.2, ablation studies; §2.1]: QAT
 that fake-quantizes both weights and activations) is the ablation the pages
@@ -37,10 +40,13 @@ from . import workloads as W
 
 
 class LayerStack:
-    def __init__(self, cfg: W.MoEConfig, seed=0, device="cuda", recorded=4):
+    def __init__(self, cfg: W.MoEConfig, seed=0, device="cuda", recorded=4, trainer_gemm="w4a16"):
         self.cfg = cfg
         self.dev = torch.device(device)
         self.recorded = min(recorded, cfg.layers)
+        if trainer_gemm not in ("w4a16", "library"):
+            raise ValueError(f"unknown trainer GEMM {trainer_gemm!r}")
+        self.trainer_gemm = trainer_gemm
         self.w_r = W.stack_router_weights(cfg, seed, device)               # [L, H, E] fp32
         T, H, E = cfg.T, cfg.H, cfg.E
         inp0 = W.moe_layer_inputs(cfg, seed, device, layer=0, with_logits=False)
@@ -59,6 +65,16 @@ class LayerStack:
             x = B.residual_add(x, out)
             self.layers.append(layer)
         self.logits = logits
+        # the trainer's own routing and expert-ordered operands (W4A16 path)
+        cap = B.moe_rows_capacity(T, cfg.k, E)
+        i32, bf = torch.int32, torch.bfloat16
+        self.t_off = torch.empty(E + 1, dtype=i32, device=self.dev)
+        self.t_row_of = torch.empty(T * cfg.k, dtype=i32, device=self.dev)
+        self.t_src_of = torch.full((cap,), -1, dtype=i32, device=self.dev)
+        self.t_ws = torch.empty(B.moe_permute_workspace_bytes(T, cfg.k, E), dtype=torch.uint8, device=self.dev)
+        self.t_x = torch.zeros(cap, H, dtype=bf, device=self.dev)
+        self.t_h = torch.empty(cap, cfg.F, dtype=bf, device=self.dev)
+        self.t_y = torch.empty(cap, H, dtype=bf, device=self.dev)
         self.x_roll = torch.empty(cfg.layers + 1, T, H, dtype=torch.bfloat16, device=self.dev)
         self.x_train = torch.empty_like(self.x_roll)
 
@@ -99,11 +115,32 @@ class LayerStack:
             y.index_add_(0, t, yd * w.reshape(-1)[pos, None])
         return y.to(torch.bfloat16)
 
+    def _trainer_ffn_w4a16(self, layer, x, idx, w):
+        """The same FFN on the W4A16 kernels: the trainer's routing permutes
+        its BF16 rows into expert order (pad rows zero), gate/up + SwiGLU and
+        down read the NVFP4 weight codes, the combine kernel sums the slots."""
+        cfg = self.cfg
+        E, H, F = cfg.E, cfg.H, cfg.F
+        cap = self.t_x.shape[0]
+        B.moe_permute(idx, E, self.t_off, self.t_row_of, self.t_src_of, self.t_ws)
+        src = self.t_src_of.long()
+        torch.where((src >= 0)[:, None], x[src.clamp_min(0)], torch.zeros((), dtype=x.dtype, device=x.device),
+                    out=self.t_x)
+        B.moe_grouped_gemm_w4a16(self.t_x, layer.w_gu_codes, layer.w_gu_scales, layer.g_w_gu, self.t_off, E, cap,
+                                 2 * F, H, y=self.t_h, swiglu=True)
+        B.moe_grouped_gemm_w4a16(self.t_h, layer.w_d_codes, layer.w_d_scales, layer.g_w_d, self.t_off, E, cap, H,
+                                 F, y=self.t_y)
+        return B.moe_unpermute_combine(self.t_y, self.t_row_of, w, cfg.T, cfg.k, H)
+
     def _trainer_down_replayed(self, layer):
         """Down projection of a recorded layer from the replayed h (the
         rollout's effective down-GEMM input, expert-ordered), combined with the
         recorded routing."""
         cfg = self.cfg
+        if self.trainer_gemm == "w4a16":
+            B.moe_grouped_gemm_w4a16(layer.h_hat, layer.w_d_codes, layer.w_d_scales, layer.g_w_d, layer.expert_off,
+                                     cfg.E, layer.cap, cfg.H, cfg.F, y=self.t_y)
+            return B.moe_unpermute_combine(self.t_y, layer.row_of, layer.topk_w, cfg.T, cfg.k, cfg.H)
         off = layer.expert_off.tolist()
         Y = torch.zeros(layer.cap, cfg.H, dtype=torch.bfloat16, device=self.dev)
         for e in range(cfg.E):
@@ -132,7 +169,10 @@ class LayerStack:
             else:
                 B.router_logits(xl, self.w_r[l], out=self.logits)
                 idx, w = B.moe_router_topk(self.logits, cfg.k, True)
-                y = self._trainer_ffn(layer, xl, idx, w, w4a4)
+                if self.trainer_gemm == "w4a16" and not w4a4 and layer.fuse_swiglu:
+                    y = self._trainer_ffn_w4a16(layer, xl, idx, w)
+                else:
+                    y = self._trainer_ffn(layer, xl, idx, w, w4a4)
             B.residual_add(xl, y, out=self.x_train[l + 1])
         return self.x_train[cfg.layers], code_mis, scale_mis
 
