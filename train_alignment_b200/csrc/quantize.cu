@@ -543,6 +543,48 @@ int launch_quantize_mode(const QuantArgs& a, size_t smem, int64_t rows_e, cudaSt
   return check_launch("quantize_kernel");
 }
 
+// Narrow rows (K <= 256) with codes and scales only: one thread per 16-element
+// block instead of one warp per row, so that a row of a few blocks does not
+// leave most lanes idle (the NVFP4 operands of the channel columns and
+// residuals are 64 to 256 wide).  Same operations as quantize_kernel.
+__global__ void __launch_bounds__(kThreads) quantize_narrow_kernel(QuantArgs a, FastDiv nkb_e_div) {
+  extern __shared__ int32_t smem_n[];
+  const int n = a.n_groups;
+  int32_t* off_s = smem_n;                                   // n + 1
+  float* g_s = reinterpret_cast<float*>(smem_n + n + 1);     // n
+  for (int i = threadIdx.x; i <= n; i += blockDim.x) {
+    if (a.group_off != nullptr) off_s[i] = a.group_off[i];
+    if (i < n) {
+      const float g = __fdiv_rn(a.amax[i], kNvfp4Range);
+      g_s[i] = g;
+      if (blockIdx.x == 0 && a.g_out != nullptr) a.g_out[i] = g;
+    }
+  }
+  __syncthreads();
+  const RowGroups grp{a.group_off ? off_s : nullptr, n, a.uniform_div};
+  const bool tiled = a.scale_layout == QUADS_SCALES_TILED;
+  const int nkb = static_cast<int>(a.K / 16);
+  const int64_t rows_valid = a.group_off ? min(a.rows, static_cast<int64_t>(off_s[n])) : a.rows;
+  const int64_t rows_e = tiled ? ceil_div(rows_valid, 128) * 128 : rows_valid;
+  const int nkb_e = static_cast<int>(nkb_e_div.d);
+  const int64_t ncol_tiles = nkb_e / 4;
+  const uint32_t total = static_cast<uint32_t>(rows_e * nkb_e);
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+    const int64_t row = fast_div(i, nkb_e_div);
+    const int kb = static_cast<int>(i - static_cast<uint32_t>(row) * nkb_e);
+    const int64_t so = tiled ? tiled_scale_offset(row, kb, ncol_tiles) : row * nkb + kb;
+    if (row >= rows_valid || kb >= nkb) {            // padding of the tiled layout
+      a.scales[so] = 0;
+      continue;
+    }
+    uint32_t w[8];
+    load_bf16x16(a.x + row * a.ld + kb * 16, w);
+    const QCore q = quant_core(w, g_s[grp.of(row)]);
+    *reinterpret_cast<uint2*>(a.codes + row * (a.K / 2) + kb * 8) = make_uint2(q.lo, q.hi);
+    a.scales[so] = static_cast<uint8_t>(q.scale);
+  }
+}
+
 int launch_quantize(QuantArgs a, cudaStream_t s) {
   if (a.rows == 0) return QUADS_OK;
   QUADS_REQUIRE(a.rows < kMaxBlocks, QUADS_ERR_UNSUPPORTED_SHAPE, "too many rows");
@@ -550,6 +592,18 @@ int launch_quantize(QuantArgs a, cudaStream_t s) {
   const size_t smem = quantize_smem(a.n_groups, a.K, a.n_chan);
   const int64_t rows_e = a.scale_layout == QUADS_SCALES_TILED ? ceil_div(a.rows, 128) * 128 : a.rows;
   const bool any_resid = a.resid != nullptr && a.n_chan > 0;
+  const int nkb = static_cast<int>(a.K / 16);
+  const int nkb_e = a.scale_layout == QUADS_SCALES_TILED ? (nkb + 3) / 4 * 4 : nkb;
+  if (a.codes && a.scales && !a.w_fq && !any_resid && a.ilv_half == 0 && nkb <= 16 &&
+      rows_e * nkb_e < (int64_t(1) << 31)) {
+    const size_t smem_n = (2 * static_cast<size_t>(a.n_groups) + 1) * 4;
+    const int64_t blocks = ceil_div(rows_e * nkb_e, kThreads);
+    const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
+    const int grid = static_cast<int>(blocks < cap ? blocks : cap);
+    quantize_narrow_kernel<<<grid, kThreads, smem_n, s>>>(a, make_fastdiv(static_cast<uint32_t>(nkb_e)));
+    count_launches(1);
+    return check_launch("quantize_narrow_kernel");
+  }
   if (a.codes && a.scales && a.w_fq && a.fold && (!any_resid || a.resid_mode == 1))
     return launch_quantize_mode<1>(a, smem, rows_e, s);
   if (a.codes && a.scales && !a.w_fq && (!any_resid || a.resid_mode == 0))

@@ -47,11 +47,14 @@ struct DirArgs {
   unsigned long long* corrections;
 };
 
-// Index of the largest E2M1 level (0, .5, 1, 1.5, 2, 3, 4, 6) at or below a >= 0.
-__device__ __forceinline__ uint32_t floor_level(float a) {
-  return static_cast<uint32_t>(a >= 0.5f) + static_cast<uint32_t>(a >= 1.0f) + static_cast<uint32_t>(a >= 1.5f) +
-         static_cast<uint32_t>(a >= 2.0f) + static_cast<uint32_t>(a >= 3.0f) + static_cast<uint32_t>(a >= 4.0f) +
-         static_cast<uint32_t>(a >= 6.0f);
+// Index of the largest E2M1 level (0, .5, 1, 1.5, 2, 3, 4, 6) at or below |v|,
+// from the bits of v: the levels from 1 up are the floats 2^e (1 + m/2) with
+// e in 0..2 and one mantissa bit m, so for |v| >= 1 the index is
+// 2 + 2 e + m = (exponent field * 2 + top mantissa bit) - 252 (capped at 7);
+// [0.5, 1) is level 1 and anything below 0.5 (zeros, subnormals) level 0.
+__device__ __forceinline__ uint32_t floor_level(float v) {
+  const int t = static_cast<int>((__float_as_uint(v) & 0x7FFFFFFFu) >> 22) - 252;
+  return t >= 2 ? static_cast<uint32_t>(min(t, 7)) : static_cast<uint32_t>(t >= 0);
 }
 
 // Shared-memory group table; returns the number of rows that belong to a group.
@@ -93,8 +96,8 @@ __global__ void __launch_bounds__(kThreads) direction_bits_kernel(DirArgs a) {
           const uint64_t y = fmul2_rn(bf16x2_to_f32x2(w[i]), inv2);
           const uint32_t cw = (i < 4) ? c.x : c.y;
           const uint32_t c0 = (cw >> (8 * (i & 3))) & 7u, c1 = (cw >> (8 * (i & 3) + 4)) & 7u;
-          out |= static_cast<uint32_t>(c0 > floor_level(fabsf(lo_f32(y)))) << (2 * i);
-          out |= static_cast<uint32_t>(c1 > floor_level(fabsf(hi_f32(y)))) << (2 * i + 1);
+          out |= static_cast<uint32_t>(c0 > floor_level(lo_f32(y))) << (2 * i);
+          out |= static_cast<uint32_t>(c1 > floor_level(hi_f32(y))) << (2 * i + 1);
         }
       }
       *reinterpret_cast<uint16_t*>(a.bits + row * (K / 8) + kb * 2) = static_cast<uint16_t>(out);
@@ -155,7 +158,7 @@ __global__ void __launch_bounds__(kThreads) replay_direction_kernel(DirArgs a) {
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float v = (i & 1) ? hi_f32(y[i >> 1]) : lo_f32(y[i >> 1]);
-            const uint32_t lvl = min(floor_level(fabsf(v)) + ((bits >> i) & 1u), 7u);
+            const uint32_t lvl = min(floor_level(v) + ((bits >> i) & 1u), 7u);
             const uint32_t code = lvl | ((__float_as_uint(v) >> 31) << 3);
             const uint32_t own = (((i < 8) ? own_lo : own_hi) >> (4 * (i & 7))) & 7u;
             fixes += (own != lvl) ? 1u : 0u;
