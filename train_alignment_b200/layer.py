@@ -191,6 +191,9 @@ class MoELayer:
         # the weight side of a step runs on its own stream (see step())
         self.side = torch.cuda.Stream(device=dev)
         self.ev_w_gu, self.ev_w_d = torch.cuda.Event(), torch.cuda.Event()
+        # and the trainer's replays on a third, as soon as their operand is recorded
+        self.trn = torch.cuda.Stream(device=dev)
+        self.ev_x, self.ev_h = torch.cuda.Event(), torch.cuda.Event()
 
     # ---------------------------------------------------------------- stages
 
@@ -311,7 +314,9 @@ class MoELayer:
             B.swiglu(self.y_gu, F, self.expert_off, E, h=self.h, amax=self.amax_h)
             t.mark("swiglu")
 
-    def _rollout_down(self, t):
+    def _rollout_down(self, t, on_h=None):
+        """quantize h (unless the gate/up GEMM did), the down GEMM and the
+        combine; on_h() runs once h's record section is written."""
         cfg = self.cfg
         T, H, E, k, F = cfg.T, cfg.H, cfg.E, cfg.k, cfg.F
         if not self.fuse_requant:
@@ -319,6 +324,8 @@ class MoELayer:
                              scale_layout=B.SCALES_TILED, chan=self.chan_h, codes=self.h_codes,
                              scales=self.h_scales, g_out=self.g_h, resid_out=self.h_resid)
             t.mark("quantize_h")
+        if on_h is not None:
+            on_h()
         if self.comp == "fp4":
             B.moe_fp4_comp_amax(self.g_h, self.g_w_d, self.g_wc_d, E, out=self.amax_r_d)
             B.quantize_nvfp4(self.h_resid, group_off=self.expert_off, n_groups=E, amax_in=self.amax_r_d,
@@ -343,22 +350,30 @@ class MoELayer:
         B.trace_export_qrecord(layer_id, self.cfg.T, self.cfg.k, self.topk_idx, self._tsrc, record=self.record)
 
     def trainer_replay(self, x_train, layer_id=0, timer=None):
-        cfg = self.cfg
         t = timer or StageTimer(False)
+        self._replay_x(x_train, layer_id, t)
+        self._replay_h(layer_id, t)
+
+    def _replay_x(self, x_train, layer_id, t):
+        cfg = self.cfg
         B.trace_replay_qrecord(self.record, layer_id, 0, cfg.T, cfg.H, x_train=x_train, x_hat=self.x_hat,
                                counts=self.counts, status=self.status)
         t.mark("replay_x")
-        B.trace_replay_qrecord(self.record, layer_id, 1, self.cap, cfg.F, x_hat=self.h_hat, status=self.status_h)
+
+    def _replay_h(self, layer_id, t):
+        B.trace_replay_qrecord(self.record, layer_id, 1, self.cap, self.cfg.F, x_hat=self.h_hat, status=self.status_h)
         t.mark("replay_h")
 
     def step(self, x, logits, x_train, grad_gu_fq, grad_d_fq, timer=None, layer_id=0):
-        """One pass of the whole path over one batch, on two streams: the
+        """One pass of the whole path over one batch, on three streams: the
         weight side (amax, fake-quant of gate/up then down, STE backward) on
-        a side stream, the rollout forward, export and replay on the calling
-        stream.  Each GEMM waits only for its own weights, and the call
-        returns with the calling stream joined to the side stream.  The
-        replay's mismatch counters accumulate across steps (zero them with
-        reset_counts())."""
+        a side stream; the rollout forward on the calling stream, each GEMM
+        waiting only for its own weights; the TRACE export (the record's
+        header: its sections are written in place by the rollout's kernels)
+        and the trainer's replays on a third stream, each replay as soon as
+        its operand is recorded.  The call returns with the calling stream
+        joined to both.  The replay's mismatch counters accumulate across
+        steps (zero them with reset_counts())."""
         cfg = self.cfg
         T, H, E, k, F = cfg.T, cfg.H, cfg.E, cfg.k, cfg.F
         t = timer or StageTimer(False)
@@ -386,15 +401,27 @@ class MoELayer:
             self.ev_w_d.record(self.side)
             self.ste_backward(grad_gu_fq, grad_d_fq, t)
         self._rollout_front(x, logits, t)
+        self.ev_x.record(main)
+        self.trn.wait_event(self.ev_x)
+        with torch.cuda.stream(self.trn):
+            t.mark("start")
+            self.export(layer_id)
+            t.mark("export")
+            self._replay_x(x_train, layer_id, t)
         main.wait_event(self.ev_w_gu)
         t.mark("wait_w_gate_up")
         self._rollout_gate_up(t)
         main.wait_event(self.ev_w_d)
         t.mark("wait_w_down")
-        out = self._rollout_down(t)
-        self.export(layer_id)
-        t.mark("export")
-        self.trainer_replay(x_train, layer_id, t)
+
+        def replay_h_when_recorded():
+            self.ev_h.record(main)
+            self.trn.wait_event(self.ev_h)
+            with torch.cuda.stream(self.trn):
+                self._replay_h(layer_id, t)
+
+        out = self._rollout_down(t, replay_h_when_recorded)
+        main.wait_stream(self.trn)
         main.wait_stream(self.side)
         t.mark("join")
         return out
