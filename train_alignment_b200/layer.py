@@ -214,6 +214,16 @@ class MoELayer:
             B.amax_bf16(self.w_d.view(E * H, F), n_groups=E, out=self.amax_w_d)
         t.mark("amax_w")
 
+    def _amax_w_gate_up(self, t):
+        E, F, H = self.cfg.E, self.cfg.F, self.cfg.H
+        B.amax_bf16(self.w_gu.view(E * 2 * F, H), n_groups=E, out=self.amax_w_gu)
+        t.mark("amax_w_gate_up")
+
+    def _amax_w_down(self, t):
+        E, F, H = self.cfg.E, self.cfg.F, self.cfg.H
+        B.amax_bf16(self.w_d.view(E * H, F), n_groups=E, out=self.amax_w_d)
+        t.mark("amax_w_down")
+
     def _fakequant_gate_up(self, t):
         B.fakequant_weight_ste(self.w_gu, True, self.chan_x, False, True, self.w_gu_fq, self.w_gu_codes,
                                self.w_gu_scales, self.g_w_gu, self.wc_gu, None, self.amax_w_gu,
@@ -393,10 +403,13 @@ class MoELayer:
             return out
         self.side.wait_stream(main)
         with torch.cuda.stream(self.side):
+            # gate/up first, so that the gate/up GEMM can start as early as
+            # possible (its amax pass leaves the weights in L2 for the fake-quant)
             t.mark("start")
-            self._amax_w(t)
+            self._amax_w_gate_up(t)
             self._fakequant_gate_up(t)
             self.ev_w_gu.record(self.side)
+            self._amax_w_down(t)
             self._fakequant_down(t)
             self.ev_w_d.record(self.side)
             self.ste_backward(grad_gu_fq, grad_d_fq, t)
