@@ -68,7 +68,7 @@ __device__ __forceinline__ int64_t load_groups(const DirArgs& a, int32_t* off_s,
   return a.group_off ? min(a.rows, static_cast<int64_t>(off_s[n])) : a.rows;
 }
 
-__global__ void __launch_bounds__(kThreads) direction_bits_kernel(DirArgs a) {
+__global__ void __launch_bounds__(kThreads, 4) direction_bits_kernel(DirArgs a) {
   extern __shared__ int32_t smem[];
   int32_t* off_s = smem;
   float* g_s = reinterpret_cast<float*>(smem + a.n_groups + 1);
@@ -82,30 +82,43 @@ __global__ void __launch_bounds__(kThreads) direction_bits_kernel(DirArgs a) {
   for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
        row += warps) {
     const float g = g_s[grp.of(row)];
-    for (int kb = lane; kb < nkb; kb += 32) {
-      const uint32_t s = a.scales[a.tiled ? tiled_scale_offset(row, kb, ncol_tiles) : row * nkb + kb];
-      const float2 e = scale_table_entry(s, g);
-      uint32_t out = 0;
-      if (e.x != 0.0f) {
-        uint32_t w[8];
-        load_bf16x16(a.x + row * K + kb * 16, w);
-        const uint2 c = __ldg(reinterpret_cast<const uint2*>(a.codes + row * (K / 2) + kb * 8));
-        const uint64_t inv2 = pack_f32x2(e.y, e.y);
+    for (int kb0 = lane; kb0 < nkb; kb0 += 64) {
+      // both blocks' loads first: two 32-byte rows of x in flight per lane
+      uint32_t w[2][8], sc[2];
+      uint2 c[2];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint64_t y = fmul2_rn(bf16x2_to_f32x2(w[i]), inv2);
-          const uint32_t cw = (i < 4) ? c.x : c.y;
-          const uint32_t c0 = (cw >> (8 * (i & 3))) & 7u, c1 = (cw >> (8 * (i & 3) + 4)) & 7u;
-          out |= static_cast<uint32_t>(c0 > floor_level(lo_f32(y))) << (2 * i);
-          out |= static_cast<uint32_t>(c1 > floor_level(hi_f32(y))) << (2 * i + 1);
+      for (int u = 0; u < 2; ++u) {
+        const int kb = kb0 + 32 * u;
+        if (kb < nkb) {
+          sc[u] = a.scales[a.tiled ? tiled_scale_offset(row, kb, ncol_tiles) : row * nkb + kb];
+          load_bf16x16(a.x + row * K + kb * 16, w[u]);
+          c[u] = __ldg(reinterpret_cast<const uint2*>(a.codes + row * (K / 2) + kb * 8));
         }
       }
-      *reinterpret_cast<uint16_t*>(a.bits + row * (K / 8) + kb * 2) = static_cast<uint16_t>(out);
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int kb = kb0 + 32 * u;
+        if (kb >= nkb) break;
+        const float2 e = scale_table_entry(sc[u], g);
+        uint32_t out = 0;
+        if (e.x != 0.0f) {
+          const uint64_t inv2 = pack_f32x2(e.y, e.y);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const uint64_t y = fmul2_rn(bf16x2_to_f32x2(w[u][i]), inv2);
+            const uint32_t cw = (i < 4) ? c[u].x : c[u].y;
+            const uint32_t c0 = (cw >> (8 * (i & 3))) & 7u, c1 = (cw >> (8 * (i & 3) + 4)) & 7u;
+            out |= static_cast<uint32_t>(c0 > floor_level(lo_f32(y))) << (2 * i);
+            out |= static_cast<uint32_t>(c1 > floor_level(hi_f32(y))) << (2 * i + 1);
+          }
+        }
+        *reinterpret_cast<uint16_t*>(a.bits + row * (K / 8) + kb * 2) = static_cast<uint16_t>(out);
+      }
     }
   }
 }
 
-__global__ void __launch_bounds__(kThreads) replay_direction_kernel(DirArgs a) {
+__global__ void __launch_bounds__(kThreads, 3) replay_direction_kernel(DirArgs a) {
   extern __shared__ int32_t smem[];
   const int n = a.n_groups;
   const int64_t K = a.K;
@@ -131,66 +144,81 @@ __global__ void __launch_bounds__(kThreads) replay_direction_kernel(DirArgs a) {
   for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
        row += warps) {
     const float g = g_s[grp.of(row)];
-    for (int p = 0; p < npass; ++p) {
-      const int kb = p * 32 + lane;
-      QCore q{0u, 0u, 0u, 0.0f};
-      if (kb < nkb) {
-        const uint32_t s = a.scales[a.tiled ? tiled_scale_offset(row, kb, ncol_tiles) : row * nkb + kb];
-        const float2 e = scale_table_entry(s, g);
-        const uint32_t bits = *reinterpret_cast<const uint16_t*>(a.bits + row * (K / 8) + kb * 2);
-        uint32_t w[8];
-        load_bf16x16(a.x + row * K + kb * 16, w);
-        q.scale = s;
-        q.sv = e4m3_value(s);
-        if (e.x == 0.0f) {
-          // signed zeros, as the quantizer writes for a zero block scale
+    for (int p0 = 0; p0 < npass; p0 += 2) {
+      // both passes' loads first: two 32-byte rows of x_train in flight per lane
+      uint32_t wx[2][8], sx[2], bx[2];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            q.lo |= ((w[i] >> 15) & 1u) << (8 * i + 3) | ((w[i] >> 31) & 1u) << (8 * i + 7);
-            q.hi |= ((w[4 + i] >> 15) & 1u) << (8 * i + 3) | ((w[4 + i] >> 31) & 1u) << (8 * i + 7);
-          }
-        } else {
-          const uint64_t inv2 = pack_f32x2(e.y, e.y);
-          uint64_t y[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) y[i] = fmul2_rn(bf16x2_to_f32x2(w[i]), inv2);
-          const uint32_t own_lo = e2m1x8_from_pairs(y), own_hi = e2m1x8_from_pairs(y + 4);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float v = (i & 1) ? hi_f32(y[i >> 1]) : lo_f32(y[i >> 1]);
-            const uint32_t lvl = min(floor_level(v) + ((bits >> i) & 1u), 7u);
-            const uint32_t code = lvl | ((__float_as_uint(v) >> 31) << 3);
-            const uint32_t own = (((i < 8) ? own_lo : own_hi) >> (4 * (i & 7))) & 7u;
-            fixes += (own != lvl) ? 1u : 0u;
-            if (i < 8) q.lo |= code << (4 * i); else q.hi |= code << (4 * (i - 8));
-          }
+      for (int u = 0; u < 2; ++u) {
+        const int kb = (p0 + u) * 32 + lane;
+        if (kb < nkb) {
+          sx[u] = a.scales[a.tiled ? tiled_scale_offset(row, kb, ncol_tiles) : row * nkb + kb];
+          bx[u] = *reinterpret_cast<const uint16_t*>(a.bits + row * (K / 8) + kb * 2);
+          load_bf16x16(a.x + row * K + kb * 16, wx[u]);
         }
-        uint32_t o[8];
-        deq_block_bf16(q, g, 1, o);
-        uint4* dst = reinterpret_cast<uint4*>(a.x_hat + row * K + kb * 16);
-        dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-        dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
-        if (a.codes_out) *reinterpret_cast<uint2*>(a.codes_out + row * (K / 2) + kb * 8) = make_uint2(q.lo, q.hi);
       }
-      if (a.n_chan) {
-        // compensation channels of this pass: x_hat = bf16(fp32(deq) + r)
-        __syncwarp();
-        const int slo = pass_slot[p], shi = pass_slot[p + 1];
-        for (int j0 = slo; j0 < shi; j0 += 32) {              // warp-uniform
-          const int j = j0 + lane;
-          const bool act = j < shi;
-          const int c = act ? chan_s[j] : 512 * p;
-          const int src = (c - 512 * p) >> 4, bit = c & 15;
-          const uint32_t cl = __shfl_sync(0xffffffffu, q.lo, src);
-          const uint32_t ch = __shfl_sync(0xffffffffu, q.hi, src);
-          const float sv = __shfl_sync(0xffffffffu, q.sv, src);
-          if (act) {
-            const uint32_t code = (((bit < 8) ? cl : ch) >> (4 * (bit & 7))) & 15u;
-            const float v = __fadd_rn(deq_f32(code, sv, g), bf16_bits_to_float(a.resid[row * a.n_chan + j]));
-            a.x_hat[row * K + c] = static_cast<uint16_t>(float_to_bf16_bits(v));
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int p = p0 + u;
+        if (p >= npass) break;                              // warp-uniform
+        const int kb = p * 32 + lane;
+        QCore q{0u, 0u, 0u, 0.0f};
+        if (kb < nkb) {
+          const uint32_t s = sx[u];
+          const float2 e = scale_table_entry(s, g);
+          const uint32_t bits = bx[u];
+          const uint32_t (&w)[8] = wx[u];
+          q.scale = s;
+          q.sv = e4m3_value(s);
+          if (e.x == 0.0f) {
+            // signed zeros, as the quantizer writes for a zero block scale
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              q.lo |= ((w[i] >> 15) & 1u) << (8 * i + 3) | ((w[i] >> 31) & 1u) << (8 * i + 7);
+              q.hi |= ((w[4 + i] >> 15) & 1u) << (8 * i + 3) | ((w[4 + i] >> 31) & 1u) << (8 * i + 7);
+            }
+          } else {
+            const uint64_t inv2 = pack_f32x2(e.y, e.y);
+            uint64_t y[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) y[i] = fmul2_rn(bf16x2_to_f32x2(w[i]), inv2);
+            const uint32_t own_lo = e2m1x8_from_pairs(y), own_hi = e2m1x8_from_pairs(y + 4);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float v = (i & 1) ? hi_f32(y[i >> 1]) : lo_f32(y[i >> 1]);
+              const uint32_t lvl = min(floor_level(v) + ((bits >> i) & 1u), 7u);
+              const uint32_t code = lvl | ((__float_as_uint(v) >> 31) << 3);
+              const uint32_t own = (((i < 8) ? own_lo : own_hi) >> (4 * (i & 7))) & 7u;
+              fixes += (own != lvl) ? 1u : 0u;
+              if (i < 8) q.lo |= code << (4 * i); else q.hi |= code << (4 * (i - 8));
+            }
           }
+          uint32_t o[8];
+          deq_block_bf16(q, g, 1, o);
+          uint4* dst = reinterpret_cast<uint4*>(a.x_hat + row * K + kb * 16);
+          dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+          dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+          if (a.codes_out) *reinterpret_cast<uint2*>(a.codes_out + row * (K / 2) + kb * 8) = make_uint2(q.lo, q.hi);
         }
-        __syncwarp();
+        if (a.n_chan) {
+          // compensation channels of this pass: x_hat = bf16(fp32(deq) + r)
+          __syncwarp();
+          const int slo = pass_slot[p], shi = pass_slot[p + 1];
+          for (int j0 = slo; j0 < shi; j0 += 32) {              // warp-uniform
+            const int j = j0 + lane;
+            const bool act = j < shi;
+            const int c = act ? chan_s[j] : 512 * p;
+            const int src = (c - 512 * p) >> 4, bit = c & 15;
+            const uint32_t cl = __shfl_sync(0xffffffffu, q.lo, src);
+            const uint32_t ch = __shfl_sync(0xffffffffu, q.hi, src);
+            const float sv = __shfl_sync(0xffffffffu, q.sv, src);
+            if (act) {
+              const uint32_t code = (((bit < 8) ? cl : ch) >> (4 * (bit & 7))) & 15u;
+              const float v = __fadd_rn(deq_f32(code, sv, g), bf16_bits_to_float(a.resid[row * a.n_chan + j]));
+              a.x_hat[row * K + c] = static_cast<uint16_t>(float_to_bf16_bits(v));
+            }
+          }
+          __syncwarp();
+        }
       }
     }
   }
