@@ -370,6 +370,8 @@ def _w4a16_problem(counts, N, K, seed):
     ([130, 0, 257], 256, 512),         # empty expert, ragged experts
     ([500, 20, 1000, 3], 384, 1024),
     ([256], 128, 4096),                # long K
+    ([300, 0, 40], 512, 256),          # 256-row weight tiles, an empty expert
+    ([129], 256, 1024),                # 256-row weight tiles, one expert
 ])
 def test_grouped_gemm_w4a16_parity(cuda_lib, counts, N, K):
     """The trainer-side W4A16 GEMM (BF16 activations, NVFP4 weights
@@ -403,7 +405,8 @@ def test_grouped_gemm_w4a16_parity(cuda_lib, counts, N, K):
         assert bool((err <= bound).all()), f"expert {e}: {int((err > bound).sum())} outside the FP32 bound"
 
 
-@pytest.mark.parametrize("counts,F_,K", [([64], 64, 64), ([500, 20, 1000, 3], 192, 1024)])
+@pytest.mark.parametrize("counts,F_,K", [([64], 64, 64), ([500, 20, 1000, 3], 192, 1024),
+                                         ([200, 0, 70], 256, 512), ([130], 128, 64)])
 def test_grouped_gemm_w4a16_swiglu(cuda_lib, counts, F_, K):
     """The W4A16 GEMM with the SwiGLU epilogue on 64-row interleaved gate/up
     weights, bit for bit against the plain W4A16 GEMM followed by the SwiGLU

@@ -56,13 +56,16 @@ constexpr int kBBytes = BN * kStageRowBytes;        // 16384
 constexpr int kSfBytes = 4 * 512;                   // scales of 4 MMAs for 128 rows
 constexpr int kStageBytes = kABytes + kBBytes + 2 * kSfBytes;   // 36864
 constexpr int kCompChunkBytes = 128 * 32;           // 128 rows x 16 BF16
-// W4A16 stage (K = 64): BF16 activations, the weights dequantized to BF16 by
-// the converter warps, the weights' FP4 codes and their 512-byte scale tile
-constexpr int kW16ABytes = BM * 128;                 // 128 rows x 64 BF16
-constexpr int kW16BBytes = BN * 128;
-constexpr int kW16CodeBytes = BN * 32;               // 128 rows x 64 FP4
-constexpr int kW16StageBytes = kW16ABytes + kW16BBytes + kW16CodeBytes + 1024;   // 37888 (1024-aligned)
-__host__ __device__ constexpr int stage_bytes(bool w4a16) { return w4a16 ? kW16StageBytes : kStageBytes; }
+// W4A16 stage (K = 64) for bn weight rows per tile: BF16 activations
+// (128 x 64), the weights dequantized to BF16 by the converter warps
+// (bn x 64), the weights' FP4 codes (bn x 32 bytes), their 512-byte scale
+// tiles (one per 128 rows), padded to 1024 bytes
+constexpr int kW16ABytes = BM * 128;
+__host__ __device__ constexpr int w16_codes_off(int bn) { return kW16ABytes + bn * 128; }
+__host__ __device__ constexpr int w16_scales_off(int bn) { return kW16ABytes + bn * 160; }
+__host__ __device__ constexpr int stage_bytes(bool w4a16, int bn) {
+  return w4a16 ? w16_scales_off(bn) + 1024 : kStageBytes;          // 37888 (bn 128), 58368 (bn 256)
+}
 constexpr int kOutChunkBytes = 32 * 64;             // 32 rows x 32 BF16 output columns
 constexpr int kOutStageBytes = 4 * 2 * kOutChunkBytes;   // 4 epilogue warps, 2 buffers each
 constexpr int kThreads = 320;                    // 10 warps
@@ -80,8 +83,10 @@ constexpr uint64_t kDrainTimeoutNs = 500000000ull;
 // bit 17, scale format UE4M3 (0) at bit 23, M>>4 at bit 24, dense K = 64.
 constexpr uint32_t kIdescFp4 = (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
 // kind::f16: D format F32 (1) at bits 4-5, A/B BF16 (1), K-major, N>>3, M>>4.
-constexpr uint32_t kIdescBf16 =
-    (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+__host__ __device__ constexpr uint32_t idesc_bf16(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(n >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+}
+constexpr uint32_t kIdescBf16 = idesc_bf16(BN);
 
 struct GemmParams {
   const uint8_t* a_scales;
@@ -343,7 +348,7 @@ __device__ __forceinline__ void quantize_h_chunk(const GemmParams& p, const uint
 // FP4 weight tile into W_fq = bf16(fp32(val(q) val(s)) g_w[e]) in shared
 // memory (the 128-byte-swizzled K-major layout the MMA reads), and the MMA
 // is kind::f16 (BF16 x BF16, FP32 accumulate); the epilogue stores fp32 acc.
-template <bool kSwiglu, bool kQuant, bool kW4A16>
+template <bool kSwiglu, bool kQuant, bool kW4A16, int kBN = BN>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                         const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_wc,
@@ -355,7 +360,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* const base_ptr = smem_raw + (base - raw);
   const int S = p.stages;
   const int nch = p.n_chan / 16;
-  constexpr int kSB = stage_bytes(kW4A16);
+  constexpr int kSB = stage_bytes(kW4A16, kBN);
+  static_assert(kBN == BN || kW4A16, "256-row weight tiles are the W4A16 kernel's only");
   const uint32_t comp_r = base + S * kSB;
   const uint32_t comp_wc = comp_r + nch * kCompChunkBytes;
   const uint32_t out_stage = comp_wc + nch * kCompChunkBytes;     // 1024-byte aligned
@@ -432,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const int n_ntiles = p.N / BN;
+  const int n_ntiles = p.N / kBN;
   // row tiles below expert_off[E], never past the buffers' rows_cap rows
   const int total = (min(off_s[p.E], p.rows_cap) / BM) * n_ntiles;
   const int nkb_total = p.K / 64;                 // MMAs along K
@@ -449,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int mt = t / n_ntiles, nt = t - mt * n_ntiles;
       const int m0 = mt * BM;
       const int e = expert_of_row(off_s, p.E, m0);
-      const int brow = e * p.N + nt * BN;
+      const int brow = e * p.N + nt * kBN;
       for (int ks = 0; ks < nks; ++ks, ++it) {
         const int s = it % S;
         const uint32_t ph = (it / S) & 1;
@@ -457,11 +463,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t st = base + s * kSB;
         if constexpr (kW4A16) {
           // BF16 activations (64 per row), FP4 weight codes, their scale tile
-          mbar_expect_tx(full_bar(s), kW16ABytes + kW16CodeBytes + 512);
+          mbar_expect_tx(full_bar(s), kW16ABytes + kBN * 32 + (kBN / 128) * 512);
           tma_load_2d(st, &tm_a, ks * 64, m0, full_bar(s));
-          tma_load_2d(st + kW16ABytes + kW16BBytes, &tm_b, ks * kMmaKBytes, brow, full_bar(s));
-          bulk_load(st + kW16ABytes + kW16BBytes + kW16CodeBytes,
-                    p.w_scales + (static_cast<int64_t>(brow / BM) * n_col_tiles + ks) * 512, 512, full_bar(s));
+          tma_load_2d(st + w16_codes_off(kBN), &tm_b, ks * kMmaKBytes, brow, full_bar(s));
+#pragma unroll
+          for (int b = 0; b < kBN / 128; ++b)
+            bulk_load(st + w16_scales_off(kBN) + b * 512,
+                      p.w_scales + (static_cast<int64_t>(brow / BM + b) * n_col_tiles + ks) * 512, 512, full_bar(s));
         } else if (ks < nks_main) {
           const int nkb = min(4, nkb_total - ks * 4);
           mbar_expect_tx(full_bar(s), kABytes + kBBytes + 2 * nkb * 512);
@@ -514,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t aph = (tc >> 1) & 1;
       if (!mbar_wait(acc_empty0 + 8 * buf, aph ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t dacc = tmem + buf * BN;
+      const uint32_t dacc = tmem + buf * kBN;
       for (int ks = 0; ks < nks; ++ks, ++it) {
         const int s = it % S;
         const uint32_t ph = (it / S) & 1;
@@ -526,8 +534,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t st = base + s * kSB;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)      // four K = 16 BF16 MMAs per stage
-            mma_bf16(dacc, desc_kmajor_sw128(st + kk * 32), desc_kmajor_sw128(st + kW16ABytes + kk * 32), kIdescBf16,
-                     (ks | kk) != 0 ? 1u : 0u);
+            mma_bf16(dacc, desc_kmajor_sw128(st + kk * 32), desc_kmajor_sw128(st + kW16ABytes + kk * 32),
+                     idesc_bf16(kBN), (ks | kk) != 0 ? 1u : 0u);
           tc_commit(empty_bar(s));
           continue;
         }
@@ -573,11 +581,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (kW4A16 && warp >= 6) {
     // ------------------------------------------- W4A16 weight converters
-    // Thread r of warps 6..9 owns weight row r of the tile: its 64 FP4 codes
-    // (32 bytes) and 4 block scales become 64 BF16 values of W_fq written as
-    // row r of the 128-byte-swizzled K-major tile (16-byte chunk j at
-    // j ^ (r % 8)), the layout a TMA load with 128-byte swizzle produces.
-    const int r = (warp - 6) * 32 + lane;
+    // Thread r of warps 6..9 owns weight rows r (and r + 128 in 256-row
+    // tiles): a row's 64 FP4 codes (32 bytes) and 4 block scales become 64
+    // BF16 values of W_fq written as that row of the 128-byte-swizzled
+    // K-major tile (16-byte chunk j at j ^ (row % 8)), the layout a TMA load
+    // with 128-byte swizzle produces.
+    const int r0 = (warp - 6) * 32 + lane;
     int it = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
@@ -588,20 +597,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool w_ok = mbar_wait(full_bar(s), (it / S) & 1, abort_flag, p.timeout_ns);
         if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
         const uint32_t st = base + s * kSB;
-        const uint32_t cw = st + kW16ABytes + kW16BBytes + r * 32;
-        const uint4 c0 = ld_shared_v4(cw), c1 = ld_shared_v4(cw + 16);
-        const uint4 sv = ld_shared_v4(st + kW16ABytes + kW16BBytes + kW16CodeBytes + (r & 31) * 16);
-        const int qr = (r >> 5) & 3;
-        const uint32_t sc = qr == 0 ? sv.x : (qr == 1 ? sv.y : (qr == 2 ? sv.z : sv.w));
-        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-        const uint32_t row = st + kW16ABytes + r * 128;
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          const QCore q{words[2 * b], words[2 * b + 1], (sc >> (8 * b)) & 0xFFu, 0.0f};
-          uint32_t o[8];
-          deq_block_bf16(q, g, 1, o);
-          st_shared_v4(row + (static_cast<uint32_t>((2 * b) ^ (r & 7)) << 4), o[0], o[1], o[2], o[3]);
-          st_shared_v4(row + (static_cast<uint32_t>((2 * b + 1) ^ (r & 7)) << 4), o[4], o[5], o[6], o[7]);
+        for (int h = 0; h < kBN / 128; ++h) {
+          const int r = r0 + 128 * h;
+          const uint32_t cw = st + w16_codes_off(kBN) + r * 32;
+          const uint4 c0 = ld_shared_v4(cw), c1 = ld_shared_v4(cw + 16);
+          const uint4 sv = ld_shared_v4(st + w16_scales_off(kBN) + h * 512 + (r & 31) * 16);
+          const int qr = (r >> 5) & 3;
+          const uint32_t sc = qr == 0 ? sv.x : (qr == 1 ? sv.y : (qr == 2 ? sv.z : sv.w));
+          const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+          const uint32_t row = st + kW16ABytes + r * 128;
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const QCore q{words[2 * b], words[2 * b + 1], (sc >> (8 * b)) & 0xFFu, 0.0f};
+            uint32_t o[8];
+            deq_block_bf16(q, g, 1, o);
+            st_shared_v4(row + (static_cast<uint32_t>((2 * b) ^ (r & 7)) << 4), o[0], o[1], o[2], o[3]);
+            st_shared_v4(row + (static_cast<uint32_t>((2 * b + 1) ^ (r & 7)) << 4), o[4], o[5], o[6], o[7]);
+          }
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -661,14 +674,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const float G = kW4A16 ? 1.0f : gscale_s[e];      // W4A16: g_w is inside W_fq
       const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
-      constexpr int kChunks = kSwiglu ? BN / 64 : BN / 32;   // 32 output columns each
+      constexpr int kChunks = kSwiglu ? kBN / 64 : kBN / 32;   // 32 output columns each
 #pragma unroll 1
       for (int c = 0; c < kChunks; ++c, ++nstore) {
         uint32_t o[16];
         unsigned int hmax = 0u;
         if constexpr (!kSwiglu) {
           uint32_t v[32], w[32];
-          tmem_load32(lane_base + buf * BN + c * 32, v);
+          tmem_load32(lane_base + buf * kBN + c * 32, v);
           if (nch) tmem_load32(lane_base + kCompCol + c * 32, w);
           tmem_wait_ld();
           if (c == kChunks - 1) {
@@ -689,10 +702,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           // read 16 at a time to keep the register footprint small
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf) {
-            const uint32_t col = c * 32 + hf * 16;
+            // gate columns of 128-column half c / 2; the up columns follow 64 later
+            const uint32_t col = (c >> 1) * 128 + (c & 1) * 32 + hf * 16;
             uint32_t vg[16], vu[16], wg[16], wu[16];
-            tmem_load16(lane_base + buf * BN + col, vg);
-            tmem_load16(lane_base + buf * BN + 64 + col, vu);
+            tmem_load16(lane_base + buf * kBN + col, vg);
+            tmem_load16(lane_base + buf * kBN + 64 + col, vu);
             if (nch) {
               tmem_load16(lane_base + kCompCol + col, wg);
               tmem_load16(lane_base + kCompCol + 64 + col, wu);
@@ -727,7 +741,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if constexpr (kQuant) quantize_h_chunk(p, o, gh_s[e], chanh_s, hslot_s, m0 + q * 32 + lane,
-                                               nt * (BN / 2) + c * 32, nt == 0 && c == 0);
+                                               nt * (kBN / 2) + c * 32, nt == 0 && c == 0);
         if (!kQuant || p.y != nullptr) {
           const uint32_t sb = stg + (nstore & 1) * kOutChunkBytes;
           if (lane == 0) bulk_wait_read_1();
@@ -742,7 +756,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&tm_y, sb, (kSwiglu ? nt * (BN / 2) : nt * BN) + c * 32, m0 + q * 32);
+            tma_store_2d(&tm_y, sb, (kSwiglu ? nt * (kBN / 2) : nt * kBN) + c * 32, m0 + q * 32);
             bulk_commit();
           }
         }
@@ -860,14 +874,14 @@ extern "C" {
 namespace quads {
 namespace {
 
-template <bool kSwiglu, bool kQuant = false, bool kW4A16 = false>
+template <bool kSwiglu, bool kQuant = false, bool kW4A16 = false, int kBN = BN>
 int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_a, int g_a_per_expert,
                 const uint8_t* w_codes, const uint8_t* w_scales, const float* g_w, const int32_t* expert_off, int E,
                 int64_t rows_cap, int64_t N, int64_t K, const uint16_t* a_resid, const uint16_t* w_resid, int n_chan,
                 uint16_t* y, float* amax_out, cudaStream_t stream, const HQuant* hq = nullptr,
                 const Fp4Comp* fc = nullptr) {
   QUADS_REQUIRE(E >= 1 && E <= 256, QUADS_ERR_UNSUPPORTED_SHAPE, "E must be in [1, 256]");
-  QUADS_REQUIRE(N > 0 && N % BN == 0 && N <= (int64_t(1) << 20), QUADS_ERR_UNSUPPORTED_SHAPE,
+  QUADS_REQUIRE(N > 0 && N % kBN == 0 && N <= (int64_t(1) << 20), QUADS_ERR_UNSUPPORTED_SHAPE,
                 "N (%lld) must be a positive multiple of 128", (long long)N);
   QUADS_REQUIRE(K > 0 && K % 64 == 0 && K <= (int64_t(1) << 20), QUADS_ERR_UNSUPPORTED_SHAPE,
                 "K (%lld) must be a positive multiple of 64", (long long)K);
@@ -909,7 +923,7 @@ int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_
     // a_codes holds the BF16 activations [rows_cap][K]; W codes come in 32-byte rows per K = 64
     QUADS_TRY(make_map_2d(&tm_a, a_codes, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, rows_cap, 64, BM,
                           CU_TENSOR_MAP_SWIZZLE_128B));
-    QUADS_TRY(make_map_2d(&tm_b, w_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, E * N, kMmaKBytes, BN,
+    QUADS_TRY(make_map_2d(&tm_b, w_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, E * N, kMmaKBytes, kBN,
                           CU_TENSOR_MAP_SWIZZLE_NONE));
   } else {
     QUADS_TRY(make_map_2d(&tm_a, a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, rows_cap, kStageRowBytes, BM,
@@ -941,11 +955,11 @@ int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_
   const size_t extra = kQuant ? static_cast<size_t>(E + hq->n_chan + N / 64 + 1) : 0;
   const size_t smem_cap = 232448;   // 227 KB per block on sm_100
   int stages = kMaxStages;
-  constexpr int kSB = stage_bytes(kW4A16);
+  constexpr int kSB = stage_bytes(kW4A16, kBN);
   while (stages >= 2 && gemm_smem_bytes(stages, n_chan, E, extra, kSB) > smem_cap) --stages;
   QUADS_REQUIRE(stages >= 2, QUADS_ERR_UNSUPPORTED_SHAPE, "not enough shared memory for two stages");
   const size_t smem = gemm_smem_bytes(stages, n_chan, E, extra, kSB);
-  if (cudaFuncSetAttribute(grouped_gemm_kernel<kSwiglu, kQuant, kW4A16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(grouped_gemm_kernel<kSwiglu, kQuant, kW4A16, kBN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return set_error(QUADS_ERR_CUDA, "cannot set %zu bytes of shared memory", smem);
   GemmParams p;
@@ -974,11 +988,11 @@ int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_
   p.n_chan = n_chan;
   p.stages = stages;
   p.timeout_ns = kGemmTimeoutNs;
-  const int64_t max_tiles = (rows_cap / BM) * (N / BN);
+  const int64_t max_tiles = (rows_cap / BM) * (N / kBN);
   int grid = num_sms();
   if (grid > max_tiles) grid = static_cast<int>(max_tiles);
-  grouped_gemm_kernel<kSwiglu, kQuant, kW4A16><<<grid, kThreads, smem, stream>>>(tm_a, tm_b, tm_r, tm_wc, tm_y,
-                                                                                 tm_a2, tm_b2, p);
+  grouped_gemm_kernel<kSwiglu, kQuant, kW4A16, kBN><<<grid, kThreads, smem, stream>>>(tm_a, tm_b, tm_r, tm_wc,
+                                                                                      tm_y, tm_a2, tm_b2, p);
   count_launches(1);
   return check_launch("grouped_gemm_kernel");
 }
@@ -1029,8 +1043,13 @@ int quads_moe_grouped_gemm_w4a16(const uint16_t* x, const uint8_t* w_codes, cons
                                  const float* g_w, const int32_t* expert_off, int E, int64_t rows_cap, int64_t N,
                                  int64_t K, uint16_t* y, quads_stream_t stream) {
   clear_error();
-  return launch_gemm<false, false, true>(reinterpret_cast<const uint8_t*>(x), nullptr, nullptr, 0, w_codes, w_scales,
-                                         g_w, expert_off, E, rows_cap, N, K, nullptr, nullptr, 0, y, nullptr, stream);
+  // 256 weight rows per tile where N allows: half the activation traffic per FLOP
+  const uint8_t* xa = reinterpret_cast<const uint8_t*>(x);
+  if (N % 256 == 0)
+    return launch_gemm<false, false, true, 256>(xa, nullptr, nullptr, 0, w_codes, w_scales, g_w, expert_off, E,
+                                                rows_cap, N, K, nullptr, nullptr, 0, y, nullptr, stream);
+  return launch_gemm<false, false, true>(xa, nullptr, nullptr, 0, w_codes, w_scales, g_w, expert_off, E, rows_cap, N,
+                                         K, nullptr, nullptr, 0, y, nullptr, stream);
 }
 
 int quads_moe_grouped_gemm_w4a16_swiglu(const uint16_t* x, const uint8_t* w_codes, const uint8_t* w_scales,
@@ -1039,9 +1058,12 @@ int quads_moe_grouped_gemm_w4a16_swiglu(const uint16_t* x, const uint8_t* w_code
   clear_error();
   QUADS_REQUIRE(F > 0 && F % 64 == 0, QUADS_ERR_UNSUPPORTED_SHAPE, "F (%lld) must be a positive multiple of 64",
                 (long long)F);
-  return launch_gemm<true, false, true>(reinterpret_cast<const uint8_t*>(x), nullptr, nullptr, 0, w_codes, w_scales,
-                                        g_w, expert_off, E, rows_cap, 2 * F, K, nullptr, nullptr, 0, h, amax_out,
-                                        stream);
+  const uint8_t* xa = reinterpret_cast<const uint8_t*>(x);
+  if (F % 128 == 0)
+    return launch_gemm<true, false, true, 256>(xa, nullptr, nullptr, 0, w_codes, w_scales, g_w, expert_off, E,
+                                               rows_cap, 2 * F, K, nullptr, nullptr, 0, h, amax_out, stream);
+  return launch_gemm<true, false, true>(xa, nullptr, nullptr, 0, w_codes, w_scales, g_w, expert_off, E, rows_cap,
+                                        2 * F, K, nullptr, nullptr, 0, h, amax_out, stream);
 }
 
 int quads_moe_fp4_comp_amax(const float* g_a, int g_a_per_expert, const float* g_w, const float* g_wc, int E,
