@@ -140,7 +140,7 @@ __global__ void __launch_bounds__(kThreads, 3) replay_direction_kernel(DirArgs a
   const int64_t ncol_tiles = ceil_div(nkb, 4);
   const int lane = threadIdx.x & 31;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  unsigned long long fixes = 0;
+  uint32_t fixes = 0;
   for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
        row += warps) {
     const float g = g_s[grp.of(row)];
@@ -181,16 +181,24 @@ __global__ void __launch_bounds__(kThreads, 3) replay_direction_kernel(DirArgs a
             uint64_t y[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) y[i] = fmul2_rn(bf16x2_to_f32x2(w[i]), inv2);
+            // the trainer's own nearest-even codes carry y's sign (negative
+            // zero included); the guided magnitudes are assembled nibble by
+            // nibble, then the sign bits are taken from the own codes and the
+            // differing magnitudes counted 8 at a time
             const uint32_t own_lo = e2m1x8_from_pairs(y), own_hi = e2m1x8_from_pairs(y + 4);
+            uint32_t mag_lo = 0, mag_hi = 0;
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const float v = (i & 1) ? hi_f32(y[i >> 1]) : lo_f32(y[i >> 1]);
               const uint32_t lvl = min(floor_level(v) + ((bits >> i) & 1u), 7u);
-              const uint32_t code = lvl | ((__float_as_uint(v) >> 31) << 3);
-              const uint32_t own = (((i < 8) ? own_lo : own_hi) >> (4 * (i & 7))) & 7u;
-              fixes += (own != lvl) ? 1u : 0u;
-              if (i < 8) q.lo |= code << (4 * i); else q.hi |= code << (4 * (i - 8));
+              if (i < 8) mag_lo |= lvl << (4 * i); else mag_hi |= lvl << (4 * (i - 8));
             }
+            q.lo = mag_lo | (own_lo & 0x88888888u);
+            q.hi = mag_hi | (own_hi & 0x88888888u);
+            uint32_t d0 = (mag_lo ^ own_lo) & 0x77777777u, d1 = (mag_hi ^ own_hi) & 0x77777777u;
+            d0 = (d0 | (d0 >> 1) | (d0 >> 2)) & 0x11111111u;
+            d1 = (d1 | (d1 >> 1) | (d1 >> 2)) & 0x11111111u;
+            fixes += __popc(d0) + __popc(d1);
           }
           uint32_t o[8];
           deq_block_bf16(q, g, 1, o);
@@ -224,8 +232,9 @@ __global__ void __launch_bounds__(kThreads, 3) replay_direction_kernel(DirArgs a
   }
   if (a.corrections) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) fixes += __shfl_xor_sync(0xffffffffu, fixes, o);
-    if (lane == 0 && fixes) atomicAdd(a.corrections, fixes);
+    unsigned long long f = fixes;
+    for (int o = 16; o > 0; o >>= 1) f += __shfl_xor_sync(0xffffffffu, f, o);
+    if (lane == 0 && f) atomicAdd(a.corrections, f);
   }
 }
 
