@@ -231,8 +231,8 @@ __global__ void __launch_bounds__(kThreads, 3) replay_direction_kernel(DirArgs a
     }
   }
   if (a.corrections) {
-#pragma unroll
     unsigned long long f = fixes;
+#pragma unroll
     for (int o = 16; o > 0; o >>= 1) f += __shfl_xor_sync(0xffffffffu, f, o);
     if (lane == 0 && f) atomicAdd(a.corrections, f);
   }
