@@ -57,6 +57,8 @@ def parse():
     ap.add_argument("--serial", action="store_true", help="run the step on one stream (no weight-side overlap)")
     ap.add_argument("--comp", choices=["bf16", "fp4"], default="bf16",
                     help="compensation: BF16 R . Wc (default) or the NVFP4 second pass")
+    ap.add_argument("--trainer-w4a16", action="store_true",
+                    help="the trainer's GEMMs read the NVFP4 codes (W4A16 kernels), so W_fq is not written")
     ap.add_argument("--fuse-requant", action="store_true",
                     help="quantize h in the gate/up GEMM epilogue with the previous step's amax (delayed scaling)")
     return ap.parse_args()
@@ -150,7 +152,7 @@ def gemm_flops(cfg, counts=None):
     return fp4, comp
 
 
-def kernel_work(cfg, rpad):
+def kernel_work(cfg, rpad, wfq=True):
     """Algorithmic bytes (HBM) or FLOPs per launch of every kernel in a step,
     and which roofline bounds it."""
     T, H, E, k, F = cfg.T, cfg.H, cfg.E, cfg.k, cfg.F
@@ -161,8 +163,8 @@ def kernel_work(cfg, rpad):
     q = 0.5 + 1.0 / 16                      # codes + scales per element
     w = {
         "amax_w": ("hbm", 2.0 * (wgu + wd)),
-        "fakequant_w_gate_up": ("hbm", wgu * (2 + 2 + q) + E * 2 * F * nc * 2),
-        "fakequant_w_down": ("hbm", wd * (2 + 2 + q) + E * H * ncf * 2),
+        "fakequant_w_gate_up": ("hbm", wgu * (2 + (2 if wfq else 0) + q) + E * 2 * F * nc * 2),
+        "fakequant_w_down": ("hbm", wd * (2 + (2 if wfq else 0) + q) + E * H * ncf * 2),
         "amax_x": ("hbm", 2.0 * T * H),
         "quantize_x": ("hbm", T * H * (2 + q) + T * nc * 2),
         "router_topk": ("hbm", T * E * 4 + R * 8),
@@ -489,7 +491,8 @@ def run_ours(args):
     B.load()
     cfg = W.CONFIGS[args.workload]
     inp = W.moe_layer_inputs(cfg, seed=rank, device=dev)
-    layer = L.build_layer(cfg, inp, dev, overlap=not args.serial, fuse_requant=args.fuse_requant, comp=args.comp)
+    layer = L.build_layer(cfg, inp, dev, overlap=not args.serial, fuse_requant=args.fuse_requant, comp=args.comp,
+                          materialize_wfq=not args.trainer_w4a16)
     x, logits = inp["x"], inp["logits"]
     x_train = W.engine_drift(x, 1e-2, seed=rank, device=dev)
     g_all, g_gu, g_d = layer.grad_fq_buffers()          # both weight gradients in one allocation
@@ -596,7 +599,7 @@ def run_ours(args):
     # roofline of the dominant kernel: its own launches timed by two events
     # around it alone, in the one-stream step, over args.steps replays
     peaks, peak_src = load_peaks()
-    work = kernel_work(cfg, rpad)
+    work = kernel_work(cfg, rpad, wfq=not args.trainer_w4a16)
     dom = max(per_kernel, key=per_kernel.get)
     bound, amount = work[dom]
     dur = per_kernel[dom] * 1e-3
@@ -695,7 +698,8 @@ def run_ours(args):
                                ("; h quantized in the gate/up GEMM epilogue (delayed amax)" if args.fuse_requant
                                 else "") +
                                ("; FP4 compensation (NVFP4 residual x NVFP4 weight columns)" if args.comp == "fp4"
-                                else ""),
+                                else "") +
+                               ("; trainer on W4A16 GEMMs (W_fq not written)" if args.trainer_w4a16 else ""),
                    "l2": "flushed between steps (256 MiB memset outside the timed events)",
                    "gemm_flops_per_step": fp4 + comp},
         "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,

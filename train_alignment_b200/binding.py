@@ -430,7 +430,7 @@ def moe_unpermute_combine(y, row_of, topk_w, T, k, H, out=None):
 
 
 def fakequant_weight_ste(w, fold_global=True, chan=None, chan_raw=False, want_codes=True, w_fq=None, codes=None,
-                         scales=None, g_out=None, w_chan=None, ws=None, amax_in=None, gate_up=False):
+                         scales=None, g_out=None, w_chan=None, ws=None, amax_in=None, gate_up=False, want_wfq=True):
     """w: [n_mat, rows, K] bf16.  Returns (w_fq, codes, scales, g, w_chan).
     gate_up=True: codes, scales and w_chan in the 64-row gate/up interleaved
     order of quads_fakequant_weight_ste_gate_up."""
@@ -439,7 +439,10 @@ def fakequant_weight_ste(w, fold_global=True, chan=None, chan_raw=False, want_co
     dev = w.device
     n_chan = 0 if chan is None else int(chan.numel())
     layout = SCALES_TILED if rows % 128 == 0 else SCALES_LINEAR
-    w_fq = w_fq if w_fq is not None else _empty((n_mat, rows, K), torch.bfloat16, dev)
+    if want_wfq:
+        w_fq = w_fq if w_fq is not None else _empty((n_mat, rows, K), torch.bfloat16, dev)
+    else:
+        w_fq = None
     if want_codes:
         codes = codes if codes is not None else _empty((n_mat, rows, K // 2), torch.uint8, dev)
         scales = scales if scales is not None else _empty((scales_bytes(n_mat * rows, K, layout),), torch.uint8,

@@ -67,7 +67,7 @@ class MoELayer:
     fixed token count; step() runs the whole path without allocating."""
 
     def __init__(self, cfg: MoEConfig, w_gu, w_d, chan_x, chan_h, device="cuda", fuse_swiglu=None, overlap=True,
-                 fuse_requant=False, amax_h_init=None, comp="bf16"):
+                 fuse_requant=False, amax_h_init=None, comp="bf16", materialize_wfq=True):
         self.cfg = cfg
         T, H, E, k, F = cfg.T, cfg.H, cfg.E, cfg.k, cfg.F
         dev = torch.device(device)
@@ -110,6 +110,10 @@ class MoELayer:
             if not self.fuse_swiglu or self.fuse_requant:
                 raise ValueError("the FP4 compensation runs with the fused SwiGLU epilogue, without fuse_requant")
             chan_x, chan_h = _pad_chan(chan_x, 64), _pad_chan(chan_h, 64)
+        # the trainer's fake-quantized weights W_fq in HBM (False: a trainer
+        # whose GEMMs are the W4A16 kernels reads the NVFP4 codes instead, so
+        # the weight sync writes codes, scales and Wc only)
+        self.materialize_wfq = bool(materialize_wfq)
         # the weight side of a step on its own stream (False: one stream)
         self.overlap = bool(overlap)
         self.nc_x = int(chan_x.numel())
@@ -227,7 +231,7 @@ class MoELayer:
     def _fakequant_gate_up(self, t):
         B.fakequant_weight_ste(self.w_gu, True, self.chan_x, False, True, self.w_gu_fq, self.w_gu_codes,
                                self.w_gu_scales, self.g_w_gu, self.wc_gu, None, self.amax_w_gu,
-                               gate_up=self.fuse_swiglu)
+                               gate_up=self.fuse_swiglu, want_wfq=self.materialize_wfq)
         t.mark("fakequant_w_gate_up")
         if self.comp == "fp4":
             E, F = self.cfg.E, self.cfg.F
@@ -237,7 +241,8 @@ class MoELayer:
 
     def _fakequant_down(self, t):
         B.fakequant_weight_ste(self.w_d, True, self.chan_h, False, True, self.w_d_fq, self.w_d_codes,
-                               self.w_d_scales, self.g_w_d, self.wc_d, None, self.amax_w_d)
+                               self.w_d_scales, self.g_w_d, self.wc_d, None, self.amax_w_d,
+                               want_wfq=self.materialize_wfq)
         t.mark("fakequant_w_down")
         if self.comp == "fp4":
             E, H = self.cfg.E, self.cfg.H
@@ -475,7 +480,8 @@ def calibrate_channels(x, n_sel):
     return out
 
 
-def build_layer(cfg: MoEConfig, inputs, device="cuda", overlap=True, fuse_requant=False, comp="bf16"):
+def build_layer(cfg: MoEConfig, inputs, device="cuda", overlap=True, fuse_requant=False, comp="bf16",
+                materialize_wfq=True):
     """Layer from generated inputs: channel sets calibrated on the layer's own
     batch (X for the gate/up input, the uncompensated h for the down input);
     with fuse_requant, h's first-step per-expert amax is calibrated on the
@@ -492,4 +498,5 @@ def build_layer(cfg: MoEConfig, inputs, device="cuda", overlap=True, fuse_requan
     amax_h = probe.amax_h.clone()
     del probe
     return MoELayer(cfg, inputs["w_gu"], inputs["w_d"], chan_x, chan_h, device, overlap=overlap,
-                    fuse_requant=fuse_requant, amax_h_init=amax_h if fuse_requant else None, comp=comp)
+                    fuse_requant=fuse_requant, amax_h_init=amax_h if fuse_requant else None, comp=comp,
+                    materialize_wfq=materialize_wfq)
