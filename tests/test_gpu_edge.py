@@ -58,10 +58,11 @@ def test_gemm_with_no_routed_rows(cuda_lib):
 
 
 def test_one_token_one_expert_layer(cuda_lib):
-    """T = 1, E = 1, k = 1, hidden 64, ffn 64: the whole step (weight sync,
+    """T = 1, E = 1, k = 1, hidden 128 (the GEMM's smallest output width), ffn
+    64: the whole step (weight sync,
     rollout, record, replay, STE) against the oracle: input codes, routing
     and replayed operand bit-exact, output within 2 % (L2)."""
-    cfg = W.MoEConfig("tiny_t1_h64_e1k1_f64", T=1, H=64, E=1, k=1, F=64, n_chan=16, n_chan_f=16)
+    cfg = W.MoEConfig("tiny_t1_h128_e1k1_f64", T=1, H=128, E=1, k=1, F=64, n_chan=16, n_chan_f=16)
     inp = W.moe_layer_inputs(cfg, seed=5, device="cpu")
     r = np.random.default_rng(5)
     chan_x = Q.pad_channels(np.sort(r.choice(cfg.H, 5, replace=False)))
