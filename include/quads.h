@@ -112,7 +112,8 @@ int quads_amax_bf16(const uint16_t* x, int64_t rows, int64_t K, int64_t ld_x,
  *   ws        device workspace of quads_quantize_workspace_bytes(n_groups)
  *             bytes (may be NULL when amax_in is given).
  * Constraints: K % 16 == 0, K <= 65536, n_groups >= 1 (<= 1024 with
- * group_off), rows >= 0. */
+ * group_off), rows >= 0.  With rows == 0 only g_out is written (zeros) and
+ * codes and scales may be NULL. */
 size_t quads_quantize_workspace_bytes(int n_groups);
 int quads_quantize_nvfp4(const uint16_t* x, int64_t rows, int64_t K, int64_t ld_x,
                          const int32_t* group_off, int n_groups, const float* amax_in,

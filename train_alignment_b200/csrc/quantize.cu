@@ -641,7 +641,8 @@ int quads_quantize_nvfp4(const uint16_t* x, int64_t rows, int64_t K, int64_t ld_
   QUADS_TRY(validate_groups(group_off, n_groups, rows));
   QUADS_REQUIRE(scale_layout == QUADS_SCALES_LINEAR || scale_layout == QUADS_SCALES_TILED,
                 QUADS_ERR_INVALID_ARG, "unknown scale layout %d", scale_layout);
-  QUADS_REQUIRE(codes && scales && g_out, QUADS_ERR_INVALID_ARG, "codes, scales and g_out must be non-null");
+  QUADS_REQUIRE(g_out && (rows == 0 || (codes && scales)), QUADS_ERR_INVALID_ARG,
+                "codes, scales and g_out must be non-null (codes and scales may be null for zero rows)");
   QUADS_REQUIRE(aligned(codes, 8), QUADS_ERR_INVALID_ARG, "codes must be 8-byte aligned");
   QUADS_REQUIRE(n_chan >= 0 && n_chan <= kMaxChan, QUADS_ERR_UNSUPPORTED_SHAPE, "n_chan must be in [0, %d]",
                 kMaxChan);
@@ -871,7 +872,8 @@ extern "C" int quads_quantize_nvfp4_noalloc(const uint16_t* x, int64_t rows, int
                 n_groups);
   QUADS_REQUIRE(scale_layout == QUADS_SCALES_LINEAR || scale_layout == QUADS_SCALES_TILED,
                 QUADS_ERR_INVALID_ARG, "unknown scale layout %d", scale_layout);
-  QUADS_REQUIRE(codes && scales && g_out, QUADS_ERR_INVALID_ARG, "codes, scales and g_out must be non-null");
+  QUADS_REQUIRE(g_out && (rows == 0 || (codes && scales)), QUADS_ERR_INVALID_ARG,
+                "codes, scales and g_out must be non-null (codes and scales may be null for zero rows)");
   QUADS_REQUIRE(aligned(codes, 8), QUADS_ERR_INVALID_ARG, "codes must be 8-byte aligned");
   QUADS_REQUIRE(n_chan >= 0 && n_chan <= kMaxChan, QUADS_ERR_UNSUPPORTED_SHAPE, "n_chan must be in [0, %d]",
                 kMaxChan);

@@ -155,7 +155,9 @@ class MoELayer:
         self.ws_x = e((B.quantize_workspace_bytes(1),), u8)
         self.topk_idx = self.record[hdr.topk_idx_off:hdr.topk_idx_off + 4 * T * k].view(i32).view(T, k)
         self.topk_w = e((T, k), f32)
-        self.expert_off, self.row_of, self.src_of = vh["group_off"], e((T * k,), i32), e((cap,), i32)
+        # one expert: the record keeps no group offsets, so they live outside it
+        goff = vh["group_off"] if vh["group_off"] is not None else e((E + 1,), i32)
+        self.expert_off, self.row_of, self.src_of = goff, e((T * k,), i32), e((cap,), i32)
         self.ws_perm = e((B.moe_permute_workspace_bytes(T, k, E),), u8)
         self.pa_codes, self.pa_scales = e((cap, H // 2), u8), e((B.scales_bytes(cap, H, B.SCALES_TILED),), u8)
         self.pa_resid = e((cap, self.nc_x), bf)
