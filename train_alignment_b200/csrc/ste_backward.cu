@@ -18,9 +18,7 @@ int ste_grid(int64_t work) {
 }
 
 // Each thread keeps kSteUnroll 16-byte vectors of both inputs in flight per
-// iteration of a grid-stride loop.  Every byte is touched once, so loads and
-// stores are streaming (evict-first): the step's other kernels keep their
-// operands in L2.
+// iteration of a grid-stride loop.
 constexpr int kSteUnroll = 4;
 
 __device__ __forceinline__ uint4 ste_add(uint4 a, uint4 b) {
@@ -45,15 +43,15 @@ __global__ void __launch_bounds__(kThreads) ste_backward_kernel(const uint16_t* 
   for (; i + (kSteUnroll - 1) * nth < nv; i += kSteUnroll * nth) {
     uint4 a[kSteUnroll], b[kSteUnroll];
 #pragma unroll
-    for (int u = 0; u < kSteUnroll; ++u) a[u] = __ldcs(src + i + u * nth);
+    for (int u = 0; u < kSteUnroll; ++u) a[u] = __ldg(src + i + u * nth);
     if (accumulate) {
 #pragma unroll
-      for (int u = 0; u < kSteUnroll; ++u) b[u] = __ldcs(dst + i + u * nth);
+      for (int u = 0; u < kSteUnroll; ++u) b[u] = dst[i + u * nth];
 #pragma unroll
       for (int u = 0; u < kSteUnroll; ++u) a[u] = ste_add(a[u], b[u]);
     }
 #pragma unroll
-    for (int u = 0; u < kSteUnroll; ++u) __stcs(dst + i + u * nth, a[u]);
+    for (int u = 0; u < kSteUnroll; ++u) dst[i + u * nth] = a[u];
   }
   for (; i < nv; i += nth) {
     uint4 a = __ldg(src + i);
