@@ -102,14 +102,24 @@ __global__ void __launch_bounds__(kThreads, 4) direction_bits_kernel(DirArgs a) 
         const float2 e = scale_table_entry(sc[u], g);
         uint32_t out = 0;
         if (e.x != 0.0f) {
+          // level nibbles F of 8 elements per word, then per nibble
+          // C > F  <=>  C + (7 - F) >= 8: bit 3 of C + (F ^ 7), no carry out
+          // of a nibble (at most 14); bit 3 of nibble i moved to bit i
           const uint64_t inv2 = pack_f32x2(e.y, e.y);
+          uint32_t f[2] = {0u, 0u};
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const uint64_t y = fmul2_rn(bf16x2_to_f32x2(w[u][i]), inv2);
-            const uint32_t cw = (i < 4) ? c[u].x : c[u].y;
-            const uint32_t c0 = (cw >> (8 * (i & 3))) & 7u, c1 = (cw >> (8 * (i & 3) + 4)) & 7u;
-            out |= static_cast<uint32_t>(c0 > floor_level(lo_f32(y))) << (2 * i);
-            out |= static_cast<uint32_t>(c1 > floor_level(hi_f32(y))) << (2 * i + 1);
+            f[i >> 2] |= (floor_level(lo_f32(y)) | (floor_level(hi_f32(y)) << 4)) << (8 * (i & 3));
+          }
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t cm = (h ? c[u].y : c[u].x) & 0x77777777u;
+            uint32_t m = ((cm + (f[h] ^ 0x77777777u)) >> 3) & 0x11111111u;   // bit 4i = element i
+            m = (m | (m >> 3)) & 0x03030303u;
+            m = (m | (m >> 6)) & 0x000F000Fu;
+            m = (m | (m >> 12)) & 0xFFu;
+            out |= m << (8 * h);
           }
         }
         *reinterpret_cast<uint16_t*>(a.bits + row * (K / 8) + kb * 2) = static_cast<uint16_t>(out);
