@@ -15,7 +15,7 @@ Method statements followed:
 * [TRACE] "Fonctionnement, côté ingénierie": the router's choice of experts
   is discrete, so small numeric differences can change which experts run.
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent:
 * Router: experts ordered by (logit descending, index ascending), first k
   taken; weights are the softmax over the k selected logits (renorm=True) or
   the full softmax restricted to them (renorm=False).
@@ -160,7 +160,7 @@ def bf16_out(v):
 # to the quantized output.  Here the residual R and the weight columns Wc are
 # themselves NVFP4-quantized and multiplied on the FP4 path.
 #
-# Reading (listed in the design doc): Wc_e is quantized per expert with its own
+# Reading: Wc_e is quantized per expert with its own
 # amax (decode scale g_wc[e]); R is quantized per expert segment with the
 # decode scale derived from amax_r[e] = fp32(fp32(G_e / g_wc[e]) * 2688),
 # G_e = fp32(g_a g_w[e]), so that g_r g_wc equals G_e up to one rounding and

@@ -23,7 +23,7 @@ Method statements followed:
   discretized weights).  The backward through the fake-quant is the
   straight-through estimator (identity).
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent:
 * g = fp32(amax / (6 * 448)), so that the largest block scale lands on 448.
 * Block scale: d = fp32(6 * g); t = fp32(a_b / d); s_b = E4M3_RN_satfinite(t).
 * Element codes: S = fp32(val(s_b) * g); inv = fp32(1 / S);

@@ -13,7 +13,7 @@ Method statements followed:
 * [TRACE] "Impact pour les développeurs": the inference engine exports its
   quantization results and the training framework consumes them.
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent:
 * What is recorded for one quantized tensor: the 4-bit codes, the E4M3 block
   scales, the FP32 per-tensor scale(s), the BF16 residual on the
   compensation channels, and, per layer, the router's top-k expert indices.
@@ -103,7 +103,7 @@ def n_blocks(rec):
 # the same choice.  [TRACE] "L'idée centrale": the cache keeps the mantissa
 # and the scale factors selectively to save memory.
 #
-# Reading (listed in the design doc): the compact record keeps, per element, one
+# Reading: the compact record keeps, per element, one
 # bit -- the rounding direction the rollout took -- in place of the 4-bit
 # code, with the block scales and per-tensor scales unchanged.  For an
 # element with scaled value y = fp32(x * fp32(1/S)):
