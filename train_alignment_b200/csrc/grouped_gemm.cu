@@ -69,6 +69,12 @@ __host__ __device__ constexpr int stage_bytes(bool w4a16, int bn) {
 constexpr int kOutChunkBytes = 32 * 64;             // 32 rows x 32 BF16 output columns
 constexpr int kOutStageBytes = 4 * 2 * kOutChunkBytes;   // 4 epilogue warps, 2 buffers each
 constexpr int kThreads = 320;                    // 10 warps
+// The quantizing epilogue does twice the work per column, so its kernel has
+// two epilogue warps per TMEM lane quarter (warps 2-5 and 10-13), each taking
+// every other 32-column chunk.
+__host__ __device__ constexpr int epi_warps(bool quant) { return quant ? 8 : 4; }
+__host__ __device__ constexpr int threads_for(bool quant) { return quant ? 448 : kThreads; }
+__host__ __device__ constexpr int out_stage_bytes(bool quant) { return epi_warps(quant) * 2 * kOutChunkBytes; }
 constexpr int kSfSlots = 4;                      // scale-factor buffers in TMEM
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kCompCol = 256;
@@ -349,7 +355,7 @@ __device__ __forceinline__ void quantize_h_chunk(const GemmParams& p, const uint
 // memory (the 128-byte-swizzled K-major layout the MMA reads), and the MMA
 // is kind::f16 (BF16 x BF16, FP32 accumulate); the epilogue stores fp32 acc.
 template <bool kSwiglu, bool kQuant, bool kW4A16, int kBN = BN>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(threads_for(kQuant), 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                         const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_wc,
                         const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_a2,
@@ -365,7 +371,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t comp_r = base + S * kSB;
   const uint32_t comp_wc = comp_r + nch * kCompChunkBytes;
   const uint32_t out_stage = comp_wc + nch * kCompChunkBytes;     // 1024-byte aligned
-  const uint32_t bar0 = out_stage + kOutStageBytes;                 // 8-byte aligned
+  constexpr int kEpi = epi_warps(kQuant);
+  const uint32_t bar0 = out_stage + out_stage_bytes(kQuant);        // 8-byte aligned
   // barrier addresses
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
@@ -399,9 +406,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(comp_empty, 1);
     mbar_init(acc_full0, 1);
     mbar_init(acc_full0 + 8, 1);
-    mbar_init(acc_empty0, 4);
-    mbar_init(acc_empty0 + 8, 4);
-    mbar_init(compacc_empty, 4);
+    mbar_init(acc_empty0, kEpi);              // one arrival per epilogue warp
+    mbar_init(acc_empty0 + 8, kEpi);
+    mbar_init(compacc_empty, kEpi);
     mbar_init(drain_bar, 1);
     for (int i = 0; i < kSfSlots; ++i) {
       mbar_init(sf_full(i), 4);                 // one arrival per scale warp
@@ -579,7 +586,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit(drain_bar);
       mbar_wait(drain_bar, 0, nullptr, kDrainTimeoutNs);
     }
-  } else if (kW4A16 && warp >= 6) {
+  } else if (kW4A16 && warp >= 6 && warp <= 9) {
     // ------------------------------------------- W4A16 weight converters
     // Thread r of warps 6..9 owns weight rows r (and r + 128 in 256-row
     // tiles): a row's 64 FP4 codes (32 bytes) and 4 block scales become 64
@@ -621,7 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(conv_bar(s));
       }
     }
-  } else if (warp >= 6) {
+  } else if (warp >= 6 && warp <= 9) {
     // ------------------------------------------------------- block scales
     // Warps 6..9, one per TMEM lane quarter q: lane i of the quarter reads
     // row i (16 bytes: rows i, i + 32, i + 64, i + 96 x 4 scales) of each of
@@ -655,14 +662,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(sf_full(slot));
       }
     }
-  } else if (warp >= 2 && warp <= 5) {
+  } else if ((warp >= 2 && warp <= 5) || warp >= 10) {
     // ----------------------------------------------------------- epilogue
     // Each warp owns 32 accumulator rows (its TMEM lane quarter).  Per
     // 32-column chunk: TMEM -> registers -> y = G * acc + comp -> BF16 row in
     // a 2 KB shared buffer -> one TMA store of the 32 x 32 box.  Two buffers
     // per warp; a buffer is rewritten only after its previous store has read it.
+    // With two warps per quarter, warp 10 + i takes the odd chunks of warp 2 + i.
     const int q = warp & 3;
-    const uint32_t stg = out_stage + (warp - 2) * 2 * kOutChunkBytes;
+    const int ew = warp <= 5 ? warp - 2 : warp - 6;                   // 0..kEpi-1
+    constexpr int kStride = kEpi / 4;
+    const int c0 = warp >= 10 ? 1 : 0;
+    const uint32_t stg = out_stage + ew * 2 * kOutChunkBytes;
     int tc = 0, nstore = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++tc) {
       const int mt = t / n_ntiles, nt = t - mt * n_ntiles;
@@ -676,7 +687,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
       constexpr int kChunks = kSwiglu ? kBN / 64 : kBN / 32;   // 32 output columns each
 #pragma unroll 1
-      for (int c = 0; c < kChunks; ++c, ++nstore) {
+      for (int c = c0; c < kChunks; c += kStride, ++nstore) {
+        const bool last = c + kStride >= kChunks;         // this warp's last TMEM read of the tile
         uint32_t o[16];
         unsigned int hmax = 0u;
         if constexpr (!kSwiglu) {
@@ -684,7 +696,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_load32(lane_base + buf * kBN + c * 32, v);
           if (nch) tmem_load32(lane_base + kCompCol + c * 32, w);
           tmem_wait_ld();
-          if (c == kChunks - 1) {
+          if (last) {
             // every TMEM read of this tile is done: hand the accumulators back
             tc_fence_before();
             __syncwarp();
@@ -712,7 +724,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               tmem_load16(lane_base + kCompCol + 64 + col, wu);
             }
             tmem_wait_ld();
-            if (c == kChunks - 1 && hf == 1) {
+            if (last && hf == 1) {
               tc_fence_before();
               __syncwarp();
               if (lane == 0) {
@@ -834,9 +846,10 @@ int make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64
 }
 
 // extra_words: the quantizing epilogue's tables (E + n_chan_h + N / 64 + 1)
-size_t gemm_smem_bytes(int stages, int n_chan, int E, size_t extra_words = 0, int stage_b = kStageBytes) {
+size_t gemm_smem_bytes(int stages, int n_chan, int E, size_t extra_words = 0, int stage_b = kStageBytes,
+                       int out_b = kOutStageBytes) {
   return 1024 + static_cast<size_t>(stages) * stage_b + static_cast<size_t>(n_chan / 16) * 2 * kCompChunkBytes +
-         kOutStageBytes + static_cast<size_t>(3 * stages + 9 + 2 * kSfSlots) * 8 + 16 +
+         out_b + static_cast<size_t>(3 * stages + 9 + 2 * kSfSlots) * 8 + 16 +
          (static_cast<size_t>(2 * E + 1) + extra_words) * 4;
 }
 
@@ -956,9 +969,10 @@ int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_
   const size_t smem_cap = 232448;   // 227 KB per block on sm_100
   int stages = kMaxStages;
   constexpr int kSB = stage_bytes(kW4A16, kBN);
-  while (stages >= 2 && gemm_smem_bytes(stages, n_chan, E, extra, kSB) > smem_cap) --stages;
+  constexpr int kOB = out_stage_bytes(kQuant);
+  while (stages >= 2 && gemm_smem_bytes(stages, n_chan, E, extra, kSB, kOB) > smem_cap) --stages;
   QUADS_REQUIRE(stages >= 2, QUADS_ERR_UNSUPPORTED_SHAPE, "not enough shared memory for two stages");
-  const size_t smem = gemm_smem_bytes(stages, n_chan, E, extra, kSB);
+  const size_t smem = gemm_smem_bytes(stages, n_chan, E, extra, kSB, kOB);
   if (cudaFuncSetAttribute(grouped_gemm_kernel<kSwiglu, kQuant, kW4A16, kBN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return set_error(QUADS_ERR_CUDA, "cannot set %zu bytes of shared memory", smem);
@@ -991,8 +1005,8 @@ int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_
   const int64_t max_tiles = (rows_cap / BM) * (N / kBN);
   int grid = num_sms();
   if (grid > max_tiles) grid = static_cast<int>(max_tiles);
-  grouped_gemm_kernel<kSwiglu, kQuant, kW4A16, kBN><<<grid, kThreads, smem, stream>>>(tm_a, tm_b, tm_r, tm_wc,
-                                                                                      tm_y, tm_a2, tm_b2, p);
+  grouped_gemm_kernel<kSwiglu, kQuant, kW4A16, kBN><<<grid, threads_for(kQuant), smem, stream>>>(
+      tm_a, tm_b, tm_r, tm_wc, tm_y, tm_a2, tm_b2, p);
   count_launches(1);
   return check_launch("grouped_gemm_kernel");
 }
