@@ -534,6 +534,10 @@ int quads_router_logits(const uint16_t* x, int64_t T, int64_t H, const float* w_
  * elements (n % 8 == 0, all three 16-byte aligned; out may alias x or y). */
 int quads_residual_add(const uint16_t* x, const uint16_t* y, int64_t n, uint16_t* out,
                        quads_stream_t stream);
+/* n floats copied device to device by a kernel (not a copy engine): the
+ * delayed-scaling amax handed from one step to the next inside a captured
+ * step, where a copy-engine copy would queue behind host transfers. */
+int quads_copy_f32(const float* src, float* dst, int64_t n, quads_stream_t stream);
 
 #ifdef __cplusplus
 }

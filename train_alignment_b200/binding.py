@@ -93,6 +93,7 @@ _SIGS = {
                                                             c_i64, c_i64, c_i64, c_vp, c_vp, c_vp, c_vp, c_i64, c_vp,
                                                             c_vp, c_vp]),
     "quads_moe_fp4_comp_amax": (c_i32, [c_vp, c_i32, c_vp, c_vp, c_i32, c_vp, c_vp]),
+    "quads_copy_f32": (c_i32, [c_vp, c_vp, c_i64, c_vp]),
     "quads_moe_grouped_gemm_w4a16": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_i32, c_i64, c_i64, c_i64, c_vp, c_vp]),
     "quads_moe_grouped_gemm_w4a16_swiglu": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_i32, c_i64, c_i64, c_i64, c_vp,
                                                     c_vp, c_vp]),
@@ -579,6 +580,11 @@ def trace_replay_direction(bits, scales, scale_layout, g, x_train, group_off=Non
                                          _p(x_train), _p(chan), n_chan, _p(resid) if n_chan else None, _p(x_hat),
                                          _p(codes_out), _p(corrections), _s()), "trace_replay_direction")
     return x_hat, codes_out, corrections
+
+
+def copy_f32(src, dst):
+    _check(load().quads_copy_f32(_p(src), _p(dst), src.numel(), _s()), "quads_copy_f32")
+    return dst
 
 
 def router_logits(x, w_r, out=None):

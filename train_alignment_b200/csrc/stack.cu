@@ -84,6 +84,14 @@ __global__ void __launch_bounds__(256) residual_add_kernel(const uint16_t* x, co
   }
 }
 
+// A few floats copied by the SMs (no copy engine, so a captured step's own
+// small copies never queue behind host transfers on the copy engines).
+__global__ void copy_f32_kernel(const float* src, float* dst, int64_t n) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    dst[i] = src[i];
+}
+
 }  // namespace
 }  // namespace quads
 
@@ -116,6 +124,17 @@ int quads_residual_add(const uint16_t* x, const uint16_t* y, int64_t n, uint16_t
   residual_add_kernel<<<grid, 256, 0, stream>>>(x, y, n, out);
   count_launches(1);
   return check_launch("residual_add_kernel");
+}
+
+int quads_copy_f32(const float* src, float* dst, int64_t n, quads_stream_t stream) {
+  clear_error();
+  QUADS_REQUIRE(n >= 0, QUADS_ERR_INVALID_ARG, "n must be >= 0");
+  if (n == 0) return QUADS_OK;
+  QUADS_REQUIRE(src && dst, QUADS_ERR_INVALID_ARG, "null pointer");
+  const int64_t blocks = ceil_div(n, int64_t(256));
+  copy_f32_kernel<<<static_cast<unsigned>(blocks < 1024 ? blocks : 1024), 256, 0, stream>>>(src, dst, n);
+  count_launches(1);
+  return check_launch("copy_f32_kernel");
 }
 
 }  // extern "C"

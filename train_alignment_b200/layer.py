@@ -317,7 +317,7 @@ class MoELayer:
                 a_resid=self.pa_resid, w_resid=self.wc_gu, h_codes=self.h_codes, h_scales=self.h_scales,
                 h_resid=self.h_resid, g_h=self.g_h, amax_h_out=self.amax_h)
             t.mark("gemm_gate_up_swiglu_quant")
-            self.amax_h_prev.copy_(self.amax_h)         # the next step's scale (a 4E-byte device copy)
+            B.copy_f32(self.amax_h, self.amax_h_prev)   # the next step's scale
         elif self.fuse_swiglu:
             B.moe_grouped_gemm_nvfp4_swiglu(self.pa_codes, self.pa_scales, self.g_x, self.w_gu_codes,
                                             self.w_gu_scales, self.g_w_gu, self.expert_off, E, self.cap, F, H,
