@@ -297,37 +297,28 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a) {
         if (has_scales && kb < nkb_e)
           a.scales[sbase + (tiled ? (kb >> 2) * 512 + (kb & 3) : kb)] = static_cast<uint8_t>(q.scale);
         if (a.resid) {
-          // Channel slot j of this pass is taken by lane j % 32.  The element
-          // itself is read back through L2 (the input row, or, for bf16(deq)
-          // with the scale folded, the W_fq row this warp has just written);
-          // its code and block scale come from the owning lane by shuffles.
+          // Channel slot j of this pass is taken by lane j % 32: the element's
+          // code and block scale come from the owning lane by shuffles (the
+          // input element, where needed, is read back through L2).
+          // bf16(deq) = bf16(fp32(val(q) val(s)) g) is the W_fq value itself.
           const int slo = pass_slot[p], shi = pass_slot[p + 1];
-          const bool from_fq = resid_mode == 1 && fold && has_wfq;
-          if (from_fq) __syncwarp();                     // this warp's W_fq stores are visible to it
           for (int j0 = slo; j0 < shi; j0 += 32) {       // warp-uniform
             const int j = j0 + lane;
             const bool act = j < shi;
             const int c = act ? chan_s[j] : 512 * p;
             const int src = (c - 512 * p) >> 4, bit = c & 15;
-            uint32_t vb;
-            if (from_fq) {
-              vb = act ? a.w_fq[row * a.K + c] : 0u;
+            const uint32_t cl = __shfl_sync(0xffffffffu, q.lo, src);
+            const uint32_t ch = __shfl_sync(0xffffffffu, q.hi, src);
+            const float sv = __shfl_sync(0xffffffffu, q.sv, src);
+            const uint32_t code = (((bit < 8) ? cl : ch) >> (4 * (bit & 7))) & 15u;
+            float v;
+            if (resid_mode == 1) {
+              v = deq_f32(code, sv, g);
             } else {
-              const uint32_t cl = __shfl_sync(0xffffffffu, q.lo, src);
-              const uint32_t ch = __shfl_sync(0xffffffffu, q.hi, src);
-              const float sv = __shfl_sync(0xffffffffu, q.sv, src);
               const float xv = act ? bf16_bits_to_float(__ldg(xr + c)) : 0.0f;
-              const uint32_t code = (((bit < 8) ? cl : ch) >> (4 * (bit & 7))) & 15u;
-              float v;
-              if (resid_mode == 2) {
-                v = xv;
-              } else {
-                const float dq = deq_f32(code, sv, g);
-                v = (resid_mode == 1) ? dq : __fsub_rn(xv, dq);
-              }
-              vb = float_to_bf16_bits(v);
+              v = (resid_mode == 2) ? xv : __fsub_rn(xv, deq_f32(code, sv, g));
             }
-            if (act) a.resid[drow * a.n_chan + j] = static_cast<uint16_t>(vb);
+            if (act) a.resid[drow * a.n_chan + j] = static_cast<uint16_t>(float_to_bf16_bits(v));
           }
         }
       }
