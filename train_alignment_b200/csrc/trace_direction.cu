@@ -18,7 +18,7 @@
 // Both kernels: one warp per row, lane = 16-element block, 32 blocks per pass;
 // HBM-bound streams (direction: 2 + 0.5 B read, 0.125 B written per element;
 // replay: 2 + 0.125 B read, 2 (+ 0.5) B written).
-#include "common.cuh"
+#include "trace_common.cuh"
 
 namespace quads {
 namespace {
@@ -217,26 +217,9 @@ __global__ void __launch_bounds__(kThreads, 3) replay_direction_kernel(DirArgs a
           dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
           if (a.codes_out) *reinterpret_cast<uint2*>(a.codes_out + row * (K / 2) + kb * 8) = make_uint2(q.lo, q.hi);
         }
-        if (a.n_chan) {
-          // compensation channels of this pass: x_hat = bf16(fp32(deq) + r)
-          __syncwarp();
-          const int slo = pass_slot[p], shi = pass_slot[p + 1];
-          for (int j0 = slo; j0 < shi; j0 += 32) {              // warp-uniform
-            const int j = j0 + lane;
-            const bool act = j < shi;
-            const int c = act ? chan_s[j] : 512 * p;
-            const int src = (c - 512 * p) >> 4, bit = c & 15;
-            const uint32_t cl = __shfl_sync(0xffffffffu, q.lo, src);
-            const uint32_t ch = __shfl_sync(0xffffffffu, q.hi, src);
-            const float sv = __shfl_sync(0xffffffffu, q.sv, src);
-            if (act) {
-              const uint32_t code = (((bit < 8) ? cl : ch) >> (4 * (bit & 7))) & 15u;
-              const float v = __fadd_rn(deq_f32(code, sv, g), bf16_bits_to_float(a.resid[row * a.n_chan + j]));
-              a.x_hat[row * K + c] = static_cast<uint16_t>(float_to_bf16_bits(v));
-            }
-          }
-          __syncwarp();
-        }
+        if (a.n_chan)                // compensation channels of this pass: x_hat = bf16(fp32(deq) + r)
+          replay_channel_pass(q, g, p, pass_slot[p], pass_slot[p + 1], chan_s, a.resid + row * a.n_chan,
+                              a.x_hat + row * K);
       }
     }
   }

@@ -13,7 +13,7 @@
 // scales its own rounding would have chosen differently.
 #include <cstring>
 
-#include "common.cuh"
+#include "trace_common.cuh"
 
 namespace quads {
 namespace {
@@ -190,25 +190,9 @@ __global__ void __launch_bounds__(kThreads, 3) replay_kernel(ReplayArgs a) {
           }
         }
         if (d.n_chan) {
-          // compensation channels of this pass: x_hat = bf16(fp32(deq) + r),
-          // rewritten after the block stores above
-          __syncwarp();
-          const int slo = pass_slot[p], shi = pass_slot[p + 1];
-          for (int j0 = slo; j0 < shi; j0 += 32) {       // warp-uniform
-            const int j = j0 + lane;
-            const bool act = j < shi;
-            const int c = act ? chan_s[j] : 512 * p;
-            const int src = (c - 512 * p) >> 4, bit = c & 15;
-            const uint32_t cl = __shfl_sync(0xffffffffu, q.lo, src);
-            const uint32_t ch = __shfl_sync(0xffffffffu, q.hi, src);
-            const float sv = __shfl_sync(0xffffffffu, q.sv, src);
-            if (act) {
-              const uint32_t code = (((bit < 8) ? cl : ch) >> (4 * (bit & 7))) & 15u;
-              const float v = __fadd_rn(deq_f32(code, sv, g), bf16_bits_to_float(resid_rec[row * d.n_chan + j]));
-              a.x_hat[row * K + c] = static_cast<uint16_t>(float_to_bf16_bits(v));
-            }
-          }
-          __syncwarp();
+          // compensation channels of this pass, rewritten after the block stores above
+          replay_channel_pass(q, g, p, pass_slot[p], pass_slot[p + 1], chan_s, resid_rec + row * d.n_chan,
+                              a.x_hat + row * K);
         }
       }
     }
