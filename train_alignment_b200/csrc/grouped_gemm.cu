@@ -73,7 +73,12 @@ constexpr int kThreads = 320;                    // 10 warps
 // two epilogue warps per TMEM lane quarter (warps 2-5 and 10-13), each taking
 // every other 32-column chunk.
 __host__ __device__ constexpr int epi_warps(bool quant) { return quant ? 8 : 4; }
-__host__ __device__ constexpr int threads_for(bool quant) { return quant ? 448 : kThreads; }
+// The W4A16 kernel's weight conversion is on its critical path, so it has
+// eight converter warps (6-13), one weight row per thread for 256-row tiles.
+__host__ __device__ constexpr int conv_warps(bool w4a16) { return w4a16 ? 8 : 0; }
+__host__ __device__ constexpr int threads_for(bool quant, bool w4a16 = false) {
+  return (quant || w4a16) ? 448 : kThreads;
+}
 __host__ __device__ constexpr int out_stage_bytes(bool quant) { return epi_warps(quant) * 2 * kOutChunkBytes; }
 constexpr int kSfSlots = 4;                      // scale-factor buffers in TMEM
 constexpr uint32_t kTmemCols = 512;
@@ -355,7 +360,7 @@ __device__ __forceinline__ void quantize_h_chunk(const GemmParams& p, const uint
 // memory (the 128-byte-swizzled K-major layout the MMA reads), and the MMA
 // is kind::f16 (BF16 x BF16, FP32 accumulate); the epilogue stores fp32 acc.
 template <bool kSwiglu, bool kQuant, bool kW4A16, int kBN = BN>
-__global__ void __launch_bounds__(threads_for(kQuant), 1)
+__global__ void __launch_bounds__(threads_for(kQuant, kW4A16), 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                         const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_wc,
                         const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_a2,
@@ -414,7 +419,7 @@ __global__ void __launch_bounds__(threads_for(kQuant), 1)
       mbar_init(sf_full(i), 4);                 // one arrival per scale warp
       mbar_init(sf_empty(i), 1);
     }
-    for (int s = 0; s < S; ++s) mbar_init(conv_bar(s), 4);   // one arrival per converter warp
+    for (int s = 0; s < S; ++s) mbar_init(conv_bar(s), conv_warps(true));   // one arrival per converter warp
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -586,14 +591,15 @@ __global__ void __launch_bounds__(threads_for(kQuant), 1)
       tc_commit(drain_bar);
       mbar_wait(drain_bar, 0, nullptr, kDrainTimeoutNs);
     }
-  } else if (kW4A16 && warp >= 6 && warp <= 9) {
+  } else if (kW4A16 && warp >= 6) {
     // ------------------------------------------- W4A16 weight converters
-    // Thread r of warps 6..9 owns weight rows r (and r + 128 in 256-row
-    // tiles): a row's 64 FP4 codes (32 bytes) and 4 block scales become 64
-    // BF16 values of W_fq written as that row of the 128-byte-swizzled
-    // K-major tile (16-byte chunk j at j ^ (row % 8)), the layout a TMA load
-    // with 128-byte swizzle produces.
-    const int r0 = (warp - 6) * 32 + lane;
+    // Thread r of warps 6..13 owns weight row r of the tile (threads past
+    // the tile's rows idle): the row's 64 FP4 codes (32 bytes) and 4 block
+    // scales (in the 512-byte tile of its 128-row band) become 64 BF16 values
+    // of W_fq written as that row of the 128-byte-swizzled K-major tile
+    // (16-byte chunk j at j ^ (row % 8)), the layout a TMA load with 128-byte
+    // swizzle produces.
+    const int r0 = (warp - 6) * 32 + lane;                            // 0..255
     int it = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
@@ -605,11 +611,12 @@ __global__ void __launch_bounds__(threads_for(kQuant), 1)
         if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
         const uint32_t st = base + s * kSB;
 #pragma unroll
-        for (int h = 0; h < kBN / 128; ++h) {
-          const int r = r0 + 128 * h;
+        for (int h = 0; h < (kBN + 255) / 256; ++h) {
+          const int r = r0 + 256 * h;
+          if (r >= kBN) break;
           const uint32_t cw = st + w16_codes_off(kBN) + r * 32;
           const uint4 c0 = ld_shared_v4(cw), c1 = ld_shared_v4(cw + 16);
-          const uint4 sv = ld_shared_v4(st + w16_scales_off(kBN) + h * 512 + (r & 31) * 16);
+          const uint4 sv = ld_shared_v4(st + w16_scales_off(kBN) + (r >> 7) * 512 + (r & 31) * 16);
           const int qr = (r >> 5) & 3;
           const uint32_t sc = qr == 0 ? sv.x : (qr == 1 ? sv.y : (qr == 2 ? sv.z : sv.w));
           const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
@@ -662,7 +669,7 @@ __global__ void __launch_bounds__(threads_for(kQuant), 1)
         if (lane == 0) mbar_arrive(sf_full(slot));
       }
     }
-  } else if ((warp >= 2 && warp <= 5) || warp >= 10) {
+  } else if ((warp >= 2 && warp <= 5) || (kQuant && warp >= 10)) {
     // ----------------------------------------------------------- epilogue
     // Each warp owns 32 accumulator rows (its TMEM lane quarter).  Per
     // 32-column chunk: TMEM -> registers -> y = G * acc + comp -> BF16 row in
@@ -1005,7 +1012,7 @@ int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_
   const int64_t max_tiles = (rows_cap / BM) * (N / kBN);
   int grid = num_sms();
   if (grid > max_tiles) grid = static_cast<int>(max_tiles);
-  grouped_gemm_kernel<kSwiglu, kQuant, kW4A16, kBN><<<grid, threads_for(kQuant), smem, stream>>>(
+  grouped_gemm_kernel<kSwiglu, kQuant, kW4A16, kBN><<<grid, threads_for(kQuant, kW4A16), smem, stream>>>(
       tm_a, tm_b, tm_r, tm_wc, tm_y, tm_a2, tm_b2, p);
   count_launches(1);
   return check_launch("grouped_gemm_kernel");
