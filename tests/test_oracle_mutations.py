@@ -6,6 +6,7 @@ import pytest
 from oracle import formats as F
 from oracle import moe as M
 from oracle import nvfp4 as Q
+from oracle import stack as ST
 from oracle import trace as TR
 from tests import oracle_pins as P
 
@@ -127,6 +128,23 @@ def _comp_amax_uses_gw(g_a, g_w, g_wc):
     return M.__dict__["_orig_comp_amax"](g_a, g_w, np.asarray(g_w, dtype=np.float64) * 4.0)
 
 
+def _w4a16_unfolded(x, w_codes, w_scales, g_w, expert_off):
+    # the per-expert scale dropped from W_fq
+    return M.__dict__["_orig_w4a16"](x, w_codes, w_scales, np.ones(len(g_w)), expert_off)
+
+
+def _residual_add_no_bf16(x, y):
+    # the BF16 rounding of the sum dropped
+    return F.f32(np.asarray(x, dtype=np.float64) + np.asarray(y, dtype=np.float64))
+
+
+def _router_logits_abs(x, w_r):
+    # the magnitude product used for the logits themselves
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(w_r, dtype=np.float64)
+    return np.abs(x) @ np.abs(w), np.abs(x) @ np.abs(w)
+
+
 MUTATIONS = {
     "e2m1_ties_away": [(F, "e2m1_rne_code", _e2m1_ties_up), (Q, "e2m1_rne_code", _e2m1_ties_up)],
     "e2m1_drops_sign": [(F, "e2m1_rne_code", _e2m1_no_sign), (Q, "e2m1_rne_code", _e2m1_no_sign)],
@@ -143,6 +161,9 @@ MUTATIONS = {
     "swiglu_gate_up_swapped": [(M, "swiglu", _swiglu_wrong)],
     "nibble_order": [(F, "pack_nibbles", _pack_swapped)],
     "channel_ties_to_high_index": [(Q, "select_channels", _select_ties_high)],
+    "w4a16_drops_weight_scale": [(M, "_orig_w4a16", M.grouped_gemm_w4a16), (M, "grouped_gemm_w4a16", _w4a16_unfolded)],
+    "residual_add_keeps_fp32": [(ST, "residual_add", _residual_add_no_bf16)],
+    "router_logits_magnitudes": [(ST, "router_logits", _router_logits_abs)],
     "fp4_comp_wrong_scale": [(M, "_orig_comp_amax", M.fp4_comp_amax), (M, "fp4_comp_amax", _comp_amax_uses_gw)],
     "direction_floor_off_by_one": [(TR, "_floor_level_index", _floor_level_left)],
     "direction_bit_ignored": [(TR, "_orig_replay_dir", TR.replay_direction),
