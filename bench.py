@@ -318,6 +318,81 @@ def trainer_gemm_timing(layer, dev, peaks, reps=20):
     return out
 
 
+def _timed_flushed(fn, flush, reps=20):
+    import torch
+    fn()
+    ts = []
+    for _ in range(reps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    ts.sort()
+    return ts[len(ts) // 2]
+
+
+def _gemm_calls(layer, comp=True):
+    """The layer's two grouped GEMMs on its current operands (after a
+    rollout): gate/up with the SwiGLU epilogue, and down."""
+    from train_alignment_b200 import binding as B
+    cfg = layer.cfg
+    E, H, F = cfg.E, cfg.H, cfg.F
+    gu = lambda: B.moe_grouped_gemm_nvfp4_swiglu(
+        layer.pa_codes, layer.pa_scales, layer.g_x, layer.w_gu_codes, layer.w_gu_scales, layer.g_w_gu,
+        layer.expert_off, E, layer.cap, F, H, layer.pa_resid if comp else None, layer.wc_gu if comp else None,
+        h=layer.h, amax=layer.amax_h)
+    dn = lambda: B.moe_grouped_gemm_nvfp4(
+        layer.h_codes, layer.h_scales, layer.g_h, layer.w_d_codes, layer.w_d_scales, layer.g_w_d, layer.expert_off,
+        E, layer.cap, H, F, layer.h_resid if comp else None, layer.wc_d if comp else None, y=layer.y_d)
+    return gu, dn
+
+
+def gemm_side_measurements(layer, dev, peaks):
+    """(1) The compensation's cost: the step layer's two grouped GEMMs with
+    and without the BF16 correction on the same operands.  (2) Decode
+    shapes (2048 hidden, 128 experts top-8, ffn 768, T = 64 and 512), judged
+    as weight-stream bandwidth: the NVFP4 weight bytes (codes, scales and the
+    BF16 Wc columns) of every expert that received rows, over the GEMM time.
+    L2 flushed before each timed launch."""
+    import torch
+    from train_alignment_b200 import layer as L
+    from train_alignment_b200 import workloads as W
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    out = {}
+    gu, dn = _gemm_calls(layer, True)
+    gu0, dn0 = _gemm_calls(layer, False)
+    t = {k: _timed_flushed(f, flush) * 1e3 for k, f in (("gate_up", gu), ("down", dn), ("gate_up_nocomp", gu0),
+                                                         ("down_nocomp", dn0))}
+    tot, tot0 = t["gate_up"] + t["down"], t["gate_up_nocomp"] + t["down_nocomp"]
+    out["compensation"] = {"us_with": tot, "us_without": tot0, "overhead_frac": tot / tot0 - 1.0,
+                           "gate_up_us": [t["gate_up"], t["gate_up_nocomp"]], "down_us": [t["down"], t["down_nocomp"]]}
+    dec = []
+    for T in (64, 512):
+        cfg = W.decode_config(T)
+        inp = W.moe_layer_inputs(cfg, seed=0, device=dev)
+        ly = L.build_layer(cfg, inp, dev)
+        ly.weight_sync()
+        ly.rollout_forward(inp["x"], inp["logits"])
+        torch.cuda.synchronize()
+        off = ly.expert_off.tolist()
+        used = sum(1 for e in range(cfg.E) if off[e + 1] > off[e])
+        g, d = _gemm_calls(ly, True)
+        tg, td = _timed_flushed(g, flush) * 1e3, _timed_flushed(d, flush) * 1e3
+        q = 0.5 + 1.0 / 16
+        wb_g = used * 2 * cfg.F * (cfg.H * q + ly.nc_x * 2)
+        wb_d = used * cfg.H * (cfg.F * q + ly.nc_h * 2)
+        dec.append({"workload": cfg.name, "experts_with_rows": used, "gate_up_us": tg, "down_us": td,
+                    "weight_bytes": wb_g + wb_d, "weight_stream_gbs": (wb_g + wb_d) / ((tg + td) * 1e-6) / 1e9,
+                    "frac_hbm": (wb_g + wb_d) / ((tg + td) * 1e-6) / 1e9 / peaks["hbm_gbs"]})
+        del ly, inp
+        torch.cuda.empty_cache()
+    out["decode"] = dec
+    return out
+
+
 # ------------------------------------------------------------------- clocks
 
 
@@ -713,6 +788,7 @@ def run_ours(args):
     if not args.no_sweep:
         sweep = quantize_replay_sweep(dev, peaks["hbm_gbs"])
     trainer = trainer_gemm_timing(layer, dev, peaks) if not args.no_sweep else None
+    gemm_side = gemm_side_measurements(layer, dev, peaks) if not args.no_sweep and layer.comp == "bf16" else None
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -753,6 +829,7 @@ def run_ours(args):
         "instrumented_ms_per_step": sum(inst_ms) / len(inst_ms),
         "quantize_replay_sweep": sweep,
         "trainer_gemm": trainer,
+        "gemm_side": gemm_side,
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)
