@@ -240,8 +240,9 @@ int quads_moe_grouped_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales
                                  const uint16_t* a_resid, const uint16_t* w_resid, int n_chan,
                                  uint16_t* y, quads_stream_t stream);
 
-/* a6 + a7 in one pass: the gate/up grouped GEMM with the SwiGLU applied in
- * the epilogue.  The operands are those of quads_moe_grouped_gemm_nvfp4 with
+/* a6 + a7 in one pass ([QUADS-fr §1]: the rollout's MoE expert GEMMs in
+ * NVFP4; the SwiGLU expert FFN is a reading, the pages name no activation):
+ * the gate/up grouped GEMM with the SwiGLU applied in the epilogue.  The operands are those of quads_moe_grouped_gemm_nvfp4 with
  * N = 2F, except that the W rows (w_codes, w_scales, w_resid) are in the
  * 64-row interleaved gate/up order that quads_fakequant_weight_ste_gate_up
  * writes.  Each 128-row tile then holds gate rows 64b..64b+63 followed by the
@@ -318,8 +319,9 @@ int quads_moe_grouped_gemm_w4a16_swiglu(const uint16_t* x, const uint8_t* w_code
 int quads_moe_fp4_comp_amax(const float* g_a, int g_a_per_expert, const float* g_w,
                             const float* g_wc, int E, float* amax_r, quads_stream_t stream);
 
-/* a6 + a7 + the re-quantization of h in one pass: the SwiGLU GEMM above
- * whose epilogue also NVFP4-quantizes h for the down projection.  Each
+/* a6 + a7 + the re-quantization of h in one pass ([QUADS-fr §1]: the down
+ * GEMM's input is NVFP4 too): the SwiGLU GEMM above whose epilogue also
+ * NVFP4-quantizes h for the down projection.  Each
  * expert uses the decode scale g_e = fp32(amax_h_in[e] / 2688), computed from
  * an amax given in advance (calibrated, or the previous step's: delayed
  * scaling).  Written:
@@ -345,6 +347,7 @@ int quads_moe_grouped_gemm_nvfp4_swiglu_quant(const uint8_t* a_codes, const uint
                                               float* amax_h_out, uint16_t* h, quads_stream_t stream);
 
 /* --------------------------------------------------------- a7: SwiGLU
+ * (reading: the pages name no activation; SwiGLU is the plainest MoE FFN)
  * h[r][j] = bf16(silu(Y[r][j]) * Y[r][F + j]) for rows r < expert_off[E],
  * silu(v) = v / (1 + exp(-v)), computed in FP32 from the BF16 gate/up GEMM
  * output y [rows_cap][2F].  amax_out (device float[E], nullable, overwritten)
@@ -354,6 +357,8 @@ int quads_swiglu(const uint16_t* y, int64_t rows_cap, int64_t F,
                  quads_stream_t stream);
 
 /* --------------------------------------------------------- a8: combine
+ * ([TRACE] "Fonctionnement": the router's discrete choice of experts; the
+ * weighted sum of the k expert outputs is the plainest reading)
  * out[t] = bf16(sum over s = 0..k-1 of topk_w[t][s] * Y[row_of[t*k + s]]),
  * FP32 accumulation in slot order.  y [rows_cap][H], out [T][H], H % 8 == 0. */
 int quads_moe_unpermute_combine(const uint16_t* y, const int32_t* row_of, const float* topk_w,
@@ -396,7 +401,8 @@ int quads_fakequant_weight_ste_gate_up(const uint16_t* w, int64_t n_mat, int64_t
                                        uint8_t* codes, uint8_t* scales, float* g_out,
                                        const int32_t* chan, int n_chan, int chan_raw, uint16_t* w_chan,
                                        void* ws, size_t ws_bytes, quads_stream_t stream);
-/* Straight-through backward: grad_w = grad_wfq (accumulate = 0) or
+/* Straight-through backward ([QUADS-fr §2.2.A]: the QAT trainer's gradient
+ * passes through the weight fake-quant): grad_w = grad_wfq (accumulate = 0) or
  * grad_w = bf16(fp32(grad_w + grad_wfq)) (accumulate = 1); n BF16 elements. */
 int quads_fakequant_weight_ste_backward(const uint16_t* grad_wfq, uint16_t* grad_w, int64_t n,
                                         int accumulate, quads_stream_t stream);
@@ -464,7 +470,9 @@ size_t trace_qrecord_layout(int layer_id, int64_t T, int k,
 int trace_export_qrecord(int layer_id, int64_t T, int k, const int32_t* topk_idx,
                          const trace_qtensor_src* tensors, int n_tensors,
                          void* record, size_t record_bytes, quads_stream_t stream);
-/* Trainer replay of slot `which` of a record (device memory):
+/* Trainer replay of slot `which` of a record (device memory) ([TRACE]
+ * "Fonctionnement": the trainer reads the record during its forward pass and
+ * reproduces the rollout's rounding):
  *   x_hat [rows][K] BF16 = bf16(fp32(deq) + r) on the compensation channels,
  *         bf16(deq) elsewhere -- the operand the rollout's compensated GEMM
  *         effectively used;
