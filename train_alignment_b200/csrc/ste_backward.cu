@@ -13,13 +13,13 @@ constexpr int kThreads = 256;
 
 int ste_grid(int64_t work) {
   int64_t g = ceil_div(work, int64_t(kThreads));
-  const int64_t cap = static_cast<int64_t>(num_sms()) * 16;
+  const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
   return static_cast<int>(g > cap ? cap : (g < 1 ? 1 : g));
 }
 
 // Each thread keeps kSteUnroll 16-byte vectors of both inputs in flight per
 // iteration of a grid-stride loop.
-constexpr int kSteUnroll = 4;
+constexpr int kSteUnroll = 2;
 
 __device__ __forceinline__ uint4 ste_add(uint4 a, uint4 b) {
   uint32_t* pa = reinterpret_cast<uint32_t*>(&a);
