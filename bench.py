@@ -353,7 +353,7 @@ def _gemm_calls(layer, comp=True):
 def gemm_side_measurements(layer, dev, peaks):
     """(1) The compensation's cost: the step layer's two grouped GEMMs with
     and without the BF16 correction on the same operands.  (2) Decode
-    shapes (2048 hidden, 128 experts top-8, ffn 768, T = 64 and 512), judged
+    shapes (2048 hidden, 128 experts top-8, ffn 768, T = 64 and 512), measured
     as weight-stream bandwidth: the NVFP4 weight bytes (codes, scales and the
     BF16 Wc columns) of every expert that received rows, over the GEMM time.
     L2 flushed before each timed launch."""
