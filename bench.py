@@ -456,12 +456,17 @@ class ClockSampler:
 
 class OracleSample:
     """Bounded CPU sample of the workload for the oracle: a fraction `frac` of
-    every part of one step -- the weight sync and straight-through backward of
-    that fraction of the weight rows, the rollout forward and record replay of
-    that fraction of the tokens.  Inputs and every expert's NVFP4 weights
-    (which the forward needs) are prepared once, outside the timing."""
+    every part of one step.  The weight sync and straight-through backward
+    run on that fraction of the weight rows.  The rollout forward and record
+    replay run on a slice of the layer: T_s of the tokens and the first F_s
+    of the ffn columns (gate and up rows of W_gate/up, columns of W_down),
+    with T_s * F_s about frac * T * F.  Slicing the ffn width as well as the
+    tokens keeps small samples small: the forward dequantizes every expert's
+    weights once per call, whatever the number of tokens.  Inputs and the
+    slice's NVFP4 weights (which the forward needs) are prepared in
+    set_fraction, outside the timing."""
 
-    def __init__(self, cfg, seed=0):
+    def __init__(self, cfg, seed=0, frac=1.0):
         import numpy as np
         from oracle import layer as OL
         from oracle import nvfp4 as Q
@@ -472,36 +477,57 @@ class OracleSample:
         self.logits = inp["logits"].numpy().astype(np.float64)
         self.w_gu = inp["w_gu"].float().numpy().astype(np.float64)
         self.w_d = inp["w_d"].float().numpy().astype(np.float64)
+        self.seed = seed
         r = np.random.default_rng(seed)
         self.chan_x = Q.pad_channels(np.sort(r.choice(cfg.H, cfg.n_chan, replace=False)))
         self.chan_h = Q.pad_channels(np.sort(r.choice(cfg.F, cfg.n_chan_f, replace=False)))
-        self.wgu_all = OL.weight_sync(self.w_gu, self.chan_x)
-        self.wd_all = OL.weight_sync(self.w_d, self.chan_h)
-        self.set_fraction(1.0)
+        self.F_s = None
+        self.set_fraction(frac)
+
+    def _slice_weights(self, F_s):
+        """NVFP4 weights and ffn channel set of the first F_s ffn columns."""
+        np, cfg, Q, OL = self.np, self.cfg, self.Q, self.OL
+        if F_s == cfg.F:
+            chan_h = self.chan_h
+            w_gu, w_d = self.w_gu, self.w_d
+        else:
+            r = np.random.default_rng(self.seed + 1)
+            chan_h = Q.pad_channels(np.sort(r.choice(F_s, min(cfg.n_chan_f, F_s // 2), replace=False)))
+            w_gu = np.concatenate([self.w_gu[:, :F_s], self.w_gu[:, cfg.F:cfg.F + F_s]], axis=1)
+            w_d = np.ascontiguousarray(self.w_d[:, :, :F_s])
+        self.chan_h_s = chan_h
+        self.wgu_all = OL.weight_sync(w_gu, self.chan_x)
+        self.wd_all = OL.weight_sync(w_d, chan_h)
+        self.F_s = F_s
 
     def set_fraction(self, frac):
-        cfg = self.cfg
+        np, cfg = self.np, self.cfg
         self.frac = frac
-        self.T_s = max(1, int(round(cfg.T * frac)))
+        F_s = min(cfg.F, max(16, int(round(cfg.F * np.sqrt(frac) / 16)) * 16))
+        if F_s != self.F_s:
+            self._slice_weights(F_s)
+        self.T_s = max(1, min(cfg.T, int(round(cfg.T * frac * cfg.F / F_s))))
         self.rows_gu = max(16, int(round(cfg.E * 2 * cfg.F * frac)))
         self.rows_d = max(16, int(round(cfg.E * cfg.H * frac)))
         R = self.T_s * cfg.k
-        self.flops = 2 * R * 2 * cfg.F * cfg.H + 2 * R * cfg.H * cfg.F + 2 * R * 2 * cfg.F * cfg.n_chan + \
-            2 * R * cfg.H * cfg.n_chan_f
-        self.desc = (f"oracle (float64 numpy) on {self.T_s} of {cfg.T} tokens and the weight sync + STE "
+        n_cx = int((self.chan_x >= 0).sum())
+        n_ch = int((self.chan_h_s >= 0).sum())
+        self.flops = 2 * R * 2 * F_s * cfg.H + 2 * R * cfg.H * F_s + 2 * R * 2 * F_s * n_cx + 2 * R * cfg.H * n_ch
+        self.desc = (f"oracle (float64 numpy): forward and replay of {self.T_s} of {cfg.T} tokens over the first "
+                     f"{F_s} of {cfg.F} ffn columns ({n_cx} + {n_ch} compensation channels), weight sync + STE "
                      f"backward of {self.rows_gu} of {cfg.E * 2 * cfg.F} gate/up and {self.rows_d} of "
                      f"{cfg.E * cfg.H} down weight rows per step")
 
     def run(self):
-        OL, Q, np = self.OL, self.Q, self.np
+        OL, Q = self.OL, self.Q
         wgu = self.w_gu.reshape(-1, self.cfg.H)[:self.rows_gu][None]
         wd = self.w_d.reshape(-1, self.cfg.F)[:self.rows_d][None]
         t0 = time.perf_counter()
         OL.weight_sync(wgu, self.chan_x)
         OL.weight_sync(wd, self.chan_h)
         fwd = OL.rollout_forward(self.x[:self.T_s], self.logits[:self.T_s], self.wgu_all, self.wd_all,
-                                 self.chan_x, self.chan_h, self.cfg.k)
-        OL.trainer_replay(fwd, self.x[:self.T_s], self.chan_x, self.chan_h)
+                                 self.chan_x, self.chan_h_s, self.cfg.k)
+        OL.trainer_replay(fwd, self.x[:self.T_s], self.chan_x, self.chan_h_s)
         Q.ste_backward(wgu, wgu)
         Q.ste_backward(wd, wd)
         return time.perf_counter() - t0
@@ -522,12 +548,24 @@ def run_reference(args):
         return 0
     from train_alignment_b200 import workloads as W
     cfg = W.CONFIGS[args.workload]
-    sample = OracleSample(cfg, seed=0)
-    # size each step so that warm-up + timed steps take about two minutes
-    sample.set_fraction(1.0 / 64)
-    probe = sample.run()
-    budget = 120.0 / max(1, args.steps + args.warmup)
-    sample.set_fraction(min(1.0, max(1.0 / 4096, budget / max(probe * 64, 1e-6))))
+    # size each step so that warm-up + timed steps take about 100 s: a few
+    # probe runs, each rescaling the fraction by budget / time (the time is
+    # not proportional to the fraction, so one probe does not suffice)
+    budget = 100.0 / max(1, args.steps + args.warmup)
+    frac = 1.0 / 64
+    sample = OracleSample(cfg, seed=0, frac=frac)
+    tried = []
+    for _ in range(8):
+        sample.set_fraction(frac)
+        t = sample.run()
+        tried.append((frac, t))
+        nxt = min(1.0, max(1e-6, frac * budget / max(t, 1e-6)))
+        if 0.7 * budget <= t <= 1.3 * budget or nxt == frac:
+            break
+        frac = nxt
+    # the largest probed fraction within the budget, else the smallest probed
+    fit = [f for f, t in tried if t <= 1.3 * budget]
+    sample.set_fraction(max(fit) if fit else min(f for f, _ in tried))
     for _ in range(args.warmup):
         sample.run()
     times = [sample.run() for _ in range(args.steps)]

@@ -1,5 +1,5 @@
-"""Host-side accounting of bench.py: the recorded DRAM traffic table and the
-algorithmic work per kernel (no GPU)."""
+"""Host-side accounting of bench.py: the recorded DRAM traffic table, the
+algorithmic work per kernel and the reference arm's oracle sample (no GPU)."""
 import bench
 from train_alignment_b200 import workloads as W
 
@@ -35,3 +35,31 @@ def test_stale_hash_gives_null(tmp_path, monkeypatch):
 
 def test_whole_job_aggregate():
     assert bench.whole_job_tflops(2e12, 4, 1000.0) == 8.0
+
+
+def test_oracle_sample_slices_stay_small_and_consistent():
+    """The reference arm's sample: the ffn slice is a whole number of
+    16-column blocks, tokens times width track the fraction, and the
+    smallest sample runs in well under a second per step."""
+    import time
+    cfg = W.CONFIGS["moe_t2048_h1024_e8k2_f2048"]
+    s = bench.OracleSample(cfg, seed=0, frac=1e-6)
+    assert (s.F_s, s.T_s, s.rows_gu, s.rows_d) == (16, 1, 16, 16)
+    t0 = time.perf_counter()
+    s.run()
+    assert time.perf_counter() - t0 < 5.0
+    for f in (1.0 / 1024, 1.0 / 64):
+        s.set_fraction(f)
+        assert s.F_s % 16 == 0 and 16 <= s.F_s <= cfg.F
+        got = s.T_s * s.F_s / (cfg.T * cfg.F)
+        assert 0.5 * f <= got <= 2.0 * f, (f, got)
+        assert s.flops > 0 and int((s.chan_h_s >= 0).sum()) <= s.F_s // 2
+
+
+def test_reference_arm_other_ranks_do_no_work(monkeypatch):
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("LOCAL_RANK", "1")
+    import argparse
+    args = argparse.Namespace(impl="reference", gpus=2, steps=1, warmup=0, workload="moe_t2048_h1024_e8k2_f2048")
+    assert bench.run_reference(args) == 0
