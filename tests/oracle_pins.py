@@ -494,6 +494,13 @@ def pin_replay_counts_drift():
     assert cm >= 1
     c2, s2 = Q.quantize_with_scale(x2, g)
     assert cm == int(np.count_nonzero(c2 != c)) and sm == int(np.count_nonzero(s2 != s))
+    # halving one block of the trainer's input halves its block maximum: the
+    # block's E4M3 scale moves (its codes need not), so exactly one scale
+    # mismatch is counted when the halved scale stays a normal E4M3 value
+    x3 = x.copy()
+    x3[1, 16:32] = x3[1, 16:32] * 0.5
+    _, _, sm3 = TR.replay_tensor(rec, x3)
+    assert s[1, 1] >= 16 and sm3 == 1, (s[1, 1], sm3)
 
 
 def _unit_scale_block(vals):

@@ -145,6 +145,27 @@ def _router_logits_abs(x, w_r):
     return np.abs(x) @ np.abs(w), np.abs(x) @ np.abs(w)
 
 
+def _ste_overwrites(grad_wfq, grad_w=None):
+    # the existing gradient dropped instead of accumulated
+    return np.asarray(grad_wfq, dtype=np.float64).copy()
+
+
+def _replay_drops_residual(rec, x_train=None):
+    # the recorded residual channels not added back
+    return TR.__dict__["_orig_replay"](dict(rec, resid=None), x_train)
+
+
+def _replay_counts_codes_only(rec, x_train=None):
+    # scale mismatches never counted
+    x_hat, cm, sm = TR.__dict__["_orig_replay"](rec, x_train)
+    return x_hat, cm, (None if sm is None else 0)
+
+
+def _dequant_unit_drops_scale(codes, scales):
+    # the E4M3 block scale left out of the dequantized value
+    return F.e2m1_value(np.asarray(codes))
+
+
 MUTATIONS = {
     "e2m1_ties_away": [(F, "e2m1_rne_code", _e2m1_ties_up), (Q, "e2m1_rne_code", _e2m1_ties_up)],
     "e2m1_drops_sign": [(F, "e2m1_rne_code", _e2m1_no_sign), (Q, "e2m1_rne_code", _e2m1_no_sign)],
@@ -170,6 +191,12 @@ MUTATIONS = {
                               (TR, "replay_direction", _guided_ignores_bit)],
     "element_scale_dropped_factor": [(Q, "_orig_qws", Q.quantize_with_scale),
                                      (Q, "quantize_with_scale", _div_instead_of_recip)],
+    "ste_overwrites_gradient": [(Q, "ste_backward", _ste_overwrites)],
+    "replay_drops_residual": [(TR, "_orig_replay", TR.replay_tensor), (TR, "replay_tensor", _replay_drops_residual)],
+    "replay_skips_scale_count": [(TR, "_orig_replay", TR.replay_tensor),
+                                 (TR, "replay_tensor", _replay_counts_codes_only)],
+    "permute_pads_to_64": [(M, "PAD", 64)],
+    "dequant_drops_block_scale": [(Q, "dequant_unit", _dequant_unit_drops_scale)],
 }
 
 
