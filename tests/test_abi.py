@@ -87,6 +87,21 @@ def test_rows_capacity(lib):
     lambda l: l.quads_moe_unpermute_combine(None, None, None, 4, 2, 12, None, None),
     lambda l: l.quads_select_channels(None, 20000, 4, None, None),
     lambda l: l.trace_replay_qrecord(None, 0, 0, 0, 4, 16, None, None, None, None, None),
+    # N not a multiple of the weight tile
+    lambda l: l.quads_moe_grouped_gemm_w4a16(None, None, None, None, None, 8, 256, 100, 256, None, None),
+    # F not a multiple of 64
+    lambda l: l.quads_moe_grouped_gemm_w4a16_swiglu(None, None, None, None, None, 8, 256, 96, 256, None, None, None),
+    # no experts
+    lambda l: l.quads_moe_fp4_comp_amax(None, 0, None, None, 0, None, None),
+    # correction operands missing
+    lambda l: l.quads_moe_grouped_gemm_nvfp4_fp4comp(None, None, None, 0, None, None, None, None, 8, 256, 256, 128,
+                                                     None, None, None, None, 32, None, None),
+    # K not a multiple of 16
+    lambda l: l.trace_direction_bits(None, 4, 24, None, None, 0, None, None, 1, None, None),
+    # rows without scales
+    lambda l: l.trace_replay_direction(None, None, 0, None, None, 1, 4, 32, None, None, 0, None, None, None, None,
+                                       None),
+    lambda l: l.quads_copy_f32(None, None, -1, None),
 ])
 def test_invalid_arguments_are_rejected_on_the_host(lib, call):
     rc = call(lib)
