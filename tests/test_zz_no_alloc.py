@@ -13,7 +13,6 @@ the first so that scratch left over from the first call would show, and
 requests beyond the scratch's size are refused before any launch.  This file
 is collected last so that a failure here leaves every other test run.
 """
-import ctypes
 
 import numpy as np
 import pytest

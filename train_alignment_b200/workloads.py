@@ -16,7 +16,7 @@ available, so these synthetic tensors stand in for them:
 * expert weights: BF16 ~ N(0, 0.02), gate/up stored [E, 2F, H] (rows =
   output features, K = H contiguous), down stored [E, H, F].
 """
-from dataclasses import dataclass, field
+from dataclasses import dataclass
 import math
 
 import torch
