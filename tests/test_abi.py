@@ -133,3 +133,15 @@ def test_trace_record_layout(lib):
     # invalid description
     s0.K = 24
     assert lib.trace_qrecord_layout(7, 50, 2, ctypes.cast(src, ctypes.c_void_p), 2, ctypes.byref(hdr)) == 0
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """Without the built library every op raises: there is no CPU fallback."""
+    import torch
+    monkeypatch.setattr(B, "_lib", None)
+    monkeypatch.setattr(B, "_LIB_PATH", str(tmp_path / "libquads.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        B.load()
+    # a host tensor is refused too, rather than computed on the CPU
+    with pytest.raises(ValueError, match="CUDA"):
+        B.amax_bf16(torch.zeros((4, 16), dtype=torch.bfloat16))
