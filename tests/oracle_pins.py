@@ -675,4 +675,44 @@ def pin_residual_add_against_torch_rounding():
     assert np.array_equal(got, ref.to(torch.float64).numpy())
 
 
+def _golden_blocks(name):
+    """Parse a tests/golden fixture: a `levels` line and `block` sections."""
+    import os
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", name)
+    levels, blocks, cur = None, [], None
+    with open(path, encoding="utf-8") as f:
+        for line in f:
+            line = line.split("#", 1)[0].split()
+            if not line:
+                continue
+            key, vals = line[0], line[1:]
+            if key == "levels":
+                levels = [float(v) for v in vals]
+            elif key == "block":
+                cur = {"name": vals[0]}
+                blocks.append(cur)
+            else:
+                cur[key] = [float(v) for v in vals]
+    return levels, blocks
+
+
+def pin_golden_worked_blocks():
+    """Hand-worked NVFP4 blocks (tests/golden/nvfp4_worked_blocks.txt, from
+    the format's definition; [QUADS-fr §1] for the 8 levels per sign and
+    [TRACE] Fonctionnement for rounding to a neighbouring grid point): the
+    oracle's level set, block scale codes and element codes, signed zeros
+    included."""
+    levels, blocks = _golden_blocks("nvfp4_worked_blocks.txt")
+    assert len(levels) == 8 and np.array_equal(F.E2M1_LEVELS, np.array(levels))
+    assert len(blocks) == 4
+    for b in blocks:
+        x = np.array(b["x"], dtype=np.float64)[None]
+        assert np.array_equal(F.bf16_rne(x), x) and np.array_equal(np.signbit(F.bf16_rne(x)), np.signbit(x))
+        codes, scales = Q.quantize_with_scale(x, b["g"][0])
+        assert int(scales[0, 0]) == int(b["scale"][0]), (b["name"], scales)
+        assert codes[0].astype(int).tolist() == [int(c) for c in b["codes"]], (b["name"], codes)
+        if "tensor_amax" in b:
+            assert float(Q.tensor_scale(b["tensor_amax"][0])) == b["g"][0]
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -22,8 +22,14 @@ def _e2m1_ties_up(v):
     return ((np.signbit(v).astype(np.int64) << 3) | idx).astype(np.uint8)
 
 
+# the unmutated functions, taken before any test patches them (a mutation
+# that called the patched name would only recurse)
+_orig_e2m1_code = F.e2m1_rne_code
+_orig_e4m3_code = F.e4m3_rn_satfinite_code
+
+
 def _e2m1_no_sign(v):
-    return F.e2m1_rne_code(np.abs(np.asarray(v, dtype=np.float64)))
+    return _orig_e2m1_code(np.abs(np.asarray(v, dtype=np.float64)))
 
 
 def _e4m3_truncate(t):
@@ -31,7 +37,7 @@ def _e4m3_truncate(t):
     with np.errstate(divide="ignore"):
         e = np.maximum(np.floor(np.log2(np.where(t > 0, t, 1.0))), -6.0)
     q = np.exp2(e - 3.0)
-    return F.e4m3_rn_satfinite_code(np.floor(t / q) * q)
+    return _orig_e4m3_code(np.floor(t / q) * q)
 
 
 def _tensor_scale_wrong(amax):
@@ -208,6 +214,6 @@ def test_mutation_is_caught(name, monkeypatch):
     for pin in P.ALL_PINS:
         try:
             pin()
-        except Exception as exc:        # noqa: BLE001 -- any failure counts as caught
-            failures.append((pin.__name__, type(exc).__name__))
-    assert failures, f"mutation {name} passed every pin"
+        except AssertionError:
+            failures.append(pin.__name__)
+    assert failures, f"mutation {name} failed no pin's assertion"
