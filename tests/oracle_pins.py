@@ -715,4 +715,158 @@ def pin_golden_worked_blocks():
             assert float(Q.tensor_scale(b["tensor_amax"][0])) == b["g"][0]
 
 
+# ---------------------------------------------------------------- one layer
+
+
+def _unit_values(codes, scales):
+    """val(q) * val(s_b) element by element (the scale of element j is the
+    one of block j // 16)."""
+    rows, K = codes.shape
+    out = np.zeros((rows, K))
+    for i in range(rows):
+        for j in range(K):
+            out[i, j] = float(F.e2m1_value(codes[i, j])) * float(F.e4m3_value(scales[i, j // 16]))
+    return out
+
+
+def _layer_by_token(x, logits, x_train, w_gu, w_d, chan_x, chan_h, k):
+    """One MoE layer on both sides recomputed token by token from the
+    definitions, with none of the oracle's composition: quantize x with its
+    own tensor scale; for each token its top-k experts by (logit desc, index
+    asc) and the softmax over them; per selected expert the dequantized
+    product with that expert's fake-quantized gate/up weights (own tensor
+    scale) plus the BF16 residual of x on C times the BF16 W_fq columns of C;
+    BF16 storage of that output; SwiGLU in FP64 stored as BF16; h quantized
+    with the scale of its expert's rows (max over every row routed there);
+    the down product with the residual of h on C_F times the down W_fq
+    columns of C_F; BF16 storage; the weighted sum over the slots in order.
+    The trainer side: x_hat = bf16(deq) with bf16(fp32(deq + r)) on C, and
+    the counts of codes and scales that x_train's own rounding (same scale)
+    changes.  Returns a dict of float64 arrays."""
+    T, H = x.shape
+    E, F2 = w_gu.shape[0], w_gu.shape[1]
+    Fh = F2 // 2
+    bf = lambda v: float(F.bf16_rne(F.f32(np.array([v])))[0])
+
+    def fq(w):
+        g = float(Q.tensor_scale(np.max(np.abs(w))))
+        c, s = Q.quantize_with_scale(w, g)
+        unit = _unit_values(c, s)
+        return unit, g, F.bf16_rne(F.f32(unit * g))
+
+    wg = [fq(w_gu[e]) for e in range(E)]
+    wdn = [fq(w_d[e]) for e in range(E)]
+    gx = float(Q.tensor_scale(np.max(np.abs(x))))
+    cx, sx = Q.quantize_with_scale(x, gx)
+    ux = _unit_values(cx, sx)
+    r_x = {}
+    for t in range(T):
+        for c in chan_x:
+            if c >= 0:
+                r_x[t, c] = bf(x[t, c] - float(F.f32(ux[t, c] * gx)))
+    sel, wts, h_of = {}, {}, {}
+    for t in range(T):
+        order = sorted(range(E), key=lambda e: (-logits[t, e], e))[:k]
+        z = [np.exp(logits[t, e] - logits[t, order[0]]) for e in order]
+        sel[t], wts[t] = order, [v / sum(z) for v in z]
+        for s, e in enumerate(order):
+            unit_w, gw, wfq = wg[e]
+            y1 = np.zeros(F2)
+            for n in range(F2):
+                acc = gx * gw * float(np.dot(ux[t], unit_w[n]))
+                for c in chan_x:
+                    if c >= 0:
+                        acc += r_x[t, c] * wfq[n, c]
+                y1[n] = bf(acc)
+            h = np.array([bf(y1[j] / (1.0 + np.exp(-y1[j])) * y1[Fh + j]) for j in range(Fh)])
+            h_of[t, s] = h
+    g_h = np.zeros(E)
+    for e in range(E):
+        rows = [h_of[t, s] for t in range(T) for s in range(k) if sel[t][s] == e]
+        g_h[e] = float(Q.tensor_scale(max(np.max(np.abs(r)) for r in rows))) if rows else 0.0
+    out = np.zeros((T, H))
+    h_hat = {}
+    for t in range(T):
+        for s, e in enumerate(sel[t]):
+            h = h_of[t, s]
+            ch, sh = Q.quantize_with_scale(h[None], g_h[e])
+            uh = _unit_values(ch, sh)[0]
+            r_h = {c: bf(h[c] - float(F.f32(uh[c] * g_h[e]))) for c in chan_h if c >= 0}
+            unit_w, gw, wfq = wdn[e]
+            y2 = np.zeros(H)
+            for n in range(H):
+                acc = g_h[e] * gw * float(np.dot(uh, unit_w[n]))
+                for c, r in r_h.items():
+                    acc += r * wfq[n, c]
+                y2[n] = bf(acc)
+            out[t] += wts[t][s] * y2
+            hh = np.array([bf(uh[j] * g_h[e]) for j in range(Fh)])
+            for c, r in r_h.items():
+                hh[c] = bf(float(F.f32(uh[c] * g_h[e])) + r)
+            h_hat[t, s] = hh
+    x_hat = np.array([[bf(ux[t, j] * gx) for j in range(H)] for t in range(T)])
+    for (t, c), r in r_x.items():
+        x_hat[t, c] = bf(float(F.f32(ux[t, c] * gx)) + r)
+    ct, st = Q.quantize_with_scale(x_train, gx)
+    return dict(out=out, h=h_of, h_hat=h_hat, g_h=g_h, x_hat=x_hat, sel=sel,
+                code_mismatches=int(np.count_nonzero(ct != cx)), scale_mismatches=int(np.count_nonzero(st != sx)))
+
+
+def pin_layer_composition_per_token():
+    """The oracle's layer composition (weight sync, rollout forward, record,
+    replay) against a token-by-token recomputation from the definitions on a
+    tiny layer (T = 8, H = F = 32, E = 3, k = 2): routing, every stored h
+    row, the per-expert scale of h, the layer output, the replayed x and h
+    and the mismatch counts of a drifted trainer input.  [QUADS-fr §2.2.B]
+    (compensation on the high-residual channels of each GEMM input),
+    [QUADS-fr §2.2.A] (fake-quantized weights on the rollout's grid), [TRACE]
+    Fonctionnement (the recorded rounding replayed by the trainer)."""
+    from oracle import layer as OL
+    T, H, Fh, E, k = 8, 32, 32, 3, 2
+    r = np.random.default_rng(77)
+    x = F.bf16_rne(F.f32(r.standard_normal((T, H))))
+    x[:, 5] *= 16.0
+    logits = F.f32(r.standard_normal((T, E)))
+    logits[0, 1] = logits[0, 2]                                       # a tie: lower index first
+    w_gu = F.bf16_rne(F.f32(r.standard_normal((E, 2 * Fh, H)) * 0.5))
+    w_d = F.bf16_rne(F.f32(r.standard_normal((E, H, Fh)) * 0.5))
+    w_d[2] *= 8.0                                                     # experts' h scales differ
+    x_train = F.bf16_rne(F.f32(x + 0.05 * r.standard_normal((T, H))))
+    chan_x = Q.pad_channels(np.array([1, 5, 20]))
+    chan_h = Q.pad_channels(np.array([0, 7, 30]))
+    ref = _layer_by_token(x, logits, x_train, w_gu, w_d, chan_x, chan_h, k)
+    got = OL.step(x, logits, x_train, w_gu, w_d, chan_x, chan_h, k)
+    f = got["fwd"]
+    assert [list(map(int, f["idx"][t])) for t in range(T)] == [ref["sel"][t] for t in range(T)]
+    for t in range(T):
+        for s in range(k):
+            row = int(f["row_of"][t * k + s])
+            assert np.array_equal(f["h"][row], ref["h"][t, s]), ("h", t, s)
+            assert np.array_equal(got["h_hat"][row], ref["h_hat"][t, s]), ("h_hat", t, s)
+    assert np.array_equal(f["gh"], ref["g_h"]), (f["gh"], ref["g_h"])
+    assert len(set(ref["g_h"].tolist())) == E
+    assert np.allclose(f["out"], ref["out"], rtol=1e-12, atol=1e-12), np.max(np.abs(f["out"] - ref["out"]))
+    assert np.array_equal(got["x_hat"], ref["x_hat"])
+    assert (got["code_mismatches"], got["scale_mismatches"]) == (ref["code_mismatches"], ref["scale_mismatches"])
+    assert ref["code_mismatches"] > 0
+
+
+def pin_gather_rows_loop():
+    r = np.random.default_rng(78)
+    a = r.integers(0, 255, (9, 6)).astype(np.uint8)
+    src = np.array([3, -1, 0, 8, -1, 3, 5])
+    g = M.gather_rows(a, src)
+    for i, s in enumerate(src):
+        assert np.array_equal(g[i], a[s] if s >= 0 else np.zeros(6, np.uint8))
+
+
+def pin_pack_bits_loop():
+    r = np.random.default_rng(79)
+    b = r.integers(0, 2, (3, 64)).astype(np.uint8)
+    p = TR.pack_bits(b)
+    for i in range(3):
+        for j in range(8):
+            assert int(p[i, j]) == sum(int(b[i, 8 * j + q]) << q for q in range(8))
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -3,7 +3,11 @@ check that at least one pin catches each of them."""
 import numpy as np
 import pytest
 
+import inspect
+import textwrap
+
 from oracle import formats as F
+from oracle import layer as OL
 from oracle import moe as M
 from oracle import nvfp4 as Q
 from oracle import stack as ST
@@ -172,6 +176,27 @@ def _dequant_unit_drops_scale(codes, scales):
     return F.e2m1_value(np.asarray(codes))
 
 
+def _source_mutation(func, old, new):
+    """A copy of `func` with one source fragment replaced, compiled in the
+    function's own module namespace (so the planted slip sits exactly where
+    it would in the oracle's code)."""
+    src = textwrap.dedent(inspect.getsource(func))
+    assert src.count(old) == 1, (func.__name__, old)
+    ns = {}
+    exec(compile(src.replace(old, new), f"<mutated {func.__name__}>", "exec"), func.__globals__, ns)
+    return ns[func.__name__]
+
+
+# slips in the layer composition: h's residuals taken with one scale for all
+# experts instead of the expert's own; the gate/up channel set used for the
+# down weights' compensation columns; the gate/up output fed to SwiGLU before
+# its BF16 storage rounding
+_layer_h_resid_one_scale = _source_mutation(OL.rollout_forward, "sh[lo:hi], gh[e], chan_h)",
+                                            "sh[lo:hi], gh.max(), chan_h)")
+_layer_down_wc_chan_x = _source_mutation(OL.step, "wd = weight_sync(w_d, chan_h)", "wd = weight_sync(w_d, chan_x)")
+_layer_no_bf16_before_swiglu = _source_mutation(OL.rollout_forward, "M.swiglu(y1b)", "M.swiglu(y1)")
+
+
 MUTATIONS = {
     "e2m1_ties_away": [(F, "e2m1_rne_code", _e2m1_ties_up), (Q, "e2m1_rne_code", _e2m1_ties_up)],
     "e2m1_drops_sign": [(F, "e2m1_rne_code", _e2m1_no_sign), (Q, "e2m1_rne_code", _e2m1_no_sign)],
@@ -203,6 +228,9 @@ MUTATIONS = {
                                  (TR, "replay_tensor", _replay_counts_codes_only)],
     "permute_pads_to_64": [(M, "PAD", 64)],
     "dequant_drops_block_scale": [(Q, "dequant_unit", _dequant_unit_drops_scale)],
+    "layer_h_residual_one_scale": [(OL, "rollout_forward", _layer_h_resid_one_scale)],
+    "layer_down_wc_from_gate_up_channels": [(OL, "step", _layer_down_wc_chan_x)],
+    "layer_swiglu_before_bf16_storage": [(OL, "rollout_forward", _layer_no_bf16_before_swiglu)],
 }
 
 
