@@ -1,6 +1,6 @@
 """Test-side conversions between torch tensors and the oracle's numpy arrays,
 and the float tolerance.  Shared by the GPU parity tests; holds none of the
-method's arithmetic."""
+method's arithmetic (the SwiGLU bound calls the oracle's SwiGLU)."""
 import numpy as np
 import torch
 
@@ -59,3 +59,19 @@ def gate_up_interleave_index(F):
     dst = np.arange(2 * F)
     b, j = dst // 128, dst % 128
     return np.where(j < 64, 64 * b + j, F + 64 * b + (j - 64))
+
+
+def swiglu_carried(y_ref, absdot, F_):
+    """The oracle's h = SwiGLU(bf16(y)) from its gate/up output y_ref [rows,
+    2F] and a per-element bound on |h_gpu - h|: the GEMM tolerance of y
+    (1e-2 |y| + 1e-3 sum|a b|) carried through SwiGLU to first order, plus
+    one BF16 rounding of h."""
+    from oracle import moe as M
+    tol_y = 1e-2 * np.abs(y_ref) + 1e-3 * absdot
+    g, u = y_ref[:, :F_], y_ref[:, F_:]
+    sig = 1.0 / (1.0 + np.exp(-g))
+    h_ref = M.swiglu(F.bf16_rne(y_ref.astype(np.float32)))
+    dsilu = np.abs(sig * (1.0 + g * (1.0 - sig)))
+    tol_h = dsilu * (np.abs(u) + tol_y[:, F_:]) * tol_y[:, :F_] + np.abs(g * sig) * tol_y[:, F_:] + \
+        2.0 ** -7 * np.abs(h_ref) + 1e-30
+    return h_ref, tol_h

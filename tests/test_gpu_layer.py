@@ -1,23 +1,26 @@
 """One full step of the 2048-token, 8-expert layer (hidden 1024, ffn 2048,
-32 + 32 compensation channels) on the GPU against the oracle's composition of
-the same steps on the same seeded inputs.
+32 + 32 compensation channels) on the GPU against the oracle on the same
+seeded inputs, stage by stage.
 
 Bit-exact: input quantization, residuals, routing, permutation, weight
 fake-quant / rollout weights / compensation columns, replayed operand and
-mismatch counts.  Float: the gate/up GEMM within the tolerance.  Past the
-first BF16 GEMM output the two paths can round an intermediate differently
-(FP32 vs FP64 accumulation order before the BF16 store), which can flip an
-NVFP4 code of h; those flips are counted and bounded, and the layer output is
-checked per element with the tolerance on all but a bounded fraction."""
+mismatch counts.  Float, on every element: the gate/up GEMM within the
+tolerance, and each later stage against the oracle fed the GPU's output of
+the stage before it: SwiGLU of the GPU's gate/up output, the NVFP4
+quantization of the GPU's h (bit-exact), the down GEMM on the GPU's
+quantized h, the combine of the GPU's down output.  Where h comes out of the
+gate/up GEMM's epilogue (y is never stored) h is checked against the
+oracle's own GEMM with the tolerance carried through SwiGLU."""
 import numpy as np
 import pytest
 import torch
 
 from oracle import formats as F
 from oracle import layer as OL
+from oracle import moe as M
 from oracle import nvfp4 as Q
-from tests.helpers import (assert_bits_equal, assert_close_tol, bf16_np, f32_of, gate_up_interleave_index, u8_np,
-                           unpack_codes)
+from tests.helpers import (assert_bits_equal, assert_close_tol, bf16_np, f32_of, gate_up_interleave_index,
+                           swiglu_carried, u8_np, unpack_codes)
 from train_alignment_b200 import layer as L
 from train_alignment_b200 import workloads as W
 
@@ -86,21 +89,92 @@ def test_gate_up_gemm(run):
     assert_close_tol(bf16_np(layer.y_gu)[:n], f["y1"], f["absdot1"], what="gate/up GEMM")
 
 
-def test_h_and_output(run):
+def test_h(run):
+    """SwiGLU: against the oracle's SwiGLU of the GPU's stored gate/up output
+    (separate pass), or of the oracle's own gate/up output with the GEMM
+    tolerance carried through (fused epilogue); every element."""
     cfg, layer, ref = run
     f = ref["fwd"]
     n = int(f["off"][-1])
     h = bf16_np(layer.h)[:n]
-    frac_h = np.mean(h != f["h"])
-    assert frac_h < 5e-3, f"h differs in {frac_h:.2e} of elements"
-    code_flip = np.mean(unpack_codes(layer.h_codes)[:n] != f["ch"])
-    assert code_flip < 5e-3, f"h codes differ in {code_flip:.2e} of elements"
+    if layer.fuse_swiglu:
+        h_ref, tol = swiglu_carried(f["y1"], f["absdot1"], cfg.F)
+    else:
+        y = bf16_np(layer.y_gu)[:n]
+        h_ref = M.swiglu(y)
+        tol = 1e-2 * np.abs(h_ref) + 1e-3 * np.abs(y[:, :cfg.F] / (1.0 + np.exp(-y[:, :cfg.F])) * y[:, cfg.F:])
+    err = np.abs(h - h_ref)
+    assert np.all(err <= tol), f"{np.sum(err > tol)} of {err.size} h values outside the tolerance"
+
+
+def _gpu_quantized_h(layer, cfg, n):
+    """The GPU's NVFP4 h of rows [0, n): codes, linear scales, per-expert
+    scale, channel residuals."""
+    codes = unpack_codes(layer.h_codes)[:n]
+    scales = F.scales_from_tiled(u8_np(layer.h_scales), n, cfg.F // 16)
+    resid = bf16_np(layer.h_resid)[:n]
+    return codes, scales, f32_of(layer.g_h).astype(np.float32).astype(np.float64), resid
+
+
+def test_h_quantization(run):
+    """The oracle's per-expert NVFP4 quantization of the GPU's h (amax of each
+    expert's rows, codes, scales, residuals on the ffn channel set): bit for
+    bit."""
+    cfg, layer, ref = run
+    f = ref["fwd"]
+    n = int(f["off"][-1])
+    h = bf16_np(layer.h)[:n]
+    codes, scales, g_h, resid = _gpu_quantized_h(layer, cfg, n)
+    c_ref, s_ref, g_ref = Q.quantize_grouped(h, f["off"])
+    assert_bits_equal(g_h.astype(np.float32), g_ref.astype(np.float32), "g_h")
+    assert_bits_equal(codes, c_ref, "h codes")
+    assert_bits_equal(scales, s_ref, "h scales")
+    chan_h = f32_of(layer.chan_h).astype(np.int64)
+    r_ref = np.zeros_like(resid)
+    for e in range(cfg.E):
+        lo, hi = int(f["off"][e]), int(f["off"][e + 1])
+        if hi > lo:
+            r_ref[lo:hi] = Q.residual_channels(h[lo:hi], c_ref[lo:hi], s_ref[lo:hi], g_ref[e], chan_h)
+    assert_bits_equal(F.bf16_bits(resid), F.bf16_bits(r_ref), "h residuals")
+
+
+def test_down_gemm(run):
+    """The oracle's down GEMM fed the GPU's quantized h: every element within
+    the tolerance."""
+    cfg, layer, ref = run
+    f = ref["fwd"]
+    n = int(f["off"][-1])
+    codes, scales, g_h, resid = _gpu_quantized_h(layer, cfg, n)
+    wd = ref["wd"]
+    y2, absdot2 = M.grouped_gemm(codes, scales, g_h, wd["codes"], wd["scales"], wd["g"], f["off"], resid, wd["wc"])
+    assert_close_tol(bf16_np(layer.y_d)[:n], y2, absdot2, what="down GEMM")
+
+
+def test_combine(run):
+    """The oracle's combine of the GPU's down output with the GPU's routing
+    weights: every element within the tolerance (sum |w y| as the scale)."""
+    cfg, layer, ref = run
+    y = bf16_np(layer.y_d)
+    w = f32_of(layer.topk_w)
+    row_of = f32_of(layer.row_of).astype(np.int64)
+    out_ref = M.combine(y, row_of, w, cfg.k)
+    rows = row_of.reshape(cfg.T, cfg.k)
+    absdot = sum(np.abs(w[:, s:s + 1] * y[rows[:, s]]) for s in range(cfg.k))
+    assert_close_tol(bf16_np(layer.out), out_ref, absdot, what="combine")
+
+
+def test_output_against_oracle_end_to_end(run):
+    """Report: the layer output against the oracle's own end-to-end result.
+    Past the first BF16 GEMM output the two can round an intermediate to
+    neighbouring values, which can flip an NVFP4 code of h; the flip rate is
+    printed, and the outputs must agree in norm."""
+    cfg, layer, ref = run
+    f = ref["fwd"]
+    n = int(f["off"][-1])
+    flips = np.mean(unpack_codes(layer.h_codes)[:n] != f["ch"])
     out = bf16_np(layer.out)
-    err = np.abs(out - f["out"])
-    scale = np.abs(f["out"]) * 1e-2 + 1e-3 * np.sqrt(np.mean(f["out"] ** 2))
-    frac_bad = np.mean(err > scale)
-    assert frac_bad < 1e-2, f"{frac_bad:.2e} of outputs outside the tolerance"
     rel = np.linalg.norm(out - f["out"]) / np.linalg.norm(f["out"])
+    print(f"h code flips against the oracle's own h: {flips:.2e}; output relative distance {rel:.2e}")
     assert rel < 1e-2, rel
 
 

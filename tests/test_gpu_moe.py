@@ -71,6 +71,38 @@ def test_gather_parity(cuda_lib):
     assert_bits_equal(F.bf16_bits(bf16_np(pr)[:n]), F.bf16_bits(M.gather_rows(resid, src_ref)), "resid")
 
 
+@pytest.mark.parametrize("T,E,k,K,nc", [(1, 4, 1, 64, 0), (300, 8, 2, 256, 16), (4096, 128, 8, 512, 32)])
+def test_route_permute_composite(cuda_lib, T, E, k, K, nc):
+    """quads_moe_route_permute (router + permutation + gather in one call)
+    against the oracle's router_topk, permute and gather_rows: indices,
+    offsets, rows, gathered codes, scales and residuals bit for bit, weights
+    within float rounding."""
+    r = np.random.default_rng(T + E + K)
+    x = F.bf16_rne(r.standard_normal((T, K)).astype(np.float32))
+    c, s, g = Q.quantize(x)
+    chan = Q.pad_channels(np.sort(r.choice(K, max(nc - 5, 1), replace=False))) if nc else np.zeros(0, np.int32)
+    resid = Q.residual_channels(x, c, s, g, chan) if nc else None
+    l = _logits(T, E, 3 * T + E, "zipf" if E >= 64 else "normal")
+    idx, w, off, row_of, src_of, pc, ps, pr = cuda_lib.moe_route_permute(
+        l.cuda(), k, torch.from_numpy(F.pack_nibbles(c)).cuda(), torch.from_numpy(s).cuda(), K,
+        bf16_torch(resid) if nc else None)
+    torch.cuda.synchronize()
+    assert cuda_lib.device_status() == cuda_lib.OK
+    idx_ref, w_ref = M.router_topk(l.numpy().astype(np.float64), k)
+    assert_bits_equal(f32_of(idx).astype(np.int64), idx_ref.astype(np.int64), "topk idx")
+    assert np.allclose(f32_of(w), w_ref, rtol=2e-6, atol=1e-7)
+    off_ref, row_ref, src_ref = M.permute(idx_ref, E)
+    assert_bits_equal(f32_of(off).astype(np.int64), off_ref.astype(np.int64), "expert_off")
+    assert_bits_equal(f32_of(row_of).astype(np.int64), row_ref.astype(np.int64), "row_of")
+    n = int(off_ref[-1])
+    assert_bits_equal(f32_of(src_of)[:n].astype(np.int64), src_ref.astype(np.int64), "src_of")
+    assert_bits_equal(u8_np(pc)[:n], F.pack_nibbles(M.gather_rows(c, src_ref)), "gathered codes")
+    cap = cuda_lib.moe_rows_capacity(T, k, E)
+    assert_bits_equal(F.scales_from_tiled(u8_np(ps), cap, K // 16)[:n], M.gather_rows(s, src_ref), "gathered scales")
+    if nc:
+        assert_bits_equal(F.bf16_bits(bf16_np(pr)[:n]), F.bf16_bits(M.gather_rows(resid, src_ref)), "gathered resid")
+
+
 def test_swiglu_parity(cuda_lib):
     E, F_ = 3, 256
     off = np.array([0, 128, 128, 384], dtype=np.int32)

@@ -308,6 +308,30 @@ def moe_gather(src_of, expert_off, E, rows_cap, a_codes, a_scales, K, a_resid=No
     return pa_codes, pa_scales, (pa_resid if n_chan else None)
 
 
+def moe_route_permute(logits, k, a_codes, a_scales, K, a_resid=None, renorm=True):
+    """Router top-k, permutation and gather in one call (quads_moe_route_permute).
+    Returns (topk_idx, topk_w, expert_off, row_of, src_of, pa_codes, pa_scales,
+    pa_resid)."""
+    _dev(logits, torch.float32, "logits")
+    T, E = logits.shape
+    dev = logits.device
+    cap = moe_rows_capacity(T, k, E)
+    n_chan = 0 if a_resid is None else a_resid.shape[1]
+    idx, w = _empty((T, k), torch.int32, dev), _empty((T, k), torch.float32, dev)
+    off, row_of, src_of = _empty((E + 1,), torch.int32, dev), _empty((T * k,), torch.int32, dev), \
+        _empty((cap,), torch.int32, dev)
+    pa_codes = _empty((cap, K // 2), torch.uint8, dev)
+    pa_scales = _empty((scales_bytes(cap, K, SCALES_TILED),), torch.uint8, dev)
+    pa_resid = _empty((cap, n_chan), torch.bfloat16, dev) if n_chan else None
+    ws = _empty((moe_permute_workspace_bytes(T, k, E),), torch.uint8, dev)
+    _check(load().quads_moe_route_permute(_p(logits), T, E, k, 1 if renorm else 0, _p(idx), _p(w), _p(off),
+                                          _p(row_of), _p(src_of), cap, _p(a_codes), _p(a_scales), K,
+                                          _p(a_resid) if n_chan else None, n_chan, _p(pa_codes), _p(pa_scales),
+                                          _p(pa_resid) if n_chan else None, _p(ws), ws.numel(), _s()),
+           "quads_moe_route_permute")
+    return idx, w, off, row_of, src_of, pa_codes, pa_scales, pa_resid
+
+
 def moe_grouped_gemm_nvfp4(a_codes, a_scales, g_a, w_codes, w_scales, g_w, expert_off, E, rows_cap, N, K,
                            a_resid=None, w_resid=None, y=None):
     n_chan = 0 if a_resid is None else a_resid.shape[1]
