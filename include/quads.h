@@ -135,9 +135,13 @@ int quads_quantize_nvfp4(const uint16_t* x, int64_t rows, int64_t K, int64_t ld_
  *   - n_groups <= 1024; larger requests return QUADS_ERR_UNSUPPORTED_SHAPE
  *     before anything is launched.  All other arguments and limits are those
  *     of quads_quantize_nvfp4.
- *   - The first call with a given device current looks up the array's device
- *     address on that device (cudaGetSymbolAddress); make that first call
- *     before any stream capture.
+ *   - The first call with a given device and CUDA context current looks up
+ *     the array's device address there (cudaGetSymbolAddress) and caches it
+ *     for that device and context; make that first call before any stream
+ *     capture.  A device reset (cudaDeviceReset) unloads the array and the
+ *     context it comes back with can carry the same handle, so the cached
+ *     address is not valid after a reset: a process that resets a device
+ *     must not call this entry point on it again.
  *   - Every call reuses the same array and clears it before use.  Calls that
  *     can run at the same time on one GPU (other streams, other host threads)
  *     race on it: serialize them. */

@@ -815,9 +815,13 @@ int quads_fakequant_weight_ste_gate_up(const uint16_t* w, int64_t n_mat, int64_t
 // is loaded and that stays there until the process exits.
 //
 // The array's name is only a host-side stand-in for the device variable, so
-// host code never passes it to a kernel: the device address is obtained once
-// per device with cudaGetSymbolAddress (on the first call made with that
-// device current) and cached.  All calls share the array and it keeps the
+// host code never passes it to a kernel: the device address is obtained with
+// cudaGetSymbolAddress on the first call made with a given device and CUDA
+// context current, and cached for that device and context.  A call under a
+// different context (a non-primary context the caller made current) looks
+// the address up again.  cudaDeviceReset destroys the module, and the
+// recreated primary context may come back with the same handle, so the
+// cached address is not valid across a device reset.  All calls share the array and it keeps the
 // last call's contents, so each call clears the part it uses before the amax
 // pass; calls that can overlap on the GPU (different streams, or different
 // host threads on one device) race on it and must be serialized by the caller.
@@ -827,23 +831,51 @@ namespace {
 constexpr int kNoAllocMaxGroups = 1024;                     // 4 KiB of scratch per GPU
 static __device__ __align__(256) float g_noalloc_amax[kNoAllocMaxGroups];
 
+struct NoAllocSlot {
+  void* ctx;          // CUcontext the address was looked up under
+  float* ptr;
+};
 std::mutex g_noalloc_mutex;
-float* g_noalloc_scratch[64] = {nullptr};
+NoAllocSlot g_noalloc_scratch[64] = {};
+
+// The calling thread's current CUDA context, through the driver entry point
+// the runtime hands out (no link against the driver library).
+int current_context(void** ctx) {
+  using GetCtx = int (*)(void**);
+  static GetCtx get = nullptr;
+  if (get == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+      return set_error(QUADS_ERR_CUDA, "cuCtxGetCurrent is not available from the CUDA runtime");
+    get = reinterpret_cast<GetCtx>(fn);
+  }
+  *ctx = nullptr;
+  if (get(ctx) != 0 || *ctx == nullptr) return set_error(QUADS_ERR_CUDA, "no current CUDA context");
+  return QUADS_OK;
+}
 
 int noalloc_scratch(float** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
     return set_error(QUADS_ERR_CUDA, "no usable current CUDA device");
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (g_noalloc_scratch[dev] == nullptr) {
+  NoAllocSlot& slot = g_noalloc_scratch[dev];
+  void* ctx = nullptr;
+  if (slot.ptr != nullptr) QUADS_TRY(current_context(&ctx));
+  if (slot.ptr == nullptr || slot.ctx != ctx) {
+    // on a device's first call this also sets up its context, so the handle
+    // is read after it
     void* p = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_amax);
     if (e != cudaSuccess || p == nullptr)
       return set_error(QUADS_ERR_CUDA, "cudaGetSymbolAddress of the quantizer scratch failed: %s",
                        cudaGetErrorString(e));
-    g_noalloc_scratch[dev] = static_cast<float*>(p);
+    QUADS_TRY(current_context(&ctx));
+    slot = NoAllocSlot{ctx, static_cast<float*>(p)};
   }
-  *out = g_noalloc_scratch[dev];
+  *out = slot.ptr;
   return QUADS_OK;
 }
 
@@ -856,11 +888,13 @@ extern "C" int quads_quantize_nvfp4_noalloc(const uint16_t* x, int64_t rows, int
                                             const int32_t* chan, int n_chan, uint16_t* resid_out,
                                             quads_stream_t stream) {
   clear_error();
-  QUADS_TRY(validate_matrix(x, rows, K, ld_x));
-  QUADS_TRY(validate_groups(group_off, n_groups, rows));
+  // the scratch's size is this entry point's own limit: checked first, so it
+  // holds whatever the general group limit below is
   QUADS_REQUIRE(n_groups <= kNoAllocMaxGroups, QUADS_ERR_UNSUPPORTED_SHAPE,
                 "the allocation-free quantizer supports at most %d row groups (got %d)", kNoAllocMaxGroups,
                 n_groups);
+  QUADS_TRY(validate_matrix(x, rows, K, ld_x));
+  QUADS_TRY(validate_groups(group_off, n_groups, rows));
   QUADS_REQUIRE(scale_layout == QUADS_SCALES_LINEAR || scale_layout == QUADS_SCALES_TILED,
                 QUADS_ERR_INVALID_ARG, "unknown scale layout %d", scale_layout);
   QUADS_REQUIRE(g_out && (rows == 0 || (codes && scales)), QUADS_ERR_INVALID_ARG,

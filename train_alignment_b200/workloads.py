@@ -141,18 +141,32 @@ def router_logits(T, E, kind, gen, device):
     return l.contiguous()
 
 
-def moe_layer_inputs(cfg: MoEConfig, seed=0, device="cpu", layer=0, with_logits=True):
+def moe_layer_inputs(cfg: MoEConfig, seed=0, device="cpu", layer=0, with_logits=True, with_weights=True):
     """Inputs of one MoE layer: x [T,H] bf16, logits [T,E] f32, w_gu [E,2F,H]
     bf16, w_d [E,H,F] bf16.  Layer l of a stack uses seed + 1000 * l for its
-    weights (the stack's activations flow from layer to layer)."""
+    weights (the stack's activations flow from layer to layer).  x and the
+    logits are drawn first, so with_weights=False gives the same x and logits
+    without the weights."""
     gen = _gen(device, seed * 7919 + layer * 1000 + 1)
     out = {}
     out["x"] = activations(cfg.T, cfg.H, cfg.x_kind, cfg.n_outlier, cfg.outlier_scale, gen, device)
     if with_logits:
         out["logits"] = router_logits(cfg.T, cfg.E, cfg.logit_kind, gen, device)
-    out["w_gu"] = _randn_bf16((cfg.E, 2 * cfg.F, cfg.H), 0.02, gen, device)
-    out["w_d"] = _randn_bf16((cfg.E, cfg.H, cfg.F), 0.02, gen, device)
+    if with_weights:
+        out["w_gu"] = _randn_bf16((cfg.E, 2 * cfg.F, cfg.H), 0.02, gen, device)
+        out["w_d"] = _randn_bf16((cfg.E, cfg.H, cfg.F), 0.02, gen, device)
     return out
+
+
+def expert_weight_slice(cfg: MoEConfig, F_s, seed=0, device="cpu"):
+    """Expert weights of the first F_s ffn columns only, with the layer's
+    distribution (BF16 ~ N(0, 0.02)) from their own seeded generator (not the
+    values moe_layer_inputs draws): w_gu [E, 2 F_s, H] (gate rows, then up
+    rows), w_d [E, H, F_s].  Used where the whole layer's weights are too
+    large to draw on the host."""
+    gen = _gen(device, seed * 7919 + 271828)
+    return {"w_gu": _randn_bf16((cfg.E, 2 * F_s, cfg.H), 0.02, gen, device),
+            "w_d": _randn_bf16((cfg.E, cfg.H, F_s), 0.02, gen, device)}
 
 
 def stack_router_weights(cfg: MoEConfig, seed=0, device="cpu"):
