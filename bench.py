@@ -767,10 +767,10 @@ def run_ours(args):
 
     # the dense FP4 peak of this GPU, measured with the library's NVFP4 GEMM
     try:
-        fp4 = fp4_library_peak(dev)
-        fp4_peak, fp4_src = fp4["burst_tflops"], "measured on this GPU: library NVFP4 GEMM, burst"
+        fp4_meas = fp4_library_peak(dev)
+        fp4_peak, fp4_src = fp4_meas["burst_tflops"], "measured on this GPU: library NVFP4 GEMM, burst"
     except Exception as exc:  # noqa: BLE001 -- the nominal ratio, said so in the line
-        fp4 = {"error": f"{type(exc).__name__}: {str(exc)[:160]}"}
+        fp4_meas = {"error": f"{type(exc).__name__}: {str(exc)[:160]}"}
         fp4_peak, fp4_src = None, None
 
     # roofline of the dominant kernel: its own launches timed by two events
@@ -825,7 +825,7 @@ def run_ours(args):
     g_flop = sum(work[n][1] for n in gemm_names)
     gemm = {"kernels": {n: kernels[n] for n in gemm_names}, "ms": g_ms, "TFLOP/s": g_flop / (g_ms * 1e-3) / 1e12,
             "frac_fp4": g_flop / (g_ms * 1e-3) / 1e12 / fp4_peak, "fp4_peak_tflops": fp4_peak,
-            "fp4_peak_source": fp4_src, "fp4_peak_measurement": fp4,
+            "fp4_peak_source": fp4_src, "fp4_peak_measurement": fp4_meas,
             "flops": "2 x routed rows x N x K per GEMM (FP4) + 2 x routed rows x N x channels (BF16 correction); "
                      "padding rows excluded",
             "timed_by": "events around each GEMM launch alone, one-stream step graph, L2 flushed before each step"}
