@@ -77,6 +77,18 @@ int quads_device_status(quads_stream_t stream);
  * wait gives up, records a timeout and the kernel returns.  A following
  * quads_device_status() returns QUADS_ERR_TIMEOUT. */
 int quads_selftest_bounded_wait(uint64_t timeout_ns, quads_stream_t stream);
+/* Output tile of the grouped FP4 GEMMs with the BF16 correction (or none)
+ * and N % 256 == 0 (a tuning and testing switch, not a reading of the pages):
+ *   0  128 x 128 on one CTA, the correction in its own FP32 accumulator;
+ *   1  128 x 256 on one CTA (the default);
+ *   2  256 x 256 on a pair of CTAs (tcgen05 cta_group::2, each CTA loads
+ *      its own half of the rows and of the weight rows).
+ * Shapes 1 and 2 accumulate the correction into the FP4 accumulator as
+ * (R / G) . Wc, with R / G = bf16(fp32(R * fp32(1 / G))) and G = g_a g_w[e].
+ * Other GEMMs (W4A16, the FP4 correction, N % 256 != 0) always take shape 0.
+ * Returns the previous shape, or QUADS_ERR_INVALID_ARG for another value.
+ * Process-wide; not synchronized with launches in flight. */
+int quads_gemm_set_tile_shape(int shape);
 
 /* Bytes of a scale array of `rows` x K/16 scales in the given layout. */
 size_t quads_scales_bytes(int64_t rows, int64_t K, int scale_layout);

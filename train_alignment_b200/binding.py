@@ -61,6 +61,7 @@ _SIGS = {
     "quads_launch_count": (c_u64, []),
     "quads_device_status": (c_i32, [c_vp]),
     "quads_selftest_bounded_wait": (c_i32, [c_u64, c_vp]),
+    "quads_gemm_set_tile_shape": (c_i32, [c_i32]),
     "quads_scales_bytes": (c_sz, [c_i64, c_i64, c_i32]),
     "quads_amax_bf16": (c_i32, [c_vp, c_i64, c_i64, c_i64, c_vp, c_i32, c_vp, c_vp]),
     "quads_quantize_workspace_bytes": (c_sz, [c_i32]),
@@ -186,6 +187,18 @@ def device_status():
 
 def selftest_bounded_wait(timeout_ns):
     _check(load().quads_selftest_bounded_wait(int(timeout_ns), _s()), "quads_selftest_bounded_wait")
+
+
+TILE_128x128, TILE_128x256, TILE_PAIR_256x256 = 0, 1, 2
+
+
+def gemm_set_tile_shape(shape):
+    """Output tile of the FP4 grouped GEMMs (0: 128 x 128, 1: 128 x 256,
+    2: 256 x 256 on a CTA pair); returns the previous shape."""
+    prev = int(load().quads_gemm_set_tile_shape(int(shape)))
+    if prev < 0:
+        _check(prev, "quads_gemm_set_tile_shape")
+    return prev
 
 
 def scales_bytes(rows, K, layout):

@@ -203,6 +203,7 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t sr
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -794,6 +795,587 @@ __global__ void __launch_bounds__(threads_for(kQuant, kW4A16), 1)
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
+// ---------------------------------------------------------------------------
+// Pair tiles: two CTAs on two SMs compute one 256-row x 256-column tile with
+// tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 64 per instruction).
+//
+// Why: the single-CTA kernel above is bound by how fast TMA fills each SM's
+// shared memory (about 30 bytes per clock per SM), not by its MMAs.  In a
+// pair, CTA r holds rows [128 r, 128 r + 128) of A and rows
+// [128 r, 128 r + 128) of the tile's 256 weight rows; the MMA issued by CTA 0
+// reads both CTAs' halves, so every SM loads 8 KB per 128 x 256 x 64 product
+// instead of 8 KB per 128 x 128 x 64: half the bytes per FLOP.  Each CTA
+// loads only its own halves (no multicast).
+//
+// Roles (448 threads, 14 warps, the same in both CTAs):
+//   warp 0 lane 0  TMA producer into this CTA's stage ring: its A rows, its
+//                  weight rows, the block scales of its A rows and of all 256
+//                  weight rows; then the BF16 correction operands R and Wc
+//                  (16-channel chunks) as extra stages after the K loop.
+//   warps 2..5     one per TMEM lane quarter: write each stage's block scales
+//                  into a TMEM slot of this CTA (tcgen05.st), or for the
+//                  correction stages rescale R in place to R / G; then
+//                  arrive on CTA 0's barrier of that slot.
+//   warp 1         allocates 512 TMEM columns in both CTAs (cta_group::2);
+//                  in CTA 0 lane 0 issues the MMAs once both CTAs' slots are
+//                  ready and commits their completion to both CTAs' barriers.
+//   warps 6..13    epilogue, two warps per lane quarter (128 accumulator
+//                  columns each): y = G * acc, BF16, TMA stores; or SwiGLU
+//                  (and the NVFP4 quantization of h) as the single-CTA kernel.
+// TMEM per CTA: [0, 256) the accumulator (one buffer), [256, 512) four
+// scale-factor slots of 64 columns (A scales in 16, B scales in 32).
+//
+// The BF16 correction is accumulated into the FP4 accumulator: the MMA adds
+// (R / G) . Wc, so y = G * acc = G * A.W + R . Wc up to the rounding of
+// R / G, computed as bf16(fp32(R * fp32(1 / G))) (a relative 2^-9 + 2^-23 of
+// each correction term).  G = g_a g_w[e] of the
+// tile's expert; a zero G (an all-zero input or expert) gives R / G = 0.
+//
+// Rows: each expert's 128-aligned segment is cut into 256-row pair blocks
+// from its first row; a segment with an odd number of 128-row blocks ends in
+// a pair block whose second half belongs to the next expert: CTA 1 loads no
+// A rows for it and its results are not stored.
+constexpr int PBM = 256;
+constexpr int PBN = 256;
+constexpr int kPairHalfBytes = 128 * kStageRowBytes;               // 16384: 128 rows x 256 FP4
+constexpr int kPairSfaBytes = 4 * 512;                              // its 128 A rows, 4 MMAs
+constexpr int kPairSfbBytes = 2 * 4 * 512;                          // all 256 weight rows, 4 MMAs
+constexpr int kPairStageBytes = 2 * kPairHalfBytes + kPairSfaBytes + kPairSfbBytes;   // 38912
+// this CTA's weight rows per stage: half of the 256 in a pair, all 256 alone
+__host__ __device__ constexpr int wide_b_bytes(bool pair) { return pair ? kPairHalfBytes : 2 * kPairHalfBytes; }
+__host__ __device__ constexpr int wide_stage_bytes(bool pair) {
+  return kPairHalfBytes + wide_b_bytes(pair) + kPairSfaBytes + kPairSfbBytes;       // 38912 or 55296
+}
+constexpr int kPairThreads = 448;
+constexpr int kPairSfSlots = 4;
+constexpr uint32_t kPairSfCol = 256;
+constexpr uint32_t kPairSlotCols = 64;
+constexpr int kPairEpiWarps = 8;
+// instruction descriptors with M = 256 (the pair's rows), N = 256
+constexpr uint32_t kIdescFp4Pair = (1u << 7) | (1u << 10) | (uint32_t(PBN >> 3) << 17) | (uint32_t(PBM >> 4) << 24);
+constexpr uint32_t kIdescBf16Pair =
+    (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(PBN >> 3) << 17) | (uint32_t(PBM >> 4) << 24);
+// one CTA alone: M = 128, N = 256
+constexpr uint32_t kIdescFp4Wide = (1u << 7) | (1u << 10) | (uint32_t(PBN >> 3) << 17) | (uint32_t(128 >> 4) << 24);
+constexpr uint32_t kIdescBf16Wide =
+    (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(PBN >> 3) << 17) | (uint32_t(128 >> 4) << 24);
+// output staging: each epilogue warp stages 32 rows x 64 columns at a time
+__host__ __device__ constexpr int pair_out_bytes() { return kPairEpiWarps * 2 * kOutChunkBytes; }
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+// Address of the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ bool mbar_test_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait (as mbar_wait) on a barrier that the peer CTA also arrives on.
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                                  uint64_t limit_ns) {
+  if (mbar_test_cluster(bar, parity)) return true;
+  const uint64_t t0 = global_timer();
+  while (true) {
+    if (mbar_test_cluster(bar, parity)) return true;
+    if (abort_flag != nullptr && *abort_flag) return false;
+    if (global_timer() - t0 > limit_ns) {
+      if (abort_flag != nullptr) *abort_flag = 1;
+      atomicOr(&g_wait_status, 1u);
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// Completion of this thread's earlier MMAs arrives on the barrier at the same
+// offset in every CTA of `mask`.
+__device__ __forceinline__ void tc_commit_pair_mc(uint32_t bar, uint16_t mask) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::
+                   "r"(bar), "h"(mask)
+               : "memory");
+}
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mma_fp4_pair(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa,
+                                             uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// h = silu(gate) * up for two packed BF16 pairs, in FP32 as quads_swiglu
+// computes it, rounded to a packed BF16 pair.
+__device__ __forceinline__ uint32_t swiglu_bf16x2(uint32_t yg, uint32_t yu) {
+  float r[2];
+#pragma unroll
+  for (int hl = 0; hl < 2; ++hl) {
+    const float gt = bf16_bits_to_float(hl ? (yg >> 16) : (yg & 0xFFFFu));
+    const float ut = bf16_bits_to_float(hl ? (yu >> 16) : (yu & 0xFFFFu));
+    r[hl] = __fmul_rn(__fdividef(gt, 1.0f + __expf(-gt)), ut);
+  }
+  return pack_bf16x2(r[0], r[1]);
+}
+
+// Stage 32 rows x 32 BF16 columns (this lane's row: 16 packed words) in a
+// 2 KB buffer with the store map's 64-byte swizzle.
+__device__ __forceinline__ void stage_chunk(uint32_t sb, int lane, const uint32_t (&o)[16]) {
+  const uint32_t row_addr = sb + lane * 64;
+  const uint32_t sw = (lane >> 1) & 3u;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) st_shared_v4(row_addr + ((j ^ sw) << 4), o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+}
+
+template <bool kSwiglu, bool kQuant, bool kPair>
+__global__ void __launch_bounds__(kPairThreads, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                             const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_wc,
+                             const __grid_constant__ CUtensorMap tm_y, GemmParams p) {
+  static_assert(kSwiglu || !kQuant, "the quantizing epilogue follows SwiGLU");
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* const base_ptr = smem_raw + (base - raw);
+  const int S = p.stages;
+  constexpr int kSB = wide_stage_bytes(kPair);
+  constexpr int kBB = wide_b_bytes(kPair);
+  constexpr int kRows = kPair ? PBM : 128;        // rows of a tile
+  constexpr int kWcChunk = kPair ? kCompChunkBytes : 2 * kCompChunkBytes;   // Wc chunk: this CTA's weight rows
+  const uint32_t rank = kPair ? cluster_ctarank() : 0u;
+  const uint32_t out_stage = base + S * kSB;
+  constexpr int kOutB = pair_out_bytes();
+  const uint32_t bar0 = out_stage + kOutB;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
+  auto sf_full = [&](int i) { return bar0 + 8u * (2 * S + i); };
+  auto sf_empty = [&](int i) { return bar0 + 8u * (2 * S + kPairSfSlots + i); };
+  const uint32_t acc_full = bar0 + 8u * (2 * S + 2 * kPairSfSlots);
+  const uint32_t acc_empty = acc_full + 8;
+  const uint32_t drain_bar = acc_full + 16;
+  uint8_t* const misc = base_ptr + (drain_bar + 8 - base);
+  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(misc);
+  volatile int* const abort_flag = reinterpret_cast<volatile int*>(misc + 4);
+  int32_t* const off_s = reinterpret_cast<int32_t*>(misc + 16);       // E + 1, clamped to rows_cap
+  int32_t* const pb_s = off_s + p.E + 1;                                 // E + 1: first pair block of each expert
+  float* const gscale_s = reinterpret_cast<float*>(pb_s + p.E + 1);     // g_a(e) * g_w[e]
+  float* const gh_s = gscale_s + p.E;                                    // kQuant: h's per-expert scale
+  int32_t* const chanh_s = reinterpret_cast<int32_t*>(gh_s + p.E);     // n_chan_h
+  int32_t* const hslot_s = chanh_s + p.n_chan_h;                        // N / 64 + 1
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int i = 0; i < kPairSfSlots; ++i) {
+      mbar_init(sf_full(i), kPair ? 2 * 4 : 4);   // four scale warps in each CTA
+      mbar_init(sf_empty(i), 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, kPair ? 2 * kPairEpiWarps : kPairEpiWarps);   // every epilogue warp of both CTAs
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    if constexpr (kPair) {
+      tmem_alloc_pair(smem_addr(tmem_slot), kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_addr(tmem_slot), kTmemCols);
+      tmem_relinquish();
+    }
+  }
+  for (int i = threadIdx.x; i <= p.E; i += blockDim.x) {
+    off_s[i] = min(p.expert_off[i], p.rows_cap);
+    if (i < p.E) gscale_s[i] = __fmul_rn(p.g_a[p.g_a_per_expert ? i : 0], p.g_w[i]);
+  }
+  if constexpr (kQuant) {
+    const int Fh = p.N / 2;
+    for (int i = threadIdx.x; i < p.E; i += blockDim.x) {
+      gh_s[i] = __fdiv_rn(p.amax_h_in[i], kNvfp4Range);
+      if (blockIdx.x == 0 && p.g_h_out != nullptr) p.g_h_out[i] = gh_s[i];
+    }
+    for (int j = threadIdx.x; j < p.n_chan_h; j += blockDim.x) chanh_s[j] = p.chan_h[j];
+    __syncthreads();
+    for (int qc = threadIdx.x; qc <= Fh / 32; qc += blockDim.x) {
+      int cnt = 0;
+      for (int j = 0; j < p.n_chan_h; ++j) cnt += (chanh_s[j] >= 0 && chanh_s[j] < Fh && chanh_s[j] < 32 * qc) ? 1 : 0;
+      hslot_s[qc] = cnt;
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    pb_s[0] = 0;
+    for (int e = 0; e < p.E; ++e) pb_s[e + 1] = pb_s[e] + (max(off_s[e + 1] - off_s[e], 0) + kRows - 1) / kRows;
+  }
+  tc_fence_before();
+  if constexpr (kPair)
+    cluster_sync_all();                // barriers initialized and TMEM allocated in both CTAs
+  else
+    __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int n_ntiles = p.N / PBN;
+  const int total = pb_s[p.E] * n_ntiles;
+  const int nkb_total = p.K / 64;
+  const int nks_main = (nkb_total + 3) / 4;
+  const int nch = p.n_chan / 16;                  // 16-channel chunks of the BF16 correction
+  const int nks = nks_main + (nch + 3) / 4;
+  const int n_col_tiles = nkb_total;
+  const int cluster_id = kPair ? blockIdx.x >> 1 : blockIdx.x, n_clusters = kPair ? gridDim.x >> 1 : gridDim.x;
+  // pair tile t: expert e, first row m0, column tile nt, and whether its
+  // second 128 rows belong to e
+  auto tile_of = [&](int t, int& e, int& m0, int& nt, bool& hi_valid) {
+    const int pb = t / n_ntiles;
+    nt = t - pb * n_ntiles;
+    e = expert_of_row(pb_s, p.E, pb);
+    m0 = off_s[e] + kRows * (pb - pb_s[e]);
+    hi_valid = !kPair || m0 + 128 < off_s[e + 1];
+  };
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ producer
+    int it = 0;
+    bool ok = true;
+    for (int t = cluster_id; t < total && ok; t += n_clusters) {
+      int e, m0, nt;
+      bool hi_valid;
+      tile_of(t, e, m0, nt, hi_valid);
+      const bool av = rank == 0 || hi_valid;      // this CTA's A rows belong to the tile's expert
+      const int row0 = m0 + 128 * static_cast<int>(rank);
+      const int brow = e * p.N + nt * PBN;        // the tile's first weight row
+      const int myb = brow + 128 * static_cast<int>(rank);
+      for (int ks = 0; ks < nks; ++ks, ++it) {
+        const int s = it % S;
+        const uint32_t ph = (it / S) & 1;
+        if (!mbar_wait_cluster(empty_bar(s), ph ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+        const uint32_t st = base + s * kSB;
+        if (ks < nks_main) {
+          const int nkb = min(4, nkb_total - ks * 4);
+          mbar_expect_tx(full_bar(s), kBB + 2 * nkb * 512 + (av ? kPairHalfBytes + nkb * 512 : 0));
+          if (av) {
+            tma_load_2d(st, &tm_a, ks * kStageRowBytes, row0, full_bar(s));
+            bulk_load(st + kPairHalfBytes + kBB,
+                      p.a_scales + (static_cast<int64_t>(row0 / 128) * n_col_tiles + ks * 4) * 512, nkb * 512,
+                      full_bar(s));
+          }
+          tma_load_2d(st + kPairHalfBytes, &tm_b, ks * kStageRowBytes, myb, full_bar(s));   // 128 or 256 rows
+#pragma unroll
+          for (int b = 0; b < 2; ++b)
+            bulk_load(st + kPairHalfBytes + kBB + kPairSfaBytes + b * 2048,
+                      p.w_scales + (static_cast<int64_t>(brow / 128 + b) * n_col_tiles + ks * 4) * 512, nkb * 512,
+                      full_bar(s));
+        } else {
+          const int j0 = (ks - nks_main) * 4, nj = min(4, nch - j0);
+          mbar_expect_tx(full_bar(s), nj * (kWcChunk + (av ? kCompChunkBytes : 0)));
+          for (int j = 0; j < nj; ++j) {
+            if (av) tma_load_2d(st + j * kCompChunkBytes, &tm_r, (j0 + j) * 16, row0, full_bar(s));
+            tma_load_2d(st + kPairHalfBytes + j * kWcChunk, &tm_wc, (j0 + j) * 16, myb, full_bar(s));
+          }
+        }
+      }
+    }
+    if (!ok) {
+      for (int i = (it > S ? it - S : 0); i < it; ++i) mbar_wait(full_bar(i % S), (i / S) & 1, nullptr, kDrainTimeoutNs);
+    }
+  } else if (warp == 1 && lane == 0 && rank == 0) {
+    // ------------------------------------------------- MMA (CTA 0 of the pair)
+    int it = 0, tc = 0;
+    bool ok = true;
+    for (int t = cluster_id; t < total && ok; t += n_clusters, ++tc) {
+      if (!mbar_wait_cluster(acc_empty, (tc & 1) ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+      tc_fence_after();
+      for (int ks = 0; ks < nks; ++ks, ++it) {
+        const int s = it % S, slot = it % kPairSfSlots;
+        if (!mbar_wait_cluster(sf_full(slot), (it / kPairSfSlots) & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+        if (!mbar_wait(full_bar(s), (it / S) & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t st = base + s * kSB;
+        const uint32_t tsfa = tmem + kPairSfCol + slot * kPairSlotCols;
+        const uint32_t tsfb = tsfa + 16;
+        if (ks < nks_main) {
+          const int nkb = min(4, nkb_total - ks * 4);
+          for (int kb = 0; kb < nkb; ++kb) {
+            const uint64_t da = desc_kmajor_sw128(st + kb * kMmaKBytes);
+            const uint64_t db = desc_kmajor_sw128(st + kPairHalfBytes + kb * kMmaKBytes);
+            const uint32_t acc = (ks | kb) != 0 ? 1u : 0u;
+            if constexpr (kPair)
+              mma_fp4_pair(tmem, da, db, kIdescFp4Pair, tsfa + 4 * kb, tsfb + 8 * kb, acc);
+            else
+              mma_fp4(tmem, da, db, kIdescFp4Wide, tsfa + 4 * kb, tsfb + 8 * kb, acc);
+          }
+        } else {
+          const int nj = min(4, nch - (ks - nks_main) * 4);
+          for (int j = 0; j < nj; ++j) {
+            const uint64_t da = desc_kmajor_sw32(st + j * kCompChunkBytes);
+            const uint64_t db = desc_kmajor_sw32(st + kPairHalfBytes + j * kWcChunk);
+            if constexpr (kPair)
+              mma_bf16_pair(tmem, da, db, kIdescBf16Pair, 1u);
+            else
+              mma_bf16(tmem, da, db, kIdescBf16Wide, 1u);
+          }
+        }
+        if constexpr (kPair) {
+          tc_commit_pair_mc(empty_bar(s), 3);
+          tc_commit_pair_mc(sf_empty(slot), 3);
+        } else {
+          tc_commit(empty_bar(s));
+          tc_commit(sf_empty(slot));
+        }
+      }
+      if (!ok) break;
+      if constexpr (kPair)
+        tc_commit_pair_mc(acc_full, 3);
+      else
+        tc_commit(acc_full);
+    }
+    if (!ok) {
+      if constexpr (kPair)
+        tc_commit_pair(drain_bar);
+      else
+        tc_commit(drain_bar);
+      mbar_wait(drain_bar, 0, nullptr, kDrainTimeoutNs);
+    }
+  } else if (warp >= 2 && warp <= 5) {
+    // ------------------------------------- block scales / rescaled residuals
+    // Lane i of the warp for lane quarter q writes TMEM lane 32 q + i of the
+    // slot: A scales of rows i + 32 j in column 4 kb + j and weight scales of
+    // rows i + 32 j (j < 8) in column 16 + 8 kb + j, for MMA kb of the stage
+    // (the layout a tcgen05.cp .32x128b.warpx4 of each 512-byte tile gives).
+    const int q = warp & 3;
+    int it = 0;
+    bool ok = true;
+    for (int t = cluster_id; t < total && ok; t += n_clusters) {
+      int e, m0, nt;
+      bool hi_valid;
+      tile_of(t, e, m0, nt, hi_valid);
+      const bool av = rank == 0 || hi_valid;
+      const float G = gscale_s[e];
+      const float Ginv = G > 0.0f ? __frcp_rn(G) : 0.0f;     // R / G as R * fp32(1 / G)
+      for (int ks = 0; ks < nks; ++ks, ++it) {
+        const int s = it % S, slot = it % kPairSfSlots;
+        bool w_ok = mbar_wait(full_bar(s), (it / S) & 1, abort_flag, p.timeout_ns);
+        if (w_ok) w_ok = mbar_wait_cluster(sf_empty(slot), ((it / kPairSfSlots) & 1) ^ 1u, abort_flag, p.timeout_ns);
+        if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t st = base + s * kSB;
+        if (ks < nks_main) {
+          const uint32_t sfa = st + kPairHalfBytes + kBB + lane * 16;
+          const uint32_t sfb = sfa + kPairSfaBytes;
+          const uint32_t tsf = tmem + (static_cast<uint32_t>(q * 32) << 16) + kPairSfCol + slot * kPairSlotCols;
+          uint32_t ra[16], rb[16], rc[16];
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb) {       // tiles past the stage's last K block are never read
+            const uint4 a = ld_shared_v4(sfa + kb * 512);
+            const uint4 b0 = ld_shared_v4(sfb + kb * 512);
+            const uint4 b1 = ld_shared_v4(sfb + 2048 + kb * 512);
+            ra[4 * kb] = a.x; ra[4 * kb + 1] = a.y; ra[4 * kb + 2] = a.z; ra[4 * kb + 3] = a.w;
+            uint32_t* d = kb < 2 ? rb : rc;
+            const int o = (kb & 1) * 8;
+            d[o] = b0.x; d[o + 1] = b0.y; d[o + 2] = b0.z; d[o + 3] = b0.w;
+            d[o + 4] = b1.x; d[o + 5] = b1.y; d[o + 6] = b1.z; d[o + 7] = b1.w;
+          }
+          tmem_store16(tsf, ra);
+          tmem_store16(tsf + 16, rb);
+          tmem_store16(tsf + 32, rc);
+          tmem_wait_st();
+          tc_fence_before();
+        } else if (av) {
+          // R / G rounded to BF16 (as R * fp32(1 / G)), in place: this lane's row of each chunk
+          // (32 bytes, wherever the 32-byte swizzle puts its halves)
+          const int nj = min(4, nch - (ks - nks_main) * 4);
+          for (int j = 0; j < nj; ++j) {
+            const uint32_t ad = st + j * kCompChunkBytes + (q * 32 + lane) * 32;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint4 v = ld_shared_v4(ad + 16 * h);
+              uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float lo = __fmul_rn(bf16_bits_to_float(w[i] & 0xFFFFu), Ginv);
+                const float hi = __fmul_rn(bf16_bits_to_float(w[i] >> 16), Ginv);
+                w[i] = pack_bf16x2(lo, hi);
+              }
+              st_shared_v4(ad + 16 * h, w[0], w[1], w[2], w[3]);
+            }
+          }
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (kPair)
+            mbar_arrive_cluster(mapa_shared(sf_full(slot), 0));
+          else
+            mbar_arrive(sf_full(slot));
+        }
+      }
+    }
+  } else if (warp >= 6) {
+    // ----------------------------------------------------------- epilogue
+    // Warp 6 + 4 hs + i reads TMEM lane quarter q = warp % 4 and accumulator
+    // columns [128 hs, 128 hs + 128).  Two 32-column chunks are read at a
+    // time; after the last read the accumulator is handed back to the MMA,
+    // and the rest of the tile's epilogue overlaps the next tile's MMAs.
+    const int q = warp & 3, hs = (warp - 6) >> 2;
+    const uint32_t stg = out_stage + (warp - 6) * (kOutB / kPairEpiWarps);
+    const uint32_t lead_acc_empty = kPair ? mapa_shared(acc_empty, 0) : acc_empty;
+    auto arrive_acc_empty = [&]() {
+      if constexpr (kPair)
+        mbar_arrive_cluster(lead_acc_empty);
+      else
+        mbar_arrive(lead_acc_empty);
+    };
+    int tc = 0;
+    for (int t = cluster_id; t < total; t += n_clusters, ++tc) {
+      int e, m0, nt;
+      bool hi_valid;
+      tile_of(t, e, m0, nt, hi_valid);
+      const bool valid = rank == 0 || hi_valid;
+      if (!mbar_wait_cluster(acc_full, tc & 1, abort_flag, p.timeout_ns)) break;
+      tc_fence_after();
+      const int row = m0 + 128 * static_cast<int>(rank) + q * 32 + lane;
+      const float G = gscale_s[e];
+      const uint32_t acc = tmem + (static_cast<uint32_t>(q * 32) << 16) + hs * 128;
+      if (!valid) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) arrive_acc_empty();
+        continue;
+      }
+      // the warp's stores of its previous tile must have read the staging buffer
+      if (lane == 0) bulk_wait_read_0();
+      __syncwarp();
+      auto release = [&]() {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) arrive_acc_empty();
+      };
+      if constexpr (!kSwiglu) {
+        // two halves of 64 columns through the warp's two 2 KB buffers
+#pragma unroll 1
+        for (int c2 = 0; c2 < 2; ++c2) {
+          uint32_t v[2][32];
+          tmem_load32(acc + c2 * 64, v[0]);
+          tmem_load32(acc + c2 * 64 + 32, v[1]);
+          tmem_wait_ld();
+          if (c2 == 1) {
+            release();
+            if (lane == 0) bulk_wait_read_0();      // the first half's stores have read the buffers
+            __syncwarp();
+          }
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint32_t o[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              o[j] = pack_bf16x2(__fmul_rn(__uint_as_float(v[h][2 * j]), G), __fmul_rn(__uint_as_float(v[h][2 * j + 1]), G));
+            stage_chunk(stg + h * kOutChunkBytes, lane, o);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              tma_store_2d(&tm_y, stg + h * kOutChunkBytes, nt * PBN + hs * 128 + c2 * 64 + h * 32, row - lane);
+            bulk_commit();
+          }
+        }
+      } else {
+        unsigned int hmax = 0u;
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          // gate columns [32 c, 32 c + 32) of the warp's 128 and the up columns 64 further
+          uint32_t vg[32], vu[32];
+          tmem_load32(acc + c * 32, vg);
+          tmem_load32(acc + 64 + c * 32, vu);
+          tmem_wait_ld();
+          if (c == 1) release();
+          uint32_t o[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const uint32_t yg = pack_bf16x2(__fmul_rn(__uint_as_float(vg[2 * j]), G),
+                                            __fmul_rn(__uint_as_float(vg[2 * j + 1]), G));
+            const uint32_t yu = pack_bf16x2(__fmul_rn(__uint_as_float(vu[2 * j]), G),
+                                            __fmul_rn(__uint_as_float(vu[2 * j + 1]), G));
+            o[j] = swiglu_bf16x2(yg, yu);
+            hmax = max(hmax, max(o[j] & 0x7FFFu, (o[j] >> 16) & 0x7FFFu));
+          }
+          const int hcol = nt * (PBN / 2) + hs * 64 + c * 32;
+          if constexpr (kQuant) quantize_h_chunk(p, o, gh_s[e], chanh_s, hslot_s, row, hcol, hcol == 0);
+          if (!kQuant || p.y != nullptr) stage_chunk(stg + c * kOutChunkBytes, lane, o);
+        }
+        if (!kQuant || p.y != nullptr) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+              tma_store_2d(&tm_y, stg + c * kOutChunkBytes, nt * (PBN / 2) + hs * 64 + c * 32, row - lane);
+            bulk_commit();
+          }
+        }
+        hmax = __reduce_max_sync(0xffffffffu, hmax);
+        if (lane == 0 && hmax != 0u && p.amax_bits != nullptr) atomicMax(&p.amax_bits[e], hmax << 16);
+      }
+    }
+    if (lane == 0) bulk_wait_all();
+  }
+  __syncwarp();
+  tc_fence_before();
+  if constexpr (kPair)
+    cluster_sync_all();                // every MMA has completed and no peer arrival is pending
+  else
+    __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    if constexpr (kPair)
+      tmem_dealloc_pair(tmem, kTmemCols);
+    else
+      tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
 // Per-expert amax for the FP4 compensation's residual:
 // amax_r[e] = fp32(fp32(G_e / g_wc[e]) * 2688), G_e = fp32(g_a g_w[e]); the
 // residual's decode scale times g_wc[e] is then G_e up to one rounding.
@@ -894,6 +1476,134 @@ extern "C" {
 namespace quads {
 namespace {
 
+// Tile shape of the FP4 grouped GEMMs with the BF16 correction (or none)
+// whose N is a multiple of 256 (quads_gemm_set_tile_shape): 0 = 128 x 128 on
+// one CTA (the kernel above), 1 = 128 x 256 on one CTA, 2 = 256 x 256 on a
+// pair of CTAs.  Other GEMMs always take the 128 x 128 kernel.
+int g_tile_shape = 1;
+
+size_t pair_smem_bytes(int stages, bool pair, int E, size_t extra_words) {
+  return 1024 + static_cast<size_t>(stages) * wide_stage_bytes(pair) + pair_out_bytes() +
+         static_cast<size_t>(2 * stages + 2 * kPairSfSlots + 3) * 8 + 16 +
+         (static_cast<size_t>(4 * E + 2) + extra_words) * 4;
+}
+
+// Clusters of two that fit on the device at once with this much shared
+// memory (one CTA per SM), cached per kernel instance.
+template <bool kSwiglu, bool kQuant>
+int pair_clusters(size_t smem) {
+  static int cached = -1;
+  static size_t cached_smem = 0;
+  if (cached > 0 && cached_smem == smem) return cached;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(2 * (num_sms() / 2), 1, 1);
+  cfg.blockDim = dim3(kPairThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr{};
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = 2;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_pair_kernel<kSwiglu, kQuant, true>, &cfg) != cudaSuccess ||
+      n <= 0) {
+    cudaGetLastError();
+    n = num_sms() / 2;
+  }
+  cached = n;
+  cached_smem = smem;
+  return n;
+}
+
+template <bool kSwiglu, bool kQuant, bool kPair>
+int launch_gemm_pair(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_a, int g_a_per_expert,
+                     const uint8_t* w_codes, const uint8_t* w_scales, const float* g_w, const int32_t* expert_off,
+                     int E, int64_t rows_cap, int64_t N, int64_t K, const uint16_t* a_resid, const uint16_t* w_resid,
+                     int n_chan, uint16_t* y, float* amax_out, cudaStream_t stream, const HQuant* hq) {
+  CUtensorMap tm_a, tm_b, tm_r, tm_wc, tm_y;
+  const uint32_t wrows = kPair ? 128 : 256;       // weight rows this CTA loads per tile
+  QUADS_TRY(make_map_2d(&tm_a, a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, rows_cap, kStageRowBytes, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B));
+  QUADS_TRY(make_map_2d(&tm_b, w_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, E * N, kStageRowBytes, wrows,
+                        CU_TENSOR_MAP_SWIZZLE_128B));
+  if (n_chan) {
+    QUADS_TRY(make_map_2d(&tm_r, a_resid, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, n_chan, rows_cap, 16, 128,
+                          CU_TENSOR_MAP_SWIZZLE_32B));
+    QUADS_TRY(make_map_2d(&tm_wc, w_resid, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, n_chan, E * N, 16, wrows,
+                          CU_TENSOR_MAP_SWIZZLE_32B));
+  } else {
+    tm_r = tm_a;
+    tm_wc = tm_a;
+  }
+  if (y)
+    QUADS_TRY(make_map_2d(&tm_y, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kSwiglu ? N / 2 : N, rows_cap, 32, 32,
+                          CU_TENSOR_MAP_SWIZZLE_64B));
+  else
+    tm_y = tm_a;                                  // never used: no h store
+  const size_t extra = kQuant ? static_cast<size_t>(hq->n_chan + N / 64 + 1) : 0;
+  const size_t smem_cap = 232448;
+  int stages = kMaxStages;
+  while (stages >= 2 && pair_smem_bytes(stages, kPair, E, extra) > smem_cap) --stages;
+  QUADS_REQUIRE(stages >= 2, QUADS_ERR_UNSUPPORTED_SHAPE, "not enough shared memory for two stages");
+  const size_t smem = pair_smem_bytes(stages, kPair, E, extra);
+  auto kernel = grouped_gemm_pair_kernel<kSwiglu, kQuant, kPair>;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+      cudaSuccess)
+    return set_error(QUADS_ERR_CUDA, "cannot set %zu bytes of shared memory", smem);
+  GemmParams p{};
+  p.a_scales = a_scales;
+  p.w_scales = w_scales;
+  p.g_a = g_a;
+  p.g_w = g_w;
+  p.expert_off = expert_off;
+  p.y = y;
+  p.amax_bits = reinterpret_cast<unsigned int*>(amax_out);
+  p.amax_h_in = kQuant ? hq->amax_in : nullptr;
+  p.chan_h = kQuant ? hq->chan : nullptr;
+  p.n_chan_h = kQuant ? hq->n_chan : 0;
+  p.h_codes = kQuant ? hq->codes : nullptr;
+  p.h_scales = kQuant ? hq->scales : nullptr;
+  p.h_resid = kQuant ? hq->resid : nullptr;
+  p.g_h_out = kQuant ? hq->g_out : nullptr;
+  p.g_a_per_expert = g_a_per_expert ? 1 : 0;
+  p.E = E;
+  p.rows_cap = static_cast<int>(rows_cap);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.n_chan = n_chan;
+  p.stages = stages;
+  p.timeout_ns = kGemmTimeoutNs;
+  // at most one tile per 128 rows and 256 columns
+  const int64_t max_tiles = (rows_cap / 128) * (N / PBN);
+  if constexpr (kPair) {
+    int64_t clusters = pair_clusters<kSwiglu, kQuant>(smem);
+    if (clusters > max_tiles) clusters = max_tiles;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
+    cfg.blockDim = dim3(kPairThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr{};
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kernel, tm_a, tm_b, tm_r, tm_wc, tm_y, p) != cudaSuccess)
+      return set_error(QUADS_ERR_CUDA, "launch of the pair-tile GEMM failed: %s",
+                       cudaGetErrorString(cudaGetLastError()));
+  } else {
+    int64_t grid = num_sms();
+    if (grid > max_tiles) grid = max_tiles;
+    kernel<<<static_cast<unsigned>(grid), kPairThreads, smem, stream>>>(tm_a, tm_b, tm_r, tm_wc, tm_y, p);
+  }
+  count_launches(1);
+  return check_launch("grouped_gemm_pair_kernel");
+}
+
 template <bool kSwiglu, bool kQuant = false, bool kW4A16 = false, int kBN = BN>
 int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_a, int g_a_per_expert,
                 const uint8_t* w_codes, const uint8_t* w_scales, const float* g_w, const int32_t* expert_off, int E,
@@ -937,6 +1647,17 @@ int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_
   if (kSwiglu && amax_out && cudaMemsetAsync(amax_out, 0, sizeof(float) * E, stream) != cudaSuccess)
     return set_error(QUADS_ERR_CUDA, "memset of amax_out failed");
   if (rows_cap == 0) return QUADS_OK;
+  if constexpr (!kW4A16 && kBN == BN) {
+    if (fc == nullptr && g_tile_shape != 0 && N % PBN == 0) {
+      if (g_tile_shape == 2)
+        return launch_gemm_pair<kSwiglu, kQuant, true>(a_codes, a_scales, g_a, g_a_per_expert, w_codes, w_scales,
+                                                       g_w, expert_off, E, rows_cap, N, K, a_resid, w_resid, n_chan,
+                                                       y, amax_out, stream, hq);
+      return launch_gemm_pair<kSwiglu, kQuant, false>(a_codes, a_scales, g_a, g_a_per_expert, w_codes, w_scales, g_w,
+                                                      expert_off, E, rows_cap, N, K, a_resid, w_resid, n_chan, y,
+                                                      amax_out, stream, hq);
+    }
+  }
 
   CUtensorMap tm_a, tm_b, tm_r, tm_wc, tm_y;
   if (kW4A16) {
@@ -1123,6 +1844,14 @@ int quads_moe_grouped_gemm_nvfp4_swiglu(const uint8_t* a_codes, const uint8_t* a
                 (long long)F);
   return launch_gemm<true>(a_codes, a_scales, g_a, g_a_per_expert, w_codes, w_scales, g_w, expert_off, E, rows_cap,
                            2 * F, K, a_resid, w_resid, n_chan, h, amax_out, stream);
+}
+
+int quads_gemm_set_tile_shape(int shape) {
+  clear_error();
+  QUADS_REQUIRE(shape >= 0 && shape <= 2, QUADS_ERR_INVALID_ARG, "tile shape must be 0, 1 or 2");
+  const int prev = g_tile_shape;
+  g_tile_shape = shape;
+  return prev;
 }
 
 int quads_device_status(quads_stream_t stream) {
