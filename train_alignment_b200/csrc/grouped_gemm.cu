@@ -1089,7 +1089,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       for (int ks = 0; ks < nks; ++ks, ++it) {
         const int s = it % S;
         const uint32_t ph = (it / S) & 1;
-        if (!mbar_wait_cluster(empty_bar(s), ph ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+        const bool e_ok = kPair ? mbar_wait_cluster(empty_bar(s), ph ^ 1u, abort_flag, p.timeout_ns)
+                                : mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, p.timeout_ns);
+        if (!e_ok) { ok = false; break; }
         const uint32_t st = base + s * kSB;
         if (ks < nks_main) {
           const int nkb = min(4, nkb_total - ks * 4);
@@ -1124,12 +1126,20 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     int it = 0, tc = 0;
     bool ok = true;
     for (int t = cluster_id; t < total && ok; t += n_clusters, ++tc) {
-      if (!mbar_wait_cluster(acc_empty, (tc & 1) ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+      const bool acc_ok = kPair ? mbar_wait_cluster(acc_empty, (tc & 1) ^ 1u, abort_flag, p.timeout_ns)
+                                : mbar_wait(acc_empty, (tc & 1) ^ 1u, abort_flag, p.timeout_ns);
+      if (!acc_ok) { ok = false; break; }
       tc_fence_after();
       for (int ks = 0; ks < nks; ++ks, ++it) {
-        const int s = it % S, slot = it % kPairSfSlots;
-        if (!mbar_wait_cluster(sf_full(slot), (it / kPairSfSlots) & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
-        if (!mbar_wait(full_bar(s), (it / S) & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+        // One CTA: a scale slot per stage, and the scale warps' arrival (made
+        // after they saw the stage's data land) is the only wait.  Pair: the
+        // slots cycle on their own and the stage's own barrier is waited too.
+        const int s = it % S, slot = kPair ? it % kPairSfSlots : s;
+        const uint32_t sph = kPair ? (it / kPairSfSlots) & 1 : (it / S) & 1;
+        const bool sf_ok = kPair ? mbar_wait_cluster(sf_full(slot), sph, abort_flag, p.timeout_ns)
+                                 : mbar_wait(sf_full(slot), sph, abort_flag, p.timeout_ns);
+        if (!sf_ok) { ok = false; break; }
+        if (kPair && !mbar_wait(full_bar(s), (it / S) & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
         tc_fence_after();
         const uint32_t st = base + s * kSB;
         const uint32_t tsfa = tmem + kPairSfCol + slot * kPairSlotCols;
@@ -1160,8 +1170,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           tc_commit_pair_mc(empty_bar(s), 3);
           tc_commit_pair_mc(sf_empty(slot), 3);
         } else {
-          tc_commit(empty_bar(s));
-          tc_commit(sf_empty(slot));
+          tc_commit(empty_bar(s));           // frees the stage and its scale slot
         }
       }
       if (!ok) break;
@@ -1194,9 +1203,12 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       const float G = gscale_s[e];
       const float Ginv = G > 0.0f ? __frcp_rn(G) : 0.0f;     // R / G as R * fp32(1 / G)
       for (int ks = 0; ks < nks; ++ks, ++it) {
-        const int s = it % S, slot = it % kPairSfSlots;
+        // one CTA: the stage's data landing implies its slot is free (the
+        // producer refilled the stage only after the MMAs that read it)
+        const int s = it % S, slot = kPair ? it % kPairSfSlots : s;
         bool w_ok = mbar_wait(full_bar(s), (it / S) & 1, abort_flag, p.timeout_ns);
-        if (w_ok) w_ok = mbar_wait_cluster(sf_empty(slot), ((it / kPairSfSlots) & 1) ^ 1u, abort_flag, p.timeout_ns);
+        if (kPair && w_ok)
+          w_ok = mbar_wait_cluster(sf_empty(slot), ((it / kPairSfSlots) & 1) ^ 1u, abort_flag, p.timeout_ns);
         if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
         tc_fence_after();
         const uint32_t st = base + s * kSB;
@@ -1272,7 +1284,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       bool hi_valid;
       tile_of(t, e, m0, nt, hi_valid);
       const bool valid = rank == 0 || hi_valid;
-      if (!mbar_wait_cluster(acc_full, tc & 1, abort_flag, p.timeout_ns)) break;
+      const bool full_ok = kPair ? mbar_wait_cluster(acc_full, tc & 1, abort_flag, p.timeout_ns)
+                                 : mbar_wait(acc_full, tc & 1, abort_flag, p.timeout_ns);
+      if (!full_ok) break;
       tc_fence_after();
       const int row = m0 + 128 * static_cast<int>(rank) + q * 32 + lane;
       const float G = gscale_s[e];
@@ -1544,7 +1558,7 @@ int launch_gemm_pair(const uint8_t* a_codes, const uint8_t* a_scales, const floa
     tm_y = tm_a;                                  // never used: no h store
   const size_t extra = kQuant ? static_cast<size_t>(hq->n_chan + N / 64 + 1) : 0;
   const size_t smem_cap = 232448;
-  int stages = kMaxStages;
+  int stages = kPair ? kMaxStages : kPairSfSlots;  // one CTA: a scale slot per stage
   while (stages >= 2 && pair_smem_bytes(stages, kPair, E, extra) > smem_cap) --stages;
   QUADS_REQUIRE(stages >= 2, QUADS_ERR_UNSUPPORTED_SHAPE, "not enough shared memory for two stages");
   const size_t smem = pair_smem_bytes(stages, kPair, E, extra);
