@@ -1089,9 +1089,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       for (int ks = 0; ks < nks; ++ks, ++it) {
         const int s = it % S;
         const uint32_t ph = (it / S) & 1;
-        const bool e_ok = kPair ? mbar_wait_cluster(empty_bar(s), ph ^ 1u, abort_flag, p.timeout_ns)
-                                : mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, p.timeout_ns);
-        if (!e_ok) { ok = false; break; }
+        if (!mbar_wait_cluster(empty_bar(s), ph ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
         const uint32_t st = base + s * kSB;
         if (ks < nks_main) {
           const int nkb = min(4, nkb_total - ks * 4);
@@ -1124,22 +1122,20 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   } else if (warp == 1 && lane == 0 && rank == 0) {
     // ------------------------------------------------- MMA (CTA 0 of the pair)
     int it = 0, tc = 0;
+    int s = 0, slot = 0;                          // stage and scale slot of `it`
+    uint32_t ph = 0, sph = 0;                     // their phases
     bool ok = true;
     for (int t = cluster_id; t < total && ok; t += n_clusters, ++tc) {
-      const bool acc_ok = kPair ? mbar_wait_cluster(acc_empty, (tc & 1) ^ 1u, abort_flag, p.timeout_ns)
-                                : mbar_wait(acc_empty, (tc & 1) ^ 1u, abort_flag, p.timeout_ns);
-      if (!acc_ok) { ok = false; break; }
+      if (!mbar_wait_cluster(acc_empty, (tc & 1) ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
       tc_fence_after();
       for (int ks = 0; ks < nks; ++ks, ++it) {
         // One CTA: a scale slot per stage, and the scale warps' arrival (made
         // after they saw the stage's data land) is the only wait.  Pair: the
         // slots cycle on their own and the stage's own barrier is waited too.
-        const int s = it % S, slot = kPair ? it % kPairSfSlots : s;
-        const uint32_t sph = kPair ? (it / kPairSfSlots) & 1 : (it / S) & 1;
-        const bool sf_ok = kPair ? mbar_wait_cluster(sf_full(slot), sph, abort_flag, p.timeout_ns)
-                                 : mbar_wait(sf_full(slot), sph, abort_flag, p.timeout_ns);
-        if (!sf_ok) { ok = false; break; }
-        if (kPair && !mbar_wait(full_bar(s), (it / S) & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+        // (the cluster-scope acquire is used even for a CTA alone: its
+        // waits measured faster at tile boundaries)
+        if (!mbar_wait_cluster(sf_full(slot), sph, abort_flag, p.timeout_ns)) { ok = false; break; }
+        if (kPair && !mbar_wait(full_bar(s), ph, abort_flag, p.timeout_ns)) { ok = false; break; }
         tc_fence_after();
         const uint32_t st = base + s * kSB;
         const uint32_t tsfa = tmem + kPairSfCol + slot * kPairSlotCols;
@@ -1171,6 +1167,13 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           tc_commit_pair_mc(sf_empty(slot), 3);
         } else {
           tc_commit(empty_bar(s));           // frees the stage and its scale slot
+        }
+        if (++s == S) { s = 0; ph ^= 1u; }
+        if constexpr (kPair) {
+          if (++slot == kPairSfSlots) { slot = 0; sph ^= 1u; }
+        } else {
+          slot = s;
+          sph = ph;
         }
       }
       if (!ok) break;
@@ -1284,9 +1287,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       bool hi_valid;
       tile_of(t, e, m0, nt, hi_valid);
       const bool valid = rank == 0 || hi_valid;
-      const bool full_ok = kPair ? mbar_wait_cluster(acc_full, tc & 1, abort_flag, p.timeout_ns)
-                                 : mbar_wait(acc_full, tc & 1, abort_flag, p.timeout_ns);
-      if (!full_ok) break;
+      if (!mbar_wait_cluster(acc_full, tc & 1, abort_flag, p.timeout_ns)) break;
       tc_fence_after();
       const int row = m0 + 128 * static_cast<int>(rank) + q * 32 + lane;
       const float G = gscale_s[e];
@@ -1306,26 +1307,32 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         if (lane == 0) arrive_acc_empty();
       };
       if constexpr (!kSwiglu) {
-        // two halves of 64 columns through the warp's two 2 KB buffers
-#pragma unroll 1
+        // all 128 columns are read and rounded to BF16 before the accumulator
+        // is handed back; then two halves of 64 columns go out through the
+        // warp's two 2 KB buffers
+        uint32_t ob[4][16];
+#pragma unroll
         for (int c2 = 0; c2 < 2; ++c2) {
           uint32_t v[2][32];
           tmem_load32(acc + c2 * 64, v[0]);
           tmem_load32(acc + c2 * 64 + 32, v[1]);
           tmem_wait_ld();
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              ob[2 * c2 + h][j] = pack_bf16x2(__fmul_rn(__uint_as_float(v[h][2 * j]), G),
+                                              __fmul_rn(__uint_as_float(v[h][2 * j + 1]), G));
+        }
+        release();
+#pragma unroll
+        for (int c2 = 0; c2 < 2; ++c2) {
           if (c2 == 1) {
-            release();
             if (lane == 0) bulk_wait_read_0();      // the first half's stores have read the buffers
             __syncwarp();
           }
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint32_t o[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-              o[j] = pack_bf16x2(__fmul_rn(__uint_as_float(v[h][2 * j]), G), __fmul_rn(__uint_as_float(v[h][2 * j + 1]), G));
-            stage_chunk(stg + h * kOutChunkBytes, lane, o);
-          }
+          for (int h = 0; h < 2; ++h) stage_chunk(stg + h * kOutChunkBytes, lane, ob[2 * c2 + h]);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
@@ -1337,22 +1344,29 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         }
       } else {
         unsigned int hmax = 0u;
-#pragma unroll 1
+        // gate columns [32 c, 32 c + 32) of the warp's 128 and the up columns
+        // 64 further, for both chunks, rounded to BF16 before the
+        // accumulator is handed back; SwiGLU follows from the rounded values
+        uint32_t yg[2][16], yu[2][16];
+#pragma unroll
         for (int c = 0; c < 2; ++c) {
-          // gate columns [32 c, 32 c + 32) of the warp's 128 and the up columns 64 further
           uint32_t vg[32], vu[32];
           tmem_load32(acc + c * 32, vg);
           tmem_load32(acc + 64 + c * 32, vu);
           tmem_wait_ld();
-          if (c == 1) release();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            yg[c][j] = pack_bf16x2(__fmul_rn(__uint_as_float(vg[2 * j]), G), __fmul_rn(__uint_as_float(vg[2 * j + 1]), G));
+            yu[c][j] = pack_bf16x2(__fmul_rn(__uint_as_float(vu[2 * j]), G), __fmul_rn(__uint_as_float(vu[2 * j + 1]), G));
+          }
+        }
+        release();
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
           uint32_t o[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const uint32_t yg = pack_bf16x2(__fmul_rn(__uint_as_float(vg[2 * j]), G),
-                                            __fmul_rn(__uint_as_float(vg[2 * j + 1]), G));
-            const uint32_t yu = pack_bf16x2(__fmul_rn(__uint_as_float(vu[2 * j]), G),
-                                            __fmul_rn(__uint_as_float(vu[2 * j + 1]), G));
-            o[j] = swiglu_bf16x2(yg, yu);
+            o[j] = swiglu_bf16x2(yg[c][j], yu[c][j]);
             hmax = max(hmax, max(o[j] & 0x7FFFu, (o[j] >> 16) & 0x7FFFu));
           }
           const int hcol = nt * (PBN / 2) + hs * 64 + c * 32;
