@@ -87,8 +87,17 @@ STACK8_T4096 = MoEConfig(
     description="8-layer MoE stack: 4096 tokens, hidden 2048, 64 experts top-4, "
                 "ffn 1024; the last 4 layers are recorded and replayed")
 
+# The prefill layer's per-expert shape (1024 routed rows per expert on
+# average, hidden 4096, ffn 1536, top-8, 128 + 128 channels) on 16 experts:
+# small enough (a few GB on the device) for kernel profiles.
+PREFILL_SLICE_T2048 = MoEConfig(
+    "prefill_slice_t2048_h4096_e16k8_f1536", T=2048, H=4096, E=16, k=8, F=1536,
+    n_chan=128, n_chan_f=128, x_kind="student_t", logit_kind="zipf",
+    description="16-expert slice of the prefill layer: 2048 tokens, hidden 4096, 16 experts top-8, "
+                "ffn 1536, Student-t(3) channel scales, 128 compensation channels (kernel profiles)")
+
 CONFIGS = {c.name: c for c in [MOE_T2048, decode_config(64), decode_config(512),
-                               decode_config(4096), PREFILL_T16384, STACK8_T4096]}
+                               decode_config(4096), PREFILL_T16384, STACK8_T4096, PREFILL_SLICE_T2048]}
 
 
 def _gen(device, seed):
