@@ -96,7 +96,8 @@ size_t quads_scales_bytes(int64_t rows, int64_t K, int scale_layout);
 /* ---------------------------------------------------------------- a1: amax
  * Per-group max |x| of a BF16 matrix (the tensor statistic behind the FP32
  * per-tensor scale, [format]).  Rows are split into groups either by
- * group_off (device int32 [n_groups + 1], ascending, group_off[0] = 0) or,
+ * group_off (device int32 [n_groups + 1], ascending, group_off[0] = 0; rows
+ * at or past group_off[n_groups] belong to no group and are not read) or,
  * when group_off is NULL, into n_groups groups of rows / n_groups rows each.
  * amax_out: device float[n_groups], overwritten.  K % 16 == 0, ld_x >= K,
  * ld_x % 8 == 0, x 16-byte aligned. */
@@ -220,6 +221,13 @@ int quads_moe_gather(const int32_t* src_of, const int32_t* expert_off, int E, in
                      const uint16_t* a_resid, int n_chan,
                      uint8_t* pa_codes, uint8_t* pa_scales, uint16_t* pa_resid,
                      quads_stream_t stream);
+/* Gathers BF16 rows into expert order: out[p] = x[src_of[p]] for
+ * p < expert_off[E], zeros on pad rows (src_of[p] == -1); rows >= expert_off[E]
+ * are untouched.  x [T][H], out [rows_cap][H], both 16-byte aligned,
+ * H % 8 == 0.  The trainer's BF16 activations for the W4A16 GEMMs
+ * ([QUADS-fr §2.2.A]: the trainer keeps BF16 activations). */
+int quads_moe_gather_bf16(const int32_t* src_of, const int32_t* expert_off, int E, int64_t rows_cap,
+                          const uint16_t* x, int64_t H, uint16_t* out, quads_stream_t stream);
 /* Router + permutation + gather in one call (same arguments as above). */
 int quads_moe_route_permute(const float* logits, int64_t T, int E, int k, int renorm,
                             int32_t* topk_idx, float* topk_w, int32_t* expert_off,

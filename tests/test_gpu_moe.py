@@ -103,6 +103,27 @@ def test_route_permute_composite(cuda_lib, T, E, k, K, nc):
         assert_bits_equal(F.bf16_bits(bf16_np(pr)[:n]), F.bf16_bits(M.gather_rows(resid, src_ref)), "gathered resid")
 
 
+@pytest.mark.parametrize("T,E,k,H", [(1, 4, 1, 64), (300, 8, 2, 1024), (4096, 64, 4, 2048)])
+def test_gather_bf16_parity(cuda_lib, T, E, k, H):
+    """BF16 rows gathered into expert order against the oracle's gather_rows:
+    bit for bit, pad rows zero, rows past expert_off[E] untouched."""
+    r = np.random.default_rng(T + E + H)
+    x = F.bf16_rne(r.standard_normal((T, H)).astype(np.float32))
+    idx_ref, _ = M.router_topk(r.standard_normal((T, E)), k)
+    off_ref, row_ref, src_ref = M.permute(idx_ref, E)
+    cap = cuda_lib.moe_rows_capacity(T, k, E)
+    src_full = np.full(cap, -7, dtype=np.int32)
+    src_full[:len(src_ref)] = src_ref
+    out = torch.full((cap, H), float("nan"), dtype=torch.bfloat16, device="cuda")
+    cuda_lib.moe_gather_bf16(torch.from_numpy(src_full).cuda(), torch.from_numpy(off_ref).cuda(), E, cap,
+                             bf16_torch(x), out=out)
+    torch.cuda.synchronize()
+    n = int(off_ref[-1])
+    got = bf16_np(out)
+    assert_bits_equal(F.bf16_bits(got[:n]), F.bf16_bits(M.gather_rows(x, src_ref)), "gathered rows")
+    assert np.all(np.isnan(got[n:])), "rows past expert_off[E] must be untouched"
+
+
 def test_swiglu_parity(cuda_lib):
     E, F_ = 3, 256
     off = np.array([0, 128, 128, 384], dtype=np.int32)

@@ -160,6 +160,22 @@ def test_amax_groups(cuda_lib):
     assert_bits_equal(got, np.array(want), "amax")
 
 
+def test_amax_ignores_rows_past_the_last_group(cuda_lib):
+    """Rows at or past group_off[n] belong to no group: huge values there
+    (the unused tail of an expert-ordered buffer) change no group's amax, in
+    the strided and the contiguous kernel, and in the quantizer's own amax."""
+    x = _x(384, 128, 21)
+    x[300:] = 3.0e38
+    off = torch.tensor([0, 100, 100, 300], dtype=torch.int32, device="cuda")
+    full = bf16_torch(np.concatenate([x, np.zeros((384, 64))], axis=1))
+    want = [np.max(np.abs(x[0:100])), 0.0, np.max(np.abs(x[100:300]))]
+    assert_bits_equal(f32_of(cuda_lib.amax_bf16(bf16_torch(x), off, 3)), np.array(want), "amax contiguous")
+    assert_bits_equal(f32_of(cuda_lib.amax_bf16(full[:, :128], off, 3)), np.array(want), "amax strided")
+    _, _, g, _ = cuda_lib.quantize_nvfp4(bf16_torch(x), group_off=off, n_groups=3, scale_layout=cuda_lib.SCALES_TILED)
+    g_ref = [Q.tensor_scale(a) for a in want]
+    assert_bits_equal(f32_of(g).astype(np.float32), np.array(g_ref, dtype=np.float32), "g")
+
+
 @pytest.mark.parametrize("layout", [0, 1])
 def test_dequant_parity(cuda_lib, layout):
     x = _x(257, 512, 11)

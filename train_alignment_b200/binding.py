@@ -79,6 +79,7 @@ _SIGS = {
     "quads_moe_permute": (c_i32, [c_vp, c_i64, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
     "quads_moe_gather": (c_i32, [c_vp, c_vp, c_i32, c_i64, c_vp, c_vp, c_i64, c_vp, c_i32, c_vp, c_vp, c_vp,
                                  c_vp]),
+    "quads_moe_gather_bf16": (c_i32, [c_vp, c_vp, c_i32, c_i64, c_vp, c_i64, c_vp, c_vp]),
     "quads_moe_route_permute": (c_i32, [c_vp, c_i64, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_i64,
                                         c_vp, c_vp, c_i64, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
     "quads_moe_grouped_gemm_nvfp4": (c_i32, [c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_i32, c_i64, c_i64,
@@ -319,6 +320,16 @@ def moe_gather(src_of, expert_off, E, rows_cap, a_codes, a_scales, K, a_resid=No
                                    _p(a_resid), n_chan, _p(pa_codes), _p(pa_scales),
                                    _p(pa_resid) if n_chan else None, _s()), "quads_moe_gather")
     return pa_codes, pa_scales, (pa_resid if n_chan else None)
+
+
+def moe_gather_bf16(src_of, expert_off, E, rows_cap, x, out=None):
+    """BF16 rows of x in expert order (pad rows zero): [rows_cap, H]."""
+    _dev(x, torch.bfloat16, "x")
+    H = x.shape[1]
+    out = out if out is not None else _empty((rows_cap, H), torch.bfloat16, x.device)
+    _check(load().quads_moe_gather_bf16(_p(src_of), _p(expert_off), E, rows_cap, _p(x), H, _p(out), _s()),
+           "quads_moe_gather_bf16")
+    return out
 
 
 def moe_route_permute(logits, k, a_codes, a_scales, K, a_resid=None, renorm=True):

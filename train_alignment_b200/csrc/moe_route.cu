@@ -313,6 +313,25 @@ __global__ void __launch_bounds__(256) gather_kernel(const int32_t* __restrict__
   }
 }
 
+// One warp per expert-ordered row: the BF16 row of its token in 16-byte
+// vectors, or zeros on a pad row (the trainer's BF16 activations gathered for
+// the W4A16 GEMMs).
+__global__ void __launch_bounds__(256) gather_bf16_kernel(const int32_t* __restrict__ src_of,
+                                                          const int32_t* __restrict__ expert_off, int E,
+                                                          const uint16_t* __restrict__ x, int64_t H,
+                                                          uint16_t* __restrict__ out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t rows = expert_off[E];
+  const int64_t nvec = H / 8;
+  for (int64_t p = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; p < rows;
+       p += (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5) {
+    const int t = src_of[p];
+    uint4* d = reinterpret_cast<uint4*>(out + p * H);
+    const uint4* sx = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t) * H);
+    for (int64_t j = lane; j < nvec; j += 32) d[j] = (t >= 0) ? __ldg(sx + j) : make_uint4(0, 0, 0, 0);
+  }
+}
+
 // ------------------------------------------------------------------- SwiGLU
 
 // Each thread: 8 outputs of one row.  Per-expert amax via shared atomics.
@@ -513,6 +532,20 @@ int quads_moe_gather(const int32_t* src_of, const int32_t* expert_off, int E, in
                                                                     pa_scales, pa_resid);
   count_launches(1);
   return check_launch("gather_kernel");
+}
+
+int quads_moe_gather_bf16(const int32_t* src_of, const int32_t* expert_off, int E, int64_t rows_cap,
+                          const uint16_t* x, int64_t H, uint16_t* out, quads_stream_t stream) {
+  clear_error();
+  QUADS_REQUIRE(E >= 1 && E <= kMaxE, QUADS_ERR_UNSUPPORTED_SHAPE, "E must be in [1, %d]", kMaxE);
+  QUADS_REQUIRE(H > 0 && H % 8 == 0, QUADS_ERR_UNSUPPORTED_SHAPE, "H must be a positive multiple of 8");
+  QUADS_REQUIRE(rows_cap >= 0 && rows_cap % 128 == 0, QUADS_ERR_INVALID_ARG, "rows_cap must be a multiple of 128");
+  QUADS_REQUIRE(src_of && expert_off && x && out, QUADS_ERR_INVALID_ARG, "null pointer");
+  QUADS_REQUIRE(aligned(x, 16) && aligned(out, 16), QUADS_ERR_INVALID_ARG, "x and out must be 16-byte aligned");
+  if (rows_cap == 0) return QUADS_OK;
+  gather_bf16_kernel<<<grid_rows(rows_cap * 32, 256), 256, 0, stream>>>(src_of, expert_off, E, x, H, out);
+  count_launches(1);
+  return check_launch("gather_bf16_kernel");
 }
 
 int quads_moe_route_permute(const float* logits, int64_t T, int E, int k, int renorm, int32_t* topk_idx,

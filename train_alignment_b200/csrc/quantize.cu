@@ -52,6 +52,7 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const uint16_t* __restri
   }
   __syncthreads();
   RowGroups grp{group_off ? off_s : nullptr, n_groups, uniform};
+  if (group_off != nullptr) rows = min(rows, static_cast<int64_t>(off_s[n_groups]));   // rows past the last group
   const int lane = threadIdx.x & 31;
   const int nkb = static_cast<int>(K / 16);
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
@@ -114,6 +115,7 @@ __global__ void __launch_bounds__(kThreads) amax_flat_kernel(const uint4* __rest
   }
   __syncthreads();
   RowGroups grp{group_off ? off_a : nullptr, n_groups, uniform};
+  if (group_off != nullptr) rows = min(rows, static_cast<int64_t>(off_a[n_groups]));   // rows past the last group
   const uint32_t nvec = static_cast<uint32_t>(rows * vec_per_row);   // < 2^31 (checked on the host)
   const uint32_t lane = threadIdx.x & 31;
   const uint32_t nwarps = gridDim.x * (blockDim.x >> 5);

@@ -30,7 +30,10 @@ report as drifting further than the asymmetric scheme: every
 layer fake-quantizes its input x (one per-tensor scale) and each expert's h
 (one scale per expert) on the NVFP4 grid, without compensation and without
 replay; its backward through those fake-quants is the same straight-through
-identity as for the weights.
+identity as for the weights.  It runs on the same kernels as the W4A16
+trainer: the fake-quant of x, the BF16 gather into expert order, the W4A16
+gate/up + SwiGLU, the per-expert quantize and dequantize of h, the W4A16
+down GEMM and the combine.
 """
 import torch
 
@@ -74,6 +77,8 @@ class LayerStack:
         self.t_ws = torch.empty(B.moe_permute_workspace_bytes(T, cfg.k, E), dtype=torch.uint8, device=self.dev)
         self.t_x = torch.zeros(cap, H, dtype=bf, device=self.dev)
         self.t_h = torch.empty(cap, cfg.F, dtype=bf, device=self.dev)
+        self.t_hq = torch.empty(cap, cfg.F, dtype=bf, device=self.dev)     # W4A4: fake-quantized h
+        self.t_amax = torch.empty(E, dtype=torch.float32, device=self.dev)
         self.t_y = torch.empty(cap, H, dtype=bf, device=self.dev)
         self.x_roll = torch.empty(cfg.layers + 1, T, H, dtype=torch.bfloat16, device=self.dev)
         self.x_train = torch.empty_like(self.x_roll)
@@ -115,20 +120,30 @@ class LayerStack:
             y.index_add_(0, t, yd * w.reshape(-1)[pos, None])
         return y.to(torch.bfloat16)
 
-    def _trainer_ffn_w4a16(self, layer, x, idx, w):
+    def _trainer_ffn_w4a16(self, layer, x, idx, w, w4a4=False):
         """The same FFN on the W4A16 kernels: the trainer's routing permutes
-        its BF16 rows into expert order (pad rows zero), gate/up + SwiGLU and
-        down read the NVFP4 weight codes, the combine kernel sums the slots."""
+        its BF16 rows into expert order (the gather kernel; pad rows zero),
+        gate/up + SwiGLU and down read the NVFP4 weight codes, the combine
+        kernel sums the slots.  w4a4: x fake-quantized first (one per-tensor
+        scale) and h quantized per expert segment and dequantized before the
+        down GEMM (one scale per expert)."""
         cfg = self.cfg
         E, H, F = cfg.E, cfg.H, cfg.F
         cap = self.t_x.shape[0]
+        if w4a4:
+            x = B.fakequant_weight_ste(x.unsqueeze(0), want_codes=False)[0][0]
         B.moe_permute(idx, E, self.t_off, self.t_row_of, self.t_src_of, self.t_ws)
-        src = self.t_src_of.long()
-        torch.where((src >= 0)[:, None], x[src.clamp_min(0)], torch.zeros((), dtype=x.dtype, device=x.device),
-                    out=self.t_x)
+        B.moe_gather_bf16(self.t_src_of, self.t_off, E, cap, x, out=self.t_x)
         B.moe_grouped_gemm_w4a16(self.t_x, layer.w_gu_codes, layer.w_gu_scales, layer.g_w_gu, self.t_off, E, cap,
-                                 2 * F, H, y=self.t_h, swiglu=True)
-        B.moe_grouped_gemm_w4a16(self.t_h, layer.w_d_codes, layer.w_d_scales, layer.g_w_d, self.t_off, E, cap, H,
+                                 2 * F, H, y=self.t_h, swiglu=True, amax=self.t_amax)
+        h = self.t_h
+        if w4a4:
+            # the per-expert max |h| comes from the SwiGLU epilogue
+            codes, scales, g_h, _ = B.quantize_nvfp4(self.t_h, group_off=self.t_off, n_groups=E,
+                                                     amax_in=self.t_amax, scale_layout=B.SCALES_TILED)
+            h = B.dequant(codes, scales, B.SCALES_TILED, g_h, cap, F, group_off=self.t_off, n_groups=E,
+                          out=self.t_hq)
+        B.moe_grouped_gemm_w4a16(h, layer.w_d_codes, layer.w_d_scales, layer.g_w_d, self.t_off, E, cap, H,
                                  F, y=self.t_y)
         return B.moe_unpermute_combine(self.t_y, self.t_row_of, w, cfg.T, cfg.k, H)
 
@@ -169,8 +184,8 @@ class LayerStack:
             else:
                 B.router_logits(xl, self.w_r[l], out=self.logits)
                 idx, w = B.moe_router_topk(self.logits, cfg.k, True)
-                if self.trainer_gemm == "w4a16" and not w4a4 and layer.fuse_swiglu:
-                    y = self._trainer_ffn_w4a16(layer, xl, idx, w)
+                if self.trainer_gemm == "w4a16" and layer.fuse_swiglu:
+                    y = self._trainer_ffn_w4a16(layer, xl, idx, w, w4a4)
                 else:
                     y = self._trainer_ffn(layer, xl, idx, w, w4a4)
             B.residual_add(xl, y, out=self.x_train[l + 1])
