@@ -277,17 +277,7 @@ def quantize_replay_sweep(dev, hbm_gbs, reps=10):
         q = lambda: B.quantize_nvfp4(x, amax_in=amax, codes=codes, scales=scales, g_out=g)
 
         def timed(fn):
-            fn()
-            ts = []
-            for _ in range(reps):
-                flush.zero_()
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record()
-                fn()
-                e1.record()
-                e1.synchronize()
-                ts.append(e0.elapsed_time(e1))
-            return sum(ts) / len(ts)
+            return _timed_flushed(fn, flush, reps)
 
         tq = timed(q)
         src = [B.qtensor_src(codes, scales, g, rows, K, B.SCALES_LINEAR)]
@@ -341,17 +331,7 @@ def trainer_gemm_timing(layer, dev, peaks, reps=20):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     def timed(fn):
-        fn()
-        ts = []
-        for _ in range(reps):
-            flush.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            fn()
-            e1.record()
-            e1.synchronize()
-            ts.append(e0.elapsed_time(e1))
-        return sum(ts) / len(ts)
+        return _timed_flushed(fn, flush, reps)
 
     t_w4 = None
     if layer.fuse_swiglu:           # the rollout's gate/up codes are in the interleaved order SwiGLU needs
@@ -377,18 +357,32 @@ def trainer_gemm_timing(layer, dev, peaks, reps=20):
 
 
 def _timed_flushed(fn, flush, reps=20):
+    """Median device time (ms) of the launches fn() makes, L2 flushed (a
+    write of a buffer larger than L2) before each.  The flush, two timing
+    events and fn are captured once in a CUDA graph (the events as external
+    event nodes, re-recorded at every replay), so the interval is the
+    kernels' own time as they run inside a step's graph: neither the host
+    work of preparing the launches (tensor maps, argument checks, the Python
+    binding) nor the graph's launch latency falls inside it, either of which
+    would dominate a kernel of tens of microseconds."""
     import torch
     fn()
-    ts = []
-    for _ in range(reps):
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    e0 = torch.cuda.Event(enable_timing=True, external=True)
+    e1 = torch.cuda.Event(enable_timing=True, external=True)
+    with torch.cuda.graph(graph):
         flush.zero_()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         fn()
         e1.record()
-        e1.synchronize()
+    ts = []
+    for _ in range(reps + 1):
+        graph.replay()
+        torch.cuda.synchronize()
         ts.append(e0.elapsed_time(e1))
-    ts.sort()
+    del graph
+    ts = sorted(ts[1:])
     return ts[len(ts) // 2]
 
 
@@ -413,8 +407,10 @@ def gemm_side_measurements(layer, dev, peaks):
     and without the BF16 correction on the same operands.  (2) Decode
     shapes (2048 hidden, 128 experts top-8, ffn 768, T = 64 and 512), measured
     as weight-stream bandwidth: the NVFP4 weight bytes (codes, scales and the
-    BF16 Wc columns) of every expert that received rows, over the GEMM time.
-    L2 flushed before each timed launch."""
+    BF16 Wc columns) of every expert that received rows, over the GEMM time,
+    on the tiles the library picks (the decode tiles, weights as the MMA's M
+    operand) and on the 128 x 256 tiles.  L2 flushed before each timed
+    launch."""
     import torch
     from train_alignment_b200 import layer as L
     from train_alignment_b200 import workloads as W
@@ -428,6 +424,7 @@ def gemm_side_measurements(layer, dev, peaks):
     out["compensation"] = {"us_with": tot, "us_without": tot0, "overhead_frac": tot / tot0 - 1.0,
                            "gate_up_us": [t["gate_up"], t["gate_up_nocomp"]], "down_us": [t["down"], t["down_nocomp"]]}
     dec = []
+    from train_alignment_b200 import binding as B
     for T in (64, 512):
         cfg = W.decode_config(T)
         inp = W.moe_layer_inputs(cfg, seed=0, device=dev)
@@ -437,14 +434,22 @@ def gemm_side_measurements(layer, dev, peaks):
         torch.cuda.synchronize()
         off = ly.expert_off.tolist()
         used = sum(1 for e in range(cfg.E) if off[e + 1] > off[e])
-        g, d = _gemm_calls(ly, True)
-        tg, td = _timed_flushed(g, flush) * 1e3, _timed_flushed(d, flush) * 1e3
         q = 0.5 + 1.0 / 16
         wb_g = used * 2 * cfg.F * (cfg.H * q + ly.nc_x * 2)
         wb_d = used * cfg.H * (cfg.F * q + ly.nc_h * 2)
-        dec.append({"workload": cfg.name, "experts_with_rows": used, "gate_up_us": tg, "down_us": td,
-                    "weight_bytes": wb_g + wb_d, "weight_stream_gbs": (wb_g + wb_d) / ((tg + td) * 1e-6) / 1e9,
-                    "frac_hbm": (wb_g + wb_d) / ((tg + td) * 1e-6) / 1e9 / peaks["hbm_gbs"]})
+        row = {"workload": cfg.name, "experts_with_rows": used, "weight_bytes": wb_g + wb_d}
+        # the library's own choice (decode tiles at these sizes), then the
+        # 128 x 256 tiles on the same operands for comparison
+        for key, rows in (("", None), ("tiles_128x256_", 0)):
+            prev = B.gemm_set_decode_rows(rows) if rows is not None else None
+            g, d = _gemm_calls(ly, True)
+            tg, td = _timed_flushed(g, flush) * 1e3, _timed_flushed(d, flush) * 1e3
+            if prev is not None:
+                B.gemm_set_decode_rows(prev)
+            gbs = (wb_g + wb_d) / ((tg + td) * 1e-6) / 1e9
+            row.update({key + "gate_up_us": tg, key + "down_us": td, key + "weight_stream_gbs": gbs,
+                        key + "frac_hbm": gbs / peaks["hbm_gbs"]})
+        dec.append(row)
         del ly, inp
         torch.cuda.empty_cache()
     out["decode"] = dec

@@ -89,6 +89,18 @@ int quads_selftest_bounded_wait(uint64_t timeout_ns, quads_stream_t stream);
  * Returns the previous shape, or QUADS_ERR_INVALID_ARG for another value.
  * Process-wide; not synchronized with launches in flight. */
 int quads_gemm_set_tile_shape(int shape);
+/* Decode tiles for the same GEMMs when they carry no fused quantization:
+ * the weights become the MMA's M operand (128 weight rows on the TMEM
+ * lanes) and the expert's rows its N operand (128 per tile); each tile
+ * computes 256 weight rows (for SwiGLU: 128 gate rows and the matching
+ * 128 up rows, so SwiGLU needs no exchange between TMEM lanes).
+ * Taken when N % 256 == 0 and the average rows per expert,
+ * max(0, rows_cap / 128 - E) * 128 / E, is at most `rows` (default 64);
+ * 0 never takes it.  The correction is folded as in shapes 1 and 2.  A
+ * tuning and testing switch, not a reading of the pages.  Returns the
+ * previous value, or QUADS_ERR_INVALID_ARG for a negative one.
+ * Process-wide; not synchronized with launches in flight. */
+int quads_gemm_set_decode_rows(int rows);
 
 /* Bytes of a scale array of `rows` x K/16 scales in the given layout. */
 size_t quads_scales_bytes(int64_t rows, int64_t K, int scale_layout);

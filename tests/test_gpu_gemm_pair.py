@@ -20,9 +20,11 @@ pytestmark = pytest.mark.gpu
 @pytest.fixture(params=[1, 2], ids=["128x256", "pair_256x256"])
 def pair_tiles(cuda_lib, request):
     prev = cuda_lib.gemm_set_tile_shape(request.param)
+    prev_dec = cuda_lib.gemm_set_decode_rows(0)         # these shapes, not the decode tiles
     cuda_lib.shape = request.param
     yield cuda_lib
     cuda_lib.gemm_set_tile_shape(prev)
+    cuda_lib.gemm_set_decode_rows(prev_dec)
 
 
 def _plain(lib, p, pair):

@@ -62,6 +62,7 @@ _SIGS = {
     "quads_device_status": (c_i32, [c_vp]),
     "quads_selftest_bounded_wait": (c_i32, [c_u64, c_vp]),
     "quads_gemm_set_tile_shape": (c_i32, [c_i32]),
+    "quads_gemm_set_decode_rows": (c_i32, [c_i32]),
     "quads_scales_bytes": (c_sz, [c_i64, c_i64, c_i32]),
     "quads_amax_bf16": (c_i32, [c_vp, c_i64, c_i64, c_i64, c_vp, c_i32, c_vp, c_vp]),
     "quads_quantize_workspace_bytes": (c_sz, [c_i32]),
@@ -199,6 +200,16 @@ def gemm_set_tile_shape(shape):
     prev = int(load().quads_gemm_set_tile_shape(int(shape)))
     if prev < 0:
         _check(prev, "quads_gemm_set_tile_shape")
+    return prev
+
+
+def gemm_set_decode_rows(rows):
+    """Average rows per expert at or below which the FP4 grouped GEMMs take
+    the decode tiles (weights as the MMA's M operand); 0: never.  Returns
+    the previous value."""
+    prev = int(load().quads_gemm_set_decode_rows(int(rows)))
+    if prev < 0:
+        _check(prev, "quads_gemm_set_decode_rows")
     return prev
 
 

@@ -126,6 +126,7 @@ struct GemmParams {
   int N;
   int K;
   int n_chan;
+  int comp_cw;               // channels per box of the correction operands (wide and decode tiles)
   int stages;
   uint64_t timeout_ns;
 };
@@ -288,6 +289,42 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t addr) {
 __device__ __forceinline__ uint64_t desc_kmajor_sw32(uint32_t addr) {
   return uint64_t((addr >> 4) & 0x3FFFu) | (uint64_t(1) << 16) | (uint64_t(256 >> 4) << 32) | (uint64_t(1) << 46) |
          (uint64_t(6) << 61);
+}
+
+// K-major descriptor for rows of row_bytes = 32, 64 or 128 bytes stored with
+// the swizzle of that width (8-row groups of 8 * row_bytes).
+__device__ __forceinline__ uint64_t desc_kmajor_rows(uint32_t addr, int row_bytes) {
+  const uint64_t layout = row_bytes == 128 ? 2u : (row_bytes == 64 ? 4u : 6u);
+  return uint64_t((addr >> 4) & 0x3FFFu) | (uint64_t(1) << 16) | (uint64_t((8 * row_bytes) >> 4) << 32) |
+         (uint64_t(1) << 46) | (layout << 61);
+}
+
+// out_s[0] = 0, out_s[e + 1] = out_s[e] + ceil(max(off_s[e + 1] - off_s[e], 0) / rows) * mult
+// for e < E <= 256; run by one whole warp (each lane a run of experts, a
+// shuffle scan across lanes).
+__device__ __forceinline__ void warp_block_prefix(int32_t* out_s, const int32_t* off_s, int E, int rows, int mult,
+                                                  int lane) {
+  const int per = (E + 31) / 32, e0 = lane * per;
+  int sum = 0;
+  for (int i = 0; i < per; ++i)
+    if (e0 + i < E) sum += (max(off_s[e0 + i + 1] - off_s[e0 + i], 0) + rows - 1) / rows * mult;
+  int incl = sum;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += v;
+  }
+  int run = incl - sum;
+  if (lane == 0) out_s[0] = 0;
+  for (int i = 0; i < per; ++i)
+    if (e0 + i < E) {
+      run += (max(off_s[e0 + i + 1] - off_s[e0 + i], 0) + rows - 1) / rows * mult;
+      out_s[e0 + i + 1] = run;
+    }
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* m) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
 
 __device__ __forceinline__ int expert_of_row(const int32_t* off_s, int E, int row) {
@@ -978,7 +1015,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   constexpr int kSB = wide_stage_bytes(kPair);
   constexpr int kBB = wide_b_bytes(kPair);
   constexpr int kRows = kPair ? PBM : 128;        // rows of a tile
-  constexpr int kWcChunk = kPair ? kCompChunkBytes : 2 * kCompChunkBytes;   // Wc chunk: this CTA's weight rows
+  // BF16 correction operands in boxes of cw channels (rows of 2 cw bytes, the
+  // swizzle of that width), 64 channels per stage: R [128 x cw] and this
+  // CTA's Wc rows [128 or 256 x cw] per box
+  const int cw = p.comp_cw, cps = 64 / cw;
+  const int rcb = 128 * 2 * cw, wcb = (kPair ? 128 : 256) * 2 * cw;
   const uint32_t rank = kPair ? cluster_ctarank() : 0u;
   const uint32_t out_stage = base + S * kSB;
   constexpr int kOutB = pair_out_bytes();
@@ -1002,6 +1043,12 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
+    prefetch_tensormap(&tm_a);
+    prefetch_tensormap(&tm_b);
+    if (p.n_chan) {
+      prefetch_tensormap(&tm_r);
+      prefetch_tensormap(&tm_wc);
+    }
     for (int s = 0; s < S; ++s) {
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
@@ -1044,10 +1091,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     }
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    pb_s[0] = 0;
-    for (int e = 0; e < p.E; ++e) pb_s[e + 1] = pb_s[e] + (max(off_s[e + 1] - off_s[e], 0) + kRows - 1) / kRows;
-  }
+  if (warp == 2) warp_block_prefix(pb_s, off_s, p.E, kRows, 1, lane);
   tc_fence_before();
   if constexpr (kPair)
     cluster_sync_all();                // barriers initialized and TMEM allocated in both CTAs
@@ -1060,8 +1104,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   const int total = pb_s[p.E] * n_ntiles;
   const int nkb_total = p.K / 64;
   const int nks_main = (nkb_total + 3) / 4;
-  const int nch = p.n_chan / 16;                  // 16-channel chunks of the BF16 correction
-  const int nks = nks_main + (nch + 3) / 4;
+  const int nch = p.n_chan / cw;                  // cw-channel boxes of the BF16 correction
+  const int nks = nks_main + (nch + cps - 1) / cps;
   const int n_col_tiles = nkb_total;
   const int cluster_id = kPair ? blockIdx.x >> 1 : blockIdx.x, n_clusters = kPair ? gridDim.x >> 1 : gridDim.x;
   // pair tile t: expert e, first row m0, column tile nt, and whether its
@@ -1107,11 +1151,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                       p.w_scales + (static_cast<int64_t>(brow / 128 + b) * n_col_tiles + ks * 4) * 512, nkb * 512,
                       full_bar(s));
         } else {
-          const int j0 = (ks - nks_main) * 4, nj = min(4, nch - j0);
-          mbar_expect_tx(full_bar(s), nj * (kWcChunk + (av ? kCompChunkBytes : 0)));
+          const int j0 = (ks - nks_main) * cps, nj = min(cps, nch - j0);
+          mbar_expect_tx(full_bar(s), nj * (wcb + (av ? rcb : 0)));
           for (int j = 0; j < nj; ++j) {
-            if (av) tma_load_2d(st + j * kCompChunkBytes, &tm_r, (j0 + j) * 16, row0, full_bar(s));
-            tma_load_2d(st + kPairHalfBytes + j * kWcChunk, &tm_wc, (j0 + j) * 16, myb, full_bar(s));
+            if (av) tma_load_2d(st + j * rcb, &tm_r, (j0 + j) * cw, row0, full_bar(s));
+            tma_load_2d(st + kPairHalfBytes + j * wcb, &tm_wc, (j0 + j) * cw, myb, full_bar(s));
           }
         }
       }
@@ -1152,15 +1196,16 @@ __global__ void __launch_bounds__(kPairThreads, 1)
               mma_fp4(tmem, da, db, kIdescFp4Wide, tsfa + 4 * kb, tsfb + 8 * kb, acc);
           }
         } else {
-          const int nj = min(4, nch - (ks - nks_main) * 4);
-          for (int j = 0; j < nj; ++j) {
-            const uint64_t da = desc_kmajor_sw32(st + j * kCompChunkBytes);
-            const uint64_t db = desc_kmajor_sw32(st + kPairHalfBytes + j * kWcChunk);
-            if constexpr (kPair)
-              mma_bf16_pair(tmem, da, db, kIdescBf16Pair, 1u);
-            else
-              mma_bf16(tmem, da, db, kIdescBf16Wide, 1u);
-          }
+          const int nj = min(cps, nch - (ks - nks_main) * cps);
+          for (int j = 0; j < nj; ++j)
+            for (int kk = 0; kk < cw / 16; ++kk) {      // K = 16 channels per MMA, 32 bytes along the row
+              const uint64_t da = desc_kmajor_rows(st + j * rcb + kk * 32, 2 * cw);
+              const uint64_t db = desc_kmajor_rows(st + kPairHalfBytes + j * wcb + kk * 32, 2 * cw);
+              if constexpr (kPair)
+                mma_bf16_pair(tmem, da, db, kIdescBf16Pair, 1u);
+              else
+                mma_bf16(tmem, da, db, kIdescBf16Wide, 1u);
+            }
         }
         if constexpr (kPair) {
           tc_commit_pair_mc(empty_bar(s), 3);
@@ -1237,13 +1282,16 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           tmem_wait_st();
           tc_fence_before();
         } else if (av) {
-          // R / G rounded to BF16 (as R * fp32(1 / G)), in place: this lane's row of each chunk
-          // (32 bytes, wherever the 32-byte swizzle puts its halves)
-          const int nj = min(4, nch - (ks - nks_main) * 4);
+          // R / G rounded to BF16 (as R * fp32(1 / G)), in place: this lane's row of each box
+          // (2 cw bytes; the swizzle permutes 16-byte pieces within the row)
+          // (each lane starts at another 16-byte piece: the rows of a
+          // quarter warp then fall in distinct banks)
+          const int nj = min(cps, nch - (ks - nks_main) * cps);
+          const int units = cw / 8, rot = (q * 32 + lane) >> (cw == 64 ? 0 : (cw == 32 ? 1 : 2));
           for (int j = 0; j < nj; ++j) {
-            const uint32_t ad = st + j * kCompChunkBytes + (q * 32 + lane) * 32;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
+            const uint32_t ad = st + j * rcb + (q * 32 + lane) * 2 * cw;
+            for (int hh = 0; hh < units; ++hh) {
+              const int h = (hh + rot) & (units - 1);
               const uint4 v = ld_shared_v4(ad + 16 * h);
               uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -1404,6 +1452,391 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Decode tiles: the weights as the MMA's M operand.
+//
+// At decode sizes an expert receives a handful of rows, so a 128-row A tile
+// is mostly padding and the GEMM is a stream of the experts' weights.  Here
+// the roles of the operands are swapped: D^T = W . A^T, with 128 weight rows
+// on the MMA's M (TMEM lanes) and up to 128 of the expert's rows on its N
+// (TMEM columns).  A work unit is (expert, 256 consecutive weight rows, a
+// block of up to 128 of the expert's rows), as two M = 128 halves sharing one
+// token tile (one 128-row box; rows past the expert's segment read as
+// zeros or belong to the next segment and only feed accumulator columns
+// that are never stored).
+//
+//   halves      plain: weight rows [0, 128) and [128, 256) of the unit.
+//               kSwiglu: the unit covers 128 h columns; half 0 holds their
+//               128 gate rows and half 1 the 128 up rows (weight rows are
+//               interleaved 64 gate / 64 up, so each half is two 64-row
+//               boxes), so lane i of both accumulators belongs to the same
+//               h column and SwiGLU needs no exchange between lanes.
+//   roles       as the one-CTA 128 x 256 kernel: warp 0 lane 0 loads, warps
+//               2..5 write each stage's scales into TMEM (the weights' as the
+//               A scales, the rows' as the B scales) or rescale R to R / G,
+//               warp 1 lane 0 issues the MMAs, warps 6..13 the epilogue (two
+//               per lane quarter, 64 accumulator columns = rows each).
+//   TMEM        [0, 128) half 0, [128, 256) half 1 (one buffer, handed back
+//               right after it is read); [256, 512) four scale slots of 64
+//               columns: half 0 A scales at 0, half 1 at 16, B scales at 32.
+//   correction  folded into the FP4 accumulator as (R / G) . Wc, R / G =
+//               bf16(fp32(R * fp32(1 / G))), as the 128 x 256 kernel.
+//   units       ordered expert, weight block, row block (row blocks
+//               innermost, so the CTAs that share a weight block run at the
+//               same time and all but one read it from L2).
+constexpr int kDecRowsPerUnit = 256;                  // weight rows per unit
+constexpr int kDecTok = 128;                          // expert rows per unit at most
+constexpr int kDecHalfBytes = 128 * kStageRowBytes;  // 16384
+constexpr int kDecXOff = 2 * kDecHalfBytes;           // token tile
+constexpr int kDecWsfOff = kDecXOff + kDecTok * kStageRowBytes;   // weight scale tiles (two 128-row blocks)
+constexpr int kDecXsfOff = kDecWsfOff + 2 * 4 * 512;             // token scale tile
+constexpr int kDecStageBytes = kDecXsfOff + 4 * 512;              // 55296
+constexpr int kDecWcOff = kDecTok * 128;                          // correction stage: Wc after R (64 channels)
+constexpr int kDecBox = 128;                          // rows per TMA box of the token tile
+constexpr int kDecSlots = 4;
+constexpr int kDecEpiWarps = 8;
+constexpr int kDecThreads = 448;
+
+// Shared-memory offset of 64-row weight box i (rows 64 i .. 64 i + 63 of the
+// unit) inside a stage holding the two halves one after the other, for boxes
+// of box_bytes: plain units keep the rows in order; SwiGLU units send the
+// gate boxes (0, 2) to half 0 and the up boxes (1, 3) to half 1.
+template <bool kSwiglu>
+__device__ __forceinline__ uint32_t dec_box_off(int i, uint32_t box_bytes) {
+  return kSwiglu ? (static_cast<uint32_t>(i & 1) * 2u + static_cast<uint32_t>(i >> 1)) * box_bytes
+                 : static_cast<uint32_t>(i) * box_bytes;
+}
+
+template <bool kSwiglu>
+__global__ void __launch_bounds__(kDecThreads, 1)
+    grouped_gemm_decode_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                               const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_wc,
+                               GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* const base_ptr = smem_raw + (base - raw);
+  const int S = p.stages;
+  const uint32_t bar0 = base + S * kDecStageBytes;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
+  auto sf_full = [&](int s) { return bar0 + 8u * (2 * S + s); };
+  const uint32_t acc_full = bar0 + 8u * (3 * S);
+  const uint32_t acc_empty = acc_full + 8;
+  const uint32_t drain_bar = acc_full + 16;
+  uint8_t* const misc = base_ptr + (drain_bar + 8 - base);
+  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(misc);
+  volatile int* const abort_flag = reinterpret_cast<volatile int*>(misc + 4);
+  int32_t* const off_s = reinterpret_cast<int32_t*>(misc + 16);       // E + 1, clamped to rows_cap
+  int32_t* const ub_s = off_s + p.E + 1;                                 // E + 1: first unit of each expert
+  float* const gscale_s = reinterpret_cast<float*>(ub_s + p.E + 1);     // g_a(e) * g_w[e]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    prefetch_tensormap(&tm_x);
+    prefetch_tensormap(&tm_w);
+    if (p.n_chan) {
+      prefetch_tensormap(&tm_r);
+      prefetch_tensormap(&tm_wc);
+    }
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+      mbar_init(sf_full(s), 4);                 // one arrival per scale warp
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, kDecEpiWarps);
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  const int nwb = p.N / kDecRowsPerUnit;
+  for (int i = threadIdx.x; i <= p.E; i += blockDim.x) {
+    off_s[i] = min(p.expert_off[i], p.rows_cap);
+    if (i < p.E) gscale_s[i] = __fmul_rn(p.g_a[p.g_a_per_expert ? i : 0], p.g_w[i]);
+  }
+  __syncthreads();
+  if (warp == 2) warp_block_prefix(ub_s, off_s, p.E, kDecTok, nwb, lane);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int total = ub_s[p.E];
+  const int nkb_total = p.K / 64;
+  const int nks_main = (nkb_total + 3) / 4;
+  // BF16 correction operands in boxes of cw channels (rows of 2 cw bytes, the
+  // swizzle of that width), 64 channels per stage: R [128 x cw] (one box)
+  // and Wc [256 x cw] (64-row boxes) per box column
+  const int cw = p.comp_cw, cps = 64 / cw;
+  const int rcb = kDecTok * 2 * cw, wcb = kDecRowsPerUnit * 2 * cw;
+  const int nch = p.n_chan / cw;
+  const int nks = nks_main + (nch + cps - 1) / cps;
+  const int n_col_tiles = nkb_total;
+  // unit u: expert e, its first weight row wrow (over all experts), the
+  // expert-local weight block wb, the first row row0 and the number of rows
+  auto unit_of = [&](int u, int& e, int& wrow, int& wb, int& row0, int& nrows) {
+    e = expert_of_row(ub_s, p.E, u);
+    const int ntb = (off_s[e + 1] - off_s[e] + kDecTok - 1) / kDecTok;
+    const int local = u - ub_s[e];
+    wb = local / ntb;
+    const int tb = local - wb * ntb;
+    wrow = e * p.N + wb * kDecRowsPerUnit;
+    row0 = off_s[e] + kDecTok * tb;
+    nrows = min(kDecTok, off_s[e + 1] - row0);
+  };
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ producer
+    int it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+      int e, wrow, wb, row0, nrows;
+      unit_of(u, e, wrow, wb, row0, nrows);
+      const int nbox = (nrows + kDecBox - 1) / kDecBox;   // boxes of the token tile that hold rows
+      for (int ks = 0; ks < nks; ++ks, ++it) {
+        const int s = it % S;
+        if (!mbar_wait(empty_bar(s), ((it / S) & 1) ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+        const uint32_t st = base + s * kDecStageBytes;
+        if (ks < nks_main) {
+          const int nkb = min(4, nkb_total - ks * 4);
+          mbar_expect_tx(full_bar(s), 2 * kDecHalfBytes + 3 * nkb * 512 + nbox * kDecBox * kStageRowBytes);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            tma_load_2d(st + dec_box_off<kSwiglu>(i, 64 * kStageRowBytes), &tm_w, ks * kStageRowBytes, wrow + 64 * i,
+                        full_bar(s));
+#pragma unroll
+          for (int b = 0; b < 2; ++b)
+            bulk_load(st + kDecWsfOff + b * 2048,
+                      p.w_scales + (static_cast<int64_t>(wrow / 128 + b) * n_col_tiles + ks * 4) * 512, nkb * 512,
+                      full_bar(s));
+          for (int i = 0; i < nbox; ++i)
+            tma_load_2d(st + kDecXOff + i * kDecBox * kStageRowBytes, &tm_x, ks * kStageRowBytes, row0 + kDecBox * i,
+                        full_bar(s));
+          bulk_load(st + kDecXsfOff, p.a_scales + (static_cast<int64_t>(row0 / 128) * n_col_tiles + ks * 4) * 512,
+                    nkb * 512, full_bar(s));
+        } else {
+          const int j0 = (ks - nks_main) * cps, nj = min(cps, nch - j0);
+          mbar_expect_tx(full_bar(s), nj * (wcb + nbox * kDecBox * 2 * cw));
+          for (int j = 0; j < nj; ++j) {
+            const uint32_t wc = st + kDecWcOff + j * wcb;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              tma_load_2d(wc + dec_box_off<kSwiglu>(i, 64 * 2 * cw), &tm_wc, (j0 + j) * cw, wrow + 64 * i, full_bar(s));
+            for (int i = 0; i < nbox; ++i)
+              tma_load_2d(st + j * rcb + i * kDecBox * 2 * cw, &tm_r, (j0 + j) * cw, row0 + kDecBox * i, full_bar(s));
+          }
+        }
+      }
+    }
+    if (!ok) {
+      for (int i = (it > S ? it - S : 0); i < it; ++i) mbar_wait(full_bar(i % S), (i / S) & 1, nullptr, kDrainTimeoutNs);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------------ MMA
+    int it = 0, tc = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < total && ok; u += gridDim.x, ++tc) {
+      if (!mbar_wait_cluster(acc_empty, (tc & 1) ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+      tc_fence_after();
+      for (int ks = 0; ks < nks; ++ks, ++it) {
+        const int s = it % S;
+        if (!mbar_wait_cluster(sf_full(s), (it / S) & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t st = base + s * kDecStageBytes;
+        const uint32_t slot = tmem + kPairSfCol + s * kPairSlotCols;
+        if (ks < nks_main) {
+          const int nkb = min(4, nkb_total - ks * 4);
+          for (int kb = 0; kb < nkb; ++kb) {
+            const uint64_t dx = desc_kmajor_sw128(st + kDecXOff + kb * kMmaKBytes);
+            const uint32_t acc = (ks | kb) != 0 ? 1u : 0u;
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              mma_fp4(tmem + 128 * h, desc_kmajor_sw128(st + h * kDecHalfBytes + kb * kMmaKBytes), dx, kIdescFp4,
+                      slot + 16 * h + 4 * kb, slot + 32 + 4 * kb, acc);
+          }
+        } else {
+          const int nj = min(cps, nch - (ks - nks_main) * cps);
+          for (int j = 0; j < nj; ++j)
+            for (int kk = 0; kk < cw / 16; ++kk) {      // K = 16 channels per MMA, 32 bytes along the row
+              const uint64_t dr = desc_kmajor_rows(st + j * rcb + kk * 32, 2 * cw);
+#pragma unroll
+              for (int h = 0; h < 2; ++h)
+                mma_bf16(tmem + 128 * h,
+                         desc_kmajor_rows(st + kDecWcOff + j * wcb + h * (wcb / 2) + kk * 32, 2 * cw), dr,
+                         kIdescBf16, 1u);
+            }
+        }
+        tc_commit(empty_bar(s));               // frees the stage and its scale slot
+      }
+      if (!ok) break;
+      tc_commit(acc_full);
+    }
+    if (!ok) {
+      tc_commit(drain_bar);
+      mbar_wait(drain_bar, 0, nullptr, kDrainTimeoutNs);
+    }
+  } else if (warp >= 2 && warp <= 5) {
+    // ------------------------------------- block scales / rescaled residuals
+    // Lane i of the warp for lane quarter q writes TMEM lane 32 q + i of the
+    // stage's slot: for MMA kb, column 4 kb + j of each half holds the scales
+    // of its A rows i + 32 j, and column 32 + 4 kb + j those of token rows
+    // i + 32 j.  A SwiGLU half takes rows 0..63 (gate) or 64..127 (up) of
+    // both 128-row weight blocks: words 0, 1 or 2, 3 of each block's tile.
+    const int q = warp & 3;
+    int it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+      int e, wrow, wb, row0, nrows;
+      unit_of(u, e, wrow, wb, row0, nrows);
+      const float G = gscale_s[e];
+      const float Ginv = G > 0.0f ? __frcp_rn(G) : 0.0f;     // R / G as R * fp32(1 / G)
+      const bool my_row = q * 32 + lane < (nrows + kDecBox - 1) / kDecBox * kDecBox;   // a loaded token row
+      for (int ks = 0; ks < nks; ++ks, ++it) {
+        const int s = it % S;
+        const bool w_ok = mbar_wait(full_bar(s), (it / S) & 1, abort_flag, p.timeout_ns);
+        if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t st = base + s * kDecStageBytes;
+        if (ks < nks_main) {
+          const uint32_t wsf = st + kDecWsfOff + lane * 16;
+          const uint32_t xsf = st + kDecXsfOff + lane * 16;
+          const uint32_t tsf = tmem + (static_cast<uint32_t>(q * 32) << 16) + kPairSfCol + s * kPairSlotCols;
+          uint32_t r0[16], r1[16], rx[16];
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb) {       // tiles past the stage's last K block are never read
+            const uint4 w0 = ld_shared_v4(wsf + kb * 512);
+            const uint4 w1 = ld_shared_v4(wsf + 2048 + kb * 512);
+            const uint4 x = ld_shared_v4(xsf + kb * 512);
+            if constexpr (kSwiglu) {
+              r0[4 * kb] = w0.x; r0[4 * kb + 1] = w0.y; r0[4 * kb + 2] = w1.x; r0[4 * kb + 3] = w1.y;
+              r1[4 * kb] = w0.z; r1[4 * kb + 1] = w0.w; r1[4 * kb + 2] = w1.z; r1[4 * kb + 3] = w1.w;
+            } else {
+              r0[4 * kb] = w0.x; r0[4 * kb + 1] = w0.y; r0[4 * kb + 2] = w0.z; r0[4 * kb + 3] = w0.w;
+              r1[4 * kb] = w1.x; r1[4 * kb + 1] = w1.y; r1[4 * kb + 2] = w1.z; r1[4 * kb + 3] = w1.w;
+            }
+            rx[4 * kb] = x.x; rx[4 * kb + 1] = x.y; rx[4 * kb + 2] = x.z; rx[4 * kb + 3] = x.w;
+          }
+          tmem_store16(tsf, r0);
+          tmem_store16(tsf + 16, r1);
+          tmem_store16(tsf + 32, rx);
+          tmem_wait_st();
+          tc_fence_before();
+        } else if (my_row) {
+          // R / G rounded to BF16 (as R * fp32(1 / G)), in place: this lane's
+          // token row of each box (2 cw bytes)
+          // (each lane starts at another 16-byte piece: the rows of a
+          // quarter warp then fall in distinct banks)
+          const int nj = min(cps, nch - (ks - nks_main) * cps);
+          const int units = cw / 8, rot = (q * 32 + lane) >> (cw == 64 ? 0 : (cw == 32 ? 1 : 2));
+          for (int j = 0; j < nj; ++j) {
+            const uint32_t ad = st + j * rcb + (q * 32 + lane) * 2 * cw;
+            for (int hh = 0; hh < units; ++hh) {
+              const int h = (hh + rot) & (units - 1);
+              const uint4 v = ld_shared_v4(ad + 16 * h);
+              uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float lo = __fmul_rn(bf16_bits_to_float(w[i] & 0xFFFFu), Ginv);
+                const float hi = __fmul_rn(bf16_bits_to_float(w[i] >> 16), Ginv);
+                w[i] = pack_bf16x2(lo, hi);
+              }
+              st_shared_v4(ad + 16 * h, w[0], w[1], w[2], w[3]);
+            }
+          }
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sf_full(s));
+      }
+    }
+  } else if (warp >= 6) {
+    // ----------------------------------------------------------- epilogue
+    // Warp 6 + 4 hs + i reads TMEM lane quarter q = warp % 4 (weight rows
+    // 32 q + lane of both halves) and accumulator columns [64 hs, 64 hs + 64)
+    // (token rows), 32 at a time; both halves are read and rounded before
+    // the accumulator is handed back.  Lane i stores its weight row's value
+    // for each token row: a warp writes 64 contiguous bytes per row.
+    const int q = warp & 3, hs = (warp - 6) >> 2;
+    int tc = 0;
+    for (int u = blockIdx.x; u < total; u += gridDim.x, ++tc) {
+      int e, wrow, wb, row0, nrows;
+      unit_of(u, e, wrow, wb, row0, nrows);
+      if (!mbar_wait_cluster(acc_full, tc & 1, abort_flag, p.timeout_ns)) break;
+      tc_fence_after();
+      const float G = gscale_s[e];
+      const int c0 = 64 * hs;                         // first token column of this warp
+      const int nvalid = max(0, min(64, nrows - c0)); // token rows this warp stores
+      uint32_t v0[2][16], v1[2][16];                  // BF16 pairs of consecutive token rows, per half
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        if (32 * c < nvalid) {
+          uint32_t a[32], b[32];
+          const uint32_t tacc = tmem + (static_cast<uint32_t>(q * 32) << 16) + c0 + 32 * c;
+          tmem_load32(tacc, a);
+          tmem_load32(tacc + 128, b);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            v0[c][j] = pack_bf16x2(__fmul_rn(__uint_as_float(a[2 * j]), G), __fmul_rn(__uint_as_float(a[2 * j + 1]), G));
+            v1[c][j] = pack_bf16x2(__fmul_rn(__uint_as_float(b[2 * j]), G), __fmul_rn(__uint_as_float(b[2 * j + 1]), G));
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+      const int feat = 32 * q + lane;
+      if constexpr (!kSwiglu) {
+        const int col = wb * kDecRowsPerUnit + feat;   // expert-local output column of half 0
+        uint16_t* const y0 = p.y + static_cast<int64_t>(row0 + c0) * p.N + col;
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int t = 32 * c + j;
+            if (t < nvalid) {
+              const uint32_t w0 = v0[c][j >> 1], w1 = v1[c][j >> 1];
+              y0[static_cast<int64_t>(t) * p.N] = static_cast<uint16_t>((j & 1) ? (w0 >> 16) : (w0 & 0xFFFFu));
+              y0[static_cast<int64_t>(t) * p.N + 128] = static_cast<uint16_t>((j & 1) ? (w1 >> 16) : (w1 & 0xFFFFu));
+            }
+          }
+      } else {
+        const int Fh = p.N / 2;
+        const int col = wb * (kDecRowsPerUnit / 2) + feat;   // h column
+        uint16_t* const h0 = p.y + static_cast<int64_t>(row0 + c0) * Fh + col;
+        unsigned int hmax = 0u;
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int t = 32 * c + 2 * j;
+            if (t < nvalid) {
+              const uint32_t o = swiglu_bf16x2(v0[c][j], v1[c][j]);
+              h0[static_cast<int64_t>(t) * Fh] = static_cast<uint16_t>(o & 0xFFFFu);
+              hmax = max(hmax, o & 0x7FFFu);
+              if (t + 1 < nvalid) {
+                h0[static_cast<int64_t>(t + 1) * Fh] = static_cast<uint16_t>(o >> 16);
+                hmax = max(hmax, (o >> 16) & 0x7FFFu);
+              }
+            }
+          }
+        hmax = __reduce_max_sync(0xffffffffu, hmax);
+        if (lane == 0 && hmax != 0u && p.amax_bits != nullptr) atomicMax(&p.amax_bits[e], hmax << 16);
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
 // Per-expert amax for the FP4 compensation's residual:
 // amax_r[e] = fp32(fp32(G_e / g_wc[e]) * 2688), G_e = fp32(g_a g_w[e]); the
 // residual's decode scale times g_wc[e] is then G_e up to one rounding.
@@ -1460,6 +1893,15 @@ int make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return set_error(QUADS_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
   return QUADS_OK;
+}
+
+// Channels per box of the wide and decode tiles' BF16 correction operands:
+// the widest of 64, 32, 16 that divides n_chan (rows of 128, 64 or 32 bytes:
+// fewer, longer rows per TMA copy).
+int comp_box_channels(int n_chan) { return n_chan % 64 == 0 ? 64 : (n_chan % 32 == 0 ? 32 : 16); }
+CUtensorMapSwizzle swizzle_of_row(int row_bytes) {
+  return row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                          : (row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
 }
 
 // extra_words: the quantizing epilogue's tables (E + n_chan_h + N / 64 + 1)
@@ -1556,11 +1998,12 @@ int launch_gemm_pair(const uint8_t* a_codes, const uint8_t* a_scales, const floa
                         CU_TENSOR_MAP_SWIZZLE_128B));
   QUADS_TRY(make_map_2d(&tm_b, w_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, E * N, kStageRowBytes, wrows,
                         CU_TENSOR_MAP_SWIZZLE_128B));
+  const int cw = comp_box_channels(n_chan);
   if (n_chan) {
-    QUADS_TRY(make_map_2d(&tm_r, a_resid, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, n_chan, rows_cap, 16, 128,
-                          CU_TENSOR_MAP_SWIZZLE_32B));
-    QUADS_TRY(make_map_2d(&tm_wc, w_resid, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, n_chan, E * N, 16, wrows,
-                          CU_TENSOR_MAP_SWIZZLE_32B));
+    QUADS_TRY(make_map_2d(&tm_r, a_resid, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, n_chan, rows_cap, cw, 128,
+                          swizzle_of_row(2 * cw)));
+    QUADS_TRY(make_map_2d(&tm_wc, w_resid, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, n_chan, E * N, cw, wrows,
+                          swizzle_of_row(2 * cw)));
   } else {
     tm_r = tm_a;
     tm_wc = tm_a;
@@ -1601,6 +2044,7 @@ int launch_gemm_pair(const uint8_t* a_codes, const uint8_t* a_scales, const floa
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
   p.n_chan = n_chan;
+  p.comp_cw = cw;
   p.stages = stages;
   p.timeout_ns = kGemmTimeoutNs;
   // at most one tile per 128 rows and 256 columns
@@ -1630,6 +2074,78 @@ int launch_gemm_pair(const uint8_t* a_codes, const uint8_t* a_scales, const floa
   }
   count_launches(1);
   return check_launch("grouped_gemm_pair_kernel");
+}
+
+// Average rows per expert at or below which the FP4 GEMMs with the BF16
+// correction (or none), N % 256 == 0 and no fused quantization take the
+// decode kernel (quads_gemm_set_decode_rows); 0: never.
+int g_decode_rows = 64;
+
+bool decode_selected(int64_t rows_cap, int E) {
+  if (g_decode_rows <= 0) return false;
+  const int64_t blocks = rows_cap / 128 - E;       // 128-row blocks beyond one padding block per expert
+  const int64_t avg = (blocks > 0 ? blocks : 0) * 128 / E;
+  return avg <= g_decode_rows;
+}
+
+size_t decode_smem_bytes(int stages, int E) {
+  return 1024 + static_cast<size_t>(stages) * kDecStageBytes + static_cast<size_t>(3 * stages + 3) * 8 + 16 +
+         static_cast<size_t>(3 * E + 2) * 4;
+}
+
+template <bool kSwiglu>
+int launch_gemm_decode(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_a, int g_a_per_expert,
+                       const uint8_t* w_codes, const uint8_t* w_scales, const float* g_w, const int32_t* expert_off,
+                       int E, int64_t rows_cap, int64_t N, int64_t K, const uint16_t* a_resid, const uint16_t* w_resid,
+                       int n_chan, uint16_t* y, float* amax_out, cudaStream_t stream) {
+  CUtensorMap tm_x, tm_w, tm_r, tm_wc;
+  QUADS_TRY(make_map_2d(&tm_x, a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, rows_cap, kStageRowBytes, kDecBox,
+                        CU_TENSOR_MAP_SWIZZLE_128B));
+  QUADS_TRY(make_map_2d(&tm_w, w_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, E * N, kStageRowBytes, 64,
+                        CU_TENSOR_MAP_SWIZZLE_128B));
+  const int cw = comp_box_channels(n_chan);
+  if (n_chan) {
+    QUADS_TRY(make_map_2d(&tm_r, a_resid, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, n_chan, rows_cap, cw, kDecBox,
+                          swizzle_of_row(2 * cw)));
+    QUADS_TRY(make_map_2d(&tm_wc, w_resid, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, n_chan, E * N, cw, 64,
+                          swizzle_of_row(2 * cw)));
+  } else {
+    tm_r = tm_x;
+    tm_wc = tm_x;
+  }
+  const size_t smem_cap = 232448;
+  int stages = kDecSlots;
+  while (stages >= 2 && decode_smem_bytes(stages, E) > smem_cap) --stages;
+  QUADS_REQUIRE(stages >= 2, QUADS_ERR_UNSUPPORTED_SHAPE, "not enough shared memory for two stages");
+  const size_t smem = decode_smem_bytes(stages, E);
+  auto kernel = grouped_gemm_decode_kernel<kSwiglu>;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+      cudaSuccess)
+    return set_error(QUADS_ERR_CUDA, "cannot set %zu bytes of shared memory", smem);
+  GemmParams p{};
+  p.a_scales = a_scales;
+  p.w_scales = w_scales;
+  p.g_a = g_a;
+  p.g_w = g_w;
+  p.expert_off = expert_off;
+  p.y = y;
+  p.amax_bits = reinterpret_cast<unsigned int*>(amax_out);
+  p.g_a_per_expert = g_a_per_expert ? 1 : 0;
+  p.E = E;
+  p.rows_cap = static_cast<int>(rows_cap);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.n_chan = n_chan;
+  p.comp_cw = cw;
+  p.stages = stages;
+  p.timeout_ns = kGemmTimeoutNs;
+  // at most one unit per 128 rows (segments are 128-aligned) and 256 weight rows
+  const int64_t max_units = (rows_cap / kDecTok) * (N / kDecRowsPerUnit);
+  int64_t grid = num_sms();
+  if (grid > max_units) grid = max_units;
+  kernel<<<static_cast<unsigned>(grid), kDecThreads, smem, stream>>>(tm_x, tm_w, tm_r, tm_wc, p);
+  count_launches(1);
+  return check_launch("grouped_gemm_decode_kernel");
 }
 
 template <bool kSwiglu, bool kQuant = false, bool kW4A16 = false, int kBN = BN>
@@ -1675,6 +2191,11 @@ int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_
   if (kSwiglu && amax_out && cudaMemsetAsync(amax_out, 0, sizeof(float) * E, stream) != cudaSuccess)
     return set_error(QUADS_ERR_CUDA, "memset of amax_out failed");
   if (rows_cap == 0) return QUADS_OK;
+  if constexpr (!kW4A16 && kBN == BN && !kQuant) {
+    if (fc == nullptr && N % kDecRowsPerUnit == 0 && decode_selected(rows_cap, E))
+      return launch_gemm_decode<kSwiglu>(a_codes, a_scales, g_a, g_a_per_expert, w_codes, w_scales, g_w, expert_off,
+                                         E, rows_cap, N, K, a_resid, w_resid, n_chan, y, amax_out, stream);
+  }
   if constexpr (!kW4A16 && kBN == BN) {
     if (fc == nullptr && g_tile_shape != 0 && N % PBN == 0) {
       if (g_tile_shape == 2)
@@ -1756,6 +2277,7 @@ int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
   p.n_chan = n_chan;
+  p.comp_cw = 16;                                 // this kernel's correction boxes are 16 channels wide
   p.stages = stages;
   p.timeout_ns = kGemmTimeoutNs;
   const int64_t max_tiles = (rows_cap / BM) * (N / kBN);
@@ -1879,6 +2401,14 @@ int quads_gemm_set_tile_shape(int shape) {
   QUADS_REQUIRE(shape >= 0 && shape <= 2, QUADS_ERR_INVALID_ARG, "tile shape must be 0, 1 or 2");
   const int prev = g_tile_shape;
   g_tile_shape = shape;
+  return prev;
+}
+
+int quads_gemm_set_decode_rows(int rows) {
+  clear_error();
+  QUADS_REQUIRE(rows >= 0, QUADS_ERR_INVALID_ARG, "decode rows must be >= 0");
+  const int prev = g_decode_rows;
+  g_decode_rows = rows;
   return prev;
 }
 
