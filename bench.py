@@ -358,7 +358,7 @@ def trainer_gemm_timing(layer, dev, peaks, reps=20):
 
 def _timed_flushed(fn, flush, reps=20):
     """Median device time (ms) of the launches fn() makes, L2 flushed (a
-    write of a buffer larger than L2) before each.  The flush, two timing
+    write of a buffer larger than L2, then a read of it) before each.  The flush, two timing
     events and fn are captured once in a CUDA graph (the events as external
     event nodes, re-recorded at every replay), so the interval is the
     kernels' own time as they run inside a step's graph: neither the host
@@ -371,8 +371,14 @@ def _timed_flushed(fn, flush, reps=20):
     graph = torch.cuda.CUDAGraph()
     e0 = torch.cuda.Event(enable_timing=True, external=True)
     e1 = torch.cuda.Event(enable_timing=True, external=True)
+    words = flush.view(torch.int32)
+    acc = torch.empty((), dtype=torch.int32, device=flush.device)
     with torch.cuda.graph(graph):
         flush.zero_()
+        # then a read of the same buffer: its dirty lines are written back
+        # here rather than during the timed kernel, which finds only clean,
+        # unrelated lines in L2
+        torch.sum(words, dim=0, out=acc)
         e0.record()
         fn()
         e1.record()
