@@ -61,6 +61,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sweep", action="store_true", help="skip the standalone quantize/replay size sweep")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the other workloads (single linear, 2048-token layer step, 8-layer alignment pass)")
     ap.add_argument("--serial", action="store_true", help="run the step on one stream (no weight-side overlap)")
     ap.add_argument("--comp", choices=["bf16", "fp4"], default="bf16",
                     help="compensation: BF16 R . Wc (default) or the NVFP4 second pass")
@@ -406,6 +408,95 @@ def _gemm_calls(layer, comp=True):
         layer.h_codes, layer.h_scales, layer.g_h, layer.w_d_codes, layer.w_d_scales, layer.g_w_d, layer.expert_off,
         E, layer.cap, H, F, layer.h_resid if comp else None, layer.wc_d if comp else None, y=layer.y_d)
     return gu, dn
+
+
+def secondary_workloads(dev, peaks, fp4_peak, steps=20):
+    """The other workloads, each timed on its own after the headline (L2
+    flushed before each timed run): the single NVFP4 linear (64 x 256 x 512,
+    8 compensation channels: quantize x + the GEMM, the weights quantized
+    once beforehand), one step of the 2048-token layer (the whole path, one
+    CUDA graph per step, as the headline step), and one train/rollout
+    alignment pass of the 8-layer stack (rollout of all 8 layers with the
+    last 4 recorded, then the trainer with those 4 replayed), host-launched,
+    with its per-token output gap (unpinned)."""
+    import torch
+    from train_alignment_b200 import binding as B
+    from train_alignment_b200 import layer as L
+    from train_alignment_b200 import stack as ST
+    from train_alignment_b200 import workloads as W
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    out = {}
+    # single NVFP4 linear
+    lc = W.LINEAR_64x256x512
+    li = W.linear_inputs(lc, seed=0, device=dev)
+    xt = torch.zeros(128, lc.K, dtype=torch.bfloat16, device=dev)
+    xt[:lc.M] = li["x"]
+    chan = torch.full((16,), -1, dtype=torch.int32, device=dev)   # 8 channels, padded to the GEMM's 16
+    chan[:lc.n_chan] = B.select_channels(B.channel_scores(xt[:lc.M]), lc.n_chan)
+    _, w_codes, w_scales, g_w, w_chan = B.fakequant_weight_ste(li["w"][None].contiguous(), chan=chan)
+    off = torch.tensor([0, 128], dtype=torch.int32, device=dev)
+    amax = torch.empty(1, dtype=torch.float32, device=dev)
+    codes = torch.empty(128, lc.K // 2, dtype=torch.uint8, device=dev)
+    scales = torch.empty(B.scales_bytes(128, lc.K, B.SCALES_TILED), dtype=torch.uint8, device=dev)
+    g = torch.empty(1, dtype=torch.float32, device=dev)
+    resid = torch.empty(128, chan.numel(), dtype=torch.bfloat16, device=dev)
+    y = torch.empty(128, lc.N, dtype=torch.bfloat16, device=dev)
+
+    def linear():
+        B.amax_bf16(xt, out=amax)
+        B.quantize_nvfp4(xt, amax_in=amax, scale_layout=B.SCALES_TILED, chan=chan, codes=codes, scales=scales,
+                         g_out=g, resid_out=resid)
+        B.moe_grouped_gemm_nvfp4(codes, scales, g, w_codes, w_scales, g_w, off, 1, 128, lc.N, lc.K, resid, w_chan,
+                                 y=y)
+    t = _timed_flushed(linear, flush) * 1e3
+    flop = 2.0 * lc.M * lc.N * (lc.K + lc.n_chan)
+    out[lc.name] = {"us": t, "TFLOP/s": flop / (t * 1e-6) / 1e12, "launches": 3,
+                    "what": "amax + quantize x (codes, tiled scales, 8 residual channels) + the grouped GEMM"}
+    assert B.device_status() == B.OK, B.last_error()
+    # one step of the 2048-token layer
+    cfg = W.CONFIGS["moe_t2048_h1024_e8k2_f2048"]
+    inp = W.moe_layer_inputs(cfg, seed=0, device=dev)
+    ly = L.build_layer(cfg, inp, dev)
+    x_train = W.engine_drift(inp["x"], 1e-2, seed=0, device=dev)
+    _, g_gu, g_d = ly.grad_fq_buffers()
+    g_gu.copy_(W.random_bf16(ly.w_gu.shape, 100, 1e-3, dev))
+    g_d.copy_(W.random_bf16(ly.w_d.shape, 200, 1e-3, dev))
+    step = lambda: ly.step(inp["x"], inp["logits"], x_train, g_gu, g_d)
+    for _ in range(3):
+        step()
+    ms = _timed_flushed(step, flush, steps)
+    fp4, comp = gemm_flops(cfg)
+    out[cfg.name] = {"ms_per_step": ms, "TFLOP/s": (fp4 + comp) / (ms * 1e-3) / 1e12,
+                     "what": "the whole step (rollout layer, TRACE export, trainer replay, weight fake-quant and "
+                             "STE backward), one CUDA graph"}
+    assert B.device_status() == B.OK, B.last_error()
+    del ly, inp, x_train, g_gu, g_d
+    torch.cuda.empty_cache()
+    # the 8-layer alignment pass
+    scfg = W.CONFIGS["stack8_t4096_h2048_e64k4_f1024"]
+    st = ST.LayerStack(scfg, seed=0, device=dev)
+    st.alignment_pass(drift=1e-3)
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(3):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        gap, cm, sm = st.alignment_pass(drift=1e-3)
+        e1.record()
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    assert B.device_status() == B.OK, B.last_error()
+    gp = gap.float()
+    out[scfg.name] = {"ms_per_pass": statistics.median(ts), "tokens_per_s": scfg.T / (statistics.median(ts) * 1e-3),
+                      "per_token_gap": {"median": float(gp.median()), "p90": float(gp.quantile(0.9)),
+                                        "max": float(gp.max()), "pinned": False},
+                      "replayed_layer_mismatches": {"codes": int(cm), "scales": int(sm)},
+                      "what": "rollout of 8 layers (last 4 recorded) + trainer with the 4 records replayed; "
+                              "host-launched, events around the pass"}
+    del st
+    torch.cuda.empty_cache()
+    return out
 
 
 def gemm_side_measurements(layer, dev, peaks):
@@ -921,6 +1012,12 @@ def run_ours(args):
         sweep = quantize_replay_sweep(dev, peaks["hbm_gbs"])
     trainer = trainer_gemm_timing(layer, dev, peaks) if not args.no_sweep else None
     gemm_side = gemm_side_measurements(layer, dev, peaks) if not args.no_sweep and layer.comp == "bf16" else None
+    secondary = None
+    if not args.no_secondary and world == 1:
+        try:
+            secondary = secondary_workloads(dev, peaks, fp4_peak)
+        except Exception as exc:  # noqa: BLE001 -- reported, the headline stands
+            secondary = {"error": f"{type(exc).__name__}: {str(exc)[:200]}"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -965,6 +1062,7 @@ def run_ours(args):
         "quantize_replay_sweep": sweep,
         "trainer_gemm": trainer,
         "gemm_side": gemm_side,
+        "secondary_workloads": secondary,
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)
