@@ -187,6 +187,13 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
       : "memory");
 }
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                "l"(src), "r"(bytes), "r"(bar)
@@ -1465,12 +1472,13 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 // zeros or belong to the next segment and only feed accumulator columns
 // that are never stored).
 //
-//   halves      plain: weight rows [0, 128) and [128, 256) of the unit.
-//               kSwiglu: the unit covers 128 h columns; half 0 holds their
-//               128 gate rows and half 1 the 128 up rows (weight rows are
-//               interleaved 64 gate / 64 up, so each half is two 64-row
-//               boxes), so lane i of both accumulators belongs to the same
-//               h column and SwiGLU needs no exchange between lanes.
+//   halves      plain: weight rows [0, 128) and [128, 256) of the unit
+//               (one 256-row box).  kSwiglu: the unit covers 128 h columns;
+//               half 0 holds their 128 gate rows and half 1 the 128 up rows
+//               (weight rows are interleaved 64 gate / 64 up, so each half
+//               is rows 0-63 or 64-127 of the unit's two 128-row blocks,
+//               one 3D box), so lane i of both accumulators belongs to the
+//               same h column and SwiGLU needs no exchange between lanes.
 //   roles       as the one-CTA 128 x 256 kernel: warp 0 lane 0 loads, warps
 //               2..5 write each stage's scales into TMEM (the weights' as the
 //               A scales, the rows' as the B scales) or rescale R to R / G,
@@ -1496,16 +1504,6 @@ constexpr int kDecBox = 128;                          // rows per TMA box of the
 constexpr int kDecSlots = 4;
 constexpr int kDecEpiWarps = 8;
 constexpr int kDecThreads = 448;
-
-// Shared-memory offset of 64-row weight box i (rows 64 i .. 64 i + 63 of the
-// unit) inside a stage holding the two halves one after the other, for boxes
-// of box_bytes: plain units keep the rows in order; SwiGLU units send the
-// gate boxes (0, 2) to half 0 and the up boxes (1, 3) to half 1.
-template <bool kSwiglu>
-__device__ __forceinline__ uint32_t dec_box_off(int i, uint32_t box_bytes) {
-  return kSwiglu ? (static_cast<uint32_t>(i & 1) * 2u + static_cast<uint32_t>(i >> 1)) * box_bytes
-                 : static_cast<uint32_t>(i) * box_bytes;
-}
 
 template <bool kSwiglu>
 __global__ void __launch_bounds__(kDecThreads, 1)
@@ -1605,10 +1603,14 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         if (ks < nks_main) {
           const int nkb = min(4, nkb_total - ks * 4);
           mbar_expect_tx(full_bar(s), 2 * kDecHalfBytes + 3 * nkb * 512 + nbox * kDecBox * kStageRowBytes);
+          if constexpr (kSwiglu) {
+            // half h: rows 64 h .. 64 h + 63 of both 128-row blocks, one 3D box
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            tma_load_2d(st + dec_box_off<kSwiglu>(i, 64 * kStageRowBytes), &tm_w, ks * kStageRowBytes, wrow + 64 * i,
-                        full_bar(s));
+            for (int h = 0; h < 2; ++h)
+              tma_load_3d(st + h * kDecHalfBytes, &tm_w, ks * kStageRowBytes, 64 * h, wrow / 128, full_bar(s));
+          } else {
+            tma_load_2d(st, &tm_w, ks * kStageRowBytes, wrow, full_bar(s));     // 256 rows
+          }
 #pragma unroll
           for (int b = 0; b < 2; ++b)
             bulk_load(st + kDecWsfOff + b * 2048,
@@ -1624,9 +1626,13 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           mbar_expect_tx(full_bar(s), nj * (wcb + nbox * kDecBox * 2 * cw));
           for (int j = 0; j < nj; ++j) {
             const uint32_t wc = st + kDecWcOff + j * wcb;
+            if constexpr (kSwiglu) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              tma_load_2d(wc + dec_box_off<kSwiglu>(i, 64 * 2 * cw), &tm_wc, (j0 + j) * cw, wrow + 64 * i, full_bar(s));
+              for (int h = 0; h < 2; ++h)
+                tma_load_3d(wc + h * (wcb / 2), &tm_wc, (j0 + j) * cw, 64 * h, wrow / 128, full_bar(s));
+            } else {
+              tma_load_2d(wc, &tm_wc, (j0 + j) * cw, wrow, full_bar(s));
+            }
             for (int i = 0; i < nbox; ++i)
               tma_load_2d(st + j * rcb + i * kDecBox * 2 * cw, &tm_r, (j0 + j) * cw, row0 + kDecBox * i, full_bar(s));
           }
@@ -1895,6 +1901,23 @@ int make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64
   return QUADS_OK;
 }
 
+// A 3D map over rows of `inner` elements grouped in blocks of 128 rows:
+// dims (inner, 128 rows, blocks), box (box_inner, box_rows, box_blocks).
+int make_map_3d_blocks(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t elem_bytes, uint64_t inner,
+                       uint64_t rows, uint32_t box_inner, uint32_t box_rows, uint32_t box_blocks,
+                       CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return set_error(QUADS_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[3] = {inner, 128, rows / 128};
+  cuuint64_t strides[2] = {inner * elem_bytes, 128 * inner * elem_bytes};
+  cuuint32_t box[3] = {box_inner, box_rows, box_blocks};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return set_error(QUADS_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return QUADS_OK;
+}
+
 // Channels per box of the wide and decode tiles' BF16 correction operands:
 // the widest of 64, 32, 16 that divides n_chan (rows of 128, 64 or 32 bytes:
 // fewer, longer rows per TMA copy).
@@ -2101,14 +2124,24 @@ int launch_gemm_decode(const uint8_t* a_codes, const uint8_t* a_scales, const fl
   CUtensorMap tm_x, tm_w, tm_r, tm_wc;
   QUADS_TRY(make_map_2d(&tm_x, a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, rows_cap, kStageRowBytes, kDecBox,
                         CU_TENSOR_MAP_SWIZZLE_128B));
-  QUADS_TRY(make_map_2d(&tm_w, w_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, E * N, kStageRowBytes, 64,
-                        CU_TENSOR_MAP_SWIZZLE_128B));
+  // weights: SwiGLU, the 64 gate (or up) rows of both 128-row blocks of a
+  // unit in one 3D box; plain, the unit's 256 rows in one box
+  if (kSwiglu)
+    QUADS_TRY(make_map_3d_blocks(&tm_w, w_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, E * N, kStageRowBytes, 64, 2,
+                                 CU_TENSOR_MAP_SWIZZLE_128B));
+  else
+    QUADS_TRY(make_map_2d(&tm_w, w_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, E * N, kStageRowBytes, 256,
+                          CU_TENSOR_MAP_SWIZZLE_128B));
   const int cw = comp_box_channels(n_chan);
   if (n_chan) {
     QUADS_TRY(make_map_2d(&tm_r, a_resid, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, n_chan, rows_cap, cw, kDecBox,
                           swizzle_of_row(2 * cw)));
-    QUADS_TRY(make_map_2d(&tm_wc, w_resid, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, n_chan, E * N, cw, 64,
-                          swizzle_of_row(2 * cw)));
+    if (kSwiglu)
+      QUADS_TRY(make_map_3d_blocks(&tm_wc, w_resid, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, n_chan, E * N, cw, 64, 2,
+                                   swizzle_of_row(2 * cw)));
+    else
+      QUADS_TRY(make_map_2d(&tm_wc, w_resid, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, n_chan, E * N, cw, 256,
+                            swizzle_of_row(2 * cw)));
   } else {
     tm_r = tm_x;
     tm_wc = tm_x;
