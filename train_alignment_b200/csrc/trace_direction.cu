@@ -26,6 +26,15 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kMaxGroups = 1024;
 constexpr int kMaxChan = 256;
+// Up to this many groups, the {S, 1/S} pair of every E4M3 scale code of each
+// group (S = fp32(val(s) g)) is tabulated in shared memory once per block
+// instead of being computed (an E4M3 decode and a reciprocal) per block of
+// 16 elements.
+constexpr int kDirTabGroups = 16;
+
+size_t dir_tab_bytes(int n_groups) {
+  return n_groups <= kDirTabGroups ? static_cast<size_t>(n_groups) * 128 * sizeof(float2) : 0;
+}
 
 struct DirArgs {
   const uint16_t* x;          // rollout input (bits) or trainer input (replay)
@@ -57,22 +66,28 @@ __device__ __forceinline__ uint32_t floor_level(float v) {
   return t >= 2 ? static_cast<uint32_t>(min(t, 7)) : static_cast<uint32_t>(t >= 0);
 }
 
-// Shared-memory group table; returns the number of rows that belong to a group.
-__device__ __forceinline__ int64_t load_groups(const DirArgs& a, int32_t* off_s, float* g_s) {
+// Shared-memory group table (and, for few groups, the scale table tab);
+// returns the number of rows that belong to a group.
+__device__ __forceinline__ int64_t load_groups(const DirArgs& a, int32_t* off_s, float* g_s, float2* tab) {
   const int n = a.n_groups;
   for (int i = threadIdx.x; i <= n; i += blockDim.x) {
     off_s[i] = a.group_off ? a.group_off[i] : 0;
     if (i < n) g_s[i] = a.g[i];
   }
+  if (n <= kDirTabGroups)
+    for (int i = threadIdx.x; i < n * 128; i += blockDim.x) tab[i] = scale_table_entry(i & 127, a.g[i >> 7]);
   __syncthreads();
   return a.group_off ? min(a.rows, static_cast<int64_t>(off_s[n])) : a.rows;
 }
 
 __global__ void __launch_bounds__(kThreads, 4) direction_bits_kernel(DirArgs a) {
-  extern __shared__ int32_t smem[];
+  extern __shared__ float2 smem_tab[];
+  const bool use_tab = a.n_groups <= kDirTabGroups;
+  float2* tab = smem_tab;                                          // n x 128 {S, 1/S} (few groups)
+  int32_t* smem = reinterpret_cast<int32_t*>(smem_tab + (use_tab ? a.n_groups * 128 : 0));
   int32_t* off_s = smem;
   float* g_s = reinterpret_cast<float*>(smem + a.n_groups + 1);
-  const int64_t rows = load_groups(a, off_s, g_s);
+  const int64_t rows = load_groups(a, off_s, g_s, tab);
   const RowGroups grp{a.group_off ? off_s : nullptr, a.n_groups, a.uniform};
   const int64_t K = a.K;
   const int nkb = static_cast<int>(K / 16);
@@ -81,7 +96,9 @@ __global__ void __launch_bounds__(kThreads, 4) direction_bits_kernel(DirArgs a) 
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
        row += warps) {
-    const float g = g_s[grp.of(row)];
+    const int gi = grp.of(row);
+    const float g = g_s[gi];
+    const float2* tab_g = tab + gi * 128;
     for (int kb0 = lane; kb0 < nkb; kb0 += 64) {
       // both blocks' loads first: two 32-byte rows of x in flight per lane
       uint32_t w[2][8], sc[2];
@@ -99,7 +116,7 @@ __global__ void __launch_bounds__(kThreads, 4) direction_bits_kernel(DirArgs a) 
       for (int u = 0; u < 2; ++u) {
         const int kb = kb0 + 32 * u;
         if (kb >= nkb) break;
-        const float2 e = scale_table_entry(sc[u], g);
+        const float2 e = use_tab ? tab_g[sc[u] & 127u] : scale_table_entry(sc[u], g);
         uint32_t out = 0;
         if (e.x != 0.0f) {
           // level nibbles F of 8 elements per word, then per nibble
@@ -129,8 +146,11 @@ __global__ void __launch_bounds__(kThreads, 4) direction_bits_kernel(DirArgs a) 
 }
 
 __global__ void __launch_bounds__(kThreads, 3) replay_direction_kernel(DirArgs a) {
-  extern __shared__ int32_t smem[];
+  extern __shared__ float2 smem_tab[];
   const int n = a.n_groups;
+  const bool use_tab = n <= kDirTabGroups;
+  float2* tab = smem_tab;                                          // n x 128 {S, 1/S} (few groups)
+  int32_t* smem = reinterpret_cast<int32_t*>(smem_tab + (use_tab ? n * 128 : 0));
   const int64_t K = a.K;
   const int nkb = static_cast<int>(K / 16);
   const int npass = (nkb + 31) / 32;
@@ -145,7 +165,7 @@ __global__ void __launch_bounds__(kThreads, 3) replay_direction_kernel(DirArgs a
     for (int j = 0; j < a.n_chan; ++j) cnt += (chan_s[j] >= 0 && chan_s[j] < K && chan_s[j] < 512 * p) ? 1 : 0;
     pass_slot[p] = cnt;
   }
-  const int64_t rows = load_groups(a, off_s, g_s);
+  const int64_t rows = load_groups(a, off_s, g_s, tab);
   const RowGroups grp{a.group_off ? off_s : nullptr, n, a.uniform};
   const int64_t ncol_tiles = ceil_div(nkb, 4);
   const int lane = threadIdx.x & 31;
@@ -153,7 +173,9 @@ __global__ void __launch_bounds__(kThreads, 3) replay_direction_kernel(DirArgs a
   uint32_t fixes = 0;
   for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
        row += warps) {
-    const float g = g_s[grp.of(row)];
+    const int gi = grp.of(row);
+    const float g = g_s[gi];
+    const float2* tab_g = tab + gi * 128;
     for (int p0 = 0; p0 < npass; p0 += 2) {
       // both passes' loads first: two 32-byte rows of x_train in flight per lane
       uint32_t wx[2][8], sx[2], bx[2];
@@ -174,7 +196,7 @@ __global__ void __launch_bounds__(kThreads, 3) replay_direction_kernel(DirArgs a
         QCore q{0u, 0u, 0u, 0.0f};
         if (kb < nkb) {
           const uint32_t s = sx[u];
-          const float2 e = scale_table_entry(s, g);
+          const float2 e = use_tab ? tab_g[s & 127u] : scale_table_entry(s, g);
           const uint32_t bits = bx[u];
           const uint32_t (&w)[8] = wx[u];
           q.scale = s;
@@ -279,7 +301,7 @@ int trace_direction_bits(const uint16_t* x, int64_t rows, int64_t K, const uint8
   a.x = x;
   a.codes = codes;
   a.bits = bits;
-  const size_t smem = (2 * static_cast<size_t>(n_groups) + 1) * 4;
+  const size_t smem = dir_tab_bytes(n_groups) + (2 * static_cast<size_t>(n_groups) + 1) * 4;
   const int grid = persistent_grid(reinterpret_cast<const void*>(direction_bits_kernel), kThreads, smem,
                                    ceil_div(rows, kThreads / 32));
   direction_bits_kernel<<<grid, kThreads, smem, stream>>>(a);
@@ -309,7 +331,8 @@ int trace_replay_direction(const uint8_t* bits, const uint8_t* scales, int scale
   a.x_hat = x_hat;
   a.codes_out = codes_out;
   a.corrections = corrections;
-  const size_t smem = (2 * static_cast<size_t>(n_groups) + 1 + (K / 16 + 31) / 32 + 1 + n_chan) * 4;
+  const size_t smem =
+      dir_tab_bytes(n_groups) + (2 * static_cast<size_t>(n_groups) + 1 + (K / 16 + 31) / 32 + 1 + n_chan) * 4;
   if (smem > 48 * 1024 && cudaFuncSetAttribute(replay_direction_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                static_cast<int>(smem)) != cudaSuccess)
     return set_error(QUADS_ERR_CUDA, "cannot raise shared memory of replay_direction_kernel");
