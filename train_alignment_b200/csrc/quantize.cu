@@ -190,6 +190,12 @@ struct QuantArgs {
 // kMode: 0 any combination of outputs (runtime checks); 1 the weight
 // fake-quant (codes, scales, W_fq with g folded, compensation columns as
 // bf16(deq)); 2 the activation quantizer (codes, scales, residual channels).
+// Eight words to 32-byte aligned shared memory.
+__device__ __forceinline__ void st_shared_u32x8(uint32_t* p, const uint32_t (&o)[8]) {
+  reinterpret_cast<uint4*>(p)[0] = make_uint4(o[0], o[1], o[2], o[3]);
+  reinterpret_cast<uint4*>(p)[1] = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
 template <int kMode>
 __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a) {
   constexpr bool kFq = kMode == 1, kAct = kMode == 2;
@@ -199,6 +205,9 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a) {
   const int fold = kFq ? 1 : a.fold;
   const int resid_mode = kFq ? 1 : (kAct ? 0 : a.resid_mode);
   extern __shared__ int32_t smem_q[];
+  // weight fake-quant: each warp's W_fq words of the current pass (32 lanes x
+  // 8 words), from which the compensation columns are picked
+  __shared__ __align__(16) uint32_t wfq_s[kFq ? (kThreads / 32) * 32 * 8 : 4];
   const int n = a.n_groups;
   const int nkb = static_cast<int>(a.K / 16);
   const int npass = (nkb + 31) / 32;
@@ -284,12 +293,12 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a) {
         if (p >= npass) break;                         // warp-uniform
         const int kb = p * 32 + lane;
         QCore q{0u, 0u, 0u, 0.0f};
+        uint32_t o[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
         if (kb < nkb) {
           q = quant_core(w[u], qc);
           if (has_codes)
             *reinterpret_cast<uint2*>(a.codes + drow * (a.K / 2) + kb * 8) = make_uint2(q.lo, q.hi);
           if (has_wfq) {
-            uint32_t o[8];
             deq_block_bf16(q, g, fold, o);
             uint4* dst = reinterpret_cast<uint4*>(a.w_fq + row * a.K + kb * 16);
             dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
@@ -298,7 +307,27 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a) {
         }
         if (has_scales && kb < nkb_e)
           a.scales[sbase + (tiled ? (kb >> 2) * 512 + (kb & 3) : kb)] = static_cast<uint8_t>(q.scale);
-        if (a.resid) {
+        if (kFq && a.resid) {
+          // The compensation column of channel c is W_fq[:, c] itself (the
+          // fold makes bf16(deq) the W_fq value): the warp stages its W_fq
+          // words of the pass and channel slot j takes lane j % 32, which
+          // picks its element there.
+          const int slo = pass_slot[p], shi = pass_slot[p + 1];
+          if (slo < shi) {                                 // warp-uniform
+            uint32_t* const ws = wfq_s + (threadIdx.x >> 5) * 256;
+            st_shared_u32x8(ws + lane * 8, o);
+            __syncwarp();
+            for (int j0 = slo; j0 < shi; j0 += 32) {
+              const int j = j0 + lane;
+              if (j < shi) {
+                const int c = chan_s[j] - 512 * p;
+                const uint32_t word = ws[(c >> 4) * 8 + ((c & 15) >> 1)];
+                a.resid[drow * a.n_chan + j] = static_cast<uint16_t>((c & 1) ? (word >> 16) : (word & 0xFFFFu));
+              }
+            }
+            __syncwarp();
+          }
+        } else if (a.resid) {
           // Channel slot j of this pass is taken by lane j % 32: the element's
           // code and block scale come from the owning lane by shuffles (the
           // input element, where needed, is read back through L2).
