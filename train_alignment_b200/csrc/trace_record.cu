@@ -93,7 +93,12 @@ __device__ bool record_ok(const ReplayArgs& a, const trace_qrecord_header& h) {
   return true;
 }
 
-__global__ void __launch_bounds__(kThreads, 3) replay_kernel(ReplayArgs a) {
+// kTrain: a trainer input is compared (x_train given); without one the lane
+// loads the codes and scales of four passes at a time instead of two (the
+// loop is latency-bound: a block's loads are only 9 bytes per lane).
+template <bool kTrain>
+__global__ void __launch_bounds__(kThreads, kTrain ? 3 : 4) replay_kernel(ReplayArgs a) {
+  constexpr int kU = kTrain ? 2 : 4;                        // passes whose loads are in flight at once
   extern __shared__ int32_t smem[];
   __shared__ trace_qrecord_header h;
   __shared__ int ok;
@@ -147,57 +152,86 @@ __global__ void __launch_bounds__(kThreads, 3) replay_kernel(ReplayArgs a) {
   const int lane = threadIdx.x & 31;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   unsigned long long code_mis = 0, scale_mis = 0;
-  for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
-       row += warps) {
-    const float g = g_s[grp.of(row)];
-    const QConsts qc = make_qconsts(g);
-    for (int p0 = 0; p0 < npass; p0 += 2) {
-      uint2 cw[2];
-      uint32_t sc[2], xw[2][8];
+  // the codes, scales (and trainer input) of passes [p0, p0 + kU) of a row
+  auto load_passes = [&](int64_t row, int p0, uint2 (&cw)[kU], uint32_t (&sc)[kU], uint32_t (&xw)[kTrain ? kU : 1][8]) {
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int kb = (p0 + u) * 32 + lane;
-        if (kb < nkb) {
-          cw[u] = *reinterpret_cast<const uint2*>(codes + row * (K / 2) + kb * 8);
-          sc[u] = scales[tiled ? tiled_scale_offset(row, kb, ncol_tiles) : row * nkb + kb];
-          if (a.x_train) load_bf16x16(a.x_train + row * K + kb * 16, xw[u]);
+    for (int u = 0; u < kU; ++u) {
+      const int kb = (p0 + u) * 32 + lane;
+      if (kb < nkb) {
+        cw[u] = *reinterpret_cast<const uint2*>(codes + row * (K / 2) + kb * 8);
+        sc[u] = scales[tiled ? tiled_scale_offset(row, kb, ncol_tiles) : row * nkb + kb];
+        if constexpr (kTrain) load_bf16x16(a.x_train + row * K + kb * 16, xw[u]);
+      }
+    }
+  };
+  // x_hat of those passes (and the mismatch counts)
+  auto replay_passes = [&](int64_t row, int p0, float g, const QConsts& qc, const uint2 (&cw)[kU],
+                           const uint32_t (&sc)[kU], const uint32_t (&xw)[kTrain ? kU : 1][8]) {
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int p = p0 + u;
+      if (p >= npass) break;                         // warp-uniform
+      const int kb = p * 32 + lane;
+      QCore q{0u, 0u, 0u, 0.0f};
+      uint32_t o[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+      if (kb < nkb) {
+        q.lo = cw[u].x;
+        q.hi = cw[u].y;
+        q.scale = sc[u];
+        q.sv = e4m3_value(sc[u]);
+        deq_block_bf16(q, g, 1, o);
+        if constexpr (kTrain) {
+          const QCore t = quant_core(xw[u], qc);
+          // nibbles that differ: OR-fold each nibble onto its low bit, count
+          uint32_t d0 = t.lo ^ q.lo, d1 = t.hi ^ q.hi;
+          d0 = (d0 | (d0 >> 1) | (d0 >> 2) | (d0 >> 3)) & 0x11111111u;
+          d1 = (d1 | (d1 >> 1) | (d1 >> 2) | (d1 >> 3)) & 0x11111111u;
+          code_mis += __popc(d0) + __popc(d1);
+          scale_mis += (t.scale != q.scale) ? 1u : 0u;
         }
       }
+      if (kb < nkb) {
+        uint4* dst = reinterpret_cast<uint4*>(a.x_hat + row * K + kb * 16);
+        dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+        dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+      }
+      if (d.n_chan) {
+        // compensation channels of this pass, rewritten after the block stores above
+        replay_channel_pass(q, g, p, pass_slot[p], pass_slot[p + 1], chan_s, resid_rec + row * d.n_chan,
+                            a.x_hat + row * K);
+      }
+    }
+  };
+  const int64_t first = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (!kTrain && npass <= kU) {
+    // a whole row per batch: the next row's codes and scales are loaded
+    // while this row is replayed
+    uint2 cw[kU], ncw[kU];
+    uint32_t sc[kU], nsc[kU], xw[kTrain ? kU : 1][8];
+    if (first < rows) load_passes(first, 0, cw, sc, xw);
+    for (int64_t row = first; row < rows; row += warps) {
+      if (row + warps < rows) load_passes(row + warps, 0, ncw, nsc, xw);
+      const float g = g_s[grp.of(row)];
+      replay_passes(row, 0, g, make_qconsts(g), cw, sc, xw);
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int p = p0 + u;
-        if (p >= npass) break;                         // warp-uniform
-        const int kb = p * 32 + lane;
-        QCore q{0u, 0u, 0u, 0.0f};
-        if (kb < nkb) {
-          q.lo = cw[u].x;
-          q.hi = cw[u].y;
-          q.scale = sc[u];
-          q.sv = e4m3_value(sc[u]);
-          uint32_t o[8];
-          deq_block_bf16(q, g, 1, o);
-          uint4* dst = reinterpret_cast<uint4*>(a.x_hat + row * K + kb * 16);
-          dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-          dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
-          if (a.x_train) {
-            const QCore t = quant_core(xw[u], qc);
-            // nibbles that differ: OR-fold each nibble onto its low bit, count
-            uint32_t d0 = t.lo ^ q.lo, d1 = t.hi ^ q.hi;
-            d0 = (d0 | (d0 >> 1) | (d0 >> 2) | (d0 >> 3)) & 0x11111111u;
-            d1 = (d1 | (d1 >> 1) | (d1 >> 2) | (d1 >> 3)) & 0x11111111u;
-            code_mis += __popc(d0) + __popc(d1);
-            scale_mis += (t.scale != q.scale) ? 1u : 0u;
-          }
-        }
-        if (d.n_chan) {
-          // compensation channels of this pass, rewritten after the block stores above
-          replay_channel_pass(q, g, p, pass_slot[p], pass_slot[p + 1], chan_s, resid_rec + row * d.n_chan,
-                              a.x_hat + row * K);
-        }
+      for (int u = 0; u < kU; ++u) {
+        cw[u] = ncw[u];
+        sc[u] = nsc[u];
+      }
+    }
+  } else {
+    for (int64_t row = first; row < rows; row += warps) {
+      const float g = g_s[grp.of(row)];
+      const QConsts qc = make_qconsts(g);
+      for (int p0 = 0; p0 < npass; p0 += kU) {
+        uint2 cw[kU];
+        uint32_t sc[kU], xw[kTrain ? kU : 1][8];
+        load_passes(row, p0, cw, sc, xw);
+        replay_passes(row, p0, g, qc, cw, sc, xw);
       }
     }
   }
-  if (a.x_train) {
+  if constexpr (kTrain) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       code_mis += __shfl_xor_sync(0xffffffffu, code_mis, o);
@@ -318,12 +352,12 @@ int trace_replay_qrecord(const void* record, size_t record_bytes, int layer_id, 
                status, make_fastdiv(static_cast<uint32_t>(K / 16))};
   // worst case: group offsets and scales of 1024 groups, the pass table and 256 channels
   size_t smem = (2 * 1024 + 1) * 4 + (static_cast<size_t>((K / 16 + 31) / 32) + 1 + 256) * 4;
+  auto kernel = x_train ? replay_kernel<true> : replay_kernel<false>;
   if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(replay_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
-          cudaSuccess)
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
     return set_error(QUADS_ERR_CUDA, "cannot raise shared memory of replay_kernel");
-  const int grid = persistent_grid(reinterpret_cast<const void*>(replay_kernel), kThreads, smem, ceil_div(rows, 8));
-  replay_kernel<<<grid, kThreads, smem, stream>>>(a);
+  const int grid = persistent_grid(reinterpret_cast<const void*>(kernel), kThreads, smem, ceil_div(rows, 8));
+  kernel<<<grid, kThreads, smem, stream>>>(a);
   count_launches(1);
   return check_launch("replay_kernel");
 }
