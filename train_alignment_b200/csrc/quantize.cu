@@ -199,6 +199,9 @@ __device__ __forceinline__ void st_shared_u32x8(uint32_t* p, const uint32_t (&o)
 template <int kMode>
 __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a) {
   constexpr bool kFq = kMode == 1, kAct = kMode == 2;
+  // passes of a row whose 32-byte loads are in flight at once (the
+  // activation quantizer's per-block work is lighter: more loads cover it)
+  constexpr int kU = kAct ? 4 : 2;
   const bool has_codes = kFq || kAct || a.codes != nullptr;
   const bool has_scales = kFq || kAct || a.scales != nullptr;
   const bool has_wfq = kFq || (!kAct && a.w_fq != nullptr);
@@ -280,15 +283,15 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a) {
     // the row's part of the scale offsets (tiled: band, lane and quarter of the row)
     const int64_t sbase = tiled ? ((drow >> 7) * ncol_tiles) * 512 + (drow & 31) * 16 + ((drow >> 5) & 3) * 4
                                 : drow * nkb;
-    for (int p0 = 0; p0 < npass; p0 += 2) {
-      uint32_t w[2][8];
+    for (int p0 = 0; p0 < npass; p0 += kU) {
+      uint32_t w[kU][8];
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
+      for (int u = 0; u < kU; ++u) {
         const int kb = (p0 + u) * 32 + lane;
         if (kb < nkb) load_bf16x16(xr + kb * 16, w[u]);
       }
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
+      for (int u = 0; u < kU; ++u) {
         const int p = p0 + u;
         if (p >= npass) break;                         // warp-uniform
         const int kb = p * 32 + lane;
