@@ -102,6 +102,23 @@ int quads_gemm_set_tile_shape(int shape);
  * Process-wide; not synchronized with launches in flight. */
 int quads_gemm_set_decode_rows(int rows);
 
+/* SM budget for kernels launched afterwards (from any host thread), so that
+ * an HBM-bound stream and the tensor-core GEMMs can run side by side on
+ * disjoint SMs.  With 0 < n < the device's SM count:
+ *   - the persistent grouped GEMMs (every tile shape, the decode tiles and
+ *     the W4A16 GEMM) launch at most n CTAs (n / 2 CTA pairs);
+ *   - quads_fakequant_weight_ste_backward launches n CTAs of 1024 threads,
+ *     each requesting more than half of an SM's shared memory, so that each
+ *     takes an SM of its own.
+ * A persistent GEMM CTA needs all of an SM's shared memory, so the two
+ * never share an SM: launched on concurrent streams with budgets n_gemm
+ * and n_ste, n_gemm + n_ste <= the SM count, they split the GPU.  Results do
+ * not depend on the budget.  n = 0 (or n >= the SM count) restores the
+ * default: grids sized to the whole device.  Returns the previous budget,
+ * or QUADS_ERR_INVALID_ARG for n < 0.  Process-wide; read at launch (and so
+ * at CUDA graph capture) time. */
+int quads_set_sm_budget(int n);
+
 /* Bytes of a scale array of `rows` x K/16 scales in the given layout. */
 size_t quads_scales_bytes(int64_t rows, int64_t K, int scale_layout);
 

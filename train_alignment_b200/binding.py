@@ -63,6 +63,7 @@ _SIGS = {
     "quads_selftest_bounded_wait": (c_i32, [c_u64, c_vp]),
     "quads_gemm_set_tile_shape": (c_i32, [c_i32]),
     "quads_gemm_set_decode_rows": (c_i32, [c_i32]),
+    "quads_set_sm_budget": (c_i32, [c_i32]),
     "quads_scales_bytes": (c_sz, [c_i64, c_i64, c_i32]),
     "quads_amax_bf16": (c_i32, [c_vp, c_i64, c_i64, c_i64, c_vp, c_i32, c_vp, c_vp]),
     "quads_quantize_workspace_bytes": (c_sz, [c_i32]),
@@ -210,6 +211,15 @@ def gemm_set_decode_rows(rows):
     prev = int(load().quads_gemm_set_decode_rows(int(rows)))
     if prev < 0:
         _check(prev, "quads_gemm_set_decode_rows")
+    return prev
+
+
+def set_sm_budget(n):
+    """SMs that the persistent GEMMs and the STE backward launched afterwards
+    may use (0: all).  Returns the previous budget."""
+    prev = int(load().quads_set_sm_budget(int(n)))
+    if prev < 0:
+        _check(prev, "quads_set_sm_budget")
     return prev
 
 

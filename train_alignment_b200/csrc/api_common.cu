@@ -13,6 +13,7 @@ thread_local char g_last_error[512] = "";
 std::atomic<uint64_t> g_launches{0};
 std::mutex g_sm_mutex;
 int g_sm_count[64] = {0};
+std::atomic<int> g_sm_budget{0};
 }  // namespace
 
 int set_error(int code, const char* fmt, ...) {
@@ -45,6 +46,17 @@ int num_sms() {
   return g_sm_count[dev];
 }
 
+int sm_budget() {
+  const int b = g_sm_budget.load(std::memory_order_relaxed);
+  const int n = num_sms();
+  return b > 0 && b < n ? b : 0;
+}
+
+int grid_sms() {
+  const int b = sm_budget();
+  return b > 0 ? b : num_sms();
+}
+
 int persistent_grid(const void* kernel, int threads, size_t smem, int64_t work_blocks) {
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) != cudaSuccess || per_sm < 1)
@@ -63,6 +75,12 @@ const char* quads_last_error(void) { return quads::g_last_error; }
 int quads_abi_version(void) { return 1; }
 
 uint64_t quads_launch_count(void) { return quads::g_launches.load(); }
+
+int quads_set_sm_budget(int n) {
+  quads::clear_error();
+  QUADS_REQUIRE(n >= 0, QUADS_ERR_INVALID_ARG, "the SM budget must be >= 0");
+  return quads::g_sm_budget.exchange(n);
+}
 
 size_t quads_scales_bytes(int64_t rows, int64_t K, int scale_layout) {
   if (rows < 0 || K < 0 || K % 16 != 0) return 0;

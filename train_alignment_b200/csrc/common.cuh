@@ -18,6 +18,13 @@ int persistent_grid(const void* kernel, int threads, size_t smem, int64_t work_b
 void clear_error();
 void count_launches(uint64_t n);
 int num_sms();
+// The SM budget set by quads_set_sm_budget (0: none, or a budget of at least
+// the device's SM count), and the SMs a persistent grid may use.
+int sm_budget();
+int grid_sms();
+// Device address of the word in which bounded device-side waits record a
+// timeout (read and cleared by quads_device_status), or null.
+unsigned int* wait_status_word();
 
 // Returns QUADS_ERR_CUDA (with a message) if the last launch failed.
 int check_launch(const char* what);

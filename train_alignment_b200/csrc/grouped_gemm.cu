@@ -45,6 +45,12 @@ namespace quads {
 
 __device__ unsigned int g_wait_status = 0u;
 
+unsigned int* wait_status_word() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_wait_status) != cudaSuccess) return nullptr;
+  return static_cast<unsigned int*>(p);
+}
+
 namespace {
 
 constexpr int BM = 128;
@@ -2074,6 +2080,7 @@ int launch_gemm_pair(const uint8_t* a_codes, const uint8_t* a_scales, const floa
   const int64_t max_tiles = (rows_cap / 128) * (N / PBN);
   if constexpr (kPair) {
     int64_t clusters = pair_clusters<kSwiglu, kQuant>(smem);
+    if (sm_budget() > 0 && clusters > sm_budget() / 2) clusters = sm_budget() / 2 > 0 ? sm_budget() / 2 : 1;
     if (clusters > max_tiles) clusters = max_tiles;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
@@ -2091,7 +2098,7 @@ int launch_gemm_pair(const uint8_t* a_codes, const uint8_t* a_scales, const floa
       return set_error(QUADS_ERR_CUDA, "launch of the pair-tile GEMM failed: %s",
                        cudaGetErrorString(cudaGetLastError()));
   } else {
-    int64_t grid = num_sms();
+    int64_t grid = grid_sms();
     if (grid > max_tiles) grid = max_tiles;
     kernel<<<static_cast<unsigned>(grid), kPairThreads, smem, stream>>>(tm_a, tm_b, tm_r, tm_wc, tm_y, p);
   }
@@ -2174,7 +2181,7 @@ int launch_gemm_decode(const uint8_t* a_codes, const uint8_t* a_scales, const fl
   p.timeout_ns = kGemmTimeoutNs;
   // at most one unit per 128 rows (segments are 128-aligned) and 256 weight rows
   const int64_t max_units = (rows_cap / kDecTok) * (N / kDecRowsPerUnit);
-  int64_t grid = num_sms();
+  int64_t grid = grid_sms();
   if (grid > max_units) grid = max_units;
   kernel<<<static_cast<unsigned>(grid), kDecThreads, smem, stream>>>(tm_x, tm_w, tm_r, tm_wc, p);
   count_launches(1);
@@ -2314,7 +2321,7 @@ int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_
   p.stages = stages;
   p.timeout_ns = kGemmTimeoutNs;
   const int64_t max_tiles = (rows_cap / BM) * (N / kBN);
-  int grid = num_sms();
+  int grid = grid_sms();
   if (grid > max_tiles) grid = static_cast<int>(max_tiles);
   grouped_gemm_kernel<kSwiglu, kQuant, kW4A16, kBN><<<grid, threads_for(kQuant, kW4A16), smem, stream>>>(
       tm_a, tm_b, tm_r, tm_wc, tm_y, tm_a2, tm_b2, p);

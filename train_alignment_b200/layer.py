@@ -14,6 +14,7 @@ compensation weight columns), the straight-through backward accumulated
 into the master gradient, the export of the rollout's quantization record
 and its replay against the trainer's activation.
 """
+import contextlib
 import math
 
 import torch
@@ -67,7 +68,7 @@ class MoELayer:
     fixed token count; step() runs the whole path without allocating."""
 
     def __init__(self, cfg: MoEConfig, w_gu, w_d, chan_x, chan_h, device="cuda", fuse_swiglu=None, overlap=True,
-                 fuse_requant=False, amax_h_init=None, comp="bf16", materialize_wfq=True):
+                 fuse_requant=False, amax_h_init=None, comp="bf16", materialize_wfq=True, side_sms=None):
         self.cfg = cfg
         T, H, E, k, F = cfg.T, cfg.H, cfg.E, cfg.k, cfg.F
         dev = torch.device(device)
@@ -116,6 +117,13 @@ class MoELayer:
         self.materialize_wfq = bool(materialize_wfq)
         # the weight side of a step on its own stream (False: one stream)
         self.overlap = bool(overlap)
+        # SMs of the overlapped step's STE backward; the rollout's GEMMs run on
+        # the others meanwhile (0: every kernel sized to the whole device)
+        n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+        self.side_sms = SIDE_SMS_DEFAULT if side_sms is None else int(side_sms)
+        if not 0 <= self.side_sms < n_sm:
+            raise ValueError(f"side_sms must be in [0, {n_sm})")
+        self.gemm_sms = n_sm - self.side_sms if self.side_sms else 0
         self.nc_x = int(chan_x.numel())
         self.nc_h = int(chan_h.numel())
         cap = B.moe_rows_capacity(T, k, E)
@@ -388,9 +396,12 @@ class MoELayer:
         waiting only for its own weights; the TRACE export (the record's
         header: its sections are written in place by the rollout's kernels)
         and the trainer's replays on a third stream, each replay as soon as
-        its operand is recorded.  The call returns with the calling stream
-        joined to both.  The replay's mismatch counters accumulate across
-        steps (zero them with reset_counts())."""
+        its operand is recorded.  While the rollout's GEMMs run, the STE
+        backward keeps to side_sms SMs and the GEMMs to the rest (the
+        library's SM budget), so that the HBM-bound and the tensor-core work
+        share the GPU instead of taking turns.  The call returns with the
+        calling stream joined to both.  The replay's mismatch counters
+        accumulate across steps (zero them with reset_counts())."""
         cfg = self.cfg
         T, H, E, k, F = cfg.T, cfg.H, cfg.E, cfg.k, cfg.F
         t = timer or StageTimer(False)
@@ -410,16 +421,29 @@ class MoELayer:
             return out
         self.side.wait_stream(main)
         with torch.cuda.stream(self.side):
-            # gate/up first, so that the gate/up GEMM can start as early as
-            # possible (its amax pass leaves the weights in L2 for the fake-quant)
             t.mark("start")
-            self._amax_w_gate_up(t)
-            self._fakequant_gate_up(t)
-            self.ev_w_gu.record(self.side)
-            self._amax_w_down(t)
-            self._fakequant_down(t)
-            self.ev_w_d.record(self.side)
-            self.ste_backward(grad_gu_fq, grad_d_fq, t)
+            if self.side_sms:
+                # SMs split between the GEMMs and the STE: the whole weight
+                # sync first (on every SM), then the STE on its own SMs
+                # beside the GEMMs
+                self._amax_w(t)
+                self._fakequant_gate_up(t)
+                self.ev_w_gu.record(self.side)
+                self._fakequant_down(t)
+                self.ev_w_d.record(self.side)
+                with _sm_budget(self.side_sms):
+                    self.ste_backward(grad_gu_fq, grad_d_fq, t)
+            else:
+                # gate/up first, so that the gate/up GEMM can start as early as
+                # possible (its amax pass leaves the weights in L2 for the
+                # fake-quant)
+                self._amax_w_gate_up(t)
+                self._fakequant_gate_up(t)
+                self.ev_w_gu.record(self.side)
+                self._amax_w_down(t)
+                self._fakequant_down(t)
+                self.ev_w_d.record(self.side)
+                self.ste_backward(grad_gu_fq, grad_d_fq, t)
         self._rollout_front(x, logits, t)
         self.ev_x.record(main)
         self.trn.wait_event(self.ev_x)
@@ -428,9 +452,12 @@ class MoELayer:
             self.export(layer_id)
             t.mark("export")
             self._replay_x(x_train, layer_id, t)
-        main.wait_event(self.ev_w_gu)
+        # with the SMs split, the gate/up GEMM starts once both weights are
+        # synced, so that it does not share the SMs with the fake-quant
+        main.wait_event(self.ev_w_d if self.side_sms else self.ev_w_gu)
         t.mark("wait_w_gate_up")
-        self._rollout_gate_up(t)
+        with _sm_budget(self.gemm_sms):
+            self._rollout_gate_up(t)
         main.wait_event(self.ev_w_d)
         t.mark("wait_w_down")
 
@@ -440,7 +467,8 @@ class MoELayer:
             with torch.cuda.stream(self.trn):
                 self._replay_h(layer_id, t)
 
-        out = self._rollout_down(t, replay_h_when_recorded)
+        with _sm_budget(self.gemm_sms):
+            out = self._rollout_down(t, replay_h_when_recorded)
         main.wait_stream(self.trn)
         main.wait_stream(self.side)
         t.mark("join")
@@ -448,6 +476,25 @@ class MoELayer:
 
     def reset_counts(self):
         self.counts.zero_()
+
+
+# SMs given to the STE backward while the rollout's GEMMs run beside it in
+# the overlapped step (the STE's bulk-copy kernel moves about 110 GB/s per
+# SM; the GEMMs keep the other 108 SMs)
+SIDE_SMS_DEFAULT = 40
+
+
+@contextlib.contextmanager
+def _sm_budget(n):
+    """The library's SM budget set to n (0: none) for the launches inside."""
+    if not n:
+        yield
+        return
+    prev = B.set_sm_budget(n)
+    try:
+        yield
+    finally:
+        B.set_sm_budget(prev)
 
 
 def _pad_chan(chan, multiple):
@@ -483,7 +530,7 @@ def calibrate_channels(x, n_sel):
 
 
 def build_layer(cfg: MoEConfig, inputs, device="cuda", overlap=True, fuse_requant=False, comp="bf16",
-                materialize_wfq=True):
+                materialize_wfq=True, side_sms=None):
     """Layer from generated inputs: channel sets calibrated on the layer's own
     batch (X for the gate/up input, the uncompensated h for the down input);
     with fuse_requant, h's first-step per-expert amax is calibrated on the
@@ -501,4 +548,4 @@ def build_layer(cfg: MoEConfig, inputs, device="cuda", overlap=True, fuse_requan
     del probe
     return MoELayer(cfg, inputs["w_gu"], inputs["w_d"], chan_x, chan_h, device, overlap=overlap,
                     fuse_requant=fuse_requant, amax_h_init=amax_h if fuse_requant else None, comp=comp,
-                    materialize_wfq=materialize_wfq)
+                    materialize_wfq=materialize_wfq, side_sms=side_sms)
