@@ -107,9 +107,9 @@ int quads_gemm_set_decode_rows(int rows);
  * disjoint SMs.  With 0 < n < the device's SM count:
  *   - the persistent grouped GEMMs (every tile shape, the decode tiles and
  *     the W4A16 GEMM) launch at most n CTAs (n / 2 CTA pairs);
- *   - quads_fakequant_weight_ste_backward launches n CTAs of 1024 threads,
- *     each requesting more than half of an SM's shared memory, so that each
- *     takes an SM of its own.
+ *   - quads_fakequant_weight_ste_backward, whose CTAs each request more
+ *     than half of an SM's shared memory (one CTA per SM), launches n of
+ *     them instead of one per SM of the device.
  * A persistent GEMM CTA needs all of an SM's shared memory, so the two
  * never share an SM: launched on concurrent streams with budgets n_gemm
  * and n_ste, n_gemm + n_ste <= the SM count, they split the GPU.  Results do
@@ -456,7 +456,9 @@ int quads_fakequant_weight_ste_gate_up(const uint16_t* w, int64_t n_mat, int64_t
                                        void* ws, size_t ws_bytes, quads_stream_t stream);
 /* Straight-through backward ([QUADS-fr §2.2.A]: the QAT trainer's gradient
  * passes through the weight fake-quant): grad_w = grad_wfq (accumulate = 0) or
- * grad_w = bf16(fp32(grad_w + grad_wfq)) (accumulate = 1); n BF16 elements. */
+ * grad_w = bf16(fp32(grad_w + grad_wfq)) (accumulate = 1); n BF16 elements,
+ * both arrays 16-byte aligned.  One CTA per SM streams 16 KB chunks of both
+ * through a shared-memory ring (see quads_set_sm_budget). */
 int quads_fakequant_weight_ste_backward(const uint16_t* grad_wfq, uint16_t* grad_w, int64_t n,
                                         int accumulate, quads_stream_t stream);
 

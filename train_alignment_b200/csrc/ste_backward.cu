@@ -9,18 +9,6 @@
 namespace quads {
 namespace {
 
-constexpr int kThreads = 256;
-
-int ste_grid(int64_t work) {
-  int64_t g = ceil_div(work, int64_t(kThreads));
-  const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
-  return static_cast<int>(g > cap ? cap : (g < 1 ? 1 : g));
-}
-
-// Each thread keeps kSteUnroll 16-byte vectors of both inputs in flight per
-// iteration of a grid-stride loop.
-constexpr int kSteUnroll = 2;
-
 __device__ __forceinline__ uint4 ste_add(uint4 a, uint4 b) {
   uint32_t* pa = reinterpret_cast<uint32_t*>(&a);
   const uint32_t* pb = reinterpret_cast<const uint32_t*>(&b);
@@ -33,48 +21,12 @@ __device__ __forceinline__ uint4 ste_add(uint4 a, uint4 b) {
   return a;
 }
 
-__global__ void __launch_bounds__(kThreads) ste_backward_kernel(const uint16_t* __restrict__ gfq,
-                                                                uint16_t* __restrict__ gw, int64_t n, int accumulate) {
-  const int64_t nv = n / 8;
-  const int64_t nth = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  const uint4* src = reinterpret_cast<const uint4*>(gfq);
-  uint4* dst = reinterpret_cast<uint4*>(gw);
-  int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  for (; i + (kSteUnroll - 1) * nth < nv; i += kSteUnroll * nth) {
-    uint4 a[kSteUnroll], b[kSteUnroll];
-#pragma unroll
-    for (int u = 0; u < kSteUnroll; ++u) a[u] = __ldg(src + i + u * nth);
-    if (accumulate) {
-#pragma unroll
-      for (int u = 0; u < kSteUnroll; ++u) b[u] = dst[i + u * nth];
-#pragma unroll
-      for (int u = 0; u < kSteUnroll; ++u) a[u] = ste_add(a[u], b[u]);
-    }
-#pragma unroll
-    for (int u = 0; u < kSteUnroll; ++u) dst[i + u * nth] = a[u];
-  }
-  for (; i < nv; i += nth) {
-    uint4 a = __ldg(src + i);
-    if (accumulate) a = ste_add(a, dst[i]);
-    dst[i] = a;
-  }
-  // tail (n % 8 elements) handled by the first thread
-  if (blockIdx.x == 0 && threadIdx.x == 0) {
-    for (int64_t i = nv * 8; i < n; ++i) {
-      if (accumulate)
-        gw[i] = static_cast<uint16_t>(
-            float_to_bf16_bits(__fadd_rn(bf16_bits_to_float(gfq[i]), bf16_bits_to_float(gw[i]))));
-      else
-        gw[i] = gfq[i];
-    }
-  }
-}
-
-// With an SM budget of n SMs: one CTA on each of n SMs, streaming through
-// shared memory.  The loads are bulk copies of one chunk of each input per
-// stage into a ring of stages; sixteen arithmetic warps each add their own
-// slice of a stage and store the sum with coalesced 16-byte stores.  The
-// rollout's persistent GEMMs keep the other SMs to themselves.
+// One CTA per SM (all SMs, or the SM budget), streaming through shared
+// memory: the loads are bulk copies of one 16 KB chunk of each input per
+// stage into a ring of six stages; sixteen arithmetic warps each add their
+// own slice of a stage and store the sum with coalesced 16-byte stores.  The
+// shared-memory request keeps a second CTA off the SM, so that under an SM
+// budget the rollout's persistent GEMMs keep the other SMs to themselves.
 constexpr int kTmaIssuers = 1;                 // loading warps per input (stages alternate between them)
 constexpr int kTmaConsumerWarps = 16;
 constexpr int kTmaThreads = 64 * kTmaIssuers + 32 * kTmaConsumerWarps;   // loading warps, then arithmetic warps
@@ -253,30 +205,24 @@ int quads_fakequant_weight_ste_backward(const uint16_t* grad_wfq, uint16_t* grad
   if (n == 0) return QUADS_OK;
   QUADS_REQUIRE(grad_wfq && grad_w && aligned(grad_wfq, 16) && aligned(grad_w, 16), QUADS_ERR_INVALID_ARG,
                 "gradients must be non-null and 16-byte aligned");
-  if (sm_budget() > 0) {
-    if (cudaFuncSetAttribute(ste_backward_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTmaSmem) !=
-        cudaSuccess)
-      return set_error(QUADS_ERR_CUDA, "cannot reserve shared memory for the STE backward");
-    const int64_t nv = n / 8;
-    int launches = 0;
-    if (nv > 0) {
-      const int64_t nchunks = ceil_div(nv, int64_t(kTmaChunk / 16));
-      const int grid = static_cast<int>(nchunks < sm_budget() ? nchunks : sm_budget());
-      ste_backward_tma_kernel<<<grid, kTmaThreads, kTmaSmem, stream>>>(grad_wfq, grad_w, nv, accumulate,
-                                                                       wait_status_word());
-      ++launches;
-    }
-    if (nv * 8 < n) {
-      ste_backward_tail_kernel<<<1, 32, 0, stream>>>(grad_wfq, grad_w, nv * 8, n, accumulate);
-      ++launches;
-    }
-    count_launches(launches);
-    return check_launch("ste_backward_tma_kernel");
+  if (cudaFuncSetAttribute(ste_backward_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTmaSmem) !=
+      cudaSuccess)
+    return set_error(QUADS_ERR_CUDA, "cannot reserve shared memory for the STE backward");
+  const int64_t nv = n / 8;
+  int launches = 0;
+  if (nv > 0) {
+    const int64_t nchunks = ceil_div(nv, int64_t(kTmaChunk / 16));
+    const int grid = static_cast<int>(nchunks < grid_sms() ? nchunks : grid_sms());
+    ste_backward_tma_kernel<<<grid, kTmaThreads, kTmaSmem, stream>>>(grad_wfq, grad_w, nv, accumulate,
+                                                                     wait_status_word());
+    ++launches;
   }
-  ste_backward_kernel<<<ste_grid(ceil_div(ceil_div(n, 8), int64_t(kSteUnroll))), kThreads, 0, stream>>>(
-      grad_wfq, grad_w, n, accumulate);
-  count_launches(1);
-  return check_launch("ste_backward_kernel");
+  if (nv * 8 < n) {
+    ste_backward_tail_kernel<<<1, 32, 0, stream>>>(grad_wfq, grad_w, nv * 8, n, accumulate);
+    ++launches;
+  }
+  count_launches(launches);
+  return check_launch("ste_backward_tma_kernel");
 }
 
 }  // extern "C"
