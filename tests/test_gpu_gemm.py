@@ -10,7 +10,7 @@ from oracle import formats as F
 from oracle import moe as M
 from oracle import nvfp4 as Q
 from tests.helpers import (assert_bits_equal, assert_close_tol, bf16_np, bf16_torch, f32_of, gate_up_interleave_index,
-                           u8_np)
+                           swiglu_carried, u8_np)
 from train_alignment_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
@@ -403,6 +403,49 @@ def test_grouped_gemm_w4a16_parity(cuda_lib, counts, N, K):
         err = (y[lo:hi].float() - yt).abs()
         bound = 2.0 ** -8 * yt.abs() + K * 2.0 ** -22 * torch.matmul(x[lo:hi].float().abs(), w_fq[e].float().abs().t())
         assert bool((err <= bound).all()), f"expert {e}: {int((err > bound).sum())} outside the FP32 bound"
+
+
+@pytest.mark.parametrize("shape", [0, 1])
+@pytest.mark.parametrize("counts,N,K,swiglu", [([300, 0, 40, 700], 512, 384, False), ([257, 1, 600], 768, 256, True)])
+def test_grouped_gemm_w4a16_both_kernels(cuda_lib, shape, counts, N, K, swiglu):
+    """Where N % 256 == 0 the W4A16 GEMM takes the weights-as-M kernel (W_fq
+    converted into tensor memory, 128 weight rows by 256 rows per unit);
+    tile shape 0 keeps the 128 x N kernel.  Both against the oracle."""
+    prev = cuda_lib.gemm_set_tile_shape(shape)
+    try:
+        p = _w4a16_problem(counts, N, K, seed=3 * sum(counts) + N + K + shape)
+        E, cap, R, off = p["E"], p["cap"], p["R"], p["off"]
+        dev = "cuda"
+        perm = gate_up_interleave_index(N // 2) if swiglu else np.arange(N)
+        w_codes = torch.from_numpy(np.ascontiguousarray(F.pack_nibbles(p["w_c"][:, perm]))).to(dev)
+        w_scales = torch.from_numpy(F.scales_to_tiled(p["w_s"][:, perm].reshape(E * N, K // 16))).to(dev)
+        g_w = torch.tensor(p["g_w"], dtype=torch.float32, device=dev)
+        x = bf16_torch(p["x"])
+        offt = torch.from_numpy(off).to(dev)
+        ref, absdot = M.grouped_gemm_w4a16(p["x"][:R], p["w_c"], p["w_s"], p["g_w"], off)
+        if not swiglu:
+            y = torch.full((cap, N), float("nan"), dtype=torch.bfloat16, device=dev)
+            cuda_lib.moe_grouped_gemm_w4a16(x, w_codes, w_scales, g_w, offt, E, cap, N, K, y=y)
+            torch.cuda.synchronize()
+            assert cuda_lib.device_status() == cuda_lib.OK
+            got = bf16_np(y)
+            assert_close_tol(got[:R], ref, absdot, what=f"W4A16 GEMM (tile shape {shape})")
+            assert np.all(np.isnan(got[R:]))
+        else:
+            h, amax = cuda_lib.moe_grouped_gemm_w4a16(x, w_codes, w_scales, g_w, offt, E, cap, N, K, swiglu=True)
+            torch.cuda.synchronize()
+            assert cuda_lib.device_status() == cuda_lib.OK
+            F_ = N // 2
+            h_ref, tol = swiglu_carried(ref, absdot, F_)
+            got = bf16_np(h)[:R]
+            err = np.abs(got - h_ref)
+            assert np.all(err <= tol), f"{int(np.sum(err > tol))} h values outside the tolerance"
+            a = f32_of(amax)
+            for e in range(E):
+                lo, hi = off[e], off[e + 1]
+                assert a[e] == (np.max(np.abs(got[lo:hi])) if hi > lo else 0.0), e
+    finally:
+        cuda_lib.gemm_set_tile_shape(prev)
 
 
 @pytest.mark.parametrize("counts,F_,K", [([64], 64, 64), ([500, 20, 1000, 3], 192, 1024),

@@ -239,6 +239,14 @@ __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
+__device__ __forceinline__ void st_shared_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
@@ -269,6 +277,17 @@ __device__ __forceinline__ void mma_bf16(uint32_t d, uint64_t a, uint64_t b, uin
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
       "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// kind::f16 with A read from tensor memory (a: its TMEM address, K-major
+// rows on the lanes, two 16-bit elements per 32-bit column)
+__device__ __forceinline__ void mma_bf16_tmem_a(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc,
+                                                uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+      "r"(a), "l"(b), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 __device__ __forceinline__ void tmem_load32(uint32_t taddr, uint32_t (&r)[32]) {
@@ -1849,6 +1868,325 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
+// ---------------------------------------------------------------------------
+// W4A16 with the weights as the MMA's M operand, converted into TMEM.
+//
+// The trainer's GEMM Y = X . W_fq^T (X BF16; the weights given as NVFP4
+// codes and scales, W_fq = bf16(fp32(val(q) val(s)) g_w[e])).  The 128 x N
+// W4A16 kernel converts each weight tile into shared memory, where the MMA
+// reads it back.  Here the converter warps store W_fq straight into tensor
+// memory and the kind::f16 MMA reads it there as its A operand; only the
+// BF16 row tile goes through shared memory to the tensor cores.  D^T = W .
+// X^T: a unit is (expert, 128 weight rows, up to 256 of the expert's rows),
+// the weight rows on the MMA's M (TMEM lanes) and the rows on its N = 256.
+// A weight tile is converted once per 256 rows, and each MMA is the full
+// 128 x 256 x 16.
+//   stage       the codes of the unit's 128 weight rows for 64 K (128 x 32
+//               bytes), their 512-byte scale tile, and the BF16 row tile
+//               (256 rows x 64 K, 128-byte swizzle): 37 KB.
+//   roles       warps 0 and 14 (lane 0) load the even and the odd stages
+//               (two issuing threads fill a stage about twice as fast as
+//               one); warp 1 lane 0 issues the MMAs; warps 2..5 convert the
+//               even stages and warps 15..18 the odd ones (lane i of the
+//               group's warp for quarter q: weight row 32 q + i), so that two
+//               stages are converted at once; warps 6..13 the epilogue (warp
+//               6 + 4 hs + q: lane quarter q, rows [128 hs, 128 hs + 128)).
+//   TMEM        [0, 256) the accumulator (one buffer); [256, 512) eight A
+//               slots of 32 columns (64 K of BF16, two per column).
+//   pipeline    up to eight stages and eight A slots (slot it % 8): a stage
+//               landing implies that its slot's previous MMAs have completed.
+//   SwiGLU      a unit's 128 weight rows are one block of the interleaved
+//               layout: 64 gate rows (lanes 0-63) and the matching 64 up
+//               rows (lanes 64-127).  The up warps (quarters 2, 3) pass their
+//               rounded values to the gate warps through shared memory
+//               (bounded barrier waits), which apply SwiGLU: 64 h columns
+//               per unit.
+constexpr int kW16Rows = 128;                                  // weight rows per unit (M)
+constexpr int kW16Tok = 256;                                   // expert rows per unit at most (N)
+constexpr int kW16SfOff = kW16Rows * 32;                       // after the codes (64 K of FP4 per row)
+constexpr int kW16XOff = kW16SfOff + 1024;                     // 5120: 1024-byte aligned row tile
+constexpr int kW16StageBytes = kW16XOff + kW16Tok * 128;       // 37888
+constexpr int kW16Slots = 8;                                   // A slots in TMEM
+constexpr int kW16MaxStages = 8;
+static_assert(kW16MaxStages <= kW16Slots, "a stage landing must imply its A slot is free");
+constexpr int kW16ACol = 256;
+constexpr int kW16ConvWarps = 4;                               // per group: even and odd stages
+constexpr int kW16EpiWarp0 = 2 + kW16ConvWarps;                // 6
+constexpr int kW16Loader1 = kW16EpiWarp0 + kDecEpiWarps;       // 14: the second loading warp
+constexpr int kW16Conv1 = kW16Loader1 + 1;                     // 15: the odd stages' converters
+constexpr int kW16Threads = 32 * (kW16Conv1 + kW16ConvWarps);  // 608
+constexpr int kW16XchgBytes = 4 * 128 * 32 * 2;                // SwiGLU: four 8 KB up-to-gate buffers
+
+template <bool kSwiglu>
+__global__ void __launch_bounds__(kW16Threads, 1)
+    grouped_gemm_w16m_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                             GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* const base_ptr = smem_raw + (base - raw);
+  const int S = p.stages;                         // <= kW16Slots
+  const uint32_t xchg = base + S * kW16StageBytes;                          // kSwiglu only
+  const uint32_t bar0 = xchg + (kSwiglu ? kW16XchgBytes : 0);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
+  auto conv_full = [&](int j) { return bar0 + 8u * (2 * S + j); };               // A slot j converted
+  auto x_full = [&](int k) { return bar0 + 8u * (2 * S + 2 * kW16Slots + k); };  // up values passed
+  auto x_empty = [&](int k) { return bar0 + 8u * (2 * S + 2 * kW16Slots + 4 + k); };
+  const uint32_t acc_full = bar0 + 8u * (2 * S + 2 * kW16Slots + 8);
+  const uint32_t acc_empty = acc_full + 8;
+  const uint32_t drain_bar = acc_full + 16;
+  uint8_t* const misc = base_ptr + (drain_bar + 8 - base);
+  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(misc);
+  volatile int* const abort_flag = reinterpret_cast<volatile int*>(misc + 4);
+  int32_t* const off_s = reinterpret_cast<int32_t*>(misc + 16);       // E + 1, clamped to rows_cap
+  int32_t* const ub_s = off_s + p.E + 1;                                 // E + 1: first unit of each expert
+  float* const gw_s = reinterpret_cast<float*>(ub_s + p.E + 1);         // g_w[e]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    prefetch_tensormap(&tm_x);
+    prefetch_tensormap(&tm_w);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int j = 0; j < kW16Slots; ++j) mbar_init(conv_full(j), kW16ConvWarps);   // one arrival per converter warp
+    for (int k = 0; k < 4; ++k) {
+      mbar_init(x_full(k), 1);
+      mbar_init(x_empty(k), 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, kDecEpiWarps);
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  const int nwb = p.N / kW16Rows;
+  for (int i = threadIdx.x; i <= p.E; i += blockDim.x) {
+    off_s[i] = min(p.expert_off[i], p.rows_cap);
+    if (i < p.E) gw_s[i] = p.g_w[i];
+  }
+  __syncthreads();
+  if (warp == 2) warp_block_prefix(ub_s, off_s, p.E, kW16Tok, nwb, lane);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int total = ub_s[p.E];
+  const int nks = p.K / 64;                       // stages of 64 K
+  const int n_col_tiles = p.K / 64;               // 128 x 4 scale tiles along K
+  // units ordered expert, row block, weight block (weight blocks innermost:
+  // the CTAs that run at the same time share a BF16 row tile, the larger
+  // operand, and read it from L2; an expert's FP4 weights stay in L2 across
+  // its row blocks)
+  auto unit_of = [&](int u, int& e, int& wrow, int& wb, int& row0, int& nrows) {
+    e = expert_of_row(ub_s, p.E, u);
+    const int local = u - ub_s[e];
+    const int tb = local / nwb;
+    wb = local - tb * nwb;
+    wrow = e * p.N + wb * kW16Rows;
+    row0 = off_s[e] + kW16Tok * tb;
+    nrows = min(kW16Tok, off_s[e + 1] - row0);
+  };
+
+  if ((warp == 0 || warp == kW16Loader1) && lane == 0) {
+    // ---------------------------------------------------- producers (two)
+    const int par = warp == 0 ? 0 : 1;            // the stages it % 2 == par
+    int it = 0, last = -1;
+    bool ok = true;
+    for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+      int e, wrow, wb, row0, nrows;
+      unit_of(u, e, wrow, wb, row0, nrows);
+      for (int ks = 0; ks < nks; ++ks, ++it) {
+        if ((it & 1) != par) continue;
+        const int s = it % S;
+        if (!mbar_wait(empty_bar(s), ((it / S) & 1) ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+        const uint32_t st = base + s * kW16StageBytes;
+        mbar_expect_tx(full_bar(s), kW16SfOff + 512 + kW16Tok * 128);
+        tma_load_2d(st, &tm_w, ks * 32, wrow, full_bar(s));                   // 128 rows x 32 bytes
+        bulk_load(st + kW16SfOff, p.w_scales + (static_cast<int64_t>(wrow / 128) * n_col_tiles + ks) * 512, 512,
+                  full_bar(s));
+        tma_load_2d(st + kW16XOff, &tm_x, ks * 64, row0, full_bar(s));       // 256 rows x 64 BF16
+        last = it;
+      }
+    }
+    if (!ok)   // this thread's copies in flight land before the CTA exits
+      for (int i = (last >= S ? last - S + 1 : 0); i <= last; ++i)
+        if ((i & 1) == par) mbar_wait(full_bar(i % S), (i / S) & 1, nullptr, kDrainTimeoutNs);
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------------ MMA
+    constexpr uint32_t kIdesc = idesc_bf16(kW16Tok);
+    int it = 0, tc = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < total && ok; u += gridDim.x, ++tc) {
+      if (!mbar_wait_cluster(acc_empty, (tc & 1) ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+      tc_fence_after();
+      for (int ks = 0; ks < nks; ++ks, ++it) {
+        const int s = it % S, j = it % kW16Slots;
+        // the converters arrive after they saw the stage land: the row tile is there too
+        if (!mbar_wait_cluster(conv_full(j), (it / kW16Slots) & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t st = base + s * kW16StageBytes;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)            // K = 16 per MMA, 32 bytes along the row tile's rows
+          mma_bf16_tmem_a(tmem, tmem + kW16ACol + 32 * j + 8 * kk, desc_kmajor_sw128(st + kW16XOff + kk * 32), kIdesc,
+                          (ks | kk) != 0 ? 1u : 0u);
+        tc_commit(empty_bar(s));               // frees the stage (and, S <= 8 stages later, the A slot)
+      }
+      if (!ok) break;
+      tc_commit(acc_full);
+    }
+    if (!ok) {
+      tc_commit(drain_bar);
+      mbar_wait(drain_bar, 0, nullptr, kDrainTimeoutNs);
+    }
+  } else if ((warp >= 2 && warp < kW16EpiWarp0) || warp >= kW16Conv1) {
+    // ------------------------------------------------------------ converters
+    // Lane i of the group's warp for quarter q: weight row 32 q + i of the
+    // unit.  Its 32 code bytes and 4 scale bytes of the stage become 64 W_fq
+    // values, stored as 32 columns of its TMEM lane in A slot it % 8 once the
+    // stage has landed and the MMAs that last read the slot have completed.
+    const int q = warp & 3;
+    const int par = warp >= kW16Conv1 ? 1 : 0;   // the stages it % 2 == par
+    const int r = 32 * q + lane;
+    const uint32_t sf_off = kW16SfOff + (r & 31) * 16 + ((r >> 5) & 3) * 4;
+    int it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+      int e, wrow, wb, row0, nrows;
+      unit_of(u, e, wrow, wb, row0, nrows);
+      const float g = gw_s[e];
+      for (int ks = 0; ks < nks; ++ks, ++it) {
+        if ((it & 1) != par) continue;
+        const int s = it % S, j = it % kW16Slots;
+        // the stage landing implies that A slot j is free: the producer
+        // refilled the stage after the MMAs of iteration it - S completed,
+        // and those of it - 8 (the slot's last use) came before them
+        const bool w_ok = mbar_wait(full_bar(s), (it / S) & 1, abort_flag, p.timeout_ns);
+        if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t st = base + s * kW16StageBytes;
+        const uint4 c0 = ld_shared_v4(st + r * 32), c1 = ld_shared_v4(st + r * 32 + 16);
+        const uint32_t sw = ld_shared_u32(st + sf_off);
+        const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + kW16ACol + 32 * j;
+#pragma unroll
+        for (int hg = 0; hg < 2; ++hg) {          // 32 K (two blocks) per 16 columns
+          uint32_t o[16];
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            const int kb = 2 * hg + b;
+            QCore qb{cw[2 * kb], cw[2 * kb + 1], (sw >> (8 * kb)) & 0xFFu, 0.0f};
+            uint32_t w8[8];
+            deq_block_bf16(qb, g, 1, w8);
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) o[8 * b + jj] = w8[jj];
+          }
+          tmem_store16(ta + 16 * hg, o);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(conv_full(j));
+      }
+    }
+  } else if (warp >= kW16EpiWarp0 && warp < kW16Loader1) {
+    // ----------------------------------------------------------- epilogue
+    // Warp 6 + 4 hs + q reads lane quarter q (weight rows 32 q + lane) and
+    // accumulator columns [128 hs, 128 hs + 128) (rows), rounded to BF16
+    // before the accumulator is handed back.  Lane i stores its weight
+    // row's value for each row: a warp writes 64 contiguous bytes per row.
+    const int q = warp & 3, hs = (warp - kW16EpiWarp0) >> 2;
+    const int pair = (q & 1) + 2 * hs;            // SwiGLU: gate warp q, up warp q + 2
+    const uint32_t xb = xchg + pair * (128 * 32 * 2);
+    int tc = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < total && ok; u += gridDim.x, ++tc) {
+      int e, wrow, wb, row0, nrows;
+      unit_of(u, e, wrow, wb, row0, nrows);
+      if (!mbar_wait_cluster(acc_full, tc & 1, abort_flag, p.timeout_ns)) break;
+      tc_fence_after();
+      const int c0 = 128 * hs;
+      const int nvalid = max(0, min(128, nrows - c0));   // rows this warp stores
+      uint32_t v[4][16];                                  // BF16 pairs of consecutive rows
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        if (32 * c < nvalid) {
+          uint32_t a[32];
+          tmem_load32(tmem + (static_cast<uint32_t>(q * 32) << 16) + c0 + 32 * c, a);
+          tmem_wait_ld();
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) v[c][jj] = pack_bf16x2(__uint_as_float(a[2 * jj]), __uint_as_float(a[2 * jj + 1]));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+      if constexpr (!kSwiglu) {
+        uint16_t* const y0 = p.y + static_cast<int64_t>(row0 + c0) * p.N + wb * kW16Rows + 32 * q + lane;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) {
+            const int t = 32 * c + jj;
+            if (t < nvalid) {
+              const uint32_t w = v[c][jj >> 1];
+              y0[static_cast<int64_t>(t) * p.N] = static_cast<uint16_t>((jj & 1) ? (w >> 16) : (w & 0xFFFFu));
+            }
+          }
+      } else if (q >= 2) {
+        // up rows: hand the rounded values to the gate warp of the pair
+        bool w_ok = mbar_wait(x_empty(pair), (tc & 1) ^ 1u, abort_flag, p.timeout_ns);
+        if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) st_shared_u32(xb + ((16 * c + jj) * 32 + lane) * 4, v[c][jj]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(x_full(pair));
+      } else {
+        bool w_ok = mbar_wait(x_full(pair), tc & 1, abort_flag, p.timeout_ns);
+        if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+        const int Fh = p.N / 2;
+        // gate lane 32 q + i: h column wb * 64 + 32 q + i of the expert
+        uint16_t* const h0 = p.y + static_cast<int64_t>(row0 + c0) * Fh + wb * (kW16Rows / 2) + 32 * q + lane;
+        unsigned int hmax = 0u;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            const int t = 32 * c + 2 * jj;
+            const uint32_t up = ld_shared_u32(xb + ((16 * c + jj) * 32 + lane) * 4);
+            if (t < nvalid) {
+              const uint32_t o = swiglu_bf16x2(v[c][jj], up);
+              h0[static_cast<int64_t>(t) * Fh] = static_cast<uint16_t>(o & 0xFFFFu);
+              hmax = max(hmax, o & 0x7FFFu);
+              if (t + 1 < nvalid) {
+                h0[static_cast<int64_t>(t + 1) * Fh] = static_cast<uint16_t>(o >> 16);
+                hmax = max(hmax, (o >> 16) & 0x7FFFu);
+              }
+            }
+          }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(x_empty(pair));
+        hmax = __reduce_max_sync(0xffffffffu, hmax);
+        if (lane == 0 && hmax != 0u && p.amax_bits != nullptr) atomicMax(&p.amax_bits[e], hmax << 16);
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
 // Per-expert amax for the FP4 compensation's residual:
 // amax_r[e] = fp32(fp32(G_e / g_wc[e]) * 2688), G_e = fp32(g_a g_w[e]); the
 // residual's decode scale times g_wc[e] is then G_e up to one rounding.
@@ -2123,6 +2461,52 @@ size_t decode_smem_bytes(int stages, int E) {
          static_cast<size_t>(3 * E + 2) * 4;
 }
 
+size_t w16m_smem_bytes(int stages, bool swiglu, int E) {
+  return 1024 + static_cast<size_t>(stages) * kW16StageBytes + (swiglu ? kW16XchgBytes : 0) +
+         static_cast<size_t>(2 * stages + 2 * kW16Slots + 8 + 3) * 8 + 16 + static_cast<size_t>(3 * E + 2) * 4;
+}
+
+// The W4A16 GEMM on the weights-as-M kernel (N % 256 == 0; arguments
+// validated by launch_gemm).
+template <bool kSwiglu>
+int launch_gemm_w16m(const uint16_t* x, const uint8_t* w_codes, const uint8_t* w_scales, const float* g_w,
+                     const int32_t* expert_off, int E, int64_t rows_cap, int64_t N, int64_t K, uint16_t* y,
+                     float* amax_out, cudaStream_t stream) {
+  CUtensorMap tm_x, tm_w;
+  QUADS_TRY(make_map_2d(&tm_x, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, rows_cap, 64, kW16Tok,
+                        CU_TENSOR_MAP_SWIZZLE_128B));
+  QUADS_TRY(make_map_2d(&tm_w, w_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, E * N, 32, kW16Rows,
+                        CU_TENSOR_MAP_SWIZZLE_NONE));
+  const size_t smem_cap = 232448;
+  int stages = kW16MaxStages;
+  while (stages >= 2 && w16m_smem_bytes(stages, kSwiglu, E) > smem_cap) --stages;
+  QUADS_REQUIRE(stages >= 2, QUADS_ERR_UNSUPPORTED_SHAPE, "not enough shared memory for two stages");
+  const size_t smem = w16m_smem_bytes(stages, kSwiglu, E);
+  auto kernel = grouped_gemm_w16m_kernel<kSwiglu>;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+      cudaSuccess)
+    return set_error(QUADS_ERR_CUDA, "cannot set %zu bytes of shared memory", smem);
+  GemmParams p{};
+  p.w_scales = w_scales;
+  p.g_w = g_w;
+  p.expert_off = expert_off;
+  p.y = y;
+  p.amax_bits = reinterpret_cast<unsigned int*>(amax_out);
+  p.E = E;
+  p.rows_cap = static_cast<int>(rows_cap);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.stages = stages;
+  p.timeout_ns = kGemmTimeoutNs;
+  // at most one unit per 128 rows (segments are 128-aligned) and 128 weight rows
+  const int64_t max_units = (rows_cap / 128) * (N / kW16Rows);
+  int64_t grid = grid_sms();
+  if (grid > max_units) grid = max_units;
+  kernel<<<static_cast<unsigned>(grid), kW16Threads, smem, stream>>>(tm_x, tm_w, p);
+  count_launches(1);
+  return check_launch("grouped_gemm_w16m_kernel");
+}
+
 template <bool kSwiglu>
 int launch_gemm_decode(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_a, int g_a_per_expert,
                        const uint8_t* w_codes, const uint8_t* w_scales, const float* g_w, const int32_t* expert_off,
@@ -2231,6 +2615,12 @@ int launch_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* g_
   if (kSwiglu && amax_out && cudaMemsetAsync(amax_out, 0, sizeof(float) * E, stream) != cudaSuccess)
     return set_error(QUADS_ERR_CUDA, "memset of amax_out failed");
   if (rows_cap == 0) return QUADS_OK;
+  if constexpr (kW4A16 && kBN == 256 && !kQuant) {
+    // the weights as M, converted into TMEM (tile shape 0 keeps the 128 x N kernel)
+    if (g_tile_shape != 0 && N % 256 == 0)
+      return launch_gemm_w16m<kSwiglu>(reinterpret_cast<const uint16_t*>(a_codes), w_codes, w_scales, g_w,
+                                       expert_off, E, rows_cap, N, K, y, amax_out, stream);
+  }
   if constexpr (!kW4A16 && kBN == BN && !kQuant) {
     if (fc == nullptr && N % kDecRowsPerUnit == 0 && decode_selected(rows_cap, E))
       return launch_gemm_decode<kSwiglu>(a_codes, a_scales, g_a, g_a_per_expert, w_codes, w_scales, g_w, expert_off,
