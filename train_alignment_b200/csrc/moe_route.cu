@@ -293,22 +293,43 @@ __global__ void __launch_bounds__(256) gather_kernel(const int32_t* __restrict__
   const int lane = threadIdx.x & 31;
   const int64_t rows = expert_off[E];
   const int64_t nkb = K / 16, ncol_tiles = nkb / 4;
-  const int64_t cbytes = K / 2;
+  const int64_t cbytes = K / 2, ncv = cbytes / 16;
+  // residual rows in 16-byte vectors when they are whole and aligned
+  const bool rvec = n_chan % 8 == 0 && (reinterpret_cast<uintptr_t>(a_resid) & 15) == 0 &&
+                    (reinterpret_cast<uintptr_t>(pa_resid) & 15) == 0;
   for (int64_t p = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; p < rows;
        p += (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5) {
     const int t = src_of[p];
-    // codes: 16-byte vectors
+    const bool has = t >= 0;
+    // codes: 16-byte vectors, four loads in flight per lane before the stores
     uint4* dc = reinterpret_cast<uint4*>(pa_codes + p * cbytes);
     const uint4* sc = reinterpret_cast<const uint4*>(a_codes + static_cast<int64_t>(t) * cbytes);
-    for (int64_t j = lane; j < cbytes / 16; j += 32) dc[j] = (t >= 0) ? __ldg(sc + j) : make_uint4(0, 0, 0, 0);
+    for (int64_t j0 = lane; j0 < ncv; j0 += 128) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t j = j0 + 32 * u;
+        v[u] = (has && j < ncv) ? __ldg(sc + j) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (j0 + 32 * u < ncv) dc[j0 + 32 * u] = v[u];
+    }
     // scales: 4 consecutive blocks are 4 contiguous bytes in both layouts
     for (int64_t q = lane; q < nkb / 4; q += 32) {
-      uint32_t v = (t >= 0) ? __ldg(reinterpret_cast<const uint32_t*>(a_scales + static_cast<int64_t>(t) * nkb) + q) : 0u;
+      uint32_t v = has ? __ldg(reinterpret_cast<const uint32_t*>(a_scales + static_cast<int64_t>(t) * nkb) + q) : 0u;
       *reinterpret_cast<uint32_t*>(pa_scales + tiled_scale_offset(p, 4 * q, ncol_tiles)) = v;
     }
     if (n_chan) {
-      for (int j = lane; j < n_chan; j += 32)
-        pa_resid[p * n_chan + j] = (t >= 0) ? a_resid[static_cast<int64_t>(t) * n_chan + j] : 0;
+      if (rvec) {
+        const int nrv = n_chan / 8;
+        const uint4* sr = reinterpret_cast<const uint4*>(a_resid + static_cast<int64_t>(t) * n_chan);
+        uint4* dr = reinterpret_cast<uint4*>(pa_resid + p * n_chan);
+        for (int j = lane; j < nrv; j += 32) dr[j] = has ? __ldg(sr + j) : make_uint4(0, 0, 0, 0);
+      } else {
+        for (int j = lane; j < n_chan; j += 32)
+          pa_resid[p * n_chan + j] = has ? a_resid[static_cast<int64_t>(t) * n_chan + j] : 0;
+      }
     }
   }
 }
@@ -326,9 +347,20 @@ __global__ void __launch_bounds__(256) gather_bf16_kernel(const int32_t* __restr
   for (int64_t p = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; p < rows;
        p += (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5) {
     const int t = src_of[p];
+    const bool has = t >= 0;
     uint4* d = reinterpret_cast<uint4*>(out + p * H);
     const uint4* sx = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t) * H);
-    for (int64_t j = lane; j < nvec; j += 32) d[j] = (t >= 0) ? __ldg(sx + j) : make_uint4(0, 0, 0, 0);
+    for (int64_t j0 = lane; j0 < nvec; j0 += 128) {     // four loads in flight per lane
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t j = j0 + 32 * u;
+        v[u] = (has && j < nvec) ? __ldg(sx + j) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (j0 + 32 * u < nvec) d[j0 + 32 * u] = v[u];
+    }
   }
 }
 
