@@ -211,6 +211,11 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a) {
   // weight fake-quant: each warp's W_fq words of the current pass (32 lanes x
   // 8 words), from which the compensation columns are picked
   __shared__ __align__(16) uint32_t wfq_s[kFq ? (kThreads / 32) * 32 * 8 : 4];
+  // residual channels of the other modes: each warp's inputs (32 lanes x 8
+  // words), codes (32 x 2 words) and block scale values (32 words) of the
+  // current pass, from which the channel slots pick their element
+  constexpr int kXqWords = 32 * 8 + 32 * 2 + 32;
+  __shared__ __align__(16) uint32_t xq_s[kFq ? 4 : (kThreads / 32) * kXqWords];
   const int n = a.n_groups;
   const int nkb = static_cast<int>(a.K / 16);
   const int npass = (nkb + 31) / 32;
@@ -331,28 +336,36 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a) {
             __syncwarp();
           }
         } else if (a.resid) {
-          // Channel slot j of this pass is taken by lane j % 32: the element's
-          // code and block scale come from the owning lane by shuffles (the
-          // input element, where needed, is read back through L2).
-          // bf16(deq) = bf16(fp32(val(q) val(s)) g) is the W_fq value itself.
+          // Channel slot j of this pass is taken by lane j % 32, which picks
+          // the element's input, code and block scale from the warp's staged
+          // pass.  bf16(deq) = bf16(fp32(val(q) val(s)) g) is the W_fq value.
           const int slo = pass_slot[p], shi = pass_slot[p + 1];
-          for (int j0 = slo; j0 < shi; j0 += 32) {       // warp-uniform
-            const int j = j0 + lane;
-            const bool act = j < shi;
-            const int c = act ? chan_s[j] : 512 * p;
-            const int src = (c - 512 * p) >> 4, bit = c & 15;
-            const uint32_t cl = __shfl_sync(0xffffffffu, q.lo, src);
-            const uint32_t ch = __shfl_sync(0xffffffffu, q.hi, src);
-            const float sv = __shfl_sync(0xffffffffu, q.sv, src);
-            const uint32_t code = (((bit < 8) ? cl : ch) >> (4 * (bit & 7))) & 15u;
-            float v;
-            if (resid_mode == 1) {
-              v = deq_f32(code, sv, g);
-            } else {
-              const float xv = act ? bf16_bits_to_float(__ldg(xr + c)) : 0.0f;
-              v = (resid_mode == 2) ? xv : __fsub_rn(xv, deq_f32(code, sv, g));
+          if (slo < shi) {                                 // warp-uniform
+            uint32_t* const xs = xq_s + (threadIdx.x >> 5) * kXqWords;
+            st_shared_u32x8(xs + lane * 8, w[u]);
+            xs[256 + 2 * lane] = q.lo;
+            xs[257 + 2 * lane] = q.hi;
+            xs[320 + lane] = __float_as_uint(q.sv);
+            __syncwarp();
+            for (int j0 = slo; j0 < shi; j0 += 32) {
+              const int j = j0 + lane;
+              if (j < shi) {
+                const int c = chan_s[j] - 512 * p;         // column within the pass
+                const int src = c >> 4, bit = c & 15;
+                const uint32_t code = (xs[256 + 2 * src + (bit >> 3)] >> (4 * (bit & 7))) & 15u;
+                const float sv = __uint_as_float(xs[320 + src]);
+                float v;
+                if (resid_mode == 1) {
+                  v = deq_f32(code, sv, g);
+                } else {
+                  const uint32_t xw = xs[8 * src + (bit >> 1)];
+                  const float xv = bf16_bits_to_float((bit & 1) ? (xw >> 16) : (xw & 0xFFFFu));
+                  v = (resid_mode == 2) ? xv : __fsub_rn(xv, deq_f32(code, sv, g));
+                }
+                a.resid[drow * a.n_chan + j] = static_cast<uint16_t>(float_to_bf16_bits(v));
+              }
             }
-            if (act) a.resid[drow * a.n_chan + j] = static_cast<uint16_t>(float_to_bf16_bits(v));
+            __syncwarp();
           }
         }
       }
