@@ -57,13 +57,21 @@ struct DirArgs {
 };
 
 // Index of the largest E2M1 level (0, .5, 1, 1.5, 2, 3, 4, 6) at or below |v|,
-// from the bits of v: the levels from 1 up are the floats 2^e (1 + m/2) with
-// e in 0..2 and one mantissa bit m, so for |v| >= 1 the index is
-// 2 + 2 e + m = (exponent field * 2 + top mantissa bit) - 252 (capped at 7);
-// [0.5, 1) is level 1 and anything below 0.5 (zeros, subnormals) level 0.
-__device__ __forceinline__ uint32_t floor_level(float v) {
-  const int t = static_cast<int>((__float_as_uint(v) & 0x7FFFFFFFu) >> 22) - 252;
-  return t >= 2 ? static_cast<uint32_t>(min(t, 7)) : static_cast<uint32_t>(t >= 0);
+// for both floats of a pair at once, in two 16-bit lanes: [level(lo) |
+// level(hi) << 16].  The levels from 1 up are the floats 2^e (1 + m/2) with e
+// in 0..2 and one mantissa bit m, so for |v| >= 1 the index is 2 + 2 e + m =
+// f - 252 with f = exponent field * 2 + top mantissa bit (capped at 7);
+// [0.5, 1) (f = 252, 253) is level 1 and anything below 0.5 (zeros,
+// subnormals) level 0.  With f clamped to [251, 259] that is f - 251, less
+// one for f >= 253.
+__device__ __forceinline__ uint32_t floor_level2(uint64_t y) {
+  const uint32_t w = __byte_perm(static_cast<uint32_t>(y), static_cast<uint32_t>(y >> 32), 0x7632);
+  const uint32_t f = (w >> 6) & 0x01FF01FFu;      // the sign bits fall outside the mask
+  uint32_t a;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(a) : "r"(f), "r"(0x00FB00FBu));
+  asm("min.u16x2 %0, %0, %1;" : "+r"(a) : "r"(0x01030103u));
+  const uint32_t ge = ((a + 0x00030003u) >> 8) & 0x00010001u;
+  return a - 0x00FB00FBu - ge;
 }
 
 // Shared-memory group table (and, for few groups, the scale table tab);
@@ -126,8 +134,8 @@ __global__ void __launch_bounds__(kThreads, 4) direction_bits_kernel(DirArgs a) 
           uint32_t f[2] = {0u, 0u};
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            const uint64_t y = fmul2_rn(bf16x2_to_f32x2(w[u][i]), inv2);
-            f[i >> 2] |= (floor_level(lo_f32(y)) | (floor_level(hi_f32(y)) << 4)) << (8 * (i & 3));
+            const uint32_t l2 = floor_level2(fmul2_rn(bf16x2_to_f32x2(w[u][i]), inv2));
+            f[i >> 2] |= ((l2 | (l2 >> 12)) & 0xFFu) << (8 * (i & 3));
           }
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
@@ -219,11 +227,14 @@ __global__ void __launch_bounds__(kThreads, 3) replay_direction_kernel(DirArgs a
             // differing magnitudes counted 8 at a time
             const uint32_t own_lo = e2m1x8_from_pairs(y), own_hi = e2m1x8_from_pairs(y + 4);
             uint32_t mag_lo = 0, mag_hi = 0;
+            // bit 2i of the record to bit 0 and bit 2i + 1 to bit 16 of pair i
+            const uint32_t spread = (bits & 0x5555u) | ((bits & 0xAAAAu) << 15);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float v = (i & 1) ? hi_f32(y[i >> 1]) : lo_f32(y[i >> 1]);
-              const uint32_t lvl = min(floor_level(v) + ((bits >> i) & 1u), 7u);
-              if (i < 8) mag_lo |= lvl << (4 * i); else mag_hi |= lvl << (4 * (i - 8));
+            for (int i = 0; i < 8; ++i) {
+              uint32_t l2 = floor_level2(y[i]) + ((spread >> (2 * i)) & 0x00010001u);
+              asm("min.u16x2 %0, %0, %1;" : "+r"(l2) : "r"(0x00070007u));
+              const uint32_t nib = (l2 | (l2 >> 12)) & 0xFFu;   // elements 2i and 2i + 1
+              if (i < 4) mag_lo |= nib << (8 * i); else mag_hi |= nib << (8 * (i - 4));
             }
             q.lo = mag_lo | (own_lo & 0x88888888u);
             q.hi = mag_hi | (own_hi & 0x88888888u);
