@@ -196,16 +196,6 @@ __device__ __forceinline__ void st_shared_u32x8(uint32_t* p, const uint32_t (&o)
   reinterpret_cast<uint4*>(p)[1] = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-// Element i (0..15) of a block given as 8 packed BF16 words, by selects (no
-// indexed access to the register array).
-__device__ __forceinline__ uint32_t pick_bf16(const uint32_t (&w)[8], int i) {
-  const int wi = i >> 1;
-  const bool b0 = wi & 1, b1 = wi & 2, b2 = wi & 4;
-  const uint32_t t0 = b0 ? w[1] : w[0], t1 = b0 ? w[3] : w[2], t2 = b0 ? w[5] : w[4], t3 = b0 ? w[7] : w[6];
-  const uint32_t word = b2 ? (b1 ? t3 : t2) : (b1 ? t1 : t0);
-  return (i & 1) ? word >> 16 : word & 0xFFFFu;
-}
-
 template <int kMode>
 __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a) {
   constexpr bool kFq = kMode == 1, kAct = kMode == 2;
@@ -221,6 +211,11 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a) {
   // weight fake-quant: each warp's W_fq words of the current pass (32 lanes x
   // 8 words), from which the compensation columns are picked
   __shared__ __align__(16) uint32_t wfq_s[kFq ? (kThreads / 32) * 32 * 8 : 4];
+  // residual channels of the other modes: each warp's inputs (32 lanes x 8
+  // words), codes (32 x 2 words) and block scale values (32 words) of the
+  // current pass, from which the channel slots pick their element
+  constexpr int kXqWords = 32 * 8 + 32 * 2 + 32;
+  __shared__ __align__(16) uint32_t xq_s[kFq ? 4 : (kThreads / 32) * kXqWords];
   const int n = a.n_groups;
   const int nkb = static_cast<int>(a.K / 16);
   const int npass = (nkb + 31) / 32;
@@ -231,9 +226,6 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a) {
   float* g_s = reinterpret_cast<float*>(smem + n + 1);     // n
   int32_t* pass_slot = smem + 2 * n + 1;                   // npass + 1 (with channels)
   int32_t* chan_s = pass_slot + npass + 1;                 // n_chan
-  // the other modes' residual channels, per 16-column block: the slot of its
-  // first channel (high 16 bits) and a bit per channel column (low 16)
-  uint32_t* chan_blk = reinterpret_cast<uint32_t*>(chan_s + a.n_chan);   // nkb (with channels)
   __shared__ int n_valid_s;
   for (int i = threadIdx.x; i <= n; i += blockDim.x) {
     if (a.group_off != nullptr) off_s[i] = a.group_off[i];
@@ -264,17 +256,6 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a) {
       for (int j = 0; j < a.n_chan; ++j) cnt += (chan_s[j] >= 0 && chan_s[j] < a.K) ? 1 : 0;
       n_valid_s = cnt;
     }
-    if constexpr (!kFq)
-      for (int kb = threadIdx.x; kb < nkb; kb += blockDim.x) {
-        uint32_t first = 0, mask = 0;
-        for (int j = 0; j < a.n_chan; ++j) {
-          const int c = chan_s[j];
-          if (c < 0 || c >= a.K) continue;
-          if (c < 16 * kb) ++first;
-          else if (c < 16 * kb + 16) mask |= 1u << (c - 16 * kb);
-        }
-        chan_blk[kb] = first << 16 | mask;
-      }
   }
   __syncthreads();
   RowGroups grp{a.group_off ? off_s : nullptr, n, a.uniform_div};
@@ -354,26 +335,37 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a) {
             }
             __syncwarp();
           }
-        } else if (a.resid && kb < nkb) {
-          // the lane's own block: each channel column in it, from the input
-          // and code in its registers.  bf16(deq) = bf16(fp32(val(q) val(s)) g)
-          // is the W_fq value.
-          const uint32_t cb = chan_blk[kb];
-          uint32_t mask = cb & 0xFFFFu;
-          int slot = static_cast<int>(cb >> 16);
-          while (mask) {
-            const int i = __ffs(mask) - 1;
-            mask &= mask - 1u;
-            const uint32_t code = (((i & 8) ? q.hi : q.lo) >> (4 * (i & 7))) & 15u;
-            float v;
-            if (resid_mode == 1) {
-              v = deq_f32(code, q.sv, g);
-            } else {
-              const float xv = bf16_bits_to_float(pick_bf16(w[u], i));
-              v = (resid_mode == 2) ? xv : __fsub_rn(xv, deq_f32(code, q.sv, g));
+        } else if (a.resid) {
+          // Channel slot j of this pass is taken by lane j % 32, which picks
+          // the element's input, code and block scale from the warp's staged
+          // pass.  bf16(deq) = bf16(fp32(val(q) val(s)) g) is the W_fq value.
+          const int slo = pass_slot[p], shi = pass_slot[p + 1];
+          if (slo < shi) {                                 // warp-uniform
+            uint32_t* const xs = xq_s + (threadIdx.x >> 5) * kXqWords;
+            st_shared_u32x8(xs + lane * 8, w[u]);
+            xs[256 + 2 * lane] = q.lo;
+            xs[257 + 2 * lane] = q.hi;
+            xs[320 + lane] = __float_as_uint(q.sv);
+            __syncwarp();
+            for (int j0 = slo; j0 < shi; j0 += 32) {
+              const int j = j0 + lane;
+              if (j < shi) {
+                const int c = chan_s[j] - 512 * p;         // column within the pass
+                const int src = c >> 4, bit = c & 15;
+                const uint32_t code = (xs[256 + 2 * src + (bit >> 3)] >> (4 * (bit & 7))) & 15u;
+                const float sv = __uint_as_float(xs[320 + src]);
+                float v;
+                if (resid_mode == 1) {
+                  v = deq_f32(code, sv, g);
+                } else {
+                  const uint32_t xw = xs[8 * src + (bit >> 1)];
+                  const float xv = bf16_bits_to_float((bit & 1) ? (xw >> 16) : (xw & 0xFFFFu));
+                  v = (resid_mode == 2) ? xv : __fsub_rn(xv, deq_f32(code, sv, g));
+                }
+                a.resid[drow * a.n_chan + j] = static_cast<uint16_t>(float_to_bf16_bits(v));
+              }
             }
-            a.resid[drow * a.n_chan + slot] = static_cast<uint16_t>(float_to_bf16_bits(v));
-            ++slot;
+            __syncwarp();
           }
         }
       }
@@ -386,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 4) quantize_kernel(QuantArgs a) {
 size_t quantize_smem(int n_groups, int64_t K, int n_chan) {
   size_t s = (2 * static_cast<size_t>(n_groups) + 1) * 4;
   if (n_groups <= kTabGroups) s += static_cast<size_t>(n_groups) * 128 * sizeof(float2);
-  if (n_chan) s += (static_cast<size_t>((K / 16 + 31) / 32) + 1 + n_chan + K / 16) * 4;
+  if (n_chan) s += (static_cast<size_t>((K / 16 + 31) / 32) + 1 + n_chan) * 4;
   return s;
 }
 
