@@ -78,3 +78,35 @@ def test_budget_switch(cuda_lib):
     assert cuda_lib.set_sm_budget(prev) == 10
     with pytest.raises(cuda_lib.QuadsError):
         cuda_lib.set_sm_budget(-1)
+
+
+def test_layer_step_split_matches_unsplit(budget):
+    """The overlapped layer step with the STE on its own SMs beside the GEMMs
+    gives the same outputs, records, replayed operands, mismatch counts and
+    master gradients, bit for bit, as the step with every kernel on all SMs."""
+    from train_alignment_b200 import layer as L
+    from train_alignment_b200 import workloads as W
+    cfg = W.MOE_T2048
+    dev = torch.device("cuda")
+    inp = W.moe_layer_inputs(cfg, seed=3, device=dev)
+    x_train = W.engine_drift(inp["x"], 1e-2, seed=3, device=dev)
+    results = []
+    for side in (0, 40):
+        layer = L.build_layer(cfg, inp, dev, side_sms=side)
+        _, g_gu, g_d = layer.grad_fq_buffers()
+        g_gu.copy_(W.random_bf16(layer.w_gu.shape, 5, 1e-3, dev))
+        g_d.copy_(W.random_bf16(layer.w_d.shape, 6, 1e-3, dev))
+        layer.grad_all.zero_()
+        layer.reset_counts()
+        out = layer.step(inp["x"], inp["logits"], x_train, g_gu, g_d)
+        torch.cuda.synchronize()
+        assert budget.device_status() == budget.OK, budget.last_error()
+        assert budget.set_sm_budget(0) == 0, "the step leaves no budget behind"
+        n_rows = int(layer.expert_off[-1].item())       # h past the last expert's rows is never written
+        results.append({k: v.detach().clone() for k, v in (("out", out), ("h", layer.h[:n_rows]),
+                                                           ("counts", layer.counts), ("grad", layer.grad_all),
+                                                           ("record", layer.record))})
+    for k in results[0]:
+        a, b = results[0][k], results[1][k]
+        assert torch.equal(a.view(torch.uint8) if a.dtype != torch.int64 else a,
+                           b.view(torch.uint8) if b.dtype != torch.int64 else b), k
