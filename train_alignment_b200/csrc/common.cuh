@@ -331,9 +331,12 @@ __device__ __forceinline__ uint32_t e4m3_splat_f16x2(uint32_t s) {
 // The quantizer on 16 BF16 values given as 8 packed words (element 2i in the
 // low half of w[i]); same operations and rounding as quantize_block.
 __device__ __forceinline__ QCore quant_core(const uint32_t (&w)[8], const QConsts& c) {
+  // lane-wise max |.| of the pairs in one instruction each (the result's sign
+  // bits, the XOR of the inputs', are cleared afterwards)
   uint32_t m = 0u;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) m = __vmaxu2(m, w[i] & 0x7FFF7FFFu);
+  for (int i = 0; i < 8; ++i) asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(m) : "r"(w[i]));
+  m &= 0x7FFF7FFFu;
   const float amax = bf16_bits_to_float(max(m & 0xFFFFu, m >> 16));
   uint32_t s = 0;
   if (c.g != 0.0f) s = e4m3_from_float(block_ratio(amax, c));
