@@ -499,15 +499,16 @@ def secondary_workloads(dev, peaks, fp4_peak, steps=20):
     return out
 
 
-def gemm_side_measurements(layer, dev, peaks):
+def gemm_side_measurements(layer, dev, peaks, fp4_peak=None):
     """(1) The compensation's cost: the step layer's two grouped GEMMs with
     and without the BF16 correction on the same operands.  (2) Decode
     shapes (2048 hidden, 128 experts top-8, ffn 768, T = 64 and 512), measured
     as weight-stream bandwidth: the NVFP4 weight bytes (codes, scales and the
     BF16 Wc columns) of every expert that received rows, over the GEMM time,
     on the tiles the library picks (the decode tiles, weights as the MMA's M
-    operand) and on the 128 x 256 tiles.  L2 flushed before each timed
-    launch."""
+    operand) and on the 128 x 256 tiles.  (3) The same layer at T = 4096,
+    near the ridge, also as FP4 TFLOP/s against the measured FP4 peak.  L2
+    flushed before each timed launch."""
     import torch
     from train_alignment_b200 import layer as L
     from train_alignment_b200 import workloads as W
@@ -522,7 +523,7 @@ def gemm_side_measurements(layer, dev, peaks):
                            "gate_up_us": [t["gate_up"], t["gate_up_nocomp"]], "down_us": [t["down"], t["down_nocomp"]]}
     dec = []
     from train_alignment_b200 import binding as B
-    for T in (64, 512):
+    for T in (64, 512, 4096):
         cfg = W.decode_config(T)
         inp = W.moe_layer_inputs(cfg, seed=0, device=dev)
         ly = L.build_layer(cfg, inp, dev)
@@ -546,6 +547,11 @@ def gemm_side_measurements(layer, dev, peaks):
             gbs = (wb_g + wb_d) / ((tg + td) * 1e-6) / 1e9
             row.update({key + "gate_up_us": tg, key + "down_us": td, key + "weight_stream_gbs": gbs,
                         key + "frac_hbm": gbs / peaks["hbm_gbs"]})
+            if T >= 4096:
+                fl = sum(gemm_flops(cfg))
+                row.update({key + "TFLOP/s": fl / ((tg + td) * 1e-6) / 1e12})
+                if fp4_peak:
+                    row[key + "frac_fp4"] = fl / ((tg + td) * 1e-6) / 1e12 / fp4_peak
         dec.append(row)
         del ly, inp
         torch.cuda.empty_cache()
@@ -1014,7 +1020,8 @@ def run_ours(args):
     if not args.no_sweep:
         sweep = quantize_replay_sweep(dev, peaks["hbm_gbs"])
     trainer = trainer_gemm_timing(layer, dev, peaks) if not args.no_sweep else None
-    gemm_side = gemm_side_measurements(layer, dev, peaks) if not args.no_sweep and layer.comp == "bf16" else None
+    gemm_side = (gemm_side_measurements(layer, dev, peaks, fp4_peak) if not args.no_sweep and layer.comp == "bf16"
+                 else None)
     secondary = None
     if not args.no_secondary and world == 1:
         try:
