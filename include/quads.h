@@ -85,7 +85,9 @@ int quads_selftest_bounded_wait(uint64_t timeout_ns, quads_stream_t stream);
  *      its own half of the rows and of the weight rows).
  * Shapes 1 and 2 accumulate the correction into the FP4 accumulator as
  * (R / G) . Wc, with R / G = bf16(fp32(R * fp32(1 / G))) and G = g_a g_w[e].
- * Other GEMMs (W4A16, the FP4 correction, N % 256 != 0) always take shape 0.
+ * Other FP4 GEMMs (the FP4 correction, N % 256 != 0) always take shape 0.
+ * The W4A16 GEMMs take their tensor-memory kernel under shapes 1 and 2
+ * (N % 256 == 0) and the 128 x N kernel under shape 0.
  * Returns the previous shape, or QUADS_ERR_INVALID_ARG for another value.
  * Process-wide; not synchronized with launches in flight. */
 int quads_gemm_set_tile_shape(int shape);
@@ -354,7 +356,10 @@ int quads_moe_grouped_gemm_nvfp4_swiglu_fp4comp(const uint8_t* a_codes, const ui
  * chip, so W_fq is never stored.  x [rows_cap][K] BF16, 16-byte aligned;
  * other arguments as quads_moe_grouped_gemm_nvfp4.  The SwiGLU variant
  * writes h [rows_cap][F] from weights in the 64-row interleaved gate/up order
- * (N = 2F) and the per-expert max |h| (amax_out, nullable). */
+ * (N = 2F) and the per-expert max |h| (amax_out, nullable).  Where N % 256
+ * == 0 (and the tile shape is not 0) W_fq is converted into tensor memory
+ * and read there by the MMA (units of 128 weight rows by up to 256 rows);
+ * otherwise, or with tile shape 0, it is converted into shared memory. */
 int quads_moe_grouped_gemm_w4a16(const uint16_t* x, const uint8_t* w_codes, const uint8_t* w_scales,
                                  const float* g_w, const int32_t* expert_off, int E,
                                  int64_t rows_cap, int64_t N, int64_t K, uint16_t* y,
