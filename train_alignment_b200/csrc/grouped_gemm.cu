@@ -909,7 +909,6 @@ constexpr int PBN = 256;
 constexpr int kPairHalfBytes = 128 * kStageRowBytes;               // 16384: 128 rows x 256 FP4
 constexpr int kPairSfaBytes = 4 * 512;                              // its 128 A rows, 4 MMAs
 constexpr int kPairSfbBytes = 2 * 4 * 512;                          // all 256 weight rows, 4 MMAs
-constexpr int kPairStageBytes = 2 * kPairHalfBytes + kPairSfaBytes + kPairSfbBytes;   // 38912
 // this CTA's weight rows per stage: half of the 256 in a pair, all 256 alone
 __host__ __device__ constexpr int wide_b_bytes(bool pair) { return pair ? kPairHalfBytes : 2 * kPairHalfBytes; }
 __host__ __device__ constexpr int wide_stage_bytes(bool pair) {
