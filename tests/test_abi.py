@@ -102,6 +102,8 @@ def test_rows_capacity(lib):
     lambda l: l.trace_replay_direction(None, None, 0, None, None, 1, 4, 32, None, None, 0, None, None, None, None,
                                        None),
     lambda l: l.quads_copy_f32(None, None, -1, None),
+    # a negative SM budget
+    lambda l: l.quads_set_sm_budget(-1),
 ])
 def test_invalid_arguments_are_rejected_on_the_host(lib, call):
     rc = call(lib)
@@ -145,3 +147,10 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     # a host tensor is refused too, rather than computed on the CPU
     with pytest.raises(ValueError, match="CUDA"):
         B.amax_bf16(torch.zeros((4, 16), dtype=torch.bfloat16))
+
+
+def test_sm_budget_switch(lib):
+    """The SM budget is host state: set, read back, restored (no launch)."""
+    prev = lib.quads_set_sm_budget(37)
+    assert lib.quads_set_sm_budget(prev) == 37
+    assert lib.quads_set_sm_budget(prev) == prev
