@@ -38,6 +38,6 @@ Pins: every function here is checked in ``tests/test_oracle_*.py`` against
 brute force, closed forms, library routines or invariants.  Functions with
 no such pin are listed as "parity unpinned" below.
 
-Parity unpinned: ``moe.per_token_gap`` (a reported diagnostic, no value is
-fixed by the pages).
+Parity unpinned: none.  ``moe.per_token_gap`` is a reported diagnostic: its
+formula is pinned by closed forms, and no page fixes the value it measures.
 """

@@ -142,7 +142,7 @@ def combine(y, row_of, w, k):
 
 def per_token_gap(y_rollout, y_trainer):
     """Per-token L2 distance between two layer outputs, relative to the
-    trainer output's norm (a reported diagnostic; parity unpinned)."""
+    trainer output's norm (a reported diagnostic: no page fixes its value)."""
     a = np.asarray(y_rollout, dtype=np.float64)
     b = np.asarray(y_trainer, dtype=np.float64)
     return np.linalg.norm(a - b, axis=1) / np.maximum(np.linalg.norm(b, axis=1), 1e-30)

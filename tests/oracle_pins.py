@@ -869,4 +869,24 @@ def pin_pack_bits_loop():
             assert int(p[i, j]) == sum(int(b[i, 8 * j + q]) << q for q in range(8))
 
 
+def pin_per_token_gap_closed_forms():
+    """The relative per-token distance ||y_r - y_t|| / ||y_t|| on rows built
+    to have a known answer: equal rows, scaled rows, an orthogonal step (a
+    3-4-5 triangle), and the trainer output as the denominator."""
+    r = np.random.default_rng(80)
+    yt = r.standard_normal((5, 16))
+    assert np.all(M.per_token_gap(yt, yt) == 0.0)
+    c = np.array([0.5, -0.25, 2.0, 1e-3, -1.0])
+    assert np.allclose(M.per_token_gap(yt * (1.0 + c)[:, None], yt), np.abs(c), rtol=1e-12, atol=0.0)
+    yt2 = np.zeros((3, 4))
+    yt2[:, 0] = 4.0
+    yr2 = yt2.copy()
+    yr2[:, 1] = 3.0
+    assert np.allclose(M.per_token_gap(yr2, yt2), 0.75, rtol=1e-15, atol=0.0)
+    assert np.allclose(M.per_token_gap(yt2, yr2), 0.6, rtol=1e-15, atol=0.0)
+    # a token whose two outputs are both zero has no gap
+    z = np.zeros((1, 8))
+    assert M.per_token_gap(z, z)[0] == 0.0
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -197,6 +197,18 @@ _layer_down_wc_chan_x = _source_mutation(OL.step, "wd = weight_sync(w_d, chan_h)
 _layer_no_bf16_before_swiglu = _source_mutation(OL.rollout_forward, "M.swiglu(y1b)", "M.swiglu(y1)")
 
 
+def _gap_over_rollout_norm(y_rollout, y_trainer):
+    a = np.asarray(y_rollout, dtype=np.float64)
+    b = np.asarray(y_trainer, dtype=np.float64)
+    return np.linalg.norm(a - b, axis=1) / np.maximum(np.linalg.norm(a, axis=1), 1e-30)
+
+
+def _gap_squared(y_rollout, y_trainer):
+    a = np.asarray(y_rollout, dtype=np.float64)
+    b = np.asarray(y_trainer, dtype=np.float64)
+    return np.sum((a - b) ** 2, axis=1) / np.maximum(np.sum(b * b, axis=1), 1e-30)
+
+
 MUTATIONS = {
     "e2m1_ties_away": [(F, "e2m1_rne_code", _e2m1_ties_up), (Q, "e2m1_rne_code", _e2m1_ties_up)],
     "e2m1_drops_sign": [(F, "e2m1_rne_code", _e2m1_no_sign), (Q, "e2m1_rne_code", _e2m1_no_sign)],
@@ -231,6 +243,8 @@ MUTATIONS = {
     "layer_h_residual_one_scale": [(OL, "rollout_forward", _layer_h_resid_one_scale)],
     "layer_down_wc_from_gate_up_channels": [(OL, "step", _layer_down_wc_chan_x)],
     "layer_swiglu_before_bf16_storage": [(OL, "rollout_forward", _layer_no_bf16_before_swiglu)],
+    "gap_over_rollout_norm": [(M, "per_token_gap", _gap_over_rollout_norm)],
+    "gap_squared_norms": [(M, "per_token_gap", _gap_squared)],
 }
 
 
