@@ -418,7 +418,7 @@ def secondary_workloads(dev, peaks, fp4_peak, steps=20):
     CUDA graph per step, as the headline step), and one train/rollout
     alignment pass of the 8-layer stack (rollout of all 8 layers with the
     last 4 recorded, then the trainer with those 4 replayed), host-launched,
-    with its per-token output gap (unpinned)."""
+    with its per-token output gap (a measured value that no page fixes)."""
     import torch
     from train_alignment_b200 import binding as B
     from train_alignment_b200 import layer as L
@@ -490,7 +490,7 @@ def secondary_workloads(dev, peaks, fp4_peak, steps=20):
     gp = gap.float()
     out[scfg.name] = {"ms_per_pass": statistics.median(ts), "tokens_per_s": scfg.T / (statistics.median(ts) * 1e-3),
                       "per_token_gap": {"median": float(gp.median()), "p90": float(gp.quantile(0.9)),
-                                        "max": float(gp.max()), "pinned": False},
+                                        "max": float(gp.max()), "fixed_by_pages": False},
                       "replayed_layer_mismatches": {"codes": int(cm), "scales": int(sm)},
                       "what": "rollout of 8 layers (last 4 recorded) + trainer with the 4 records replayed; "
                               "host-launched, events around the pass"}
